@@ -1,0 +1,380 @@
+"""Benchmark of the CCA / CCGQA layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl cca|reference]
+
+A step is one prefill forward (down-projection, latent stencil, latent attention,
+up-projection) of the whole batch of the workload (default: CCGQA bf16 long prefill,
+B=2 x 16384 tokens, E=2048, 16 query / 4 kv heads, C=2), inputs resident in HBM.  The L2
+is flushed (256 MiB write) between timed steps, outside each step's CUDA events.  The
+single-token decode step over the compressed cache (B=64, 8192 cached tokens) is timed in
+the same run and reported under "decode".  One JSON line is printed by rank 0.
+
+With --gpus N > 1 (under torchrun) every rank runs its own replica of the workload (the
+path has no exchange step); times are the max over ranks.
+
+--impl reference times the CPU oracle (the plain float64 restatement of the method) on a
+bounded sample of the same workload, on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import workloads as W  # noqa: E402
+
+METRIC = "CCA/CCGQA prefill tokens/s & TFLOP/s (% bf16 peak); decode GB/s (% HBM) on 1 B200"
+DEFAULT_WORKLOAD = "ccgqa_prefill_16k"
+DECODE_WORKLOAD = "ccgqa_decode_8k"
+
+
+def prefill_flops(w) -> float:
+    """Algorithmic flops of one prefill forward: 2 E (n_q + 2 n_kv) + 2 n_q E per token for
+    the projections, 4 d~ per visible (query, key, head) for the causal attention."""
+    tokens = w.batch * w.seq
+    proj = 2.0 * tokens * w.d_model * (w.n_q + 2 * w.n_kv) + 2.0 * tokens * w.n_q * w.d_model
+    return proj + attention_flops(w)
+
+
+def attention_flops(w) -> float:
+    return 2.0 * w.batch * w.n_heads * w.dl * w.seq * (w.seq + 1)
+
+
+def decode_bytes(w, es=2) -> float:
+    """Algorithmic HBM bytes of one decode step: the K/V cache read (L+1 rows), both weight
+    matrices, the conv / value-shift state read and written, x read and y written."""
+    B, ctx = w.batch, w.seq
+    cache = 2.0 * B * w.n_kv_heads * (ctx + 1) * w.dl * es
+    weights = ((w.n_q + 2 * w.n_kv) * w.d_model + w.d_model * w.n_q) * es
+    state = 2.0 * B * ((w.conv_kernel - 1) * (w.n_q + w.n_kv) + (w.n_kv - w.n_kv // 2)) * es
+    io = 2.0 * B * w.d_model * es
+    return cache + weights + state + io
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d["hbm_gbs"], d["bf16_tflops"], d.get("bf16_tflops_sustained"), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples while the GPU is busy."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out = ""
+        else:
+            self.out = ""
+
+    def summary(self):
+        rows = []
+        for line in self.out.splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                rows.append((float(parts[0]), float(parts[1]), parts[3:7]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r) if v.lower() == "active"})
+        loaded = [r for r in rows if r[0] > 0.5 * r[1]] or rows
+        return {"sm_mhz": statistics.median(r[0] for r in loaded), "sm_max_mhz": rows[0][1],
+                "reasons": reasons, "samples": len(rows)}
+
+
+def dist_setup(n):
+    if n <= 1:
+        return 0, 1, 0
+    import torch.distributed as dist
+    rank = int(os.environ["RANK"])
+    world = int(os.environ["WORLD_SIZE"])
+    local = int(os.environ.get("LOCAL_RANK", rank))
+    torch.cuda.set_device(local)
+    from datetime import timedelta
+    dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                            device_id=torch.device("cuda", local))
+    return rank, world, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world <= 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ------------------------------------------------------------------ the CUDA arm
+def bench_prefill(cls, w, steps, warmup, world, seed):
+    inp = W.make_inputs(w, seed=seed)
+    layer = cls.CCALayer.from_workload(w, inp)
+    x = inp.x.cuda()
+    y = torch.empty_like(x)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    for _ in range(warmup):
+        layer.prefill(x, out=y)
+    torch.cuda.synchronize()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    cls.cca_stage_timing(True)
+    for i in range(steps):
+        flush.fill_(i & 0xFF)
+        starts[i].record()
+        layer.prefill(x, out=y)
+        ends[i].record()
+    torch.cuda.synchronize()
+    barrier(world)
+    cls.cca_stage_timing(False)
+    stage_ms, calls = cls.cca_stage_times(8)
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    ms = statistics.fmean(step_ms)
+    stages = {n: t / max(calls, 1) for n, t in
+              zip(["qkv_projection", "latent_stencil", "latent_attention", "out_projection"], stage_ms)}
+
+    # end to end through the public API: pinned host x -> device, forward, y -> pinned host
+    xh = inp.x.pin_memory()
+    yh = torch.empty(xh.shape, dtype=xh.dtype).pin_memory()
+    for _ in range(2):
+        x.copy_(xh, non_blocking=True)
+        layer.prefill(x, out=y)
+        yh.copy_(y, non_blocking=True)
+    torch.cuda.synchronize()
+    e2e_s = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    e2e_e = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    for i in range(steps):
+        flush.fill_(i & 0xFF)
+        e2e_s[i].record()
+        x.copy_(xh, non_blocking=True)
+        layer.prefill(x, out=y)
+        yh.copy_(y, non_blocking=True)
+        e2e_e[i].record()
+    torch.cuda.synchronize()
+    e2e_ms = statistics.fmean(s.elapsed_time(e) for s, e in zip(e2e_s, e2e_e))
+    nbytes = x.numel() * x.element_size()
+    return dict(ms=ms, stages=stages, calls=calls, e2e_ms=e2e_ms, h2d=nbytes, d2h=nbytes,
+                launches=4 * steps)
+
+
+def bench_decode(cls, w, steps, warmup, seed):
+    inp = W.make_inputs(w, seed=seed)
+    layer = cls.CCALayer.from_workload(w, inp)
+    max_seq = w.seq + steps + warmup + 8
+    cache = layer.new_cache(w.batch, max_seq)
+    cache.k[:, :, :w.seq] = inp.k_cache.cuda()
+    cache.v[:, :, :w.seq] = inp.v_cache.cuda()
+    cache.conv_state.copy_(inp.conv_state.cuda())
+    cache.vshift_state.copy_(inp.vshift_state.cuda())
+    cache.lengths.copy_(inp.lengths.cuda())
+    x = inp.x.cuda()
+    y = torch.empty_like(x)
+    for _ in range(warmup):
+        layer.decode(x, cache, out=y)
+    torch.cuda.synchronize()
+    s = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    e = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    cls.cca_stage_timing(True)
+    for i in range(steps):
+        s[i].record()
+        layer.decode(x, cache, out=y)
+        e[i].record()
+    torch.cuda.synchronize()
+    cls.cca_stage_timing(False)
+    stage_ms, calls = cls.cca_stage_times(8)
+    cls.cca_cache_check(cache.struct)
+    ms = statistics.fmean(a.elapsed_time(b) for a, b in zip(s, e))
+    names = ["qkv_projection", "stencil_append", "split_kv_attention", "merge", "out_projection"]
+    return dict(ms=ms, stages={n: t / max(calls, 1) for n, t in zip(names, stage_ms)},
+                launches=6 * steps)
+
+
+def cpu_oracle_sample(w, budget_s=12.0, seed=0):
+    """Times the float64 oracle on the causal prefix of sequence 0 of the workload, doubling
+    the prefix from 512 tokens while the run stays within the budget."""
+    import numpy as np
+    import oracle.cca_oracle as O
+    from oracle.cca_oracle import OracleConfig, OracleWeights
+    inp = W.make_inputs(w, seed=seed)
+    cfg = OracleConfig(d_model=w.d_model, n_heads=w.n_heads, n_kv_heads=w.n_kv_heads,
+                       compression=w.compression, conv_kernel=w.conv_kernel)
+    f64 = lambda t: t.to(torch.float64).numpy()
+    ow = OracleWeights.from_arrays(cfg, f64(inp.w_qkv), f64(inp.w_o), f64(inp.conv_seq),
+                                   f64(inp.conv_chan))
+    x0 = f64(inp.x[0])
+    T = 512
+    best = None
+    spent = 0.0
+    while T <= w.seq:
+        t0 = time.perf_counter()
+        O.prefill_sequence(cfg, ow, x0[:T])
+        dt = time.perf_counter() - t0
+        spent += dt
+        best = (T, dt)
+        if spent + 4.5 * dt > budget_s or T == w.seq:
+            break
+        T = min(2 * T, w.seq)
+    T, dt = best
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    return dict(value=T / dt, unit="tokens/s", cores=cores, kind="oracle",
+                sample=f"float64 oracle forward of the first {T} tokens of sequence 0 of "
+                       f"{w.name} ({dt:.2f} s; per-token attention cost grows with the prefix, so "
+                       f"this overstates the oracle's full-length rate)")
+
+
+def run_cuda(args):
+    rank, world, local = dist_setup(args.gpus)
+    import compressed_latent_space_b200 as cls
+    cls.load()
+    w = W.WORKLOADS[args.workload]
+    hbm, bf16_peak, bf16_sus, peak_src = measured_peaks()
+    with ClockSampler(local) as clk:
+        pre = bench_prefill(cls, w, args.steps, args.warmup, world, seed=rank)
+        dec = None
+        if not args.no_decode:
+            dw = W.WORKLOADS[DECODE_WORKLOAD]
+            dec = bench_decode(cls, dw, args.steps, args.warmup, seed=rank)
+    ms = max_over_ranks(pre["ms"], world)
+    e2e_ms = max_over_ranks(pre["e2e_ms"], world)
+    tokens = w.batch * w.seq
+    flops = prefill_flops(w)
+    attn_ms = pre["stages"].get("latent_attention", float("nan"))
+    attn_tflops = attention_flops(w) / (attn_ms * 1e-3) / 1e12
+    line = {
+        "metric": METRIC,
+        "value": tokens * world / (ms * 1e-3),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": w.dtype,
+        "data": "synthetic (seeded N(0,1) x, N(0,0.02^2) weights)",
+        "config": {"workload": w.name, "description": w.description, "batch": w.batch,
+                   "seq_len": w.seq, "d_model": w.d_model, "n_heads": w.n_heads,
+                   "n_kv_heads": w.n_kv_heads, "compression": w.compression,
+                   "latent_head_dim": w.dl, "conv_kernel": w.conv_kernel,
+                   "parallelism": f"replicas x{world}",
+                   "l2": "flushed between timed steps (256 MiB write outside the step events)"},
+        "tflops": flops / (ms * 1e-3) / 1e12,
+        "tflops_frac_of_bf16_peak": flops / (ms * 1e-3) / 1e12 / bf16_peak,
+        "stages_ms": pre["stages"],
+        "roofline": {"kernel": "latent_attention", "bound": "tensor", "achieved": attn_tflops,
+                     "peak": bf16_peak, "unit": "TFLOP/s", "frac": attn_tflops / bf16_peak,
+                     "traffic": None, "peak_source": f"{peak_src} bf16 burst"},
+        "e2e": {"value": tokens * world / (e2e_ms * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": pre["h2d"], "d2h_bytes_per_step": pre["d2h"]},
+        "gpu_launches": pre["launches"] + (dec["launches"] if dec else 0),
+    }
+    if dec:
+        dw = W.WORKLOADS[DECODE_WORKLOAD]
+        dms = max_over_ranks(dec["ms"], world)
+        gbs = decode_bytes(dw) / (dms * 1e-3) / 1e9
+        line["decode"] = {"workload": dw.name, "description": dw.description, "ms_per_step": dms,
+                          "tokens_per_s": dw.batch * world / (dms * 1e-3), "GB/s": gbs,
+                          "frac_of_hbm": gbs / hbm, "hbm_peak_GB/s": hbm,
+                          "bytes_per_step": decode_bytes(dw), "stages_ms": dec["stages"],
+                          "peak_source": peak_src}
+    line["clocks"] = clk.summary()
+    if rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_oracle_sample(w)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# ------------------------------------------------------------------ the reference arm
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    w = W.WORKLOADS[args.workload]
+    per_step_budget = max(2.0, 150.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        cpu_oracle_sample(w, budget_s=per_step_budget)
+    vals = []
+    samples = []
+    for _ in range(args.steps):
+        r = cpu_oracle_sample(w, budget_s=per_step_budget)
+        vals.append(r["value"])
+        samples.append(r)
+    v = statistics.fmean(vals)
+    line = {"metric": METRIC, "value": v, "unit": "tokens/s", "impl": "reference",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": w.name, "description": w.description},
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": samples[-1]["cores"],
+                             "kind": "oracle", "sample": samples[-1]["sample"]},
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.WORKLOADS))
+    ap.add_argument("--impl", default="cca", choices=["cca", "reference"])
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)      # at least 3 untimed warm-up steps
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_cuda(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,458 @@
+// Single-token decode step over the compressed cache (gist.science explainer, 1. Problem
+// Statement: during generation the cache is streamed once per token; 2. Methodology:
+// the cache holds latent keys/values only, Hkv*d~ wide each).
+//
+// For each sequence b with L = lengths[b] cached tokens, one new token x[b]:
+//   D1  p = x W_qkv^T                                   (split-K partial sums, fp32)
+//   D2  latent stencil of the new row: the causal conv reads the stored KC-1 pre-conv rows,
+//       the value-shift reads the stored upper-half value row; q-k-mean, RMS norm, RoPE at
+//       position L; k, v appended at position L; conv / value-shift state advanced
+//   D3  split-KV attention of the G query heads of each group over keys 0..L
+//   D3b merge of the splits (log-sum-exp), o [B, NQ]
+//   D4  y = o W_o^T, then lengths[b] += 1
+// A sequence with L >= max_seq is left untouched (y row zero) and the cache status word is
+// set to a "full" code.
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace cca {
+namespace {
+
+constexpr int CHUNK = 256;        // keys per split-KV block
+
+// ------------------------------------------------------------------ D1 / D4 skinny GEMM
+// C[M, N] = A[M, K] * B[N, K]^T for small M (the batch), bf16 operands on mma.sync.
+// Grid (N / NB, ksplit, ceil(M/64)); 4 warps share the K slice of the block and reduce
+// through shared memory.  OUT_F32: write fp32 partial sums to C + ks*M*N; else write bf16.
+template <int NB, bool OUT_F32>
+__global__ void __launch_bounds__(128) skinny_gemm_kernel(const __nv_bfloat16 *__restrict__ A,
+                                                          const __nv_bfloat16 *__restrict__ B,
+                                                          void *__restrict__ C, int M, int N,
+                                                          int K, int k_per_split) {
+  constexpr int NT = NB / 8;
+  __shared__ float red[4][64][NB + 1];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gr = lane >> 2, qc = lane & 3;
+  const int n0 = blockIdx.x * NB;
+  const int ks = blockIdx.y;
+  const int mbase = blockIdx.z * 64;
+  const int kbeg = ks * k_per_split;
+  const int kend = min(K, kbeg + k_per_split);
+  float acc[4][NT][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < NT; ++j) acc[i][j][0] = acc[i][j][1] = acc[i][j][2] = acc[i][j][3] = 0.f;
+  for (int k0 = kbeg + warp * 16; k0 < kend; k0 += 64) {
+    uint32_t bf[NT][2];
+#pragma unroll
+    for (int j = 0; j < NT; ++j) {
+      const int n = n0 + j * 8 + gr;
+      const __nv_bfloat16 *bp = B + static_cast<size_t>(n) * K + k0 + 2 * qc;
+      bf[j][0] = n < N ? *reinterpret_cast<const uint32_t *>(bp) : 0u;
+      bf[j][1] = n < N ? *reinterpret_cast<const uint32_t *>(bp + 8) : 0u;
+    }
+#pragma unroll
+    for (int mt = 0; mt < 4; ++mt) {
+      const int ma = mbase + mt * 16 + gr, mb = ma + 8;
+      uint32_t af[4];
+      const __nv_bfloat16 *pa = A + static_cast<size_t>(ma) * K + k0 + 2 * qc;
+      const __nv_bfloat16 *pb = A + static_cast<size_t>(mb) * K + k0 + 2 * qc;
+      af[0] = ma < M ? *reinterpret_cast<const uint32_t *>(pa) : 0u;
+      af[1] = mb < M ? *reinterpret_cast<const uint32_t *>(pb) : 0u;
+      af[2] = ma < M ? *reinterpret_cast<const uint32_t *>(pa + 8) : 0u;
+      af[3] = mb < M ? *reinterpret_cast<const uint32_t *>(pb + 8) : 0u;
+#pragma unroll
+      for (int j = 0; j < NT; ++j) mma_bf16_16816(acc[mt][j], af, bf[j]);
+    }
+  }
+#pragma unroll
+  for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+    for (int j = 0; j < NT; ++j) {
+      red[warp][mt * 16 + gr][j * 8 + 2 * qc] = acc[mt][j][0];
+      red[warp][mt * 16 + gr][j * 8 + 2 * qc + 1] = acc[mt][j][1];
+      red[warp][mt * 16 + gr + 8][j * 8 + 2 * qc] = acc[mt][j][2];
+      red[warp][mt * 16 + gr + 8][j * 8 + 2 * qc + 1] = acc[mt][j][3];
+    }
+  __syncthreads();
+  for (int i = threadIdx.x; i < 64 * NB; i += blockDim.x) {
+    const int r = i / NB, c = i % NB;
+    const int m = mbase + r, n = n0 + c;
+    if (m >= M || n >= N) continue;
+    const float v = red[0][r][c] + red[1][r][c] + red[2][r][c] + red[3][r][c];
+    if (OUT_F32)
+      static_cast<float *>(C)[(static_cast<size_t>(ks) * M + m) * N + n] = v;
+    else
+      static_cast<__nv_bfloat16 *>(C)[static_cast<size_t>(m) * N + n] = __float2bfloat16_rn(v);
+  }
+}
+
+// ------------------------------------------------------------------ D2 decode stencil
+template <typename T>
+struct D2Params {
+  const float *p_part;
+  int ksplit;
+  const float *conv_seq, *conv_chan;
+  T *k_cache, *v_cache, *conv_state, *vshift_state;
+  int *lengths, *status;
+  float *q_new;
+  int B, H, Hkv, G, DL, NQ, NKV, NQKV, KC, max_seq;
+  unsigned flags;
+  float eps, rope_base;
+};
+
+template <typename T>
+__global__ void __launch_bounds__(128) decode_stencil_kernel(const D2Params<T> p) {
+  extern __shared__ float sm[];
+  const int g = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+  const int G = p.G, DL = p.DL, CH = (G + 2) * DL, QKC = (G + 1) * DL;
+  float *pn = sm;               // [CH] new projections (rounded like the prefill's P)
+  float *a = pn + CH;           // [QKC] after the sequence conv
+  float *u = a + QKC;           // [QKC] after channel conv / q-k-mean
+  float *inv = u + QKC;         // [G+1]
+  const int L = p.lengths[b];
+  if (L >= p.max_seq) {
+    if (tid == 0) report(p.status, DEV_CACHE_FULL);
+    return;
+  }
+  const int qcol0 = g * G * DL, kcol0 = p.NQ + g * DL, vcol0 = p.NQ + p.NKV + g * DL;
+  auto gch = [&](int c) {
+    return c < G * DL ? qcol0 + c : (c < QKC ? kcol0 + (c - G * DL) : vcol0 + (c - QKC));
+  };
+  for (int c = tid; c < CH; c += blockDim.x) {
+    const int gc = gch(c);
+    float s = 0.f;
+    for (int ks = 0; ks < p.ksplit; ++ks) s += p.p_part[(static_cast<size_t>(ks) * p.B + b) * p.NQKV + gc];
+    pn[c] = to_f32(from_f32<T>(s));
+  }
+  __syncthreads();
+  const int KC1 = p.KC - 1, W = p.NQ + p.NKV;
+  T *cs = p.conv_state + static_cast<size_t>(b) * KC1 * W;
+  for (int c = tid; c < QKC; c += blockDim.x) {
+    const int gc = gch(c);
+    const float *w = p.conv_seq + static_cast<size_t>(gc) * p.KC;
+    float acc = 0.f;
+    for (int j = 0; j < KC1; ++j) acc = fmaf(w[j], to_f32(cs[static_cast<size_t>(j) * W + gc]), acc);
+    a[c] = fmaf(w[KC1], pn[c], acc);
+  }
+  __syncthreads();
+  for (int o = tid; o < QKC; o += blockDim.x) {
+    const int hh = o / DL, i = o % DL;
+    const bool is_q = hh < G;
+    const int head_w = is_q ? g * G + hh : p.H + g;
+    const float *wr = p.conv_chan + (static_cast<size_t>(head_w) * DL + i) * DL;
+    float acc = 0.f;
+    for (int j = 0; j < DL; ++j) acc = fmaf(wr[j], a[hh * DL + j], acc);
+    if (p.flags & F_QK_MEAN) {
+      const float pk = pn[G * DL + i];
+      if (is_q) {
+        acc += 0.5f * (pn[hh * DL + i] + pk);
+      } else {
+        float mq = 0.f;
+        for (int h2 = 0; h2 < G; ++h2) mq += pn[h2 * DL + i];
+        acc += 0.5f * (mq / static_cast<float>(G) + pk);
+      }
+    }
+    u[o] = acc;
+  }
+  __syncthreads();
+  // RMS norm per head: one warp per head
+  const int warp = tid >> 5, lane = tid & 31;
+  for (int hh = warp; hh <= G; hh += blockDim.x / 32) {
+    float ss = 0.f;
+    for (int i = lane; i < DL; i += 32) ss += u[hh * DL + i] * u[hh * DL + i];
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+    if (lane == 0)
+      inv[hh] = (p.flags & F_QK_NORM) ? 1.0f / sqrtf(ss / static_cast<float>(DL) + p.eps) : 1.0f;
+  }
+  __syncthreads();
+  // RoPE at position L on (i, i + DL/2) pairs, then store q (workspace) and k (cache)
+  const int HALF = DL / 2;
+  for (int o = tid; o < (G + 1) * HALF; o += blockDim.x) {
+    const int hh = o / HALF, ip = o % HALF;
+    float x1 = u[hh * DL + ip] * inv[hh], x2 = u[hh * DL + ip + HALF] * inv[hh];
+    if (p.flags & F_ROPE) {
+      const double theta = pow(static_cast<double>(p.rope_base), -2.0 * ip / DL);
+      double sd, cd;
+      sincos(static_cast<double>(L) * theta, &sd, &cd);
+      const float c = static_cast<float>(cd), s = static_cast<float>(sd);
+      const float y1 = x1 * c - x2 * s, y2 = x1 * s + x2 * c;
+      x1 = y1;
+      x2 = y2;
+    }
+    if (hh < G) {
+      float *qd = p.q_new + (static_cast<size_t>(b) * p.H + g * G + hh) * DL;
+      qd[ip] = x1;
+      qd[ip + HALF] = x2;
+    } else {
+      T *kd = p.k_cache + ((static_cast<size_t>(b) * p.Hkv + g) * p.max_seq + L) * DL;
+      kd[ip] = from_f32<T>(x1);
+      kd[ip + HALF] = from_f32<T>(x2);
+    }
+  }
+  // value with the value-shift, appended at position L
+  const int vhalf = p.NKV / 2;
+  T *vs = p.vshift_state + static_cast<size_t>(b) * (p.NKV - vhalf);
+  for (int c = tid; c < DL; c += blockDim.x) {
+    const int vc = g * DL + c;
+    const bool shifted = vc >= vhalf;
+    const float val = ((p.flags & F_VALUE_SHIFT) && shifted) ? to_f32(vs[vc - vhalf]) : pn[QKC + c];
+    p.v_cache[((static_cast<size_t>(b) * p.Hkv + g) * p.max_seq + L) * DL + c] = from_f32<T>(val);
+  }
+  __syncthreads();   // every read of the old state is done
+  for (int c = tid; c < QKC; c += blockDim.x) {
+    const int gc = gch(c);
+    for (int j = 0; j + 1 < KC1; ++j) cs[static_cast<size_t>(j) * W + gc] = cs[static_cast<size_t>(j + 1) * W + gc];
+    if (KC1 > 0) cs[static_cast<size_t>(KC1 - 1) * W + gc] = from_f32<T>(pn[c]);
+  }
+  for (int c = tid; c < DL; c += blockDim.x) {
+    const int vc = g * DL + c;
+    if (vc >= vhalf) vs[vc - vhalf] = from_f32<T>(pn[QKC + c]);
+  }
+}
+
+// ------------------------------------------------------------------ D3 split-KV attention
+template <typename T>
+__global__ void __launch_bounds__(128) decode_attn_kernel(
+    const float *__restrict__ q_new, const T *__restrict__ k_cache, const T *__restrict__ v_cache,
+    const int *__restrict__ lengths, float *__restrict__ part_o, float *__restrict__ part_ml, int H,
+    int Hkv, int G, int DL, int max_seq, int nchunk, float scale_log2) {
+  extern __shared__ float sm[];
+  const int ch = blockIdx.x, g = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
+  const int L = lengths[b];
+  const int nkeys = L + 1;
+  const int s0 = ch * CHUNK;
+  const int n = L < max_seq ? min(CHUNK, nkeys - s0) : 0;
+  float *qs = sm;                   // [G][DL]
+  float *sc = qs + G * DL;          // [G][CHUNK]
+  float *ks = sc + G * CHUNK;       // [CHUNK][DL+1]
+  float *vsm = ks + CHUNK * (DL + 1);  // [CHUNK][DL]
+  float *ml = vsm + CHUNK * DL;     // [G][2]
+  if (n <= 0) {
+    for (int i = tid; i < G * DL; i += blockDim.x) {
+      const int hh = i / DL, d = i % DL;
+      part_o[((static_cast<size_t>(b) * H + g * G + hh) * nchunk + ch) * DL + d] = 0.f;
+    }
+    for (int hh = tid; hh < G; hh += blockDim.x) {
+      float *o = part_ml + ((static_cast<size_t>(b) * H + g * G + hh) * nchunk + ch) * 2;
+      o[0] = -INFINITY;
+      o[1] = 0.f;
+    }
+    return;
+  }
+  for (int i = tid; i < G * DL; i += blockDim.x)
+    qs[i] = q_new[(static_cast<size_t>(b) * H + g * G) * DL + i] * scale_log2;
+  const T *kb = k_cache + ((static_cast<size_t>(b) * Hkv + g) * max_seq + s0) * DL;
+  const T *vb = v_cache + ((static_cast<size_t>(b) * Hkv + g) * max_seq + s0) * DL;
+  for (int i = tid; i < n * DL / 8; i += blockDim.x) {
+    const int r = i / (DL / 8), c = (i % (DL / 8)) * 8;
+    float k8[8], v8[8];
+    load8(kb + static_cast<size_t>(r) * DL + c, k8);
+    load8(vb + static_cast<size_t>(r) * DL + c, v8);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      ks[r * (DL + 1) + c + e] = k8[e];
+      vsm[r * DL + c + e] = v8[e];
+    }
+  }
+  __syncthreads();
+  for (int i = tid; i < G * n; i += blockDim.x) {
+    const int hh = i / n, s = i % n;
+    float acc = 0.f;
+    for (int d = 0; d < DL; ++d) acc = fmaf(qs[hh * DL + d], ks[s * (DL + 1) + d], acc);
+    sc[hh * CHUNK + s] = acc;
+  }
+  __syncthreads();
+  const int warp = tid >> 5, lane = tid & 31;
+  for (int hh = warp; hh < G; hh += blockDim.x / 32) {
+    float mx = -INFINITY;
+    for (int s = lane; s < n; s += 32) mx = fmaxf(mx, sc[hh * CHUNK + s]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    float sum = 0.f;
+    for (int s = lane; s < n; s += 32) {
+      const float e = exp2f(sc[hh * CHUNK + s] - mx);
+      sc[hh * CHUNK + s] = e;
+      sum += e;
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+    if (lane == 0) {
+      ml[2 * hh] = mx;
+      ml[2 * hh + 1] = sum;
+    }
+  }
+  __syncthreads();
+  for (int i = tid; i < G * DL; i += blockDim.x) {
+    const int hh = i / DL, d = i % DL;
+    float acc = 0.f;
+    for (int s = 0; s < n; ++s) acc = fmaf(sc[hh * CHUNK + s], vsm[s * DL + d], acc);
+    part_o[((static_cast<size_t>(b) * H + g * G + hh) * nchunk + ch) * DL + d] = acc;
+  }
+  for (int hh = tid; hh < G; hh += blockDim.x) {
+    float *o = part_ml + ((static_cast<size_t>(b) * H + g * G + hh) * nchunk + ch) * 2;
+    o[0] = ml[2 * hh];
+    o[1] = ml[2 * hh + 1];
+  }
+}
+
+// ------------------------------------------------------------------ D3b merge
+template <typename T>
+__global__ void decode_merge_kernel(const float *__restrict__ part_o,
+                                    const float *__restrict__ part_ml, const int *__restrict__ lengths,
+                                    T *__restrict__ o, int H, int DL, int max_seq, int nchunk) {
+  const int b = blockIdx.x;
+  const bool full = lengths[b] >= max_seq;
+  const int nused = full ? 0 : min(nchunk, (lengths[b] + 1 + CHUNK - 1) / CHUNK);
+  for (int i = threadIdx.x; i < H * DL; i += blockDim.x) {
+    const int h = i / DL, d = i % DL;
+    const float *ml = part_ml + (static_cast<size_t>(b) * H + h) * nchunk * 2;
+    float mx = -INFINITY;
+    for (int c = 0; c < nused; ++c) mx = fmaxf(mx, ml[2 * c]);
+    float l = 0.f, acc = 0.f;
+    for (int c = 0; c < nused; ++c) {
+      const float w = exp2f(ml[2 * c] - mx);
+      l += w * ml[2 * c + 1];
+      acc += w * part_o[((static_cast<size_t>(b) * H + h) * nchunk + c) * DL + d];
+    }
+    o[static_cast<size_t>(b) * H * DL + i] = from_f32<T>(nused > 0 ? acc / l : 0.f);
+  }
+}
+
+__global__ void decode_advance_kernel(int *lengths, int B, int max_seq) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b < B && lengths[b] < max_seq) lengths[b] += 1;
+}
+
+int decode_ksplit(const Dims &d) {
+  // enough blocks to keep every SM streaming the weight matrix
+  const int nblk = (d.NQKV + 31) / 32;
+  int ks = (num_sms() + nblk - 1) / nblk;
+  if (ks < 1) ks = 1;
+  while (ks > 1 && d.E / ks < 64) --ks;
+  return ks;
+}
+
+inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+}  // namespace
+
+size_t decode_workspace_bytes(const Dims &d, int max_seq) {
+  const int nchunk = (max_seq + CHUNK - 1) / CHUNK;
+  const int ks = d.bf16 ? decode_ksplit(d) : 1;
+  const size_t es = d.bf16 ? 2 : 4;
+  size_t s = 0;
+  s += align256(static_cast<size_t>(ks) * d.B * d.NQKV * 4);
+  s += align256(static_cast<size_t>(d.B) * d.H * d.DL * 4);
+  s += align256(static_cast<size_t>(d.B) * d.H * nchunk * d.DL * 4);
+  s += align256(static_cast<size_t>(d.B) * d.H * nchunk * 2 * 4);
+  s += align256(static_cast<size_t>(d.B) * d.NQ * es);
+  return s;
+}
+
+void decode_workspace_carve(const Dims &d, int max_seq, void *ws, DecodeArgs &a) {
+  const int nchunk = (max_seq + CHUNK - 1) / CHUNK;
+  const int ks = d.bf16 ? decode_ksplit(d) : 1;
+  const size_t es = d.bf16 ? 2 : 4;
+  char *p = static_cast<char *>(ws);
+  a.p_part = reinterpret_cast<float *>(p);
+  p += align256(static_cast<size_t>(ks) * d.B * d.NQKV * 4);
+  a.q_new = reinterpret_cast<float *>(p);
+  p += align256(static_cast<size_t>(d.B) * d.H * d.DL * 4);
+  a.part_o = reinterpret_cast<float *>(p);
+  p += align256(static_cast<size_t>(d.B) * d.H * nchunk * d.DL * 4);
+  a.part_ml = reinterpret_cast<float *>(p);
+  p += align256(static_cast<size_t>(d.B) * d.H * nchunk * 2 * 4);
+  a.o = p;
+  a.ksplit = ks;
+  a.nchunk = nchunk;
+  a.chunk = CHUNK;
+}
+
+template <typename T>
+static cudaError_t decode_typed(const Dims &d, const DecodeArgs &a, cudaStream_t st,
+                                const StageMarker &mark) {
+  cudaError_t e;
+  // D1
+  if constexpr (sizeof(T) == 2) {
+    const int kps = ((d.E + a.ksplit - 1) / a.ksplit + 63) / 64 * 64;
+    dim3 g1((d.NQKV + 31) / 32, a.ksplit, (d.B + 63) / 64);
+    skinny_gemm_kernel<32, true><<<g1, 128, 0, st>>>(
+        static_cast<const __nv_bfloat16 *>(a.x), static_cast<const __nv_bfloat16 *>(a.w_qkv),
+        a.p_part, d.B, d.NQKV, d.E, kps);
+  } else {
+    e = gemm_simt(0, a.x, a.w_qkv, a.p_part, d.B, d.NQKV, d.E, st);
+    if (e != cudaSuccess) return e;
+  }
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  mark();
+  // D2
+  D2Params<T> p2;
+  p2.p_part = a.p_part;
+  p2.ksplit = sizeof(T) == 2 ? a.ksplit : 1;
+  p2.conv_seq = a.conv_seq;
+  p2.conv_chan = a.conv_chan;
+  p2.k_cache = static_cast<T *>(a.k_cache);
+  p2.v_cache = static_cast<T *>(a.v_cache);
+  p2.conv_state = static_cast<T *>(a.conv_state);
+  p2.vshift_state = static_cast<T *>(a.vshift_state);
+  p2.lengths = a.lengths;
+  p2.status = a.status;
+  p2.q_new = a.q_new;
+  p2.B = d.B; p2.H = d.H; p2.Hkv = d.Hkv; p2.G = d.G; p2.DL = d.DL;
+  p2.NQ = d.NQ; p2.NKV = d.NKV; p2.NQKV = d.NQKV; p2.KC = d.KC; p2.max_seq = a.max_seq;
+  p2.flags = d.flags;
+  p2.eps = d.eps;
+  p2.rope_base = d.rope_base;
+  const size_t sm2 = (static_cast<size_t>(d.G + 2) * d.DL + 2 * (d.G + 1) * d.DL + (d.G + 1)) * 4;
+  decode_stencil_kernel<T><<<dim3(d.Hkv, d.B), 128, sm2, st>>>(p2);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  mark();
+  // D3
+  const float scale_log2 = static_cast<float>(1.4426950408889634 / sqrt(static_cast<double>(d.DL)));
+  const size_t sm3 = (static_cast<size_t>(d.G) * d.DL + d.G * CHUNK + CHUNK * (d.DL + 1) +
+                      CHUNK * d.DL + 2 * d.G) * 4;
+  if (sm3 > 48 * 1024) {
+    e = cudaFuncSetAttribute(decode_attn_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(sm3));
+    if (e != cudaSuccess) return e;
+  }
+  decode_attn_kernel<T><<<dim3(a.nchunk, d.Hkv, d.B), 128, sm3, st>>>(
+      a.q_new, static_cast<const T *>(a.k_cache), static_cast<const T *>(a.v_cache), a.lengths,
+      a.part_o, a.part_ml, d.H, d.Hkv, d.G, d.DL, a.max_seq, a.nchunk, scale_log2);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  mark();
+  decode_merge_kernel<T><<<d.B, 256, 0, st>>>(a.part_o, a.part_ml, a.lengths,
+                                               static_cast<T *>(a.o), d.H, d.DL, a.max_seq,
+                                               a.nchunk);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  mark();
+  // D4
+  if constexpr (sizeof(T) == 2) {
+    dim3 g4((d.E + 15) / 16, 1, (d.B + 63) / 64);
+    skinny_gemm_kernel<16, false><<<g4, 128, 0, st>>>(
+        static_cast<const __nv_bfloat16 *>(a.o), static_cast<const __nv_bfloat16 *>(a.w_o),
+        a.y, d.B, d.E, d.NQ, d.NQ);
+  } else {
+    e = gemm_simt(0, a.o, a.w_o, a.y, d.B, d.E, d.NQ, st);
+    if (e != cudaSuccess) return e;
+  }
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  decode_advance_kernel<<<(d.B + 127) / 128, 128, 0, st>>>(a.lengths, d.B, a.max_seq);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  mark();
+  return cudaSuccess;
+}
+
+cudaError_t decode_step(const Dims &d, const DecodeArgs &a, cudaStream_t st,
+                        const StageMarker &mark) {
+  if (d.B == 0) return cudaSuccess;
+  return d.bf16 ? decode_typed<__nv_bfloat16>(d, a, st, mark)
+                : decode_typed<float>(d, a, st, mark);
+}
+
+}  // namespace cca

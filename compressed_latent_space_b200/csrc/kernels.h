@@ -1,0 +1,94 @@
+// Host-side launchers of the CCA kernels (internal to libcca; not part of the C ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace cca {
+
+// Shape of one layer plus the switches, as the kernels consume it.
+struct Dims {
+  int B = 0, S = 0;              // batch, tokens per sequence (prefill)
+  int E = 0, H = 0, Hkv = 0;     // d_model, query heads, key/value heads
+  int G = 0, DL = 0;             // group size H/Hkv, latent head width
+  int NQ = 0, NKV = 0, NQKV = 0; // H*DL, Hkv*DL, NQ + 2*NKV
+  int KC = 0;                    // sequence-conv taps
+  unsigned flags = 0;
+  float eps = 1e-6f;
+  float rope_base = 10000.f;
+  int bf16 = 1;                  // element type of activations / weights / cache
+};
+
+// Called after each kernel launch of a C-ABI call; records a timing event when stage
+// timing is on (see cca_stage_timing).
+struct StageMarker {
+  void *ctx = nullptr;
+  void (*fn)(void *) = nullptr;
+  void operator()() const {
+    if (fn) fn(ctx);
+  }
+};
+
+enum : unsigned { F_QK_MEAN = 1u, F_VALUE_SHIFT = 2u, F_QK_NORM = 4u, F_ROPE = 8u };
+
+// C[M, N] = A[M, K] * B[N, K]^T, bf16 in, fp32 accumulate, bf16 out (tcgen05 + TMA).
+cudaError_t gemm_bf16_tcgen05(const void *A, const void *B, void *C, int M, int N, int K,
+                              int *status, cudaStream_t st);
+// Same contraction on CUDA cores; element type float (bf16 == 0) or bf16.
+cudaError_t gemm_simt(int bf16, const void *A, const void *B, void *C, int M, int N, int K,
+                      cudaStream_t st);
+
+// Latent stencil of a prefill: P [B*S, NQKV] -> q [B, H, S, DL], k/v [B, Hkv, kv_stride, DL]
+// (kv_stride >= S: the cache's max_seq, or S for workspace buffers).  When conv_state is
+// non-null the last KC-1 pre-conv q|k rows and the last upper-half value row are stored
+// and lengths[b] = S.
+struct StencilArgs {
+  const void *P;
+  const float *conv_seq;
+  const float *conv_chan;
+  void *q, *k, *v;
+  int kv_stride;
+  void *conv_state;     // [B, KC-1, NQ+NKV] or null
+  void *vshift_state;   // [B, NKV - NKV/2]
+  int *lengths;         // [B]
+  bool write_state = false;
+};
+cudaError_t latent_stencil(const Dims &d, const StencilArgs &a, cudaStream_t st);
+
+// Causal latent attention: q [B, H, S, DL], k/v [B, Hkv, kv_stride, DL] -> o [B*S, NQ].
+cudaError_t latent_attention(const Dims &d, const void *q, const void *k, const void *v,
+                             int kv_stride, void *o, int *status, cudaStream_t st);
+
+// Decode step kernels.
+struct DecodeArgs {
+  const void *x;            // [B, E]
+  const void *w_qkv;        // [NQKV, E]
+  const void *w_o;          // [E, NQ]
+  const float *conv_seq;
+  const float *conv_chan;
+  void *y;                  // [B, E]
+  void *k_cache, *v_cache;  // [B, Hkv, max_seq, DL]
+  void *conv_state;         // [B, KC-1, NQ+NKV]
+  void *vshift_state;       // [B, NKV - NKV/2]
+  int *lengths;             // [B]
+  int *status;              // cache status word
+  int max_seq;
+  // workspace
+  float *p_part;            // [ksplit, B, NQKV]
+  float *q_new;             // [B, H, DL]
+  float *part_o;            // [B, H, nchunk, DL]
+  float *part_ml;           // [B, H, nchunk, 2]
+  void *o;                  // [B, NQ]
+  int ksplit;
+  int nchunk;
+  int chunk;
+};
+size_t decode_workspace_bytes(const Dims &d, int max_seq);
+void decode_workspace_carve(const Dims &d, int max_seq, void *ws, DecodeArgs &a);
+cudaError_t decode_step(const Dims &d, const DecodeArgs &a, cudaStream_t st,
+                        const StageMarker &mark);
+
+int num_sms();
+
+}  // namespace cca

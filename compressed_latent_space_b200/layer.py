@@ -1,0 +1,94 @@
+"""Convenience wrapper: one CCA / CCGQA layer whose parameters, workspace and caches are
+torch CUDA tensors, driving the C ABI of libcca.  Holds memory only; every step of the
+computation runs in the library's kernels."""
+from __future__ import annotations
+
+import torch
+
+from . import (CCA_BF16, CCA_DEFAULT_FLAGS, CCA_F32, cca_cache_alloc, cca_decode_step,
+               cca_decode_workspace_size, cca_prefill_forward, cca_prefill_workspace_size,
+               make_config, make_weights)
+
+
+class Cache:
+    """A decode cache laid out by cca_cache_alloc inside one uint8 CUDA buffer, with torch
+    views of its regions (k, v, conv_state, vshift_state, lengths)."""
+
+    def __init__(self, layer: "CCALayer", batch: int, max_seq: int, stream=None):
+        nbytes = cca_cache_alloc(layer.cfg, batch, max_seq)
+        self.buf = torch.empty(nbytes, dtype=torch.uint8, device=layer.device)
+        self.struct = cca_cache_alloc(layer.cfg, batch, max_seq, self.buf, stream)
+        self.batch, self.max_seq = batch, max_seq
+        base = self.buf.data_ptr()
+        dt, es = layer.dtype, layer.esize
+
+        def view(ptr, numel, dtype, esz, shape):
+            off = ptr - base
+            assert off % esz == 0
+            return self.buf[off:off + numel * esz].view(dtype).view(*shape)
+
+        c = layer.cfg
+        dl = layer.dl
+        self.k = view(self.struct.k, batch * c.n_kv_heads * max_seq * dl, dt, es,
+                      (batch, c.n_kv_heads, max_seq, dl))
+        self.v = view(self.struct.v, batch * c.n_kv_heads * max_seq * dl, dt, es,
+                      (batch, c.n_kv_heads, max_seq, dl))
+        kc1 = c.conv_kernel - 1
+        if kc1 > 0:
+            self.conv_state = view(self.struct.conv_state, batch * kc1 * (layer.n_q + layer.n_kv), dt,
+                                   es, (batch, kc1, layer.n_q + layer.n_kv))
+        else:
+            self.conv_state = None
+        half = layer.n_kv - layer.n_kv // 2
+        self.vshift_state = view(self.struct.vshift_state, batch * half, dt, es, (batch, half))
+        self.lengths = view(self.struct.lengths, batch, torch.int32, 4, (batch,))
+
+
+class CCALayer:
+    def __init__(self, d_model, n_heads, n_kv_heads, compression, w_qkv, w_o, conv_seq, conv_chan,
+                 conv_kernel=4, rope_base=10000.0, norm_eps=1e-6, flags=CCA_DEFAULT_FLAGS,
+                 dtype="bf16", device="cuda"):
+        self.dtype = torch.bfloat16 if dtype == "bf16" else torch.float32
+        self.esize = 2 if dtype == "bf16" else 4
+        self.device = torch.device(device)
+        self.cfg = make_config(d_model, n_heads, n_kv_heads, compression, conv_kernel, 1, rope_base,
+                               norm_eps, flags, CCA_BF16 if dtype == "bf16" else CCA_F32)
+        self.dl = d_model // n_heads // compression
+        self.n_q = n_heads * self.dl
+        self.n_kv = n_kv_heads * self.dl
+        self.w_qkv = w_qkv.to(self.device, self.dtype).contiguous()
+        self.w_o = w_o.to(self.device, self.dtype).contiguous()
+        self.conv_seq = conv_seq.to(self.device, torch.float32).contiguous()
+        self.conv_chan = conv_chan.to(self.device, torch.float32).contiguous()
+        self.weights = make_weights(self.w_qkv, self.w_o, self.conv_seq, self.conv_chan)
+        self._ws = None
+
+    @classmethod
+    def from_workload(cls, w, inputs, flags=CCA_DEFAULT_FLAGS, device="cuda"):
+        return cls(w.d_model, w.n_heads, w.n_kv_heads, w.compression, inputs.w_qkv, inputs.w_o,
+                   inputs.conv_seq, inputs.conv_chan, conv_kernel=w.conv_kernel,
+                   rope_base=w.rope_base, flags=flags, dtype=w.dtype, device=device)
+
+    def workspace(self, nbytes: int) -> torch.Tensor:
+        if self._ws is None or self._ws.numel() < nbytes:
+            self._ws = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=self.device)
+        return self._ws
+
+    def new_cache(self, batch: int, max_seq: int, stream=None) -> Cache:
+        return Cache(self, batch, max_seq, stream)
+
+    def prefill(self, x: torch.Tensor, cache: Cache | None = None, out: torch.Tensor | None = None,
+                stream=None) -> torch.Tensor:
+        B, S, E = x.shape
+        y = out if out is not None else torch.empty_like(x)
+        ws = self.workspace(cca_prefill_workspace_size(self.cfg, B, S))
+        cca_prefill_forward(self.cfg, self.weights, x, B, S, y,
+                            cache.struct if cache is not None else None, ws, stream)
+        return y
+
+    def decode(self, x: torch.Tensor, cache: Cache, out: torch.Tensor | None = None,
+               stream=None) -> torch.Tensor:
+        y = out if out is not None else torch.empty_like(x)
+        ws = self.workspace(cca_decode_workspace_size(self.cfg, cache.batch, cache.max_seq))
+        cca_decode_step(self.cfg, self.weights, x, y, cache.struct, ws, stream)
+        return y

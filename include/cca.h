@@ -1,0 +1,159 @@
+/*
+ * cca.h -- C ABI of the B200 (sm_100a) implementation of Compressed Convolutional
+ * Attention (CCA) and its grouped variant CCGQA.
+ *
+ * The operator (arXiv 2510.04476, "Compressed Convolutional Attention: Efficient
+ * Attention in a Compressed Latent Space"; gist.science explainer, 2. Methodology, Core
+ * Mechanism and Extension: CCGQA; arXiv abstract):
+ *   1. x [tokens, E] is projected to latent q (H heads), k and v (Hkv heads), each head
+ *      d~ = (E/H)/C wide, so the query latent is E/C wide ("Down-Projection").
+ *   2. q and k pass a causal depthwise convolution along the sequence (conv_kernel taps,
+ *      tap conv_kernel-1 on the current token) and a per-head channel convolution
+ *      (d~ x d~ per head, pointwise in time) ("Convolutional Mixing"); half of
+ *      (pre-conv q + pre-conv k) is added back to both ("Q-K-Mean"); the upper half of the
+ *      value channels of token t is taken from token t-1 ("Value-Shift"); q and k are
+ *      RMS-normalised per head and rotated by RoPE ("RoPE Integration").
+ *   3. causal softmax attention runs on the latent heads, query head h reading key/value
+ *      head h / (H/Hkv) (CCGQA), scale 1/sqrt(d~).
+ *   4. the latent result [tokens, E/C] is projected back to E.
+ *
+ * Conventions for every entry point:
+ *   - All device pointers are caller-owned; the library never allocates or frees device
+ *     memory.  Scratch comes from the caller's `workspace`, sized by the *_size queries.
+ *   - Work is enqueued asynchronously on `stream` (a cudaStream_t passed as void*; NULL =
+ *     the legacy default stream).  Arguments are validated on the host before any launch;
+ *     a failed check returns an error and launches nothing.
+ *   - Return value: CCA_OK (0) or a negative CCA_ERR_* code; the text of the last error of
+ *     the calling thread is in cca_last_error_string().  No C++ exception crosses the ABI.
+ *   - Tensors are dense and row-major in the listed index order.  Activations, projection
+ *     weights and the cache use the config's dtype (float32 or bfloat16); conv filters are
+ *     always float32.  Device pointers must be 16-byte aligned (CCA_ERR_ALIGNMENT).
+ */
+#ifndef CCA_H
+#define CCA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define CCA_API __attribute__((visibility("default")))
+
+typedef enum { CCA_F32 = 0, CCA_BF16 = 1 } cca_dtype_t;
+
+enum {
+  CCA_OK = 0,
+  CCA_ERR_INVALID_ARG = -1,   /* null pointer, non-positive size, inconsistent shape      */
+  CCA_ERR_UNSUPPORTED = -2,   /* valid operator, but outside what the kernels implement   */
+  CCA_ERR_WORKSPACE = -3,     /* workspace pointer null or smaller than the size query    */
+  CCA_ERR_CACHE_FULL = -4,    /* a sequence would pass max_seq                             */
+  CCA_ERR_ALIGNMENT = -5,     /* a device pointer is not 16-byte aligned                  */
+  CCA_ERR_CUDA = -6,          /* a CUDA call or kernel launch failed                      */
+  CCA_ERR_DEVICE = -7         /* a kernel reported an internal error (bounded wait ran out) */
+};
+
+/* Switches of the method's three expressivity steps and of normalisation / RoPE. */
+enum {
+  CCA_QK_MEAN = 1u,
+  CCA_VALUE_SHIFT = 2u,
+  CCA_QK_NORM = 4u,
+  CCA_ROPE = 8u,
+  CCA_DEFAULT_FLAGS = 15u
+};
+
+/* One CCA / CCGQA layer.  d_model = E, n_heads = H, n_kv_heads = Hkv (H % Hkv == 0;
+ * Hkv == H is CCA), compression = C with (E/H) % C == 0.  Supported by the kernels:
+ * d~ = E/H/C in {16, 32, 64}, conv_kernel in [1, 8], chan_conv_kernel == 1.  norm_eps is
+ * added to the mean square before the square root (1e-6 by default). */
+typedef struct {
+  int d_model;
+  int n_heads;
+  int n_kv_heads;
+  int compression;
+  int conv_kernel;
+  int chan_conv_kernel;
+  float rope_base;
+  float norm_eps;
+  unsigned flags;
+  int dtype;                /* cca_dtype_t */
+} cca_config_t;
+
+/* Layer parameters (device pointers).
+ *   w_qkv     [n_q + 2*n_kv, E]  rows: W_q (n_q = H*d~), W_k (n_kv = Hkv*d~), W_v
+ *   w_o       [E, n_q]
+ *   conv_seq  [n_q + n_kv, conv_kernel] float32, one causal filter per latent q/k channel
+ *   conv_chan [H + Hkv, d~, d~, chan_conv_kernel] float32 (head, out, in, tap)          */
+typedef struct {
+  const void *w_qkv;
+  const void *w_o;
+  const float *conv_seq;
+  const float *conv_chan;
+} cca_weights_t;
+
+/* Compressed decode state, laid out by cca_cache_alloc inside one caller buffer.
+ *   k, v          [batch, Hkv, max_seq, d~]  final latent keys (after conv, q-k-mean, norm
+ *                 and RoPE) and values (after value-shift)
+ *   conv_state    [batch, conv_kernel-1, n_q + n_kv]  pre-conv q|k projections of the last
+ *                 conv_kernel-1 tokens, oldest first, zero before position 0
+ *   vshift_state  [batch, n_kv - n_kv/2]  upper-half value projection of the last token
+ *   lengths       [batch] int32, tokens held per sequence (the RoPE position of the next)
+ *   status        int32 sticky error word set by kernels that met a full sequence       */
+typedef struct {
+  void *k;
+  void *v;
+  void *conv_state;
+  void *vshift_state;
+  int *lengths;
+  int *status;
+  int batch;
+  int max_seq;
+} cca_cache_t;
+
+/* Lays out a decode cache for `batch` sequences of up to `max_seq` tokens.
+ * dev_buf == NULL: only writes the byte count to *bytes.  Otherwise *bytes must be at
+ * least that count; fills *out with pointers into dev_buf and enqueues on `stream` the
+ * zeroing of the whole buffer (lengths = 0, status = 0).  Errors: INVALID_ARG,
+ * UNSUPPORTED, WORKSPACE (buffer too small), ALIGNMENT, CUDA. */
+CCA_API int cca_cache_alloc(const cca_config_t *cfg, int batch, int max_seq, void *dev_buf,
+                            size_t *bytes, cca_cache_t *out, void *stream);
+
+/* Scratch bytes needed by cca_prefill_forward (0 if the config is invalid). */
+CCA_API size_t cca_prefill_workspace_size(const cca_config_t *cfg, int batch, int seq);
+
+/* Scratch bytes needed by cca_decode_step for a cache of this shape (0 if invalid). */
+CCA_API size_t cca_decode_workspace_size(const cca_config_t *cfg, int batch, int max_seq);
+
+/* Full layer forward of `batch` sequences of `seq` tokens each, from position 0.
+ *   x [batch, seq, E] -> y [batch, seq, E]   (x and y must not overlap)
+ * cache == NULL: keys/values live in the workspace only.  Otherwise (cache->batch ==
+ * batch, seq <= max_seq) the final keys/values of every token are written to the cache,
+ * the conv and value-shift state of the last token are stored and lengths[b] = seq.
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CACHE_FULL (seq > max_seq), ALIGNMENT, CUDA. */
+CCA_API int cca_prefill_forward(const cca_config_t *cfg, const cca_weights_t *w, const void *x,
+                                int batch, int seq, void *y, cca_cache_t *cache,
+                                void *workspace, size_t ws_bytes, void *stream);
+
+/* One new token per sequence: x [batch, E] -> y [batch, E], batch = cache->batch.
+ * The token's key/value are appended at position lengths[b], its query attends to
+ * positions 0..lengths[b], the conv / value-shift state advance and lengths[b] += 1.
+ * A sequence already holding max_seq tokens is left untouched, its y row is zero and the
+ * cache status word is set to CCA_ERR_CACHE_FULL (read it with cca_cache_check).
+ * Errors (host): INVALID_ARG, UNSUPPORTED, WORKSPACE, ALIGNMENT, CUDA. */
+CCA_API int cca_decode_step(const cca_config_t *cfg, const cca_weights_t *w, const void *x,
+                            void *y, cca_cache_t *cache, void *workspace, size_t ws_bytes,
+                            void *stream);
+
+/* Waits for `stream`, then returns the cache's sticky status word (CCA_OK or
+ * CCA_ERR_CACHE_FULL) and clears it. */
+CCA_API int cca_cache_check(cca_cache_t *cache, void *stream);
+
+/* Text of the calling thread's last error ("" if none). */
+CCA_API const char *cca_last_error_string(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CCA_H */

@@ -1,0 +1,58 @@
+/*
+ * cca_stages.h -- the kernels of the CCA forward one at a time, for per-stage testing and
+ * timing.  Same conventions as cca.h (caller-owned device memory, asynchronous on
+ * `stream`, host-side validation, CCA_* status codes).  `status` is an optional device
+ * int (may be NULL) in which a kernel whose bounded wait ran out records a nonzero code.
+ */
+#ifndef CCA_STAGES_H
+#define CCA_STAGES_H
+
+#include "cca.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* C[m, n] = sum_k A[m, k] * B[n, k]  (A [M, K], B [N, K], C [M, N], all row-major, dtype
+ * as given).  bf16 runs on the tcgen05 tensor-core kernel when K % 8 == 0, float32 on CUDA
+ * cores.  This is the contraction of the down-projection (x W_qkv^T) and of the
+ * up-projection (o W_o^T) of the layer (gist.science explainer, 2. Methodology, Core
+ * Mechanism, "Down-Projection"). */
+CCA_API int cca_gemm(int dtype, const void *A, const void *B, void *C, int M, int N, int K,
+                     int *status, void *stream);
+
+/* Latent stencil: P [batch*seq, n_q + 2 n_kv] (the projections) ->
+ * q [batch, H, seq, d~], k and v [batch, Hkv, kv_stride, d~] with kv_stride >= seq.
+ * Sequence conv, channel conv, q-k-mean, value-shift, RMS norm and RoPE (positions 0..seq-1),
+ * as selected by cfg->flags (gist.science explainer, 2. Methodology, Core Mechanism). */
+CCA_API int cca_stage_stencil(const cca_config_t *cfg, const void *P, int batch, int seq,
+                              const float *conv_seq, const float *conv_chan, void *q, void *k,
+                              void *v, int kv_stride, void *stream);
+
+/* Causal latent attention: q [batch, H, seq, d~], k/v [batch, Hkv, kv_stride, d~] ->
+ * o [batch*seq, H*d~] (token-major), scale 1/sqrt(d~), query head h reads kv head
+ * h / (H/Hkv) (gist.science/de explainer, 2. Methodik: Softmax(QK^T)V in the compressed
+ * space; gist.science explainer, Extension: CCGQA). */
+CCA_API int cca_stage_attention(const cca_config_t *cfg, const void *q, const void *k,
+                                const void *v, int batch, int seq, int kv_stride, void *o,
+                                int *status, void *stream);
+
+/* Waits for `stream` and returns CCA_OK, or CCA_ERR_DEVICE if a kernel of the last
+ * cca_prefill_forward that used this workspace recorded an internal error. */
+CCA_API int cca_workspace_status(const void *workspace, void *stream);
+
+/* Per-kernel timing for benchmarks.  cca_stage_timing(1) starts a session: from then on
+ * every cca_prefill_forward / cca_decode_step records a CUDA event on its stream before its
+ * first kernel and after each kernel (events only; nothing else changes).
+ * cca_stage_timing(0) ends recording.  cca_stage_times waits for the recorded events and
+ * writes, for up to n kernels of the recorded calls (in launch order), the summed
+ * milliseconds to ms[] and the number of recorded calls to *calls; it returns the number
+ * of kernel slots per call.  Recording holds at most 4096 calls. */
+CCA_API int cca_stage_timing(int enable);
+CCA_API int cca_stage_times(double *ms, int n, int *calls);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CCA_STAGES_H */

@@ -1,0 +1,53 @@
+"""Shared helpers of the GPU parity tests: oracle configs from workloads, tolerances, and
+row samples.  Imports the oracle (tests may) and the product binding; neither imports
+the other."""
+import numpy as np
+import torch
+
+import oracle.cca_oracle as O
+from oracle.cca_oracle import OracleConfig, OracleWeights
+
+FLAG_BITS = dict(qk_mean=1, value_shift=2, qk_norm=4, rope=8)
+
+
+def oracle_config(w, flags=15) -> OracleConfig:
+    return OracleConfig(d_model=w.d_model, n_heads=w.n_heads, n_kv_heads=w.n_kv_heads,
+                        compression=w.compression, conv_kernel=w.conv_kernel,
+                        chan_conv_kernel=w.chan_conv_kernel, rope_base=w.rope_base,
+                        **{k: bool(flags & b) for k, b in FLAG_BITS.items()})
+
+
+def f64(t) -> np.ndarray:
+    return t.detach().to("cpu", torch.float64).numpy()
+
+
+def oracle_weights(cfg: OracleConfig, inp) -> OracleWeights:
+    return OracleWeights.from_arrays(cfg, f64(inp.w_qkv), f64(inp.w_o), f64(inp.conv_seq),
+                                     f64(inp.conv_chan))
+
+
+def bf16_err(y, ref) -> float:
+    """max |y - ref| / rms(ref): the bf16 parity measure (bound 2e-2)."""
+    y = np.asarray(y, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    return float(np.max(np.abs(y - ref)) / np.sqrt(np.mean(ref * ref)))
+
+
+BF16_TOL = 2e-2
+
+
+def assert_fp32_close(y, ref):
+    """|y - ref| <= 1e-4 + 1e-4 |ref| elementwise (the float32 parity bound)."""
+    y = np.asarray(y, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    bad = np.abs(y - ref) > 1e-4 + 1e-4 * np.abs(ref)
+    assert not bad.any(), f"{bad.sum()} elements off, max err {np.max(np.abs(y - ref)):.3e}"
+
+
+def sample_rows(S: int, rng, tile=128, n_random=512):
+    """First 16, last 16, every tile boundary +-1, and n_random seeded rows."""
+    rows = set(range(min(16, S))) | set(range(max(0, S - 16), S))
+    for t in range(0, S, tile):
+        rows |= {r for r in (t - 1, t, t + 1) if 0 <= r < S}
+    rows |= set(rng.choice(S, size=min(n_random, S), replace=False).tolist())
+    return np.array(sorted(rows))

@@ -1,0 +1,328 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Bounds: float32 |y - y_oracle| <= 1e-4 + 1e-4 |y_oracle| elementwise; bf16
+max |y - y_oracle| / rms(y_oracle) <= 2e-2.  The oracle computes in float64 from the exact
+(rounded) values handed to the GPU.  Full-size workloads are checked on sampled rows
+(first/last 16, tile boundaries +-1, 512 seeded rows per sequence) in the launch
+configuration the benchmark times.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle.cca_oracle as O
+import workloads as W
+from gpu_helpers import (BF16_TOL, assert_fp32_close, bf16_err, f64, oracle_config,
+                         oracle_weights, sample_rows)
+
+pytestmark = pytest.mark.gpu
+
+
+def small(name, **kw):
+    base = dict(batch=2, seq=200, d_model=256, n_heads=4, n_kv_heads=2, compression=2,
+                description=name)
+    base.update(kw)
+    return W.Workload(name, **base)
+
+
+# ------------------------------------------------------------------ single kernels
+@pytest.mark.parametrize("M,N,K", [(128, 256, 64), (300, 520, 200), (1000, 1536, 2048),
+                                   (257, 768, 512), (64, 2048, 512), (4096, 2048, 1024)])
+def test_gemm_bf16_tcgen05(cuda_lib, M, N, K):
+    cls = cuda_lib
+    g = torch.Generator("cpu").manual_seed(M + N + K)
+    A = torch.randn(M, K, generator=g).to(torch.bfloat16)
+    B = (torch.randn(N, K, generator=g) * 0.05).to(torch.bfloat16)
+    ref = A.double() @ B.double().T
+    C = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    cls.cca_gemm(cls.CCA_BF16, A.cuda(), B.cuda(), C, M, N, K, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    err = (C.double().cpu() - ref).abs()
+    assert (err <= 8e-3 * ref.abs() + 2e-3 * ref.pow(2).mean().sqrt()).all(), float(err.max())
+
+
+@pytest.mark.parametrize("M,N,K", [(128, 192, 256), (77, 130, 48)])
+def test_gemm_f32_simt(cuda_lib, M, N, K):
+    cls = cuda_lib
+    g = torch.Generator("cpu").manual_seed(7)
+    A = torch.randn(M, K, generator=g)
+    B = torch.randn(N, K, generator=g) * 0.05
+    C = torch.empty(M, N, device="cuda")
+    cls.cca_gemm(cls.CCA_F32, A.cuda(), B.cuda(), C, M, N, K)
+    torch.cuda.synchronize()
+    assert_fp32_close(f64(C), (A.double() @ B.double().T).numpy())
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("H,Hkv,C,E,S", [(4, 4, 4, 256, 130), (8, 2, 2, 512, 77), (6, 3, 1, 96, 65),
+                                         (4, 1, 2, 512, 33)])
+def test_stencil_matches_oracle(cuda_lib, dtype, H, Hkv, C, E, S):
+    cls = cuda_lib
+    w = W.Workload("t", 2, S, E, H, Hkv, C, dtype=dtype)
+    ocfg = oracle_config(w)
+    inp = W.make_inputs(w, seed=3, conv_std=0.3, identity_conv=True)
+    dt = w.torch_dtype
+    g = torch.Generator("cpu").manual_seed(11)
+    P = torch.randn(2 * S, w.n_q + 2 * w.n_kv, generator=g).to(dt)
+    q = torch.empty(2, H, S, w.dl, dtype=dt, device="cuda")
+    k = torch.empty(2, Hkv, S + 5, w.dl, dtype=dt, device="cuda")
+    v = torch.empty_like(k)
+    cfg = cls.make_config(E, H, Hkv, C, dtype=cls.CCA_BF16 if dtype == "bf16" else cls.CCA_F32)
+    cls.cca_stage_stencil(cfg, P.cuda(), 2, S, inp.conv_seq.cuda(), inp.conv_chan.cuda(), q, k, v,
+                          S + 5)
+    torch.cuda.synchronize()
+    ow = oracle_weights(ocfg, inp)
+    for b in range(2):
+        p = f64(P[b * S:(b + 1) * S])
+        pq, pk, pv = p[:, :w.n_q], p[:, w.n_q:w.n_q + w.n_kv], p[:, w.n_q + w.n_kv:]
+        rq, rk, rv, _ = O.latent_qkv(ocfg, ow, pq, pk, pv, np.arange(S))
+        gq = f64(q[b]).transpose(1, 0, 2).reshape(S, -1)
+        gk = f64(k[b, :, :S]).transpose(1, 0, 2).reshape(S, -1)
+        gv = f64(v[b, :, :S]).transpose(1, 0, 2).reshape(S, -1)
+        for got, ref in ((gq, rq), (gk, rk), (gv, rv)):
+            if dtype == "f32":
+                assert_fp32_close(got, ref)
+            else:
+                assert bf16_err(got, ref) < 1e-2
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("H,Hkv,DL,S", [(4, 4, 16, 130), (4, 2, 32, 200), (8, 2, 64, 129),
+                                        (3, 1, 32, 64), (2, 2, 64, 1)])
+def test_attention_matches_oracle(cuda_lib, dtype, H, Hkv, DL, S):
+    cls = cuda_lib
+    dt = torch.float32 if dtype == "f32" else torch.bfloat16
+    g = torch.Generator("cpu").manual_seed(5)
+    B = 2
+    q = torch.randn(B, H, S, DL, generator=g).to(dt)
+    k = torch.randn(B, Hkv, S, DL, generator=g).to(dt)
+    v = torch.randn(B, Hkv, S, DL, generator=g).to(dt)
+    o = torch.empty(B * S, H * DL, dtype=dt, device="cuda")
+    E = H * DL * 2
+    cfg = cls.make_config(E, H, Hkv, 2, dtype=cls.CCA_BF16 if dtype == "bf16" else cls.CCA_F32)
+    cls.cca_stage_attention(cfg, q.cuda(), k.cuda(), v.cuda(), B, S, S, o)
+    torch.cuda.synchronize()
+    ocfg = O.OracleConfig(d_model=E, n_heads=H, n_kv_heads=Hkv, compression=2)
+    for b in range(B):
+        ref = O.causal_attention(f64(q[b]).transpose(1, 0, 2).reshape(S, -1),
+                                 f64(k[b]).transpose(1, 0, 2).reshape(S, -1),
+                                 f64(v[b]).transpose(1, 0, 2).reshape(S, -1), ocfg)
+        got = f64(o[b * S:(b + 1) * S])
+        if dtype == "f32":
+            assert_fp32_close(got, ref)
+        else:
+            assert bf16_err(got, ref) < 1e-2
+
+
+# ------------------------------------------------------------------ whole layer
+def run_prefill(cls, w, inp, flags=15):
+    layer = cls.CCALayer.from_workload(w, inp, flags=flags)
+    y = layer.prefill(inp.x.cuda())
+    torch.cuda.synchronize()
+    return layer, y
+
+
+@pytest.mark.parametrize("conv_std", [0.02, 0.5])
+def test_prefill_tiny_fp32(cuda_lib, conv_std):
+    """CCA tiny fp32: B=1 S=128 E=256 H=4 Hkv=4 C=4 (d~=16)."""
+    w = W.WORKLOADS["cca_tiny_fp32"]
+    inp = W.make_inputs(w, seed=0, conv_std=conv_std)
+    _, y = run_prefill(cuda_lib, w, inp)
+    ocfg = oracle_config(w)
+    ref = O.prefill(ocfg, oracle_weights(ocfg, inp), f64(inp.x))
+    assert_fp32_close(f64(y), ref)
+
+
+@pytest.mark.parametrize("flags", [15, 14, 13, 11, 7, 0])
+@pytest.mark.parametrize("shape", [
+    dict(n_heads=4, n_kv_heads=4, compression=4, seq=129),              # CCA, d~=16
+    dict(n_heads=4, n_kv_heads=2, compression=2, seq=200),              # CCGQA, d~=32
+    dict(n_heads=8, n_kv_heads=2, compression=1, d_model=512, seq=77),  # d~=64, G=4
+])
+def test_prefill_bf16_flags(cuda_lib, shape, flags):
+    w = small("bf16", **shape)
+    inp = W.make_inputs(w, seed=1, conv_std=0.4, identity_conv=True)
+    _, y = run_prefill(cuda_lib, w, inp, flags)
+    ocfg = oracle_config(w, flags)
+    ref = O.prefill(ocfg, oracle_weights(ocfg, inp), f64(inp.x))
+    assert bf16_err(f64(y), ref) <= BF16_TOL
+
+
+@pytest.mark.parametrize("seq", [1, 2, 3, 4, 63, 64, 65, 127, 128, 129, 300])
+def test_prefill_ragged_lengths(cuda_lib, seq):
+    w = small("ragged", seq=seq, n_heads=6, n_kv_heads=3, d_model=192, compression=1)   # d~=32
+    inp = W.make_inputs(w, seed=seq, conv_std=0.4)
+    _, y = run_prefill(cuda_lib, w, inp)
+    ocfg = oracle_config(w)
+    ref = O.prefill(ocfg, oracle_weights(ocfg, inp), f64(inp.x))
+    assert bf16_err(f64(y), ref) <= BF16_TOL
+
+
+def test_prefill_causality_gpu(cuda_lib):
+    w = small("causal", seq=257)
+    inp = W.make_inputs(w, seed=2, conv_std=0.4)
+    layer, y0 = run_prefill(cuda_lib, w, inp)
+    x2 = inp.x.clone()
+    x2[:, 130:] = torch.randn(x2[:, 130:].shape, generator=torch.Generator().manual_seed(9)).to(x2.dtype)
+    y1 = layer.prefill(x2.cuda())
+    torch.cuda.synchronize()
+    assert torch.equal(y0[:, :130], y1[:, :130])
+    assert not torch.equal(y0[:, 130:], y1[:, 130:])
+
+
+def test_ccgqa_kv_eq_heads_equals_cca(cuda_lib):
+    """The GPU path with Hkv = H is CCA: equal to the oracle's CCA."""
+    w = small("cca", n_heads=4, n_kv_heads=4, compression=2, seq=150)
+    inp = W.make_inputs(w, seed=4, conv_std=0.3)
+    _, y = run_prefill(cuda_lib, w, inp)
+    ocfg = oracle_config(w)
+    assert bf16_err(f64(y), O.prefill(ocfg, oracle_weights(ocfg, inp), f64(inp.x))) <= BF16_TOL
+
+
+@pytest.mark.parametrize("name", ["cca_prefill_4k", "ccgqa_prefill_16k", "ccgqa_prefill_32k"])
+def test_full_size_prefill_sampled(cuda_lib, name):
+    w = W.WORKLOADS[name]
+    inp = W.make_inputs(w, seed=0)
+    _, y = run_prefill(cuda_lib, w, inp)
+    ocfg = oracle_config(w)
+    ow = oracle_weights(ocfg, inp)
+    rng = np.random.default_rng(0)
+    for b in range(w.batch):
+        rows = sample_rows(w.seq, rng)
+        ref = O.prefill_rows(ocfg, ow, f64(inp.x[b]), rows)
+        got = f64(y[b, torch.as_tensor(rows)])
+        assert np.isfinite(got).all()
+        assert bf16_err(got, ref) <= BF16_TOL, (b, bf16_err(got, ref))
+
+
+def test_prefill_fills_cache_and_state(cuda_lib):
+    cls = cuda_lib
+    w = small("cache", seq=70)
+    inp = W.make_inputs(w, seed=6, conv_std=0.4)
+    layer = cls.CCALayer.from_workload(w, inp)
+    cache = layer.new_cache(w.batch, 96)
+    layer.prefill(inp.x.cuda(), cache=cache)
+    torch.cuda.synchronize()
+    ocfg = oracle_config(w)
+    ow = oracle_weights(ocfg, inp)
+    assert cache.lengths.tolist() == [70, 70]
+    for b in range(w.batch):
+        _, st = O.prefill_sequence(ocfg, ow, f64(inp.x[b]))
+        gk = f64(cache.k[b, :, :70]).transpose(1, 0, 2).reshape(70, -1)
+        gv = f64(cache.v[b, :, :70]).transpose(1, 0, 2).reshape(70, -1)
+        assert bf16_err(gk, st.k_cache) < 1e-2
+        assert bf16_err(gv, st.v_cache) < 1e-2
+        assert bf16_err(f64(cache.conv_state[b]), st.conv_state) < 1e-2
+        assert bf16_err(f64(cache.vshift_state[b]), st.vshift_state) < 1e-2
+
+
+# ------------------------------------------------------------------ decode
+def load_cache(cache, inp, ctx):
+    cache.k[:, :, :ctx] = inp.k_cache.cuda()
+    cache.v[:, :, :ctx] = inp.v_cache.cuda()
+    cache.conv_state.copy_(inp.conv_state.cuda())
+    cache.vshift_state.copy_(inp.vshift_state.cuda())
+    cache.lengths.copy_(inp.lengths.cuda())
+
+
+def decode_vs_oracle(cls, w, inp, max_seq):
+    layer = cls.CCALayer.from_workload(w, inp)
+    cache = layer.new_cache(w.batch, max_seq)
+    load_cache(cache, inp, w.seq)
+    y = layer.decode(inp.x.cuda(), cache)
+    cls.cca_cache_check(cache.struct)
+    ocfg = oracle_config(w)
+    ow = oracle_weights(ocfg, inp)
+    ref_y, ref_k, ref_v, ref_conv, ref_vs = O.decode_batch(
+        ocfg, ow, f64(inp.x), f64(inp.k_cache), f64(inp.v_cache), inp.lengths.numpy(),
+        f64(inp.conv_state), f64(inp.vshift_state))
+    return layer, cache, y, (ref_y, ref_k, ref_v, ref_conv, ref_vs)
+
+
+def test_decode_step_full_size(cuda_lib):
+    """CCGQA bf16 decode: B=64, 8192 cached tokens, one new token each."""
+    w = W.WORKLOADS["ccgqa_decode_8k"]
+    inp = W.make_inputs(w, seed=0)
+    layer, cache, y, (ry, rk, rv, rc, rvs) = decode_vs_oracle(cuda_lib, w, inp, w.seq + 64)
+    assert bf16_err(f64(y), ry) <= BF16_TOL
+    L = w.seq
+    gk = f64(cache.k[:, :, L]).reshape(w.batch, -1)
+    gv = f64(cache.v[:, :, L]).reshape(w.batch, -1)
+    assert bf16_err(gk, rk) < 1e-2 and bf16_err(gv, rv) < 1e-2
+    assert bf16_err(f64(cache.conv_state), rc) < 1e-2
+    assert bf16_err(f64(cache.vshift_state), rvs) < 1e-2
+    assert (cache.lengths.cpu() == L + 1).all()
+
+
+def test_decode_ragged_lengths(cuda_lib):
+    w = W.Workload("dec", 5, 300, 256, 4, 2, 2, decode=True)
+    lengths = [0, 1, 255, 256, 300]
+    inp = W.make_inputs(w, seed=2, conv_std=0.4, lengths=lengths)
+    _, cache, y, (ry, *_rest) = decode_vs_oracle(cuda_lib, w, inp, 320)
+    assert bf16_err(f64(y), ry) <= BF16_TOL
+    assert cache.lengths.cpu().tolist() == [l + 1 for l in lengths]
+
+
+def test_decode_equals_prefill_gpu(cuda_lib):
+    """Prefill S0 tokens into the cache, then n decode steps == prefill of S0 + n tokens."""
+    cls = cuda_lib
+    w = small("dp", seq=40, batch=3)
+    inp = W.make_inputs(w, seed=8, conv_std=0.4)
+    layer = cls.CCALayer.from_workload(w, inp)
+    s0, n = 33, 7
+    x = inp.x.cuda()
+    y_full = layer.prefill(x)
+    cache = layer.new_cache(w.batch, 64)
+    layer.prefill(x[:, :s0].contiguous(), cache=cache)
+    for i in range(n):
+        yi = layer.decode(x[:, s0 + i].contiguous(), cache)
+        torch.cuda.synchronize()
+        assert bf16_err(f64(yi), f64(y_full[:, s0 + i])) <= BF16_TOL
+    ocfg = oracle_config(w)
+    ref = O.prefill(ocfg, oracle_weights(ocfg, inp), f64(inp.x))
+    assert bf16_err(f64(yi), ref[:, s0 + n - 1]) <= BF16_TOL
+    assert cache.lengths.tolist() == [s0 + n] * w.batch
+
+
+def test_decode_f32_equals_prefill(cuda_lib):
+    cls = cuda_lib
+    w = W.WORKLOADS["cca_tiny_fp32"].with_(batch=2, seq=20)
+    inp = W.make_inputs(w, seed=3, conv_std=0.4)
+    layer = cls.CCALayer.from_workload(w, inp)
+    cache = layer.new_cache(2, 32)
+    x = inp.x.cuda()
+    layer.prefill(x[:, :15].contiguous(), cache=cache)
+    ocfg = oracle_config(w)
+    ref = O.prefill(ocfg, oracle_weights(ocfg, inp), f64(inp.x))
+    for i in range(15, 20):
+        yi = layer.decode(x[:, i].contiguous(), cache)
+        torch.cuda.synchronize()
+        assert_fp32_close(f64(yi), ref[:, i])
+
+
+def test_decode_cache_full(cuda_lib):
+    cls = cuda_lib
+    w = W.Workload("full", 2, 16, 256, 4, 2, 2, decode=True)
+    inp = W.make_inputs(w, seed=1, lengths=[16, 10])
+    layer = cls.CCALayer.from_workload(w, inp)
+    cache = layer.new_cache(2, 16)
+    load_cache(cache, inp, 16)
+    k_before = cache.k.clone()
+    y = layer.decode(inp.x.cuda(), cache)
+    with pytest.raises(cls.CCAError) as e:
+        cls.cca_cache_check(cache.struct)
+    assert e.value.code == cls.CCA_ERR_CACHE_FULL
+    cls.cca_cache_check(cache.struct)          # the status word was cleared
+    assert torch.equal(y[0].float().cpu(), torch.zeros(w.d_model))
+    assert torch.equal(cache.k[0], k_before[0])
+    assert cache.lengths.tolist() == [16, 11]
+
+
+def test_prefill_workspace_status_clean(cuda_lib):
+    cls = cuda_lib
+    w = small("st", seq=300)
+    inp = W.make_inputs(w, seed=0)
+    layer, _ = run_prefill(cls, w, inp)
+    cls.cca_workspace_status(layer._ws)
