@@ -14,7 +14,7 @@ from ctypes import POINTER, c_float, c_int, c_size_t, c_uint, c_void_p
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libcca.so")
 
-CCA_F32, CCA_BF16 = 0, 1
+CCA_F32, CCA_BF16, CCA_F16 = 0, 1, 2
 CCA_OK = 0
 CCA_ERR_INVALID_ARG = -1
 CCA_ERR_UNSUPPORTED = -2
@@ -23,6 +23,7 @@ CCA_ERR_CACHE_FULL = -4
 CCA_ERR_ALIGNMENT = -5
 CCA_ERR_CUDA = -6
 CCA_ERR_DEVICE = -7
+CCA_ERR_RANGE = -8
 CCA_QK_MEAN, CCA_VALUE_SHIFT, CCA_QK_NORM, CCA_ROPE = 1, 2, 4, 8
 CCA_DEFAULT_FLAGS = 15
 
@@ -64,8 +65,8 @@ _SIGS = {
     "cca_decode_step": (c_int, [POINTER(cca_config_t), POINTER(cca_weights_t), c_void_p, c_void_p,
                                 POINTER(cca_cache_t), c_void_p, c_size_t, c_void_p]),
     "cca_cache_check": (c_int, [POINTER(cca_cache_t), c_void_p]),
-    "cca_gemm": (c_int, [c_int, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_void_p,
-                         c_void_p]),
+    "cca_gemm": (c_int, [c_int, c_int, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int,
+                         c_void_p, c_void_p]),
     "cca_stage_stencil": (c_int, [POINTER(cca_config_t), c_void_p, c_int, c_int, c_void_p,
                                   c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_void_p]),
     "cca_stage_attention": (c_int, [POINTER(cca_config_t), c_void_p, c_void_p, c_void_p, c_int,
@@ -171,8 +172,8 @@ def cca_cache_check(cache, stream=None):
     _check(load().cca_cache_check(ctypes.byref(cache), _stream(stream)))
 
 
-def cca_gemm(dtype, A, B, C, M, N, K, status=None, stream=None):
-    _check(load().cca_gemm(dtype, _ptr(A), _ptr(B), _ptr(C), M, N, K, _ptr(status), _stream(stream)))
+def cca_gemm(dtype, out_dtype, A, B, C, M, N, K, status=None, stream=None):
+    _check(load().cca_gemm(dtype, out_dtype, _ptr(A), _ptr(B), _ptr(C), M, N, K, _ptr(status), _stream(stream)))
 
 
 def cca_stage_stencil(cfg, P, batch, seq, conv_seq, conv_chan, q, k, v, kv_stride, stream=None):

@@ -5,10 +5,13 @@
 //   O[b, t, h*d~ + :] = sum_{s <= t} softmax_s(q[b,h,t] . k[b,g,s] / sqrt(d~)) v[b,g,s]
 //
 // Two kernels:
-//  * attn_mma_kernel (bf16): flash-style online softmax over 64-key tiles, mma.sync
-//    m16n8k16 for QK^T and PV, fp32 softmax; causal tiles above the diagonal are skipped.
+//  * attn_mma_kernel (16-bit layers): flash-style online softmax over 64-key tiles, mma.sync
+//    m16n8k16 f16 x f16 -> f32 for QK^T and PV (float16 latents and probabilities), fp32
+//    softmax, float16 output; causal tiles above the diagonal are skipped.
 //  * attn_simt_kernel (float32): one warp per query row, exact fp32 arithmetic.
 #include <math.h>
+
+#include <type_traits>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -20,13 +23,13 @@ constexpr int BM = 64, BN = 64;
 
 template <int DL>
 __global__ void __launch_bounds__(128) attn_mma_kernel(
-    const __nv_bfloat16 *__restrict__ Q, const __nv_bfloat16 *__restrict__ K,
-    const __nv_bfloat16 *__restrict__ V, __nv_bfloat16 *__restrict__ O, int S, int H, int Hkv,
+    const __half *__restrict__ Q, const __half *__restrict__ K,
+    const __half *__restrict__ V, __half *__restrict__ O, int S, int H, int Hkv,
     int G, int kv_stride, float scale_log2) {
   constexpr int KP = DL + 8;      // padded K row (bf16)
   constexpr int VP = BN + 8;      // padded V^T row (bf16)
-  __shared__ __align__(16) __nv_bfloat16 Ks[BN * KP];
-  __shared__ __align__(16) __nv_bfloat16 Vt[DL * VP];
+  __shared__ __align__(16) __half Ks[BN * KP];
+  __shared__ __align__(16) __half Vt[DL * VP];
   const int nqt = (S + BM - 1) / BM;
   const int qt = nqt - 1 - blockIdx.x;            // longest rows first
   const int h = blockIdx.y, b = blockIdx.z, g = h / G;
@@ -35,9 +38,9 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(
   const int q0 = qt * BM;
   const int qa = q0 + warp * 16 + gr, qb = qa + 8;
 
-  const __nv_bfloat16 *Qh = Q + (static_cast<size_t>(b) * H + h) * S * DL;
-  const __nv_bfloat16 *Kg = K + (static_cast<size_t>(b) * Hkv + g) * kv_stride * DL;
-  const __nv_bfloat16 *Vg = V + (static_cast<size_t>(b) * Hkv + g) * kv_stride * DL;
+  const __half *Qh = Q + (static_cast<size_t>(b) * H + h) * S * DL;
+  const __half *Kg = K + (static_cast<size_t>(b) * Hkv + g) * kv_stride * DL;
+  const __half *Vg = V + (static_cast<size_t>(b) * Hkv + g) * kv_stride * DL;
 
   // Q fragments (A operand), zero for rows past the sequence end.
   uint32_t qf[DL / 16][4];
@@ -71,7 +74,7 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(
         vv = *reinterpret_cast<const uint4 *>(Vg + static_cast<size_t>(kv0 + r) * DL + c);
       }
       *reinterpret_cast<uint4 *>(Ks + r * KP + c) = kv;
-      const __nv_bfloat16 *ve = reinterpret_cast<const __nv_bfloat16 *>(&vv);
+      const __half *ve = reinterpret_cast<const __half *>(&vv);
 #pragma unroll
       for (int e = 0; e < 8; ++e) Vt[(c + e) * VP + r] = ve[e];
     }
@@ -83,10 +86,10 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(
       s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.f;
 #pragma unroll
       for (int kk = 0; kk < DL / 16; ++kk) {
-        const __nv_bfloat16 *kr = Ks + (j * 8 + gr) * KP + kk * 16 + 2 * qc;
+        const __half *kr = Ks + (j * 8 + gr) * KP + kk * 16 + 2 * qc;
         uint32_t bf[2] = {*reinterpret_cast<const uint32_t *>(kr),
                           *reinterpret_cast<const uint32_t *>(kr + 8)};
-        mma_bf16_16816(s[j], qf[kk], bf);
+        mma_f16_16816(s[j], qf[kk], bf);
       }
     }
     // scale, causal mask, running max
@@ -126,11 +129,11 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(
       sum_b += p2 + p3;
       const int kk = j >> 1;
       if ((j & 1) == 0) {
-        pf[kk][0] = pack_bf16x2(p0, p1);
-        pf[kk][1] = pack_bf16x2(p2, p3);
+        pf[kk][0] = pack_f16x2(p0, p1);
+        pf[kk][1] = pack_f16x2(p2, p3);
       } else {
-        pf[kk][2] = pack_bf16x2(p0, p1);
-        pf[kk][3] = pack_bf16x2(p2, p3);
+        pf[kk][2] = pack_f16x2(p0, p1);
+        pf[kk][3] = pack_f16x2(p2, p3);
       }
     }
     l_a = l_a * corr_a + sum_a;
@@ -143,10 +146,10 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(
       o[dt][3] *= corr_b;
 #pragma unroll
       for (int kk = 0; kk < BN / 16; ++kk) {
-        const __nv_bfloat16 *vr = Vt + (dt * 8 + gr) * VP + kk * 16 + 2 * qc;
+        const __half *vr = Vt + (dt * 8 + gr) * VP + kk * 16 + 2 * qc;
         uint32_t bf[2] = {*reinterpret_cast<const uint32_t *>(vr),
                           *reinterpret_cast<const uint32_t *>(vr + 8)};
-        mma_bf16_16816(o[dt], pf[kk], bf);
+        mma_f16_16816(o[dt], pf[kk], bf);
       }
     }
   }
@@ -161,10 +164,10 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(
     const int col = h * DL + dt * 8 + 2 * qc;
     if (qa < S)
       *reinterpret_cast<uint32_t *>(O + (static_cast<size_t>(b) * S + qa) * NQ + col) =
-          pack_bf16x2(o[dt][0] * ia, o[dt][1] * ia);
+          pack_f16x2(o[dt][0] * ia, o[dt][1] * ia);
     if (qb < S)
       *reinterpret_cast<uint32_t *>(O + (static_cast<size_t>(b) * S + qb) * NQ + col) =
-          pack_bf16x2(o[dt][2] * ib, o[dt][3] * ib);
+          pack_f16x2(o[dt][2] * ib, o[dt][3] * ib);
   }
 }
 
@@ -221,25 +224,31 @@ __global__ void __launch_bounds__(256) attn_simt_kernel(const float *__restrict_
 
 }  // namespace
 
+static cudaError_t launch_mma(const Dims &d, const void *q, const void *k, const void *v,
+                              int kv_stride, void *o, float scale_log2, cudaStream_t st) {
+  dim3 grid((d.S + BM - 1) / BM, d.H, d.B);
+  auto Q = static_cast<const __half *>(q);
+  auto Kp = static_cast<const __half *>(k);
+  auto Vp = static_cast<const __half *>(v);
+  auto Op = static_cast<__half *>(o);
+  if (d.DL == 16)
+    attn_mma_kernel<16><<<grid, 128, 0, st>>>(Q, Kp, Vp, Op, d.S, d.H, d.Hkv, d.G, kv_stride, scale_log2);
+  else if (d.DL == 32)
+    attn_mma_kernel<32><<<grid, 128, 0, st>>>(Q, Kp, Vp, Op, d.S, d.H, d.Hkv, d.G, kv_stride, scale_log2);
+  else if (d.DL == 64)
+    attn_mma_kernel<64><<<grid, 128, 0, st>>>(Q, Kp, Vp, Op, d.S, d.H, d.Hkv, d.G, kv_stride, scale_log2);
+  else
+    return cudaErrorInvalidValue;
+  return cudaGetLastError();
+}
+
 cudaError_t latent_attention(const Dims &d, const void *q, const void *k, const void *v,
                              int kv_stride, void *o, int *status, cudaStream_t st) {
   (void)status;
   if (d.B == 0 || d.S == 0) return cudaSuccess;
   const float scale_log2 = static_cast<float>(1.4426950408889634 / sqrt(static_cast<double>(d.DL)));
   if (d.bf16) {
-    dim3 grid((d.S + BM - 1) / BM, d.H, d.B);
-    auto Q = static_cast<const __nv_bfloat16 *>(q);
-    auto Kp = static_cast<const __nv_bfloat16 *>(k);
-    auto Vp = static_cast<const __nv_bfloat16 *>(v);
-    auto Op = static_cast<__nv_bfloat16 *>(o);
-    if (d.DL == 16)
-      attn_mma_kernel<16><<<grid, 128, 0, st>>>(Q, Kp, Vp, Op, d.S, d.H, d.Hkv, d.G, kv_stride, scale_log2);
-    else if (d.DL == 32)
-      attn_mma_kernel<32><<<grid, 128, 0, st>>>(Q, Kp, Vp, Op, d.S, d.H, d.Hkv, d.G, kv_stride, scale_log2);
-    else if (d.DL == 64)
-      attn_mma_kernel<64><<<grid, 128, 0, st>>>(Q, Kp, Vp, Op, d.S, d.H, d.Hkv, d.G, kv_stride, scale_log2);
-    else
-      return cudaErrorInvalidValue;
+    return launch_mma(d, q, k, v, kv_stride, o, scale_log2, st);
   } else {
     const long long rows = static_cast<long long>(d.B) * d.H * d.S;
     const int grid = static_cast<int>((rows + 7) / 8);

@@ -93,7 +93,7 @@ int make_dims(const cca_config_t *cfg, cca::Dims &d) {
 size_t esize(const cca::Dims &d) { return d.bf16 ? 2 : 4; }
 
 struct PrefillLayout {
-  size_t status, P, q, k, v, o, total;
+  size_t status, wo16, P, q, k, v, o, total;
 };
 
 PrefillLayout prefill_layout(const cca::Dims &d, int B, int S) {
@@ -101,7 +101,8 @@ PrefillLayout prefill_layout(const cca::Dims &d, int B, int S) {
   const size_t M = static_cast<size_t>(B) * S, es = esize(d);
   size_t off = 0;
   L.status = off; off += 256;
-  L.P = off; off += align256(M * d.NQKV * es);
+  L.wo16 = off; off += d.bf16 ? align256(static_cast<size_t>(d.E) * d.NQ * 2) : 0;
+  L.P = off; off += align256(M * d.NQKV * 4);   // projections stay float32
   L.q = off; off += align256(M * d.NQ * es);
   L.k = off; off += align256(M * d.NKV * es);
   L.v = off; off += align256(M * d.NKV * es);
@@ -120,8 +121,8 @@ CacheLayout cache_layout(const cca::Dims &d, int B, int max_seq) {
   size_t off = 0;
   L.k = off; off += align256(static_cast<size_t>(B) * d.Hkv * max_seq * d.DL * es);
   L.v = off; off += align256(static_cast<size_t>(B) * d.Hkv * max_seq * d.DL * es);
-  L.conv = off; off += align256(static_cast<size_t>(B) * (d.KC - 1) * (d.NQ + d.NKV) * es);
-  L.vshift = off; off += align256(static_cast<size_t>(B) * (d.NKV - d.NKV / 2) * es);
+  L.conv = off; off += align256(static_cast<size_t>(B) * (d.KC - 1) * (d.NQ + d.NKV) * 4);
+  L.vshift = off; off += align256(static_cast<size_t>(B) * (d.NKV - d.NKV / 2) * 4);
   L.lengths = off; off += align256(static_cast<size_t>(B) * 4);
   L.status = off; off += 256;
   L.total = off;
@@ -138,13 +139,14 @@ int check_cache(const cca::Dims &d, const cca_cache_t *c) {
   return CCA_OK;
 }
 
-int gemm_dispatch(int bf16, const void *A, const void *B, void *C, int M, int N, int K,
-                  int *status, cudaStream_t st) {
+// dtype of the operands: CCA_F32 (CUDA cores), CCA_BF16 or CCA_F16 (tensor cores).
+int gemm_dispatch(int dtype, int out_f32, const void *A, const void *B, void *C, int M, int N,
+                  int K, int *status, cudaStream_t st) {
   cudaError_t e;
-  if (bf16 && K % 8 == 0)
-    e = cca::gemm_bf16_tcgen05(A, B, C, M, N, K, status, st);
+  if (dtype != CCA_F32)
+    e = cca::gemm_tcgen05(A, B, C, M, N, K, dtype == CCA_F16, out_f32, status, st);
   else
-    e = cca::gemm_simt(bf16, A, B, C, M, N, K, st);
+    e = cca::gemm_simt(0, A, B, C, M, N, K, st);
   return e == cudaSuccess ? CCA_OK : cuda_fail(e, "projection GEMM launch");
 }
 
@@ -321,31 +323,44 @@ CCA_API int cca_prefill_forward(const cca_config_t *cfg, const cca_weights_t *w,
   const int M = batch * seq;
   CallRecorder rec(st);
   rec.mark();
+  // 16-bit layers: the up-projection runs on float16 operands (the attention output is
+  // float16), so W_o is converted once per call.
+  void *wo = const_cast<void *>(w->w_o);
+  if (d.bf16) {
+    wo = ws + L.wo16;
+    if ((e = cca::convert_bf16_to_f16(w->w_o, wo, static_cast<size_t>(d.E) * d.NQ, status, st)) !=
+        cudaSuccess)
+      return cuda_fail(e, "W_o conversion launch");
+  }
+  rec.mark();
   void *P = ws + L.P, *q = ws + L.q, *o = ws + L.o;
   void *k = cache ? cache->k : ws + L.k;
   void *v = cache ? cache->v : ws + L.v;
   const int kv_stride = cache ? cache->max_seq : seq;
 
-  if ((rc = gemm_dispatch(d.bf16, x, w->w_qkv, P, M, d.NQKV, d.E, status, st))) return rc;
+  const int dt = d.bf16 ? CCA_BF16 : CCA_F32;
+  if ((rc = gemm_dispatch(dt, 1, x, w->w_qkv, P, M, d.NQKV, d.E, status, st))) return rc;
   rec.mark();
   cca::StencilArgs sa;
-  sa.P = P;
+  sa.P = static_cast<const float *>(P);
   sa.conv_seq = w->conv_seq;
   sa.conv_chan = w->conv_chan;
   sa.q = q;
   sa.k = k;
   sa.v = v;
   sa.kv_stride = kv_stride;
-  sa.conv_state = cache ? cache->conv_state : nullptr;
-  sa.vshift_state = cache ? cache->vshift_state : nullptr;
+  sa.conv_state = cache ? static_cast<float *>(cache->conv_state) : nullptr;
+  sa.vshift_state = cache ? static_cast<float *>(cache->vshift_state) : nullptr;
   sa.lengths = cache ? cache->lengths : nullptr;
   sa.write_state = cache != nullptr;
+  sa.status = status;
   if ((e = cca::latent_stencil(d, sa, st)) != cudaSuccess) return cuda_fail(e, "stencil launch");
   rec.mark();
   if ((e = cca::latent_attention(d, q, k, v, kv_stride, o, status, st)) != cudaSuccess)
     return cuda_fail(e, "attention launch");
   rec.mark();
-  if ((rc = gemm_dispatch(d.bf16, o, w->w_o, y, M, d.E, d.NQ, status, st))) return rc;
+  if ((rc = gemm_dispatch(d.bf16 ? CCA_F16 : CCA_F32, 0, o, wo, y, M, d.E, d.NQ, status, st)))
+    return rc;
   rec.mark();
   return ok();
 }
@@ -379,8 +394,8 @@ CCA_API int cca_decode_step(const cca_config_t *cfg, const cca_weights_t *w, con
   a.y = y;
   a.k_cache = cache->k;
   a.v_cache = cache->v;
-  a.conv_state = cache->conv_state;
-  a.vshift_state = cache->vshift_state;
+  a.conv_state = static_cast<float *>(cache->conv_state);
+  a.vshift_state = static_cast<float *>(cache->vshift_state);
   a.lengths = cache->lengths;
   a.status = cache->status;
   a.max_seq = cache->max_seq;
@@ -402,6 +417,7 @@ CCA_API int cca_cache_check(cca_cache_t *cache, void *stream) {
   if (s == 0) return ok();
   if ((e = cudaMemset(cache->status, 0, sizeof(int))) != cudaSuccess) return cuda_fail(e, "status clear");
   if (s == cca::DEV_CACHE_FULL) return fail(CCA_ERR_CACHE_FULL, "a sequence reached max_seq");
+  if (s == cca::DEV_RANGE) return fail(CCA_ERR_RANGE, "a latent key or value exceeded the float16 range");
   return fail(CCA_ERR_DEVICE, "kernel status %d", s);
 }
 
@@ -412,18 +428,26 @@ CCA_API int cca_workspace_status(const void *workspace, void *stream) {
   int s = 0;
   if ((e = cudaMemcpy(&s, workspace, sizeof(int), cudaMemcpyDeviceToHost)) != cudaSuccess)
     return cuda_fail(e, "status read");
+  if (s == cca::DEV_RANGE) return fail(CCA_ERR_RANGE, "a latent query, key or value exceeded the float16 range");
   if (s) return fail(CCA_ERR_DEVICE, "kernel status %d (bounded wait ran out)", s);
   return ok();
 }
 
-CCA_API int cca_gemm(int dtype, const void *A, const void *B, void *C, int M, int N, int K,
+CCA_API int cca_gemm(int dtype, int out_dtype, const void *A, const void *B, void *C, int M, int N, int K,
                      int *status, void *stream) {
-  if (dtype != CCA_F32 && dtype != CCA_BF16) return fail(CCA_ERR_INVALID_ARG, "bad dtype %d", dtype);
+  if ((dtype != CCA_F32 && dtype != CCA_BF16 && dtype != CCA_F16) ||
+      (out_dtype != CCA_F32 && out_dtype != CCA_BF16))
+    return fail(CCA_ERR_INVALID_ARG, "bad dtype %d / %d", dtype, out_dtype);
   if (M < 0 || N < 0 || K <= 0) return fail(CCA_ERR_INVALID_ARG, "bad shape %d x %d x %d", M, N, K);
   if (M > 0 && N > 0 && (!A || !B || !C)) return fail(CCA_ERR_INVALID_ARG, "NULL operand");
   if (!aligned16(A) || !aligned16(B) || !aligned16(C)) return fail(CCA_ERR_ALIGNMENT, "operands must be 16-byte aligned");
   if (injected_launch_failure()) return fail(CCA_ERR_CUDA, "injected launch failure");
-  int rc = gemm_dispatch(dtype == CCA_BF16, A, B, C, M, N, K, status, static_cast<cudaStream_t>(stream));
+  if (dtype == CCA_F32 && out_dtype != CCA_F32)
+    return fail(CCA_ERR_UNSUPPORTED, "float32 operands give a float32 result");
+  if (dtype != CCA_F32 && K % 8 != 0)
+    return fail(CCA_ERR_UNSUPPORTED, "16-bit rows must be a multiple of 16 bytes (K %% 8 == 0)");
+  int rc = gemm_dispatch(dtype, out_dtype == CCA_F32, A, B, C, M, N, K, status,
+                         static_cast<cudaStream_t>(stream));
   return rc ? rc : ok();
 }
 
@@ -441,7 +465,7 @@ CCA_API int cca_stage_stencil(const cca_config_t *cfg, const void *P, int batch,
   d.B = batch;
   d.S = seq;
   cca::StencilArgs sa{};
-  sa.P = P;
+  sa.P = static_cast<const float *>(P);
   sa.conv_seq = conv_seq;
   sa.conv_chan = conv_chan;
   sa.q = q;

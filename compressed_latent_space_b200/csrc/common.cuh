@@ -4,6 +4,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -12,15 +13,41 @@ namespace cca {
 // ----------------------------------------------------------------------------- elements
 __device__ __forceinline__ float to_f32(float v) { return v; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
+__device__ __forceinline__ float to_f32(__half v) { return __half2float(v); }
 template <typename T> __device__ __forceinline__ T from_f32(float v);
 template <> __device__ __forceinline__ float from_f32<float>(float v) { return v; }
 template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float v) {
   return __float2bfloat16_rn(v);
 }
+template <> __device__ __forceinline__ __half from_f32<__half>(float v) {
+  return __float2half_rn(v);
+}
+
+// Element type of the latent queries, keys and values (and of the K/V cache) of a layer whose
+// activations are T.  16-bit layers keep them in float16: three more significand bits than
+// bfloat16 at the same size and tensor-core rate (normalised q and k are bounded by sqrt(d~);
+// a value beyond the float16 range is reported through the status word).
+template <typename T> struct LatentType { using type = __half; };
+template <> struct LatentType<float> { using type = float; };
+constexpr float kF16Max = 65504.f;
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t *>(&h);
+}
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t *>(&h);
+}
+
+// Splits a pair of floats into bf16x2 leading terms and bf16x2 remainders (v = hi + lo to
+// about 16 significand bits).
+__device__ __forceinline__ void split_bf16x2(float2 v, uint32_t &hi, uint32_t &lo) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(v.x, v.y);
+  const float2 hf = __bfloat1622float2(h);
+  hi = *reinterpret_cast<uint32_t *>(&h);
+  lo = pack_bf16x2(v.x - hf.x, v.y - hf.y);
 }
 
 // Loads 8 consecutive elements (16 bytes for bf16, 32 for f32) into floats.
@@ -30,6 +57,16 @@ __device__ __forceinline__ void load8(const __nv_bfloat16 *p, float (&o)[8]) {
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     float2 f = __bfloat1622float2(h[i]);
+    o[2 * i] = f.x;
+    o[2 * i + 1] = f.y;
+  }
+}
+__device__ __forceinline__ void load8(const __half *p, float (&o)[8]) {
+  uint4 u = *reinterpret_cast<const uint4 *>(p);
+  const __half2 *h = reinterpret_cast<const __half2 *>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float2 f = __half22float2(h[i]);
     o[2 * i] = f.x;
     o[2 * i + 1] = f.y;
   }
@@ -55,10 +92,19 @@ __device__ __forceinline__ void store8(float *p, const float (&v)[8]) {
 
 // ----------------------------------------------------------------------------- status
 // Codes a kernel can leave in its status word (first error wins).
-enum : int { DEV_OK = 0, DEV_WAIT_TIMEOUT = 1, DEV_CACHE_FULL = 2 };
+enum : int { DEV_OK = 0, DEV_WAIT_TIMEOUT = 1, DEV_CACHE_FULL = 2, DEV_RANGE = 3 };
+
 
 __device__ __forceinline__ void report(int *status, int code) {
   if (status) atomicCAS(status, 0, code);
+}
+
+// Records DEV_RANGE when a latent about to be stored as float16 is not finite in float16.
+template <typename TL>
+__device__ __forceinline__ void check_latent(float v, int *status) {
+  if constexpr (sizeof(TL) == 2) {
+    if (!(fabsf(v) <= kF16Max)) report(status, DEV_RANGE);
+  }
 }
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {
@@ -249,10 +295,11 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes
   return d;
 }
 
-// Instruction descriptor of tcgen05.mma kind::f16 with bf16 A and B, f32 accumulator.
-// a_mn / b_mn select MN-major (transposed) operands.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn, int b_mn) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(a_mn) << 15) |
+// Instruction descriptor of tcgen05.mma kind::f16 with f32 accumulator; A and B both bf16
+// (ab_f16 == 0) or both f16 (ab_f16 == 1).  a_mn / b_mn select MN-major (transposed) operands.
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, int a_mn, int b_mn, int ab_f16 = 0) {
+  return (1u << 4) | (static_cast<uint32_t>(ab_f16 ? 0 : 1) << 7) |
+         (static_cast<uint32_t>(ab_f16 ? 0 : 1) << 10) | (static_cast<uint32_t>(a_mn) << 15) |
          (static_cast<uint32_t>(b_mn) << 16) | (static_cast<uint32_t>(N >> 3) << 17) |
          (static_cast<uint32_t>(M >> 4) << 24);
 }
@@ -263,6 +310,15 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a
                                                const uint32_t (&b)[2]) {
   asm volatile(
       "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+// m16n8k16 f16 x f16 -> f32.
+__device__ __forceinline__ void mma_f16_16816(float (&d)[4], const uint32_t (&a)[4],
+                                              const uint32_t (&b)[2]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
       "{%8, %9}, {%0, %1, %2, %3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));

@@ -26,8 +26,10 @@ constexpr int CHUNK = 256;        // keys per split-KV block
 // C[M, N] = A[M, K] * B[N, K]^T for small M (the batch), bf16 operands on mma.sync.
 // Grid (N / NB, ksplit, ceil(M/64)); 4 warps share the K slice of the block and reduce
 // through shared memory.  OUT_F32: write fp32 partial sums to C + ks*M*N; else write bf16.
-template <int NB, bool OUT_F32>
-__global__ void __launch_bounds__(128) skinny_gemm_kernel(const __nv_bfloat16 *__restrict__ A,
+// TA = float: A is float32 and enters the tensor cores as two bf16 terms, hi = bf16(a) and
+// lo = bf16(a - hi), so the product keeps ~16 significand bits of A at no extra traffic.
+template <int NB, bool OUT_F32, typename TA = __nv_bfloat16>
+__global__ void __launch_bounds__(128) skinny_gemm_kernel(const TA *__restrict__ A,
                                                           const __nv_bfloat16 *__restrict__ B,
                                                           void *__restrict__ C, int M, int N,
                                                           int K, int k_per_split) {
@@ -57,15 +59,33 @@ __global__ void __launch_bounds__(128) skinny_gemm_kernel(const __nv_bfloat16 *_
 #pragma unroll
     for (int mt = 0; mt < 4; ++mt) {
       const int ma = mbase + mt * 16 + gr, mb = ma + 8;
-      uint32_t af[4];
-      const __nv_bfloat16 *pa = A + static_cast<size_t>(ma) * K + k0 + 2 * qc;
-      const __nv_bfloat16 *pb = A + static_cast<size_t>(mb) * K + k0 + 2 * qc;
-      af[0] = ma < M ? *reinterpret_cast<const uint32_t *>(pa) : 0u;
-      af[1] = mb < M ? *reinterpret_cast<const uint32_t *>(pb) : 0u;
-      af[2] = ma < M ? *reinterpret_cast<const uint32_t *>(pa + 8) : 0u;
-      af[3] = mb < M ? *reinterpret_cast<const uint32_t *>(pb + 8) : 0u;
+      const TA *pa = A + static_cast<size_t>(ma) * K + k0 + 2 * qc;
+      const TA *pb = A + static_cast<size_t>(mb) * K + k0 + 2 * qc;
+      if constexpr (sizeof(TA) == 2) {
+        uint32_t af[4];
+        af[0] = ma < M ? *reinterpret_cast<const uint32_t *>(pa) : 0u;
+        af[1] = mb < M ? *reinterpret_cast<const uint32_t *>(pb) : 0u;
+        af[2] = ma < M ? *reinterpret_cast<const uint32_t *>(pa + 8) : 0u;
+        af[3] = mb < M ? *reinterpret_cast<const uint32_t *>(pb + 8) : 0u;
 #pragma unroll
-      for (int j = 0; j < NT; ++j) mma_bf16_16816(acc[mt][j], af, bf[j]);
+        for (int j = 0; j < NT; ++j) mma_bf16_16816(acc[mt][j], af, bf[j]);
+      } else {
+        const float2 z = make_float2(0.f, 0.f);
+        const float2 v0 = ma < M ? *reinterpret_cast<const float2 *>(pa) : z;
+        const float2 v1 = mb < M ? *reinterpret_cast<const float2 *>(pb) : z;
+        const float2 v2 = ma < M ? *reinterpret_cast<const float2 *>(pa + 8) : z;
+        const float2 v3 = mb < M ? *reinterpret_cast<const float2 *>(pb + 8) : z;
+        uint32_t hi[4], lo[4];
+        split_bf16x2(v0, hi[0], lo[0]);
+        split_bf16x2(v1, hi[1], lo[1]);
+        split_bf16x2(v2, hi[2], lo[2]);
+        split_bf16x2(v3, hi[3], lo[3]);
+#pragma unroll
+        for (int j = 0; j < NT; ++j) {
+          mma_bf16_16816(acc[mt][j], hi, bf[j]);
+          mma_bf16_16816(acc[mt][j], lo, bf[j]);
+        }
+      }
     }
   }
 #pragma unroll
@@ -93,10 +113,12 @@ __global__ void __launch_bounds__(128) skinny_gemm_kernel(const __nv_bfloat16 *_
 // ------------------------------------------------------------------ D2 decode stencil
 template <typename T>
 struct D2Params {
+  using TL = typename LatentType<T>::type;
   const float *p_part;
   int ksplit;
   const float *conv_seq, *conv_chan;
-  T *k_cache, *v_cache, *conv_state, *vshift_state;
+  TL *k_cache, *v_cache;
+  float *conv_state, *vshift_state;
   int *lengths, *status;
   float *q_new;
   int B, H, Hkv, G, DL, NQ, NKV, NQKV, KC, max_seq;
@@ -106,6 +128,7 @@ struct D2Params {
 
 template <typename T>
 __global__ void __launch_bounds__(128) decode_stencil_kernel(const D2Params<T> p) {
+  using TL = typename D2Params<T>::TL;
   extern __shared__ float sm[];
   const int g = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
   const int G = p.G, DL = p.DL, CH = (G + 2) * DL, QKC = (G + 1) * DL;
@@ -126,11 +149,11 @@ __global__ void __launch_bounds__(128) decode_stencil_kernel(const D2Params<T> p
     const int gc = gch(c);
     float s = 0.f;
     for (int ks = 0; ks < p.ksplit; ++ks) s += p.p_part[(static_cast<size_t>(ks) * p.B + b) * p.NQKV + gc];
-    pn[c] = to_f32(from_f32<T>(s));
+    pn[c] = s;
   }
   __syncthreads();
   const int KC1 = p.KC - 1, W = p.NQ + p.NKV;
-  T *cs = p.conv_state + static_cast<size_t>(b) * KC1 * W;
+  float *cs = p.conv_state + static_cast<size_t>(b) * KC1 * W;
   for (int c = tid; c < QKC; c += blockDim.x) {
     const int gc = gch(c);
     const float *w = p.conv_seq + static_cast<size_t>(gc) * p.KC;
@@ -189,36 +212,40 @@ __global__ void __launch_bounds__(128) decode_stencil_kernel(const D2Params<T> p
       qd[ip] = x1;
       qd[ip + HALF] = x2;
     } else {
-      T *kd = p.k_cache + ((static_cast<size_t>(b) * p.Hkv + g) * p.max_seq + L) * DL;
-      kd[ip] = from_f32<T>(x1);
-      kd[ip + HALF] = from_f32<T>(x2);
+      auto *kd = p.k_cache + ((static_cast<size_t>(b) * p.Hkv + g) * p.max_seq + L) * DL;
+      check_latent<TL>(x1, p.status);
+      check_latent<TL>(x2, p.status);
+      kd[ip] = from_f32<TL>(x1);
+      kd[ip + HALF] = from_f32<TL>(x2);
     }
   }
   // value with the value-shift, appended at position L
   const int vhalf = p.NKV / 2;
-  T *vs = p.vshift_state + static_cast<size_t>(b) * (p.NKV - vhalf);
+  float *vs = p.vshift_state + static_cast<size_t>(b) * (p.NKV - vhalf);
   for (int c = tid; c < DL; c += blockDim.x) {
     const int vc = g * DL + c;
     const bool shifted = vc >= vhalf;
     const float val = ((p.flags & F_VALUE_SHIFT) && shifted) ? to_f32(vs[vc - vhalf]) : pn[QKC + c];
-    p.v_cache[((static_cast<size_t>(b) * p.Hkv + g) * p.max_seq + L) * DL + c] = from_f32<T>(val);
+    check_latent<TL>(val, p.status);
+    p.v_cache[((static_cast<size_t>(b) * p.Hkv + g) * p.max_seq + L) * DL + c] = from_f32<TL>(val);
   }
   __syncthreads();   // every read of the old state is done
   for (int c = tid; c < QKC; c += blockDim.x) {
     const int gc = gch(c);
     for (int j = 0; j + 1 < KC1; ++j) cs[static_cast<size_t>(j) * W + gc] = cs[static_cast<size_t>(j + 1) * W + gc];
-    if (KC1 > 0) cs[static_cast<size_t>(KC1 - 1) * W + gc] = from_f32<T>(pn[c]);
+    if (KC1 > 0) cs[static_cast<size_t>(KC1 - 1) * W + gc] = pn[c];
   }
   for (int c = tid; c < DL; c += blockDim.x) {
     const int vc = g * DL + c;
-    if (vc >= vhalf) vs[vc - vhalf] = from_f32<T>(pn[QKC + c]);
+    if (vc >= vhalf) vs[vc - vhalf] = pn[QKC + c];
   }
 }
 
 // ------------------------------------------------------------------ D3 split-KV attention
-template <typename T>
+template <typename TL>
 __global__ void __launch_bounds__(128) decode_attn_kernel(
-    const float *__restrict__ q_new, const T *__restrict__ k_cache, const T *__restrict__ v_cache,
+    const float *__restrict__ q_new, const TL *__restrict__ k_cache,
+    const TL *__restrict__ v_cache,
     const int *__restrict__ lengths, float *__restrict__ part_o, float *__restrict__ part_ml, int H,
     int Hkv, int G, int DL, int max_seq, int nchunk, float scale_log2) {
   extern __shared__ float sm[];
@@ -246,8 +273,8 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(
   }
   for (int i = tid; i < G * DL; i += blockDim.x)
     qs[i] = q_new[(static_cast<size_t>(b) * H + g * G) * DL + i] * scale_log2;
-  const T *kb = k_cache + ((static_cast<size_t>(b) * Hkv + g) * max_seq + s0) * DL;
-  const T *vb = v_cache + ((static_cast<size_t>(b) * Hkv + g) * max_seq + s0) * DL;
+  const auto *kb = k_cache + ((static_cast<size_t>(b) * Hkv + g) * max_seq + s0) * DL;
+  const TL *vb = v_cache + ((static_cast<size_t>(b) * Hkv + g) * max_seq + s0) * DL;
   for (int i = tid; i < n * DL / 8; i += blockDim.x) {
     const int r = i / (DL / 8), c = (i % (DL / 8)) * 8;
     float k8[8], v8[8];
@@ -301,10 +328,9 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(
 }
 
 // ------------------------------------------------------------------ D3b merge
-template <typename T>
 __global__ void decode_merge_kernel(const float *__restrict__ part_o,
                                     const float *__restrict__ part_ml, const int *__restrict__ lengths,
-                                    T *__restrict__ o, int H, int DL, int max_seq, int nchunk) {
+                                    float *__restrict__ o, int H, int DL, int max_seq, int nchunk) {
   const int b = blockIdx.x;
   const bool full = lengths[b] >= max_seq;
   const int nused = full ? 0 : min(nchunk, (lengths[b] + 1 + CHUNK - 1) / CHUNK);
@@ -319,7 +345,7 @@ __global__ void decode_merge_kernel(const float *__restrict__ part_o,
       l += w * ml[2 * c + 1];
       acc += w * part_o[((static_cast<size_t>(b) * H + h) * nchunk + c) * DL + d];
     }
-    o[static_cast<size_t>(b) * H * DL + i] = from_f32<T>(nused > 0 ? acc / l : 0.f);
+    o[static_cast<size_t>(b) * H * DL + i] = nused > 0 ? acc / l : 0.f;
   }
 }
 
@@ -344,20 +370,18 @@ inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255);
 size_t decode_workspace_bytes(const Dims &d, int max_seq) {
   const int nchunk = (max_seq + CHUNK - 1) / CHUNK;
   const int ks = d.bf16 ? decode_ksplit(d) : 1;
-  const size_t es = d.bf16 ? 2 : 4;
   size_t s = 0;
   s += align256(static_cast<size_t>(ks) * d.B * d.NQKV * 4);
   s += align256(static_cast<size_t>(d.B) * d.H * d.DL * 4);
   s += align256(static_cast<size_t>(d.B) * d.H * nchunk * d.DL * 4);
   s += align256(static_cast<size_t>(d.B) * d.H * nchunk * 2 * 4);
-  s += align256(static_cast<size_t>(d.B) * d.NQ * es);
+  s += align256(static_cast<size_t>(d.B) * d.NQ * 4);
   return s;
 }
 
 void decode_workspace_carve(const Dims &d, int max_seq, void *ws, DecodeArgs &a) {
   const int nchunk = (max_seq + CHUNK - 1) / CHUNK;
   const int ks = d.bf16 ? decode_ksplit(d) : 1;
-  const size_t es = d.bf16 ? 2 : 4;
   char *p = static_cast<char *>(ws);
   a.p_part = reinterpret_cast<float *>(p);
   p += align256(static_cast<size_t>(ks) * d.B * d.NQKV * 4);
@@ -391,15 +415,16 @@ static cudaError_t decode_typed(const Dims &d, const DecodeArgs &a, cudaStream_t
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   mark();
   // D2
+  using TL = typename LatentType<T>::type;
   D2Params<T> p2;
   p2.p_part = a.p_part;
   p2.ksplit = sizeof(T) == 2 ? a.ksplit : 1;
   p2.conv_seq = a.conv_seq;
   p2.conv_chan = a.conv_chan;
-  p2.k_cache = static_cast<T *>(a.k_cache);
-  p2.v_cache = static_cast<T *>(a.v_cache);
-  p2.conv_state = static_cast<T *>(a.conv_state);
-  p2.vshift_state = static_cast<T *>(a.vshift_state);
+  p2.k_cache = static_cast<TL *>(a.k_cache);
+  p2.v_cache = static_cast<TL *>(a.v_cache);
+  p2.conv_state = a.conv_state;
+  p2.vshift_state = a.vshift_state;
   p2.lengths = a.lengths;
   p2.status = a.status;
   p2.q_new = a.q_new;
@@ -417,25 +442,26 @@ static cudaError_t decode_typed(const Dims &d, const DecodeArgs &a, cudaStream_t
   const size_t sm3 = (static_cast<size_t>(d.G) * d.DL + d.G * CHUNK + CHUNK * (d.DL + 1) +
                       CHUNK * d.DL + 2 * d.G) * 4;
   if (sm3 > 48 * 1024) {
-    e = cudaFuncSetAttribute(decode_attn_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(decode_attn_kernel<TL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(sm3));
     if (e != cudaSuccess) return e;
   }
-  decode_attn_kernel<T><<<dim3(a.nchunk, d.Hkv, d.B), 128, sm3, st>>>(
-      a.q_new, static_cast<const T *>(a.k_cache), static_cast<const T *>(a.v_cache), a.lengths,
+  decode_attn_kernel<TL><<<dim3(a.nchunk, d.Hkv, d.B), 128, sm3, st>>>(
+      a.q_new, static_cast<const TL *>(a.k_cache), static_cast<const TL *>(a.v_cache),
+      a.lengths,
       a.part_o, a.part_ml, d.H, d.Hkv, d.G, d.DL, a.max_seq, a.nchunk, scale_log2);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   mark();
-  decode_merge_kernel<T><<<d.B, 256, 0, st>>>(a.part_o, a.part_ml, a.lengths,
-                                               static_cast<T *>(a.o), d.H, d.DL, a.max_seq,
+  decode_merge_kernel<<<d.B, 256, 0, st>>>(a.part_o, a.part_ml, a.lengths,
+                                            static_cast<float *>(a.o), d.H, d.DL, a.max_seq,
                                                a.nchunk);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   mark();
   // D4
   if constexpr (sizeof(T) == 2) {
     dim3 g4((d.E + 15) / 16, 1, (d.B + 63) / 64);
-    skinny_gemm_kernel<16, false><<<g4, 128, 0, st>>>(
-        static_cast<const __nv_bfloat16 *>(a.o), static_cast<const __nv_bfloat16 *>(a.w_o),
+    skinny_gemm_kernel<16, false, float><<<g4, 128, 0, st>>>(
+        static_cast<const float *>(a.o), static_cast<const __nv_bfloat16 *>(a.w_o),
         a.y, d.B, d.E, d.NQ, d.NQ);
   } else {
     e = gemm_simt(0, a.o, a.w_o, a.y, d.B, d.E, d.NQ, st);
@@ -451,8 +477,7 @@ static cudaError_t decode_typed(const Dims &d, const DecodeArgs &a, cudaStream_t
 cudaError_t decode_step(const Dims &d, const DecodeArgs &a, cudaStream_t st,
                         const StageMarker &mark) {
   if (d.B == 0) return cudaSuccess;
-  return d.bf16 ? decode_typed<__nv_bfloat16>(d, a, st, mark)
-                : decode_typed<float>(d, a, st, mark);
+  return d.bf16 ? decode_typed<__nv_bfloat16>(d, a, st, mark) : decode_typed<float>(d, a, st, mark);
 }
 
 }  // namespace cca

@@ -3,7 +3,7 @@
 // Used for the down-projection x W_qkv^T and the up-projection o W_o^T of the layer
 // (gist.science explainer, 2. Methodology, Core Mechanism: "Down-Projection"; the result of
 // the latent attention returns to width E through one output matrix).  Both operands are
-// K-major (PyTorch Linear layout), bf16, accumulated in fp32 in tensor memory.
+// K-major (PyTorch Linear layout), bf16 or f16, accumulated in fp32 in tensor memory.
 //
 // Persistent, warp-specialised kernel, one CTA per SM:
 //   warp 0  : TMA producer, 4-stage ring of 128x64 (A) + 256x64 (B) tiles, 128B swizzle
@@ -38,9 +38,10 @@ struct Bars {
 };
 constexpr size_t SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + sizeof(Bars);
 
+template <typename OutT, int AB_F16>
 __global__ void __launch_bounds__(THREADS, 1)
     gemm_bf16_kernel(const __grid_constant__ CUtensorMap mapA,
-                     const __grid_constant__ CUtensorMap mapB, __nv_bfloat16 *__restrict__ C,
+                     const __grid_constant__ CUtensorMap mapB, OutT *__restrict__ C,
                      int M, int N, int K, int *status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -98,7 +99,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, 0, 0);
+      constexpr uint32_t idesc = idesc_f16_f32(BM, BN, 0, 0, AB_F16);
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
@@ -150,21 +151,28 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         const int n = n0 + c * 32;
         if (m < M && n < N) {
-          __nv_bfloat16 *dst = C + static_cast<size_t>(m) * N + n;
+          OutT *dst = C + static_cast<size_t>(m) * N + n;
           if (n + 32 <= N && (N & 7) == 0) {
+            if constexpr (sizeof(OutT) == 2) {
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              uint4 u;
-              u.x = pack_bf16x2(__uint_as_float(r[8 * v + 0]), __uint_as_float(r[8 * v + 1]));
-              u.y = pack_bf16x2(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3]));
-              u.z = pack_bf16x2(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5]));
-              u.w = pack_bf16x2(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7]));
-              reinterpret_cast<uint4 *>(dst)[v] = u;
+              for (int v = 0; v < 4; ++v) {
+                uint4 u;
+                u.x = pack_bf16x2(__uint_as_float(r[8 * v + 0]), __uint_as_float(r[8 * v + 1]));
+                u.y = pack_bf16x2(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3]));
+                u.z = pack_bf16x2(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5]));
+                u.w = pack_bf16x2(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7]));
+                reinterpret_cast<uint4 *>(dst)[v] = u;
+              }
+            } else {
+#pragma unroll
+              for (int v = 0; v < 8; ++v)
+                reinterpret_cast<uint4 *>(dst)[v] =
+                    make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
             }
           } else {
 #pragma unroll
             for (int j = 0; j < 32; ++j)
-              if (n + j < N) dst[j] = __float2bfloat16_rn(__uint_as_float(r[j]));
+              if (n + j < N) dst[j] = from_f32<OutT>(__uint_as_float(r[j]));
           }
         }
       }
@@ -199,14 +207,14 @@ EncodeTiledFn encode_fn() {
 }
 
 // 2-D bf16 row-major tensor [rows, cols] -> box [box_rows, 64 cols], 128B swizzle.
-bool make_map_2d(CUtensorMap *map, const void *ptr, int rows, int cols, int box_rows) {
+bool make_map_2d(CUtensorMap *map, const void *ptr, int rows, int cols, int box_rows, int f16) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
   cuuint32_t box[2] = {static_cast<cuuint32_t>(BK), static_cast<cuuint32_t>(box_rows)};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides,
+  CUresult r = fn(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -225,16 +233,12 @@ int num_sms() {
   return n;
 }
 
-cudaError_t gemm_bf16_tcgen05(const void *A, const void *B, void *C, int M, int N, int K,
-                              int *status, cudaStream_t st) {
-  if (M <= 0 || N <= 0) return cudaSuccess;
-  if (K % 8 != 0) return cudaErrorInvalidValue;   // TMA row pitch must be a multiple of 16 B
-  CUtensorMap ma, mb;
-  if (!make_map_2d(&ma, A, M, K, BM) || !make_map_2d(&mb, B, N, K, BN))
-    return cudaErrorInvalidValue;
+template <typename OutT, int AB_F16>
+static cudaError_t launch_gemm(const CUtensorMap &ma, const CUtensorMap &mb, void *C, int M,
+                               int N, int K, int *status, cudaStream_t st) {
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_bf16_kernel,
+    cudaError_t e = cudaFuncSetAttribute(gemm_bf16_kernel<OutT, AB_F16>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(SMEM_BYTES));
     if (e != cudaSuccess) return e;
@@ -242,8 +246,61 @@ cudaError_t gemm_bf16_tcgen05(const void *A, const void *B, void *C, int M, int 
   }
   const int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
   const int grid = tiles < num_sms() ? tiles : num_sms();
-  gemm_bf16_kernel<<<grid, THREADS, SMEM_BYTES, st>>>(
-      ma, mb, static_cast<__nv_bfloat16 *>(C), M, N, K, status);
+  gemm_bf16_kernel<OutT, AB_F16><<<grid, THREADS, SMEM_BYTES, st>>>(ma, mb, static_cast<OutT *>(C), M,
+                                                             N, K, status);
+  return cudaGetLastError();
+}
+
+cudaError_t gemm_tcgen05(const void *A, const void *B, void *C, int M, int N, int K, int ab_f16,
+                         int out_f32, int *status, cudaStream_t st) {
+  if (M <= 0 || N <= 0) return cudaSuccess;
+  if (K % 8 != 0) return cudaErrorInvalidValue;   // TMA row pitch must be a multiple of 16 B
+  CUtensorMap ma, mb;
+  if (!make_map_2d(&ma, A, M, K, BM, ab_f16) || !make_map_2d(&mb, B, N, K, BN, ab_f16))
+    return cudaErrorInvalidValue;
+  if (ab_f16)
+    return out_f32 ? launch_gemm<float, 1>(ma, mb, C, M, N, K, status, st)
+                   : launch_gemm<__nv_bfloat16, 1>(ma, mb, C, M, N, K, status, st);
+  return out_f32 ? launch_gemm<float, 0>(ma, mb, C, M, N, K, status, st)
+                 : launch_gemm<__nv_bfloat16, 0>(ma, mb, C, M, N, K, status, st);
+}
+
+}  // namespace cca
+
+namespace cca {
+namespace {
+
+__global__ void __launch_bounds__(256) bf16_to_f16_kernel(const __nv_bfloat16 *__restrict__ src,
+                                                          __half *__restrict__ dst, size_t n8,
+                                                          int *status) {
+  for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    float v[8];
+    load8(src + i * 8, v);
+    bool ok = true;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) ok = ok && (fabsf(v[e]) <= kF16Max);
+    if (!ok) report(status, DEV_RANGE);
+    uint4 u;
+    u.x = pack_f16x2(v[0], v[1]);
+    u.y = pack_f16x2(v[2], v[3]);
+    u.z = pack_f16x2(v[4], v[5]);
+    u.w = pack_f16x2(v[6], v[7]);
+    reinterpret_cast<uint4 *>(dst)[i] = u;
+  }
+}
+
+}  // namespace
+
+cudaError_t convert_bf16_to_f16(const void *src, void *dst, size_t n, int *status, cudaStream_t st) {
+  if (n == 0) return cudaSuccess;
+  if (n % 8) return cudaErrorInvalidValue;
+  const size_t n8 = n / 8;
+  size_t blocks = (n8 + 255) / 256;
+  const size_t cap = static_cast<size_t>(num_sms()) * 8;
+  if (blocks > cap) blocks = cap;
+  bf16_to_f16_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+      static_cast<const __nv_bfloat16 *>(src), static_cast<__half *>(dst), n8, status);
   return cudaGetLastError();
 }
 

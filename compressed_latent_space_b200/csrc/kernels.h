@@ -17,7 +17,7 @@ struct Dims {
   unsigned flags = 0;
   float eps = 1e-6f;
   float rope_base = 10000.f;
-  int bf16 = 1;                  // element type of activations / weights / cache
+  int bf16 = 1;                  // activations and weights bf16 (latents and cache float16)
 };
 
 // Called after each kernel launch of a C-ABI call; records a timing event when stage
@@ -32,26 +32,31 @@ struct StageMarker {
 
 enum : unsigned { F_QK_MEAN = 1u, F_VALUE_SHIFT = 2u, F_QK_NORM = 4u, F_ROPE = 8u };
 
-// C[M, N] = A[M, K] * B[N, K]^T, bf16 in, fp32 accumulate, bf16 out (tcgen05 + TMA).
-cudaError_t gemm_bf16_tcgen05(const void *A, const void *B, void *C, int M, int N, int K,
-                              int *status, cudaStream_t st);
+// C[M, N] = A[M, K] * B[N, K]^T, bf16 (or f16 with ab_f16) in, fp32 accumulate, bf16 or fp32
+// out (tcgen05 + TMA).
+cudaError_t gemm_tcgen05(const void *A, const void *B, void *C, int M, int N, int K, int ab_f16,
+                         int out_f32, int *status, cudaStream_t st);
+// dst[i] = float16(src[i]) for a bf16 tensor of n elements (n % 8 == 0); a value beyond the
+// float16 range records DEV_RANGE in *status.
+cudaError_t convert_bf16_to_f16(const void *src, void *dst, size_t n, int *status, cudaStream_t st);
 // Same contraction on CUDA cores; element type float (bf16 == 0) or bf16.
 cudaError_t gemm_simt(int bf16, const void *A, const void *B, void *C, int M, int N, int K,
                       cudaStream_t st);
 
-// Latent stencil of a prefill: P [B*S, NQKV] -> q [B, H, S, DL], k/v [B, Hkv, kv_stride, DL]
-// (kv_stride >= S: the cache's max_seq, or S for workspace buffers).  When conv_state is
-// non-null the last KC-1 pre-conv q|k rows and the last upper-half value row are stored
-// and lengths[b] = S.
+// Latent stencil of a prefill: P [B*S, NQKV] (float32) -> q [B, H, S, DL],
+// k/v [B, Hkv, kv_stride, DL] (float16 for 16-bit layers) (kv_stride >= S: the cache's max_seq, or S for workspace
+// buffers).  With write_state the last KC-1 pre-conv q|k rows and the last upper-half value
+// row are stored (float32) and lengths[b] = S.
 struct StencilArgs {
-  const void *P;
+  const float *P;
   const float *conv_seq;
   const float *conv_chan;
   void *q, *k, *v;
   int kv_stride;
-  void *conv_state;     // [B, KC-1, NQ+NKV] or null
-  void *vshift_state;   // [B, NKV - NKV/2]
+  float *conv_state;    // [B, KC-1, NQ+NKV]
+  float *vshift_state;  // [B, NKV - NKV/2]
   int *lengths;         // [B]
+  int *status = nullptr;  // receives DEV_RANGE for a latent beyond the float16 range
   bool write_state = false;
 };
 cudaError_t latent_stencil(const Dims &d, const StencilArgs &a, cudaStream_t st);
@@ -69,8 +74,8 @@ struct DecodeArgs {
   const float *conv_chan;
   void *y;                  // [B, E]
   void *k_cache, *v_cache;  // [B, Hkv, max_seq, DL]
-  void *conv_state;         // [B, KC-1, NQ+NKV]
-  void *vshift_state;       // [B, NKV - NKV/2]
+  float *conv_state;        // [B, KC-1, NQ+NKV]
+  float *vshift_state;      // [B, NKV - NKV/2]
   int *lengths;             // [B]
   int *status;              // cache status word
   int max_seq;

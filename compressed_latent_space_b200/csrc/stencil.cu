@@ -12,7 +12,7 @@
 // One CTA owns a tile of TT tokens of one group of one sequence: it stages the group's
 // P rows (plus a halo of KC-1 earlier tokens) in shared memory once, and writes q in
 // head-major layout [B, H, S, d~] and k, v in [B, Hkv, kv_stride, d~] (the decode cache when
-// one is given).  Float32 arithmetic throughout.
+// one is given), as float16 for 16-bit layers.  Float32 arithmetic throughout.
 #include <math.h>
 
 #include "common.cuh"
@@ -23,12 +23,14 @@ namespace {
 
 template <typename T>
 struct StencilParams {
-  const T *P;
+  using TL = typename LatentType<T>::type;
+  const float *P;
   const float *conv_seq;
   const float *conv_chan;
-  T *q, *k, *v;
-  T *conv_state, *vshift_state;
+  TL *q, *k, *v;
+  float *conv_state, *vshift_state;
   int *lengths;
+  int *status;
   int write_state;
   int B, S, H, Hkv, G, NQ, NKV, NQKV, KC, halo, TT, kv_stride;
   unsigned flags;
@@ -48,6 +50,7 @@ __host__ __device__ inline size_t stencil_smem_floats(int G, int TT, int halo) {
 
 template <typename T, int DL>
 __global__ void __launch_bounds__(256) stencil_kernel(const StencilParams<T> p) {
+  using TL = typename StencilParams<T>::TL;
   constexpr int LPI = DL < 32 ? DL : 32;   // lanes per (token, head) item
   constexpr int EPL = DL / LPI;            // elements per lane
   constexpr int IPW = 32 / LPI;            // items per warp pass
@@ -170,12 +173,13 @@ __global__ void __launch_bounds__(256) stencil_kernel(const StencilParams<T> p) 
 #pragma unroll
         for (int e = 0; e < EPL; ++e) {
           const int i = e * LPI + li;
+          check_latent<TL>(u[e], p.status);
           if (is_q) {
             const int h = g * G + hh;
-            p.q[((static_cast<size_t>(b) * p.H + h) * p.S + t) * DL + i] = from_f32<T>(u[e]);
+            p.q[((static_cast<size_t>(b) * p.H + h) * p.S + t) * DL + i] = from_f32<TL>(u[e]);
           } else {
             p.k[((static_cast<size_t>(b) * p.Hkv + g) * p.kv_stride + t) * DL + i] =
-                from_f32<T>(u[e]);
+                from_f32<TL>(u[e]);
           }
         }
       }
@@ -190,7 +194,8 @@ __global__ void __launch_bounds__(256) stencil_kernel(const StencilParams<T> p) 
     if (t >= p.S) continue;
     const bool shifted = (p.flags & F_VALUE_SHIFT) && (g * DL + c >= vhalf);
     const float val = Ps[(tt + halo - (shifted ? 1 : 0)) * CH + QKC + c];
-    p.v[((static_cast<size_t>(b) * p.Hkv + g) * p.kv_stride + t) * DL + c] = from_f32<T>(val);
+    check_latent<TL>(val, p.status);
+    p.v[((static_cast<size_t>(b) * p.Hkv + g) * p.kv_stride + t) * DL + c] = from_f32<TL>(val);
   }
 
   // 5. decode state after the last token, written by the tile that holds it.
@@ -202,14 +207,14 @@ __global__ void __launch_bounds__(256) stencil_kernel(const StencilParams<T> p) 
       const int ts = p.S - KC1 + j;
       const int r = ts - t0 + halo;
       const int gc = c < G * DL ? qcol0 + c : p.NQ + g * DL + (c - G * DL);
-      p.conv_state[(static_cast<size_t>(b) * KC1 + j) * W + gc] = from_f32<T>(Ps[r * CH + c]);
+      p.conv_state[(static_cast<size_t>(b) * KC1 + j) * W + gc] = Ps[r * CH + c];
     }
     const int rl = p.S - 1 - t0 + halo;
     for (int c = tid; c < DL; c += blockDim.x) {
       const int gch = g * DL + c;
       if (gch >= vhalf)
         p.vshift_state[static_cast<size_t>(b) * (p.NKV - vhalf) + (gch - vhalf)] =
-            from_f32<T>(Ps[rl * CH + QKC + c]);
+            Ps[rl * CH + QKC + c];
     }
     if (g == 0 && tid == 0) p.lengths[b] = p.S;
   }
@@ -217,15 +222,17 @@ __global__ void __launch_bounds__(256) stencil_kernel(const StencilParams<T> p) 
 
 template <typename T, int DL>
 cudaError_t launch(const Dims &d, const StencilArgs &a, cudaStream_t st) {
+  using TL = typename LatentType<T>::type;
   StencilParams<T> p;
-  p.P = static_cast<const T *>(a.P);
+  p.P = a.P;
   p.conv_seq = a.conv_seq;
   p.conv_chan = a.conv_chan;
-  p.q = static_cast<T *>(a.q);
-  p.k = static_cast<T *>(a.k);
-  p.v = static_cast<T *>(a.v);
-  p.conv_state = static_cast<T *>(a.conv_state);
-  p.vshift_state = static_cast<T *>(a.vshift_state);
+  p.q = static_cast<TL *>(a.q);
+  p.k = static_cast<TL *>(a.k);
+  p.v = static_cast<TL *>(a.v);
+  p.status = a.status;
+  p.conv_state = a.conv_state;
+  p.vshift_state = a.vshift_state;
   p.lengths = a.lengths;
   p.write_state = a.write_state ? 1 : 0;
   p.B = d.B; p.S = d.S; p.H = d.H; p.Hkv = d.Hkv; p.G = d.G;

@@ -29,18 +29,19 @@ class Cache:
 
         c = layer.cfg
         dl = layer.dl
-        self.k = view(self.struct.k, batch * c.n_kv_heads * max_seq * dl, dt, es,
+        self.k = view(self.struct.k, batch * c.n_kv_heads * max_seq * dl, layer.latent_dtype, es,
                       (batch, c.n_kv_heads, max_seq, dl))
-        self.v = view(self.struct.v, batch * c.n_kv_heads * max_seq * dl, dt, es,
+        self.v = view(self.struct.v, batch * c.n_kv_heads * max_seq * dl, layer.latent_dtype, es,
                       (batch, c.n_kv_heads, max_seq, dl))
         kc1 = c.conv_kernel - 1
         if kc1 > 0:
-            self.conv_state = view(self.struct.conv_state, batch * kc1 * (layer.n_q + layer.n_kv), dt,
-                                   es, (batch, kc1, layer.n_q + layer.n_kv))
+            self.conv_state = view(self.struct.conv_state, batch * kc1 * (layer.n_q + layer.n_kv),
+                                   torch.float32, 4, (batch, kc1, layer.n_q + layer.n_kv))
         else:
             self.conv_state = None
         half = layer.n_kv - layer.n_kv // 2
-        self.vshift_state = view(self.struct.vshift_state, batch * half, dt, es, (batch, half))
+        self.vshift_state = view(self.struct.vshift_state, batch * half, torch.float32, 4,
+                                 (batch, half))
         self.lengths = view(self.struct.lengths, batch, torch.int32, 4, (batch,))
 
 
@@ -49,6 +50,8 @@ class CCALayer:
                  conv_kernel=4, rope_base=10000.0, norm_eps=1e-6, flags=CCA_DEFAULT_FLAGS,
                  dtype="bf16", device="cuda"):
         self.dtype = torch.bfloat16 if dtype == "bf16" else torch.float32
+        # latent q, k, v and the K/V cache: float16 in 16-bit layers, float32 otherwise
+        self.latent_dtype = torch.float16 if dtype == "bf16" else torch.float32
         self.esize = 2 if dtype == "bf16" else 4
         self.device = torch.device(device)
         self.cfg = make_config(d_model, n_heads, n_kv_heads, compression, conv_kernel, 1, rope_base,

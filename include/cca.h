@@ -25,9 +25,14 @@
  *     a failed check returns an error and launches nothing.
  *   - Return value: CCA_OK (0) or a negative CCA_ERR_* code; the text of the last error of
  *     the calling thread is in cca_last_error_string().  No C++ exception crosses the ABI.
- *   - Tensors are dense and row-major in the listed index order.  Activations, projection
- *     weights and the cache use the config's dtype (float32 or bfloat16); conv filters are
- *     always float32.  Device pointers must be 16-byte aligned (CCA_ERR_ALIGNMENT).
+ *   - Tensors are dense and row-major in the listed index order.  Activations x, y and the
+ *     projection weights use the config's dtype (float32 or bfloat16); conv filters and the
+ *     conv / value-shift state are always float32.  The latent queries, keys and values (and
+ *     so the K/V cache) are float32 in float32 layers and float16 in bfloat16 layers: the
+ *     same size and tensor-core rate as bfloat16 with three more significand bits (after
+ *     the per-head RMS norm q and k are bounded by sqrt(d~); a latent beyond the float16
+ *     range is reported as CCA_ERR_RANGE through cca_workspace_status / cca_cache_check).
+ *     Device pointers must be 16-byte aligned (CCA_ERR_ALIGNMENT).
  */
 #ifndef CCA_H
 #define CCA_H
@@ -41,7 +46,9 @@ extern "C" {
 
 #define CCA_API __attribute__((visibility("default")))
 
-typedef enum { CCA_F32 = 0, CCA_BF16 = 1 } cca_dtype_t;
+/* Element types.  A layer is CCA_F32 or CCA_BF16; CCA_F16 (the latent type of bfloat16
+ * layers) is accepted only by the stage entry points of cca_stages.h. */
+typedef enum { CCA_F32 = 0, CCA_BF16 = 1, CCA_F16 = 2 } cca_dtype_t;
 
 enum {
   CCA_OK = 0,
@@ -51,7 +58,8 @@ enum {
   CCA_ERR_CACHE_FULL = -4,    /* a sequence would pass max_seq                             */
   CCA_ERR_ALIGNMENT = -5,     /* a device pointer is not 16-byte aligned                  */
   CCA_ERR_CUDA = -6,          /* a CUDA call or kernel launch failed                      */
-  CCA_ERR_DEVICE = -7         /* a kernel reported an internal error (bounded wait ran out) */
+  CCA_ERR_DEVICE = -7,        /* a kernel reported an internal error (bounded wait ran out) */
+  CCA_ERR_RANGE = -8          /* a latent q, k or v exceeded the float16 range (16-bit layers) */
 };
 
 /* Switches of the method's three expressivity steps and of normalisation / RoPE. */
@@ -94,10 +102,11 @@ typedef struct {
 
 /* Compressed decode state, laid out by cca_cache_alloc inside one caller buffer.
  *   k, v          [batch, Hkv, max_seq, d~]  final latent keys (after conv, q-k-mean, norm
- *                 and RoPE) and values (after value-shift)
- *   conv_state    [batch, conv_kernel-1, n_q + n_kv]  pre-conv q|k projections of the last
- *                 conv_kernel-1 tokens, oldest first, zero before position 0
- *   vshift_state  [batch, n_kv - n_kv/2]  upper-half value projection of the last token
+ *                 and RoPE) and values (after value-shift), latent element type (above)
+ *   conv_state    [batch, conv_kernel-1, n_q + n_kv] float32: pre-conv q|k projections of
+ *                 the last conv_kernel-1 tokens, oldest first, zero before position 0
+ *   vshift_state  [batch, n_kv - n_kv/2] float32: upper-half value projection of the last
+ *                 token
  *   lengths       [batch] int32, tokens held per sequence (the RoPE position of the next)
  *   status        int32 sticky error word set by kernels that met a full sequence       */
 typedef struct {
@@ -139,7 +148,8 @@ CCA_API int cca_prefill_forward(const cca_config_t *cfg, const cca_weights_t *w,
  * The token's key/value are appended at position lengths[b], its query attends to
  * positions 0..lengths[b], the conv / value-shift state advance and lengths[b] += 1.
  * A sequence already holding max_seq tokens is left untouched, its y row is zero and the
- * cache status word is set to CCA_ERR_CACHE_FULL (read it with cca_cache_check).
+ * cache status word is set to CCA_ERR_CACHE_FULL (read it with cca_cache_check).  A new
+ * latent key or value beyond the float16 range sets it to CCA_ERR_RANGE.
  * Errors (host): INVALID_ARG, UNSUPPORTED, WORKSPACE, ALIGNMENT, CUDA. */
 CCA_API int cca_decode_step(const cca_config_t *cfg, const cca_weights_t *w, const void *x,
                             void *y, cca_cache_t *cache, void *workspace, size_t ws_bytes,

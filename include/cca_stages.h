@@ -13,16 +13,18 @@
 extern "C" {
 #endif
 
-/* C[m, n] = sum_k A[m, k] * B[n, k]  (A [M, K], B [N, K], C [M, N], all row-major, dtype
- * as given).  bf16 runs on the tcgen05 tensor-core kernel when K % 8 == 0, float32 on CUDA
- * cores.  This is the contraction of the down-projection (x W_qkv^T) and of the
- * up-projection (o W_o^T) of the layer (gist.science explainer, 2. Methodology, Core
- * Mechanism, "Down-Projection"). */
-CCA_API int cca_gemm(int dtype, const void *A, const void *B, void *C, int M, int N, int K,
-                     int *status, void *stream);
+/* C[m, n] = sum_k A[m, k] * B[n, k]  (A [M, K], B [N, K], C [M, N], all row-major; A and B
+ * of `dtype`, C of `out_dtype`).  bf16 or f16 operands run on the tcgen05 tensor-core kernel
+ * (K % 8 == 0, result bf16 or float32), float32 operands on CUDA cores (result float32).
+ * This is the contraction of the down-projection (x W_qkv^T) and of the up-projection
+ * (o W_o^T) of the layer (gist.science explainer, 2. Methodology, Core Mechanism,
+ * "Down-Projection"). */
+CCA_API int cca_gemm(int dtype, int out_dtype, const void *A, const void *B, void *C, int M,
+                     int N, int K, int *status, void *stream);
 
-/* Latent stencil: P [batch*seq, n_q + 2 n_kv] (the projections) ->
- * q [batch, H, seq, d~], k and v [batch, Hkv, kv_stride, d~] with kv_stride >= seq.
+/* Latent stencil: P [batch*seq, n_q + 2 n_kv] (the projections, float32) ->
+ * q [batch, H, seq, d~], k and v [batch, Hkv, kv_stride, d~] with kv_stride >= seq
+ * (q, k and v of the latent element type of cca.h: float16 for bfloat16 layers).
  * Sequence conv, channel conv, q-k-mean, value-shift, RMS norm and RoPE (positions 0..seq-1),
  * as selected by cfg->flags (gist.science explainer, 2. Methodology, Core Mechanism). */
 CCA_API int cca_stage_stencil(const cca_config_t *cfg, const void *P, int batch, int seq,
@@ -30,15 +32,16 @@ CCA_API int cca_stage_stencil(const cca_config_t *cfg, const void *P, int batch,
                               void *v, int kv_stride, void *stream);
 
 /* Causal latent attention: q [batch, H, seq, d~], k/v [batch, Hkv, kv_stride, d~] ->
- * o [batch*seq, H*d~] (token-major), scale 1/sqrt(d~), query head h reads kv head
+ * o [batch*seq, H*d~] (token-major; q, k, v and o of the latent element type of cca.h), scale 1/sqrt(d~), query head h reads kv head
  * h / (H/Hkv) (gist.science/de explainer, 2. Methodik: Softmax(QK^T)V in the compressed
  * space; gist.science explainer, Extension: CCGQA). */
 CCA_API int cca_stage_attention(const cca_config_t *cfg, const void *q, const void *k,
                                 const void *v, int batch, int seq, int kv_stride, void *o,
                                 int *status, void *stream);
 
-/* Waits for `stream` and returns CCA_OK, or CCA_ERR_DEVICE if a kernel of the last
- * cca_prefill_forward that used this workspace recorded an internal error. */
+/* Waits for `stream` and returns CCA_OK, CCA_ERR_RANGE if the last cca_prefill_forward
+ * that used this workspace met a latent beyond the float16 range, or CCA_ERR_DEVICE if one
+ * of its kernels recorded an internal error. */
 CCA_API int cca_workspace_status(const void *workspace, void *stream);
 
 /* Per-kernel timing for benchmarks.  cca_stage_timing(1) starts a session: from then on

@@ -54,12 +54,12 @@ def test_workspace_and_cache_sizes(lib):
     M = B * S
     nq, nkv = 16 * 32, 4 * 32
     al = lambda x: (x + 255) // 256 * 256
-    expect = 256 + al(M * (nq + 2 * nkv) * 2) + al(M * nq * 2) + 2 * al(M * nkv * 2) + al(M * nq * 2)
+    expect = 256 + al(2048 * nq * 2) + al(M * (nq + 2 * nkv) * 4) + al(M * nq * 2) + 2 * al(M * nkv * 2) + al(M * nq * 2)
     assert cls.cca_prefill_workspace_size(c, B, S) == expect
     # cache: keys and values are n_kv wide per token: C * H/Hkv = 16x smaller than MHA's 2E
     nbytes = cls.cca_cache_alloc(c, 3, 1000)
     kv = 2 * al(3 * 4 * 1000 * 32 * 2)
-    state = al(3 * 3 * (nq + nkv) * 2) + al(3 * (nkv // 2) * 2) + al(3 * 4) + 256
+    state = al(3 * 3 * (nq + nkv) * 4) + al(3 * (nkv // 2) * 4) + al(3 * 4) + 256
     assert nbytes == kv + state
     assert cls.cca_decode_workspace_size(c, 3, 1000) > 0
 

@@ -7,8 +7,10 @@ Recipe (every workload): ``torch.Generator('cpu').manual_seed(seed)`` draws, in 
 order, x, W_q, W_k, W_v, W_o, conv_seq, conv_chan, and for the decode workload then the
 key cache, value cache, conv state, value-shift state and the new tokens.  x and the
 cache contents are N(0, 1); every weight (projections and conv filters) is N(0, 0.02^2)
-unless a test overrides the conv scale.  Values are rounded to the workload's dtype on
-the host; the oracle receives exactly the rounded values.
+unless a test overrides the conv scale.  x and the projection weights are rounded to the
+workload's dtype, the K/V cache to its latent type (float16 for bf16 workloads), conv
+filters and the conv / value-shift state stay float32; the oracle receives exactly these
+values.
 """
 from __future__ import annotations
 
@@ -55,6 +57,11 @@ class Workload:
     def torch_dtype(self):
         return torch.float32 if self.dtype == "f32" else torch.bfloat16
 
+    @property
+    def latent_dtype(self):
+        """Storage type of the latent q, k, v and the K/V cache (float16 in 16-bit workloads)."""
+        return torch.float32 if self.dtype == "f32" else torch.float16
+
     def with_(self, **kw) -> "Workload":
         return replace(self, **kw)
 
@@ -85,8 +92,8 @@ class Inputs:
     conv_chan: torch.Tensor         # [H + Hkv, d~, d~, k_c]    float32
     k_cache: torch.Tensor | None = None       # [B, Hkv, ctx, d~]
     v_cache: torch.Tensor | None = None       # [B, Hkv, ctx, d~]
-    conv_state: torch.Tensor | None = None    # [B, k-1, n_q + n_kv]
-    vshift_state: torch.Tensor | None = None  # [B, n_kv - n_kv/2]
+    conv_state: torch.Tensor | None = None    # [B, k-1, n_q + n_kv] float32
+    vshift_state: torch.Tensor | None = None  # [B, n_kv - n_kv/2] float32
     lengths: torch.Tensor | None = None       # [B] int32
     extra: dict = field(default_factory=dict)
 
@@ -126,10 +133,10 @@ def make_inputs(w: Workload, seed: int = 0, conv_std: float = WEIGHT_STD,
         inp.x = x
         return inp
     B, ctx = w.batch, w.seq
-    inp.k_cache = randn(B, w.n_kv_heads, ctx, d).to(dt)
-    inp.v_cache = randn(B, w.n_kv_heads, ctx, d).to(dt)
-    inp.conv_state = randn(B, w.conv_kernel - 1, nq + nkv).to(dt)
-    inp.vshift_state = randn(B, nkv - nkv // 2).to(dt)
+    inp.k_cache = randn(B, w.n_kv_heads, ctx, d).to(w.latent_dtype)
+    inp.v_cache = randn(B, w.n_kv_heads, ctx, d).to(w.latent_dtype)
+    inp.conv_state = randn(B, w.conv_kernel - 1, nq + nkv)          # float32 state
+    inp.vshift_state = randn(B, nkv - nkv // 2)
     inp.x = randn(B, E).to(dt)
     if lengths is None:
         inp.lengths = torch.full((B,), ctx, dtype=torch.int32)
