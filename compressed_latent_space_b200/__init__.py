@@ -72,6 +72,8 @@ _SIGS = {
     "cca_stage_attention": (c_int, [POINTER(cca_config_t), c_void_p, c_void_p, c_void_p, c_int,
                                     c_int, c_int, c_void_p, c_void_p, c_void_p]),
     "cca_workspace_status": (c_int, [c_void_p, c_void_p]),
+    "cca_decode_step_static": (c_int, [POINTER(cca_config_t), POINTER(cca_weights_t), c_void_p,
+                                       c_void_p, POINTER(cca_cache_t), c_void_p]),
     "cca_stage_timing": (c_int, [c_int]),
     "cca_stage_times": (c_int, [POINTER(ctypes.c_double), c_int, POINTER(c_int)]),
 }
@@ -166,6 +168,12 @@ def cca_decode_step(cfg, weights, x, y, cache, workspace=None, stream=None):
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib.cca_decode_step(ctypes.byref(cfg), ctypes.byref(weights), _ptr(x), _ptr(y),
                                ctypes.byref(cache), _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def cca_decode_step_static(cfg, weights, x, y, cache, stream=None):
+    """Decode step whose scratch is the library's built-in device array (no workspace)."""
+    _check(load().cca_decode_step_static(ctypes.byref(cfg), ctypes.byref(weights), _ptr(x), _ptr(y),
+                                         ctypes.byref(cache), _stream(stream)))
 
 
 def cca_cache_check(cache, stream=None):

@@ -494,3 +494,8 @@ CCA_API int cca_stage_attention(const cca_config_t *cfg, const void *q, const vo
 }
 
 }  // extern "C"
+
+namespace cca {
+// Records `msg` as the calling thread's last error and returns `code`.
+int set_last_error(int code, const char *msg) { return fail(code, "%s", msg); }
+}  // namespace cca

@@ -96,4 +96,7 @@ cudaError_t decode_step(const Dims &d, const DecodeArgs &a, cudaStream_t st,
 
 int num_sms();
 
+// Records `msg` as the calling thread's last error (cca_last_error_string) and returns `code`.
+int set_last_error(int code, const char *msg);
+
 }  // namespace cca

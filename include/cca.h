@@ -155,6 +155,22 @@ CCA_API int cca_decode_step(const cca_config_t *cfg, const cca_weights_t *w, con
                             void *y, cca_cache_t *cache, void *workspace, size_t ws_bytes,
                             void *stream);
 
+/* cca_decode_step without a caller workspace; it allocates nothing.  (The paper has no
+ * counterpart: this exists for callers.)  Meant for callers that cannot allocate device
+ * memory on their decode path, e.g. a serving loop whose memory is fixed at start-up, or a
+ * program running under another framework's allocator that it does not control.  Inputs,
+ * outputs, weights and the cache are the caller's as in cca_decode_step; the step's scratch
+ * lives in an 8 MiB array built into the library, held by every GPU that loads the library
+ * until the process exits.  A step that needs more scratch (cca_decode_workspace_size above
+ * 8 MiB, e.g. 64 sequences of 16 heads with d~ = 32 beyond ~12k cached tokens) is rejected
+ * with CCA_ERR_WORKSPACE before anything is launched.  The first call on each device looks
+ * up the array's device address (cudaGetSymbolAddress) with that device current; make that
+ * first call before any stream capture.  Every call uses the same array and leaves its
+ * contents there; nothing in it needs to start at zero, but two calls whose kernels overlap
+ * on the GPU (different streams without ordering) race on it.  Errors as cca_decode_step. */
+CCA_API int cca_decode_step_static(const cca_config_t *cfg, const cca_weights_t *w,
+                                   const void *x, void *y, cca_cache_t *cache, void *stream);
+
 /* Waits for `stream`, then returns the cache's sticky status word (CCA_OK or
  * CCA_ERR_CACHE_FULL) and clears it. */
 CCA_API int cca_cache_check(cca_cache_t *cache, void *stream);
