@@ -92,7 +92,7 @@ __device__ __forceinline__ void store8(float *p, const float (&v)[8]) {
 
 // ----------------------------------------------------------------------------- status
 // Codes a kernel can leave in its status word (first error wins).
-enum : int { DEV_OK = 0, DEV_WAIT_TIMEOUT = 1, DEV_CACHE_FULL = 2, DEV_RANGE = 3 };
+enum : int { DEV_OK = 0, DEV_WAIT_TIMEOUT = 1, DEV_CACHE_FULL = 2, DEV_RANGE = 3, DEV_LAYOUT = 4 };
 
 
 __device__ __forceinline__ void report(int *status, int code) {

@@ -1,6 +1,7 @@
 // Host-side launchers of the CCA kernels (internal to libcca; not part of the C ABI).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -64,6 +65,9 @@ cudaError_t latent_stencil(const Dims &d, const StencilArgs &a, cudaStream_t st)
 // Causal latent attention: q [B, H, S, DL], k/v [B, Hkv, kv_stride, DL] -> o [B*S, NQ].
 cudaError_t latent_attention(const Dims &d, const void *q, const void *k, const void *v,
                              int kv_stride, void *o, int *status, cudaStream_t st);
+// The tcgen05 kernel behind latent_attention for 16-bit layers (float16 q, k, v, o).
+cudaError_t latent_attention_tc(const Dims &d, const void *q, const void *k, const void *v,
+                                int kv_stride, void *o, int *status, cudaStream_t st);
 
 // Decode step kernels.
 struct DecodeArgs {
@@ -95,6 +99,13 @@ cudaError_t decode_step(const Dims &d, const DecodeArgs &a, cudaStream_t st,
                         const StageMarker &mark);
 
 int num_sms();
+
+// Tiled TMA descriptor of a 16-bit tensor of `rank` dims (dims[0] innermost, in elements;
+// strides_bytes[i] is the byte stride of dim i+1), box in elements, swizzle span in bytes
+// (0, 32, 64 or 128); out-of-range elements of a box read as zero.
+bool make_tma_16bit(CUtensorMap *map, const void *ptr, int rank, const uint64_t *dims,
+                    const uint64_t *strides_bytes, const uint32_t *box, int swizzle_bytes,
+                    int f16);
 
 // Records `msg` as the calling thread's last error (cca_last_error_string) and returns `code`.
 int set_last_error(int code, const char *msg);
