@@ -267,11 +267,19 @@ def cpu_oracle_sample(w, budget_s=12.0, seed=0):
                        f"this overstates the oracle's full-length rate)")
 
 
+def workload_from_args(args):
+    w = W.WORKLOADS[args.workload]
+    over = {k: v for k, v in (("batch", args.batch), ("seq", args.seq)) if v is not None}
+    if over:
+        w = w.with_(name=w.name + "[" + ",".join(f"{k}={v}" for k, v in over.items()) + "]", **over)
+    return w
+
+
 def run_cuda(args):
     rank, world, local = dist_setup(args.gpus)
     import compressed_latent_space_b200 as cls
     cls.load()
-    w = W.WORKLOADS[args.workload]
+    w = workload_from_args(args)
     hbm, bf16_peak, bf16_sus, peak_src = measured_peaks()
     with ClockSampler(local) as clk:
         pre = bench_prefill(cls, w, args.steps, args.warmup, world, seed=rank)
@@ -338,7 +346,7 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    w = W.WORKLOADS[args.workload]
+    w = workload_from_args(args)
     per_step_budget = max(2.0, 150.0 / max(1, args.steps + args.warmup))
     for _ in range(args.warmup):
         cpu_oracle_sample(w, budget_s=per_step_budget)
@@ -369,6 +377,10 @@ def main():
     ap.add_argument("--impl", default="cca", choices=["cca", "reference"])
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the workload's batch (smaller cases for profiling)")
+    ap.add_argument("--seq", type=int, default=None,
+                    help="override the workload's sequence length (smaller cases for profiling)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)      # at least 3 untimed warm-up steps
     if args.impl == "reference":
