@@ -175,7 +175,7 @@ def bench_prefill(cls, w, steps, warmup, world, seed):
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     ms = statistics.fmean(step_ms)
     stages = {n: t / max(calls, 1) for n, t in
-              zip(["w_o_to_f16", "qkv_projection", "latent_stencil", "latent_attention",
+              zip(["weights_to_16bit", "qkv_projection", "latent_stencil", "latent_attention",
                    "out_projection"], stage_ms)}
 
     # end to end through the public API: pinned host x -> device, forward, y -> pinned host
@@ -199,7 +199,7 @@ def bench_prefill(cls, w, steps, warmup, world, seed):
     e2e_ms = statistics.fmean(s.elapsed_time(e) for s, e in zip(e2e_s, e2e_e))
     nbytes = x.numel() * x.element_size()
     return dict(ms=ms, stages=stages, calls=calls, e2e_ms=e2e_ms, h2d=nbytes, d2h=nbytes,
-                launches=5 * steps)
+                launches=6 * steps)
 
 
 def bench_decode(cls, w, steps, warmup, seed):

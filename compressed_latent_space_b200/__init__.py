@@ -68,7 +68,9 @@ _SIGS = {
     "cca_gemm": (c_int, [c_int, c_int, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int,
                          c_void_p, c_void_p]),
     "cca_stage_stencil": (c_int, [POINTER(cca_config_t), c_void_p, c_int, c_int, c_void_p,
-                                  c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_void_p]),
+                                  c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_void_p,
+                                  c_size_t, c_void_p]),
+    "cca_stage_stencil_workspace_size": (c_size_t, [POINTER(cca_config_t)]),
     "cca_stage_attention": (c_int, [POINTER(cca_config_t), c_void_p, c_void_p, c_void_p, c_int,
                                     c_int, c_int, c_void_p, c_void_p, c_void_p]),
     "cca_workspace_status": (c_int, [c_void_p, c_void_p]),
@@ -184,10 +186,16 @@ def cca_gemm(dtype, out_dtype, A, B, C, M, N, K, status=None, stream=None):
     _check(load().cca_gemm(dtype, out_dtype, _ptr(A), _ptr(B), _ptr(C), M, N, K, _ptr(status), _stream(stream)))
 
 
-def cca_stage_stencil(cfg, P, batch, seq, conv_seq, conv_chan, q, k, v, kv_stride, stream=None):
+def cca_stage_stencil_workspace_size(cfg):
+    return load().cca_stage_stencil_workspace_size(ctypes.byref(cfg))
+
+
+def cca_stage_stencil(cfg, P, batch, seq, conv_seq, conv_chan, q, k, v, kv_stride, workspace,
+                      stream=None):
+    ws_bytes = workspace.numel() * workspace.element_size()
     _check(load().cca_stage_stencil(ctypes.byref(cfg), _ptr(P), batch, seq, _ptr(conv_seq),
                                     _ptr(conv_chan), _ptr(q), _ptr(k), _ptr(v), kv_stride,
-                                    _stream(stream)))
+                                    _ptr(workspace), ws_bytes, _stream(stream)))
 
 
 def cca_stage_attention(cfg, q, k, v, batch, seq, kv_stride, o, status=None, stream=None):

@@ -202,16 +202,25 @@ __global__ void __launch_bounds__(192, 2)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->s_free);
 
-      float mx = -INFINITY;
-      const bool diag = (j == nkv - 1);
-      const int key0 = j * TN;
+      // Row max of the raw scores (the 1/sqrt(d~) * log2(e) scale is positive, so it is
+      // applied afterwards): eight independent partial maxima keep the dependency chains
+      // short.  Keys past this row's position are masked on the diagonal tile only.
+      float mx8[8];
 #pragma unroll
-      for (int i = 0; i < TN; ++i) {
-        float x = __uint_as_float(r[i]) * scale_log2;
-        if (diag && key0 + i > qpos) x = -INFINITY;
-        r[i] = __float_as_uint(x);
-        mx = fmaxf(mx, x);
+      for (int e = 0; e < 8; ++e) mx8[e] = -INFINITY;
+      if (j == nkv - 1) {
+        const int last = qpos - j * TN;               // keys 0..last of this tile are visible
+#pragma unroll
+        for (int i = 0; i < TN; ++i) {
+          if (i > last) r[i] = __float_as_uint(-INFINITY);
+          mx8[i & 7] = fmaxf(mx8[i & 7], __uint_as_float(r[i]));
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < TN; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], __uint_as_float(r[i]));
       }
+      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * scale_log2;
       bool resc = false;
       float m_new = m_ref;
       if (mx > m_ref + kTau) {
@@ -239,13 +248,18 @@ __global__ void __launch_bounds__(192, 2)
         }
       }
       m_ref = m_new;
+      // p = 2^(s * scale - m_ref): one FFMA and one MUFU ex2 per score; eight partial sums.
+      const float neg_m = -m_ref;
+      float l8[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) l8[e] = 0.f;
 #pragma unroll
       for (int c = 0; c < TN / 8; ++c) {
         float p[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          p[e] = ex2(__uint_as_float(r[c * 8 + e]) - m_ref);
-          l += p[e];
+          p[e] = ex2(fmaf(__uint_as_float(r[c * 8 + e]), scale_log2, neg_m));
+          l8[e] += p[e];
         }
         uint4 u;
         u.x = pack_f16x2(p[0], p[1]);
@@ -255,6 +269,7 @@ __global__ void __launch_bounds__(192, 2)
         const int atom = c >> 3, chunk = (c & 7) ^ (row & 7);
         *reinterpret_cast<uint4 *>(p_row + atom * (TM * 128) + chunk * 16) = u;
       }
+      l += ((l8[0] + l8[1]) + (l8[2] + l8[3])) + ((l8[4] + l8[5]) + (l8[6] + l8[7]));
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();

@@ -93,7 +93,7 @@ int make_dims(const cca_config_t *cfg, cca::Dims &d) {
 size_t esize(const cca::Dims &d) { return d.bf16 ? 2 : 4; }
 
 struct PrefillLayout {
-  size_t status, wo16, P, q, k, v, o, total;
+  size_t status, wo16, wsplit, P, q, k, v, o, total;
 };
 
 PrefillLayout prefill_layout(const cca::Dims &d, int B, int S) {
@@ -102,6 +102,7 @@ PrefillLayout prefill_layout(const cca::Dims &d, int B, int S) {
   size_t off = 0;
   L.status = off; off += 256;
   L.wo16 = off; off += d.bf16 ? align256(static_cast<size_t>(d.E) * d.NQ * 2) : 0;
+  L.wsplit = off; off += align256(cca::conv_chan_split_bytes(d));
   L.P = off; off += align256(M * d.NQKV * 4);   // projections stay float32
   L.q = off; off += align256(M * d.NQ * es);
   L.k = off; off += align256(M * d.NKV * es);
@@ -331,6 +332,8 @@ CCA_API int cca_prefill_forward(const cca_config_t *cfg, const cca_weights_t *w,
     if ((e = cca::convert_bf16_to_f16(w->w_o, wo, static_cast<size_t>(d.E) * d.NQ, status, st)) !=
         cudaSuccess)
       return cuda_fail(e, "W_o conversion launch");
+    if ((e = cca::split_conv_chan(d, w->conv_chan, ws + L.wsplit, st)) != cudaSuccess)
+      return cuda_fail(e, "channel-conv weight split launch");
   }
   rec.mark();
   void *P = ws + L.P, *q = ws + L.q, *o = ws + L.o;
@@ -345,6 +348,7 @@ CCA_API int cca_prefill_forward(const cca_config_t *cfg, const cca_weights_t *w,
   sa.P = static_cast<const float *>(P);
   sa.conv_seq = w->conv_seq;
   sa.conv_chan = w->conv_chan;
+  sa.conv_chan_split = ws + L.wsplit;
   sa.q = q;
   sa.k = k;
   sa.v = v;
@@ -451,9 +455,16 @@ CCA_API int cca_gemm(int dtype, int out_dtype, const void *A, const void *B, voi
   return rc ? rc : ok();
 }
 
+CCA_API size_t cca_stage_stencil_workspace_size(const cca_config_t *cfg) {
+  cca::Dims d;
+  if (make_dims(cfg, d)) return 0;
+  return align256(cca::conv_chan_split_bytes(d)) + 256;
+}
+
 CCA_API int cca_stage_stencil(const cca_config_t *cfg, const void *P, int batch, int seq,
                               const float *conv_seq, const float *conv_chan, void *q, void *k,
-                              void *v, int kv_stride, void *stream) {
+                              void *v, int kv_stride, void *workspace, size_t ws_bytes,
+                              void *stream) {
   cca::Dims d;
   int rc = make_dims(cfg, d);
   if (rc) return rc;
@@ -464,15 +475,27 @@ CCA_API int cca_stage_stencil(const cca_config_t *cfg, const void *P, int batch,
   if (injected_launch_failure()) return fail(CCA_ERR_CUDA, "injected launch failure");
   d.B = batch;
   d.S = seq;
+  const size_t need = align256(cca::conv_chan_split_bytes(d)) + 256;
+  if (!workspace || ws_bytes < need)
+    return fail(CCA_ERR_WORKSPACE, "workspace of %zu bytes, %zu needed", workspace ? ws_bytes : 0, need);
+  if (!aligned16(workspace)) return fail(CCA_ERR_ALIGNMENT, "workspace must be 16-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char *wsp = static_cast<char *>(workspace);
+  int *status = reinterpret_cast<int *>(wsp);
+  cudaError_t e0 = cudaMemsetAsync(status, 0, 256, st);
+  if (e0 == cudaSuccess && d.bf16) e0 = cca::split_conv_chan(d, conv_chan, wsp + 256, st);
+  if (e0 != cudaSuccess) return cuda_fail(e0, "stencil preparation");
   cca::StencilArgs sa{};
   sa.P = static_cast<const float *>(P);
   sa.conv_seq = conv_seq;
   sa.conv_chan = conv_chan;
+  sa.conv_chan_split = wsp + 256;
+  sa.status = status;
   sa.q = q;
   sa.k = k;
   sa.v = v;
   sa.kv_stride = kv_stride;
-  cudaError_t e = cca::latent_stencil(d, sa, static_cast<cudaStream_t>(stream));
+  cudaError_t e = cca::latent_stencil(d, sa, st);
   return e == cudaSuccess ? ok() : cuda_fail(e, "stencil launch");
 }
 

@@ -167,6 +167,30 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
   }
 }
 
+// ----------------------------------------------------------------------------- RoPE
+// cos and sin of a rotary angle t * theta (radians; |angle| < 2^20 here).  The angle is first
+// reduced to [-pi, pi] in double by subtracting the nearest multiple of 2*pi (Cody-Waite
+// additive reduction with a one-term constant, exact to ~1e-11 at these magnitudes), then
+// evaluated in float.  Evaluating sin/cos of the unreduced double angle would send large
+// arguments down a much slower reduction path.
+__device__ __forceinline__ void rope_cos_sin(double angle, float &c, float &s) {
+  const double two_pi = 6.283185307179586;
+  const double k = rint(angle * (1.0 / two_pi));
+  const float r = static_cast<float>(fma(-k, two_pi, angle));
+  sincosf(r, &s, &c);
+}
+
+// ----------------------------------------------------------------------------- cp.async
+// 16-byte global -> shared copy that bypasses L1; writes zeros instead when !valid.
+__device__ __forceinline__ void cp_async16_zfill(void *dst, const void *src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src),
+               "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;" ::: "memory");
+}
+
 // ----------------------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");

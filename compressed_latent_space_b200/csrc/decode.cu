@@ -20,7 +20,7 @@
 namespace cca {
 namespace {
 
-constexpr int CHUNK = 256;        // keys per split-KV block
+constexpr int CHUNK = 512;        // keys per split-KV block
 
 // ------------------------------------------------------------------ D1 / D4 skinny GEMM
 // C[M, N] = A[M, K] * B[N, K]^T for small M (the batch), bf16 operands on mma.sync.
@@ -123,7 +123,8 @@ struct D2Params {
   float *q_new;
   int B, H, Hkv, G, DL, NQ, NKV, NQKV, KC, max_seq;
   unsigned flags;
-  float eps, rope_base;
+  float eps;
+  double theta[32];        // RoPE frequencies base^(-2i/d~), i < d~/2, computed on the host
 };
 
 template <typename T>
@@ -199,10 +200,8 @@ __global__ void __launch_bounds__(128) decode_stencil_kernel(const D2Params<T> p
     const int hh = o / HALF, ip = o % HALF;
     float x1 = u[hh * DL + ip] * inv[hh], x2 = u[hh * DL + ip + HALF] * inv[hh];
     if (p.flags & F_ROPE) {
-      const double theta = pow(static_cast<double>(p.rope_base), -2.0 * ip / DL);
-      double sd, cd;
-      sincos(static_cast<double>(L) * theta, &sd, &cd);
-      const float c = static_cast<float>(cd), s = static_cast<float>(sd);
+      float c, s;
+      rope_cos_sin(static_cast<double>(L) * p.theta[ip], c, s);
       const float y1 = x1 * c - x2 * s, y2 = x1 * s + x2 * c;
       x1 = y1;
       x2 = y2;
@@ -242,116 +241,193 @@ __global__ void __launch_bounds__(128) decode_stencil_kernel(const D2Params<T> p
 }
 
 // ------------------------------------------------------------------ D3 split-KV attention
-template <typename TL>
+// One CTA per (sequence, kv group, chunk of CHUNK keys).  The chunk's keys and values are
+// brought into shared memory with 16-byte asynchronous copies issued all at once (keys with
+// their 16-byte pieces XOR-swizzled by row, so the one-row-per-thread reads below hit eight
+// different bank groups), then:
+//   scores  one thread per key, the G queries of the group broadcast from shared memory
+//   softmax one warp per head: chunk max m, p = 2^(s - m), chunk sum l
+//   P V     thread (dim pair, key slice) accumulates G heads x 2 dims, slices summed at the end
+// Partial results (unnormalised o, m, l) go to the workspace for the merge.
+template <int CPR>
+__device__ __forceinline__ int kv_swz(int r) {       // swizzle of a row's 16-byte pieces
+  constexpr int SPAN = CPR < 8 ? CPR : 8;
+  constexpr int DIV = CPR < 8 ? 8 / CPR : 1;
+  return (r / DIV) & (SPAN - 1);
+}
+
+template <int DL, typename TL>
 __global__ void __launch_bounds__(128) decode_attn_kernel(
     const float *__restrict__ q_new, const TL *__restrict__ k_cache,
-    const TL *__restrict__ v_cache,
-    const int *__restrict__ lengths, float *__restrict__ part_o, float *__restrict__ part_ml, int H,
-    int Hkv, int G, int DL, int max_seq, int nchunk, float scale_log2) {
-  extern __shared__ float sm[];
+    const TL *__restrict__ v_cache, const int *__restrict__ lengths, float *__restrict__ part_o,
+    float *__restrict__ part_ml, int H, int Hkv, int G, int max_seq, int nchunk,
+    float scale_log2) {
+  constexpr int EPC = 16 / sizeof(TL);               // elements per 16-byte piece
+  constexpr int CPR = DL / EPC;                      // pieces per row
+  constexpr int PAIRS = DL / 2;
+  constexpr int KS = 128 / PAIRS;                    // key slices in the P V phase
+  extern __shared__ __align__(16) uint8_t smraw[];
+  TL *Ks = reinterpret_cast<TL *>(smraw);            // [CHUNK][DL], swizzled pieces
+  TL *Vs = Ks + CHUNK * DL;                          // [CHUNK][DL]
+  float *qs = reinterpret_cast<float *>(Vs + CHUNK * DL);   // [G][DL], pre-scaled
+  float *sc = qs + G * DL;                           // [G][CHUNK]
+  float *red = sc + G * CHUNK;                       // [KS][G][DL]
+  float *mls = red + KS * G * DL;                    // [G][2]
   const int ch = blockIdx.x, g = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
   const int L = lengths[b];
-  const int nkeys = L + 1;
   const int s0 = ch * CHUNK;
-  const int n = L < max_seq ? min(CHUNK, nkeys - s0) : 0;
-  float *qs = sm;                   // [G][DL]
-  float *sc = qs + G * DL;          // [G][CHUNK]
-  float *ks = sc + G * CHUNK;       // [CHUNK][DL+1]
-  float *vsm = ks + CHUNK * (DL + 1);  // [CHUNK][DL]
-  float *ml = vsm + CHUNK * DL;     // [G][2]
+  const int n = L < max_seq ? min(CHUNK, L + 1 - s0) : 0;
+  float *po = part_o + ((static_cast<size_t>(b) * H + g * G) * nchunk + ch) * DL;
+  float *pml = part_ml + ((static_cast<size_t>(b) * H + g * G) * nchunk + ch) * 2;
   if (n <= 0) {
-    for (int i = tid; i < G * DL; i += blockDim.x) {
-      const int hh = i / DL, d = i % DL;
-      part_o[((static_cast<size_t>(b) * H + g * G + hh) * nchunk + ch) * DL + d] = 0.f;
-    }
-    for (int hh = tid; hh < G; hh += blockDim.x) {
-      float *o = part_ml + ((static_cast<size_t>(b) * H + g * G + hh) * nchunk + ch) * 2;
-      o[0] = -INFINITY;
-      o[1] = 0.f;
+    for (int i = tid; i < G * DL; i += blockDim.x)
+      po[static_cast<size_t>(i / DL) * nchunk * DL + (i % DL)] = 0.f;
+    for (int h = tid; h < G; h += blockDim.x) {
+      pml[static_cast<size_t>(h) * nchunk * 2] = -INFINITY;
+      pml[static_cast<size_t>(h) * nchunk * 2 + 1] = 0.f;
     }
     return;
   }
+  const size_t row0 = (static_cast<size_t>(b) * Hkv + g) * max_seq + s0;
+  for (int i = tid; i < n * CPR; i += blockDim.x) {
+    const int r = i / CPR, j = i % CPR;
+    cp_async16_zfill(Ks + r * DL + (j ^ kv_swz<CPR>(r)) * EPC, k_cache + (row0 + r) * DL + j * EPC, true);
+    cp_async16_zfill(Vs + r * DL + j * EPC, v_cache + (row0 + r) * DL + j * EPC, true);
+  }
   for (int i = tid; i < G * DL; i += blockDim.x)
     qs[i] = q_new[(static_cast<size_t>(b) * H + g * G) * DL + i] * scale_log2;
-  const auto *kb = k_cache + ((static_cast<size_t>(b) * Hkv + g) * max_seq + s0) * DL;
-  const TL *vb = v_cache + ((static_cast<size_t>(b) * Hkv + g) * max_seq + s0) * DL;
-  for (int i = tid; i < n * DL / 8; i += blockDim.x) {
-    const int r = i / (DL / 8), c = (i % (DL / 8)) * 8;
-    float k8[8], v8[8];
-    load8(kb + static_cast<size_t>(r) * DL + c, k8);
-    load8(vb + static_cast<size_t>(r) * DL + c, v8);
+  cp_async_wait_all();
+  __syncthreads();
+
+  // scores
+  for (int r = tid; r < n; r += blockDim.x) {
+    float kf[DL];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      ks[r * (DL + 1) + c + e] = k8[e];
-      vsm[r * DL + c + e] = v8[e];
+    for (int j = 0; j < CPR; ++j) {
+      float e8[EPC];
+      const TL *src = Ks + r * DL + (j ^ kv_swz<CPR>(r)) * EPC;
+      if constexpr (EPC == 8) {
+        load8(src, *reinterpret_cast<float(*)[8]>(e8));
+      } else {
+        const float4 f = *reinterpret_cast<const float4 *>(src);
+        e8[0] = f.x; e8[1] = f.y; e8[2] = f.z; e8[3] = f.w;
+      }
+#pragma unroll
+      for (int e = 0; e < EPC; ++e) kf[j * EPC + e] = e8[e];
+    }
+    for (int h = 0; h < G; ++h) {
+      const float4 *qh = reinterpret_cast<const float4 *>(qs + h * DL);
+      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+      for (int d4 = 0; d4 < DL / 4; ++d4) {
+        const float4 qv = qh[d4];
+        a0 = fmaf(qv.x, kf[4 * d4 + 0], a0);
+        a1 = fmaf(qv.y, kf[4 * d4 + 1], a1);
+        a2 = fmaf(qv.z, kf[4 * d4 + 2], a2);
+        a3 = fmaf(qv.w, kf[4 * d4 + 3], a3);
+      }
+      sc[h * CHUNK + r] = (a0 + a1) + (a2 + a3);
     }
   }
   __syncthreads();
-  for (int i = tid; i < G * n; i += blockDim.x) {
-    const int hh = i / n, s = i % n;
-    float acc = 0.f;
-    for (int d = 0; d < DL; ++d) acc = fmaf(qs[hh * DL + d], ks[s * (DL + 1) + d], acc);
-    sc[hh * CHUNK + s] = acc;
-  }
-  __syncthreads();
-  const int warp = tid >> 5, lane = tid & 31;
-  for (int hh = warp; hh < G; hh += blockDim.x / 32) {
+  // per-head chunk max and sum
+  for (int h = warp; h < G; h += blockDim.x / 32) {
     float mx = -INFINITY;
-    for (int s = lane; s < n; s += 32) mx = fmaxf(mx, sc[hh * CHUNK + s]);
+    for (int r = lane; r < n; r += 32) mx = fmaxf(mx, sc[h * CHUNK + r]);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
     float sum = 0.f;
-    for (int s = lane; s < n; s += 32) {
-      const float e = exp2f(sc[hh * CHUNK + s] - mx);
-      sc[hh * CHUNK + s] = e;
+    for (int r = lane; r < n; r += 32) {
+      const float e = exp2f(sc[h * CHUNK + r] - mx);
+      sc[h * CHUNK + r] = e;
       sum += e;
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
     if (lane == 0) {
-      ml[2 * hh] = mx;
-      ml[2 * hh + 1] = sum;
+      mls[2 * h] = mx;
+      mls[2 * h + 1] = sum;
+    }
+  }
+  __syncthreads();
+  // P V: thread (key slice ks, dim pair dp), 8 heads at a time
+  const int dp = tid % PAIRS, ks = tid / PAIRS;
+  for (int hb = 0; hb < G; hb += 8) {
+    float acc[8][2];
+#pragma unroll
+    for (int h = 0; h < 8; ++h) acc[h][0] = acc[h][1] = 0.f;
+    for (int r = ks; r < n; r += KS) {
+      float2 v;
+      if constexpr (sizeof(TL) == 2) {
+        v = __half22float2(*reinterpret_cast<const __half2 *>(Vs + r * DL + 2 * dp));
+      } else {
+        v = *reinterpret_cast<const float2 *>(Vs + r * DL + 2 * dp);
+      }
+#pragma unroll
+      for (int h = 0; h < 8; ++h) {
+        if (hb + h < G) {
+          const float pr = sc[(hb + h) * CHUNK + r];
+          acc[h][0] = fmaf(pr, v.x, acc[h][0]);
+          acc[h][1] = fmaf(pr, v.y, acc[h][1]);
+        }
+      }
+    }
+#pragma unroll
+    for (int h = 0; h < 8; ++h) {
+      if (hb + h < G) {
+        red[(ks * G + hb + h) * DL + 2 * dp] = acc[h][0];
+        red[(ks * G + hb + h) * DL + 2 * dp + 1] = acc[h][1];
+      }
     }
   }
   __syncthreads();
   for (int i = tid; i < G * DL; i += blockDim.x) {
-    const int hh = i / DL, d = i % DL;
-    float acc = 0.f;
-    for (int s = 0; s < n; ++s) acc = fmaf(sc[hh * CHUNK + s], vsm[s * DL + d], acc);
-    part_o[((static_cast<size_t>(b) * H + g * G + hh) * nchunk + ch) * DL + d] = acc;
+    float o = 0.f;
+#pragma unroll
+    for (int k = 0; k < KS; ++k) o += red[k * G * DL + i];
+    po[static_cast<size_t>(i / DL) * nchunk * DL + (i % DL)] = o;
   }
-  for (int hh = tid; hh < G; hh += blockDim.x) {
-    float *o = part_ml + ((static_cast<size_t>(b) * H + g * G + hh) * nchunk + ch) * 2;
-    o[0] = ml[2 * hh];
-    o[1] = ml[2 * hh + 1];
+  for (int h = tid; h < G; h += blockDim.x) {
+    pml[static_cast<size_t>(h) * nchunk * 2] = mls[2 * h];
+    pml[static_cast<size_t>(h) * nchunk * 2 + 1] = mls[2 * h + 1];
   }
 }
 
-// ------------------------------------------------------------------ D3b merge
-__global__ void decode_merge_kernel(const float *__restrict__ part_o,
-                                    const float *__restrict__ part_ml, const int *__restrict__ lengths,
-                                    float *__restrict__ o, int H, int DL, int max_seq, int nchunk) {
+// ------------------------------------------------------------------ D3b merge (+ advance)
+// One CTA per sequence: all (m, l) of its heads and chunks are staged in shared memory with
+// one parallel load, then each thread (head, dim) combines its chunks' partial outputs.  The
+// sequence's length advances here, after every kernel of the step that reads it.
+__global__ void __launch_bounds__(512) decode_merge_kernel(
+    const float *__restrict__ part_o, const float *__restrict__ part_ml, int *__restrict__ lengths,
+    float *__restrict__ o, int H, int DL, int max_seq, int nchunk) {
+  extern __shared__ float mls[];                      // [H][nused][2]
   const int b = blockIdx.x;
-  const bool full = lengths[b] >= max_seq;
-  const int nused = full ? 0 : min(nchunk, (lengths[b] + 1 + CHUNK - 1) / CHUNK);
+  const int L = lengths[b];
+  const bool full = L >= max_seq;
+  const int nused = full ? 0 : min(nchunk, (L + 1 + CHUNK - 1) / CHUNK);
+  for (int i = threadIdx.x; i < H * nused * 2; i += blockDim.x) {
+    const int h = i / (nused * 2), r = i % (nused * 2);
+    mls[i] = part_ml[(static_cast<size_t>(b) * H + h) * nchunk * 2 + r];
+  }
+  __syncthreads();
   for (int i = threadIdx.x; i < H * DL; i += blockDim.x) {
     const int h = i / DL, d = i % DL;
-    const float *ml = part_ml + (static_cast<size_t>(b) * H + h) * nchunk * 2;
+    const float *ml = mls + h * nused * 2;
     float mx = -INFINITY;
     for (int c = 0; c < nused; ++c) mx = fmaxf(mx, ml[2 * c]);
+    const float *po = part_o + (static_cast<size_t>(b) * H + h) * nchunk * DL + d;
     float l = 0.f, acc = 0.f;
+#pragma unroll 4
     for (int c = 0; c < nused; ++c) {
       const float w = exp2f(ml[2 * c] - mx);
-      l += w * ml[2 * c + 1];
-      acc += w * part_o[((static_cast<size_t>(b) * H + h) * nchunk + c) * DL + d];
+      l = fmaf(w, ml[2 * c + 1], l);
+      acc = fmaf(w, po[static_cast<size_t>(c) * DL], acc);
     }
     o[static_cast<size_t>(b) * H * DL + i] = nused > 0 ? acc / l : 0.f;
   }
-}
-
-__global__ void decode_advance_kernel(int *lengths, int B, int max_seq) {
-  const int b = blockIdx.x * blockDim.x + threadIdx.x;
-  if (b < B && lengths[b] < max_seq) lengths[b] += 1;
+  __syncthreads();
+  if (threadIdx.x == 0 && !full) lengths[b] = L + 1;
 }
 
 int decode_ksplit(const Dims &d) {
@@ -397,6 +473,23 @@ void decode_workspace_carve(const Dims &d, int max_seq, void *ws, DecodeArgs &a)
   a.chunk = CHUNK;
 }
 
+template <int DL, typename TL>
+static cudaError_t launch_decode_attn(const Dims &d, const DecodeArgs &a, float scale_log2,
+                                      cudaStream_t st) {
+  const int KS = 128 / (DL / 2);
+  const size_t smem = 2 * static_cast<size_t>(CHUNK) * DL * sizeof(TL) +
+                      (static_cast<size_t>(d.G) * DL + static_cast<size_t>(d.G) * CHUNK +
+                       static_cast<size_t>(KS) * d.G * DL + 2 * d.G) * 4;
+  cudaError_t e = cudaFuncSetAttribute(decode_attn_kernel<DL, TL>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  decode_attn_kernel<DL, TL><<<dim3(a.nchunk, d.Hkv, d.B), 128, smem, st>>>(
+      a.q_new, static_cast<const TL *>(a.k_cache), static_cast<const TL *>(a.v_cache), a.lengths,
+      a.part_o, a.part_ml, d.H, d.Hkv, d.G, a.max_seq, a.nchunk, scale_log2);
+  return cudaGetLastError();
+}
+
 template <typename T>
 static cudaError_t decode_typed(const Dims &d, const DecodeArgs &a, cudaStream_t st,
                                 const StageMarker &mark) {
@@ -432,30 +525,34 @@ static cudaError_t decode_typed(const Dims &d, const DecodeArgs &a, cudaStream_t
   p2.NQ = d.NQ; p2.NKV = d.NKV; p2.NQKV = d.NQKV; p2.KC = d.KC; p2.max_seq = a.max_seq;
   p2.flags = d.flags;
   p2.eps = d.eps;
-  p2.rope_base = d.rope_base;
+  for (int i = 0; i < d.DL / 2; ++i)
+    p2.theta[i] = pow(static_cast<double>(d.rope_base), -2.0 * i / d.DL);
   const size_t sm2 = (static_cast<size_t>(d.G + 2) * d.DL + 2 * (d.G + 1) * d.DL + (d.G + 1)) * 4;
   decode_stencil_kernel<T><<<dim3(d.Hkv, d.B), 128, sm2, st>>>(p2);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   mark();
   // D3
   const float scale_log2 = static_cast<float>(1.4426950408889634 / sqrt(static_cast<double>(d.DL)));
-  const size_t sm3 = (static_cast<size_t>(d.G) * d.DL + d.G * CHUNK + CHUNK * (d.DL + 1) +
-                      CHUNK * d.DL + 2 * d.G) * 4;
-  if (sm3 > 48 * 1024) {
-    e = cudaFuncSetAttribute(decode_attn_kernel<TL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(sm3));
-    if (e != cudaSuccess) return e;
-  }
-  decode_attn_kernel<TL><<<dim3(a.nchunk, d.Hkv, d.B), 128, sm3, st>>>(
-      a.q_new, static_cast<const TL *>(a.k_cache), static_cast<const TL *>(a.v_cache),
-      a.lengths,
-      a.part_o, a.part_ml, d.H, d.Hkv, d.G, d.DL, a.max_seq, a.nchunk, scale_log2);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (d.DL == 16) e = launch_decode_attn<16, TL>(d, a, scale_log2, st);
+  else if (d.DL == 32) e = launch_decode_attn<32, TL>(d, a, scale_log2, st);
+  else e = launch_decode_attn<64, TL>(d, a, scale_log2, st);
+  if (e != cudaSuccess) return e;
   mark();
-  decode_merge_kernel<<<d.B, 256, 0, st>>>(a.part_o, a.part_ml, a.lengths,
-                                            static_cast<float *>(a.o), d.H, d.DL, a.max_seq,
-                                               a.nchunk);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  // D3b (+ lengths advance)
+  {
+    const int nused_max = a.nchunk;
+    const size_t smm = static_cast<size_t>(d.H) * nused_max * 2 * 4;
+    if (smm > 48 * 1024) {
+      e = cudaFuncSetAttribute(decode_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smm));
+      if (e != cudaSuccess) return e;
+    }
+    const int threads = d.H * d.DL < 512 ? ((d.H * d.DL + 31) / 32) * 32 : 512;
+    decode_merge_kernel<<<d.B, threads, smm, st>>>(a.part_o, a.part_ml, a.lengths,
+                                                   static_cast<float *>(a.o), d.H, d.DL,
+                                                   a.max_seq, a.nchunk);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
   mark();
   // D4
   if constexpr (sizeof(T) == 2) {
@@ -467,8 +564,6 @@ static cudaError_t decode_typed(const Dims &d, const DecodeArgs &a, cudaStream_t
     e = gemm_simt(0, a.o, a.w_o, a.y, d.B, d.E, d.NQ, st);
     if (e != cudaSuccess) return e;
   }
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  decode_advance_kernel<<<(d.B + 127) / 128, 128, 0, st>>>(a.lengths, d.B, a.max_seq);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   mark();
   return cudaSuccess;

@@ -52,6 +52,7 @@ struct StencilArgs {
   const float *P;
   const float *conv_seq;
   const float *conv_chan;
+  const void *conv_chan_split = nullptr;   // 16-bit layers: output of split_conv_chan
   void *q, *k, *v;
   int kv_stride;
   float *conv_state;    // [B, KC-1, NQ+NKV]
@@ -61,6 +62,10 @@ struct StencilArgs {
   bool write_state = false;
 };
 cudaError_t latent_stencil(const Dims &d, const StencilArgs &a, cudaStream_t st);
+// The channel-conv weights of a 16-bit layer as {bf16x2 hi, bf16x2 lo} per pair of inputs
+// (conv_chan_split_bytes of scratch); the stencil's tensor-core path reads them.
+size_t conv_chan_split_bytes(const Dims &d);
+cudaError_t split_conv_chan(const Dims &d, const float *conv_chan, void *out, cudaStream_t st);
 
 // Causal latent attention: q [B, H, S, DL], k/v [B, Hkv, kv_stride, DL] -> o [B*S, NQ].
 cudaError_t latent_attention(const Dims &d, const void *q, const void *k, const void *v,

@@ -1,5 +1,5 @@
 // Latent stencil of the prefill: everything between the down-projection and the attention,
-// fused into one pass over the projected latents P = x W_qkv^T.
+// fused into one pass over the projected latents P = x W_qkv^T (float32).
 //
 // For every token t and key/value group g (gist.science explainer, 2. Methodology, Core
 // Mechanism; edgentiq, "How Compressed Convolutional Attention Works"):
@@ -12,7 +12,13 @@
 // One CTA owns a tile of TT tokens of one group of one sequence: it stages the group's
 // P rows (plus a halo of KC-1 earlier tokens) in shared memory once, and writes q in
 // head-major layout [B, H, S, d~] and k, v in [B, Hkv, kv_stride, d~] (the decode cache when
-// one is given), as float16 for 16-bit layers.  Float32 arithmetic throughout.
+// one is given), as float16 for 16-bit layers.
+//
+// Channel conv: for 16-bit layers on the tensor cores (mma.sync m16n8k16), one warp per
+// (head, 16 tokens), with both operands split into bfloat16 leading terms and remainders
+// (a w ~ a_hi w_hi + a_hi w_lo + a_lo w_hi, about 16 significand bits); the norm and RoPE
+// then run in the accumulator layout (a quad of lanes holds one token's head vector, and
+// channels i and i + d~/2 sit in the same lane).  Float32 layers use exact fp32 FMAs.
 #include <math.h>
 
 #include "common.cuh"
@@ -27,6 +33,7 @@ struct StencilParams {
   const float *P;
   const float *conv_seq;
   const float *conv_chan;
+  const uint2 *conv_chan_split;   // 16-bit layers: conv_chan as bf16 hi/lo pairs
   TL *q, *k, *v;
   float *conv_state, *vshift_state;
   int *lengths;
@@ -35,151 +42,245 @@ struct StencilParams {
   int B, S, H, Hkv, G, NQ, NKV, NQKV, KC, halo, TT, kv_stride;
   unsigned flags;
   float eps;
-  float rope_base;
+  double theta[32];        // RoPE frequencies base^(-2i/d~), i < d~/2, computed on the host
 };
 
-__host__ __device__ inline int stencil_ch(int G, int DL) { return (G + 2) * DL; }
+// Padded row strides (floats) of the staged P rows and of the sequence-conv output: +4 keeps
+// the 8-row fragment loads of the tensor-core path free of bank conflicts.
+__host__ __device__ inline int ch_pad(int G, int DL) { return (G + 2) * DL + 4; }
+__host__ __device__ inline int qkc_pad(int G, int DL) { return (G + 1) * DL + 4; }
+
+__host__ __device__ inline size_t stencil_smem_floats(int G, int DL, int TT, int halo, bool simt) {
+  return static_cast<size_t>(TT + halo) * ch_pad(G, DL)        // Ps
+         + static_cast<size_t>(TT) * qkc_pad(G, DL)            // As
+         + static_cast<size_t>(TT) * DL                        // cos/sin table
+         + (simt ? static_cast<size_t>(DL) * (DL + 1) : 0);   // Ws (float32 path)
+}
 
 template <int DL>
-__host__ __device__ inline size_t stencil_smem_floats(int G, int TT, int halo) {
-  return static_cast<size_t>(TT + halo) * stencil_ch(G, DL)      // Ps
-         + static_cast<size_t>(TT) * (G + 1) * DL                // As
-         + static_cast<size_t>(DL) * (DL + 1)                    // Ws
-         + static_cast<size_t>(TT) * DL;                         // cos/sin table
+__device__ __forceinline__ float qk_mean_term(const float *prow, int G, int hh, int i) {
+  const float pk = prow[G * DL + i];
+  if (hh < G) return 0.5f * (prow[hh * DL + i] + pk);
+  float mq = 0.f;
+  for (int h2 = 0; h2 < G; ++h2) mq += prow[h2 * DL + i];
+  return 0.5f * (mq / static_cast<float>(G) + pk);
 }
 
 template <typename T, int DL>
-__global__ void __launch_bounds__(256) stencil_kernel(const StencilParams<T> p) {
+__global__ void __launch_bounds__(512) stencil_kernel(const StencilParams<T> p) {
   using TL = typename StencilParams<T>::TL;
-  constexpr int LPI = DL < 32 ? DL : 32;   // lanes per (token, head) item
-  constexpr int EPL = DL / LPI;            // elements per lane
-  constexpr int IPW = 32 / LPI;            // items per warp pass
+  constexpr bool kTensor = sizeof(T) == 2;
   constexpr int HALF = DL / 2;
   extern __shared__ float sm[];
-  const int G = p.G, CH = stencil_ch(G, DL), QKC = (G + 1) * DL;
+  const int G = p.G, QKC = (G + 1) * DL;
+  const int CHP = ch_pad(G, DL), QKCP = qkc_pad(G, DL);
   const int TT = p.TT, halo = p.halo;
-  float *Ps = sm;                                   // [TT+halo][CH]
-  float *As = Ps + (TT + halo) * CH;                // [TT][QKC]
-  float *Ws = As + TT * QKC;                        // [DL][DL+1]
-  float *Rt = Ws + DL * (DL + 1);                   // [TT][HALF][2]
+  float *Ps = sm;                                   // [TT+halo][CHP]
+  float *As = Ps + (TT + halo) * CHP;               // [TT][QKCP]
+  float *Rt = As + TT * QKCP;                       // [TT][HALF][2]
+  float *Ws = Rt + TT * DL;                         // [DL][DL+1] (float32 path)
 
   const int g = blockIdx.y, b = blockIdx.z;
   const int t0 = blockIdx.x * TT;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nwarps = blockDim.x >> 5;
   const int qcol0 = g * G * DL;                     // group's q channels in P
   const int kcol0 = p.NQ + g * DL;
   const int vcol0 = p.NQ + p.NKV + g * DL;
+  const int CH = (G + 2) * DL;
 
-  // 1. stage P rows t0-halo .. t0+TT-1 of the group's channels (zero outside [0, S)).
-  const int vec_per_row = CH / 8;
+  // 1. stage P rows t0-halo .. t0+TT-1 of the group's channels (zero outside [0, S)) with
+  //    16-byte asynchronous copies, so every thread has all of its loads in flight at once.
+  const int vec_per_row = CH / 4;
   for (int i = tid; i < (TT + halo) * vec_per_row; i += blockDim.x) {
-    const int r = i / vec_per_row, c = (i % vec_per_row) * 8;
+    const int r = i / vec_per_row, c = (i % vec_per_row) * 4;
     const int t = t0 - halo + r;
-    float v8[8];
-    if (t >= 0 && t < p.S) {
-      const int gc = c < G * DL ? qcol0 + c : (c < QKC ? kcol0 + (c - G * DL) : vcol0 + (c - QKC));
-      load8(p.P + (static_cast<size_t>(b) * p.S + t) * p.NQKV + gc, v8);
-    } else {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) v8[e] = 0.f;
-    }
-#pragma unroll
-    for (int e = 0; e < 8; ++e) Ps[r * CH + c + e] = v8[e];
+    const bool in = t >= 0 && t < p.S;
+    const int gc = c < G * DL ? qcol0 + c : (c < QKC ? kcol0 + (c - G * DL) : vcol0 + (c - QKC));
+    const float *src = in ? p.P + (static_cast<size_t>(b) * p.S + t) * p.NQKV + gc : p.P;
+    cp_async16_zfill(Ps + r * CHP + c, src, in);
   }
-  // RoPE table for this tile: angle = t * base^(-2i/d~), evaluated in double.
+  cp_async_wait_all();
+  // RoPE table for this tile: angle = t * base^(-2i/d~).
   if (p.flags & F_ROPE) {
     for (int i = tid; i < TT * HALF; i += blockDim.x) {
       const int tt = i / HALF, ip = i % HALF;
-      const double theta = pow(static_cast<double>(p.rope_base), -2.0 * ip / DL);
-      double s, c;
-      sincos(static_cast<double>(t0 + tt) * theta, &s, &c);
-      Rt[2 * i] = static_cast<float>(c);
-      Rt[2 * i + 1] = static_cast<float>(s);
+      rope_cos_sin(static_cast<double>(t0 + tt) * p.theta[ip], Rt[2 * i], Rt[2 * i + 1]);
     }
   }
   __syncthreads();
 
-  // 2. causal depthwise sequence conv of the q|k channels.
-  for (int i = tid; i < TT * QKC; i += blockDim.x) {
-    const int tt = i / QKC, c = i % QKC;
+  // 2. causal depthwise sequence conv of the q|k channels: one thread per channel, its
+  //    filter in registers, sliding along the tile's tokens (KC <= 8).
+  for (int c = tid; c < QKC; c += blockDim.x) {
     const int gc = c < G * DL ? qcol0 + c : p.NQ + g * DL + (c - G * DL);
-    const float *w = p.conv_seq + static_cast<size_t>(gc) * p.KC;
-    float a = 0.f;
-    const int r0 = tt + halo - (p.KC - 1);
-    for (int j = 0; j < p.KC; ++j) a = fmaf(w[j], Ps[(r0 + j) * CH + c], a);
-    As[tt * QKC + c] = a;
+    const int KC1 = p.KC - 1;
+    float wprev[7], prev[7], wcur = 0.f;
+    const int r0 = halo - KC1;                      // Ps row of token t0 - (KC-1)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float wj = j < p.KC ? __ldg(p.conv_seq + static_cast<size_t>(gc) * p.KC + j) : 0.f;
+      if (j < 7) wprev[j] = j < KC1 ? wj : 0.f;
+      if (j == KC1) wcur = wj;
+    }
+#pragma unroll
+    for (int j = 0; j < 7; ++j) prev[j] = j < KC1 ? Ps[(r0 + j) * CHP + c] : 0.f;
+    for (int tt = 0; tt < TT; ++tt) {
+      const float cur = Ps[(halo + tt) * CHP + c];  // token t0 + tt
+      float a = wcur * cur;
+#pragma unroll
+      for (int j = 0; j < 7; ++j) a = fmaf(wprev[j], prev[j], a);
+      As[tt * QKCP + c] = a;
+#pragma unroll
+      for (int j = 0; j < 7; ++j) prev[j] = j + 1 < KC1 ? prev[j + 1] : (j + 1 == KC1 ? cur : prev[j]);
+    }
   }
+  __syncthreads();
 
   // 3. per head: channel conv, q-k-mean, RMS norm, RoPE, store.
-  for (int hh = 0; hh <= G; ++hh) {
-    const bool is_q = hh < G;
-    const int head_w = is_q ? g * G + hh : p.H + g;     // row block of conv_chan
-    __syncthreads();                                    // As ready / previous Ws consumed
-    for (int i = tid; i < DL * DL; i += blockDim.x)
-      Ws[(i / DL) * (DL + 1) + (i % DL)] = p.conv_chan[static_cast<size_t>(head_w) * DL * DL + i];
-    __syncthreads();
-    const int sub = lane / LPI, li = lane % LPI;
-    for (int tt0 = warp * IPW; tt0 < TT; tt0 += (blockDim.x / 32) * IPW) {
-      const int tt = tt0 + sub;
-      const bool valid_tt = tt < TT;
-      const int ttc = valid_tt ? tt : TT - 1;
-      float u[EPL];
+  if constexpr (kTensor) {
+    constexpr int NT = DL / 8;                      // n-tiles of 8 output channels
+    const int MT = TT / 16;
+    const int gr = lane >> 2, qc = lane & 3;
+    for (int task = warp; task < (G + 1) * MT; task += nwarps) {
+      const int hh = task / MT, mt = task % MT;
+      const bool is_q = hh < G;
+      // pre-split weights: for (head, n, k-pair) one uint2 {bf16x2 hi, bf16x2 lo}
+      const uint2 *wb = p.conv_chan_split +
+                        static_cast<size_t>(is_q ? g * G + hh : p.H + g) * DL * (DL / 2);
+      float acc[NT][4];
 #pragma unroll
-      for (int e = 0; e < EPL; ++e) {
-        const int i = e * LPI + li;
-        const float *arow = As + ttc * QKC + hh * DL;
-        const float *wrow = Ws + i * (DL + 1);
-        float acc = 0.f;
-#pragma unroll 8
-        for (int j = 0; j < DL; ++j) acc = fmaf(wrow[j], arow[j], acc);
-        if (p.flags & F_QK_MEAN) {
-          const float *prow = Ps + (ttc + halo) * CH;
-          const float pk = prow[G * DL + i];
-          if (is_q) {
-            acc += 0.5f * (prow[hh * DL + i] + pk);
-          } else {
-            float mq = 0.f;
-            for (int h2 = 0; h2 < G; ++h2) mq += prow[h2 * DL + i];
-            acc += 0.5f * (mq / static_cast<float>(G) + pk);
+      for (int n = 0; n < NT; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
+      const float *a0p = As + (mt * 16 + gr) * QKCP + hh * DL;
+      const float *a1p = a0p + 8 * QKCP;
+#pragma unroll
+      for (int ks = 0; ks < DL / 16; ++ks) {
+        const int k0 = ks * 16 + 2 * qc;
+        uint32_t ah[4], al[4];
+        split_bf16x2(*reinterpret_cast<const float2 *>(a0p + k0), ah[0], al[0]);
+        split_bf16x2(*reinterpret_cast<const float2 *>(a1p + k0), ah[1], al[1]);
+        split_bf16x2(*reinterpret_cast<const float2 *>(a0p + k0 + 8), ah[2], al[2]);
+        split_bf16x2(*reinterpret_cast<const float2 *>(a1p + k0 + 8), ah[3], al[3]);
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+          const uint2 *wr = wb + (n * 8 + gr) * (DL / 2) + k0 / 2;
+          const uint2 w0 = __ldg(wr), w1 = __ldg(wr + 4);
+          const uint32_t bh[2] = {w0.x, w1.x}, bl[2] = {w0.y, w1.y};
+          mma_bf16_16816(acc[n], ah, bh);
+          mma_bf16_16816(acc[n], ah, bl);
+          mma_bf16_16816(acc[n], al, bh);
+        }
+      }
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int tt = mt * 16 + gr + half * 8;
+        const float *prow = Ps + (tt + halo) * CHP;
+        float u[NT][2];
+#pragma unroll
+        for (int n = 0; n < NT; ++n)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int i = n * 8 + 2 * qc + e;
+            float v = acc[n][half * 2 + e];
+            if (p.flags & F_QK_MEAN) v += qk_mean_term<DL>(prow, G, hh, i);
+            u[n][e] = v;
+          }
+        if (p.flags & F_QK_NORM) {
+          float ss = 0.f;
+#pragma unroll
+          for (int n = 0; n < NT; ++n) ss += u[n][0] * u[n][0] + u[n][1] * u[n][1];
+          ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+          ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+          const float inv = 1.0f / sqrtf(ss / static_cast<float>(DL) + p.eps);
+#pragma unroll
+          for (int n = 0; n < NT; ++n) {
+            u[n][0] *= inv;
+            u[n][1] *= inv;
           }
         }
-        u[e] = acc;
-      }
-      if (p.flags & F_QK_NORM) {
-        float ss = 0.f;
+        if (p.flags & F_ROPE) {
 #pragma unroll
-        for (int e = 0; e < EPL; ++e) ss += u[e] * u[e];
+          for (int n = 0; n < NT / 2; ++n)
 #pragma unroll
-        for (int off = LPI / 2; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-        const float inv = 1.0f / sqrtf(ss / static_cast<float>(DL) + p.eps);
+            for (int e = 0; e < 2; ++e) {
+              const int i = n * 8 + 2 * qc + e;      // < d~/2; partner i + d~/2 is n-tile n+NT/2
+              const float c = Rt[(tt * HALF + i) * 2], s = Rt[(tt * HALF + i) * 2 + 1];
+              const float x1 = u[n][e], x2 = u[n + NT / 2][e];
+              u[n][e] = x1 * c - x2 * s;
+              u[n + NT / 2][e] = x1 * s + x2 * c;
+            }
+        }
+        const int t = t0 + tt;
+        if (t < p.S) {
+          TL *dst = is_q ? p.q + ((static_cast<size_t>(b) * p.H + g * G + hh) * p.S + t) * DL
+                         : p.k + ((static_cast<size_t>(b) * p.Hkv + g) * p.kv_stride + t) * DL;
 #pragma unroll
-        for (int e = 0; e < EPL; ++e) u[e] *= inv;
-      }
-      if (p.flags & F_ROPE) {
-        if constexpr (EPL == 2) {
-          const float c = Rt[(ttc * HALF + li) * 2], s = Rt[(ttc * HALF + li) * 2 + 1];
-          const float x1 = u[0], x2 = u[1];
-          u[0] = x1 * c - x2 * s;
-          u[1] = x1 * s + x2 * c;
-        } else {
-          const float other = __shfl_xor_sync(0xffffffffu, u[0], HALF);
-          const int ip = li % HALF;
-          const float c = Rt[(ttc * HALF + ip) * 2], s = Rt[(ttc * HALF + ip) * 2 + 1];
-          u[0] = li < HALF ? u[0] * c - other * s : other * s + u[0] * c;
+          for (int n = 0; n < NT; ++n) {
+            check_latent<TL>(u[n][0], p.status);
+            check_latent<TL>(u[n][1], p.status);
+            *reinterpret_cast<uint32_t *>(dst + n * 8 + 2 * qc) = pack_f16x2(u[n][0], u[n][1]);
+          }
         }
       }
-      const int t = t0 + tt;
-      if (valid_tt && t < p.S) {
+    }
+  } else {
+    constexpr int LPI = DL < 32 ? DL : 32;   // lanes per (token, head) item
+    constexpr int EPL = DL / LPI;            // elements per lane
+    constexpr int IPW = 32 / LPI;            // items per warp pass
+    for (int hh = 0; hh <= G; ++hh) {
+      const bool is_q = hh < G;
+      const int head_w = is_q ? g * G + hh : p.H + g;
+      __syncthreads();                                  // previous Ws consumed
+      for (int i = tid; i < DL * DL; i += blockDim.x)
+        Ws[(i / DL) * (DL + 1) + (i % DL)] = p.conv_chan[static_cast<size_t>(head_w) * DL * DL + i];
+      __syncthreads();
+      const int sub = lane / LPI, li = lane % LPI;
+      for (int tt0 = warp * IPW; tt0 < TT; tt0 += nwarps * IPW) {
+        const int tt = tt0 + sub;
+        float u[EPL];
 #pragma unroll
         for (int e = 0; e < EPL; ++e) {
           const int i = e * LPI + li;
-          check_latent<TL>(u[e], p.status);
-          if (is_q) {
-            const int h = g * G + hh;
-            p.q[((static_cast<size_t>(b) * p.H + h) * p.S + t) * DL + i] = from_f32<TL>(u[e]);
+          const float *arow = As + tt * QKCP + hh * DL;
+          const float *wrow = Ws + i * (DL + 1);
+          float acc = 0.f;
+#pragma unroll 8
+          for (int j = 0; j < DL; ++j) acc = fmaf(wrow[j], arow[j], acc);
+          if (p.flags & F_QK_MEAN) acc += qk_mean_term<DL>(Ps + (tt + halo) * CHP, G, hh, i);
+          u[e] = acc;
+        }
+        if (p.flags & F_QK_NORM) {
+          float ss = 0.f;
+#pragma unroll
+          for (int e = 0; e < EPL; ++e) ss += u[e] * u[e];
+#pragma unroll
+          for (int off = LPI / 2; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+          const float inv = 1.0f / sqrtf(ss / static_cast<float>(DL) + p.eps);
+#pragma unroll
+          for (int e = 0; e < EPL; ++e) u[e] *= inv;
+        }
+        if (p.flags & F_ROPE) {
+          if constexpr (EPL == 2) {
+            const float c = Rt[(tt * HALF + li) * 2], s = Rt[(tt * HALF + li) * 2 + 1];
+            const float x1 = u[0], x2 = u[1];
+            u[0] = x1 * c - x2 * s;
+            u[1] = x1 * s + x2 * c;
           } else {
-            p.k[((static_cast<size_t>(b) * p.Hkv + g) * p.kv_stride + t) * DL + i] =
-                from_f32<TL>(u[e]);
+            const float other = __shfl_xor_sync(0xffffffffu, u[0], HALF);
+            const int ip = li % HALF;
+            const float c = Rt[(tt * HALF + ip) * 2], s = Rt[(tt * HALF + ip) * 2 + 1];
+            u[0] = li < HALF ? u[0] * c - other * s : other * s + u[0] * c;
+          }
+        }
+        const int t = t0 + tt;
+        if (t < p.S) {
+#pragma unroll
+          for (int e = 0; e < EPL; ++e) {
+            const int i = e * LPI + li;
+            if (is_q)
+              p.q[((static_cast<size_t>(b) * p.H + g * G + hh) * p.S + t) * DL + i] = from_f32<TL>(u[e]);
+            else
+              p.k[((static_cast<size_t>(b) * p.Hkv + g) * p.kv_stride + t) * DL + i] = from_f32<TL>(u[e]);
           }
         }
       }
@@ -188,14 +289,20 @@ __global__ void __launch_bounds__(256) stencil_kernel(const StencilParams<T> p) 
 
   // 4. values with the value-shift: upper half of the value channels from token t-1.
   const int vhalf = p.NKV / 2;
-  for (int i = tid; i < TT * DL; i += blockDim.x) {
-    const int tt = i / DL, c = i % DL;
+  for (int i = tid; i < TT * (DL / 2); i += blockDim.x) {
+    const int tt = i / (DL / 2), c = (i % (DL / 2)) * 2;
     const int t = t0 + tt;
     if (t >= p.S) continue;
-    const bool shifted = (p.flags & F_VALUE_SHIFT) && (g * DL + c >= vhalf);
-    const float val = Ps[(tt + halo - (shifted ? 1 : 0)) * CH + QKC + c];
-    check_latent<TL>(val, p.status);
-    p.v[((static_cast<size_t>(b) * p.Hkv + g) * p.kv_stride + t) * DL + c] = from_f32<TL>(val);
+    float val[2];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const bool shifted = (p.flags & F_VALUE_SHIFT) && (g * DL + c + e >= vhalf);
+      val[e] = Ps[(tt + halo - (shifted ? 1 : 0)) * CHP + QKC + c + e];
+      check_latent<TL>(val[e], p.status);
+    }
+    TL *dst = p.v + ((static_cast<size_t>(b) * p.Hkv + g) * p.kv_stride + t) * DL + c;
+    dst[0] = from_f32<TL>(val[0]);
+    dst[1] = from_f32<TL>(val[1]);
   }
 
   // 5. decode state after the last token, written by the tile that holds it.
@@ -207,14 +314,14 @@ __global__ void __launch_bounds__(256) stencil_kernel(const StencilParams<T> p) 
       const int ts = p.S - KC1 + j;
       const int r = ts - t0 + halo;
       const int gc = c < G * DL ? qcol0 + c : p.NQ + g * DL + (c - G * DL);
-      p.conv_state[(static_cast<size_t>(b) * KC1 + j) * W + gc] = Ps[r * CH + c];
+      p.conv_state[(static_cast<size_t>(b) * KC1 + j) * W + gc] = Ps[r * CHP + c];
     }
     const int rl = p.S - 1 - t0 + halo;
     for (int c = tid; c < DL; c += blockDim.x) {
       const int gch = g * DL + c;
       if (gch >= vhalf)
         p.vshift_state[static_cast<size_t>(b) * (p.NKV - vhalf) + (gch - vhalf)] =
-            Ps[rl * CH + QKC + c];
+            Ps[rl * CHP + QKC + c];
     }
     if (g == 0 && tid == 0) p.lengths[b] = p.S;
   }
@@ -223,10 +330,12 @@ __global__ void __launch_bounds__(256) stencil_kernel(const StencilParams<T> p) 
 template <typename T, int DL>
 cudaError_t launch(const Dims &d, const StencilArgs &a, cudaStream_t st) {
   using TL = typename LatentType<T>::type;
+  constexpr bool simt = sizeof(T) == 4;
   StencilParams<T> p;
   p.P = a.P;
   p.conv_seq = a.conv_seq;
   p.conv_chan = a.conv_chan;
+  p.conv_chan_split = static_cast<const uint2 *>(a.conv_chan_split);
   p.q = static_cast<TL *>(a.q);
   p.k = static_cast<TL *>(a.k);
   p.v = static_cast<TL *>(a.v);
@@ -241,22 +350,51 @@ cudaError_t launch(const Dims &d, const StencilArgs &a, cudaStream_t st) {
   p.kv_stride = a.kv_stride;
   p.flags = d.flags;
   p.eps = d.eps;
-  p.rope_base = d.rope_base;
+  for (int i = 0; i < DL / 2; ++i)
+    p.theta[i] = pow(static_cast<double>(d.rope_base), -2.0 * i / DL);
+  // Largest token tile (a multiple of 16) whose staging fits two CTAs per SM.
+  const size_t budget = (simt ? 72 : 110) * 1024;
   int TT = 64;
-  while (TT > 4 && stencil_smem_floats<DL>(d.G, TT, p.halo) * 4 > 72 * 1024) TT /= 2;
+  while (TT > 16 && stencil_smem_floats(d.G, DL, TT, p.halo, simt) * 4 > budget) TT /= 2;
   p.TT = TT;
-  const size_t smem = stencil_smem_floats<DL>(d.G, TT, p.halo) * 4;
-  if (smem > 200 * 1024) return cudaErrorInvalidConfiguration;
+  const size_t smem = stencil_smem_floats(d.G, DL, TT, p.halo, simt) * 4;
+  if (smem > 220 * 1024) return cudaErrorInvalidConfiguration;
   cudaError_t e = cudaFuncSetAttribute(stencil_kernel<T, DL>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
+  int threads = 256;
+  if (!simt) {
+    const int tasks = (d.G + 1) * (TT / 16);      // (head, 16-token) channel-conv tasks
+    threads = 32 * (tasks < 4 ? 4 : tasks > 16 ? 16 : tasks);
+  }
   dim3 grid((d.S + TT - 1) / TT, d.Hkv, d.B);
-  stencil_kernel<T, DL><<<grid, 256, smem, st>>>(p);
+  stencil_kernel<T, DL><<<grid, threads, smem, st>>>(p);
   return cudaGetLastError();
 }
 
+__global__ void split_conv_chan_kernel(const float *__restrict__ w, uint2 *__restrict__ out,
+                                       size_t npairs) {
+  for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < npairs;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    uint2 r;
+    split_bf16x2(*reinterpret_cast<const float2 *>(w + 2 * i), r.x, r.y);
+    out[i] = r;
+  }
+}
+
 }  // namespace
+
+size_t conv_chan_split_bytes(const Dims &d) {
+  return d.bf16 ? static_cast<size_t>(d.H + d.Hkv) * d.DL * d.DL * 4 : 0;
+}
+
+cudaError_t split_conv_chan(const Dims &d, const float *conv_chan, void *out, cudaStream_t st) {
+  const size_t npairs = static_cast<size_t>(d.H + d.Hkv) * d.DL * d.DL / 2;
+  const unsigned blocks = static_cast<unsigned>((npairs + 255) / 256 < 1024 ? (npairs + 255) / 256 : 1024);
+  split_conv_chan_kernel<<<blocks, 256, 0, st>>>(conv_chan, static_cast<uint2 *>(out), npairs);
+  return cudaGetLastError();
+}
 
 cudaError_t latent_stencil(const Dims &d, const StencilArgs &a, cudaStream_t st) {
   if (d.B == 0 || d.S == 0) return cudaSuccess;

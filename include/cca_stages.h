@@ -29,7 +29,12 @@ CCA_API int cca_gemm(int dtype, int out_dtype, const void *A, const void *B, voi
  * as selected by cfg->flags (gist.science explainer, 2. Methodology, Core Mechanism). */
 CCA_API int cca_stage_stencil(const cca_config_t *cfg, const void *P, int batch, int seq,
                               const float *conv_seq, const float *conv_chan, void *q, void *k,
-                              void *v, int kv_stride, void *stream);
+                              void *v, int kv_stride, void *workspace, size_t ws_bytes,
+                              void *stream);
+
+/* Scratch bytes cca_stage_stencil needs (its first 256 bytes are a status word read by
+ * cca_workspace_status; the rest holds the channel-conv weights split for the tensor cores). */
+CCA_API size_t cca_stage_stencil_workspace_size(const cca_config_t *cfg);
 
 /* Causal latent attention: q [batch, H, seq, d~], k/v [batch, Hkv, kv_stride, d~] ->
  * o [batch*seq, H*d~] (token-major; q, k, v and o of the latent element type of cca.h), scale 1/sqrt(d~), query head h reads kv head

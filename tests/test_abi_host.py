@@ -54,7 +54,7 @@ def test_workspace_and_cache_sizes(lib):
     M = B * S
     nq, nkv = 16 * 32, 4 * 32
     al = lambda x: (x + 255) // 256 * 256
-    expect = 256 + al(2048 * nq * 2) + al(M * (nq + 2 * nkv) * 4) + al(M * nq * 2) + 2 * al(M * nkv * 2) + al(M * nq * 2)
+    expect = 256 + al(2048 * nq * 2) + al((16 + 4) * 32 * 32 * 4) + al(M * (nq + 2 * nkv) * 4) + al(M * nq * 2) + 2 * al(M * nkv * 2) + al(M * nq * 2)
     assert cls.cca_prefill_workspace_size(c, B, S) == expect
     # cache: keys and values are n_kv wide per token: C * H/Hkv = 16x smaller than MHA's 2E
     nbytes = cls.cca_cache_alloc(c, 3, 1000)

@@ -82,9 +82,10 @@ def test_stencil_matches_oracle(cuda_lib, dtype, H, Hkv, C, E, S):
     k = torch.empty(2, Hkv, S + 5, w.dl, dtype=w.latent_dtype, device="cuda")
     v = torch.empty(2, Hkv, S + 5, w.dl, dtype=w.latent_dtype, device="cuda")
     cfg = cls.make_config(E, H, Hkv, C, dtype=cls.CCA_BF16 if dtype == "bf16" else cls.CCA_F32)
+    ws = torch.empty(cls.cca_stage_stencil_workspace_size(cfg), dtype=torch.uint8, device="cuda")
     cls.cca_stage_stencil(cfg, P.cuda(), 2, S, inp.conv_seq.cuda(), inp.conv_chan.cuda(), q, k, v,
-                          S + 5)
-    torch.cuda.synchronize()
+                          S + 5, ws)
+    cls.cca_workspace_status(ws)
     ow = oracle_weights(ocfg, inp)
     for b in range(2):
         p = f64(P[b * S:(b + 1) * S])
