@@ -379,6 +379,8 @@ CCA_API int cca_decode_step(const cca_config_t *cfg, const cca_weights_t *w, con
     return fail(CCA_ERR_INVALID_ARG, "weights (or one of their pointers) NULL");
   if (!cache) return fail(CCA_ERR_INVALID_ARG, "cache is NULL");
   if ((rc = check_cache(d, cache))) return rc;
+  if (d.G > 8)
+    return fail(CCA_ERR_UNSUPPORTED, "decode takes at most 8 query heads per kv head (got %d)", d.G);
   if (!x || !y) return fail(CCA_ERR_INVALID_ARG, "x or y NULL");
   if (!aligned16(x) || !aligned16(y) || !aligned16(w->w_qkv) || !aligned16(w->w_o) ||
       !aligned16(workspace))

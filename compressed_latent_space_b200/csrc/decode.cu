@@ -20,7 +20,7 @@
 namespace cca {
 namespace {
 
-constexpr int CHUNK = 512;        // keys per split-KV block
+constexpr int CHUNK = 1024;       // keys per split-KV block
 
 // ------------------------------------------------------------------ D1 / D4 skinny GEMM
 // C[M, N] = A[M, K] * B[N, K]^T for small M (the batch), bf16 operands on mma.sync.
@@ -241,14 +241,18 @@ __global__ void __launch_bounds__(128) decode_stencil_kernel(const D2Params<T> p
 }
 
 // ------------------------------------------------------------------ D3 split-KV attention
-// One CTA per (sequence, kv group, chunk of CHUNK keys).  The chunk's keys and values are
-// brought into shared memory with 16-byte asynchronous copies issued all at once (keys with
-// their 16-byte pieces XOR-swizzled by row, so the one-row-per-thread reads below hit eight
-// different bank groups), then:
-//   scores  one thread per key, the G queries of the group broadcast from shared memory
-//   softmax one warp per head: chunk max m, p = 2^(s - m), chunk sum l
-//   P V     thread (dim pair, key slice) accumulates G heads x 2 dims, slices summed at the end
-// Partial results (unnormalised o, m, l) go to the workspace for the merge.
+// One CTA per (sequence, kv group, split of CHUNK keys).  The split is walked in sub-chunks of
+// SUB keys through a two-deep ring of 16-byte asynchronous copies, so the copy of sub-chunk
+// i+1 is in flight while sub-chunk i is computed.  Keys land with their 16-byte pieces
+// XOR-swizzled by row (the one-row-per-thread reads below then hit eight bank groups).
+// Per sub-chunk:
+//   scores  one thread per key, the group's G queries broadcast from shared memory
+//   softmax one warp per head: running max m and sum l across sub-chunks; the P V
+//           accumulators are rescaled by 2^(m_old - m_new) when the max moves
+//   P V     thread (dim pair, key slice) accumulates G heads x 2 dims
+// The split's unnormalised o and its (m, l) go to the workspace for the merge.
+constexpr int SUB = 256;
+
 template <int CPR>
 __device__ __forceinline__ int kv_swz(int r) {       // swizzle of a row's 16-byte pieces
   constexpr int SPAN = CPR < 8 ? CPR : 8;
@@ -266,13 +270,15 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(
   constexpr int CPR = DL / EPC;                      // pieces per row
   constexpr int PAIRS = DL / 2;
   constexpr int KS = 128 / PAIRS;                    // key slices in the P V phase
+  constexpr int GMAX = 8;                            // heads per P V pass
   extern __shared__ __align__(16) uint8_t smraw[];
-  TL *Ks = reinterpret_cast<TL *>(smraw);            // [CHUNK][DL], swizzled pieces
-  TL *Vs = Ks + CHUNK * DL;                          // [CHUNK][DL]
-  float *qs = reinterpret_cast<float *>(Vs + CHUNK * DL);   // [G][DL], pre-scaled
-  float *sc = qs + G * DL;                           // [G][CHUNK]
-  float *red = sc + G * CHUNK;                       // [KS][G][DL]
-  float *mls = red + KS * G * DL;                    // [G][2]
+  TL *Kb = reinterpret_cast<TL *>(smraw);            // [2][SUB][DL], swizzled pieces
+  TL *Vb = Kb + 2 * SUB * DL;                        // [2][SUB][DL]
+  float *qs = reinterpret_cast<float *>(Vb + 2 * SUB * DL);   // [G][DL], pre-scaled
+  float *sc = qs + G * DL;                           // [G][SUB]
+  float *red = sc + G * SUB;                         // [KS][G][DL]
+  float *mls = red + KS * G * DL;                    // [G][2] running (m, l)
+  float *scl = mls + 2 * G;                          // [G] rescale of this sub-chunk
   const int ch = blockIdx.x, g = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   const int L = lengths[b];
@@ -290,74 +296,105 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(
     return;
   }
   const size_t row0 = (static_cast<size_t>(b) * Hkv + g) * max_seq + s0;
-  for (int i = tid; i < n * CPR; i += blockDim.x) {
-    const int r = i / CPR, j = i % CPR;
-    cp_async16_zfill(Ks + r * DL + (j ^ kv_swz<CPR>(r)) * EPC, k_cache + (row0 + r) * DL + j * EPC, true);
-    cp_async16_zfill(Vs + r * DL + j * EPC, v_cache + (row0 + r) * DL + j * EPC, true);
-  }
+  const int nsub = (n + SUB - 1) / SUB;
+  auto issue = [&](int sbi) {                        // copies of sub-chunk sbi into slot sbi&1
+    const int base = sbi * SUB, cnt = min(SUB, n - base);
+    TL *kd = Kb + (sbi & 1) * SUB * DL, *vd = Vb + (sbi & 1) * SUB * DL;
+    for (int i = tid; i < cnt * CPR; i += blockDim.x) {
+      const int r = i / CPR, j = i % CPR;
+      const size_t src = (row0 + base + r) * DL + j * EPC;
+      cp_async16_zfill(kd + r * DL + (j ^ kv_swz<CPR>(r)) * EPC, k_cache + src, true);
+      cp_async16_zfill(vd + r * DL + j * EPC, v_cache + src, true);
+    }
+    cp_async_commit();
+  };
+  issue(0);
   for (int i = tid; i < G * DL; i += blockDim.x)
     qs[i] = q_new[(static_cast<size_t>(b) * H + g * G) * DL + i] * scale_log2;
-  cp_async_wait_all();
-  __syncthreads();
-
-  // scores
-  for (int r = tid; r < n; r += blockDim.x) {
-    float kf[DL];
-#pragma unroll
-    for (int j = 0; j < CPR; ++j) {
-      float e8[EPC];
-      const TL *src = Ks + r * DL + (j ^ kv_swz<CPR>(r)) * EPC;
-      if constexpr (EPC == 8) {
-        load8(src, *reinterpret_cast<float(*)[8]>(e8));
-      } else {
-        const float4 f = *reinterpret_cast<const float4 *>(src);
-        e8[0] = f.x; e8[1] = f.y; e8[2] = f.z; e8[3] = f.w;
-      }
-#pragma unroll
-      for (int e = 0; e < EPC; ++e) kf[j * EPC + e] = e8[e];
-    }
-    for (int h = 0; h < G; ++h) {
-      const float4 *qh = reinterpret_cast<const float4 *>(qs + h * DL);
-      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll
-      for (int d4 = 0; d4 < DL / 4; ++d4) {
-        const float4 qv = qh[d4];
-        a0 = fmaf(qv.x, kf[4 * d4 + 0], a0);
-        a1 = fmaf(qv.y, kf[4 * d4 + 1], a1);
-        a2 = fmaf(qv.z, kf[4 * d4 + 2], a2);
-        a3 = fmaf(qv.w, kf[4 * d4 + 3], a3);
-      }
-      sc[h * CHUNK + r] = (a0 + a1) + (a2 + a3);
-    }
+  for (int h = tid; h < G; h += blockDim.x) {
+    mls[2 * h] = -INFINITY;
+    mls[2 * h + 1] = 0.f;
   }
-  __syncthreads();
-  // per-head chunk max and sum
-  for (int h = warp; h < G; h += blockDim.x / 32) {
-    float mx = -INFINITY;
-    for (int r = lane; r < n; r += 32) mx = fmaxf(mx, sc[h * CHUNK + r]);
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-    float sum = 0.f;
-    for (int r = lane; r < n; r += 32) {
-      const float e = exp2f(sc[h * CHUNK + r] - mx);
-      sc[h * CHUNK + r] = e;
-      sum += e;
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-    if (lane == 0) {
-      mls[2 * h] = mx;
-      mls[2 * h + 1] = sum;
-    }
-  }
-  __syncthreads();
-  // P V: thread (key slice ks, dim pair dp), 8 heads at a time
   const int dp = tid % PAIRS, ks = tid / PAIRS;
-  for (int hb = 0; hb < G; hb += 8) {
-    float acc[8][2];
+  float acc[GMAX][2];                                // P V accumulators (G <= 8 here)
 #pragma unroll
-    for (int h = 0; h < 8; ++h) acc[h][0] = acc[h][1] = 0.f;
-    for (int r = ks; r < n; r += KS) {
+  for (int h = 0; h < GMAX; ++h) acc[h][0] = acc[h][1] = 0.f;
+
+  for (int sbi = 0; sbi < nsub; ++sbi) {
+    if (sbi + 1 < nsub) {
+      issue(sbi + 1);
+      cp_async_wait_one();                           // sub-chunk sbi has landed
+    } else {
+      cp_async_wait_none();
+    }
+    __syncthreads();
+    const TL *Ks = Kb + (sbi & 1) * SUB * DL, *Vs = Vb + (sbi & 1) * SUB * DL;
+    const int cnt = min(SUB, n - sbi * SUB);
+    // scores
+    for (int r = tid; r < cnt; r += blockDim.x) {
+      float kf[DL];
+#pragma unroll
+      for (int j = 0; j < CPR; ++j) {
+        float e8[EPC];
+        const TL *src = Ks + r * DL + (j ^ kv_swz<CPR>(r)) * EPC;
+        if constexpr (EPC == 8) {
+          load8(src, *reinterpret_cast<float(*)[8]>(e8));
+        } else {
+          const float4 f = *reinterpret_cast<const float4 *>(src);
+          e8[0] = f.x; e8[1] = f.y; e8[2] = f.z; e8[3] = f.w;
+        }
+#pragma unroll
+        for (int e = 0; e < EPC; ++e) kf[j * EPC + e] = e8[e];
+      }
+      for (int h = 0; h < G; ++h) {
+        const float4 *qh = reinterpret_cast<const float4 *>(qs + h * DL);
+        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+        for (int d4 = 0; d4 < DL / 4; ++d4) {
+          const float4 qv = qh[d4];
+          a0 = fmaf(qv.x, kf[4 * d4 + 0], a0);
+          a1 = fmaf(qv.y, kf[4 * d4 + 1], a1);
+          a2 = fmaf(qv.z, kf[4 * d4 + 2], a2);
+          a3 = fmaf(qv.w, kf[4 * d4 + 3], a3);
+        }
+        sc[h * SUB + r] = (a0 + a1) + (a2 + a3);
+      }
+    }
+    __syncthreads();
+    // running max and sum per head
+    for (int h = warp; h < G; h += blockDim.x / 32) {
+      float mx = -INFINITY;
+      for (int r = lane; r < cnt; r += 32) mx = fmaxf(mx, sc[h * SUB + r]);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+      const float m_old = mls[2 * h];
+      const float m_new = fmaxf(m_old, mx);
+      float sum = 0.f;
+      for (int r = lane; r < cnt; r += 32) {
+        const float e = exp2f(sc[h * SUB + r] - m_new);
+        sc[h * SUB + r] = e;
+        sum += e;
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+      if (lane == 0) {
+        const float f = exp2f(m_old - m_new);        // 0 on the first sub-chunk
+        scl[h] = f;
+        mls[2 * h] = m_new;
+        mls[2 * h + 1] = mls[2 * h + 1] * f + sum;
+      }
+    }
+    __syncthreads();
+    // P V
+#pragma unroll
+    for (int h = 0; h < GMAX; ++h) {
+      if (h < G) {
+        const float f = scl[h];
+        acc[h][0] *= f;
+        acc[h][1] *= f;
+      }
+    }
+    for (int r = ks; r < cnt; r += KS) {
       float2 v;
       if constexpr (sizeof(TL) == 2) {
         v = __half22float2(*reinterpret_cast<const __half2 *>(Vs + r * DL + 2 * dp));
@@ -365,20 +402,21 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(
         v = *reinterpret_cast<const float2 *>(Vs + r * DL + 2 * dp);
       }
 #pragma unroll
-      for (int h = 0; h < 8; ++h) {
-        if (hb + h < G) {
-          const float pr = sc[(hb + h) * CHUNK + r];
+      for (int h = 0; h < GMAX; ++h) {
+        if (h < G) {
+          const float pr = sc[h * SUB + r];
           acc[h][0] = fmaf(pr, v.x, acc[h][0]);
           acc[h][1] = fmaf(pr, v.y, acc[h][1]);
         }
       }
     }
+    __syncthreads();                                 // slot sbi&1 and sc are reused next
+  }
 #pragma unroll
-    for (int h = 0; h < 8; ++h) {
-      if (hb + h < G) {
-        red[(ks * G + hb + h) * DL + 2 * dp] = acc[h][0];
-        red[(ks * G + hb + h) * DL + 2 * dp + 1] = acc[h][1];
-      }
+  for (int h = 0; h < GMAX; ++h) {
+    if (h < G) {
+      red[(ks * G + h) * DL + 2 * dp] = acc[h][0];
+      red[(ks * G + h) * DL + 2 * dp + 1] = acc[h][1];
     }
   }
   __syncthreads();
@@ -477,9 +515,9 @@ template <int DL, typename TL>
 static cudaError_t launch_decode_attn(const Dims &d, const DecodeArgs &a, float scale_log2,
                                       cudaStream_t st) {
   const int KS = 128 / (DL / 2);
-  const size_t smem = 2 * static_cast<size_t>(CHUNK) * DL * sizeof(TL) +
-                      (static_cast<size_t>(d.G) * DL + static_cast<size_t>(d.G) * CHUNK +
-                       static_cast<size_t>(KS) * d.G * DL + 2 * d.G) * 4;
+  const size_t smem = 4 * static_cast<size_t>(SUB) * DL * sizeof(TL) +
+                      (static_cast<size_t>(d.G) * DL + static_cast<size_t>(d.G) * SUB +
+                       static_cast<size_t>(KS) * d.G * DL + 3 * d.G) * 4;
   cudaError_t e = cudaFuncSetAttribute(decode_attn_kernel<DL, TL>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));

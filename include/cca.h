@@ -148,7 +148,8 @@ CCA_API int cca_prefill_forward(const cca_config_t *cfg, const cca_weights_t *w,
  * The token's key/value are appended at position lengths[b], its query attends to
  * positions 0..lengths[b], the conv / value-shift state advance and lengths[b] += 1.
  * A sequence already holding max_seq tokens is left untouched, its y row is zero and the
- * cache status word is set to CCA_ERR_CACHE_FULL (read it with cca_cache_check).  A new
+ * cache status word is set to CCA_ERR_CACHE_FULL (read it with cca_cache_check).  The decode
+ * kernels take at most 8 query heads per kv head (CCA_ERR_UNSUPPORTED otherwise).  A new
  * latent key or value beyond the float16 range sets it to CCA_ERR_RANGE.
  * Errors (host): INVALID_ARG, UNSUPPORTED, WORKSPACE, ALIGNMENT, CUDA. */
 CCA_API int cca_decode_step(const cca_config_t *cfg, const cca_weights_t *w, const void *x,
@@ -162,7 +163,7 @@ CCA_API int cca_decode_step(const cca_config_t *cfg, const cca_weights_t *w, con
  * outputs, weights and the cache are the caller's as in cca_decode_step; the step's scratch
  * lives in an 8 MiB array built into the library, held by every GPU that loads the library
  * until the process exits.  A step that needs more scratch (cca_decode_workspace_size above
- * 8 MiB, e.g. 64 sequences of 16 heads with d~ = 32 beyond ~12k cached tokens) is rejected
+ * 8 MiB, e.g. 64 sequences of 16 heads with d~ = 32 beyond ~48k cached tokens) is rejected
  * with CCA_ERR_WORKSPACE before anything is launched.  The first call on each device looks
  * up the array's device address (cudaGetSymbolAddress) with that device current; make that
  * first call before any stream capture.  Every call uses the same array and leaves its

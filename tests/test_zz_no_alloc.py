@@ -54,13 +54,14 @@ def test_static_scratch_decode_matches_workspace_decode(cuda_lib):
 def test_static_scratch_rejects_oversized_steps(cuda_lib):
     cls = cuda_lib
     w = W.WORKLOADS["ccgqa_decode_8k"]
-    inp = W.make_inputs(w.with_(batch=2, seq=16), seed=0)
-    layer = cls.CCALayer.from_workload(w.with_(batch=2, seq=16), inp)
-    max_seq = 1 << 20                                # needs far more than the 8 MiB array
-    need = cls.cca_decode_workspace_size(layer.cfg, 2, max_seq)
-    assert need > 8 << 20
-    fake = cls.cca_cache_t(16, 32, 48, 64, 80, 96, 2, max_seq)     # rejected before any use
-    x = torch.zeros(2, w.d_model, dtype=torch.bfloat16, device="cuda")
+    B = w.batch
+    inp = W.make_inputs(w.with_(seq=16), seed=0)
+    layer = cls.CCALayer.from_workload(w.with_(seq=16), inp)
+    max_seq = 1 << 16
+    while cls.cca_decode_workspace_size(layer.cfg, B, max_seq) <= 8 << 20:
+        max_seq *= 2                                 # a step that needs more than 8 MiB
+    fake = cls.cca_cache_t(16, 32, 48, 64, 80, 96, B, max_seq)     # rejected before any use
+    x = torch.zeros(B, w.d_model, dtype=torch.bfloat16, device="cuda")
     y = torch.empty_like(x)
     rc = cls.load().cca_decode_step_static(ctypes.byref(layer.cfg), ctypes.byref(layer.weights),
                                            ctypes.c_void_p(x.data_ptr()),
