@@ -432,6 +432,223 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(
   }
 }
 
+// ------------------------------------------------------------------ D3 on tensor cores
+// The float16-cache variant of D3.  Same blocking (CTA = sequence x kv group x CHUNK-key
+// split, SUB-key sub-chunks through the two-deep copy ring), but each warp owns a 64-key
+// quarter of every sub-chunk and runs its own online softmax on mma.sync tiles:
+//   S = Q K^T   m16n8k16, rows = the G query heads (rows G..15 zero), 8 keys per n-tile,
+//               Q rounded to float16 like the prefill's latent q, in registers; K through
+//               ldmatrix; the scores are scaled by log2(e)/sqrt(d~) in fp32
+//   P V         the S accumulators of two n-tiles are, after exp2 and rounding to float16,
+//               exactly the A fragment of the next m16n8k16 (keys as K); V enters through
+//               ldmatrix.trans
+// Row max and sum are per head row, reduced over the four lanes that hold a row.  The four
+// warps' (m, l, o) are combined in shared memory before the split's partials are written.
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2,
+                                        uint32_t &r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t &r0, uint32_t &r1,
+                                          uint32_t &r2, uint32_t &r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+template <int DL>
+__global__ void __launch_bounds__(128, 1) decode_attn_tc_kernel(
+    const float *__restrict__ q_new, const __half *__restrict__ k_cache,
+    const __half *__restrict__ v_cache, const int *__restrict__ lengths,
+    float *__restrict__ part_o, float *__restrict__ part_ml, int H, int Hkv, int G, int max_seq,
+    int nchunk, float scale_log2) {
+  constexpr int CPR = DL / 8;                        // 16-byte pieces (8 dims) per row
+  constexpr int NT = 8;                              // 8-key n-tiles per warp step (64 keys)
+  constexpr int WK = NT * 8;                         // keys per warp per sub-chunk
+  static_assert(4 * WK == SUB, "four warps cover a sub-chunk");
+  extern __shared__ __align__(16) uint8_t smraw[];
+  __half *Kb = reinterpret_cast<__half *>(smraw);    // [2][SUB][DL], swizzled pieces
+  __half *Vb = Kb + 2 * SUB * DL;                    // [2][SUB][DL], swizzled pieces
+  float *wst = reinterpret_cast<float *>(Vb + 2 * SUB * DL);  // [4 warps][8 heads][DL + 2]
+  const int ch = blockIdx.x, g = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31, gr = lane >> 2, qd = lane & 3;
+  const int L = lengths[b];
+  const int s0 = ch * CHUNK;
+  const int n = L < max_seq ? min(CHUNK, L + 1 - s0) : 0;
+  float *po = part_o + ((static_cast<size_t>(b) * H + g * G) * nchunk + ch) * DL;
+  float *pml = part_ml + ((static_cast<size_t>(b) * H + g * G) * nchunk + ch) * 2;
+  if (n <= 0) {
+    for (int i = tid; i < G * DL; i += blockDim.x)
+      po[static_cast<size_t>(i / DL) * nchunk * DL + (i % DL)] = 0.f;
+    for (int h = tid; h < G; h += blockDim.x) {
+      pml[static_cast<size_t>(h) * nchunk * 2] = -INFINITY;
+      pml[static_cast<size_t>(h) * nchunk * 2 + 1] = 0.f;
+    }
+    return;
+  }
+  const size_t row0 = (static_cast<size_t>(b) * Hkv + g) * max_seq + s0;
+  const int nsub = (n + SUB - 1) / SUB;
+  auto issue = [&](int sbi) {                        // sub-chunk sbi into slot sbi & 1;
+    const int base = sbi * SUB, cnt = min(SUB, n - base);   // rows past cnt are zero-filled
+    __half *kd = Kb + (sbi & 1) * SUB * DL, *vd = Vb + (sbi & 1) * SUB * DL;
+    for (int i = tid; i < SUB * CPR; i += blockDim.x) {
+      const int r = i / CPR, j = i % CPR;
+      const bool ok = r < cnt;
+      const size_t src = (row0 + base + (ok ? r : 0)) * DL + j * 8;
+      const int dst = r * DL + (j ^ kv_swz<CPR>(r)) * 8;
+      cp_async16_zfill(kd + dst, k_cache + src, ok);
+      cp_async16_zfill(vd + dst, v_cache + src, ok);
+    }
+    cp_async_commit();
+  };
+  issue(0);
+
+  // Q fragments (rows = heads; a1, a3 are rows 8..15 and stay zero)
+  uint32_t qa[DL / 16][2];
+  {
+    const float *qh = q_new + (static_cast<size_t>(b) * H + g * G + gr) * DL;
+#pragma unroll
+    for (int kk = 0; kk < DL / 16; ++kk) {
+      float v0 = 0.f, v1 = 0.f, v2 = 0.f, v3 = 0.f;
+      if (gr < G) {
+        v0 = qh[16 * kk + 2 * qd];
+        v1 = qh[16 * kk + 2 * qd + 1];
+        v2 = qh[16 * kk + 2 * qd + 8];
+        v3 = qh[16 * kk + 2 * qd + 9];
+      }
+      qa[kk][0] = pack_f16x2(v0, v1);
+      qa[kk][1] = pack_f16x2(v2, v3);
+    }
+  }
+  float o[DL / 8][4];
+#pragma unroll
+  for (int t = 0; t < DL / 8; ++t) o[t][0] = o[t][1] = o[t][2] = o[t][3] = 0.f;
+  float m_run = -INFINITY, l_run = 0.f;              // of head row gr (lanes of one quad agree)
+
+  for (int sbi = 0; sbi < nsub; ++sbi) {
+    if (sbi + 1 < nsub) {
+      issue(sbi + 1);
+      cp_async_wait_one();                           // sub-chunk sbi has landed
+    } else {
+      cp_async_wait_none();
+    }
+    __syncthreads();
+    const uint32_t ks_base = smem_u32(Kb + (sbi & 1) * SUB * DL);
+    const uint32_t vs_base = smem_u32(Vb + (sbi & 1) * SUB * DL);
+    const int kb = warp * WK;                        // this warp's first key in the sub-chunk
+    const int valid = n - sbi * SUB - kb;            // keys of this warp's slice that exist
+    if (valid > 0) {
+      // ---- S = Q K^T over 8 n-tiles
+      float sc[NT][4];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+#pragma unroll
+      for (int m0 = 0; m0 < NT * CPR; m0 += 4) {      // four (n-tile, piece) matrices per load
+        const int id = m0 + (lane >> 3);
+        const int nt = id / CPR, j = id % CPR;
+        const int r = kb + nt * 8 + (lane & 7);
+        uint32_t f[4];
+        ldsm_x4(ks_base + (r * DL + (j ^ kv_swz<CPR>(r)) * 8) * 2, f[0], f[1], f[2], f[3]);
+#pragma unroll
+        for (int e = 0; e < 4; e += 2) {
+          // matrices m0+e, m0+e+1 = pieces (2c, 2c+1) of one n-tile = one 16-dim k step
+          const int idm = m0 + e, ntm = idm / CPR, kk = (idm % CPR) / 2;
+          const uint32_t a[4] = {qa[kk][0], 0u, qa[kk][1], 0u};
+          const uint32_t bb[2] = {f[e], f[e + 1]};
+          mma_f16_16816(sc[ntm], a, bb);
+        }
+      }
+      // ---- online softmax of row gr over this warp's 64 keys (scores to log2 units here,
+      // after the product, as in the prefill attention)
+      float mx = -INFINITY;
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          sc[nt][e] = nt * 8 + 2 * qd + e < valid ? sc[nt][e] * scale_log2 : -INFINITY;
+          mx = fmaxf(mx, sc[nt][e]);
+        }
+      }
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+      const float m_new = fmaxf(m_run, mx);          // finite: key kb of this slice is valid
+      const float f = exp2f(m_run - m_new);          // 0 while m_run = -inf
+      m_run = m_new;
+      float ls = 0.f;
+      uint32_t pa[NT / 2][2];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const float p0 = exp2f(sc[nt][0] - m_new), p1 = exp2f(sc[nt][1] - m_new);
+        ls += p0 + p1;
+        pa[nt / 2][nt & 1] = pack_f16x2(p0, p1);
+      }
+      l_run = l_run * f + ls;
+#pragma unroll
+      for (int t = 0; t < DL / 8; ++t) {
+        o[t][0] *= f;
+        o[t][1] *= f;
+      }
+      // ---- O += P V: 4 k-steps of 16 keys x DL/8 n-tiles of dims
+#pragma unroll
+      for (int kk = 0; kk < NT / 2; ++kk) {
+        const uint32_t a[4] = {pa[kk][0], 0u, pa[kk][1], 0u};
+#pragma unroll
+        for (int t0 = 0; t0 < DL / 8; t0 += 2) {      // two dim n-tiles (4 matrices) per load
+          const int id = lane >> 3;                  // (dim tile t0 + id/2, key half id&1)
+          const int r = kb + kk * 16 + (id & 1) * 8 + (lane & 7);
+          const int j = t0 + (id >> 1);
+          uint32_t f4[4];
+          ldsm_x4_t(vs_base + (r * DL + (j ^ kv_swz<CPR>(r)) * 8) * 2, f4[0], f4[1], f4[2], f4[3]);
+          const uint32_t b0[2] = {f4[0], f4[1]}, b1[2] = {f4[2], f4[3]};
+          mma_f16_16816(o[t0], a, b0);
+          mma_f16_16816(o[t0 + 1], a, b1);
+        }
+      }
+    }
+    __syncthreads();                                 // slot sbi & 1 is refilled next
+  }
+
+  // ---- combine the four warps: each posts (m, l, o) of its head rows
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
+  constexpr int WS = DL + 2;
+  if (gr < G) {
+    float *w = wst + (warp * 8 + gr) * WS;
+#pragma unroll
+    for (int t = 0; t < DL / 8; ++t) {
+      w[t * 8 + 2 * qd] = o[t][0];
+      w[t * 8 + 2 * qd + 1] = o[t][1];
+    }
+    if (qd == 0) {
+      w[DL] = m_run;
+      w[DL + 1] = l_run;
+    }
+  }
+  __syncthreads();
+  for (int i = tid; i < G * DL; i += blockDim.x) {
+    const int h = i / DL, d = i % DL;
+    float mw[4], M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      mw[w] = wst[(w * 8 + h) * WS + DL];
+      M = fmaxf(M, mw[w]);
+    }
+    float acc = 0.f, lsum = 0.f;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const float c = mw[w] == -INFINITY ? 0.f : exp2f(mw[w] - M);
+      acc = fmaf(c, wst[(w * 8 + h) * WS + d], acc);
+      lsum = fmaf(c, wst[(w * 8 + h) * WS + DL + 1], lsum);
+    }
+    po[static_cast<size_t>(h) * nchunk * DL + d] = acc;
+    if (d == 0) {
+      pml[static_cast<size_t>(h) * nchunk * 2] = M;
+      pml[static_cast<size_t>(h) * nchunk * 2 + 1] = lsum;
+    }
+  }
+}
+
 // ------------------------------------------------------------------ D3b merge (+ advance)
 // One CTA per sequence: all (m, l) of its heads and chunks are staged in shared memory with
 // one parallel load, then each thread (head, dim) combines its chunks' partial outputs.  The
@@ -514,6 +731,18 @@ void decode_workspace_carve(const Dims &d, int max_seq, void *ws, DecodeArgs &a)
 template <int DL, typename TL>
 static cudaError_t launch_decode_attn(const Dims &d, const DecodeArgs &a, float scale_log2,
                                       cudaStream_t st) {
+  if constexpr (sizeof(TL) == 2) {
+    const size_t smem = 4 * static_cast<size_t>(SUB) * DL * sizeof(TL) +
+                        static_cast<size_t>(4 * 8 * (DL + 2)) * 4;
+    cudaError_t e = cudaFuncSetAttribute(decode_attn_tc_kernel<DL>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    decode_attn_tc_kernel<DL><<<dim3(a.nchunk, d.Hkv, d.B), 128, smem, st>>>(
+        a.q_new, static_cast<const __half *>(a.k_cache), static_cast<const __half *>(a.v_cache),
+        a.lengths, a.part_o, a.part_ml, d.H, d.Hkv, d.G, a.max_seq, a.nchunk, scale_log2);
+    return cudaGetLastError();
+  }
   const int KS = 128 / (DL / 2);
   const size_t smem = 4 * static_cast<size_t>(SUB) * DL * sizeof(TL) +
                       (static_cast<size_t>(d.G) * DL + static_cast<size_t>(d.G) * SUB +
