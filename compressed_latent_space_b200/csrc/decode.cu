@@ -22,92 +22,147 @@ namespace {
 
 constexpr int CHUNK = 1024;       // keys per split-KV block
 
-// ------------------------------------------------------------------ D1 / D4 skinny GEMM
-// C[M, N] = A[M, K] * B[N, K]^T for small M (the batch), bf16 operands on mma.sync.
-// Grid (N / NB, ksplit, ceil(M/64)); 4 warps share the K slice of the block and reduce
-// through shared memory.  OUT_F32: write fp32 partial sums to C + ks*M*N; else write bf16.
-// TA = float: A is float32 and enters the tensor cores as two bf16 terms, hi = bf16(a) and
-// lo = bf16(a - hi), so the product keeps ~16 significand bits of A at no extra traffic.
-template <int NB, bool OUT_F32, typename TA = __nv_bfloat16>
-__global__ void __launch_bounds__(128) skinny_gemm_kernel(const TA *__restrict__ A,
-                                                          const __nv_bfloat16 *__restrict__ B,
-                                                          void *__restrict__ C, int M, int N,
-                                                          int K, int k_per_split) {
-  constexpr int NT = NB / 8;
-  __shared__ float red[4][64][NB + 1];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int gr = lane >> 2, qc = lane & 3;
-  const int n0 = blockIdx.x * NB;
-  const int ks = blockIdx.y;
-  const int mbase = blockIdx.z * 64;
-  const int kbeg = ks * k_per_split;
-  const int kend = min(K, kbeg + k_per_split);
-  float acc[4][NT][4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < NT; ++j) acc[i][j][0] = acc[i][j][1] = acc[i][j][2] = acc[i][j][3] = 0.f;
-  for (int k0 = kbeg + warp * 16; k0 < kend; k0 += 64) {
-    uint32_t bf[NT][2];
-#pragma unroll
-    for (int j = 0; j < NT; ++j) {
-      const int n = n0 + j * 8 + gr;
-      const __nv_bfloat16 *bp = B + static_cast<size_t>(n) * K + k0 + 2 * qc;
-      bf[j][0] = n < N ? *reinterpret_cast<const uint32_t *>(bp) : 0u;
-      bf[j][1] = n < N ? *reinterpret_cast<const uint32_t *>(bp + 8) : 0u;
+// ------------------------------------------------------------------ D1 / D4 on staged tiles
+// C[M, N] = A[M, K] B[N, K]^T (+ A2[M, K] B^T) for M <= 64 per CTA row block, bfloat16
+// operands, fp32 accumulation.  Grid (ceil(N / 16), ksplit, ceil(M / 64)): a CTA owns 16
+// columns and one K slice, which it walks in 64-wide chunks staged in shared memory by 16-byte
+// cp.async through an S-deep ring (S - 1 chunks in flight while one is computed; rows padded
+// by 16 bytes so the ldmatrix reads are conflict-free).  Warp w computes rows 16w..16w+15 x
+// the 16 columns with mma.sync.  TWO_A adds a second A operand (the low bf16 halves of an fp32
+// A split hi + lo).  OUT_F32: fp32 partial sums to C + ks*M*N; else bf16.  `lengths`
+// (optional): block (0, 0, 0) advances lengths[m] for m < M where it is below max_seq (the
+// last kernel of a decode step).
+constexpr int SK_KC = 64;           // K chunk
+constexpr int SK_LD = SK_KC + 8;    // padded row, in elements
+
+template <bool TWO_A>
+__host__ __device__ constexpr int skinny_stage_elems() {
+  return ((TWO_A ? 2 : 1) * 64 + 16) * SK_LD;
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2,
+                                        uint32_t &r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t &r0, uint32_t &r1,
+                                          uint32_t &r2, uint32_t &r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+template <bool OUT_F32, bool TWO_A, int S>
+__global__ void __launch_bounds__(128) skinny_mma_kernel(
+    const __nv_bfloat16 *__restrict__ A, const __nv_bfloat16 *__restrict__ A2,
+    const __nv_bfloat16 *__restrict__ B, void *__restrict__ C, int M, int N, int K,
+    int k_per_split, int *lengths, int max_seq) {
+  constexpr int STAGE = skinny_stage_elems<TWO_A>();
+  extern __shared__ __align__(16) __nv_bfloat16 sk_smem[];     // [S][A (A2) B]
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n0 = blockIdx.x * 16, ks = blockIdx.y, m0 = blockIdx.z * 64;
+  if (lengths && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0)
+    for (int m = tid; m < M; m += 128)
+      if (lengths[m] < max_seq) lengths[m] += 1;
+  const int kbeg = ks * k_per_split, kend = min(K, kbeg + k_per_split);
+  const int nchunks = kend > kbeg ? (kend - kbeg + SK_KC - 1) / SK_KC : 0;
+  auto issue = [&](int c) {                           // an empty group past the last chunk
+    if (c < nchunks) {
+      const int k0 = kbeg + c * SK_KC;
+      __nv_bfloat16 *st = sk_smem + (c % S) * STAGE;
+      for (int i = tid; i < 64 * (SK_KC / 8); i += 128) {     // A (and A2): 64 x SK_KC
+        const int r = i / (SK_KC / 8), j = i % (SK_KC / 8);
+        const int k = k0 + j * 8;
+        const bool ok = m0 + r < M && k < kend;
+        const size_t off = ok ? static_cast<size_t>(m0 + r) * K + k : 0;
+        cp_async16_zfill(st + r * SK_LD + j * 8, A + off, ok);
+        if constexpr (TWO_A) cp_async16_zfill(st + (64 + r) * SK_LD + j * 8, A2 + off, ok);
+      }
+      __nv_bfloat16 *bs = st + (TWO_A ? 128 : 64) * SK_LD;
+      for (int i = tid; i < 16 * (SK_KC / 8); i += 128) {     // B: 16 x SK_KC
+        const int r = i / (SK_KC / 8), j = i % (SK_KC / 8);
+        const int k = k0 + j * 8;
+        const bool ok = n0 + r < N && k < kend;
+        cp_async16_zfill(bs + r * SK_LD + j * 8,
+                         B + (ok ? static_cast<size_t>(n0 + r) * K + k : 0), ok);
+      }
     }
+    cp_async_commit();
+  };
+  float acc[2][4];
 #pragma unroll
-    for (int mt = 0; mt < 4; ++mt) {
-      const int ma = mbase + mt * 16 + gr, mb = ma + 8;
-      const TA *pa = A + static_cast<size_t>(ma) * K + k0 + 2 * qc;
-      const TA *pb = A + static_cast<size_t>(mb) * K + k0 + 2 * qc;
-      if constexpr (sizeof(TA) == 2) {
-        uint32_t af[4];
-        af[0] = ma < M ? *reinterpret_cast<const uint32_t *>(pa) : 0u;
-        af[1] = mb < M ? *reinterpret_cast<const uint32_t *>(pb) : 0u;
-        af[2] = ma < M ? *reinterpret_cast<const uint32_t *>(pa + 8) : 0u;
-        af[3] = mb < M ? *reinterpret_cast<const uint32_t *>(pb + 8) : 0u;
+  for (int t = 0; t < 2; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
 #pragma unroll
-        for (int j = 0; j < NT; ++j) mma_bf16_16816(acc[mt][j], af, bf[j]);
+  for (int c = 0; c < S - 1; ++c) issue(c);
+  for (int c = 0; c < nchunks; ++c) {
+    issue(c + S - 1);
+    cp_async_wait_group<S - 1>();                      // chunk c has landed
+    __syncthreads();
+    const __nv_bfloat16 *st = sk_smem + (c % S) * STAGE;
+    const uint32_t a_base = smem_u32(st + (warp * 16 + (lane & 15)) * SK_LD + (lane >> 4) * 8);
+    const uint32_t b_base = smem_u32(st + ((TWO_A ? 128 : 64) + (lane & 7) + (lane >> 4) * 8) * SK_LD +
+                                     ((lane >> 3) & 1) * 8);
+#pragma unroll
+    for (int kk = 0; kk < SK_KC / 16; ++kk) {
+      uint32_t a[4], bq[4];
+      ldsm_x4(a_base + kk * 32, a[0], a[1], a[2], a[3]);
+      ldsm_x4(b_base + kk * 32, bq[0], bq[1], bq[2], bq[3]);
+      const uint32_t b0[2] = {bq[0], bq[1]}, b1[2] = {bq[2], bq[3]};
+      mma_bf16_16816(acc[0], a, b0);
+      mma_bf16_16816(acc[1], a, b1);
+      if constexpr (TWO_A) {
+        uint32_t a2[4];
+        ldsm_x4(a_base + kk * 32 + 64 * SK_LD * 2, a2[0], a2[1], a2[2], a2[3]);
+        mma_bf16_16816(acc[0], a2, b0);
+        mma_bf16_16816(acc[1], a2, b1);
+      }
+    }
+    __syncthreads();                                  // stage c % S is refilled next
+  }
+  cp_async_wait_group<0>();
+  const int gr = lane >> 2, qc = lane & 3;
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    const int n = n0 + t * 8 + 2 * qc;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int m = m0 + warp * 16 + gr + h * 8;
+      if (m >= M) continue;
+      const float v0 = acc[t][2 * h], v1 = acc[t][2 * h + 1];
+      if constexpr (OUT_F32) {
+        float *cp = static_cast<float *>(C) + (static_cast<size_t>(ks) * M + m) * N + n;
+        if (n < N) cp[0] = v0;
+        if (n + 1 < N) cp[1] = v1;
       } else {
-        const float2 z = make_float2(0.f, 0.f);
-        const float2 v0 = ma < M ? *reinterpret_cast<const float2 *>(pa) : z;
-        const float2 v1 = mb < M ? *reinterpret_cast<const float2 *>(pb) : z;
-        const float2 v2 = ma < M ? *reinterpret_cast<const float2 *>(pa + 8) : z;
-        const float2 v3 = mb < M ? *reinterpret_cast<const float2 *>(pb + 8) : z;
-        uint32_t hi[4], lo[4];
-        split_bf16x2(v0, hi[0], lo[0]);
-        split_bf16x2(v1, hi[1], lo[1]);
-        split_bf16x2(v2, hi[2], lo[2]);
-        split_bf16x2(v3, hi[3], lo[3]);
-#pragma unroll
-        for (int j = 0; j < NT; ++j) {
-          mma_bf16_16816(acc[mt][j], hi, bf[j]);
-          mma_bf16_16816(acc[mt][j], lo, bf[j]);
+        __nv_bfloat16 *cp = static_cast<__nv_bfloat16 *>(C) + static_cast<size_t>(m) * N + n;
+        if (n + 1 < N) {
+          *reinterpret_cast<uint32_t *>(cp) = pack_bf16x2(v0, v1);
+        } else if (n < N) {
+          cp[0] = __float2bfloat16_rn(v0);
         }
       }
     }
   }
-#pragma unroll
-  for (int mt = 0; mt < 4; ++mt)
-#pragma unroll
-    for (int j = 0; j < NT; ++j) {
-      red[warp][mt * 16 + gr][j * 8 + 2 * qc] = acc[mt][j][0];
-      red[warp][mt * 16 + gr][j * 8 + 2 * qc + 1] = acc[mt][j][1];
-      red[warp][mt * 16 + gr + 8][j * 8 + 2 * qc] = acc[mt][j][2];
-      red[warp][mt * 16 + gr + 8][j * 8 + 2 * qc + 1] = acc[mt][j][3];
-    }
-  __syncthreads();
-  for (int i = threadIdx.x; i < 64 * NB; i += blockDim.x) {
-    const int r = i / NB, c = i % NB;
-    const int m = mbase + r, n = n0 + c;
-    if (m >= M || n >= N) continue;
-    const float v = red[0][r][c] + red[1][r][c] + red[2][r][c] + red[3][r][c];
-    if (OUT_F32)
-      static_cast<float *>(C)[(static_cast<size_t>(ks) * M + m) * N + n] = v;
-    else
-      static_cast<__nv_bfloat16 *>(C)[static_cast<size_t>(m) * N + n] = __float2bfloat16_rn(v);
-  }
+}
+
+template <bool OUT_F32, bool TWO_A, int S>
+static cudaError_t launch_skinny(dim3 grid, const __nv_bfloat16 *A, const __nv_bfloat16 *A2,
+                                 const __nv_bfloat16 *B, void *C, int M, int N, int K, int kps,
+                                 int *lengths, int max_seq, cudaStream_t st) {
+  const size_t smem = static_cast<size_t>(S) * skinny_stage_elems<TWO_A>() * 2;
+  cudaError_t e = cudaFuncSetAttribute(skinny_mma_kernel<OUT_F32, TWO_A, S>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  skinny_mma_kernel<OUT_F32, TWO_A, S><<<grid, 128, smem, st>>>(A, A2, B, C, M, N, K, kps,
+                                                                lengths, max_seq);
+  return cudaGetLastError();
 }
 
 // ------------------------------------------------------------------ D2 decode stencil
@@ -444,19 +499,6 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(
 //               ldmatrix.trans
 // Row max and sum are per head row, reduced over the four lanes that hold a row.  The four
 // warps' (m, l, o) are combined in shared memory before the split's partials are written.
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2,
-                                        uint32_t &r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
-}
-__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t &r0, uint32_t &r1,
-                                          uint32_t &r2, uint32_t &r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
-}
-
 template <int DL>
 __global__ void __launch_bounds__(128, 1) decode_attn_tc_kernel(
     const float *__restrict__ q_new, const __half *__restrict__ k_cache,
@@ -685,9 +727,38 @@ __global__ void __launch_bounds__(512) decode_merge_kernel(
   if (threadIdx.x == 0 && !full) lengths[b] = L + 1;
 }
 
+// D3b for 16-bit layers: one CTA per (head, sequence), one thread per latent dim; the merged
+// o is written as bfloat16 hi + lo terms (o = hi + lo to ~16 significand bits), the A operands
+// of the D4 projection.
+__global__ void __launch_bounds__(64) decode_merge16_kernel(
+    const float *__restrict__ part_o, const float *__restrict__ part_ml,
+    const int *__restrict__ lengths, __nv_bfloat16 *__restrict__ o_hi,
+    __nv_bfloat16 *__restrict__ o_lo, int H, int DL, int max_seq, int nchunk) {
+  const int h = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
+  if (d >= DL) return;
+  const int L = lengths[b];
+  const int nused = L >= max_seq ? 0 : min(nchunk, (L + 1 + CHUNK - 1) / CHUNK);
+  const float *ml = part_ml + (static_cast<size_t>(b) * H + h) * nchunk * 2;
+  const float *po = part_o + (static_cast<size_t>(b) * H + h) * nchunk * DL + d;
+  float mx = -INFINITY;
+  for (int c = 0; c < nused; ++c) mx = fmaxf(mx, ml[2 * c]);
+  float l = 0.f, acc = 0.f;
+#pragma unroll 4
+  for (int c = 0; c < nused; ++c) {
+    const float w = exp2f(ml[2 * c] - mx);
+    l = fmaf(w, ml[2 * c + 1], l);
+    acc = fmaf(w, po[static_cast<size_t>(c) * DL], acc);
+  }
+  const float v = nused > 0 ? acc / l : 0.f;
+  const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+  const size_t idx = (static_cast<size_t>(b) * H + h) * DL + d;
+  o_hi[idx] = hi;
+  o_lo[idx] = __float2bfloat16_rn(v - __bfloat162float(hi));
+}
+
 int decode_ksplit(const Dims &d) {
   // enough blocks to keep every SM streaming the weight matrix
-  const int nblk = (d.NQKV + 31) / 32;
+  const int nblk = (d.NQKV + 15) / 16;
   int ks = (num_sms() + nblk - 1) / nblk;
   if (ks < 1) ks = 1;
   while (ks > 1 && d.E / ks < 64) --ks;
@@ -763,11 +834,12 @@ static cudaError_t decode_typed(const Dims &d, const DecodeArgs &a, cudaStream_t
   cudaError_t e;
   // D1
   if constexpr (sizeof(T) == 2) {
-    const int kps = ((d.E + a.ksplit - 1) / a.ksplit + 63) / 64 * 64;
-    dim3 g1((d.NQKV + 31) / 32, a.ksplit, (d.B + 63) / 64);
-    skinny_gemm_kernel<32, true><<<g1, 128, 0, st>>>(
-        static_cast<const __nv_bfloat16 *>(a.x), static_cast<const __nv_bfloat16 *>(a.w_qkv),
-        a.p_part, d.B, d.NQKV, d.E, kps);
+    const int kps = ((d.E + a.ksplit - 1) / a.ksplit + SK_KC - 1) / SK_KC * SK_KC;
+    dim3 g1((d.NQKV + 15) / 16, a.ksplit, (d.B + 63) / 64);
+    e = launch_skinny<true, false, 8>(g1, static_cast<const __nv_bfloat16 *>(a.x), nullptr,
+                                      static_cast<const __nv_bfloat16 *>(a.w_qkv), a.p_part, d.B,
+                                      d.NQKV, d.E, kps, nullptr, 0, st);
+    if (e != cudaSuccess) return e;
   } else {
     e = gemm_simt(0, a.x, a.w_qkv, a.p_part, d.B, d.NQKV, d.E, st);
     if (e != cudaSuccess) return e;
@@ -805,8 +877,14 @@ static cudaError_t decode_typed(const Dims &d, const DecodeArgs &a, cudaStream_t
   else e = launch_decode_attn<64, TL>(d, a, scale_log2, st);
   if (e != cudaSuccess) return e;
   mark();
-  // D3b (+ lengths advance)
-  {
+  // D3b (+ lengths advance for float32 layers; the 16-bit D4 advances them)
+  if constexpr (sizeof(T) == 2) {
+    __nv_bfloat16 *o_hi = static_cast<__nv_bfloat16 *>(a.o);
+    decode_merge16_kernel<<<dim3(d.H, d.B), d.DL < 32 ? 32 : d.DL, 0, st>>>(
+        a.part_o, a.part_ml, a.lengths, o_hi, o_hi + static_cast<size_t>(d.B) * d.NQ, d.H, d.DL,
+        a.max_seq, a.nchunk);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  } else {
     const int nused_max = a.nchunk;
     const size_t smm = static_cast<size_t>(d.H) * nused_max * 2 * 4;
     if (smm > 48 * 1024) {
@@ -821,12 +899,14 @@ static cudaError_t decode_typed(const Dims &d, const DecodeArgs &a, cudaStream_t
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   mark();
-  // D4
+  // D4 (+ lengths advance for 16-bit layers)
   if constexpr (sizeof(T) == 2) {
+    const __nv_bfloat16 *o_hi = static_cast<const __nv_bfloat16 *>(a.o);
     dim3 g4((d.E + 15) / 16, 1, (d.B + 63) / 64);
-    skinny_gemm_kernel<16, false, float><<<g4, 128, 0, st>>>(
-        static_cast<const float *>(a.o), static_cast<const __nv_bfloat16 *>(a.w_o),
-        a.y, d.B, d.E, d.NQ, d.NQ);
+    e = launch_skinny<false, true, 8>(g4, o_hi, o_hi + static_cast<size_t>(d.B) * d.NQ,
+                                      static_cast<const __nv_bfloat16 *>(a.w_o), a.y, d.B, d.E,
+                                      d.NQ, d.NQ, a.lengths, a.max_seq, st);
+    if (e != cudaSuccess) return e;
   } else {
     e = gemm_simt(0, a.o, a.w_o, a.y, d.B, d.E, d.NQ, st);
     if (e != cudaSuccess) return e;
