@@ -67,10 +67,20 @@ __global__ void __launch_bounds__(128) skinny_mma_kernel(
   extern __shared__ __align__(16) __nv_bfloat16 sk_smem[];     // [S][A (A2) B]
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int n0 = blockIdx.x * 16, ks = blockIdx.y, m0 = blockIdx.z * 64;
+  const int kbeg = ks * k_per_split, kend = min(K, kbeg + k_per_split);
+  pdl_launch_dependents();
+  {
+    // the weight slab does not depend on the previous kernel: pull it towards L2 meanwhile
+    const int lines = kend > kbeg ? ((kend - kbeg) * 2 + 127) / 128 : 0;
+    for (int i = tid; i < 16 * lines; i += 128) {
+      const int r = i / lines, c = i % lines;
+      if (n0 + r < N) prefetch_l2(B + static_cast<size_t>(n0 + r) * K + kbeg + c * 64);
+    }
+  }
+  pdl_wait();
   if (lengths && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0)
     for (int m = tid; m < M; m += 128)
       if (lengths[m] < max_seq) lengths[m] += 1;
-  const int kbeg = ks * k_per_split, kend = min(K, kbeg + k_per_split);
   const int nchunks = kend > kbeg ? (kend - kbeg + SK_KC - 1) / SK_KC : 0;
   auto issue = [&](int c) {                           // an empty group past the last chunk
     if (c < nchunks) {
@@ -160,9 +170,8 @@ static cudaError_t launch_skinny(dim3 grid, const __nv_bfloat16 *A, const __nv_b
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  skinny_mma_kernel<OUT_F32, TWO_A, S><<<grid, 128, smem, st>>>(A, A2, B, C, M, N, K, kps,
-                                                                lengths, max_seq);
-  return cudaGetLastError();
+  return launch_pdl(skinny_mma_kernel<OUT_F32, TWO_A, S>, grid, dim3(128), smem, st, A, A2, B,
+                    C, M, N, K, kps, lengths, max_seq);
 }
 
 // ------------------------------------------------------------------ D2 decode stencil
@@ -182,16 +191,44 @@ struct D2Params {
   double theta[32];        // RoPE frequencies base^(-2i/d~), i < d~/2, computed on the host
 };
 
-template <typename T>
-__global__ void __launch_bounds__(128) decode_stencil_kernel(const D2Params<T> p) {
+// D2 keeps the group's channel filters transposed in shared memory, wt[j][o] = the weight of
+// input j for output channel o (o over the G q heads and the k head, d~ each), rows padded to
+// an odd length so both the transposing writes and the per-output reads are conflict-free.
+// The filters, which no earlier kernel writes, are staged before the grid-dependency wait.
+__host__ __device__ constexpr int d2_ld(int QKC) { return QKC | 1; }
+__host__ __device__ inline size_t d2_smem_floats(int G, int DL, int KC) {
+  const int QKC = (G + 1) * DL, CH = (G + 2) * DL;
+  return static_cast<size_t>(DL) * d2_ld(QKC)   // wt
+         + QKC * KC                             // sequence filters
+         + CH + 2 * QKC + 16;                   // pn, av, uv, inv
+}
+
+template <typename T, int DL>
+__global__ void __launch_bounds__(256) decode_stencil_kernel(const D2Params<T> p) {
   using TL = typename D2Params<T>::TL;
-  extern __shared__ float sm[];
-  const int g = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
-  const int G = p.G, DL = p.DL, CH = (G + 2) * DL, QKC = (G + 1) * DL;
-  float *pn = sm;               // [CH] new projections (rounded like the prefill's P)
-  float *a = pn + CH;           // [QKC] after the sequence conv
-  float *u = a + QKC;           // [QKC] after channel conv / q-k-mean
-  float *inv = u + QKC;         // [G+1]
+  extern __shared__ __align__(16) float sm[];
+  const int g = blockIdx.x, b = blockIdx.y, tid = threadIdx.x, nt = blockDim.x;
+  const int G = p.G, CH = (G + 2) * DL, QKC = (G + 1) * DL, KC = p.KC, KC1 = KC - 1;
+  const int LD = d2_ld(QKC);
+  float *wt = sm;
+  float *wseq = wt + DL * LD;
+  float *pn = wseq + QKC * KC;
+  float *a = pn + CH;
+  float *u = a + QKC;
+  float *inv = u + QKC;
+  pdl_launch_dependents();
+  // filters: q heads g*G.., then k head H+g; W_head[i][j] -> wt[j][head * DL + i]
+  for (int e = tid; e < (G + 1) * DL * DL; e += nt) {
+    const int hh = e / (DL * DL), r = e % (DL * DL), i = r / DL, j = r % DL;
+    const int head = hh < G ? g * G + hh : p.H + g;
+    wt[j * LD + hh * DL + i] = p.conv_chan[static_cast<size_t>(head) * DL * DL + r];
+  }
+  for (int e = tid; e < QKC * KC; e += nt) {
+    const int c = e / KC, t = e % KC;
+    const int gc = c < G * DL ? g * G * DL + c : p.NQ + g * DL + (c - G * DL);
+    wseq[e] = p.conv_seq[static_cast<size_t>(gc) * KC + t];
+  }
+  pdl_wait();
   const int L = p.lengths[b];
   if (L >= p.max_seq) {
     if (tid == 0) report(p.status, DEV_CACHE_FULL);
@@ -201,34 +238,33 @@ __global__ void __launch_bounds__(128) decode_stencil_kernel(const D2Params<T> p
   auto gch = [&](int c) {
     return c < G * DL ? qcol0 + c : (c < QKC ? kcol0 + (c - G * DL) : vcol0 + (c - QKC));
   };
-  for (int c = tid; c < CH; c += blockDim.x) {
-    const int gc = gch(c);
-    float s = 0.f;
-    for (int ks = 0; ks < p.ksplit; ++ks) s += p.p_part[(static_cast<size_t>(ks) * p.B + b) * p.NQKV + gc];
-    pn[c] = s;
-  }
-  __syncthreads();
-  const int KC1 = p.KC - 1, W = p.NQ + p.NKV;
+  const int W = p.NQ + p.NKV;
   float *cs = p.conv_state + static_cast<size_t>(b) * KC1 * W;
-  for (int c = tid; c < QKC; c += blockDim.x) {
+  // new projections (sum of the split-K partials) and the sequence conv of the q|k channels
+  for (int c = tid; c < CH; c += nt) {
     const int gc = gch(c);
-    const float *w = p.conv_seq + static_cast<size_t>(gc) * p.KC;
-    float acc = 0.f;
-    for (int j = 0; j < KC1; ++j) acc = fmaf(w[j], to_f32(cs[static_cast<size_t>(j) * W + gc]), acc);
-    a[c] = fmaf(w[KC1], pn[c], acc);
+    float v = 0.f;
+    for (int ks = 0; ks < p.ksplit; ++ks) v += p.p_part[(static_cast<size_t>(ks) * p.B + b) * p.NQKV + gc];
+    pn[c] = v;
+    if (c < QKC) {
+      const float *w = wseq + c * KC;
+      float acc = 0.f;
+      for (int j = 0; j < KC1; ++j) acc = fmaf(w[j], cs[static_cast<size_t>(j) * W + gc], acc);
+      a[c] = fmaf(w[KC1], v, acc);
+    }
   }
   __syncthreads();
-  for (int o = tid; o < QKC; o += blockDim.x) {
+  // channel conv (thread per output) and q-k-mean
+  for (int o = tid; o < QKC; o += nt) {
     const int hh = o / DL, i = o % DL;
-    const bool is_q = hh < G;
-    const int head_w = is_q ? g * G + hh : p.H + g;
-    const float *wr = p.conv_chan + (static_cast<size_t>(head_w) * DL + i) * DL;
+    const float *ah = a + hh * DL;
     float acc = 0.f;
-    for (int j = 0; j < DL; ++j) acc = fmaf(wr[j], a[hh * DL + j], acc);
+#pragma unroll 8
+    for (int j = 0; j < DL; ++j) acc = fmaf(wt[j * LD + o], ah[j], acc);
     if (p.flags & F_QK_MEAN) {
       const float pk = pn[G * DL + i];
-      if (is_q) {
-        acc += 0.5f * (pn[hh * DL + i] + pk);
+      if (hh < G) {
+        acc += 0.5f * (pn[o] + pk);
       } else {
         float mq = 0.f;
         for (int h2 = 0; h2 < G; ++h2) mq += pn[h2 * DL + i];
@@ -240,7 +276,7 @@ __global__ void __launch_bounds__(128) decode_stencil_kernel(const D2Params<T> p
   __syncthreads();
   // RMS norm per head: one warp per head
   const int warp = tid >> 5, lane = tid & 31;
-  for (int hh = warp; hh <= G; hh += blockDim.x / 32) {
+  for (int hh = warp; hh <= G; hh += nt / 32) {
     float ss = 0.f;
     for (int i = lane; i < DL; i += 32) ss += u[hh * DL + i] * u[hh * DL + i];
 #pragma unroll
@@ -250,14 +286,14 @@ __global__ void __launch_bounds__(128) decode_stencil_kernel(const D2Params<T> p
   }
   __syncthreads();
   // RoPE at position L on (i, i + DL/2) pairs, then store q (workspace) and k (cache)
-  const int HALF = DL / 2;
-  for (int o = tid; o < (G + 1) * HALF; o += blockDim.x) {
+  constexpr int HALF = DL / 2;
+  for (int o = tid; o < (G + 1) * HALF; o += nt) {
     const int hh = o / HALF, ip = o % HALF;
     float x1 = u[hh * DL + ip] * inv[hh], x2 = u[hh * DL + ip + HALF] * inv[hh];
     if (p.flags & F_ROPE) {
-      float c, s;
-      rope_cos_sin(static_cast<double>(L) * p.theta[ip], c, s);
-      const float y1 = x1 * c - x2 * s, y2 = x1 * s + x2 * c;
+      float c, sn;
+      rope_cos_sin(static_cast<double>(L) * p.theta[ip], c, sn);
+      const float y1 = x1 * c - x2 * sn, y2 = x1 * sn + x2 * c;
       x1 = y1;
       x2 = y2;
     }
@@ -276,20 +312,20 @@ __global__ void __launch_bounds__(128) decode_stencil_kernel(const D2Params<T> p
   // value with the value-shift, appended at position L
   const int vhalf = p.NKV / 2;
   float *vs = p.vshift_state + static_cast<size_t>(b) * (p.NKV - vhalf);
-  for (int c = tid; c < DL; c += blockDim.x) {
+  for (int c = tid; c < DL; c += nt) {
     const int vc = g * DL + c;
     const bool shifted = vc >= vhalf;
-    const float val = ((p.flags & F_VALUE_SHIFT) && shifted) ? to_f32(vs[vc - vhalf]) : pn[QKC + c];
+    const float val = ((p.flags & F_VALUE_SHIFT) && shifted) ? vs[vc - vhalf] : pn[QKC + c];
     check_latent<TL>(val, p.status);
     p.v_cache[((static_cast<size_t>(b) * p.Hkv + g) * p.max_seq + L) * DL + c] = from_f32<TL>(val);
   }
   __syncthreads();   // every read of the old state is done
-  for (int c = tid; c < QKC; c += blockDim.x) {
+  for (int c = tid; c < QKC; c += nt) {
     const int gc = gch(c);
     for (int j = 0; j + 1 < KC1; ++j) cs[static_cast<size_t>(j) * W + gc] = cs[static_cast<size_t>(j + 1) * W + gc];
     if (KC1 > 0) cs[static_cast<size_t>(KC1 - 1) * W + gc] = pn[c];
   }
-  for (int c = tid; c < DL; c += blockDim.x) {
+  for (int c = tid; c < DL; c += nt) {
     const int vc = g * DL + c;
     if (vc >= vhalf) vs[vc - vhalf] = pn[QKC + c];
   }
@@ -515,6 +551,8 @@ __global__ void __launch_bounds__(128, 1) decode_attn_tc_kernel(
   float *wst = reinterpret_cast<float *>(Vb + 2 * SUB * DL);  // [4 warps][8 heads][DL + 2]
   const int ch = blockIdx.x, g = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31, gr = lane >> 2, qd = lane & 3;
+  pdl_launch_dependents();
+  pdl_wait();
   const int L = lengths[b];
   const int s0 = ch * CHUNK;
   const int n = L < max_seq ? min(CHUNK, L + 1 - s0) : 0;
@@ -735,6 +773,8 @@ __global__ void __launch_bounds__(64) decode_merge16_kernel(
     const int *__restrict__ lengths, __nv_bfloat16 *__restrict__ o_hi,
     __nv_bfloat16 *__restrict__ o_lo, int H, int DL, int max_seq, int nchunk) {
   const int h = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
+  pdl_launch_dependents();
+  pdl_wait();
   if (d >= DL) return;
   const int L = lengths[b];
   const int nused = L >= max_seq ? 0 : min(nchunk, (L + 1 + CHUNK - 1) / CHUNK);
@@ -809,10 +849,10 @@ static cudaError_t launch_decode_attn(const Dims &d, const DecodeArgs &a, float 
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    decode_attn_tc_kernel<DL><<<dim3(a.nchunk, d.Hkv, d.B), 128, smem, st>>>(
-        a.q_new, static_cast<const __half *>(a.k_cache), static_cast<const __half *>(a.v_cache),
-        a.lengths, a.part_o, a.part_ml, d.H, d.Hkv, d.G, a.max_seq, a.nchunk, scale_log2);
-    return cudaGetLastError();
+    return launch_pdl(decode_attn_tc_kernel<DL>, dim3(a.nchunk, d.Hkv, d.B), dim3(128), smem, st,
+                      a.q_new, static_cast<const __half *>(a.k_cache),
+                      static_cast<const __half *>(a.v_cache), a.lengths, a.part_o, a.part_ml,
+                      d.H, d.Hkv, d.G, a.max_seq, a.nchunk, scale_log2);
   }
   const int KS = 128 / (DL / 2);
   const size_t smem = 4 * static_cast<size_t>(SUB) * DL * sizeof(TL) +
@@ -866,9 +906,14 @@ static cudaError_t decode_typed(const Dims &d, const DecodeArgs &a, cudaStream_t
   p2.eps = d.eps;
   for (int i = 0; i < d.DL / 2; ++i)
     p2.theta[i] = pow(static_cast<double>(d.rope_base), -2.0 * i / d.DL);
-  const size_t sm2 = (static_cast<size_t>(d.G + 2) * d.DL + 2 * (d.G + 1) * d.DL + (d.G + 1)) * 4;
-  decode_stencil_kernel<T><<<dim3(d.Hkv, d.B), 128, sm2, st>>>(p2);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const size_t sm2 = d2_smem_floats(d.G, d.DL, d.KC) * 4;
+  auto d2 = d.DL == 16 ? decode_stencil_kernel<T, 16>
+                       : (d.DL == 32 ? decode_stencil_kernel<T, 32> : decode_stencil_kernel<T, 64>);
+  if (sm2 > 48 * 1024) {
+    e = cudaFuncSetAttribute(d2, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sm2));
+    if (e != cudaSuccess) return e;
+  }
+  if ((e = launch_pdl(d2, dim3(d.Hkv, d.B), dim3(256), sm2, st, p2)) != cudaSuccess) return e;
   mark();
   // D3
   const float scale_log2 = static_cast<float>(1.4426950408889634 / sqrt(static_cast<double>(d.DL)));
@@ -880,10 +925,10 @@ static cudaError_t decode_typed(const Dims &d, const DecodeArgs &a, cudaStream_t
   // D3b (+ lengths advance for float32 layers; the 16-bit D4 advances them)
   if constexpr (sizeof(T) == 2) {
     __nv_bfloat16 *o_hi = static_cast<__nv_bfloat16 *>(a.o);
-    decode_merge16_kernel<<<dim3(d.H, d.B), d.DL < 32 ? 32 : d.DL, 0, st>>>(
-        a.part_o, a.part_ml, a.lengths, o_hi, o_hi + static_cast<size_t>(d.B) * d.NQ, d.H, d.DL,
-        a.max_seq, a.nchunk);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    e = launch_pdl(decode_merge16_kernel, dim3(d.H, d.B), dim3(d.DL < 32 ? 32 : d.DL), 0, st,
+                   a.part_o, a.part_ml, a.lengths, o_hi, o_hi + static_cast<size_t>(d.B) * d.NQ,
+                   d.H, d.DL, a.max_seq, a.nchunk);
+    if (e != cudaSuccess) return e;
   } else {
     const int nused_max = a.nchunk;
     const size_t smm = static_cast<size_t>(d.H) * nused_max * 2 * 4;
