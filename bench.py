@@ -272,12 +272,34 @@ def cpu_oracle_sample(w, budget_s=12.0, seed=0):
                        f"this overstates the oracle's full-length rate)")
 
 
+# DRAM bytes (read + write) of one latent-attention launch on the default workload: the
+# ncu capture of the same kernel on one 8192-token sequence of it (profiles/
+# attn_tc_ccgqa_prefill_16k.md) read 25.2 MB, exactly its q, k and v (the k / v tiles that
+# later query tiles re-read stay in L2); q, k and v grow with the token count, so a launch
+# of 2 x 16384 tokens moves 4x that.  Only valid for the kernel version that was profiled.
+ATTN_TRAFFIC = {"ccgqa_prefill_16k": 25198336 * 4}
+
+
 def workload_from_args(args):
     w = W.WORKLOADS[args.workload]
     over = {k: v for k, v in (("batch", args.batch), ("seq", args.seq)) if v is not None}
     if over:
         w = w.with_(name=w.name + "[" + ",".join(f"{k}={v}" for k, v in over.items()) + "]", **over)
     return w
+
+
+def run_decode_only(args):
+    """Only the decode step (a profiling case for the decode kernels): one JSON line."""
+    import compressed_latent_space_b200 as cls
+    cls.load()
+    hbm, _, _, peak_src = measured_peaks()
+    dw = W.WORKLOADS[DECODE_WORKLOAD]
+    dec = bench_decode(cls, dw, args.steps, args.warmup, seed=0)
+    gbs = decode_bytes(dw) / (dec["ms"] * 1e-3) / 1e9
+    print(json.dumps({"metric": "decode GB/s", "value": gbs, "unit": "GB/s",
+                      "ms_per_step": dec["ms"], "frac_of_hbm": gbs / hbm, "peak_source": peak_src,
+                      "workload": dw.name, "stages_ms": dec["stages"],
+                      "gpu_launches": dec["launches"]}), flush=True)
 
 
 def run_cuda(args):
@@ -322,7 +344,7 @@ def run_cuda(args):
         "stages_ms": pre["stages"],
         "roofline": {"kernel": "latent_attention", "bound": "tensor", "achieved": attn_tflops,
                      "peak": bf16_peak, "unit": "TFLOP/s", "frac": attn_tflops / bf16_peak,
-                     "traffic": None, "peak_source": f"{peak_src} bf16 burst"},
+                     "traffic": ATTN_TRAFFIC.get(w.name), "peak_source": f"{peak_src} bf16 burst"},
         "e2e": {"value": tokens * world / (e2e_ms * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": pre["h2d"], "d2h_bytes_per_step": pre["d2h"]},
         "gpu_launches": pre["launches"] + (dec["launches"] if dec else 0),
@@ -382,6 +404,8 @@ def main():
     ap.add_argument("--impl", default="cca", choices=["cca", "reference"])
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--decode-only", action="store_true",
+                    help="time only the decode step (a profiling case for its kernels)")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch (smaller cases for profiling)")
     ap.add_argument("--seq", type=int, default=None,
@@ -390,6 +414,8 @@ def main():
     args.warmup = max(args.warmup, 3)      # at least 3 untimed warm-up steps
     if args.impl == "reference":
         run_reference(args)
+    elif args.decode_only:
+        run_decode_only(args)
     else:
         run_cuda(args)
 
