@@ -5,25 +5,23 @@
 // (gist.science/de explainer, 2. Methodik: Softmax(QK^T)V evaluated entirely in the
 // compressed space; gist.science explainer, Extension: CCGQA.)
 //
-// One CTA owns a 128-row query tile of one head and streams the 128-key tiles 0..qt of its
-// key/value head (causal: tiles past the diagonal are never touched).  Two CTAs share an SM,
-// so one CTA's softmax overlaps the other's tensor-core work.  Per CTA:
-//   warps 0-7 : softmax.  Warp w reads TMEM lanes 32*(w%4).. (one query row per thread) and
-//               key half w/4 of every tile (keys 0-63 or 64-127).  The two warps of a lane
-//               quadrant swap their partial row maxima through shared memory each tile, so
-//               both hold the same reference max.  Online softmax in fp32 with lazy
-//               rescaling (the reference max only moves when a row max grows by more than
-//               2^8); probabilities are packed to float16 pairs and stored into tensor memory,
-//               where the P*V MMA reads them as its A operand.  Each half keeps a partial
-//               row sum and rescales / normalises its half of the output columns.
-//   warp 8    : TMA producer: the Q tile once, then K and V tiles into two rings (K deeper
-//               than V: a K tile is released as soon as its QK^T is done, so the next scores
-//               never wait on the P*V two tiles back).
-//   warp 9    : allocates TMEM and issues tcgen05.mma from one thread: S = Q K^T (M=128,
-//               N=128, K=d~, both from shared memory) and O += P V (M=128, N=d~, K=128, P
-//               from TMEM, V MN-major from shared memory); QK^T of tile j+1 is issued as soon
-//               as every softmax warp has read S of tile j, so it runs under tile j's softmax.
-// TMEM columns: S [0, 128), O [128, 128 + d~), P [128 + d~, 192 + d~) (float16 pairs).
+// One CTA per SM owns two adjacent 128-row query tiles A (2i) and B (2i+1) of one head and
+// streams the 128-key tiles of its key/value head once for both (causal: A reads tiles
+// 0..2i, B 0..2i+1).  The two tiles alternate on the tensor cores, so each tile's softmax
+// runs while the other tile's MMAs execute:
+//   warps 0-3 : softmax of tile A, warps 4-7 : softmax of tile B.  One query row per thread
+//               (warp w reads TMEM lanes 32*(w%4)..), all 128 keys of a tile in registers.
+//               Online softmax in fp32 with lazy rescaling (the reference max only moves when
+//               a row max grows by more than 2^8, and then the warp rescales its rows of O);
+//               the probabilities are packed to float16 pairs and written over the tile's own
+//               scores in TMEM, where the P*V MMA reads them as its A operand.
+//   warp 8    : TMA producer: both Q tiles once, then K and V tiles into two rings.
+//   warp 9    : allocates TMEM (S_A, S_B: 128 fp32 columns each; O_A, O_B: d~ each) and
+//               issues the MMAs (whole warp runs the loop, one elected lane issues).  Per
+//               key tile j: O_A += P_A V_j, S_A = Q_A K_{j+1}^T, O_B += P_B V_j,
+//               S_B = Q_B K_{j+1}^T.  The tensor pipe executes in issue order, so a tile's
+//               next S overwrites its P only after P*V has read it, and a tile's O is final
+//               for the softmax whenever its next S is ready.
 // Every wait is bounded; on a timeout the CTA records it in the status word, stops, and
 // releases its tensor memory.
 #include <math.h>
@@ -36,8 +34,7 @@ namespace {
 
 constexpr int TM = 128;          // query rows per tile (M of all MMAs)
 constexpr int TN = 128;          // keys per tile
-constexpr int KH = TN / 2;       // keys per softmax half
-constexpr int NSOFT = 8;         // softmax warps
+constexpr int NSOFT = 8;         // softmax warps: 4 per query tile
 constexpr int W_TMA = 8, W_MMA = 9;
 constexpr int THREADS = (NSOFT + 2) * 32;
 constexpr float kTau = 8.0f;     // lazy-rescale threshold, log2 units
@@ -45,36 +42,27 @@ constexpr float kTau = 8.0f;     // lazy-rescale threshold, log2 units
 template <int DL>
 struct AttnCfg {
   static constexpr int SK = DL >= 64 ? 3 : 4;          // K ring depth
-  static constexpr int SV = DL >= 64 ? 2 : 3;          // V ring depth
+  static constexpr int SV = DL >= 64 ? 3 : 4;          // V ring depth
   static constexpr int ROWB = DL * 2;                  // bytes of one q / k / v row
   static constexpr int Q_BYTES = TM * ROWB;
   static constexpr int KV_BYTES = TN * ROWB;           // one K or one V tile
   static constexpr uint32_t SW_MODE = ROWB == 128 ? 2u : ROWB == 64 ? 4u : 6u;
   static constexpr int SBO = 8 * ROWB;                 // stride of 8-row core groups
-  static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + Q_BYTES;
+  static constexpr int OFF_Q = 0;                      // Q_A, Q_B
+  static constexpr int OFF_K = OFF_Q + 2 * Q_BYTES;
   static constexpr int OFF_V = OFF_K + SK * KV_BYTES;
-  static constexpr int OFF_X = OFF_V + SV * KV_BYTES;   // row-max swap [2][2][TM] fp32
-  static constexpr int OFF_L = OFF_X + 2 * 2 * TM * 4;      // row-sum swap [2][TM] fp32
-  static constexpr int OFF_BAR = OFF_L + 2 * TM * 4;
+  static constexpr int OFF_BAR = OFF_V + SV * KV_BYTES;
   static constexpr int SMEM = OFF_BAR + 256;
-  static constexpr uint32_t TMEM_COLS = 256;
-  static constexpr uint32_t COL_O = TN;
-  static constexpr uint32_t COL_P = TN + DL;
-  static_assert(COL_P + TN / 2 <= TMEM_COLS, "S, O and P must fit the TMEM allocation");
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t COL_O = 2 * TN;            // O_A at 256, O_B at 256 + d~
+  static_assert(COL_O + 2 * DL <= TMEM_COLS, "S and O of both tiles must fit the TMEM allocation");
 };
 
 struct AttnBars {
   uint64_t q_full;
-  uint64_t k_full[4];
-  uint64_t k_empty[4];
-  uint64_t v_full[4];
-  uint64_t v_empty[4];
-  uint64_t s_full;
-  uint64_t s_free;
-  uint64_t p_full;
-  uint64_t pv_done;
-  uint64_t swap[4];              // per lane quadrant: both halves posted their row values
+  uint64_t k_full[4], k_empty[4];
+  uint64_t v_full[4], v_empty[4];
+  uint64_t s_full[2], p_full[2], o_done[2];
   uint32_t tmem_base;
   int abort;
 };
@@ -121,19 +109,21 @@ __device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
 }
 
 template <int DL>
-__global__ void __launch_bounds__(THREADS, 2)
+__global__ void __launch_bounds__(THREADS, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap mapQ,
                    const __grid_constant__ CUtensorMap mapK,
                    const __grid_constant__ CUtensorMap mapV, __half *__restrict__ O, int S,
-                   int H, int Hkv, int G, float scale_log2, int *status) {
+                   int H, int Hkv, int G, int nqt, float scale_log2, int *status) {
   using C = AttnCfg<DL>;
   extern __shared__ __align__(1024) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h = blockIdx.x, b = blockIdx.y;
-  const int qt = static_cast<int>(gridDim.z) - 1 - static_cast<int>(blockIdx.z);  // long first
+  const int pair = static_cast<int>(gridDim.z) - 1 - static_cast<int>(blockIdx.z);  // long first
+  const int qt0 = 2 * pair;                          // tile A; tile B = qt0 + 1 when it exists
+  const bool hasB = qt0 + 1 < nqt;
+  const int nkvA = qt0 + 1, nkvB = qt0 + 2;
+  const int nsteps = hasB ? nkvB : nkvA;
   const int g = h / G;
-  const int q0 = qt * TM;
-  const int nkv = qt + 1;
   AttnBars *bars = reinterpret_cast<AttnBars *>(smem + C::OFF_BAR);
 
   // The swizzled tiles need 1024-byte alignment; refuse to run otherwise.
@@ -149,11 +139,11 @@ __global__ void __launch_bounds__(THREADS, 2)
       mbar_init(&bars->v_full[s], 1);
       mbar_init(&bars->v_empty[s], 1);
     }
-    mbar_init(&bars->s_full, 1);
-    mbar_init(&bars->s_free, NSOFT);
-    mbar_init(&bars->p_full, NSOFT);
-    mbar_init(&bars->pv_done, 1);
-    for (int e = 0; e < 4; ++e) mbar_init(&bars->swap[e], 2);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&bars->s_full[t], 1);
+      mbar_init(&bars->p_full[t], NSOFT / 2);
+      mbar_init(&bars->o_done[t], 1);
+    }
     bars->abort = 0;
     fence_mbar_init();
   }
@@ -165,7 +155,6 @@ __global__ void __launch_bounds__(THREADS, 2)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
-  const uint32_t tS = tmem, tO = tmem + C::COL_O, tP = tmem + C::COL_P;
   volatile int *abort = &bars->abort;
 
   if (warp == W_TMA) {
@@ -174,9 +163,11 @@ __global__ void __launch_bounds__(THREADS, 2)
       tma_prefetch_desc(&mapQ);
       tma_prefetch_desc(&mapK);
       tma_prefetch_desc(&mapV);
-      mbar_arrive_expect_tx(&bars->q_full, C::Q_BYTES);
-      tma_load_3d(smem + C::OFF_Q, &mapQ, &bars->q_full, 0, q0, b * H + h);
-      for (int j = 0; j < nkv; ++j) {
+      mbar_arrive_expect_tx(&bars->q_full, (hasB ? 2 : 1) * C::Q_BYTES);
+      tma_load_3d(smem + C::OFF_Q, &mapQ, &bars->q_full, 0, qt0 * TM, b * H + h);
+      if (hasB)
+        tma_load_3d(smem + C::OFF_Q + C::Q_BYTES, &mapQ, &bars->q_full, 0, (qt0 + 1) * TM, b * H + h);
+      for (int j = 0; j < nsteps; ++j) {
         const int sk = j % C::SK, sv = j % C::SV;
         if (!mbar_wait(&bars->k_empty[sk], ((j / C::SK) & 1) ^ 1u, abort, status)) break;
         mbar_arrive_expect_tx(&bars->k_full[sk], C::KV_BYTES);
@@ -190,23 +181,20 @@ __global__ void __launch_bounds__(THREADS, 2)
     }
   } else if (warp == W_MMA) {
     // ---------------------------------------------------------------- MMA issuer
-    // The whole warp runs the loop (waits and descriptor arithmetic stay warp-uniform) and
-    // one elected lane issues.  Descriptors advance by adding to their start-address field:
-    // +2 (32 bytes) per 16-wide K step of Q / K, +2*SBO/16 per 16 keys of V.
+    // Descriptors advance by adding to their start-address field: +2 (32 bytes) per 16-wide
+    // K step of Q / K, +2*SBO/16 per 16 keys of V.
     const bool leader = elect_one();
     constexpr uint32_t idesc_qk = idesc_f16_f32(TM, TN, 0, 0, 1);
     constexpr uint32_t idesc_pv = idesc_f16_f32(TM, DL, 0, 1, 1);
-    const uint64_t qd = smem_desc(smem_u32(smem + C::OFF_Q), 16, C::SBO, C::SW_MODE);
-    auto issue_qk = [&](int j) {
-      const int sk = j % C::SK;
-      const uint64_t kd = smem_desc(smem_u32(smem + C::OFF_K + sk * C::KV_BYTES), 16, C::SBO,
-                                    C::SW_MODE);
+    auto issue_qk = [&](int t, int j) {              // S_t = Q_t K_j^T
+      const uint64_t qd = smem_desc(smem_u32(smem + C::OFF_Q + t * C::Q_BYTES), 16, C::SBO, C::SW_MODE);
+      const uint64_t kd = smem_desc(smem_u32(smem + C::OFF_K + (j % C::SK) * C::KV_BYTES), 16,
+                                    C::SBO, C::SW_MODE);
       if (leader) {
 #pragma unroll
         for (int kk = 0; kk < DL / 16; ++kk)
-          umma_f16_ss(tS, qd + 2 * kk, kd + 2 * kk, idesc_qk, kk > 0 ? 1u : 0u);
-        umma_commit(&bars->s_full);
-        umma_commit(&bars->k_empty[sk]);
+          umma_f16_ss(tmem + t * TN, qd + 2 * kk, kd + 2 * kk, idesc_qk, kk > 0 ? 1u : 0u);
+        umma_commit(&bars->s_full[t]);
       }
       __syncwarp();
     };
@@ -214,119 +202,113 @@ __global__ void __launch_bounds__(THREADS, 2)
                                           mbar_wait(&bars->k_full[0], 0, abort, status));
     if (ok) {
       tc_fence_after();
-      issue_qk(0);
+      issue_qk(0, 0);
+      if (hasB) issue_qk(1, 0);
+      if (leader) umma_commit(&bars->k_empty[0]);
+      __syncwarp();
     }
-    for (int j = 0; ok && j < nkv; ++j) {
-      if (j + 1 < nkv) {
-        const int s1 = (j + 1) % C::SK;
-        const uint32_t ph1 = ((j + 1) / C::SK) & 1;
-        ok = __all_sync(0xffffffffu, mbar_wait(&bars->k_full[s1], ph1, abort, status) &&
-                                         mbar_wait(&bars->s_free, j & 1, abort, status));
+    for (int j = 0; ok && j < nsteps; ++j) {
+      const int sv = j % C::SV;
+      const bool nextK = j + 1 < nsteps;
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->v_full[sv], (j / C::SV) & 1, abort, status));
+      if (ok && nextK)
+        ok = __all_sync(0xffffffffu, mbar_wait(&bars->k_full[(j + 1) % C::SK],
+                                               ((j + 1) / C::SK) & 1, abort, status));
+      if (!ok) break;
+      const uint64_t vd = smem_desc(smem_u32(smem + C::OFF_V + sv * C::KV_BYTES), C::KV_BYTES,
+                                    C::SBO, C::SW_MODE);
+      for (int t = 0; t < 2; ++t) {
+        const int nk = t ? nkvB : nkvA;
+        if ((t == 1 && !hasB) || j >= nk) continue;
+        ok = __all_sync(0xffffffffu, mbar_wait(&bars->p_full[t], j & 1, abort, status));
         if (!ok) break;
         tc_fence_after();
-        issue_qk(j + 1);
-      }
-      const int s = j % C::SV;
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars->v_full[s], (j / C::SV) & 1, abort, status) &&
-                                       mbar_wait(&bars->p_full, j & 1, abort, status));
-      if (!ok) break;
-      tc_fence_after();
-      const uint64_t vd = smem_desc(smem_u32(smem + C::OFF_V + s * C::KV_BYTES), C::KV_BYTES,
-                                    C::SBO, C::SW_MODE);
-      if (leader) {
+        const uint32_t tS = tmem + t * TN, tO = tmem + C::COL_O + t * DL;
+        if (leader) {
 #pragma unroll
-        for (int kk = 0; kk < TN / 16; ++kk)      // 16 keys of P = 8 TMEM columns of f16 pairs
-          umma_f16_ts(tO, tP + kk * 8, vd + kk * (2 * C::SBO / 16), idesc_pv,
-                      (j > 0 || kk > 0) ? 1u : 0u);
-        umma_commit(&bars->pv_done);
-        umma_commit(&bars->v_empty[s]);
+          for (int kk = 0; kk < TN / 16; ++kk)    // 16 keys of P = 8 TMEM columns of f16 pairs
+            umma_f16_ts(tO, tS + kk * 8, vd + kk * (2 * C::SBO / 16), idesc_pv,
+                        (j > 0 || kk > 0) ? 1u : 0u);
+          if (j + 1 >= nk) umma_commit(&bars->o_done[t]);
+        }
+        __syncwarp();
+        if (j + 1 < nk) issue_qk(t, j + 1);       // runs after this P*V: it overwrites P_t
+      }
+      if (!ok) break;
+      if (leader) {
+        umma_commit(&bars->v_empty[sv]);
+        if (nextK) umma_commit(&bars->k_empty[(j + 1) % C::SK]);
       }
       __syncwarp();
     }
   } else {
     // ---------------------------------------------------------------- softmax warps 0-7
-    const int quad = warp & 3, hf = warp >> 2;
+    const int t = warp >> 2, quad = warp & 3;
     const int row = quad * 32 + lane;                 // TMEM lane of this thread
-    const int qpos = q0 + row;
+    const int nk = t ? nkvB : nkvA;
+    const int qpos = (qt0 + t) * TM + row;
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-    float *xmax = reinterpret_cast<float *>(smem + C::OFF_X);    // [parity][half][row]
-    float *xsum = reinterpret_cast<float *>(smem + C::OFF_L);    // [half][row]
-    constexpr int OC = DL / 2;                                   // O columns per half
+    const uint32_t tS = tmem + t * TN + lane_off, tO = tmem + C::COL_O + t * DL + lane_off;
+    const uint64_t sc2 = f2(scale_log2, scale_log2);
     float m_ref = -INFINITY, l = 0.f;
-    bool ok = true;
-    for (int j = 0; j < nkv; ++j) {
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full, j & 1, abort, status));
+    bool ok = t == 0 || hasB;
+    for (int j = 0; ok && j < nk; ++j) {
+      // S_t of tile j is ready, and every earlier MMA (this tile's P*V of j-1) is done
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full[t], j & 1, abort, status));
       if (!ok) break;
       tc_fence_after();
-      uint32_t r[KH];
-      tmem_ld32(tS + lane_off + hf * KH, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-      tmem_ld32(tS + lane_off + hf * KH + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+      uint32_t r[TN];
+#pragma unroll
+      for (int c = 0; c < TN / 32; ++c)
+        tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[c * 32]));
       tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->s_free);
-
       // Row max of the raw scores (the 1/sqrt(d~) * log2(e) scale is positive, so it is
       // applied afterwards), in four independent three-input chains.  Keys past this row's
       // position are masked on the diagonal tile only.
-      if (j == nkv - 1) {
-        const int last = qpos - j * TN - hf * KH;     // keys 0..last of this half are visible
+      if (j == nk - 1) {
+        const int last = qpos - j * TN;               // keys 0..last of this tile are visible
 #pragma unroll
-        for (int i = 0; i < KH; ++i)
+        for (int i = 0; i < TN; ++i)
           if (i > last) r[i] = __float_as_uint(-INFINITY);
       }
       float mx4[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) mx4[e] = __uint_as_float(r[e]);
 #pragma unroll
-      for (int i = 4; i < KH; i += 8)
+      for (int i = 4; i < TN; i += 8)
 #pragma unroll
         for (int e = 0; e < 4; ++e)
           mx4[e] = max3(mx4[e], __uint_as_float(r[i + 2 * e]), __uint_as_float(r[i + 2 * e + 1]));
-      float mx = max3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3])) * scale_log2;
-      // swap with the other half of the row (double-buffered by tile parity)
-      xmax[((j & 1) * 2 + hf) * TM + row] = mx;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->swap[quad]);
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars->swap[quad], j & 1, abort, status));
-      if (!ok) break;
-      mx = fmaxf(mx, xmax[((j & 1) * 2 + (hf ^ 1)) * TM + row]);   // finite: key 0 is visible
-
+      const float mx = max3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3])) * scale_log2;  // finite
       const bool resc = mx > m_ref + kTau;
       const float scale = resc ? ex2(m_ref - mx) : 1.f;
       if (resc) m_ref = mx;
       l *= scale;
-      if (j > 0) {
-        // the P columns and O are free once the previous P*V is done
-        ok = __all_sync(0xffffffffu, mbar_wait(&bars->pv_done, (j - 1) & 1, abort, status));
-        if (!ok) break;
-        tc_fence_after();
-        // the tcgen05 loads and stores are warp-wide: the warp rescales together, with
-        // factor 1 in rows that keep their max
-        if (__any_sync(0xffffffffu, resc)) {
+      // O is final up to tile j-1 here; the tcgen05 loads and stores are warp-wide, so the
+      // warp rescales together, with factor 1 in rows that keep their max
+      if (j > 0 && __any_sync(0xffffffffu, resc)) {
 #pragma unroll
-          for (int c = 0; c < OC / 8; ++c) {
-            uint32_t o[8];
-            tmem_ld8(tO + lane_off + hf * OC + c * 8, o);
-            tmem_ld_wait();
+        for (int c = 0; c < DL / 16; ++c) {
+          uint32_t o[16];
+          tmem_ld16(tO + c * 16, o);
+          tmem_ld_wait();
 #pragma unroll
-            for (int e = 0; e < 8; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * scale);
-            tmem_st8(tO + lane_off + hf * OC + c * 8, o);
-          }
+          for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * scale);
+          tmem_st16(tO + c * 16, o);
         }
       }
       // p = 2^(s * scale - m_ref): pairs scaled with one packed FMA, one MUFU ex2 each,
-      // rounded to float16 pairs; four paired partial sums.
-      const uint64_t sc2 = f2(scale_log2, scale_log2), nm2 = f2(-m_ref, -m_ref);
+      // rounded to float16 pairs (written over this tile's scores), four paired partial sums.
+      const uint64_t nm2 = f2(-m_ref, -m_ref);
       uint64_t l2[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) l2[e] = 0;
 #pragma unroll
-      for (int hc = 0; hc < 2; ++hc) {                 // 32 keys -> 16 TMEM columns
+      for (int c = 0; c < TN / 32; ++c) {             // 32 keys -> 16 TMEM columns
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const int i = hc * 32 + 2 * e;
+          const int i = c * 32 + 2 * e;
           const uint64_t x2 = fma2(f2(__uint_as_float(r[i]), __uint_as_float(r[i + 1])), sc2, nm2);
           float x0, x1;
           unf2(x2, x0, x1);
@@ -334,7 +316,7 @@ __global__ void __launch_bounds__(THREADS, 2)
           l2[e & 3] = add2(l2[e & 3], f2(p0, p1));
           pk[e] = pack_f16x2(p0, p1);
         }
-        tmem_st16(tP + lane_off + hf * (KH / 2) + hc * 16, pk);
+        tmem_st16(tS + c * 16, pk);
       }
       {
         const uint64_t s01 = add2(add2(l2[0], l2[1]), add2(l2[2], l2[3]));
@@ -345,26 +327,17 @@ __global__ void __launch_bounds__(THREADS, 2)
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->p_full);
+      if (lane == 0) mbar_arrive(&bars->p_full[t]);
     }
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars->pv_done, (nkv - 1) & 1, abort, status));
-    if (ok) {
-      // row sum = both halves' partial sums (same reference max)
-      xsum[hf * TM + row] = l;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->swap[quad]);
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars->swap[quad], nkv & 1, abort, status));
-    }
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_done[t], 0, abort, status));
     if (ok) {
       tc_fence_after();
-      const float lt = l + xsum[(hf ^ 1) * TM + row];
-      const float inv = lt > 0.f ? 1.f / lt : 0.f;
-      __half *dst = O + (static_cast<size_t>(b) * S + qpos) * (static_cast<size_t>(H) * DL) +
-                    h * DL + hf * OC;
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      __half *dst = O + (static_cast<size_t>(b) * S + qpos) * (static_cast<size_t>(H) * DL) + h * DL;
 #pragma unroll
-      for (int c = 0; c < OC / 8; ++c) {
+      for (int c = 0; c < DL / 8; ++c) {
         uint32_t o[8];
-        tmem_ld8(tO + lane_off + hf * OC + c * 8, o);
+        tmem_ld8(tO + c * 8, o);
         tmem_ld_wait();
         uint4 u;
         u.x = pack_f16x2(__uint_as_float(o[0]) * inv, __uint_as_float(o[1]) * inv);
@@ -414,9 +387,10 @@ cudaError_t launch_tc(const Dims &d, const void *q, const void *k, const void *v
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  dim3 grid(d.H, d.B, (d.S + TM - 1) / TM);
-  attn_tc_kernel<DL><<<grid, THREADS, C::SMEM, st>>>(mq, mk, mv, static_cast<__half *>(o), d.S, d.H,
-                                                  d.Hkv, d.G, scale_log2, status);
+  const int nqt = (d.S + TM - 1) / TM;
+  dim3 grid(d.H, d.B, (nqt + 1) / 2);
+  attn_tc_kernel<DL><<<grid, THREADS, C::SMEM, st>>>(mq, mk, mv, static_cast<__half *>(o), d.S,
+                                                     d.H, d.Hkv, d.G, nqt, scale_log2, status);
   return cudaGetLastError();
 }
 
