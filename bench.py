@@ -277,7 +277,7 @@ def cpu_oracle_sample(w, budget_s=12.0, seed=0):
 # attn_tc_ccgqa_prefill_16k.md) read 25.2 MB, exactly its q, k and v (the k / v tiles that
 # later query tiles re-read stay in L2); q, k and v grow with the token count, so a launch
 # of 2 x 16384 tokens moves 4x that.  Only valid for the kernel version that was profiled.
-ATTN_TRAFFIC = {"ccgqa_prefill_16k": 25198336 * 4}
+ATTN_TRAFFIC = {"ccgqa_prefill_16k": 25204992 * 4}
 
 
 def workload_from_args(args):
