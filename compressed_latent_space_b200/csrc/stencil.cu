@@ -9,8 +9,9 @@
 //   v  = pv[t] on the lower half of the value channels, pv[t-1] on the upper half (Value-Shift)
 //   q, k <- RMS-normalised per head, then rotated by RoPE at position t (RoPE Integration)
 //
-// One CTA owns a tile of TT tokens of one group of one sequence: it stages the group's
-// P rows (plus a halo of KC-1 earlier tokens) in shared memory once, and writes q in
+// One CTA owns a tile of TT tokens of one sequence and walks its key/value groups in turn
+// (the RoPE table of the tile is built once for all of them): per group it stages the
+// group's P rows (plus a halo of KC-1 earlier tokens) in shared memory, and writes q in
 // head-major layout [B, H, S, d~] and k, v in [B, Hkv, kv_stride, d~] (the decode cache when
 // one is given), as float16 for 16-bit layers.
 //
@@ -66,7 +67,8 @@ __device__ __forceinline__ float qk_mean_term(const float *prow, int G, int hh, 
   return 0.5f * (mq / static_cast<float>(G) + pk);
 }
 
-template <typename T, int DL>
+// KCT: the sequence-conv width when it is the common 4 (taps unrolled exactly), 0 = any.
+template <typename T, int DL, int KCT>
 __global__ void __launch_bounds__(512) stencil_kernel(const StencilParams<T> p) {
   using TL = typename StencilParams<T>::TL;
   constexpr bool kTensor = sizeof(T) == 2;
@@ -80,14 +82,25 @@ __global__ void __launch_bounds__(512) stencil_kernel(const StencilParams<T> p) 
   float *Rt = As + TT * QKCP;                       // [TT][HALF][2]
   float *Ws = Rt + TT * DL;                         // [DL][DL+1] (float32 path)
 
-  const int g = blockIdx.y, b = blockIdx.z;
+  const int b = blockIdx.z;
   const int t0 = blockIdx.x * TT;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nwarps = blockDim.x >> 5;
+  const int CH = (G + 2) * DL;
+
+  // RoPE table for this tile, shared by every group: angle = t * base^(-2i/d~).
+  if (p.flags & F_ROPE) {
+    for (int i = tid; i < TT * HALF; i += blockDim.x) {
+      const int tt = i / HALF, ip = i % HALF;
+      rope_cos_sin(static_cast<double>(t0 + tt) * p.theta[ip], Rt[2 * i], Rt[2 * i + 1]);
+    }
+  }
+
+  for (int g = 0; g < p.Hkv; ++g) {
   const int qcol0 = g * G * DL;                     // group's q channels in P
   const int kcol0 = p.NQ + g * DL;
   const int vcol0 = p.NQ + p.NKV + g * DL;
-  const int CH = (G + 2) * DL;
+  if (g > 0) __syncthreads();                       // the previous group is done with Ps / As
 
   // 1. stage P rows t0-halo .. t0+TT-1 of the group's channels (zero outside [0, S)) with
   //    16-byte asynchronous copies, so every thread has all of its loads in flight at once.
@@ -101,38 +114,38 @@ __global__ void __launch_bounds__(512) stencil_kernel(const StencilParams<T> p) 
     cp_async16_zfill(Ps + r * CHP + c, src, in);
   }
   cp_async_wait_all();
-  // RoPE table for this tile: angle = t * base^(-2i/d~).
-  if (p.flags & F_ROPE) {
-    for (int i = tid; i < TT * HALF; i += blockDim.x) {
-      const int tt = i / HALF, ip = i % HALF;
-      rope_cos_sin(static_cast<double>(t0 + tt) * p.theta[ip], Rt[2 * i], Rt[2 * i + 1]);
-    }
-  }
   __syncthreads();
 
   // 2. causal depthwise sequence conv of the q|k channels: one thread per channel, its
   //    filter in registers, sliding along the tile's tokens (KC <= 8).
   for (int c = tid; c < QKC; c += blockDim.x) {
     const int gc = c < G * DL ? qcol0 + c : p.NQ + g * DL + (c - G * DL);
-    const int KC1 = p.KC - 1;
-    float wprev[7], prev[7], wcur = 0.f;
+    constexpr int NP = KCT ? KCT - 1 : 7;           // previous-token taps held in registers
+    const int KC1 = KCT ? KCT - 1 : p.KC - 1;
+    float wprev[NP], prev[NP], wcur = 0.f;
     const int r0 = halo - KC1;                      // Ps row of token t0 - (KC-1)
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const float wj = j < p.KC ? __ldg(p.conv_seq + static_cast<size_t>(gc) * p.KC + j) : 0.f;
-      if (j < 7) wprev[j] = j < KC1 ? wj : 0.f;
+    for (int j = 0; j <= NP; ++j) {
+      const float wj = j <= KC1 ? __ldg(p.conv_seq + static_cast<size_t>(gc) * (KC1 + 1) + j) : 0.f;
+      if (j < NP) wprev[j] = j < KC1 ? wj : 0.f;
       if (j == KC1) wcur = wj;
     }
 #pragma unroll
-    for (int j = 0; j < 7; ++j) prev[j] = j < KC1 ? Ps[(r0 + j) * CHP + c] : 0.f;
+    for (int j = 0; j < NP; ++j) prev[j] = j < KC1 ? Ps[(r0 + j) * CHP + c] : 0.f;
     for (int tt = 0; tt < TT; ++tt) {
       const float cur = Ps[(halo + tt) * CHP + c];  // token t0 + tt
       float a = wcur * cur;
 #pragma unroll
-      for (int j = 0; j < 7; ++j) a = fmaf(wprev[j], prev[j], a);
+      for (int j = 0; j < NP; ++j) a = fmaf(wprev[j], prev[j], a);
       As[tt * QKCP + c] = a;
+      if constexpr (KCT != 0) {
 #pragma unroll
-      for (int j = 0; j < 7; ++j) prev[j] = j + 1 < KC1 ? prev[j + 1] : (j + 1 == KC1 ? cur : prev[j]);
+        for (int j = 0; j + 1 < NP; ++j) prev[j] = prev[j + 1];
+        if (NP > 0) prev[NP - 1] = cur;
+      } else {
+#pragma unroll
+        for (int j = 0; j < NP; ++j) prev[j] = j + 1 < KC1 ? prev[j + 1] : (j + 1 == KC1 ? cur : prev[j]);
+      }
     }
   }
   __syncthreads();
@@ -214,12 +227,13 @@ __global__ void __launch_bounds__(512) stencil_kernel(const StencilParams<T> p) 
         if (t < p.S) {
           TL *dst = is_q ? p.q + ((static_cast<size_t>(b) * p.H + g * G + hh) * p.S + t) * DL
                          : p.k + ((static_cast<size_t>(b) * p.Hkv + g) * p.kv_stride + t) * DL;
+          bool fits = true;                            // every value within the float16 range
 #pragma unroll
           for (int n = 0; n < NT; ++n) {
-            check_latent<TL>(u[n][0], p.status);
-            check_latent<TL>(u[n][1], p.status);
+            fits &= fabsf(u[n][0]) <= kF16Max && fabsf(u[n][1]) <= kF16Max;
             *reinterpret_cast<uint32_t *>(dst + n * 8 + 2 * qc) = pack_f16x2(u[n][0], u[n][1]);
           }
+          if (!fits) report(p.status, DEV_RANGE);
         }
       }
     }
@@ -298,11 +312,14 @@ __global__ void __launch_bounds__(512) stencil_kernel(const StencilParams<T> p) 
     for (int e = 0; e < 2; ++e) {
       const bool shifted = (p.flags & F_VALUE_SHIFT) && (g * DL + c + e >= vhalf);
       val[e] = Ps[(tt + halo - (shifted ? 1 : 0)) * CHP + QKC + c + e];
-      check_latent<TL>(val[e], p.status);
     }
     TL *dst = p.v + ((static_cast<size_t>(b) * p.Hkv + g) * p.kv_stride + t) * DL + c;
-    dst[0] = from_f32<TL>(val[0]);
-    dst[1] = from_f32<TL>(val[1]);
+    if constexpr (sizeof(TL) == 2) {
+      if (!(fabsf(val[0]) <= kF16Max && fabsf(val[1]) <= kF16Max)) report(p.status, DEV_RANGE);
+      *reinterpret_cast<uint32_t *>(dst) = pack_f16x2(val[0], val[1]);
+    } else {
+      *reinterpret_cast<float2 *>(dst) = make_float2(val[0], val[1]);
+    }
   }
 
   // 5. decode state after the last token, written by the tile that holds it.
@@ -325,6 +342,7 @@ __global__ void __launch_bounds__(512) stencil_kernel(const StencilParams<T> p) 
     }
     if (g == 0 && tid == 0) p.lengths[b] = p.S;
   }
+  }  // groups
 }
 
 template <typename T, int DL>
@@ -359,7 +377,7 @@ cudaError_t launch(const Dims &d, const StencilArgs &a, cudaStream_t st) {
   p.TT = TT;
   const size_t smem = stencil_smem_floats(d.G, DL, TT, p.halo, simt) * 4;
   if (smem > 220 * 1024) return cudaErrorInvalidConfiguration;
-  cudaError_t e = cudaFuncSetAttribute(stencil_kernel<T, DL>,
+  cudaError_t e = cudaFuncSetAttribute(d.KC == 4 ? stencil_kernel<T, DL, 4> : stencil_kernel<T, DL, 0>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
@@ -368,8 +386,9 @@ cudaError_t launch(const Dims &d, const StencilArgs &a, cudaStream_t st) {
     const int tasks = (d.G + 1) * (TT / 16);      // (head, 16-token) channel-conv tasks
     threads = 32 * (tasks < 4 ? 4 : tasks > 16 ? 16 : tasks);
   }
-  dim3 grid((d.S + TT - 1) / TT, d.Hkv, d.B);
-  stencil_kernel<T, DL><<<grid, threads, smem, st>>>(p);
+  dim3 grid((d.S + TT - 1) / TT, 1, d.B);
+  if (d.KC == 4) stencil_kernel<T, DL, 4><<<grid, threads, smem, st>>>(p);
+  else stencil_kernel<T, DL, 0><<<grid, threads, smem, st>>>(p);
   return cudaGetLastError();
 }
 
