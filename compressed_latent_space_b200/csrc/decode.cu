@@ -228,6 +228,7 @@ __global__ void __launch_bounds__(256) decode_stencil_kernel(const D2Params<T> p
     const int gc = c < G * DL ? g * G * DL + c : p.NQ + g * DL + (c - G * DL);
     wseq[e] = p.conv_seq[static_cast<size_t>(gc) * KC + t];
   }
+  __syncthreads();                                   // staged filters visible to every thread
   pdl_wait();
   const int L = p.lengths[b];
   if (L >= p.max_seq) {
@@ -796,10 +797,12 @@ __global__ void __launch_bounds__(64) decode_merge16_kernel(
   o_lo[idx] = __float2bfloat16_rn(v - __bfloat162float(hi));
 }
 
+constexpr int kQkvBlocksPerSm = 1;   // QKV projection blocks per SM (split-K fills the rest)
+
 int decode_ksplit(const Dims &d) {
   // enough blocks to keep every SM streaming the weight matrix
   const int nblk = (d.NQKV + 15) / 16;
-  int ks = (num_sms() + nblk - 1) / nblk;
+  int ks = (kQkvBlocksPerSm * num_sms() + nblk - 1) / nblk;
   if (ks < 1) ks = 1;
   while (ks > 1 && d.E / ks < 64) --ks;
   return ks;
