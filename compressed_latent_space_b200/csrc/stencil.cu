@@ -345,6 +345,8 @@ __global__ void __launch_bounds__(512) stencil_kernel(const StencilParams<T> p) 
   }  // groups
 }
 
+constexpr int kTensorSmemKB = 110;   // staging budget per CTA of the 16-bit path
+
 template <typename T, int DL>
 cudaError_t launch(const Dims &d, const StencilArgs &a, cudaStream_t st) {
   using TL = typename LatentType<T>::type;
@@ -371,7 +373,7 @@ cudaError_t launch(const Dims &d, const StencilArgs &a, cudaStream_t st) {
   for (int i = 0; i < DL / 2; ++i)
     p.theta[i] = pow(static_cast<double>(d.rope_base), -2.0 * i / DL);
   // Largest token tile (a multiple of 16) whose staging fits two CTAs per SM.
-  const size_t budget = (simt ? 72 : 110) * 1024;
+  const size_t budget = (simt ? 72 : kTensorSmemKB) * 1024;
   int TT = 64;
   while (TT > 16 && stencil_smem_floats(d.G, DL, TT, p.halo, simt) * 4 > budget) TT /= 2;
   p.TT = TT;
