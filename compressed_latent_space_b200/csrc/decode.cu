@@ -540,8 +540,9 @@ template <int DL>
 __global__ void __launch_bounds__(128, 1) decode_attn_tc_kernel(
     const float *__restrict__ q_new, const __half *__restrict__ k_cache,
     const __half *__restrict__ v_cache, const int *__restrict__ lengths,
-    float *__restrict__ part_o, float *__restrict__ part_ml, int H, int Hkv, int G, int max_seq,
-    int nchunk, float scale_log2) {
+    float *__restrict__ part_o, float *__restrict__ part_ml, __nv_bfloat16 *__restrict__ o_hi,
+    __nv_bfloat16 *__restrict__ o_lo, int H, int Hkv, int G, int max_seq, int chunk, int nchunk,
+    float scale_log2) {
   constexpr int CPR = DL / 8;                        // 16-byte pieces (8 dims) per row
   constexpr int NT = 8;                              // 8-key n-tiles per warp step (64 keys)
   constexpr int WK = NT * 8;                         // keys per warp per sub-chunk
@@ -555,14 +556,21 @@ __global__ void __launch_bounds__(128, 1) decode_attn_tc_kernel(
   pdl_launch_dependents();
   pdl_wait();
   const int L = lengths[b];
-  const int s0 = ch * CHUNK;
-  const int n = L < max_seq ? min(CHUNK, L + 1 - s0) : 0;
+  const int s0 = ch * chunk;
+  const int n = L < max_seq ? min(chunk, L + 1 - s0) : 0;
   float *po = part_o + ((static_cast<size_t>(b) * H + g * G) * nchunk + ch) * DL;
   float *pml = part_ml + ((static_cast<size_t>(b) * H + g * G) * nchunk + ch) * 2;
+  const bool whole = nchunk == 1;                    // one split: write the merged o itself
   if (n <= 0) {
-    for (int i = tid; i < G * DL; i += blockDim.x)
-      po[static_cast<size_t>(i / DL) * nchunk * DL + (i % DL)] = 0.f;
-    for (int h = tid; h < G; h += blockDim.x) {
+    for (int i = tid; i < G * DL; i += blockDim.x) {
+      if (whole) {
+        o_hi[(static_cast<size_t>(b) * H + g * G) * DL + i] = __float2bfloat16_rn(0.f);
+        o_lo[(static_cast<size_t>(b) * H + g * G) * DL + i] = __float2bfloat16_rn(0.f);
+      } else {
+        po[static_cast<size_t>(i / DL) * nchunk * DL + (i % DL)] = 0.f;
+      }
+    }
+    for (int h = tid; h < G && !whole; h += blockDim.x) {
       pml[static_cast<size_t>(h) * nchunk * 2] = -INFINITY;
       pml[static_cast<size_t>(h) * nchunk * 2 + 1] = 0.f;
     }
@@ -722,10 +730,18 @@ __global__ void __launch_bounds__(128, 1) decode_attn_tc_kernel(
       acc = fmaf(c, wst[(w * 8 + h) * WS + d], acc);
       lsum = fmaf(c, wst[(w * 8 + h) * WS + DL + 1], lsum);
     }
-    po[static_cast<size_t>(h) * nchunk * DL + d] = acc;
-    if (d == 0) {
-      pml[static_cast<size_t>(h) * nchunk * 2] = M;
-      pml[static_cast<size_t>(h) * nchunk * 2 + 1] = lsum;
+    if (whole) {
+      const float v = acc / lsum;
+      const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+      const size_t idx = (static_cast<size_t>(b) * H + g * G) * DL + i;
+      o_hi[idx] = hi;
+      o_lo[idx] = __float2bfloat16_rn(v - __bfloat162float(hi));
+    } else {
+      po[static_cast<size_t>(h) * nchunk * DL + d] = acc;
+      if (d == 0) {
+        pml[static_cast<size_t>(h) * nchunk * 2] = M;
+        pml[static_cast<size_t>(h) * nchunk * 2 + 1] = lsum;
+      }
     }
   }
 }
@@ -772,13 +788,13 @@ __global__ void __launch_bounds__(512) decode_merge_kernel(
 __global__ void __launch_bounds__(64) decode_merge16_kernel(
     const float *__restrict__ part_o, const float *__restrict__ part_ml,
     const int *__restrict__ lengths, __nv_bfloat16 *__restrict__ o_hi,
-    __nv_bfloat16 *__restrict__ o_lo, int H, int DL, int max_seq, int nchunk) {
+    __nv_bfloat16 *__restrict__ o_lo, int H, int DL, int max_seq, int chunk, int nchunk) {
   const int h = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
   pdl_launch_dependents();
   pdl_wait();
   if (d >= DL) return;
   const int L = lengths[b];
-  const int nused = L >= max_seq ? 0 : min(nchunk, (L + 1 + CHUNK - 1) / CHUNK);
+  const int nused = L >= max_seq ? 0 : min(nchunk, (L + 1 + chunk - 1) / chunk);
   const float *ml = part_ml + (static_cast<size_t>(b) * H + h) * nchunk * 2;
   const float *po = part_o + (static_cast<size_t>(b) * H + h) * nchunk * DL + d;
   float mx = -INFINITY;
@@ -812,8 +828,19 @@ inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255);
 
 }  // namespace
 
+// Keys per split of the attention: 16-bit layers split each (sequence, group) only as far as
+// needed for one CTA per SM (a batch with enough groups runs unsplit and skips the merge);
+// float32 layers use fixed CHUNK-key splits.
+int decode_chunk(const Dims &d, int max_seq) {
+  if (!d.bf16) return CHUNK;
+  const long units = static_cast<long>(d.B) * d.Hkv;
+  const long nsplit = (num_sms() + units - 1) / units;
+  const long per = (max_seq + nsplit - 1) / nsplit;
+  return static_cast<int>((per + SUB - 1) / SUB * SUB);
+}
+
 size_t decode_workspace_bytes(const Dims &d, int max_seq) {
-  const int nchunk = (max_seq + CHUNK - 1) / CHUNK;
+  const int nchunk = (max_seq + decode_chunk(d, max_seq) - 1) / decode_chunk(d, max_seq);
   const int ks = d.bf16 ? decode_ksplit(d) : 1;
   size_t s = 0;
   s += align256(static_cast<size_t>(ks) * d.B * d.NQKV * 4);
@@ -825,7 +852,8 @@ size_t decode_workspace_bytes(const Dims &d, int max_seq) {
 }
 
 void decode_workspace_carve(const Dims &d, int max_seq, void *ws, DecodeArgs &a) {
-  const int nchunk = (max_seq + CHUNK - 1) / CHUNK;
+  const int chunk = decode_chunk(d, max_seq);
+  const int nchunk = (max_seq + chunk - 1) / chunk;
   const int ks = d.bf16 ? decode_ksplit(d) : 1;
   char *p = static_cast<char *>(ws);
   a.p_part = reinterpret_cast<float *>(p);
@@ -839,7 +867,7 @@ void decode_workspace_carve(const Dims &d, int max_seq, void *ws, DecodeArgs &a)
   a.o = p;
   a.ksplit = ks;
   a.nchunk = nchunk;
-  a.chunk = CHUNK;
+  a.chunk = chunk;
 }
 
 template <int DL, typename TL>
@@ -852,10 +880,12 @@ static cudaError_t launch_decode_attn(const Dims &d, const DecodeArgs &a, float 
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
+    __nv_bfloat16 *o_hi = static_cast<__nv_bfloat16 *>(a.o);
     return launch_pdl(decode_attn_tc_kernel<DL>, dim3(a.nchunk, d.Hkv, d.B), dim3(128), smem, st,
                       a.q_new, static_cast<const __half *>(a.k_cache),
                       static_cast<const __half *>(a.v_cache), a.lengths, a.part_o, a.part_ml,
-                      d.H, d.Hkv, d.G, a.max_seq, a.nchunk, scale_log2);
+                      o_hi, o_hi + static_cast<size_t>(d.B) * d.NQ, d.H, d.Hkv, d.G, a.max_seq,
+                      a.chunk, a.nchunk, scale_log2);
   }
   const int KS = 128 / (DL / 2);
   const size_t smem = 4 * static_cast<size_t>(SUB) * DL * sizeof(TL) +
@@ -927,11 +957,13 @@ static cudaError_t decode_typed(const Dims &d, const DecodeArgs &a, cudaStream_t
   mark();
   // D3b (+ lengths advance for float32 layers; the 16-bit D4 advances them)
   if constexpr (sizeof(T) == 2) {
-    __nv_bfloat16 *o_hi = static_cast<__nv_bfloat16 *>(a.o);
-    e = launch_pdl(decode_merge16_kernel, dim3(d.H, d.B), dim3(d.DL < 32 ? 32 : d.DL), 0, st,
-                   a.part_o, a.part_ml, a.lengths, o_hi, o_hi + static_cast<size_t>(d.B) * d.NQ,
-                   d.H, d.DL, a.max_seq, a.nchunk);
-    if (e != cudaSuccess) return e;
+    if (a.nchunk > 1) {                              // an unsplit attention wrote o itself
+      __nv_bfloat16 *o_hi = static_cast<__nv_bfloat16 *>(a.o);
+      e = launch_pdl(decode_merge16_kernel, dim3(d.H, d.B), dim3(d.DL < 32 ? 32 : d.DL), 0, st,
+                     a.part_o, a.part_ml, a.lengths, o_hi, o_hi + static_cast<size_t>(d.B) * d.NQ,
+                     d.H, d.DL, a.max_seq, a.chunk, a.nchunk);
+      if (e != cudaSuccess) return e;
+    }
   } else {
     const int nused_max = a.nchunk;
     const size_t smm = static_cast<size_t>(d.H) * nused_max * 2 * 4;

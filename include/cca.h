@@ -163,7 +163,7 @@ CCA_API int cca_decode_step(const cca_config_t *cfg, const cca_weights_t *w, con
  * outputs, weights and the cache are the caller's as in cca_decode_step; the step's scratch
  * lives in an 8 MiB array built into the library, held by every GPU that loads the library
  * until the process exits.  A step that needs more scratch (cca_decode_workspace_size above
- * 8 MiB, e.g. 64 sequences of 16 heads with d~ = 32 and a max_seq above 53248) is rejected
+ * 8 MiB, e.g. more than 451 sequences of 16 heads with d~ = 32 and 4 kv heads) is rejected
  * with CCA_ERR_WORKSPACE before anything is launched.  The first call on each device looks
  * up the array's device address (cudaGetSymbolAddress) with that device current; make that
  * first call before any stream capture.  Every call uses the same array and leaves its

@@ -54,12 +54,11 @@ def test_static_scratch_decode_matches_workspace_decode(cuda_lib):
 def test_static_scratch_rejects_oversized_steps(cuda_lib):
     cls = cuda_lib
     w = W.WORKLOADS["ccgqa_decode_8k"]
-    B = w.batch
     inp = W.make_inputs(w.with_(seq=16), seed=0)
     layer = cls.CCALayer.from_workload(w.with_(seq=16), inp)
-    max_seq = 1 << 16
+    B, max_seq = w.batch, w.seq + 16
     while cls.cca_decode_workspace_size(layer.cfg, B, max_seq) <= 8 << 20:
-        max_seq *= 2                                 # a step that needs more than 8 MiB
+        B *= 2                                       # a step that needs more than 8 MiB
     fake = cls.cca_cache_t(16, 32, 48, 64, 80, 96, B, max_seq)     # rejected before any use
     x = torch.zeros(B, w.d_model, dtype=torch.bfloat16, device="cuda")
     y = torch.empty_like(x)
