@@ -133,13 +133,19 @@ def dist_setup(n):
     return rank, world, local
 
 
-def max_over_ranks(x: float, world: int) -> float:
+def max_over_ranks(x: float, world: int, device: str = "cuda") -> float:
+    """The slowest rank's time: every rank contributes, every rank gets the max."""
     if world <= 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(units_per_rank: float, world: int, ms: float) -> float:
+    """Whole-job rate of weak-scaled replicas: every rank's units over the slowest rank's time."""
+    return units_per_rank * world / (ms * 1e-3)
 
 
 def barrier(world):
@@ -325,7 +331,7 @@ def run_cuda(args):
     attn_tflops = attention_flops(w) / (attn_ms * 1e-3) / 1e12
     line = {
         "metric": METRIC,
-        "value": tokens * world / (ms * 1e-3),
+        "value": job_throughput(tokens, world, ms),
         "unit": "tokens/s",
         "n_gpus": world,
         "steps": args.steps,
@@ -348,7 +354,7 @@ def run_cuda(args):
         "roofline": {"kernel": "latent_attention", "bound": "tensor", "achieved": attn_tflops,
                      "peak": bf16_peak, "unit": "TFLOP/s", "frac": attn_tflops / bf16_peak,
                      "traffic": ATTN_TRAFFIC.get(w.name), "peak_source": f"{peak_src} bf16 burst"},
-        "e2e": {"value": tokens * world / (e2e_ms * 1e-3), "unit": "tokens/s",
+        "e2e": {"value": job_throughput(tokens, world, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": pre["h2d"], "d2h_bytes_per_step": pre["d2h"]},
         "gpu_launches": pre["launches"] + (dec["launches"] if dec else 0),
     }
@@ -357,7 +363,7 @@ def run_cuda(args):
         dms = max_over_ranks(dec["ms"], world)
         gbs = decode_bytes(dw) / (dms * 1e-3) / 1e9
         line["decode"] = {"workload": dw.name, "description": dw.description, "ms_per_step": dms,
-                          "tokens_per_s": dw.batch * world / (dms * 1e-3), "GB/s": gbs,
+                          "tokens_per_s": job_throughput(dw.batch, world, dms), "GB/s": gbs,
                           "frac_of_hbm": gbs / hbm, "hbm_peak_GB/s": hbm,
                           "bytes_per_step": decode_bytes(dw), "stages_ms": dec["stages"],
                           "peak_source": peak_src}
