@@ -380,13 +380,7 @@ cudaError_t launch_tc(const Dims &d, const void *q, const void *k, const void *v
         !make_tma_16bit(&mv, v, 3, dims, strides, box, C::ROWB, 1))
       return cudaErrorInvalidValue;
   }
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<DL>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+  if (cudaError_t e = ensure_dyn_smem<attn_tc_kernel<DL>>(C::SMEM); e != cudaSuccess) return e;
   const int nqt = (d.S + TM - 1) / TM;
   dim3 grid(d.H, d.B, (nqt + 1) / 2);
   attn_tc_kernel<DL><<<grid, THREADS, C::SMEM, st>>>(mq, mk, mv, static_cast<__half *>(o), d.S,

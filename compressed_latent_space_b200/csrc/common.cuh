@@ -8,6 +8,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 namespace cca {
 
 // ----------------------------------------------------------------------------- elements
@@ -187,6 +189,19 @@ __device__ __forceinline__ void cp_async16_zfill(void *dst, const void *src, boo
                "r"(valid ? 16 : 0)
                : "memory");
 }
+// The same copy marked for early eviction from L2: for data streamed once (the decode step's
+// cache), so that the stream does not push out what the next kernels read again.
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ void cp_async16_zfill_stream(void *dst, const void *src, bool valid,
+                                                        uint64_t pol) {
+  asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2, %3;"
+               ::"r"(smem_u32(dst)), "l"(src), "r"(valid ? 16 : 0), "l"(pol)
+               : "memory");
+}
 __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;" ::: "memory");
 }
@@ -213,6 +228,29 @@ __device__ __forceinline__ void pdl_launch_dependents() {
 }
 __device__ __forceinline__ void prefetch_l2(const void *p) {
   asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
+// Raises a kernel's dynamic shared-memory limit on the current device, once per (kernel,
+// device, size): the attribute lasts as long as the context, and setting it before every launch
+// adds host time to the launch path of short kernels.  (A context reset in the same process
+// is not tracked: after cudaDeviceReset the library is not usable again.)
+template <auto Kernel>
+inline cudaError_t ensure_dyn_smem(size_t bytes) {
+  constexpr int kDevices = 64;
+  static std::atomic<int> granted[kDevices];          // static storage: starts at zero
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const int want = static_cast<int>(bytes);
+  const bool tracked = dev >= 0 && dev < kDevices;
+  if (tracked && granted[dev].load(std::memory_order_acquire) >= want) return cudaSuccess;
+  e = cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, want);
+  if (e == cudaSuccess && tracked) {
+    int cur = granted[dev].load(std::memory_order_relaxed);
+    while (cur < want && !granted[dev].compare_exchange_weak(cur, want)) {
+    }
+  }
+  return e;
 }
 
 template <typename... KArgs, typename... Args>

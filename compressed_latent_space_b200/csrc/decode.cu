@@ -166,9 +166,7 @@ static cudaError_t launch_skinny(dim3 grid, const __nv_bfloat16 *A, const __nv_b
                                  const __nv_bfloat16 *B, void *C, int M, int N, int K, int kps,
                                  int *lengths, int max_seq, cudaStream_t st) {
   const size_t smem = static_cast<size_t>(S) * skinny_stage_elems<TWO_A>() * 2;
-  cudaError_t e = cudaFuncSetAttribute(skinny_mma_kernel<OUT_F32, TWO_A, S>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  cudaError_t e = ensure_dyn_smem<skinny_mma_kernel<OUT_F32, TWO_A, S>>(smem);
   if (e != cudaSuccess) return e;
   return launch_pdl(skinny_mma_kernel<OUT_F32, TWO_A, S>, grid, dim3(128), smem, st, A, A2, B,
                     C, M, N, K, kps, lengths, max_seq);
@@ -525,9 +523,12 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(
 }
 
 // ------------------------------------------------------------------ D3 on tensor cores
-// The float16-cache variant of D3.  Same blocking (CTA = sequence x kv group x CHUNK-key
-// split, SUB-key sub-chunks through the two-deep copy ring), but each warp owns a 64-key
-// quarter of every sub-chunk and runs its own online softmax on mma.sync tiles:
+// The float16-cache variant of D3.  CTA = sequence x kv group x key split; the split's keys
+// stream through an NSLOT-deep ring of TC_SUB-key sub-chunks (NSLOT - 1 sub-chunks in flight
+// while one is computed: one CTA has to keep enough bytes in flight to draw its share of the
+// memory bandwidth), loaded with an L2 evict-first hint so the stream does not push out the
+// weights and activations the step's other kernels read.  Each warp owns a quarter of every
+// sub-chunk and runs its own online softmax on mma.sync tiles:
 //   S = Q K^T   m16n8k16, rows = the G query heads (rows G..15 zero), 8 keys per n-tile,
 //               Q rounded to float16 like the prefill's latent q, in registers; K through
 //               ldmatrix; the scores are scaled by log2(e)/sqrt(d~) in fp32
@@ -536,6 +537,19 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(
 //               ldmatrix.trans
 // Row max and sum are per head row, reduced over the four lanes that hold a row.  The four
 // warps' (m, l, o) are combined in shared memory before the split's partials are written.
+constexpr int TC_SUB = 256;                  // keys per sub-chunk
+constexpr int TC_RING_BYTES = 96 * 1024;     // copy ring budget (two CTAs per SM at d~ = 32)
+
+template <int DL>
+__host__ __device__ constexpr int tc_slots() {
+  return TC_RING_BYTES / (TC_SUB * DL * 4) > 2 ? TC_RING_BYTES / (TC_SUB * DL * 4) : 2;
+}
+
+template <int DL>
+__host__ __device__ constexpr size_t tc_smem_bytes() {
+  return static_cast<size_t>(tc_slots<DL>()) * TC_SUB * DL * 4 + 4 * 8 * (DL + 2) * 4;
+}
+
 template <int DL>
 __global__ void __launch_bounds__(128, 1) decode_attn_tc_kernel(
     const float *__restrict__ q_new, const __half *__restrict__ k_cache,
@@ -544,13 +558,14 @@ __global__ void __launch_bounds__(128, 1) decode_attn_tc_kernel(
     __nv_bfloat16 *__restrict__ o_lo, int H, int Hkv, int G, int max_seq, int chunk, int nchunk,
     float scale_log2) {
   constexpr int CPR = DL / 8;                        // 16-byte pieces (8 dims) per row
-  constexpr int NT = 8;                              // 8-key n-tiles per warp step (64 keys)
+  constexpr int NSLOT = tc_slots<DL>();
+  constexpr int NT = TC_SUB / 32;                    // 8-key n-tiles per warp step
   constexpr int WK = NT * 8;                         // keys per warp per sub-chunk
-  static_assert(4 * WK == SUB, "four warps cover a sub-chunk");
+  static_assert(4 * WK == TC_SUB && NT % 2 == 0, "four warps cover a sub-chunk");
   extern __shared__ __align__(16) uint8_t smraw[];
-  __half *Kb = reinterpret_cast<__half *>(smraw);    // [2][SUB][DL], swizzled pieces
-  __half *Vb = Kb + 2 * SUB * DL;                    // [2][SUB][DL], swizzled pieces
-  float *wst = reinterpret_cast<float *>(Vb + 2 * SUB * DL);  // [4 warps][8 heads][DL + 2]
+  __half *Kb = reinterpret_cast<__half *>(smraw);    // [NSLOT][TC_SUB][DL], swizzled pieces
+  __half *Vb = Kb + NSLOT * TC_SUB * DL;             // [NSLOT][TC_SUB][DL], swizzled pieces
+  float *wst = reinterpret_cast<float *>(Vb + NSLOT * TC_SUB * DL);  // [4][8 heads][DL + 2]
   const int ch = blockIdx.x, g = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31, gr = lane >> 2, qd = lane & 3;
   pdl_launch_dependents();
@@ -577,21 +592,25 @@ __global__ void __launch_bounds__(128, 1) decode_attn_tc_kernel(
     return;
   }
   const size_t row0 = (static_cast<size_t>(b) * Hkv + g) * max_seq + s0;
-  const int nsub = (n + SUB - 1) / SUB;
-  auto issue = [&](int sbi) {                        // sub-chunk sbi into slot sbi & 1;
-    const int base = sbi * SUB, cnt = min(SUB, n - base);   // rows past cnt are zero-filled
-    __half *kd = Kb + (sbi & 1) * SUB * DL, *vd = Vb + (sbi & 1) * SUB * DL;
-    for (int i = tid; i < SUB * CPR; i += blockDim.x) {
-      const int r = i / CPR, j = i % CPR;
-      const bool ok = r < cnt;
-      const size_t src = (row0 + base + (ok ? r : 0)) * DL + j * 8;
-      const int dst = r * DL + (j ^ kv_swz<CPR>(r)) * 8;
-      cp_async16_zfill(kd + dst, k_cache + src, ok);
-      cp_async16_zfill(vd + dst, v_cache + src, ok);
+  const int nsub = (n + TC_SUB - 1) / TC_SUB;
+  const uint64_t stream_pol = l2_evict_first_policy();
+  auto issue = [&](int sbi) {                        // sub-chunk sbi into slot sbi % NSLOT;
+    if (sbi < nsub) {                                // an empty group past the last one
+      const int base = sbi * TC_SUB, cnt = min(TC_SUB, n - base);  // rows past cnt: zeros
+      __half *kd = Kb + (sbi % NSLOT) * TC_SUB * DL, *vd = Vb + (sbi % NSLOT) * TC_SUB * DL;
+      for (int i = tid; i < TC_SUB * CPR; i += blockDim.x) {
+        const int r = i / CPR, j = i % CPR;
+        const bool ok = r < cnt;
+        const size_t src = (row0 + base + (ok ? r : 0)) * DL + j * 8;
+        const int dst = r * DL + (j ^ kv_swz<CPR>(r)) * 8;
+        cp_async16_zfill_stream(kd + dst, k_cache + src, ok, stream_pol);
+        cp_async16_zfill_stream(vd + dst, v_cache + src, ok, stream_pol);
+      }
     }
     cp_async_commit();
   };
-  issue(0);
+#pragma unroll
+  for (int s = 0; s < NSLOT - 1; ++s) issue(s);
 
   // Q fragments (rows = heads; a1, a3 are rows 8..15 and stay zero)
   uint32_t qa[DL / 16][2];
@@ -616,17 +635,13 @@ __global__ void __launch_bounds__(128, 1) decode_attn_tc_kernel(
   float m_run = -INFINITY, l_run = 0.f;              // of head row gr (lanes of one quad agree)
 
   for (int sbi = 0; sbi < nsub; ++sbi) {
-    if (sbi + 1 < nsub) {
-      issue(sbi + 1);
-      cp_async_wait_one();                           // sub-chunk sbi has landed
-    } else {
-      cp_async_wait_none();
-    }
-    __syncthreads();
-    const uint32_t ks_base = smem_u32(Kb + (sbi & 1) * SUB * DL);
-    const uint32_t vs_base = smem_u32(Vb + (sbi & 1) * SUB * DL);
+    cp_async_wait_group<NSLOT - 2>();                // sub-chunk sbi has landed
+    __syncthreads();                                 // ... for every thread; and every warp
+    issue(sbi + NSLOT - 1);                          // is done with the slot refilled here
+    const uint32_t ks_base = smem_u32(Kb + (sbi % NSLOT) * TC_SUB * DL);
+    const uint32_t vs_base = smem_u32(Vb + (sbi % NSLOT) * TC_SUB * DL);
     const int kb = warp * WK;                        // this warp's first key in the sub-chunk
-    const int valid = n - sbi * SUB - kb;            // keys of this warp's slice that exist
+    const int valid = n - sbi * TC_SUB - kb;         // keys of this warp's slice that exist
     if (valid > 0) {
       // ---- S = Q K^T over 8 n-tiles
       float sc[NT][4];
@@ -695,8 +710,8 @@ __global__ void __launch_bounds__(128, 1) decode_attn_tc_kernel(
         }
       }
     }
-    __syncthreads();                                 // slot sbi & 1 is refilled next
   }
+  cp_async_wait_group<0>();                          // only empty groups can be left
 
   // ---- combine the four warps: each posts (m, l, o) of its head rows
   l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
@@ -836,7 +851,7 @@ int decode_chunk(const Dims &d, int max_seq) {
   const long units = static_cast<long>(d.B) * d.Hkv;
   const long nsplit = (num_sms() + units - 1) / units;
   const long per = (max_seq + nsplit - 1) / nsplit;
-  return static_cast<int>((per + SUB - 1) / SUB * SUB);
+  return static_cast<int>((per + TC_SUB - 1) / TC_SUB * TC_SUB);
 }
 
 size_t decode_workspace_bytes(const Dims &d, int max_seq) {
@@ -874,11 +889,8 @@ template <int DL, typename TL>
 static cudaError_t launch_decode_attn(const Dims &d, const DecodeArgs &a, float scale_log2,
                                       cudaStream_t st) {
   if constexpr (sizeof(TL) == 2) {
-    const size_t smem = 4 * static_cast<size_t>(SUB) * DL * sizeof(TL) +
-                        static_cast<size_t>(4 * 8 * (DL + 2)) * 4;
-    cudaError_t e = cudaFuncSetAttribute(decode_attn_tc_kernel<DL>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
+    const size_t smem = tc_smem_bytes<DL>();
+    cudaError_t e = ensure_dyn_smem<decode_attn_tc_kernel<DL>>(smem);
     if (e != cudaSuccess) return e;
     __nv_bfloat16 *o_hi = static_cast<__nv_bfloat16 *>(a.o);
     return launch_pdl(decode_attn_tc_kernel<DL>, dim3(a.nchunk, d.Hkv, d.B), dim3(128), smem, st,
@@ -891,9 +903,7 @@ static cudaError_t launch_decode_attn(const Dims &d, const DecodeArgs &a, float 
   const size_t smem = 4 * static_cast<size_t>(SUB) * DL * sizeof(TL) +
                       (static_cast<size_t>(d.G) * DL + static_cast<size_t>(d.G) * SUB +
                        static_cast<size_t>(KS) * d.G * DL + 3 * d.G) * 4;
-  cudaError_t e = cudaFuncSetAttribute(decode_attn_kernel<DL, TL>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  cudaError_t e = ensure_dyn_smem<decode_attn_kernel<DL, TL>>(smem);
   if (e != cudaSuccess) return e;
   decode_attn_kernel<DL, TL><<<dim3(a.nchunk, d.Hkv, d.B), 128, smem, st>>>(
       a.q_new, static_cast<const TL *>(a.k_cache), static_cast<const TL *>(a.v_cache), a.lengths,
@@ -943,7 +953,9 @@ static cudaError_t decode_typed(const Dims &d, const DecodeArgs &a, cudaStream_t
   auto d2 = d.DL == 16 ? decode_stencil_kernel<T, 16>
                        : (d.DL == 32 ? decode_stencil_kernel<T, 32> : decode_stencil_kernel<T, 64>);
   if (sm2 > 48 * 1024) {
-    e = cudaFuncSetAttribute(d2, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sm2));
+    e = d.DL == 16 ? ensure_dyn_smem<decode_stencil_kernel<T, 16>>(sm2)
+                   : (d.DL == 32 ? ensure_dyn_smem<decode_stencil_kernel<T, 32>>(sm2)
+                                 : ensure_dyn_smem<decode_stencil_kernel<T, 64>>(sm2));
     if (e != cudaSuccess) return e;
   }
   if ((e = launch_pdl(d2, dim3(d.Hkv, d.B), dim3(256), sm2, st, p2)) != cudaSuccess) return e;
@@ -968,8 +980,7 @@ static cudaError_t decode_typed(const Dims &d, const DecodeArgs &a, cudaStream_t
     const int nused_max = a.nchunk;
     const size_t smm = static_cast<size_t>(d.H) * nused_max * 2 * 4;
     if (smm > 48 * 1024) {
-      e = cudaFuncSetAttribute(decode_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(smm));
+      e = ensure_dyn_smem<decode_merge_kernel>(smm);
       if (e != cudaSuccess) return e;
     }
     const int threads = d.H * d.DL < 512 ? ((d.H * d.DL + 31) / 32) * 32 : 512;

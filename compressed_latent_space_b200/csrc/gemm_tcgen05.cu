@@ -236,14 +236,9 @@ int num_sms() {
 template <typename OutT, int AB_F16>
 static cudaError_t launch_gemm(const CUtensorMap &ma, const CUtensorMap &mb, void *C, int M,
                                int N, int K, int *status, cudaStream_t st) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_bf16_kernel<OutT, AB_F16>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(SMEM_BYTES));
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  if (cudaError_t e = ensure_dyn_smem<gemm_bf16_kernel<OutT, AB_F16>>(SMEM_BYTES);
+      e != cudaSuccess)
+    return e;
   const int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
   const int grid = tiles < num_sms() ? tiles : num_sms();
   gemm_bf16_kernel<OutT, AB_F16><<<grid, THREADS, SMEM_BYTES, st>>>(ma, mb, static_cast<OutT *>(C), M,

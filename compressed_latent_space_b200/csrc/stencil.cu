@@ -379,9 +379,8 @@ cudaError_t launch(const Dims &d, const StencilArgs &a, cudaStream_t st) {
   p.TT = TT;
   const size_t smem = stencil_smem_floats(d.G, DL, TT, p.halo, simt) * 4;
   if (smem > 220 * 1024) return cudaErrorInvalidConfiguration;
-  cudaError_t e = cudaFuncSetAttribute(d.KC == 4 ? stencil_kernel<T, DL, 4> : stencil_kernel<T, DL, 0>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  cudaError_t e = d.KC == 4 ? ensure_dyn_smem<stencil_kernel<T, DL, 4>>(smem)
+                            : ensure_dyn_smem<stencil_kernel<T, DL, 0>>(smem);
   if (e != cudaSuccess) return e;
   int threads = 256;
   if (!simt) {
