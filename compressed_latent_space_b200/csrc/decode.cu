@@ -24,20 +24,21 @@ constexpr int CHUNK = 1024;       // keys per split-KV block
 
 // ------------------------------------------------------------------ D1 / D4 on staged tiles
 // C[M, N] = A[M, K] B[N, K]^T (+ A2[M, K] B^T) for M <= 64 per CTA row block, bfloat16
-// operands, fp32 accumulation.  Grid (ceil(N / 16), ksplit, ceil(M / 64)): a CTA owns 16
+// operands, fp32 accumulation.  Grid (ceil(N / NC), ksplit, ceil(M / 64)): a CTA owns NC
 // columns and one K slice, which it walks in 64-wide chunks staged in shared memory by 16-byte
 // cp.async through an S-deep ring (S - 1 chunks in flight while one is computed; rows padded
 // by 16 bytes so the ldmatrix reads are conflict-free).  Warp w computes rows 16w..16w+15 x
-// the 16 columns with mma.sync.  TWO_A adds a second A operand (the low bf16 halves of an fp32
+// the NC columns with mma.sync.  Each staged A row serves NC columns, so A crosses from L2
+// N / NC times in all.  TWO_A adds a second A operand (the low bf16 halves of an fp32
 // A split hi + lo).  OUT_F32: fp32 partial sums to C + ks*M*N; else bf16.  `lengths`
 // (optional): block (0, 0, 0) advances lengths[m] for m < M where it is below max_seq (the
 // last kernel of a decode step).
 constexpr int SK_KC = 64;           // K chunk
 constexpr int SK_LD = SK_KC + 8;    // padded row, in elements
 
-template <bool TWO_A>
+template <bool TWO_A, int NC>
 __host__ __device__ constexpr int skinny_stage_elems() {
-  return ((TWO_A ? 2 : 1) * 64 + 16) * SK_LD;
+  return ((TWO_A ? 2 : 1) * 64 + NC) * SK_LD;
 }
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2,
@@ -58,21 +59,22 @@ __device__ __forceinline__ void cp_async_wait_group() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-template <bool OUT_F32, bool TWO_A, int S>
+template <bool OUT_F32, bool TWO_A, int S, int NC>
 __global__ void __launch_bounds__(128) skinny_mma_kernel(
     const __nv_bfloat16 *__restrict__ A, const __nv_bfloat16 *__restrict__ A2,
     const __nv_bfloat16 *__restrict__ B, void *__restrict__ C, int M, int N, int K,
     int k_per_split, int *lengths, int max_seq) {
-  constexpr int STAGE = skinny_stage_elems<TWO_A>();
+  static_assert(NC % 16 == 0, "16 columns per B load");
+  constexpr int STAGE = skinny_stage_elems<TWO_A, NC>();
   extern __shared__ __align__(16) __nv_bfloat16 sk_smem[];     // [S][A (A2) B]
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int n0 = blockIdx.x * 16, ks = blockIdx.y, m0 = blockIdx.z * 64;
+  const int n0 = blockIdx.x * NC, ks = blockIdx.y, m0 = blockIdx.z * 64;
   const int kbeg = ks * k_per_split, kend = min(K, kbeg + k_per_split);
   pdl_launch_dependents();
   {
     // the weight slab does not depend on the previous kernel: pull it towards L2 meanwhile
     const int lines = kend > kbeg ? ((kend - kbeg) * 2 + 127) / 128 : 0;
-    for (int i = tid; i < 16 * lines; i += 128) {
+    for (int i = tid; i < NC * lines; i += 128) {
       const int r = i / lines, c = i % lines;
       if (n0 + r < N) prefetch_l2(B + static_cast<size_t>(n0 + r) * K + kbeg + c * 64);
     }
@@ -95,7 +97,7 @@ __global__ void __launch_bounds__(128) skinny_mma_kernel(
         if constexpr (TWO_A) cp_async16_zfill(st + (64 + r) * SK_LD + j * 8, A2 + off, ok);
       }
       __nv_bfloat16 *bs = st + (TWO_A ? 128 : 64) * SK_LD;
-      for (int i = tid; i < 16 * (SK_KC / 8); i += 128) {     // B: 16 x SK_KC
+      for (int i = tid; i < NC * (SK_KC / 8); i += 128) {     // B: NC x SK_KC
         const int r = i / (SK_KC / 8), j = i % (SK_KC / 8);
         const int k = k0 + j * 8;
         const bool ok = n0 + r < N && k < kend;
@@ -105,9 +107,9 @@ __global__ void __launch_bounds__(128) skinny_mma_kernel(
     }
     cp_async_commit();
   };
-  float acc[2][4];
+  float acc[NC / 8][4];
 #pragma unroll
-  for (int t = 0; t < 2; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
+  for (int t = 0; t < NC / 8; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
 #pragma unroll
   for (int c = 0; c < S - 1; ++c) issue(c);
   for (int c = 0; c < nchunks; ++c) {
@@ -120,17 +122,20 @@ __global__ void __launch_bounds__(128) skinny_mma_kernel(
                                      ((lane >> 3) & 1) * 8);
 #pragma unroll
     for (int kk = 0; kk < SK_KC / 16; ++kk) {
-      uint32_t a[4], bq[4];
+      uint32_t a[4], a2[4];
       ldsm_x4(a_base + kk * 32, a[0], a[1], a[2], a[3]);
-      ldsm_x4(b_base + kk * 32, bq[0], bq[1], bq[2], bq[3]);
-      const uint32_t b0[2] = {bq[0], bq[1]}, b1[2] = {bq[2], bq[3]};
-      mma_bf16_16816(acc[0], a, b0);
-      mma_bf16_16816(acc[1], a, b1);
-      if constexpr (TWO_A) {
-        uint32_t a2[4];
-        ldsm_x4(a_base + kk * 32 + 64 * SK_LD * 2, a2[0], a2[1], a2[2], a2[3]);
-        mma_bf16_16816(acc[0], a2, b0);
-        mma_bf16_16816(acc[1], a2, b1);
+      if constexpr (TWO_A) ldsm_x4(a_base + kk * 32 + 64 * SK_LD * 2, a2[0], a2[1], a2[2], a2[3]);
+#pragma unroll
+      for (int t = 0; t < NC / 8; t += 2) {           // 16 columns per B load
+        uint32_t bq[4];
+        ldsm_x4(b_base + t * 8 * SK_LD * 2 + kk * 32, bq[0], bq[1], bq[2], bq[3]);
+        const uint32_t b0[2] = {bq[0], bq[1]}, b1[2] = {bq[2], bq[3]};
+        mma_bf16_16816(acc[t], a, b0);
+        mma_bf16_16816(acc[t + 1], a, b1);
+        if constexpr (TWO_A) {
+          mma_bf16_16816(acc[t], a2, b0);
+          mma_bf16_16816(acc[t + 1], a2, b1);
+        }
       }
     }
     __syncthreads();                                  // stage c % S is refilled next
@@ -138,7 +143,7 @@ __global__ void __launch_bounds__(128) skinny_mma_kernel(
   cp_async_wait_group<0>();
   const int gr = lane >> 2, qc = lane & 3;
 #pragma unroll
-  for (int t = 0; t < 2; ++t) {
+  for (int t = 0; t < NC / 8; ++t) {
     const int n = n0 + t * 8 + 2 * qc;
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
@@ -161,15 +166,17 @@ __global__ void __launch_bounds__(128) skinny_mma_kernel(
   }
 }
 
-template <bool OUT_F32, bool TWO_A, int S>
-static cudaError_t launch_skinny(dim3 grid, const __nv_bfloat16 *A, const __nv_bfloat16 *A2,
-                                 const __nv_bfloat16 *B, void *C, int M, int N, int K, int kps,
+template <bool OUT_F32, bool TWO_A, int S, int NC>
+static cudaError_t launch_skinny(int ksplit, const __nv_bfloat16 *A, const __nv_bfloat16 *A2,
+                                 const __nv_bfloat16 *B, void *C, int M, int N, int K,
                                  int *lengths, int max_seq, cudaStream_t st) {
-  const size_t smem = static_cast<size_t>(S) * skinny_stage_elems<TWO_A>() * 2;
-  cudaError_t e = ensure_dyn_smem<skinny_mma_kernel<OUT_F32, TWO_A, S>>(smem);
+  const int kps = ((K + ksplit - 1) / ksplit + SK_KC - 1) / SK_KC * SK_KC;
+  const dim3 grid((N + NC - 1) / NC, ksplit, (M + 63) / 64);
+  const size_t smem = static_cast<size_t>(S) * skinny_stage_elems<TWO_A, NC>() * 2;
+  cudaError_t e = ensure_dyn_smem<skinny_mma_kernel<OUT_F32, TWO_A, S, NC>>(smem);
   if (e != cudaSuccess) return e;
-  return launch_pdl(skinny_mma_kernel<OUT_F32, TWO_A, S>, grid, dim3(128), smem, st, A, A2, B,
-                    C, M, N, K, kps, lengths, max_seq);
+  return launch_pdl(skinny_mma_kernel<OUT_F32, TWO_A, S, NC>, grid, dim3(128), smem, st, A, A2,
+                    B, C, M, N, K, kps, lengths, max_seq);
 }
 
 // ------------------------------------------------------------------ D2 decode stencil
@@ -192,12 +199,16 @@ struct D2Params {
 // D2 keeps the group's channel filters transposed in shared memory, wt[j][o] = the weight of
 // input j for output channel o (o over the G q heads and the k head, d~ each), rows padded to
 // an odd length so both the transposing writes and the per-output reads are conflict-free.
-// The filters, which no earlier kernel writes, are staged before the grid-dependency wait.
+// The filters, which no earlier kernel writes, are staged before the grid-dependency wait;
+// the sequence's conv state is only prefetched into L2 then (the previous step may still be
+// writing it, and L2 keeps a prefetched line coherent).  After the wait the projections and
+// the state are loaded together, and the old state stays in shared memory for the shift.
 __host__ __device__ constexpr int d2_ld(int QKC) { return QKC | 1; }
 __host__ __device__ inline size_t d2_smem_floats(int G, int DL, int KC) {
   const int QKC = (G + 1) * DL, CH = (G + 2) * DL;
   return static_cast<size_t>(DL) * d2_ld(QKC)   // wt
          + QKC * KC                             // sequence filters
+         + static_cast<size_t>(QKC) * (KC - 1)  // old conv state
          + CH + 2 * QKC + 16;                   // pn, av, uv, inv
 }
 
@@ -210,7 +221,8 @@ __global__ void __launch_bounds__(256) decode_stencil_kernel(const D2Params<T> p
   const int LD = d2_ld(QKC);
   float *wt = sm;
   float *wseq = wt + DL * LD;
-  float *pn = wseq + QKC * KC;
+  float *old = wseq + QKC * KC;                      // [KC-1][QKC] conv state before the step
+  float *pn = old + QKC * KC1;
   float *a = pn + CH;
   float *u = a + QKC;
   float *inv = u + QKC;
@@ -226,31 +238,46 @@ __global__ void __launch_bounds__(256) decode_stencil_kernel(const D2Params<T> p
     const int gc = c < G * DL ? g * G * DL + c : p.NQ + g * DL + (c - G * DL);
     wseq[e] = p.conv_seq[static_cast<size_t>(gc) * KC + t];
   }
-  __syncthreads();                                   // staged filters visible to every thread
-  pdl_wait();
-  const int L = p.lengths[b];
-  if (L >= p.max_seq) {
-    if (tid == 0) report(p.status, DEV_CACHE_FULL);
-    return;
-  }
   const int qcol0 = g * G * DL, kcol0 = p.NQ + g * DL, vcol0 = p.NQ + p.NKV + g * DL;
   auto gch = [&](int c) {
     return c < G * DL ? qcol0 + c : (c < QKC ? kcol0 + (c - G * DL) : vcol0 + (c - QKC));
   };
   const int W = p.NQ + p.NKV;
   float *cs = p.conv_state + static_cast<size_t>(b) * KC1 * W;
-  // new projections (sum of the split-K partials) and the sequence conv of the q|k channels
+  for (int e = tid; e < KC1 * (G + 1); e += nt) {   // the state rows of this group's channels
+    const int j = e / (G + 1), part = e % (G + 1);  // (G q heads' DL run is contiguous)
+    const float *row = cs + static_cast<size_t>(j) * W;
+    const float *seg = part == 0 ? row + qcol0 : row + kcol0;
+    const int len = part == 0 ? G * DL : DL;
+    for (int off = 0; off < len; off += 32) prefetch_l2(seg + off);
+  }
+  __syncthreads();                                   // staged filters visible to every thread
+  pdl_wait();
+  // the token's projections (sum of the split-K partials) and the old conv state, loaded
+  // together before the position is known
   for (int c = tid; c < CH; c += nt) {
     const int gc = gch(c);
     float v = 0.f;
     for (int ks = 0; ks < p.ksplit; ++ks) v += p.p_part[(static_cast<size_t>(ks) * p.B + b) * p.NQKV + gc];
     pn[c] = v;
-    if (c < QKC) {
-      const float *w = wseq + c * KC;
-      float acc = 0.f;
-      for (int j = 0; j < KC1; ++j) acc = fmaf(w[j], cs[static_cast<size_t>(j) * W + gc], acc);
-      a[c] = fmaf(w[KC1], v, acc);
-    }
+    if (c < QKC)
+      for (int j = 0; j < KC1; ++j) old[j * QKC + c] = cs[static_cast<size_t>(j) * W + gc];
+  }
+  const int L = p.lengths[b];
+  if (L >= p.max_seq) {
+    if (tid == 0) report(p.status, DEV_CACHE_FULL);
+    return;
+  }
+  constexpr int HALF = DL / 2;
+  float rc = 1.f, rs = 0.f;                          // RoPE rotation of this thread's pairs
+  if ((p.flags & F_ROPE) && tid < (G + 1) * HALF)
+    rope_cos_sin(static_cast<double>(L) * p.theta[tid % HALF], rc, rs);
+  // the sequence conv of the q|k channels (each thread reads only what it loaded)
+  for (int c = tid; c < QKC; c += nt) {
+    const float *w = wseq + c * KC;
+    float acc = 0.f;
+    for (int j = 0; j < KC1; ++j) acc = fmaf(w[j], old[j * QKC + c], acc);
+    a[c] = fmaf(w[KC1], pn[c], acc);
   }
   __syncthreads();
   // channel conv (thread per output) and q-k-mean
@@ -284,15 +311,14 @@ __global__ void __launch_bounds__(256) decode_stencil_kernel(const D2Params<T> p
       inv[hh] = (p.flags & F_QK_NORM) ? 1.0f / sqrtf(ss / static_cast<float>(DL) + p.eps) : 1.0f;
   }
   __syncthreads();
-  // RoPE at position L on (i, i + DL/2) pairs, then store q (workspace) and k (cache)
-  constexpr int HALF = DL / 2;
+  // RoPE at position L on (i, i + DL/2) pairs, then store q (workspace) and k (cache); every
+  // pair a thread takes has i = tid mod DL/2 (DL/2 divides the block size), whose rotation it
+  // computed above
   for (int o = tid; o < (G + 1) * HALF; o += nt) {
     const int hh = o / HALF, ip = o % HALF;
     float x1 = u[hh * DL + ip] * inv[hh], x2 = u[hh * DL + ip + HALF] * inv[hh];
     if (p.flags & F_ROPE) {
-      float c, sn;
-      rope_cos_sin(static_cast<double>(L) * p.theta[ip], c, sn);
-      const float y1 = x1 * c - x2 * sn, y2 = x1 * sn + x2 * c;
+      const float y1 = x1 * rc - x2 * rs, y2 = x1 * rs + x2 * rc;
       x1 = y1;
       x2 = y2;
     }
@@ -318,10 +344,9 @@ __global__ void __launch_bounds__(256) decode_stencil_kernel(const D2Params<T> p
     check_latent<TL>(val, p.status);
     p.v_cache[((static_cast<size_t>(b) * p.Hkv + g) * p.max_seq + L) * DL + c] = from_f32<TL>(val);
   }
-  __syncthreads();   // every read of the old state is done
   for (int c = tid; c < QKC; c += nt) {
     const int gc = gch(c);
-    for (int j = 0; j + 1 < KC1; ++j) cs[static_cast<size_t>(j) * W + gc] = cs[static_cast<size_t>(j + 1) * W + gc];
+    for (int j = 0; j + 1 < KC1; ++j) cs[static_cast<size_t>(j) * W + gc] = old[(j + 1) * QKC + c];
     if (KC1 > 0) cs[static_cast<size_t>(KC1 - 1) * W + gc] = pn[c];
   }
   for (int c = tid; c < DL; c += nt) {
@@ -556,7 +581,7 @@ __global__ void __launch_bounds__(128, 1) decode_attn_tc_kernel(
     const __half *__restrict__ v_cache, const int *__restrict__ lengths,
     float *__restrict__ part_o, float *__restrict__ part_ml, __nv_bfloat16 *__restrict__ o_hi,
     __nv_bfloat16 *__restrict__ o_lo, int H, int Hkv, int G, int max_seq, int chunk, int nchunk,
-    float scale_log2) {
+    float scale_log2, const uint8_t *__restrict__ next_w, size_t next_w_bytes) {
   constexpr int CPR = DL / 8;                        // 16-byte pieces (8 dims) per row
   constexpr int NSLOT = tc_slots<DL>();
   constexpr int NT = TC_SUB / 32;                    // 8-key n-tiles per warp step
@@ -569,6 +594,16 @@ __global__ void __launch_bounds__(128, 1) decode_attn_tc_kernel(
   const int ch = blockIdx.x, g = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31, gr = lane >> 2, qd = lane & 3;
   pdl_launch_dependents();
+  {
+    // the up-projection weights, which nothing in the step writes, towards L2 for the step's
+    // last kernel (the evict-first cache stream leaves them there); an equal share per CTA
+    const size_t lines = (next_w_bytes + 127) / 128;
+    const size_t ctas = static_cast<size_t>(gridDim.x) * gridDim.y * gridDim.z;
+    const size_t id = (static_cast<size_t>(b) * gridDim.y + g) * gridDim.x + ch;
+    const size_t per = (lines + ctas - 1) / ctas;
+    for (size_t i = id * per + tid; i < min(lines, (id + 1) * per); i += blockDim.x)
+      prefetch_l2(next_w + i * 128);
+  }
   pdl_wait();
   const int L = lengths[b];
   const int s0 = ch * chunk;
@@ -829,10 +864,11 @@ __global__ void __launch_bounds__(64) decode_merge16_kernel(
 }
 
 constexpr int kQkvBlocksPerSm = 1;   // QKV projection blocks per SM (split-K fills the rest)
+constexpr int kQkvCols = 32;         // QKV projection columns per block
 
 int decode_ksplit(const Dims &d) {
   // enough blocks to keep every SM streaming the weight matrix
-  const int nblk = (d.NQKV + 15) / 16;
+  const int nblk = (d.NQKV + kQkvCols - 1) / kQkvCols;
   int ks = (kQkvBlocksPerSm * num_sms() + nblk - 1) / nblk;
   if (ks < 1) ks = 1;
   while (ks > 1 && d.E / ks < 64) --ks;
@@ -897,7 +933,8 @@ static cudaError_t launch_decode_attn(const Dims &d, const DecodeArgs &a, float 
                       a.q_new, static_cast<const __half *>(a.k_cache),
                       static_cast<const __half *>(a.v_cache), a.lengths, a.part_o, a.part_ml,
                       o_hi, o_hi + static_cast<size_t>(d.B) * d.NQ, d.H, d.Hkv, d.G, a.max_seq,
-                      a.chunk, a.nchunk, scale_log2);
+                      a.chunk, a.nchunk, scale_log2, static_cast<const uint8_t *>(a.w_o),
+                      static_cast<size_t>(d.E) * d.NQ * sizeof(TL));
   }
   const int KS = 128 / (DL / 2);
   const size_t smem = 4 * static_cast<size_t>(SUB) * DL * sizeof(TL) +
@@ -917,11 +954,9 @@ static cudaError_t decode_typed(const Dims &d, const DecodeArgs &a, cudaStream_t
   cudaError_t e;
   // D1
   if constexpr (sizeof(T) == 2) {
-    const int kps = ((d.E + a.ksplit - 1) / a.ksplit + SK_KC - 1) / SK_KC * SK_KC;
-    dim3 g1((d.NQKV + 15) / 16, a.ksplit, (d.B + 63) / 64);
-    e = launch_skinny<true, false, 8>(g1, static_cast<const __nv_bfloat16 *>(a.x), nullptr,
-                                      static_cast<const __nv_bfloat16 *>(a.w_qkv), a.p_part, d.B,
-                                      d.NQKV, d.E, kps, nullptr, 0, st);
+    e = launch_skinny<true, false, 8, kQkvCols>(
+        a.ksplit, static_cast<const __nv_bfloat16 *>(a.x), nullptr,
+        static_cast<const __nv_bfloat16 *>(a.w_qkv), a.p_part, d.B, d.NQKV, d.E, nullptr, 0, st);
     if (e != cudaSuccess) return e;
   } else {
     e = gemm_simt(0, a.x, a.w_qkv, a.p_part, d.B, d.NQKV, d.E, st);
@@ -993,10 +1028,9 @@ static cudaError_t decode_typed(const Dims &d, const DecodeArgs &a, cudaStream_t
   // D4 (+ lengths advance for 16-bit layers)
   if constexpr (sizeof(T) == 2) {
     const __nv_bfloat16 *o_hi = static_cast<const __nv_bfloat16 *>(a.o);
-    dim3 g4((d.E + 15) / 16, 1, (d.B + 63) / 64);
-    e = launch_skinny<false, true, 8>(g4, o_hi, o_hi + static_cast<size_t>(d.B) * d.NQ,
-                                      static_cast<const __nv_bfloat16 *>(a.w_o), a.y, d.B, d.E,
-                                      d.NQ, d.NQ, a.lengths, a.max_seq, st);
+    e = launch_skinny<false, true, 8, 16>(1, o_hi, o_hi + static_cast<size_t>(d.B) * d.NQ,
+                                          static_cast<const __nv_bfloat16 *>(a.w_o), a.y, d.B,
+                                          d.E, d.NQ, a.lengths, a.max_seq, st);
     if (e != cudaSuccess) return e;
   } else {
     e = gemm_simt(0, a.o, a.w_o, a.y, d.B, d.E, d.NQ, st);

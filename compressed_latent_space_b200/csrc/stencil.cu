@@ -345,6 +345,265 @@ __global__ void __launch_bounds__(512) stencil_kernel(const StencilParams<T> p) 
   }  // groups
 }
 
+// ------------------------------------------------------------------ persistent 16-bit path
+// One CTA per SM, each bound to one key/value group for its whole life: the group's channel
+// filters (split into bf16 hi / lo pairs) and sequence taps are staged in shared memory once,
+// and the CTA then walks a contiguous run of (sequence, TT-token tile) units, the P rows of the
+// next unit copied in (cp.async, second buffer) while the current one is computed.  Against
+// one CTA per tile walking the groups, the filters cross from L2 once per CTA instead of once
+// per (tile, group, 16-token task), and no unit waits for its own P rows.  The sequence conv is
+// evaluated straight into the MMA's A fragments (each fragment element belongs to one task),
+// so there is no intermediate buffer.  Same arithmetic as the per-tile kernel above.
+constexpr int GT = 32;                  // tokens per unit
+constexpr int kGroupSmemLimit = 220 * 1024;
+
+__host__ __device__ inline int wsp_ld(int DL) { return DL / 2 + 4; }   // uint2 per filter row
+// P row pitch (floats): = 8 mod 16 banks' worth, so the 8 rows x 4 column pairs of an A
+// fragment's float2 reads fall on distinct banks
+__host__ __device__ inline int gps_pitch(int G, int DL) { return (G + 2) * DL + 8; }
+
+struct GroupSmem {                      // byte offsets of the persistent kernel's buffers
+  size_t w, wseq, ps, rt, mq, total;
+};
+__host__ __device__ inline GroupSmem group_smem(int G, int DL, int KC, int halo) {
+  GroupSmem m;
+  m.w = 0;                                                             // [G+1][DL][wsp_ld] uint2
+  m.wseq = m.w + static_cast<size_t>(G + 1) * DL * wsp_ld(DL) * 8;     // [QKC][KC] float
+  m.ps = m.wseq + ((static_cast<size_t>(G + 1) * DL * KC * 4 + 15) / 16) * 16;  // [2][GT+halo][CHP]
+  m.rt = m.ps + static_cast<size_t>(2) * (GT + halo) * gps_pitch(G, DL) * 4;    // [GT][HALF][2]
+  m.mq = m.rt + static_cast<size_t>(GT) * DL * 4;                     // [GT][DL]
+  m.total = m.mq + static_cast<size_t>(GT) * DL * 4;
+  return m;
+}
+
+template <int DL, int KCT>
+__global__ void __launch_bounds__(576, 1) stencil_group_kernel(const StencilParams<__nv_bfloat16> p,
+                                                               int ctas_per_group, int tiles) {
+  using TL = __half;
+  constexpr int HALF = DL / 2;
+  constexpr int NT = DL / 8;
+  constexpr int MT = GT / 16;
+  extern __shared__ __align__(16) uint8_t gsm[];
+  const int G = p.G, QKC = (G + 1) * DL, CH = (G + 2) * DL;
+  const int CHP = gps_pitch(G, DL), WLD = wsp_ld(DL);
+  const int halo = p.halo, KC = p.KC;
+  const int KC1 = KCT ? KCT - 1 : KC - 1;
+  const GroupSmem L = group_smem(G, DL, KC, halo);
+  uint2 *Wsp = reinterpret_cast<uint2 *>(gsm + L.w);
+  float *wseq = reinterpret_cast<float *>(gsm + L.wseq);
+  float *PsBuf = reinterpret_cast<float *>(gsm + L.ps);
+  float *Rt = reinterpret_cast<float *>(gsm + L.rt);   // rotations of the unit's tokens
+  float *Mq = reinterpret_cast<float *>(gsm + L.mq);   // mean of the group's q heads' P rows
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nwarps = blockDim.x >> 5;
+  const int g = blockIdx.x / ctas_per_group, r = blockIdx.x % ctas_per_group;
+  const int units = p.B * tiles;
+  const int u_beg = static_cast<int>(static_cast<long>(units) * r / ctas_per_group);
+  const int u_end = static_cast<int>(static_cast<long>(units) * (r + 1) / ctas_per_group);
+  const int qcol0 = g * G * DL, kcol0 = p.NQ + g * DL, vcol0 = p.NQ + p.NKV + g * DL;
+
+  // the group's filters: heads g*G .. g*G+G-1, then k head H+g; rows padded to WLD uint2
+  for (int i = tid; i < (G + 1) * DL * (HALF / 2); i += blockDim.x) {   // 16-byte pieces
+    const int hh = i / (DL * (HALF / 2)), rem = i % (DL * (HALF / 2));
+    const int row = rem / (HALF / 2), piece = rem % (HALF / 2);
+    const int head = hh < G ? g * G + hh : p.H + g;
+    cp_async16_zfill(Wsp + (hh * DL + row) * WLD + piece * 2,
+                     p.conv_chan_split + (static_cast<size_t>(head) * DL + row) * HALF + piece * 2,
+                     true);
+  }
+  for (int e = tid; e < QKC * KC; e += blockDim.x) {
+    const int c = e / KC, t = e % KC;
+    const int gc = c < G * DL ? qcol0 + c : kcol0 + (c - G * DL);
+    wseq[e] = p.conv_seq[static_cast<size_t>(gc) * KC + t];
+  }
+  auto issue = [&](int u, int buf) {              // P rows of unit u into buffer buf
+    if (u < u_end) {
+      const int b = u / tiles, t0 = (u % tiles) * GT;
+      float *Ps = PsBuf + static_cast<size_t>(buf) * (GT + halo) * CHP;
+      for (int rr = warp; rr < GT + halo; rr += nwarps) {     // a warp per row
+        const int t = t0 - halo + rr;
+        const bool in = t >= 0 && t < p.S;
+        const float *row = p.P + (static_cast<size_t>(b) * p.S + (in ? t : 0)) * p.NQKV;
+        for (int c = lane * 4; c < CH; c += 128) {
+          const int gc = c < G * DL ? qcol0 + c : (c < QKC ? kcol0 + (c - G * DL) : vcol0 + (c - QKC));
+          cp_async16_zfill(Ps + rr * CHP + c, row + gc, in);
+        }
+      }
+    }
+    cp_async_commit();
+  };
+  issue(u_beg, 0);                                  // (the filter copies join this group)
+
+  const int gr = lane >> 2, qc = lane & 3;
+  const int vhalf = p.NKV / 2;
+  for (int u = u_beg, k = 0; u < u_end; ++u, ++k) {
+    const int buf = k & 1;
+    issue(u + 1, buf ^ 1);
+    const int b = u / tiles, t0 = (u % tiles) * GT;
+    if (p.flags & F_ROPE)                           // this unit's rotations
+      for (int i = tid; i < GT * HALF; i += blockDim.x)
+        rope_cos_sin(static_cast<double>(t0 + i / HALF) * p.theta[i % HALF], Rt[2 * i], Rt[2 * i + 1]);
+    asm volatile("cp.async.wait_group 1;" ::: "memory");   // unit u's rows have landed
+    __syncthreads();
+    const float *Ps = PsBuf + static_cast<size_t>(buf) * (GT + halo) * CHP;
+    if (p.flags & F_QK_MEAN) {                      // the k head's share of Q-K-Mean, once
+      for (int i = tid; i < GT * DL; i += blockDim.x) {
+        const float *prow = Ps + (i / DL + halo) * CHP + (i % DL);
+        float m = 0.f;
+        for (int h2 = 0; h2 < G; ++h2) m += prow[h2 * DL];
+        Mq[i] = m / static_cast<float>(G);
+      }
+      __syncthreads();
+    }
+
+    // channel conv tasks: (head, 16 tokens) per warp
+    for (int task = warp; task < (G + 1) * MT; task += nwarps) {
+      const int hh = task / MT, mt = task % MT;
+      const bool is_q = hh < G;
+      const uint2 *wb = Wsp + static_cast<size_t>(hh) * DL * WLD;
+      float acc[NT][4];
+#pragma unroll
+      for (int n = 0; n < NT; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
+      const int tr0 = mt * 16 + gr;                 // fragment rows tr0, tr0 + 8
+#pragma unroll
+      for (int ks = 0; ks < DL / 16; ++ks) {
+        // A = the sequence conv of channels hh*DL + ks*16 + {2qc, 2qc+1, 2qc+8, 2qc+9}
+        float2 av[4];
+#pragma unroll
+        for (int hp = 0; hp < 2; ++hp) {            // column pair 2qc (+0 / +8)
+          const int c = hh * DL + ks * 16 + 2 * qc + hp * 8;
+          const float *w0 = wseq + c * KC, *w1 = w0 + KC;
+#pragma unroll
+          for (int rh = 0; rh < 2; ++rh) {          // row tr0 (+0 / +8)
+            const int rbase = tr0 + rh * 8 + halo - KC1;   // Ps row of the first tap
+            float x = 0.f, y = 0.f;
+            if constexpr (KCT != 0) {
+#pragma unroll
+              for (int j = 0; j < KCT; ++j) {
+                const float2 pv = *reinterpret_cast<const float2 *>(Ps + (rbase + j) * CHP + c);
+                x = fmaf(w0[j], pv.x, x);
+                y = fmaf(w1[j], pv.y, y);
+              }
+            } else {
+              for (int j = 0; j <= KC1; ++j) {
+                const float2 pv = *reinterpret_cast<const float2 *>(Ps + (rbase + j) * CHP + c);
+                x = fmaf(w0[j], pv.x, x);
+                y = fmaf(w1[j], pv.y, y);
+              }
+            }
+            av[hp * 2 + rh] = make_float2(x, y);
+          }
+        }
+        uint32_t ah[4], al[4];                      // a0: (r, k), a1: (r+8, k), a2: (r, k+8), a3
+        split_bf16x2(av[0], ah[0], al[0]);
+        split_bf16x2(av[1], ah[1], al[1]);
+        split_bf16x2(av[2], ah[2], al[2]);
+        split_bf16x2(av[3], ah[3], al[3]);
+        const int k0 = ks * 16 + 2 * qc;
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+          const uint2 *wr = wb + (n * 8 + gr) * WLD + k0 / 2;
+          const uint2 w0 = wr[0], w1 = wr[4];
+          const uint32_t bh[2] = {w0.x, w1.x}, bl[2] = {w0.y, w1.y};
+          mma_bf16_16816(acc[n], ah, bh);
+          mma_bf16_16816(acc[n], ah, bl);
+          mma_bf16_16816(acc[n], al, bh);
+        }
+      }
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int tt = tr0 + half * 8;
+        const float *prow = Ps + (tt + halo) * CHP;
+        float uv[NT][2];
+#pragma unroll
+        for (int n = 0; n < NT; ++n)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int i = n * 8 + 2 * qc + e;
+            float v = acc[n][half * 2 + e];
+            if (p.flags & F_QK_MEAN)
+              v += 0.5f * ((is_q ? prow[hh * DL + i] : Mq[tt * DL + i]) + prow[G * DL + i]);
+            uv[n][e] = v;
+          }
+        if (p.flags & F_QK_NORM) {
+          float ss = 0.f;
+#pragma unroll
+          for (int n = 0; n < NT; ++n) ss += uv[n][0] * uv[n][0] + uv[n][1] * uv[n][1];
+          ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+          ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+          const float inv = 1.0f / sqrtf(ss / static_cast<float>(DL) + p.eps);
+#pragma unroll
+          for (int n = 0; n < NT; ++n) {
+            uv[n][0] *= inv;
+            uv[n][1] *= inv;
+          }
+        }
+        if (p.flags & F_ROPE) {
+#pragma unroll
+          for (int n = 0; n < NT / 2; ++n)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int i = n * 8 + 2 * qc + e;      // < d~/2; partner i + d~/2 is n-tile n+NT/2
+              const float c = Rt[(tt * HALF + i) * 2], sn = Rt[(tt * HALF + i) * 2 + 1];
+              const float x1 = uv[n][e], x2 = uv[n + NT / 2][e];
+              uv[n][e] = x1 * c - x2 * sn;
+              uv[n + NT / 2][e] = x1 * sn + x2 * c;
+            }
+        }
+        const int t = t0 + tt;
+        if (t < p.S) {
+          TL *dst = is_q ? p.q + ((static_cast<size_t>(b) * p.H + g * G + hh) * p.S + t) * DL
+                         : p.k + ((static_cast<size_t>(b) * p.Hkv + g) * p.kv_stride + t) * DL;
+          bool fits = true;                            // every value within the float16 range
+#pragma unroll
+          for (int n = 0; n < NT; ++n) {
+            fits &= fabsf(uv[n][0]) <= kF16Max && fabsf(uv[n][1]) <= kF16Max;
+            *reinterpret_cast<uint32_t *>(dst + n * 8 + 2 * qc) = pack_f16x2(uv[n][0], uv[n][1]);
+          }
+          if (!fits) report(p.status, DEV_RANGE);
+        }
+      }
+    }
+
+    // values with the value-shift: upper half of the value channels from token t-1
+    for (int i = tid; i < GT * HALF; i += blockDim.x) {
+      const int tt = i / HALF, c = (i % HALF) * 2;
+      const int t = t0 + tt;
+      if (t >= p.S) continue;
+      float val[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const bool shifted = (p.flags & F_VALUE_SHIFT) && (g * DL + c + e >= vhalf);
+        val[e] = Ps[(tt + halo - (shifted ? 1 : 0)) * CHP + QKC + c + e];
+      }
+      if (!(fabsf(val[0]) <= kF16Max && fabsf(val[1]) <= kF16Max)) report(p.status, DEV_RANGE);
+      *reinterpret_cast<uint32_t *>(
+          p.v + ((static_cast<size_t>(b) * p.Hkv + g) * p.kv_stride + t) * DL + c) =
+          pack_f16x2(val[0], val[1]);
+    }
+
+    // decode state after the sequence's last token, by the unit that holds it
+    if (p.write_state && t0 <= p.S - 1 && p.S - 1 < t0 + GT) {
+      const int W = p.NQ + p.NKV;
+      for (int i = tid; i < KC1 * QKC; i += blockDim.x) {
+        const int j = i / QKC, c = i % QKC;
+        const int rr = p.S - KC1 + j - t0 + halo;
+        const int gc = c < G * DL ? qcol0 + c : kcol0 + (c - G * DL);
+        p.conv_state[(static_cast<size_t>(b) * KC1 + j) * W + gc] = Ps[rr * CHP + c];
+      }
+      const int rl = p.S - 1 - t0 + halo;
+      for (int c = tid; c < DL; c += blockDim.x) {
+        const int gch = g * DL + c;
+        if (gch >= vhalf)
+          p.vshift_state[static_cast<size_t>(b) * (p.NKV - vhalf) + (gch - vhalf)] =
+              Ps[rl * CHP + QKC + c];
+      }
+      if (g == 0 && tid == 0) p.lengths[b] = p.S;
+    }
+    __syncthreads();                                // buffer buf and Rt are rewritten next
+  }
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+}
+
 constexpr int kTensorSmemKB = 110;   // staging budget per CTA of the 16-bit path
 
 template <typename T, int DL>
@@ -372,6 +631,25 @@ cudaError_t launch(const Dims &d, const StencilArgs &a, cudaStream_t st) {
   p.eps = d.eps;
   for (int i = 0; i < DL / 2; ++i)
     p.theta[i] = pow(static_cast<double>(d.rope_base), -2.0 * i / DL);
+  if constexpr (!simt) {
+    const GroupSmem gs = group_smem(d.G, DL, d.KC, p.halo);
+    const int warps = (d.G + 1) * (GT / 16);
+    if (gs.total <= static_cast<size_t>(kGroupSmemLimit) && warps <= 18) {
+      const int tiles = (d.S + GT - 1) / GT;
+      const int units = d.B * tiles;
+      int cpg = num_sms() / d.Hkv;                   // CTAs per group: one per SM in all
+      if (cpg < 1) cpg = 1;
+      if (cpg > units) cpg = units;
+      p.TT = GT;
+      cudaError_t e = d.KC == 4 ? ensure_dyn_smem<stencil_group_kernel<DL, 4>>(gs.total)
+                                : ensure_dyn_smem<stencil_group_kernel<DL, 0>>(gs.total);
+      if (e != cudaSuccess) return e;
+      const dim3 grid(d.Hkv * cpg), block(32 * (warps < 4 ? 4 : warps));
+      if (d.KC == 4) stencil_group_kernel<DL, 4><<<grid, block, gs.total, st>>>(p, cpg, tiles);
+      else stencil_group_kernel<DL, 0><<<grid, block, gs.total, st>>>(p, cpg, tiles);
+      return cudaGetLastError();
+    }
+  }
   // Largest token tile (a multiple of 16) whose staging fits two CTAs per SM.
   const size_t budget = (simt ? 72 : kTensorSmemKB) * 1024;
   int TT = 64;
