@@ -376,9 +376,11 @@ __host__ __device__ inline GroupSmem group_smem(int G, int DL, int KC, int halo)
   return m;
 }
 
-template <int DL, int KCT>
-__global__ void __launch_bounds__(576, 1) stencil_group_kernel(const StencilParams<__nv_bfloat16> p,
-                                                               int ctas_per_group, int tiles) {
+// MAXW: the most warps a launch uses ((G + 1) * GT / 16); a smaller bound leaves each thread
+// more registers.
+template <int DL, int KCT, int MAXW>
+__global__ void __launch_bounds__(32 * MAXW, 1) stencil_group_kernel(
+    const StencilParams<__nv_bfloat16> p, int ctas_per_group, int tiles) {
   using TL = __half;
   constexpr int HALF = DL / 2;
   constexpr int NT = DL / 8;
@@ -641,13 +643,22 @@ cudaError_t launch(const Dims &d, const StencilArgs &a, cudaStream_t st) {
       if (cpg < 1) cpg = 1;
       if (cpg > units) cpg = units;
       p.TT = GT;
-      cudaError_t e = d.KC == 4 ? ensure_dyn_smem<stencil_group_kernel<DL, 4>>(gs.total)
-                                : ensure_dyn_smem<stencil_group_kernel<DL, 0>>(gs.total);
-      if (e != cudaSuccess) return e;
       const dim3 grid(d.Hkv * cpg), block(32 * (warps < 4 ? 4 : warps));
-      if (d.KC == 4) stencil_group_kernel<DL, 4><<<grid, block, gs.total, st>>>(p, cpg, tiles);
-      else stencil_group_kernel<DL, 0><<<grid, block, gs.total, st>>>(p, cpg, tiles);
-      return cudaGetLastError();
+      auto go = [&](auto kernel) -> cudaError_t {
+        kernel<<<grid, block, gs.total, st>>>(p, cpg, tiles);
+        return cudaGetLastError();
+      };
+      cudaError_t e;
+      if (warps <= 12) {
+        e = d.KC == 4 ? ensure_dyn_smem<stencil_group_kernel<DL, 4, 12>>(gs.total)
+                      : ensure_dyn_smem<stencil_group_kernel<DL, 0, 12>>(gs.total);
+        if (e != cudaSuccess) return e;
+        return d.KC == 4 ? go(stencil_group_kernel<DL, 4, 12>) : go(stencil_group_kernel<DL, 0, 12>);
+      }
+      e = d.KC == 4 ? ensure_dyn_smem<stencil_group_kernel<DL, 4, 18>>(gs.total)
+                    : ensure_dyn_smem<stencil_group_kernel<DL, 0, 18>>(gs.total);
+      if (e != cudaSuccess) return e;
+      return d.KC == 4 ? go(stencil_group_kernel<DL, 4, 18>) : go(stencil_group_kernel<DL, 0, 18>);
     }
   }
   // Largest token tile (a multiple of 16) whose staging fits two CTAs per SM.
