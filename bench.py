@@ -215,12 +215,12 @@ def bench_prefill(cls, w, steps, warmup, world, seed):
 DECODE_LAYERS = 32
 
 
-def decode_launches(w):
-    """Kernels one 16-bit decode step launches: QKV projection, stencil, attention, output
-    projection, and the merge of the attention's key splits when the (sequence, group) pairs
-    are fewer than the SMs (the library splits the keys only then)."""
-    sms = torch.cuda.get_device_properties(0).multi_processor_count
-    return 4 + (1 if w.batch * w.n_kv_heads < sms else 0)
+def decode_launches(cls, layer, batch, max_seq):
+    """Kernels one decode step launches, as the library reports them for this shape."""
+    n = cls.cca_decode_kernel_count(layer.cfg, batch, max_seq)
+    if n <= 0:
+        raise RuntimeError(cls.cca_last_error_string())
+    return n
 
 
 def bench_decode(cls, w, steps, warmup, seed, layers=DECODE_LAYERS):
@@ -268,7 +268,7 @@ def bench_decode(cls, w, steps, warmup, seed, layers=DECODE_LAYERS):
         cls.cca_cache_check(cache.struct)
     names = ["qkv_projection", "stencil_append", "split_kv_attention", "merge", "out_projection"]
     return dict(ms=ms, stages={n: t / max(calls, 1) for n, t in zip(names, stage_ms)},
-                launches=decode_launches(w) * steps, layers=layers)
+                launches=decode_launches(cls, stack[0][0], w.batch, max_seq) * steps, layers=layers)
 
 
 def cpu_oracle_sample(w, budget_s=12.0, seed=0):

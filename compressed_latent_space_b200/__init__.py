@@ -59,6 +59,7 @@ _SIGS = {
                                 POINTER(cca_cache_t), c_void_p]),
     "cca_prefill_workspace_size": (c_size_t, [POINTER(cca_config_t), c_int, c_int]),
     "cca_decode_workspace_size": (c_size_t, [POINTER(cca_config_t), c_int, c_int]),
+    "cca_decode_kernel_count": (c_int, [POINTER(cca_config_t), c_int, c_int]),
     "cca_prefill_forward": (c_int, [POINTER(cca_config_t), POINTER(cca_weights_t), c_void_p, c_int,
                                     c_int, c_void_p, POINTER(cca_cache_t), c_void_p, c_size_t,
                                     c_void_p]),
@@ -140,6 +141,10 @@ def cca_prefill_workspace_size(cfg: cca_config_t, batch: int, seq: int) -> int:
 
 def cca_decode_workspace_size(cfg: cca_config_t, batch: int, max_seq: int) -> int:
     return load().cca_decode_workspace_size(ctypes.byref(cfg), batch, max_seq)
+
+
+def cca_decode_kernel_count(cfg: cca_config_t, batch: int, max_seq: int) -> int:
+    return load().cca_decode_kernel_count(ctypes.byref(cfg), batch, max_seq)
 
 
 def cca_cache_alloc(cfg: cca_config_t, batch: int, max_seq: int, buf=None, stream=None):

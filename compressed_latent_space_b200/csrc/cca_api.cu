@@ -287,6 +287,15 @@ CCA_API size_t cca_decode_workspace_size(const cca_config_t *cfg, int batch, int
   return cca::decode_workspace_bytes(d, max_seq);
 }
 
+CCA_API int cca_decode_kernel_count(const cca_config_t *cfg, int batch, int max_seq) {
+  cca::Dims d;
+  int rc = make_dims(cfg, d);
+  if (rc) return rc;
+  if (batch <= 0 || max_seq <= 0) return fail(CCA_ERR_INVALID_ARG, "batch and max_seq must be positive");
+  d.B = batch;
+  return cca::decode_kernel_count(d, max_seq);
+}
+
 CCA_API int cca_prefill_forward(const cca_config_t *cfg, const cca_weights_t *w, const void *x,
                                 int batch, int seq, void *y, cca_cache_t *cache,
                                 void *workspace, size_t ws_bytes, void *stream) {

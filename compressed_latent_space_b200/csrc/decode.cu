@@ -212,38 +212,43 @@ __host__ __device__ inline size_t d2_smem_floats(int G, int DL, int KC) {
          + CH + 2 * QKC + 16;                   // pn, av, uv, inv
 }
 
+// D2's shared-memory carve ([wt | wseq | old | pn | a | u | inv], floats)
+template <int DL>
+struct D2Smem {
+  float *wt, *wseq, *old, *pn, *a, *u, *inv;
+  __device__ D2Smem(float *sm, int G, int KC) {
+    const int QKC = (G + 1) * DL, CH = (G + 2) * DL;
+    wt = sm;
+    wseq = wt + DL * d2_ld(QKC);
+    old = wseq + QKC * KC;                           // [KC-1][QKC] conv state before the step
+    pn = old + QKC * (KC - 1);
+    a = pn + CH;
+    u = a + QKC;
+    inv = u + QKC;
+  }
+};
+
+// Before the grid-dependency wait: the group's filters into shared memory (no __syncthreads),
+// the sequence's conv state towards L2.
 template <typename T, int DL>
-__global__ void __launch_bounds__(256) decode_stencil_kernel(const D2Params<T> p) {
-  using TL = typename D2Params<T>::TL;
-  extern __shared__ __align__(16) float sm[];
-  const int g = blockIdx.x, b = blockIdx.y, tid = threadIdx.x, nt = blockDim.x;
-  const int G = p.G, CH = (G + 2) * DL, QKC = (G + 1) * DL, KC = p.KC, KC1 = KC - 1;
+__device__ __forceinline__ void d2_stage(const D2Params<T> &p, int g, int b, const D2Smem<DL> &m) {
+  const int tid = threadIdx.x, nt = blockDim.x;
+  const int G = p.G, QKC = (G + 1) * DL, KC = p.KC, KC1 = KC - 1;
   const int LD = d2_ld(QKC);
-  float *wt = sm;
-  float *wseq = wt + DL * LD;
-  float *old = wseq + QKC * KC;                      // [KC-1][QKC] conv state before the step
-  float *pn = old + QKC * KC1;
-  float *a = pn + CH;
-  float *u = a + QKC;
-  float *inv = u + QKC;
-  pdl_launch_dependents();
   // filters: q heads g*G.., then k head H+g; W_head[i][j] -> wt[j][head * DL + i]
   for (int e = tid; e < (G + 1) * DL * DL; e += nt) {
     const int hh = e / (DL * DL), r = e % (DL * DL), i = r / DL, j = r % DL;
     const int head = hh < G ? g * G + hh : p.H + g;
-    wt[j * LD + hh * DL + i] = p.conv_chan[static_cast<size_t>(head) * DL * DL + r];
+    m.wt[j * LD + hh * DL + i] = p.conv_chan[static_cast<size_t>(head) * DL * DL + r];
   }
+  const int qcol0 = g * G * DL, kcol0 = p.NQ + g * DL;
   for (int e = tid; e < QKC * KC; e += nt) {
     const int c = e / KC, t = e % KC;
-    const int gc = c < G * DL ? g * G * DL + c : p.NQ + g * DL + (c - G * DL);
-    wseq[e] = p.conv_seq[static_cast<size_t>(gc) * KC + t];
+    const int gc = c < G * DL ? qcol0 + c : kcol0 + (c - G * DL);
+    m.wseq[e] = p.conv_seq[static_cast<size_t>(gc) * KC + t];
   }
-  const int qcol0 = g * G * DL, kcol0 = p.NQ + g * DL, vcol0 = p.NQ + p.NKV + g * DL;
-  auto gch = [&](int c) {
-    return c < G * DL ? qcol0 + c : (c < QKC ? kcol0 + (c - G * DL) : vcol0 + (c - QKC));
-  };
   const int W = p.NQ + p.NKV;
-  float *cs = p.conv_state + static_cast<size_t>(b) * KC1 * W;
+  const float *cs = p.conv_state + static_cast<size_t>(b) * KC1 * W;
   for (int e = tid; e < KC1 * (G + 1); e += nt) {   // the state rows of this group's channels
     const int j = e / (G + 1), part = e % (G + 1);  // (G q heads' DL run is contiguous)
     const float *row = cs + static_cast<size_t>(j) * W;
@@ -251,81 +256,96 @@ __global__ void __launch_bounds__(256) decode_stencil_kernel(const D2Params<T> p
     const int len = part == 0 ? G * DL : DL;
     for (int off = 0; off < len; off += 32) prefetch_l2(seg + off);
   }
-  __syncthreads();                                   // staged filters visible to every thread
-  pdl_wait();
-  // the token's projections (sum of the split-K partials) and the old conv state, loaded
-  // together before the position is known
+}
+
+// After the wait: the token's projections (sum of the split-K partials) and the old conv
+// state into shared memory, thread c taking channel c (the compute below keeps that mapping).
+template <typename T, int DL>
+__device__ __forceinline__ void d2_load(const D2Params<T> &p, int g, int b, const D2Smem<DL> &m) {
+  const int tid = threadIdx.x, nt = blockDim.x;
+  const int G = p.G, CH = (G + 2) * DL, QKC = (G + 1) * DL, KC1 = p.KC - 1;
+  const int qcol0 = g * G * DL, kcol0 = p.NQ + g * DL, vcol0 = p.NQ + p.NKV + g * DL;
+  const int W = p.NQ + p.NKV;
+  const float *cs = p.conv_state + static_cast<size_t>(b) * KC1 * W;
   for (int c = tid; c < CH; c += nt) {
-    const int gc = gch(c);
+    const int gc = c < G * DL ? qcol0 + c : (c < QKC ? kcol0 + (c - G * DL) : vcol0 + (c - QKC));
     float v = 0.f;
     for (int ks = 0; ks < p.ksplit; ++ks) v += p.p_part[(static_cast<size_t>(ks) * p.B + b) * p.NQKV + gc];
-    pn[c] = v;
+    m.pn[c] = v;
     if (c < QKC)
-      for (int j = 0; j < KC1; ++j) old[j * QKC + c] = cs[static_cast<size_t>(j) * W + gc];
+      for (int j = 0; j < KC1; ++j) m.old[j * QKC + c] = cs[static_cast<size_t>(j) * W + gc];
   }
-  const int L = p.lengths[b];
-  if (L >= p.max_seq) {
-    if (tid == 0) report(p.status, DEV_CACHE_FULL);
-    return;
-  }
+}
+
+// The stencil of the new token at position L (< max_seq): k and v rows appended to the cache,
+// the G query heads' rotated latents to q (head hh at q + hh * DL; global or shared memory),
+// conv / value-shift state advanced.  Every thread of the block takes part (__syncthreads).
+template <typename T, int DL>
+__device__ __forceinline__ void d2_compute(const D2Params<T> &p, int g, int b, int L,
+                                           const D2Smem<DL> &m, float *q) {
+  using TL = typename D2Params<T>::TL;
+  const int tid = threadIdx.x, nt = blockDim.x;
+  const int G = p.G, QKC = (G + 1) * DL, KC = p.KC, KC1 = KC - 1;
+  const int LD = d2_ld(QKC);
+  const int qcol0 = g * G * DL, kcol0 = p.NQ + g * DL;
+  const int W = p.NQ + p.NKV;
+  float *cs = p.conv_state + static_cast<size_t>(b) * KC1 * W;
   constexpr int HALF = DL / 2;
   float rc = 1.f, rs = 0.f;                          // RoPE rotation of this thread's pairs
   if ((p.flags & F_ROPE) && tid < (G + 1) * HALF)
     rope_cos_sin(static_cast<double>(L) * p.theta[tid % HALF], rc, rs);
   // the sequence conv of the q|k channels (each thread reads only what it loaded)
   for (int c = tid; c < QKC; c += nt) {
-    const float *w = wseq + c * KC;
+    const float *w = m.wseq + c * KC;
     float acc = 0.f;
-    for (int j = 0; j < KC1; ++j) acc = fmaf(w[j], old[j * QKC + c], acc);
-    a[c] = fmaf(w[KC1], pn[c], acc);
+    for (int j = 0; j < KC1; ++j) acc = fmaf(w[j], m.old[j * QKC + c], acc);
+    m.a[c] = fmaf(w[KC1], m.pn[c], acc);
   }
   __syncthreads();
   // channel conv (thread per output) and q-k-mean
   for (int o = tid; o < QKC; o += nt) {
     const int hh = o / DL, i = o % DL;
-    const float *ah = a + hh * DL;
+    const float *ah = m.a + hh * DL;
     float acc = 0.f;
 #pragma unroll 8
-    for (int j = 0; j < DL; ++j) acc = fmaf(wt[j * LD + o], ah[j], acc);
+    for (int j = 0; j < DL; ++j) acc = fmaf(m.wt[j * LD + o], ah[j], acc);
     if (p.flags & F_QK_MEAN) {
-      const float pk = pn[G * DL + i];
+      const float pk = m.pn[G * DL + i];
       if (hh < G) {
-        acc += 0.5f * (pn[o] + pk);
+        acc += 0.5f * (m.pn[o] + pk);
       } else {
         float mq = 0.f;
-        for (int h2 = 0; h2 < G; ++h2) mq += pn[h2 * DL + i];
+        for (int h2 = 0; h2 < G; ++h2) mq += m.pn[h2 * DL + i];
         acc += 0.5f * (mq / static_cast<float>(G) + pk);
       }
     }
-    u[o] = acc;
+    m.u[o] = acc;
   }
   __syncthreads();
   // RMS norm per head: one warp per head
   const int warp = tid >> 5, lane = tid & 31;
   for (int hh = warp; hh <= G; hh += nt / 32) {
     float ss = 0.f;
-    for (int i = lane; i < DL; i += 32) ss += u[hh * DL + i] * u[hh * DL + i];
+    for (int i = lane; i < DL; i += 32) ss += m.u[hh * DL + i] * m.u[hh * DL + i];
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
     if (lane == 0)
-      inv[hh] = (p.flags & F_QK_NORM) ? 1.0f / sqrtf(ss / static_cast<float>(DL) + p.eps) : 1.0f;
+      m.inv[hh] = (p.flags & F_QK_NORM) ? 1.0f / sqrtf(ss / static_cast<float>(DL) + p.eps) : 1.0f;
   }
   __syncthreads();
-  // RoPE at position L on (i, i + DL/2) pairs, then store q (workspace) and k (cache); every
-  // pair a thread takes has i = tid mod DL/2 (DL/2 divides the block size), whose rotation it
-  // computed above
+  // RoPE at position L on (i, i + DL/2) pairs, then store q and k (cache); every pair a thread
+  // takes has i = tid mod DL/2 (DL/2 divides the block size), whose rotation it computed above
   for (int o = tid; o < (G + 1) * HALF; o += nt) {
     const int hh = o / HALF, ip = o % HALF;
-    float x1 = u[hh * DL + ip] * inv[hh], x2 = u[hh * DL + ip + HALF] * inv[hh];
+    float x1 = m.u[hh * DL + ip] * m.inv[hh], x2 = m.u[hh * DL + ip + HALF] * m.inv[hh];
     if (p.flags & F_ROPE) {
       const float y1 = x1 * rc - x2 * rs, y2 = x1 * rs + x2 * rc;
       x1 = y1;
       x2 = y2;
     }
     if (hh < G) {
-      float *qd = p.q_new + (static_cast<size_t>(b) * p.H + g * G + hh) * DL;
-      qd[ip] = x1;
-      qd[ip + HALF] = x2;
+      q[hh * DL + ip] = x1;
+      q[hh * DL + ip + HALF] = x2;
     } else {
       auto *kd = p.k_cache + ((static_cast<size_t>(b) * p.Hkv + g) * p.max_seq + L) * DL;
       check_latent<TL>(x1, p.status);
@@ -340,19 +360,38 @@ __global__ void __launch_bounds__(256) decode_stencil_kernel(const D2Params<T> p
   for (int c = tid; c < DL; c += nt) {
     const int vc = g * DL + c;
     const bool shifted = vc >= vhalf;
-    const float val = ((p.flags & F_VALUE_SHIFT) && shifted) ? vs[vc - vhalf] : pn[QKC + c];
+    const float val = ((p.flags & F_VALUE_SHIFT) && shifted) ? vs[vc - vhalf] : m.pn[QKC + c];
     check_latent<TL>(val, p.status);
     p.v_cache[((static_cast<size_t>(b) * p.Hkv + g) * p.max_seq + L) * DL + c] = from_f32<TL>(val);
   }
+  // state advance (thread c rewrites only channel c's state, which it alone read)
   for (int c = tid; c < QKC; c += nt) {
-    const int gc = gch(c);
-    for (int j = 0; j + 1 < KC1; ++j) cs[static_cast<size_t>(j) * W + gc] = old[(j + 1) * QKC + c];
-    if (KC1 > 0) cs[static_cast<size_t>(KC1 - 1) * W + gc] = pn[c];
+    const int gc = c < G * DL ? qcol0 + c : kcol0 + (c - G * DL);
+    for (int j = 0; j + 1 < KC1; ++j) cs[static_cast<size_t>(j) * W + gc] = m.old[(j + 1) * QKC + c];
+    if (KC1 > 0) cs[static_cast<size_t>(KC1 - 1) * W + gc] = m.pn[c];
   }
   for (int c = tid; c < DL; c += nt) {
     const int vc = g * DL + c;
-    if (vc >= vhalf) vs[vc - vhalf] = pn[QKC + c];
+    if (vc >= vhalf) vs[vc - vhalf] = m.pn[QKC + c];
   }
+}
+
+template <typename T, int DL>
+__global__ void __launch_bounds__(256) decode_stencil_kernel(const D2Params<T> p) {
+  extern __shared__ __align__(16) float sm[];
+  const int g = blockIdx.x, b = blockIdx.y;
+  const D2Smem<DL> m(sm, p.G, p.KC);
+  pdl_launch_dependents();
+  d2_stage(p, g, b, m);
+  __syncthreads();                                   // staged filters visible to every thread
+  pdl_wait();
+  d2_load(p, g, b, m);                               // loads in flight before the position
+  const int L = p.lengths[b];
+  if (L >= p.max_seq) {
+    if (threadIdx.x == 0) report(p.status, DEV_CACHE_FULL);
+    return;
+  }
+  d2_compute(p, g, b, L, m, p.q_new + (static_cast<size_t>(b) * p.H + g * p.G) * DL);
 }
 
 // ------------------------------------------------------------------ D3 split-KV attention
@@ -586,11 +625,11 @@ __global__ void __launch_bounds__(128, 1) decode_attn_tc_kernel(
   constexpr int NSLOT = tc_slots<DL>();
   constexpr int NT = TC_SUB / 32;                    // 8-key n-tiles per warp step
   constexpr int WK = NT * 8;                         // keys per warp per sub-chunk
+  constexpr int SLOT = 2 * TC_SUB * DL;              // halves per slot: [K | V]
   static_assert(4 * WK == TC_SUB && NT % 2 == 0, "four warps cover a sub-chunk");
   extern __shared__ __align__(16) uint8_t smraw[];
-  __half *Kb = reinterpret_cast<__half *>(smraw);    // [NSLOT][TC_SUB][DL], swizzled pieces
-  __half *Vb = Kb + NSLOT * TC_SUB * DL;             // [NSLOT][TC_SUB][DL], swizzled pieces
-  float *wst = reinterpret_cast<float *>(Vb + NSLOT * TC_SUB * DL);  // [4][8 heads][DL + 2]
+  __half *ring = reinterpret_cast<__half *>(smraw);  // [NSLOT][K, V][TC_SUB][DL], swizzled
+  float *wst = reinterpret_cast<float *>(ring + NSLOT * SLOT);     // [4][8 heads][DL + 2]
   const int ch = blockIdx.x, g = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31, gr = lane >> 2, qd = lane & 3;
   pdl_launch_dependents();
@@ -632,7 +671,7 @@ __global__ void __launch_bounds__(128, 1) decode_attn_tc_kernel(
   auto issue = [&](int sbi) {                        // sub-chunk sbi into slot sbi % NSLOT;
     if (sbi < nsub) {                                // an empty group past the last one
       const int base = sbi * TC_SUB, cnt = min(TC_SUB, n - base);  // rows past cnt: zeros
-      __half *kd = Kb + (sbi % NSLOT) * TC_SUB * DL, *vd = Vb + (sbi % NSLOT) * TC_SUB * DL;
+      __half *kd = ring + (sbi % NSLOT) * SLOT, *vd = kd + TC_SUB * DL;
       for (int i = tid; i < TC_SUB * CPR; i += blockDim.x) {
         const int r = i / CPR, j = i % CPR;
         const bool ok = r < cnt;
@@ -673,8 +712,8 @@ __global__ void __launch_bounds__(128, 1) decode_attn_tc_kernel(
     cp_async_wait_group<NSLOT - 2>();                // sub-chunk sbi has landed
     __syncthreads();                                 // ... for every thread; and every warp
     issue(sbi + NSLOT - 1);                          // is done with the slot refilled here
-    const uint32_t ks_base = smem_u32(Kb + (sbi % NSLOT) * TC_SUB * DL);
-    const uint32_t vs_base = smem_u32(Vb + (sbi % NSLOT) * TC_SUB * DL);
+    const uint32_t ks_base = smem_u32(ring + (sbi % NSLOT) * SLOT);
+    const uint32_t vs_base = ks_base + TC_SUB * DL * 2;
     const int kb = warp * WK;                        // this warp's first key in the sub-chunk
     const int valid = n - sbi * TC_SUB - kb;         // keys of this warp's slice that exist
     if (valid > 0) {
@@ -888,6 +927,14 @@ int decode_chunk(const Dims &d, int max_seq) {
   const long nsplit = (num_sms() + units - 1) / units;
   const long per = (max_seq + nsplit - 1) / nsplit;
   return static_cast<int>((per + TC_SUB - 1) / TC_SUB * TC_SUB);
+}
+
+// projection, stencil, attention, output projection, and the merge of the attention's key
+// splits (16-bit layers merge only when they split; float32 layers always run it)
+int decode_kernel_count(const Dims &d, int max_seq) {
+  const int chunk = decode_chunk(d, max_seq);
+  const int nchunk = (max_seq + chunk - 1) / chunk;
+  return d.bf16 && nchunk == 1 ? 4 : 5;
 }
 
 size_t decode_workspace_bytes(const Dims &d, int max_seq) {

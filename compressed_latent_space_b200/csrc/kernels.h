@@ -99,6 +99,7 @@ struct DecodeArgs {
   int chunk;
 };
 size_t decode_workspace_bytes(const Dims &d, int max_seq);
+int decode_kernel_count(const Dims &d, int max_seq);
 void decode_workspace_carve(const Dims &d, int max_seq, void *ws, DecodeArgs &a);
 cudaError_t decode_step(const Dims &d, const DecodeArgs &a, cudaStream_t st,
                         const StageMarker &mark);

@@ -134,6 +134,11 @@ CCA_API size_t cca_prefill_workspace_size(const cca_config_t *cfg, int batch, in
 /* Scratch bytes needed by cca_decode_step for a cache of this shape (0 if invalid). */
 CCA_API size_t cca_decode_workspace_size(const cca_config_t *cfg, int batch, int max_seq);
 
+/* Kernels one cca_decode_step launches for a cache of this shape, on the current device
+ * (the split of the attention's keys depends on its SM count); for launch accounting and
+ * profiling.  (Not in the paper.)  Negative CCA_ERR_* code if the config is invalid. */
+CCA_API int cca_decode_kernel_count(const cca_config_t *cfg, int batch, int max_seq);
+
 /* Full layer forward of `batch` sequences of `seq` tokens each, from position 0.
  *   x [batch, seq, E] -> y [batch, seq, E]   (x and y must not overlap)
  * cache == NULL: keys/values live in the workspace only.  Otherwise (cache->batch ==
