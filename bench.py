@@ -347,7 +347,7 @@ def run_decode_only(args):
     cls.load()
     hbm, _, _, peak_src = measured_peaks()
     dw = W.WORKLOADS[DECODE_WORKLOAD]
-    dec = bench_decode(cls, dw, args.steps, args.warmup, seed=0)
+    dec = bench_decode(cls, dw, args.steps, args.warmup, seed=0, layers=args.decode_layers)
     gbs = decode_bytes(dw) / (dec["ms"] * 1e-3) / 1e9
     print(json.dumps({"metric": "decode GB/s", "value": gbs, "unit": "GB/s",
                       "ms_per_step": dec["ms"], "frac_of_hbm": gbs / hbm, "peak_source": peak_src,
@@ -366,7 +366,8 @@ def run_cuda(args):
         dec = None
         if not args.no_decode:
             dw = W.WORKLOADS[DECODE_WORKLOAD]
-            dec = bench_decode(cls, dw, args.steps, args.warmup, seed=rank)
+            dec = bench_decode(cls, dw, args.steps, args.warmup, seed=rank,
+                               layers=args.decode_layers)
     ms = max_over_ranks(pre["ms"], world)
     e2e_ms = max_over_ranks(pre["e2e_ms"], world)
     tokens = w.batch * w.seq
@@ -461,6 +462,9 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.WORKLOADS))
     ap.add_argument("--impl", default="cca", choices=["cca", "reference"])
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--decode-layers", type=int, default=DECODE_LAYERS,
+                    help="independent layers the decode steps rotate over (fewer for profiling "
+                         "captures that must stay small; the timing needs the default)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--decode-only", action="store_true",
                     help="time only the decode step (a profiling case for its kernels)")
