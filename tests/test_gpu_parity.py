@@ -67,12 +67,17 @@ def test_gemm_f32_simt(cuda_lib, M, N, K):
     assert_fp32_close(f64(C), (A.double() @ B.double().T).numpy())
 
 
+# Shapes cover d~ = 16 / 32 / 64, G = 1..8, token counts off the 32-token unit, sequence-conv
+# widths other than 4 (the generic-tap code paths; width 1 has no halo of its own), and G = 8 at
+# d~ = 64, whose filters and P tiles do not fit the persistent kernel (the per-tile fallback).
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-@pytest.mark.parametrize("H,Hkv,C,E,S", [(4, 4, 4, 256, 130), (8, 2, 2, 512, 77), (6, 3, 1, 96, 65),
-                                         (4, 1, 2, 512, 33)])
-def test_stencil_matches_oracle(cuda_lib, dtype, H, Hkv, C, E, S):
+@pytest.mark.parametrize("H,Hkv,C,E,S,KC", [(4, 4, 4, 256, 130, 4), (8, 2, 2, 512, 77, 4),
+                                            (6, 3, 1, 96, 65, 4), (4, 1, 2, 512, 33, 4),
+                                            (8, 2, 2, 512, 70, 2), (4, 2, 4, 256, 45, 6),
+                                            (4, 4, 4, 256, 40, 1), (8, 1, 1, 512, 70, 4)])
+def test_stencil_matches_oracle(cuda_lib, dtype, H, Hkv, C, E, S, KC):
     cls = cuda_lib
-    w = W.Workload("t", 2, S, E, H, Hkv, C, dtype=dtype)
+    w = W.Workload("t", 2, S, E, H, Hkv, C, dtype=dtype, conv_kernel=KC)
     ocfg = oracle_config(w)
     inp = W.make_inputs(w, seed=3, conv_std=0.3, identity_conv=True)
     dt = w.torch_dtype
@@ -81,7 +86,8 @@ def test_stencil_matches_oracle(cuda_lib, dtype, H, Hkv, C, E, S):
     q = torch.empty(2, H, S, w.dl, dtype=w.latent_dtype, device="cuda")
     k = torch.empty(2, Hkv, S + 5, w.dl, dtype=w.latent_dtype, device="cuda")
     v = torch.empty(2, Hkv, S + 5, w.dl, dtype=w.latent_dtype, device="cuda")
-    cfg = cls.make_config(E, H, Hkv, C, dtype=cls.CCA_BF16 if dtype == "bf16" else cls.CCA_F32)
+    cfg = cls.make_config(E, H, Hkv, C, conv_kernel=KC,
+                          dtype=cls.CCA_BF16 if dtype == "bf16" else cls.CCA_F32)
     ws = torch.empty(cls.cca_stage_stencil_workspace_size(cfg), dtype=torch.uint8, device="cuda")
     cls.cca_stage_stencil(cfg, P.cuda(), 2, S, inp.conv_seq.cuda(), inp.conv_chan.cuda(), q, k, v,
                           S + 5, ws)
@@ -270,6 +276,18 @@ def test_decode_step_full_size(cuda_lib):
     assert (cache.lengths.cpu() == L + 1).all()
 
 
+def test_decode_kernel_count(cuda_lib):
+    """The step launches projection, stencil, attention and output kernels, plus the merge of
+    the attention's key splits when the (sequence, group) pairs are fewer than the SMs."""
+    cls = cuda_lib
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    cfg = cls.make_config(2048, 16, 4, 4)
+    assert cls.cca_decode_kernel_count(cfg, 64, 8300) == (4 if 64 * 4 >= sms else 5)
+    assert cls.cca_decode_kernel_count(cfg, 2, 8300) == 5
+    assert cls.cca_decode_kernel_count(cls.make_config(256, 4, 4, 4, dtype=cls.CCA_F32), 64, 300) == 5
+    assert cls.cca_decode_kernel_count(cfg, 0, 8300) < 0
+
+
 def test_decode_ragged_lengths(cuda_lib):
     w = W.Workload("dec", 5, 300, 256, 4, 2, 2, decode=True)
     lengths = [0, 1, 255, 256, 300]
@@ -279,10 +297,12 @@ def test_decode_ragged_lengths(cuda_lib):
     assert cache.lengths.cpu().tolist() == [l + 1 for l in lengths]
 
 
-def test_decode_equals_prefill_gpu(cuda_lib):
-    """Prefill S0 tokens into the cache, then n decode steps == prefill of S0 + n tokens."""
+@pytest.mark.parametrize("KC", [4, 2, 6])
+def test_decode_equals_prefill_gpu(cuda_lib, KC):
+    """Prefill S0 tokens into the cache, then n decode steps == prefill of S0 + n tokens (the
+    conv state carries KC - 1 pre-conv rows from the prefill into the decode)."""
     cls = cuda_lib
-    w = small("dp", seq=40, batch=3)
+    w = small("dp", seq=40, batch=3, conv_kernel=KC)
     inp = W.make_inputs(w, seed=8, conv_std=0.4)
     layer = cls.CCALayer.from_workload(w, inp)
     s0, n = 33, 7
