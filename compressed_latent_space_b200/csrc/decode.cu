@@ -7,8 +7,9 @@
 //   D2  latent stencil of the new row: the causal conv reads the stored KC-1 pre-conv rows,
 //       the value-shift reads the stored upper-half value row; q-k-mean, RMS norm, RoPE at
 //       position L; k, v appended at position L; conv / value-shift state advanced
-//   D3  split-KV attention of the G query heads of each group over keys 0..L
-//   D3b merge of the splits (log-sum-exp), o [B, NQ]
+//   D3  attention of the G query heads of each group over keys 0..L, its keys split across
+//       CTAs only when the (sequence, group) pairs are fewer than the SMs
+//   D3b merge of the splits (log-sum-exp) into o [B, NQ], when there are splits
 //   D4  y = o W_o^T, then lengths[b] += 1
 // A sequence with L >= max_seq is left untouched (y row zero) and the cache status word is
 // set to a "full" code.
