@@ -67,6 +67,80 @@ __device__ __forceinline__ float qk_mean_term(const float *prow, int G, int hh, 
   return 0.5f * (mq / static_cast<float>(G) + pk);
 }
 
+// The tensor-core paths' epilogue for one warp's (head hh, 16 tokens from row tr0) channel-conv
+// tile, in the m16n8k16 accumulator layout (a quad of lanes holds one token's head vector,
+// channels i and i + d~/2 in the same lane): Q-K-Mean skip, RMS norm, RoPE, float16 store.
+// Ps: the group's staged P rows (row tt + halo = token t0 + tt, pitch CHP); Rt: the tile's
+// rotations [tt][d~/2][2]; MQ: Mq holds the mean of the group's q heads' P rows per token
+// [tt][d~] for the k head's skip term (else it is summed here).
+template <int DL, bool MQ>
+__device__ __forceinline__ void store_head_tile(const StencilParams<__nv_bfloat16> &p,
+                                                const float (&acc)[DL / 8][4], const float *Ps,
+                                                int CHP, int halo, const float *Rt,
+                                                const float *Mq, int b, int g, int hh, int t0,
+                                                int tr0, int qc) {
+  constexpr int NT = DL / 8, HALF = DL / 2;
+  const int G = p.G;
+  const bool is_q = hh < G;
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    const int tt = tr0 + half * 8;
+    const float *prow = Ps + (tt + halo) * CHP;
+    float u[NT][2];
+#pragma unroll
+    for (int n = 0; n < NT; ++n)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int i = n * 8 + 2 * qc + e;
+        float v = acc[n][half * 2 + e];
+        if (p.flags & F_QK_MEAN) {
+          if constexpr (MQ)
+            v += 0.5f * ((is_q ? prow[hh * DL + i] : Mq[tt * DL + i]) + prow[G * DL + i]);
+          else
+            v += qk_mean_term<DL>(prow, G, hh, i);
+        }
+        u[n][e] = v;
+      }
+    if (p.flags & F_QK_NORM) {
+      float ss = 0.f;
+#pragma unroll
+      for (int n = 0; n < NT; ++n) ss += u[n][0] * u[n][0] + u[n][1] * u[n][1];
+      ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+      ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+      const float inv = 1.0f / sqrtf(ss / static_cast<float>(DL) + p.eps);
+#pragma unroll
+      for (int n = 0; n < NT; ++n) {
+        u[n][0] *= inv;
+        u[n][1] *= inv;
+      }
+    }
+    if (p.flags & F_ROPE) {
+#pragma unroll
+      for (int n = 0; n < NT / 2; ++n)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int i = n * 8 + 2 * qc + e;          // < d~/2; partner i + d~/2 is n-tile n+NT/2
+          const float c = Rt[(tt * HALF + i) * 2], s = Rt[(tt * HALF + i) * 2 + 1];
+          const float x1 = u[n][e], x2 = u[n + NT / 2][e];
+          u[n][e] = x1 * c - x2 * s;
+          u[n + NT / 2][e] = x1 * s + x2 * c;
+        }
+    }
+    const int t = t0 + tt;
+    if (t < p.S) {
+      __half *dst = is_q ? p.q + ((static_cast<size_t>(b) * p.H + g * G + hh) * p.S + t) * DL
+                         : p.k + ((static_cast<size_t>(b) * p.Hkv + g) * p.kv_stride + t) * DL;
+      bool fits = true;                                // every value within the float16 range
+#pragma unroll
+      for (int n = 0; n < NT; ++n) {
+        fits &= fabsf(u[n][0]) <= kF16Max && fabsf(u[n][1]) <= kF16Max;
+        *reinterpret_cast<uint32_t *>(dst + n * 8 + 2 * qc) = pack_f16x2(u[n][0], u[n][1]);
+      }
+      if (!fits) report(p.status, DEV_RANGE);
+    }
+  }
+}
+
 // KCT: the sequence-conv width when it is the common 4 (taps unrolled exactly), 0 = any.
 template <typename T, int DL, int KCT>
 __global__ void __launch_bounds__(512) stencil_kernel(const StencilParams<T> p) {
@@ -184,58 +258,7 @@ __global__ void __launch_bounds__(512) stencil_kernel(const StencilParams<T> p) 
           mma_bf16_16816(acc[n], al, bh);
         }
       }
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const int tt = mt * 16 + gr + half * 8;
-        const float *prow = Ps + (tt + halo) * CHP;
-        float u[NT][2];
-#pragma unroll
-        for (int n = 0; n < NT; ++n)
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int i = n * 8 + 2 * qc + e;
-            float v = acc[n][half * 2 + e];
-            if (p.flags & F_QK_MEAN) v += qk_mean_term<DL>(prow, G, hh, i);
-            u[n][e] = v;
-          }
-        if (p.flags & F_QK_NORM) {
-          float ss = 0.f;
-#pragma unroll
-          for (int n = 0; n < NT; ++n) ss += u[n][0] * u[n][0] + u[n][1] * u[n][1];
-          ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-          ss += __shfl_xor_sync(0xffffffffu, ss, 2);
-          const float inv = 1.0f / sqrtf(ss / static_cast<float>(DL) + p.eps);
-#pragma unroll
-          for (int n = 0; n < NT; ++n) {
-            u[n][0] *= inv;
-            u[n][1] *= inv;
-          }
-        }
-        if (p.flags & F_ROPE) {
-#pragma unroll
-          for (int n = 0; n < NT / 2; ++n)
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const int i = n * 8 + 2 * qc + e;      // < d~/2; partner i + d~/2 is n-tile n+NT/2
-              const float c = Rt[(tt * HALF + i) * 2], s = Rt[(tt * HALF + i) * 2 + 1];
-              const float x1 = u[n][e], x2 = u[n + NT / 2][e];
-              u[n][e] = x1 * c - x2 * s;
-              u[n + NT / 2][e] = x1 * s + x2 * c;
-            }
-        }
-        const int t = t0 + tt;
-        if (t < p.S) {
-          TL *dst = is_q ? p.q + ((static_cast<size_t>(b) * p.H + g * G + hh) * p.S + t) * DL
-                         : p.k + ((static_cast<size_t>(b) * p.Hkv + g) * p.kv_stride + t) * DL;
-          bool fits = true;                            // every value within the float16 range
-#pragma unroll
-          for (int n = 0; n < NT; ++n) {
-            fits &= fabsf(u[n][0]) <= kF16Max && fabsf(u[n][1]) <= kF16Max;
-            *reinterpret_cast<uint32_t *>(dst + n * 8 + 2 * qc) = pack_f16x2(u[n][0], u[n][1]);
-          }
-          if (!fits) report(p.status, DEV_RANGE);
-        }
-      }
+      store_head_tile<DL, false>(p, acc, Ps, CHP, halo, Rt, nullptr, b, g, hh, t0, mt * 16 + gr, qc);
     }
   } else {
     constexpr int LPI = DL < 32 ? DL : 32;   // lanes per (token, head) item
@@ -460,7 +483,6 @@ __global__ void __launch_bounds__(32 * MAXW, 1) stencil_group_kernel(
     // channel conv tasks: (head, 16 tokens) per warp
     for (int task = warp; task < (G + 1) * MT; task += nwarps) {
       const int hh = task / MT, mt = task % MT;
-      const bool is_q = hh < G;
       const uint2 *wb = Wsp + static_cast<size_t>(hh) * DL * WLD;
       float acc[NT][4];
 #pragma unroll
@@ -511,59 +533,7 @@ __global__ void __launch_bounds__(32 * MAXW, 1) stencil_group_kernel(
           mma_bf16_16816(acc[n], al, bh);
         }
       }
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const int tt = tr0 + half * 8;
-        const float *prow = Ps + (tt + halo) * CHP;
-        float uv[NT][2];
-#pragma unroll
-        for (int n = 0; n < NT; ++n)
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int i = n * 8 + 2 * qc + e;
-            float v = acc[n][half * 2 + e];
-            if (p.flags & F_QK_MEAN)
-              v += 0.5f * ((is_q ? prow[hh * DL + i] : Mq[tt * DL + i]) + prow[G * DL + i]);
-            uv[n][e] = v;
-          }
-        if (p.flags & F_QK_NORM) {
-          float ss = 0.f;
-#pragma unroll
-          for (int n = 0; n < NT; ++n) ss += uv[n][0] * uv[n][0] + uv[n][1] * uv[n][1];
-          ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-          ss += __shfl_xor_sync(0xffffffffu, ss, 2);
-          const float inv = 1.0f / sqrtf(ss / static_cast<float>(DL) + p.eps);
-#pragma unroll
-          for (int n = 0; n < NT; ++n) {
-            uv[n][0] *= inv;
-            uv[n][1] *= inv;
-          }
-        }
-        if (p.flags & F_ROPE) {
-#pragma unroll
-          for (int n = 0; n < NT / 2; ++n)
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const int i = n * 8 + 2 * qc + e;      // < d~/2; partner i + d~/2 is n-tile n+NT/2
-              const float c = Rt[(tt * HALF + i) * 2], sn = Rt[(tt * HALF + i) * 2 + 1];
-              const float x1 = uv[n][e], x2 = uv[n + NT / 2][e];
-              uv[n][e] = x1 * c - x2 * sn;
-              uv[n + NT / 2][e] = x1 * sn + x2 * c;
-            }
-        }
-        const int t = t0 + tt;
-        if (t < p.S) {
-          TL *dst = is_q ? p.q + ((static_cast<size_t>(b) * p.H + g * G + hh) * p.S + t) * DL
-                         : p.k + ((static_cast<size_t>(b) * p.Hkv + g) * p.kv_stride + t) * DL;
-          bool fits = true;                            // every value within the float16 range
-#pragma unroll
-          for (int n = 0; n < NT; ++n) {
-            fits &= fabsf(uv[n][0]) <= kF16Max && fabsf(uv[n][1]) <= kF16Max;
-            *reinterpret_cast<uint32_t *>(dst + n * 8 + 2 * qc) = pack_f16x2(uv[n][0], uv[n][1]);
-          }
-          if (!fits) report(p.status, DEV_RANGE);
-        }
-      }
+      store_head_tile<DL, true>(p, acc, Ps, CHP, halo, Rt, Mq, b, g, hh, t0, tr0, qc);
     }
 
     // values with the value-shift: upper half of the value channels from token t-1
