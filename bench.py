@@ -355,21 +355,10 @@ def run_decode_only(args):
                       "gpu_launches": dec["launches"]}), flush=True)
 
 
-def run_cuda(args):
-    rank, world, local = dist_setup(args.gpus)
-    import compressed_latent_space_b200 as cls
-    cls.load()
-    w = workload_from_args(args)
-    hbm, bf16_peak, bf16_sus, peak_src = measured_peaks()
-    with ClockSampler(local) as clk:
-        pre = bench_prefill(cls, w, args.steps, args.warmup, world, seed=rank)
-        dec = None
-        if not args.no_decode:
-            dw = W.WORKLOADS[DECODE_WORKLOAD]
-            dec = bench_decode(cls, dw, args.steps, args.warmup, seed=rank,
-                               layers=args.decode_layers)
-    ms = max_over_ranks(pre["ms"], world)
-    e2e_ms = max_over_ranks(pre["e2e_ms"], world)
+def result_line(w, world, steps, warmup, pre, ms, e2e_ms, dec, dms, peaks):
+    """The JSON line of the CUDA arm from the per-rank results (`pre` / `dec` as the bench
+    functions return them) and the step times already maximised over ranks."""
+    hbm, bf16_peak, _, peak_src = peaks
     tokens = w.batch * w.seq
     flops = prefill_flops(w)
     attn_ms = pre["stages"].get("latent_attention", float("nan"))
@@ -379,8 +368,8 @@ def run_cuda(args):
         "value": job_throughput(tokens, world, ms),
         "unit": "tokens/s",
         "n_gpus": world,
-        "steps": args.steps,
-        "warmup": args.warmup,
+        "steps": steps,
+        "warmup": warmup,
         "ms_per_step": ms,
         "higher_is_better": True,
         "scaling": "weak",
@@ -408,7 +397,6 @@ def run_cuda(args):
     }
     if dec:
         dw = W.WORKLOADS[DECODE_WORKLOAD]
-        dms = max_over_ranks(dec["ms"], world)
         gbs = decode_bytes(dw) / (dms * 1e-3) / 1e9
         line["decode"] = {"workload": dw.name, "description": dw.description, "ms_per_step": dms,
                           "tokens_per_s": job_throughput(dw.batch, world, dms), "GB/s": gbs,
@@ -417,6 +405,26 @@ def run_cuda(args):
                           "peak_source": peak_src,
                           "layers": f"steps rotate over {dec['layers']} independent layers "
                                     "(weights + caches), so none is in L2 from its last use"}
+    return line
+
+
+def run_cuda(args):
+    rank, world, local = dist_setup(args.gpus)
+    import compressed_latent_space_b200 as cls
+    cls.load()
+    w = workload_from_args(args)
+    with ClockSampler(local) as clk:
+        pre = bench_prefill(cls, w, args.steps, args.warmup, world, seed=rank)
+        dec = None
+        if not args.no_decode:
+            dw = W.WORKLOADS[DECODE_WORKLOAD]
+            dec = bench_decode(cls, dw, args.steps, args.warmup, seed=rank,
+                               layers=args.decode_layers)
+    ms = max_over_ranks(pre["ms"], world)
+    e2e_ms = max_over_ranks(pre["e2e_ms"], world)
+    dms = max_over_ranks(dec["ms"], world) if dec else None
+    line = result_line(w, world, args.steps, args.warmup, pre, ms, e2e_ms, dec, dms,
+                       measured_peaks())
     line["clocks"] = clk.summary()
     if rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_oracle_sample(w)
