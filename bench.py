@@ -257,6 +257,7 @@ def bench_decode(cls, w, steps, warmup, seed, layers=DECODE_LAYERS):
         cache.conv_state.copy_(inp.conv_state.cuda())
         cache.vshift_state.copy_(inp.vshift_state.cuda())
         cache.lengths.copy_(inp.lengths.cuda())
+        layer.workspace(cls.cca_decode_workspace_size(layer.cfg, w.batch, max_seq))  # not in a step
         stack.append((layer, cache))
     del k0, v0
     x = inp.x.cuda()
