@@ -271,11 +271,13 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int i = 0; i < TN; ++i)
           if (i > last) r[i] = __float_as_uint(-INFINITY);
       }
+      static_assert(TN % 8 == 0, "four chains of pairs cover the tile");
       float mx4[4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) mx4[e] = __uint_as_float(r[e]);
+      for (int e = 0; e < 4; ++e)
+        mx4[e] = fmaxf(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1]));
 #pragma unroll
-      for (int i = 4; i < TN; i += 8)
+      for (int i = 8; i < TN; i += 8)
 #pragma unroll
         for (int e = 0; e < 4; ++e)
           mx4[e] = max3(mx4[e], __uint_as_float(r[i + 2 * e]), __uint_as_float(r[i + 2 * e + 1]));
