@@ -326,12 +326,12 @@ def cpu_oracle_sample(w, budget_s=12.0, seed=0):
                        f"this overstates the oracle's full-length rate)")
 
 
-# DRAM bytes (read + write) of one latent-attention launch on the default workload: the
-# ncu capture of the same kernel on one 8192-token sequence of it (profiles/
-# attn_tc_ccgqa_prefill_16k.md) read 25.2 MB, exactly its q, k and v (the k / v tiles that
-# later query tiles re-read stay in L2); q, k and v grow with the token count, so a launch
-# of 2 x 16384 tokens moves 4x that.  Only valid for the kernel version that was profiled.
-ATTN_TRAFFIC = {"ccgqa_prefill_16k": 25204992 * 4}
+# DRAM bytes (read + write) of one latent-attention launch on a workload, from an ncu
+# capture of the current kernel (scaled by tokens from a smaller case of the same shape); a
+# workload without one reports null.  The capture in profiles/attn_tc_ccgqa_prefill_16k.md
+# (25.2 MB = exactly q, k and v on one 8192-token sequence) belongs to the earlier two-tile
+# kernel, so none is listed for the current one.
+ATTN_TRAFFIC = {}
 
 
 def workload_from_args(args):

@@ -5,23 +5,25 @@
 // (gist.science/de explainer, 2. Methodik: Softmax(QK^T)V evaluated entirely in the
 // compressed space; gist.science explainer, Extension: CCGQA.)
 //
-// One CTA per SM owns two adjacent 128-row query tiles A (2i) and B (2i+1) of one head and
-// streams the 128-key tiles of its key/value head once for both (causal: A reads tiles
-// 0..2i, B 0..2i+1).  The two tiles alternate on the tensor cores, so each tile's softmax
-// runs while the other tile's MMAs execute:
-//   warps 0-3 : softmax of tile A, warps 4-7 : softmax of tile B.  One query row per thread
-//               (warp w reads TMEM lanes 32*(w%4)..), all 128 keys of a tile in registers.
-//               Online softmax in fp32 with lazy rescaling (the reference max only moves when
-//               a row max grows by more than 2^8, and then the warp rescales its rows of O);
-//               the probabilities are packed to float16 pairs and written over the tile's own
-//               scores in TMEM, where the P*V MMA reads them as its A operand.
-//   warp 8    : TMA producer: both Q tiles once, then K and V tiles into two rings.
-//   warp 9    : allocates TMEM (S_A, S_B: 128 fp32 columns each; O_A, O_B: d~ each) and
-//               issues the MMAs (whole warp runs the loop, one elected lane issues).  Per
-//               key tile j: O_A += P_A V_j, S_A = Q_A K_{j+1}^T, O_B += P_B V_j,
-//               S_B = Q_B K_{j+1}^T.  The tensor pipe executes in issue order, so a tile's
-//               next S overwrites its P only after P*V has read it, and a tile's O is final
-//               for the softmax whenever its next S is ready.
+// One CTA per SM owns NTILE (3) adjacent 128-row query tiles of one head and streams the
+// TN-key (96) tiles of its key/value head once for all of them (causal: tile t reads the key
+// tiles through its last row).  The tiles take turns on the tensor cores, so each tile's
+// softmax runs while the others' MMAs execute, and three softmax warps per scheduler keep the
+// exponential unit busier than two (the softmax, not the tensor pipe, bounds this kernel):
+//   warps 4t..4t+3 : softmax of tile t.  One query row per thread (warp w reads TMEM lanes
+//               32*(w%4)..), all TN keys of a tile in registers.  Online softmax in fp32 with
+//               lazy rescaling (the reference max only moves when a row max grows by more than
+//               2^8, and then the warp rescales its rows of O); the probabilities are packed to
+//               float16 pairs and written over the tile's own scores in TMEM, where the P*V
+//               MMA reads them as its A operand.  Key tiles that straddle the diagonal are
+//               masked per row.
+//   warp W_TMA : TMA producer: the Q tiles once, then K and V tiles into two rings.
+//   warp W_MMA : allocates TMEM (S_t: TN fp32 columns each; O_t: d~ each, from a 64-aligned
+//               column) and issues the MMAs (whole warp runs the loop, one elected lane
+//               issues).  Per key tile j and tile t: O_t += P_t V_j, S_t = Q_t K_{j+1}^T.  The
+//               tensor pipe executes in issue order, so a tile's next S overwrites its P only
+//               after P*V has read it, and a tile's O is final for the softmax whenever its
+//               next S is ready.
 // Every wait is bounded; on a timeout the CTA records it in the status word, stops, and
 // releases its tensor memory.
 #include <math.h>
@@ -33,36 +35,37 @@ namespace cca {
 namespace {
 
 constexpr int TM = 128;          // query rows per tile (M of all MMAs)
-constexpr int TN = 128;          // keys per tile
-constexpr int NSOFT = 8;         // softmax warps: 4 per query tile
-constexpr int W_TMA = 8, W_MMA = 9;
+constexpr int TN = 96;           // keys per tile
+constexpr int NTILE = 3;         // query tiles per CTA
+constexpr int NSOFT = 4 * NTILE; // softmax warps: 4 per query tile
+constexpr int W_TMA = NSOFT, W_MMA = NSOFT + 1;
 constexpr int THREADS = (NSOFT + 2) * 32;
 constexpr float kTau = 8.0f;     // lazy-rescale threshold, log2 units
 
 template <int DL>
 struct AttnCfg {
-  static constexpr int SK = DL >= 64 ? 3 : 4;          // K ring depth
-  static constexpr int SV = DL >= 64 ? 3 : 4;          // V ring depth
+  static constexpr int SK = 4;                         // K ring depth
+  static constexpr int SV = 4;                         // V ring depth
   static constexpr int ROWB = DL * 2;                  // bytes of one q / k / v row
   static constexpr int Q_BYTES = TM * ROWB;
   static constexpr int KV_BYTES = TN * ROWB;           // one K or one V tile
   static constexpr uint32_t SW_MODE = ROWB == 128 ? 2u : ROWB == 64 ? 4u : 6u;
   static constexpr int SBO = 8 * ROWB;                 // stride of 8-row core groups
-  static constexpr int OFF_Q = 0;                      // Q_A, Q_B
-  static constexpr int OFF_K = OFF_Q + 2 * Q_BYTES;
+  static constexpr int OFF_Q = 0;                      // the NTILE query tiles
+  static constexpr int OFF_K = OFF_Q + NTILE * Q_BYTES;
   static constexpr int OFF_V = OFF_K + SK * KV_BYTES;
   static constexpr int OFF_BAR = OFF_V + SV * KV_BYTES;
-  static constexpr int SMEM = OFF_BAR + 256;
+  static constexpr int SMEM = OFF_BAR + 512;
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr uint32_t COL_O = 2 * TN;            // O_A at 256, O_B at 256 + d~
-  static_assert(COL_O + 2 * DL <= TMEM_COLS, "S and O of both tiles must fit the TMEM allocation");
+  static constexpr uint32_t COL_O = (NTILE * TN + 63) / 64 * 64;  // S_t at t * TN; O_t 64-aligned
+  static_assert(COL_O + NTILE * DL <= TMEM_COLS, "S and O of all tiles must fit the TMEM allocation");
 };
 
 struct AttnBars {
   uint64_t q_full;
   uint64_t k_full[4], k_empty[4];
   uint64_t v_full[4], v_empty[4];
-  uint64_t s_full[2], p_full[2], o_done[2];
+  uint64_t s_full[NTILE], p_full[NTILE], o_done[NTILE];
   uint32_t tmem_base;
   int abort;
 };
@@ -118,11 +121,12 @@ __global__ void __launch_bounds__(THREADS, 1)
   extern __shared__ __align__(1024) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h = blockIdx.x, b = blockIdx.y;
-  const int pair = static_cast<int>(gridDim.z) - 1 - static_cast<int>(blockIdx.z);  // long first
-  const int qt0 = 2 * pair;                          // tile A; tile B = qt0 + 1 when it exists
-  const bool hasB = qt0 + 1 < nqt;
-  const int nkvA = qt0 + 1, nkvB = qt0 + 2;
-  const int nsteps = hasB ? nkvB : nkvA;
+  const int grp = static_cast<int>(gridDim.z) - 1 - static_cast<int>(blockIdx.z);  // long first
+  const int qt0 = NTILE * grp;                       // tiles qt0 .. qt0 + ntile - 1
+  const int ntile = min(NTILE, nqt - qt0);
+  // key tiles of query tile t: through its last row (the diagonal band is masked)
+  auto nkv = [&](int t) { return ((qt0 + t + 1) * TM + TN - 1) / TN; };
+  const int nsteps = nkv(ntile - 1);
   const int g = h / G;
   AttnBars *bars = reinterpret_cast<AttnBars *>(smem + C::OFF_BAR);
 
@@ -139,9 +143,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&bars->v_full[s], 1);
       mbar_init(&bars->v_empty[s], 1);
     }
-    for (int t = 0; t < 2; ++t) {
+    for (int t = 0; t < NTILE; ++t) {
       mbar_init(&bars->s_full[t], 1);
-      mbar_init(&bars->p_full[t], NSOFT / 2);
+      mbar_init(&bars->p_full[t], 4);
       mbar_init(&bars->o_done[t], 1);
     }
     bars->abort = 0;
@@ -163,10 +167,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       tma_prefetch_desc(&mapQ);
       tma_prefetch_desc(&mapK);
       tma_prefetch_desc(&mapV);
-      mbar_arrive_expect_tx(&bars->q_full, (hasB ? 2 : 1) * C::Q_BYTES);
-      tma_load_3d(smem + C::OFF_Q, &mapQ, &bars->q_full, 0, qt0 * TM, b * H + h);
-      if (hasB)
-        tma_load_3d(smem + C::OFF_Q + C::Q_BYTES, &mapQ, &bars->q_full, 0, (qt0 + 1) * TM, b * H + h);
+      mbar_arrive_expect_tx(&bars->q_full, ntile * C::Q_BYTES);
+      for (int t = 0; t < ntile; ++t)
+        tma_load_3d(smem + C::OFF_Q + t * C::Q_BYTES, &mapQ, &bars->q_full, 0, (qt0 + t) * TM,
+                    b * H + h);
       for (int j = 0; j < nsteps; ++j) {
         const int sk = j % C::SK, sv = j % C::SV;
         if (!mbar_wait(&bars->k_empty[sk], ((j / C::SK) & 1) ^ 1u, abort, status)) break;
@@ -202,8 +206,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                                           mbar_wait(&bars->k_full[0], 0, abort, status));
     if (ok) {
       tc_fence_after();
-      issue_qk(0, 0);
-      if (hasB) issue_qk(1, 0);
+      for (int t = 0; t < ntile; ++t) issue_qk(t, 0);
       if (leader) umma_commit(&bars->k_empty[0]);
       __syncwarp();
     }
@@ -217,9 +220,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (!ok) break;
       const uint64_t vd = smem_desc(smem_u32(smem + C::OFF_V + sv * C::KV_BYTES), C::KV_BYTES,
                                     C::SBO, C::SW_MODE);
-      for (int t = 0; t < 2; ++t) {
-        const int nk = t ? nkvB : nkvA;
-        if ((t == 1 && !hasB) || j >= nk) continue;
+      for (int t = 0; t < ntile; ++t) {
+        const int nk = nkv(t);
+        if (j >= nk) continue;
         ok = __all_sync(0xffffffffu, mbar_wait(&bars->p_full[t], j & 1, abort, status));
         if (!ok) break;
         tc_fence_after();
@@ -245,13 +248,13 @@ __global__ void __launch_bounds__(THREADS, 1)
     // ---------------------------------------------------------------- softmax warps 0-7
     const int t = warp >> 2, quad = warp & 3;
     const int row = quad * 32 + lane;                 // TMEM lane of this thread
-    const int nk = t ? nkvB : nkvA;
+    const int nk = nkv(t);
     const int qpos = (qt0 + t) * TM + row;
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
     const uint32_t tS = tmem + t * TN + lane_off, tO = tmem + C::COL_O + t * DL + lane_off;
     const uint64_t sc2 = f2(scale_log2, scale_log2);
     float m_ref = -INFINITY, l = 0.f;
-    bool ok = t == 0 || hasB;
+    bool ok = t < ntile;
     for (int j = 0; ok && j < nk; ++j) {
       // S_t of tile j is ready, and every earlier MMA (this tile's P*V of j-1) is done
       ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full[t], j & 1, abort, status));
@@ -265,7 +268,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       // Row max of the raw scores (the 1/sqrt(d~) * log2(e) scale is positive, so it is
       // applied afterwards), in four independent three-input chains.  Keys past this row's
       // position are masked on the diagonal tile only.
-      if (j == nk - 1) {
+      if ((j + 1) * TN > (qt0 + t) * TM) {           // a tile of the diagonal band
         const int last = qpos - j * TN;               // keys 0..last of this tile are visible
 #pragma unroll
         for (int i = 0; i < TN; ++i)
@@ -367,6 +370,7 @@ cudaError_t launch_tc(const Dims &d, const void *q, const void *k, const void *v
   CUtensorMap mq, mk, mv;
   const uint64_t row = static_cast<uint64_t>(DL) * 2;
   const uint32_t box[3] = {static_cast<uint32_t>(DL), static_cast<uint32_t>(TM), 1u};
+  const uint32_t box_kv[3] = {static_cast<uint32_t>(DL), static_cast<uint32_t>(TN), 1u};
   {
     const uint64_t dims[3] = {static_cast<uint64_t>(DL), static_cast<uint64_t>(d.S),
                               static_cast<uint64_t>(d.B) * d.H};
@@ -378,13 +382,13 @@ cudaError_t launch_tc(const Dims &d, const void *q, const void *k, const void *v
     const uint64_t dims[3] = {static_cast<uint64_t>(DL), static_cast<uint64_t>(d.S),
                               static_cast<uint64_t>(d.B) * d.Hkv};
     const uint64_t strides[2] = {row, row * static_cast<uint64_t>(kv_stride)};
-    if (!make_tma_16bit(&mk, k, 3, dims, strides, box, C::ROWB, 1) ||
-        !make_tma_16bit(&mv, v, 3, dims, strides, box, C::ROWB, 1))
+    if (!make_tma_16bit(&mk, k, 3, dims, strides, box_kv, C::ROWB, 1) ||
+        !make_tma_16bit(&mv, v, 3, dims, strides, box_kv, C::ROWB, 1))
       return cudaErrorInvalidValue;
   }
   if (cudaError_t e = ensure_dyn_smem<attn_tc_kernel<DL>>(C::SMEM); e != cudaSuccess) return e;
   const int nqt = (d.S + TM - 1) / TM;
-  dim3 grid(d.H, d.B, (nqt + 1) / 2);
+  dim3 grid(d.H, d.B, (nqt + NTILE - 1) / NTILE);
   attn_tc_kernel<DL><<<grid, THREADS, C::SMEM, st>>>(mq, mk, mv, static_cast<__half *>(o), d.S,
                                                      d.H, d.Hkv, d.G, nqt, scale_log2, status);
   return cudaGetLastError();
