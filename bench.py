@@ -50,14 +50,20 @@ def attention_flops(w) -> float:
 
 
 def decode_bytes(w, es=2) -> float:
-    """Algorithmic HBM bytes of one decode step: the K/V cache read (L+1 rows), both weight
-    matrices, the conv / value-shift state read and written, x read and y written."""
+    """Algorithmic HBM bytes of one decode step: the K/V cache read (L+1 rows, 16-bit), both
+    weight matrices, the float32 conv / value-shift state read and written, x read and y
+    written."""
     B, ctx = w.batch, w.seq
     cache = 2.0 * B * w.n_kv_heads * (ctx + 1) * w.dl * es
     weights = ((w.n_q + 2 * w.n_kv) * w.d_model + w.d_model * w.n_q) * es
-    state = 2.0 * B * ((w.conv_kernel - 1) * (w.n_q + w.n_kv) + (w.n_kv - w.n_kv // 2)) * es
+    state = 2.0 * B * ((w.conv_kernel - 1) * (w.n_q + w.n_kv) + (w.n_kv - w.n_kv // 2)) * 4
     io = 2.0 * B * w.d_model * es
     return cache + weights + state + io
+
+
+# Rated dense bf16 tensor throughput of one B200 (the sparsity-free half of NVIDIA's figure),
+# reported beside the measured cuBLAS peak.
+RATED_BF16_TFLOPS = 2250.0
 
 
 def measured_peaks():
@@ -66,6 +72,14 @@ def measured_peaks():
         d = json.load(open(p))
         return d["hbm_gbs"], d["bf16_tflops"], d.get("bf16_tflops_sustained"), "measured"
     return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def measured_peak_clock():
+    """Median SM clock under load while MEASURED_PEAKS.json's GEMM peak was taken (or None)."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        return json.load(open(p)).get("clocks_under_load", {}).get("sm_mhz_median")
+    return None
 
 
 class ClockSampler:
@@ -155,7 +169,7 @@ def barrier(world):
 
 
 # ------------------------------------------------------------------ the CUDA arm
-def bench_prefill(cls, w, steps, warmup, world, seed):
+def bench_prefill(cls, w, steps, warmup, world, seed, e2e=True):
     inp = W.make_inputs(w, seed=seed)
     layer = cls.CCALayer.from_workload(w, inp)
     x = inp.x.cuda()
@@ -179,10 +193,13 @@ def bench_prefill(cls, w, steps, warmup, world, seed):
     cls.cca_stage_timing(False)
     stage_ms, calls = cls.cca_stage_times(8)
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    ms = statistics.fmean(step_ms)
+    ms = statistics.median(step_ms)
     stages = {n: t / max(calls, 1) for n, t in
               zip(["weights_to_16bit", "qkv_projection", "latent_stencil", "latent_attention",
                    "out_projection"], stage_ms)}
+
+    if not e2e:
+        return dict(ms=ms, stages=stages, calls=calls, launches=6 * steps)
 
     # end to end through the public API, the way a server would overlap the copies: each
     # sequence's x goes host -> device on one copy stream, its forward runs on the compute
@@ -223,7 +240,7 @@ def bench_prefill(cls, w, steps, warmup, world, seed):
         e2e_step(e2e_s[i])
         e2e_e[i].record()
     torch.cuda.synchronize()
-    e2e_ms = statistics.fmean(s.elapsed_time(e) for s, e in zip(e2e_s, e2e_e))
+    e2e_ms = statistics.median(s.elapsed_time(e) for s, e in zip(e2e_s, e2e_e))
     nbytes = x.numel() * x.element_size()
     return dict(ms=ms, stages=stages, calls=calls, e2e_ms=e2e_ms, h2d=nbytes, d2h=nbytes,
                 launches=6 * steps)
@@ -288,14 +305,39 @@ def bench_decode(cls, w, steps, warmup, seed, layers=DECODE_LAYERS):
     stage_ms, calls = cls.cca_stage_times(8)
     for layer, cache in stack:
         cls.cca_cache_check(cache.struct)
-    names = ["qkv_projection", "stencil_append", "split_kv_attention", "merge", "out_projection"]
+    nk = decode_launches(cls, stack[0][0], w.batch, max_seq)
+    names = (["qkv_projection", "stencil_append", "split_kv_attention", "merge", "out_projection"]
+             if nk == 5 else ["qkv_projection", "stencil_append", "attention", "out_projection"])
     return dict(ms=ms, stages={n: t / max(calls, 1) for n, t in zip(names, stage_ms)},
-                launches=decode_launches(cls, stack[0][0], w.batch, max_seq) * steps, layers=layers)
+                launches=nk * steps, layers=layers)
 
 
-def cpu_oracle_sample(w, budget_s=12.0, seed=0):
-    """Times the float64 oracle on the causal prefix of sequence 0 of the workload, doubling
-    the prefix from 512 tokens while the run stays within the budget."""
+def cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def host_cores() -> int:
+    return len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+
+
+# The oracle's sample of a prefill workload: the causal prefix of sequence 0, this many tokens
+# (the whole workload when it is smaller).  Both the CUDA arm's cpu_baseline and the reference
+# arm time exactly this sample.
+CPU_SAMPLE_TOKENS = 4096
+
+
+def cpu_oracle_sample(w, seed=0, full=False):
+    """Times the float64 oracle once on a fixed sample of the workload and returns the rate.
+
+    Prefill: a full forward of the first CPU_SAMPLE_TOKENS tokens of sequence 0 (all B*S
+    tokens with full=True); per-token attention cost grows with the prefix, so a prefix sample
+    overstates the oracle's full-length rate.  Decode: one decode step of the whole batch."""
     import numpy as np
     import oracle.cca_oracle as O
     from oracle.cca_oracle import OracleConfig, OracleWeights
@@ -305,33 +347,40 @@ def cpu_oracle_sample(w, budget_s=12.0, seed=0):
     f64 = lambda t: t.to(torch.float64).numpy()
     ow = OracleWeights.from_arrays(cfg, f64(inp.w_qkv), f64(inp.w_o), f64(inp.conv_seq),
                                    f64(inp.conv_chan))
-    x0 = f64(inp.x[0])
-    T = 512
-    best = None
-    spent = 0.0
-    while T <= w.seq:
+    base = dict(unit="tokens/s", cores=host_cores(), kind="oracle", cpu=cpu_model())
+    if w.decode:
         t0 = time.perf_counter()
-        O.prefill_sequence(cfg, ow, x0[:T])
+        O.decode_batch(cfg, ow, f64(inp.x), f64(inp.k_cache), f64(inp.v_cache),
+                       inp.lengths.numpy(), f64(inp.conv_state), f64(inp.vshift_state))
         dt = time.perf_counter() - t0
-        spent += dt
-        best = (T, dt)
-        if spent + 4.5 * dt > budget_s or T == w.seq:
-            break
-        T = min(2 * T, w.seq)
-    T, dt = best
-    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
-    return dict(value=T / dt, unit="tokens/s", cores=cores, kind="oracle",
+        return dict(base, value=w.batch / dt, seconds=dt,
+                    sample=f"float64 oracle decode step of all {w.batch} sequences of {w.name} "
+                           f"({w.seq} cached tokens each; {dt:.2f} s)")
+    if full or w.batch * w.seq <= CPU_SAMPLE_TOKENS:
+        t0 = time.perf_counter()
+        O.prefill(cfg, ow, f64(inp.x))
+        dt = time.perf_counter() - t0
+        return dict(base, value=w.batch * w.seq / dt, seconds=dt,
+                    sample=f"float64 oracle full forward of {w.name} ({w.batch} x {w.seq} "
+                           f"tokens; {dt:.2f} s)")
+    T = min(CPU_SAMPLE_TOKENS, w.seq)
+    x0 = f64(inp.x[0, :T])
+    t0 = time.perf_counter()
+    O.prefill_sequence(cfg, ow, x0)
+    dt = time.perf_counter() - t0
+    return dict(base, value=T / dt, seconds=dt,
                 sample=f"float64 oracle forward of the first {T} tokens of sequence 0 of "
-                       f"{w.name} ({dt:.2f} s; per-token attention cost grows with the prefix, so "
-                       f"this overstates the oracle's full-length rate)")
+                       f"{w.name} ({dt:.2f} s; per-token attention cost grows with the prefix, "
+                       f"so this overstates the oracle's full-length rate)")
 
 
 # DRAM bytes (read + write) of one latent-attention launch on a workload, from an ncu
 # capture of the current kernel (scaled by tokens from a smaller case of the same shape); a
-# workload without one reports null.  The capture in profiles/attn_tc_ccgqa_prefill_16k.md
-# (25.2 MB = exactly q, k and v on one 8192-token sequence) belongs to the earlier two-tile
-# kernel, so none is listed for the current one.
-ATTN_TRAFFIC = {}
+# workload without one reports null.
+ATTN_TRAFFIC = {
+    # 25.43 MB read on one 8192-token sequence (B=1) of the same shape, x 4 for 2 x 16384 tokens
+    "ccgqa_prefill_16k": 4 * 25.428992e6,
+}
 
 
 def workload_from_args(args):
@@ -348,12 +397,17 @@ def run_decode_only(args):
     cls.load()
     hbm, _, _, peak_src = measured_peaks()
     dw = W.WORKLOADS[DECODE_WORKLOAD]
-    dec = bench_decode(cls, dw, args.steps, args.warmup, seed=0, layers=args.decode_layers)
+    with ClockSampler(0) as clk:
+        dec = bench_decode(cls, dw, args.steps, args.warmup, seed=0, layers=args.decode_layers)
     gbs = decode_bytes(dw) / (dec["ms"] * 1e-3) / 1e9
-    print(json.dumps({"metric": "decode GB/s", "value": gbs, "unit": "GB/s",
-                      "ms_per_step": dec["ms"], "frac_of_hbm": gbs / hbm, "peak_source": peak_src,
-                      "workload": dw.name, "stages_ms": dec["stages"], "layers": dec["layers"],
-                      "gpu_launches": dec["launches"]}), flush=True)
+    line = {"metric": "decode GB/s", "value": gbs, "unit": "GB/s",
+            "ms_per_step": dec["ms"], "frac_of_hbm": gbs / hbm, "peak_source": peak_src,
+            "tokens_per_s": dw.batch / (dec["ms"] * 1e-3), "bytes_per_step": decode_bytes(dw),
+            "workload": dw.name, "stages_ms": dec["stages"], "layers": dec["layers"],
+            "gpu_launches": dec["launches"], "clocks": clk.summary()}
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_oracle_sample(dw)
+    print(json.dumps(line), flush=True)
 
 
 def result_line(w, world, steps, warmup, pre, ms, e2e_ms, dec, dms, peaks):
@@ -384,11 +438,15 @@ def result_line(w, world, steps, warmup, pre, ms, e2e_ms, dec, dms, peaks):
                    "parallelism": f"replicas x{world}",
                    "l2": "flushed between timed steps (256 MiB write outside the step events)"},
         "tflops": flops / (ms * 1e-3) / 1e12,
-        "tflops_frac_of_bf16_peak": flops / (ms * 1e-3) / 1e12 / bf16_peak,
+        "tflops_frac_of_measured_bf16_peak": flops / (ms * 1e-3) / 1e12 / bf16_peak,
+        "tflops_frac_of_rated_bf16_peak": flops / (ms * 1e-3) / 1e12 / RATED_BF16_TFLOPS,
         "stages_ms": pre["stages"],
         "roofline": {"kernel": "latent_attention", "bound": "tensor", "achieved": attn_tflops,
                      "peak": bf16_peak, "unit": "TFLOP/s", "frac": attn_tflops / bf16_peak,
-                     "traffic": ATTN_TRAFFIC.get(w.name), "peak_source": f"{peak_src} bf16 burst"},
+                     "traffic": ATTN_TRAFFIC.get(w.name),
+                     "peak_source": f"{peak_src} cuBLAS bf16 burst",
+                     "frac_of_rated": attn_tflops / RATED_BF16_TFLOPS,
+                     "rated_peak": RATED_BF16_TFLOPS},
         "e2e": {"value": job_throughput(tokens, world, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": pre["h2d"], "d2h_bytes_per_step": pre["d2h"],
                 "ms_per_step": e2e_ms,
@@ -409,11 +467,33 @@ def result_line(w, world, steps, warmup, pre, ms, e2e_ms, dec, dms, peaks):
     return line
 
 
+def bench_baselines(cls, steps, warmup, world, seed, ccgqa_ms):
+    """The systems the pages compare CCA / CCGQA prefill with at 16k tokens (MHA and GQA-8,
+    head width 128, RoPE, same d_model / heads / batch as the CCGQA workload), run on this
+    library's own GEMM, pointwise latent kernel and attention kernel, timed like the CCGQA
+    step.  The ratios set this B200's numbers beside the pages' H100 ones (1.7x, 1.3x)."""
+    out = {}
+    for name, w in W.BASELINES.items():
+        r = bench_prefill(cls, w, steps, warmup, world, seed, e2e=False)
+        out[name] = {"description": w.description, "ms_per_step": r["ms"],
+                     "tokens_per_s": job_throughput(w.batch * w.seq, world, r["ms"]),
+                     "tflops": prefill_flops(w) / (r["ms"] * 1e-3) / 1e12,
+                     "attention_tflops": attention_flops(w) / (r["stages"]["latent_attention"] * 1e-3) / 1e12,
+                     "stages_ms": r["stages"],
+                     "ccgqa_speedup": r["ms"] / ccgqa_ms}
+    out["pages_h100"] = "CCA/CCGQA prefill 1.7x faster than MHA and 1.3x faster than GQA-8 at 16k (context only)"
+    return out
+
+
 def run_cuda(args):
     rank, world, local = dist_setup(args.gpus)
     import compressed_latent_space_b200 as cls
     cls.load()
     w = workload_from_args(args)
+    if w.decode:                      # a decode workload named directly: its own line
+        if world > 1:
+            raise SystemExit("the decode workload line is a 1-GPU profiling case")
+        return run_decode_only(args)
     with ClockSampler(local) as clk:
         pre = bench_prefill(cls, w, args.steps, args.warmup, world, seed=rank)
         dec = None
@@ -421,12 +501,28 @@ def run_cuda(args):
             dw = W.WORKLOADS[DECODE_WORKLOAD]
             dec = bench_decode(cls, dw, args.steps, args.warmup, seed=rank,
                                layers=args.decode_layers)
+        base = None
+        if not args.no_baselines and w.name == DEFAULT_WORKLOAD:
+            base = bench_baselines(cls, args.steps, args.warmup, world, rank, pre["ms"])
     ms = max_over_ranks(pre["ms"], world)
     e2e_ms = max_over_ranks(pre["e2e_ms"], world)
     dms = max_over_ranks(dec["ms"], world) if dec else None
     line = result_line(w, world, args.steps, args.warmup, pre, ms, e2e_ms, dec, dms,
                        measured_peaks())
+    if base:
+        for name in W.BASELINES:
+            base[name]["ms_per_step"] = max_over_ranks(base[name]["ms_per_step"], world)
+        line["baselines"] = base
+        line["gpu_launches"] += sum(6 * args.steps for _ in W.BASELINES)
     line["clocks"] = clk.summary()
+    peak_clk = measured_peak_clock()
+    if peak_clk and line["clocks"].get("sm_mhz"):
+        # the measured GEMM peak ran power-capped at a lower SM clock than this run: the
+        # fraction at equal clocks scales the achieved rate by peak clock / this run's clock
+        r = line["roofline"]
+        r["sm_mhz"] = line["clocks"]["sm_mhz"]
+        r["peak_sm_mhz"] = peak_clk
+        r["frac_at_peak_clock"] = r["frac"] * peak_clk / line["clocks"]["sm_mhz"]
     if rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_oracle_sample(w)
     if rank == 0:
@@ -442,22 +538,18 @@ def run_reference(args):
     if rank != 0:
         return
     w = workload_from_args(args)
-    per_step_budget = max(2.0, 150.0 / max(1, args.steps + args.warmup))
-    for _ in range(args.warmup):
-        cpu_oracle_sample(w, budget_s=per_step_budget)
-    vals = []
-    samples = []
-    for _ in range(args.steps):
-        r = cpu_oracle_sample(w, budget_s=per_step_budget)
-        vals.append(r["value"])
-        samples.append(r)
-    v = statistics.fmean(vals)
+    for _ in range(args.warmup if not args.cpu_full else 0):
+        cpu_oracle_sample(w)
+    runs = [cpu_oracle_sample(w, full=args.cpu_full) for _ in range(args.steps if not args.cpu_full else 1)]
+    v = statistics.median(r["value"] for r in runs)
     line = {"metric": METRIC, "value": v, "unit": "tokens/s", "impl": "reference",
-            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "n_gpus": args.gpus, "steps": len(runs), "warmup": args.warmup,
+            "ms_per_step": statistics.median(r["seconds"] for r in runs) * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": {"workload": w.name, "description": w.description},
-            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": samples[-1]["cores"],
-                             "kind": "oracle", "sample": samples[-1]["sample"]},
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": runs[-1]["cores"],
+                             "kind": "oracle", "sample": runs[-1]["sample"],
+                             "cpu": runs[-1]["cpu"]},
             "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -475,6 +567,11 @@ def main():
                     help="independent layers the decode steps rotate over (fewer for profiling "
                          "captures that must stay small; the timing needs the default)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-baselines", action="store_true",
+                    help="skip the same-box MHA / GQA-8 prefill baselines")
+    ap.add_argument("--cpu-full", action="store_true",
+                    help="reference arm: one full forward of the whole workload instead of the "
+                         "fixed prefix sample (minutes for the large workloads)")
     ap.add_argument("--decode-only", action="store_true",
                     help="time only the decode step (a profiling case for its kernels)")
     ap.add_argument("--batch", type=int, default=None,

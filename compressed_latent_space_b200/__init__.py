@@ -26,6 +26,7 @@ CCA_ERR_DEVICE = -7
 CCA_ERR_RANGE = -8
 CCA_QK_MEAN, CCA_VALUE_SHIFT, CCA_QK_NORM, CCA_ROPE = 1, 2, 4, 8
 CCA_DEFAULT_FLAGS = 15
+CCA_NO_CONV = 16
 
 
 class CCAError(RuntimeError):
@@ -77,6 +78,7 @@ _SIGS = {
     "cca_workspace_status": (c_int, [c_void_p, c_void_p]),
     "cca_decode_step_static": (c_int, [POINTER(cca_config_t), POINTER(cca_weights_t), c_void_p,
                                        c_void_p, POINTER(cca_cache_t), c_void_p]),
+    "cca_stage_wait_probe": (c_int, [ctypes.c_longlong, c_int, c_void_p, c_void_p]),
     "cca_stage_timing": (c_int, [c_int]),
     "cca_stage_times": (c_int, [POINTER(ctypes.c_double), c_int, POINTER(c_int)]),
 }
@@ -128,7 +130,9 @@ def make_config(d_model, n_heads, n_kv_heads, compression, conv_kernel=4, chan_c
 
 
 def make_weights(w_qkv, w_o, conv_seq, conv_chan) -> cca_weights_t:
-    return cca_weights_t(w_qkv.data_ptr(), w_o.data_ptr(), conv_seq.data_ptr(), conv_chan.data_ptr())
+    """Conv filters may be None for CCA_NO_CONV layers (passed as NULL)."""
+    ptr = lambda t: None if t is None else t.data_ptr()
+    return cca_weights_t(w_qkv.data_ptr(), w_o.data_ptr(), ptr(conv_seq), ptr(conv_chan))
 
 
 def cca_last_error_string() -> str:
@@ -210,6 +214,11 @@ def cca_stage_attention(cfg, q, k, v, batch, seq, kv_stride, o, status=None, str
 
 def cca_workspace_status(workspace, stream=None):
     _check(load().cca_workspace_status(_ptr(workspace), _stream(stream)))
+
+
+def cca_stage_wait_probe(limit_ns: int, arm: bool, status, stream=None):
+    _check(load().cca_stage_wait_probe(int(limit_ns), 1 if arm else 0, _ptr(status),
+                                       _stream(stream)))
 
 
 def cca_stage_timing(enable: bool):

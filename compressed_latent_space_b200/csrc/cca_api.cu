@@ -61,15 +61,17 @@ int make_dims(const cca_config_t *cfg, cca::Dims &d) {
   if (hd % cfg->compression)
     return fail(CCA_ERR_INVALID_ARG, "head width %d is not a multiple of compression %d", hd, cfg->compression);
   const int dl = hd / cfg->compression;
-  if (dl != 16 && dl != 32 && dl != 64)
-    return fail(CCA_ERR_UNSUPPORTED, "latent head width %d: kernels take 16, 32 or 64", dl);
+  if (dl != 16 && dl != 32 && dl != 64 && dl != 128)
+    return fail(CCA_ERR_UNSUPPORTED, "latent head width %d: kernels take 16, 32, 64 or 128", dl);
+  if (dl == 128 && cfg->dtype != CCA_BF16)
+    return fail(CCA_ERR_UNSUPPORTED, "latent head width 128 is supported for bfloat16 layers only");
   if (cfg->conv_kernel < 1 || cfg->conv_kernel > 8)
     return fail(CCA_ERR_UNSUPPORTED, "conv_kernel %d: kernels take 1..8", cfg->conv_kernel);
   if (cfg->chan_conv_kernel != 1)
     return fail(CCA_ERR_UNSUPPORTED, "chan_conv_kernel %d: kernels take 1 (pointwise)", cfg->chan_conv_kernel);
   if (cfg->dtype != CCA_F32 && cfg->dtype != CCA_BF16)
     return fail(CCA_ERR_INVALID_ARG, "dtype %d is neither CCA_F32 nor CCA_BF16", cfg->dtype);
-  if (cfg->flags & ~static_cast<unsigned>(CCA_DEFAULT_FLAGS))
+  if (cfg->flags & ~static_cast<unsigned>(CCA_DEFAULT_FLAGS | CCA_NO_CONV))
     return fail(CCA_ERR_INVALID_ARG, "unknown flag bits 0x%x", cfg->flags);
   if (!(cfg->norm_eps >= 0.f)) return fail(CCA_ERR_INVALID_ARG, "norm_eps must be >= 0");
   if ((cfg->flags & CCA_ROPE) && !(cfg->rope_base > 1.f))
@@ -83,6 +85,7 @@ int make_dims(const cca_config_t *cfg, cca::Dims &d) {
   d.NKV = d.Hkv * dl;
   d.NQKV = d.NQ + 2 * d.NKV;
   d.KC = cfg->conv_kernel;
+  d.VS0 = d.NKV / 2;
   d.flags = cfg->flags;
   d.eps = cfg->norm_eps;
   d.rope_base = cfg->rope_base;
@@ -102,7 +105,7 @@ PrefillLayout prefill_layout(const cca::Dims &d, int B, int S) {
   size_t off = 0;
   L.status = off; off += 256;
   L.wo16 = off; off += d.bf16 ? align256(static_cast<size_t>(d.E) * d.NQ * 2) : 0;
-  L.wsplit = off; off += align256(cca::conv_chan_split_bytes(d));
+  L.wsplit = off; off += (d.flags & CCA_NO_CONV) ? 0 : align256(cca::conv_chan_split_bytes(d));
   L.P = off; off += align256(M * d.NQKV * 4);   // projections stay float32
   L.q = off; off += align256(M * d.NQ * es);
   L.k = off; off += align256(M * d.NKV * es);
@@ -123,11 +126,28 @@ CacheLayout cache_layout(const cca::Dims &d, int B, int max_seq) {
   L.k = off; off += align256(static_cast<size_t>(B) * d.Hkv * max_seq * d.DL * es);
   L.v = off; off += align256(static_cast<size_t>(B) * d.Hkv * max_seq * d.DL * es);
   L.conv = off; off += align256(static_cast<size_t>(B) * (d.KC - 1) * (d.NQ + d.NKV) * 4);
-  L.vshift = off; off += align256(static_cast<size_t>(B) * (d.NKV - d.NKV / 2) * 4);
+  L.vshift = off; off += align256(static_cast<size_t>(B) * (d.NKV - d.VS0) * 4);
   L.lengths = off; off += align256(static_cast<size_t>(B) * 4);
   L.status = off; off += 256;
   L.total = off;
   return L;
+}
+
+// The decode kernels (and so the cache) cover latent widths up to 64 with the convolutions.
+int check_decode_shape(const cca::Dims &d) {
+  if (d.DL > 64)
+    return fail(CCA_ERR_UNSUPPORTED, "decode and the cache take latent head widths 16, 32 or 64");
+  if (d.flags & CCA_NO_CONV)
+    return fail(CCA_ERR_UNSUPPORTED, "decode and the cache need the convolutions (CCA_NO_CONV is prefill-only)");
+  return CCA_OK;
+}
+
+// The convolution stencil covers latent widths up to 64; CCA_NO_CONV layers take up to 128.
+int check_stencil_shape(const cca::Dims &d) {
+  if (d.DL > 64 && !(d.flags & CCA_NO_CONV))
+    return fail(CCA_ERR_UNSUPPORTED, "latent head width %d needs CCA_NO_CONV (the convolution "
+                "stencil takes 16, 32 or 64)", d.DL);
+  return CCA_OK;
 }
 
 int check_cache(const cca::Dims &d, const cca_cache_t *c) {
@@ -248,6 +268,7 @@ CCA_API int cca_cache_alloc(const cca_config_t *cfg, int batch, int max_seq, voi
   cca::Dims d;
   int rc = make_dims(cfg, d);
   if (rc) return rc;
+  if ((rc = check_decode_shape(d))) return rc;
   if (!bytes) return fail(CCA_ERR_INVALID_ARG, "bytes is NULL");
   if (batch <= 0 || max_seq <= 0) return fail(CCA_ERR_INVALID_ARG, "batch and max_seq must be positive");
   const CacheLayout L = cache_layout(d, batch, max_seq);
@@ -276,13 +297,13 @@ CCA_API int cca_cache_alloc(const cca_config_t *cfg, int batch, int max_seq, voi
 
 CCA_API size_t cca_prefill_workspace_size(const cca_config_t *cfg, int batch, int seq) {
   cca::Dims d;
-  if (make_dims(cfg, d) || batch < 0 || seq < 0) return 0;
+  if (make_dims(cfg, d) || check_stencil_shape(d) || batch < 0 || seq < 0) return 0;
   return prefill_layout(d, batch, seq).total;
 }
 
 CCA_API size_t cca_decode_workspace_size(const cca_config_t *cfg, int batch, int max_seq) {
   cca::Dims d;
-  if (make_dims(cfg, d) || batch <= 0 || max_seq <= 0) return 0;
+  if (make_dims(cfg, d) || check_decode_shape(d) || batch <= 0 || max_seq <= 0) return 0;
   d.B = batch;
   return cca::decode_workspace_bytes(d, max_seq);
 }
@@ -291,6 +312,7 @@ CCA_API int cca_decode_kernel_count(const cca_config_t *cfg, int batch, int max_
   cca::Dims d;
   int rc = make_dims(cfg, d);
   if (rc) return rc;
+  if ((rc = check_decode_shape(d))) return rc;
   if (batch <= 0 || max_seq <= 0) return fail(CCA_ERR_INVALID_ARG, "batch and max_seq must be positive");
   d.B = batch;
   return cca::decode_kernel_count(d, max_seq);
@@ -302,7 +324,9 @@ CCA_API int cca_prefill_forward(const cca_config_t *cfg, const cca_weights_t *w,
   cca::Dims d;
   int rc = make_dims(cfg, d);
   if (rc) return rc;
-  if (!w || !w->w_qkv || !w->w_o || !w->conv_seq || !w->conv_chan)
+  if ((rc = check_stencil_shape(d))) return rc;
+  const bool no_conv = (d.flags & CCA_NO_CONV) != 0;
+  if (!w || !w->w_qkv || !w->w_o || (!no_conv && (!w->conv_seq || !w->conv_chan)))
     return fail(CCA_ERR_INVALID_ARG, "weights (or one of their pointers) NULL");
   if (batch < 0 || seq < 0) return fail(CCA_ERR_INVALID_ARG, "batch and seq must be >= 0");
   if (batch > 0 && seq > 0 && (!x || !y)) return fail(CCA_ERR_INVALID_ARG, "x or y NULL");
@@ -312,6 +336,7 @@ CCA_API int cca_prefill_forward(const cca_config_t *cfg, const cca_weights_t *w,
       !aligned16(workspace))
     return fail(CCA_ERR_ALIGNMENT, "x, y, weights and workspace must be 16-byte aligned");
   if (cache) {
+    if ((rc = check_decode_shape(d))) return rc;
     if ((rc = check_cache(d, cache))) return rc;
     if (cache->batch != batch)
       return fail(CCA_ERR_INVALID_ARG, "cache batch %d != batch %d", cache->batch, batch);
@@ -341,7 +366,7 @@ CCA_API int cca_prefill_forward(const cca_config_t *cfg, const cca_weights_t *w,
     if ((e = cca::convert_bf16_to_f16(w->w_o, wo, static_cast<size_t>(d.E) * d.NQ, status, st)) !=
         cudaSuccess)
       return cuda_fail(e, "W_o conversion launch");
-    if ((e = cca::split_conv_chan(d, w->conv_chan, ws + L.wsplit, st)) != cudaSuccess)
+    if (!no_conv && (e = cca::split_conv_chan(d, w->conv_chan, ws + L.wsplit, st)) != cudaSuccess)
       return cuda_fail(e, "channel-conv weight split launch");
   }
   rec.mark();
@@ -386,6 +411,7 @@ CCA_API int cca_decode_step(const cca_config_t *cfg, const cca_weights_t *w, con
   if (rc) return rc;
   if (!w || !w->w_qkv || !w->w_o || !w->conv_seq || !w->conv_chan)
     return fail(CCA_ERR_INVALID_ARG, "weights (or one of their pointers) NULL");
+  if ((rc = check_decode_shape(d))) return rc;
   if (!cache) return fail(CCA_ERR_INVALID_ARG, "cache is NULL");
   if ((rc = check_cache(d, cache))) return rc;
   if (d.G > 8)
@@ -479,8 +505,10 @@ CCA_API int cca_stage_stencil(const cca_config_t *cfg, const void *P, int batch,
   cca::Dims d;
   int rc = make_dims(cfg, d);
   if (rc) return rc;
+  if ((rc = check_stencil_shape(d))) return rc;
+  const bool no_conv = (d.flags & CCA_NO_CONV) != 0;
   if (batch < 0 || seq < 0 || kv_stride < seq) return fail(CCA_ERR_INVALID_ARG, "bad batch/seq/kv_stride");
-  if (batch > 0 && seq > 0 && (!P || !conv_seq || !conv_chan || !q || !k || !v))
+  if (batch > 0 && seq > 0 && (!P || (!no_conv && (!conv_seq || !conv_chan)) || !q || !k || !v))
     return fail(CCA_ERR_INVALID_ARG, "NULL pointer");
   if (!aligned16(P)) return fail(CCA_ERR_ALIGNMENT, "P must be 16-byte aligned");
   if (injected_launch_failure()) return fail(CCA_ERR_CUDA, "injected launch failure");
@@ -494,7 +522,7 @@ CCA_API int cca_stage_stencil(const cca_config_t *cfg, const void *P, int batch,
   char *wsp = static_cast<char *>(workspace);
   int *status = reinterpret_cast<int *>(wsp);
   cudaError_t e0 = cudaMemsetAsync(status, 0, 256, st);
-  if (e0 == cudaSuccess && d.bf16) e0 = cca::split_conv_chan(d, conv_chan, wsp + 256, st);
+  if (e0 == cudaSuccess && d.bf16 && !no_conv) e0 = cca::split_conv_chan(d, conv_chan, wsp + 256, st);
   if (e0 != cudaSuccess) return cuda_fail(e0, "stencil preparation");
   cca::StencilArgs sa{};
   sa.P = static_cast<const float *>(P);

@@ -150,17 +150,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 // Waits for the phase of `bar` with the given parity to complete.  Gives up (returns
-// false) when *abort is set by another warp or after kWaitLimitNs; the first warp to give
-// up records DEV_WAIT_TIMEOUT and sets *abort so the others stop waiting too.
+// false) when *abort is set by another warp or after limit_ns (kWaitLimitNs unless a caller
+// passes another); the first warp to give up records DEV_WAIT_TIMEOUT and sets *abort so the
+// others stop waiting too.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
-                                          int *status) {
+                                          int *status, uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t n = 1;; ++n) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((n & 255u) == 0) {
       if (*abort) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (globaltimer_ns() - t0 > limit_ns) {
         *abort = 1;
         report(status, DEV_WAIT_TIMEOUT);
         return false;

@@ -191,7 +191,7 @@ struct D2Params {
   float *conv_state, *vshift_state;
   int *lengths, *status;
   float *q_new;
-  int B, H, Hkv, G, DL, NQ, NKV, NQKV, KC, max_seq;
+  int B, H, Hkv, G, DL, NQ, NKV, NQKV, KC, VS0, max_seq;
   unsigned flags;
   float eps;
   double theta[32];        // RoPE frequencies base^(-2i/d~), i < d~/2, computed on the host
@@ -356,7 +356,7 @@ __device__ __forceinline__ void d2_compute(const D2Params<T> &p, int g, int b, i
     }
   }
   // value with the value-shift, appended at position L
-  const int vhalf = p.NKV / 2;
+  const int vhalf = p.VS0;
   float *vs = p.vshift_state + static_cast<size_t>(b) * (p.NKV - vhalf);
   for (int c = tid; c < DL; c += nt) {
     const int vc = g * DL + c;
@@ -1027,7 +1027,8 @@ static cudaError_t decode_typed(const Dims &d, const DecodeArgs &a, cudaStream_t
   p2.status = a.status;
   p2.q_new = a.q_new;
   p2.B = d.B; p2.H = d.H; p2.Hkv = d.Hkv; p2.G = d.G; p2.DL = d.DL;
-  p2.NQ = d.NQ; p2.NKV = d.NKV; p2.NQKV = d.NQKV; p2.KC = d.KC; p2.max_seq = a.max_seq;
+  p2.NQ = d.NQ; p2.NKV = d.NKV; p2.NQKV = d.NQKV; p2.KC = d.KC; p2.VS0 = d.VS0;
+  p2.max_seq = a.max_seq;
   p2.flags = d.flags;
   p2.eps = d.eps;
   for (int i = 0; i < d.DL / 2; ++i)
@@ -1058,6 +1059,7 @@ static cudaError_t decode_typed(const Dims &d, const DecodeArgs &a, cudaStream_t
                      a.part_o, a.part_ml, a.lengths, o_hi, o_hi + static_cast<size_t>(d.B) * d.NQ,
                      d.H, d.DL, a.max_seq, a.chunk, a.nchunk);
       if (e != cudaSuccess) return e;
+      mark();
     }
   } else {
     const int nused_max = a.nchunk;
@@ -1071,8 +1073,8 @@ static cudaError_t decode_typed(const Dims &d, const DecodeArgs &a, cudaStream_t
                                                    static_cast<float *>(a.o), d.H, d.DL,
                                                    a.max_seq, a.nchunk);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    mark();
   }
-  mark();
   // D4 (+ lengths advance for 16-bit layers)
   if constexpr (sizeof(T) == 2) {
     const __nv_bfloat16 *o_hi = static_cast<const __nv_bfloat16 *>(a.o);

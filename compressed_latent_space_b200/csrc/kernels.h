@@ -15,6 +15,7 @@ struct Dims {
   int G = 0, DL = 0;             // group size H/Hkv, latent head width
   int NQ = 0, NKV = 0, NQKV = 0; // H*DL, Hkv*DL, NQ + 2*NKV
   int KC = 0;                    // sequence-conv taps
+  int VS0 = 0;                   // first value channel taken from the previous token (value-shift)
   unsigned flags = 0;
   float eps = 1e-6f;
   float rope_base = 10000.f;
@@ -31,7 +32,7 @@ struct StageMarker {
   }
 };
 
-enum : unsigned { F_QK_MEAN = 1u, F_VALUE_SHIFT = 2u, F_QK_NORM = 4u, F_ROPE = 8u };
+enum : unsigned { F_QK_MEAN = 1u, F_VALUE_SHIFT = 2u, F_QK_NORM = 4u, F_ROPE = 8u, F_NO_CONV = 16u };
 
 // C[M, N] = A[M, K] * B[N, K]^T, bf16 (or f16 with ab_f16) in, fp32 accumulate, bf16 or fp32
 // out (tcgen05 + TMA).

@@ -40,7 +40,7 @@ struct StencilParams {
   int *lengths;
   int *status;
   int write_state;
-  int B, S, H, Hkv, G, NQ, NKV, NQKV, KC, halo, TT, kv_stride;
+  int B, S, H, Hkv, G, NQ, NKV, NQKV, KC, VS0, halo, TT, kv_stride;
   unsigned flags;
   float eps;
   double theta[32];        // RoPE frequencies base^(-2i/d~), i < d~/2, computed on the host
@@ -325,7 +325,7 @@ __global__ void __launch_bounds__(512) stencil_kernel(const StencilParams<T> p) 
   }
 
   // 4. values with the value-shift: upper half of the value channels from token t-1.
-  const int vhalf = p.NKV / 2;
+  const int vhalf = p.VS0;
   for (int i = tid; i < TT * (DL / 2); i += blockDim.x) {
     const int tt = i / (DL / 2), c = (i % (DL / 2)) * 2;
     const int t = t0 + tt;
@@ -459,7 +459,7 @@ __global__ void __launch_bounds__(32 * MAXW, 1) stencil_group_kernel(
   issue(u_beg, 0);                                  // (the filter copies join this group)
 
   const int gr = lane >> 2, qc = lane & 3;
-  const int vhalf = p.NKV / 2;
+  const int vhalf = p.VS0;
   for (int u = u_beg, k = 0; u < u_end; ++u, ++k) {
     const int buf = k & 1;
     issue(u + 1, buf ^ 1);
@@ -596,7 +596,7 @@ cudaError_t launch(const Dims &d, const StencilArgs &a, cudaStream_t st) {
   p.lengths = a.lengths;
   p.write_state = a.write_state ? 1 : 0;
   p.B = d.B; p.S = d.S; p.H = d.H; p.Hkv = d.Hkv; p.G = d.G;
-  p.NQ = d.NQ; p.NKV = d.NKV; p.NQKV = d.NQKV; p.KC = d.KC;
+  p.NQ = d.NQ; p.NKV = d.NKV; p.NQKV = d.NQKV; p.KC = d.KC; p.VS0 = d.VS0;
   p.halo = d.KC - 1 > 1 ? d.KC - 1 : 1;
   p.kv_stride = a.kv_stride;
   p.flags = d.flags;
@@ -652,6 +652,139 @@ cudaError_t launch(const Dims &d, const StencilArgs &a, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------ identity convolutions
+// The latent step with both convolutions the identity (CCA_NO_CONV): q = pq, k = pk before
+// Q-K-Mean (whose pre- and post-conv terms then coincide), value-shift, RMS norm and RoPE as
+// selected.  With C = 1 and only RoPE on, this is the projection-to-attention step of plain
+// multi-head (or grouped-query) attention with rotary embeddings, for any latent width up to
+// 128.  One warp per (token, head) item, reading its P row segment straight from global
+// memory (lane i holds channels i and i + d~/2, the RoPE pair, of the row); no shared memory,
+// so many warps per SM hide the load latency of this memory-bound pass.
+template <typename T>
+struct PointParams {
+  using TL = typename LatentType<T>::type;
+  const float *P;
+  TL *q, *k, *v;
+  int *status;
+  int B, S, H, Hkv, G, DL, NQ, NKV, NQKV, VS0, kv_stride;
+  unsigned flags;
+  float eps;
+  double theta[64];        // RoPE frequencies base^(-2i/d~), i < d~/2, computed on the host
+};
+
+template <typename T>
+__global__ void __launch_bounds__(256) pointwise_kernel(const PointParams<T> p) {
+  using TL = typename LatentType<T>::type;
+  const int lane = threadIdx.x & 31;
+  const int per_tok = p.H + 2 * p.Hkv;
+  const long long items = static_cast<long long>(p.B) * p.S * per_tok;
+  const long long nwarps = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
+  const int DL = p.DL, HALF = DL / 2;
+  for (long long it = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+       it < items; it += nwarps) {
+    const long long bt = it / per_tok;               // b * S + t
+    const int hh = static_cast<int>(it % per_tok);
+    const int b = static_cast<int>(bt / p.S), t = static_cast<int>(bt % p.S);
+    const float *row = p.P + bt * p.NQKV;
+    if (hh < p.H + p.Hkv) {                         // a query or key head
+      const bool is_q = hh < p.H;
+      const int g = is_q ? hh / p.G : hh - p.H;
+      const int off = is_q ? hh * DL : p.NQ + g * DL;
+      float u[2][2];                                // pairs (i, i + d~/2), i = lane + 32e
+      float ss = 0.f;
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int i = lane + 32 * e;
+#pragma unroll
+        for (int s2 = 0; s2 < 2; ++s2) {
+          float x = 0.f;
+          if (i < HALF) {
+            const int c = i + s2 * HALF;
+            x = row[off + c];
+            if (p.flags & F_QK_MEAN) {              // post-conv == pre-conv here
+              const float pk = row[p.NQ + g * DL + c];
+              float pq;
+              if (is_q) {
+                pq = x;
+              } else {
+                pq = 0.f;
+                for (int h2 = 0; h2 < p.G; ++h2) pq += row[(g * p.G + h2) * DL + c];
+                pq /= static_cast<float>(p.G);
+              }
+              x += 0.5f * (pq + pk);
+            }
+          }
+          u[e][s2] = x;
+          ss += x * x;
+        }
+      }
+      if (p.flags & F_QK_NORM) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        const float inv = 1.0f / sqrtf(ss / static_cast<float>(DL) + p.eps);
+#pragma unroll
+        for (int e = 0; e < 2; ++e) { u[e][0] *= inv; u[e][1] *= inv; }
+      }
+      TL *dst = is_q ? p.q + ((static_cast<size_t>(b) * p.H + hh) * p.S + t) * DL
+                     : p.k + ((static_cast<size_t>(b) * p.Hkv + g) * p.kv_stride + t) * DL;
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int i = lane + 32 * e;
+        if (i < HALF) {
+          float a = u[e][0], c2 = u[e][1];
+          if (p.flags & F_ROPE) {
+            float cs, sn;
+            rope_cos_sin(static_cast<double>(t) * p.theta[i], cs, sn);
+            const float x1 = a, x2 = c2;
+            a = x1 * cs - x2 * sn;
+            c2 = x1 * sn + x2 * cs;
+          }
+          check_latent<TL>(a, p.status);
+          check_latent<TL>(c2, p.status);
+          dst[i] = from_f32<TL>(a);
+          dst[i + HALF] = from_f32<TL>(c2);
+        }
+      }
+    } else {                                        // a value head, with the value-shift
+      const int g = hh - p.H - p.Hkv;
+      TL *dst = p.v + ((static_cast<size_t>(b) * p.Hkv + g) * p.kv_stride + t) * DL;
+      for (int c = lane; c < DL; c += 32) {
+        const bool shifted = (p.flags & F_VALUE_SHIFT) && (g * DL + c >= p.VS0);
+        float x = 0.f;
+        if (!shifted) x = row[p.NQ + p.NKV + g * DL + c];
+        else if (t > 0) x = row[static_cast<long long>(-p.NQKV) + p.NQ + p.NKV + g * DL + c];
+        check_latent<TL>(x, p.status);
+        dst[c] = from_f32<TL>(x);
+      }
+    }
+  }
+}
+
+template <typename T>
+cudaError_t launch_pointwise(const Dims &d, const StencilArgs &a, cudaStream_t st) {
+  using TL = typename LatentType<T>::type;
+  if (d.DL > 128) return cudaErrorInvalidValue;
+  PointParams<T> p;
+  p.P = a.P;
+  p.q = static_cast<TL *>(a.q);
+  p.k = static_cast<TL *>(a.k);
+  p.v = static_cast<TL *>(a.v);
+  p.status = a.status;
+  p.B = d.B; p.S = d.S; p.H = d.H; p.Hkv = d.Hkv; p.G = d.G; p.DL = d.DL;
+  p.NQ = d.NQ; p.NKV = d.NKV; p.NQKV = d.NQKV; p.VS0 = d.VS0;
+  p.kv_stride = a.kv_stride;
+  p.flags = d.flags;
+  p.eps = d.eps;
+  for (int i = 0; i < 64; ++i)
+    p.theta[i] = i < d.DL / 2 ? pow(static_cast<double>(d.rope_base), -2.0 * i / d.DL) : 0.0;
+  const long long items = static_cast<long long>(d.B) * d.S * (d.H + 2 * d.Hkv);
+  long long blocks = (items + 7) / 8;
+  const long long cap = static_cast<long long>(num_sms()) * 8 * 16;   // a grid-stride loop beyond
+  if (blocks > cap) blocks = cap;
+  pointwise_kernel<T><<<static_cast<unsigned>(blocks), 256, 0, st>>>(p);
+  return cudaGetLastError();
+}
+
 __global__ void split_conv_chan_kernel(const float *__restrict__ w, uint2 *__restrict__ out,
                                        size_t npairs) {
   for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < npairs;
@@ -677,6 +810,10 @@ cudaError_t split_conv_chan(const Dims &d, const float *conv_chan, void *out, cu
 
 cudaError_t latent_stencil(const Dims &d, const StencilArgs &a, cudaStream_t st) {
   if (d.B == 0 || d.S == 0) return cudaSuccess;
+  if (d.flags & F_NO_CONV) {
+    if (a.write_state) return cudaErrorInvalidValue;   // no decode state without the convs
+    return d.bf16 ? launch_pointwise<__nv_bfloat16>(d, a, st) : launch_pointwise<float>(d, a, st);
+  }
   if (d.bf16) {
     if (d.DL == 16) return launch<__nv_bfloat16, 16>(d, a, st);
     if (d.DL == 32) return launch<__nv_bfloat16, 32>(d, a, st);

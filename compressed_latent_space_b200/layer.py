@@ -61,16 +61,21 @@ class CCALayer:
         self.n_kv = n_kv_heads * self.dl
         self.w_qkv = w_qkv.to(self.device, self.dtype).contiguous()
         self.w_o = w_o.to(self.device, self.dtype).contiguous()
-        self.conv_seq = conv_seq.to(self.device, torch.float32).contiguous()
-        self.conv_chan = conv_chan.to(self.device, torch.float32).contiguous()
+        # CCA_NO_CONV layers take no conv filters
+        self.conv_seq = None if conv_seq is None else conv_seq.to(self.device, torch.float32).contiguous()
+        self.conv_chan = None if conv_chan is None else conv_chan.to(self.device, torch.float32).contiguous()
         self.weights = make_weights(self.w_qkv, self.w_o, self.conv_seq, self.conv_chan)
         self._ws = None
 
     @classmethod
-    def from_workload(cls, w, inputs, flags=CCA_DEFAULT_FLAGS, device="cuda"):
+    def from_workload(cls, w, inputs, flags=None, device="cuda"):
+        """flags None: the workload's own switches."""
+        flags = w.flags if flags is None else flags
+        no_conv = bool(flags & 16)
         return cls(w.d_model, w.n_heads, w.n_kv_heads, w.compression, inputs.w_qkv, inputs.w_o,
-                   inputs.conv_seq, inputs.conv_chan, conv_kernel=w.conv_kernel,
-                   rope_base=w.rope_base, flags=flags, dtype=w.dtype, device=device)
+                   None if no_conv else inputs.conv_seq, None if no_conv else inputs.conv_chan,
+                   conv_kernel=w.conv_kernel, rope_base=w.rope_base, flags=flags, dtype=w.dtype,
+                   device=device)
 
     def workspace(self, nbytes: int) -> torch.Tensor:
         if self._ws is None or self._ws.numel() < nbytes:

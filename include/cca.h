@@ -62,19 +62,28 @@ enum {
   CCA_ERR_RANGE = -8          /* a latent q, k or v exceeded the float16 range (16-bit layers) */
 };
 
-/* Switches of the method's three expressivity steps and of normalisation / RoPE. */
+/* Switches of the method's three expressivity steps and of normalisation / RoPE.
+ * CCA_NO_CONV makes both convolutions the identity (Convolutional Mixing off; not part of
+ * CCA_DEFAULT_FLAGS).  With compression 1 and CCA_ROPE alone the layer is plain multi-head
+ * (Hkv == H) or grouped-query attention with rotary embeddings, the systems the pages compare
+ * CCA against (gist.science explainer, 4. Experimental Results: prefill against MHA and GQA-8
+ * at 16k); such layers run up to a latent width of 128, prefill only (no cache, no decode). */
 enum {
   CCA_QK_MEAN = 1u,
   CCA_VALUE_SHIFT = 2u,
   CCA_QK_NORM = 4u,
   CCA_ROPE = 8u,
-  CCA_DEFAULT_FLAGS = 15u
+  CCA_DEFAULT_FLAGS = 15u,
+  CCA_NO_CONV = 16u
 };
 
 /* One CCA / CCGQA layer.  d_model = E, n_heads = H, n_kv_heads = Hkv (H % Hkv == 0;
- * Hkv == H is CCA), compression = C with (E/H) % C == 0.  Supported by the kernels:
- * d~ = E/H/C in {16, 32, 64}, conv_kernel in [1, 8], chan_conv_kernel == 1.  norm_eps is
- * added to the mean square before the square root (1e-6 by default). */
+ * Hkv == H is CCA), compression = C with (E/H) % C == 0.  Queries are compressed by C (latent
+ * width E/C) and keys / values by C * H/Hkv (latent width Hkv * d~): CCGQA's decoupled
+ * compression rates (gist.science explainer, Extension: CCGQA).  Supported by the kernels:
+ * d~ = E/H/C in {16, 32, 64} (and 128 for bfloat16 CCA_NO_CONV prefill), conv_kernel in
+ * [1, 8], chan_conv_kernel == 1.  norm_eps is added to the mean square before the square
+ * root (1e-6 by default). */
 typedef struct {
   int d_model;
   int n_heads;
@@ -120,7 +129,12 @@ typedef struct {
   int max_seq;
 } cca_cache_t;
 
-/* Lays out a decode cache for `batch` sequences of up to `max_seq` tokens.
+/* Lays out a decode cache for `batch` sequences of up to `max_seq` tokens.  The cache holds
+ * the compressed latent keys and values, the thing decoding streams per generated token
+ * (gist.science explainer, 1. Problem Statement), Hkv heads of d~ each (Extension: CCGQA:
+ * grouped key/value heads in the compressed space), plus the conv and value-shift state that
+ * the causal convolutions and Value-Shift of the next token need (2. Methodology, Core
+ * Mechanism).
  * dev_buf == NULL: only writes the byte count to *bytes.  Otherwise *bytes must be at
  * least that count; fills *out with pointers into dev_buf and enqueues on `stream` the
  * zeroing of the whole buffer (lengths = 0, status = 0).  Errors: INVALID_ARG,
@@ -139,8 +153,16 @@ CCA_API size_t cca_decode_workspace_size(const cca_config_t *cfg, int batch, int
  * profiling.  (Not in the paper.)  Negative CCA_ERR_* code if the config is invalid. */
 CCA_API int cca_decode_kernel_count(const cca_config_t *cfg, int batch, int max_seq);
 
-/* Full layer forward of `batch` sequences of `seq` tokens each, from position 0.
+/* Full layer forward of `batch` sequences of `seq` tokens each, from position 0: the
+ * down-projection, convolutional mixing, Q-K-Mean, Value-Shift, normalisation and RoPE,
+ * attention in the compressed space and the up-projection (gist.science explainer,
+ * 2. Methodology, Core Mechanism; Extension: CCGQA for Hkv < H).
  *   x [batch, seq, E] -> y [batch, seq, E]   (x and y must not overlap)
+ * In bfloat16 layers the up-projection runs on float16 operands (the attention output is
+ * float16), so W_o is converted to float16 in the workspace on every call: an entry beyond
+ * the float16 range (|w| > 65504) sets CCA_ERR_RANGE in the workspace status word
+ * (cca_workspace_status), and entries below 2^-14 keep float16's subnormal spacing of 2^-24
+ * (an absolute change below 3e-8 per weight).
  * cache == NULL: keys/values live in the workspace only.  Otherwise (cache->batch ==
  * batch, seq <= max_seq) the final keys/values of every token are written to the cache,
  * the conv and value-shift state of the last token are stored and lengths[b] = seq.
@@ -149,7 +171,11 @@ CCA_API int cca_prefill_forward(const cca_config_t *cfg, const cca_weights_t *w,
                                 int batch, int seq, void *y, cca_cache_t *cache,
                                 void *workspace, size_t ws_bytes, void *stream);
 
-/* One new token per sequence: x [batch, E] -> y [batch, E], batch = cache->batch.
+/* One new token per sequence over the compressed cache: the same operator as
+ * cca_prefill_forward evaluated for the next position only, reading the cached latent keys
+ * and values that decoding streams (gist.science explainer, 1. Problem Statement; Extension:
+ * CCGQA: the grouped latent cache is what shrinks).
+ * x [batch, E] -> y [batch, E], batch = cache->batch.
  * The token's key/value are appended at position lengths[b], its query attends to
  * positions 0..lengths[b], the conv / value-shift state advance and lengths[b] += 1.
  * A sequence already holding max_seq tokens is left untouched, its y row is zero and the
@@ -173,7 +199,9 @@ CCA_API int cca_decode_step(const cca_config_t *cfg, const cca_weights_t *w, con
  * up the array's device address (cudaGetSymbolAddress) with that device current; make that
  * first call before any stream capture.  Every call uses the same array and leaves its
  * contents there; nothing in it needs to start at zero, but two calls whose kernels overlap
- * on the GPU (different streams without ordering) race on it.  Errors as cca_decode_step. */
+ * on the GPU (different streams without ordering) race on it.  The looked-up address is kept
+ * for the life of the process: after cudaDeviceReset on a device, this entry point must not be
+ * called again on that device.  Errors as cca_decode_step. */
 CCA_API int cca_decode_step_static(const cca_config_t *cfg, const cca_weights_t *w,
                                    const void *x, void *y, cca_cache_t *cache, void *stream);
 

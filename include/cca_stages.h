@@ -49,6 +49,15 @@ CCA_API int cca_stage_attention(const cca_config_t *cfg, const void *q, const vo
  * of its kernels recorded an internal error. */
 CCA_API int cca_workspace_status(const void *workspace, void *stream);
 
+/* Failure-detection diagnostic (the paper has no counterpart).  Launches one CTA that runs
+ * the bounded mbarrier wait of the tcgen05 kernels on a shared-memory barrier, with a limit of
+ * limit_ns nanoseconds (1e3 .. 1e9) instead of the kernels' 2 s.  arm == 0: nothing ever
+ * arrives on the barrier, so the wait gives up after the limit, writes DEV_WAIT_TIMEOUT (1) to
+ * *status (a caller-owned device int, expected to hold 0) and the kernel returns; the context
+ * stays usable.  arm != 0: one thread arrives first, the wait completes and *status is left
+ * unchanged.  Errors: INVALID_ARG (limit out of range, status NULL), CUDA (launch). */
+CCA_API int cca_stage_wait_probe(long long limit_ns, int arm, int *status, void *stream);
+
 /* Per-kernel timing for benchmarks.  cca_stage_timing(1) starts a session: from then on
  * every cca_prefill_forward / cca_decode_step records a CUDA event on its stream before its
  * first kernel and after each kernel (events only; nothing else changes).

@@ -21,7 +21,16 @@ def f64(t) -> np.ndarray:
     return t.detach().to("cpu", torch.float64).numpy()
 
 
-def oracle_weights(cfg: OracleConfig, inp) -> OracleWeights:
+def oracle_weights(cfg: OracleConfig, inp, no_conv=False) -> OracleWeights:
+    """The oracle's copy of a workload's weights; no_conv (a CCA_NO_CONV layer) gives it
+    identity convolutions instead of the drawn filters."""
+    if no_conv:
+        conv_seq = np.zeros((cfg.n_q + cfg.n_kv, cfg.conv_kernel))
+        conv_seq[:, -1] = 1.0
+        conv_chan = np.zeros((cfg.n_heads + cfg.n_kv_heads, cfg.dl, cfg.dl, cfg.chan_conv_kernel))
+        idx = np.arange(cfg.dl)
+        conv_chan[:, idx, idx, -1] = 1.0
+        return OracleWeights.from_arrays(cfg, f64(inp.w_qkv), f64(inp.w_o), conv_seq, conv_chan)
     return OracleWeights.from_arrays(cfg, f64(inp.w_qkv), f64(inp.w_o), f64(inp.conv_seq),
                                      f64(inp.conv_chan))
 

@@ -74,7 +74,7 @@ def test_workspace_and_cache_sizes(lib):
     (dict(conv_kernel=9), -2),
     (dict(chan_conv_kernel=2), -2),
     (dict(dtype=7), -1),
-    (dict(flags=16), -1),
+    (dict(flags=32), -1),                       # unknown flag bit
     (dict(norm_eps=-1.0), -1),
 ])
 def test_config_validation(lib, kw, code):
@@ -140,3 +140,23 @@ def test_errors_are_thread_local(lib):
     t.start()
     t.join()
     assert mine != "" and seen == [""]
+
+
+def test_latent_width_128_rules(lib):
+    """d~ = 128 runs only in bfloat16 layers without the convolutions (CCA_NO_CONV), and
+    prefill only: the cache and decode kernels take widths up to 64."""
+    import compressed_latent_space_b200 as cls
+    n = ctypes.c_size_t(0)
+    f32 = cfg(d_model=512, n_heads=4, n_kv_heads=4, compression=1, flags=8 | 16)
+    assert cls.cca_prefill_workspace_size(f32, 1, 8) == 0
+    conv = cfg(d_model=512, n_heads=4, n_kv_heads=4, compression=1, dtype=cls.CCA_BF16)
+    assert cls.cca_prefill_workspace_size(conv, 1, 8) == 0
+    plain = cfg(d_model=512, n_heads=4, n_kv_heads=2, compression=1, dtype=cls.CCA_BF16,
+                flags=8 | 16)
+    assert cls.cca_prefill_workspace_size(plain, 1, 8) > 0
+    assert lib.cca_cache_alloc(ctypes.byref(plain), 1, 8, None, ctypes.byref(n), None, None) == -2
+    assert cls.cca_decode_workspace_size(plain, 1, 8) == 0
+    # the same switch at d~ = 32 is prefill-only too
+    small = cfg(flags=15 | 16, dtype=cls.CCA_BF16)
+    assert cls.cca_prefill_workspace_size(small, 1, 8) > 0
+    assert lib.cca_cache_alloc(ctypes.byref(small), 1, 8, None, ctypes.byref(n), None, None) == -2

@@ -108,10 +108,18 @@ def test_stencil_matches_oracle(cuda_lib, dtype, H, Hkv, C, E, S, KC):
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
+# S = 385, 769 and 1000 give CTAs with all their query tiles in use and several tile groups
+# per head, including rows whose whole diagonal key tile is masked.
 @pytest.mark.parametrize("H,Hkv,DL,S", [(4, 4, 16, 130), (4, 2, 32, 200), (8, 2, 64, 129),
-                                        (3, 1, 32, 64), (2, 2, 64, 1)])
+                                        (3, 1, 32, 64), (2, 2, 64, 1), (4, 1, 64, 385),
+                                        (4, 2, 64, 769), (2, 1, 64, 1000), (8, 2, 32, 385),
+                                        (4, 4, 32, 1000), (8, 1, 32, 769), (8, 8, 16, 1000),
+                                        (4, 4, 128, 385), (4, 2, 128, 200), (2, 1, 128, 1000),
+                                        (8, 1, 128, 130)])
 def test_attention_matches_oracle(cuda_lib, dtype, H, Hkv, DL, S):
     cls = cuda_lib
+    if DL == 128 and dtype == "f32":
+        pytest.skip("latent width 128 is a 16-bit path")
     dt = torch.float32 if dtype == "f32" else torch.bfloat16
     qkt = torch.float32 if dtype == "f32" else torch.float16
     g = torch.Generator("cpu").manual_seed(5)
@@ -137,7 +145,7 @@ def test_attention_matches_oracle(cuda_lib, dtype, H, Hkv, DL, S):
 
 
 # ------------------------------------------------------------------ whole layer
-def run_prefill(cls, w, inp, flags=15):
+def run_prefill(cls, w, inp, flags=None):
     layer = cls.CCALayer.from_workload(w, inp, flags=flags)
     y = layer.prefill(inp.x.cuda())
     torch.cuda.synchronize()
@@ -374,3 +382,46 @@ def test_latent_range_is_reported(cuda_lib):
     assert e.value.code == cls.CCA_ERR_RANGE
     layer.prefill(inp.x.cuda())
     cls.cca_workspace_status(layer._ws)        # the status word is reset by every call
+
+
+# ------------------------------------------------------------------ identity convolutions
+@pytest.mark.parametrize("flags", [8 | 16, 15 | 16, 16])
+@pytest.mark.parametrize("shape", [
+    dict(d_model=512, n_heads=4, n_kv_heads=4, compression=1, seq=300),   # MHA, hd=128
+    dict(d_model=512, n_heads=4, n_kv_heads=2, compression=1, seq=257),   # GQA, hd=128
+    dict(d_model=256, n_heads=4, n_kv_heads=2, compression=2, seq=130),   # d~=32
+])
+def test_prefill_no_conv(cuda_lib, shape, flags):
+    """CCA_NO_CONV: both convolutions are the identity.  With C = 1 and RoPE alone this is
+    textbook causal MHA / GQA with rotary embeddings (the oracle's MHA reduction)."""
+    w = small("noconv", **shape)
+    inp = W.make_inputs(w, seed=7)
+    _, y = run_prefill(cuda_lib, w, inp, flags)
+    ocfg = oracle_config(w, flags)
+    ref = O.prefill(ocfg, oracle_weights(ocfg, inp, no_conv=True), f64(inp.x))
+    assert bf16_err(f64(y), ref) <= BF16_TOL
+
+
+@pytest.mark.parametrize("name", ["mha_prefill_16k", "gqa8_prefill_16k"])
+def test_baseline_prefill_sampled(cuda_lib, name):
+    """The MHA and GQA-8 baselines the benchmark times, at full size, on sampled rows."""
+    w = W.BASELINES[name]
+    inp = W.make_inputs(w, seed=0)
+    _, y = run_prefill(cuda_lib, w, inp)
+    ocfg = oracle_config(w, w.flags)
+    ow = oracle_weights(ocfg, inp, no_conv=True)
+    rng = np.random.default_rng(1)
+    b = 1
+    rows = sample_rows(w.seq, rng, n_random=128)
+    ref = O.prefill_rows(ocfg, ow, f64(inp.x[b]), rows)
+    got = f64(y[b, torch.as_tensor(rows)])
+    assert np.isfinite(got).all()
+    assert bf16_err(got, ref) <= BF16_TOL
+
+
+def test_no_conv_rejects_decode(cuda_lib):
+    cls = cuda_lib
+    cfg = cls.make_config(512, 4, 4, 1, flags=8 | 16)
+    with pytest.raises(cls.CCAError) as e:
+        cls.cca_cache_alloc(cfg, 2, 64)
+    assert e.value.code == cls.CCA_ERR_UNSUPPORTED

@@ -36,6 +36,7 @@ class Workload:
     dtype: str = "bf16"      # "f32" or "bf16"
     decode: bool = False
     description: str = ""
+    flags: int = 15          # CCA_* switches of the layer (16 = CCA_NO_CONV: identity convs)
 
     @property
     def head_dim(self) -> int:
@@ -78,6 +79,18 @@ WORKLOADS = {
                  description="CCGQA bf16 large prefill: B=1 S=32768 E=4096 H=32 Hkv=8 C=4 (d~=32)"),
         Workload("ccgqa_decode_8k", 64, 8192, 2048, 16, 4, 4, decode=True,
                  description="CCGQA bf16 decode: B=64, 8192 cached tokens, E=2048 H=16 Hkv=4 C=4 (d~=32)"),
+    ]
+}
+
+# The systems the pages compare CCA / CCGQA prefill against at 16k tokens, on the same
+# d_model, heads and batch as ccgqa_prefill_16k: multi-head attention and grouped-query
+# attention with 8 key/value heads (GQA-8), head width 128 (C = 1), RoPE only, no convs.
+BASELINES = {
+    w.name: w for w in [
+        Workload("mha_prefill_16k", 2, 16384, 2048, 16, 16, 1, flags=8 | 16,
+                 description="MHA bf16 prefill baseline: B=2 S=16384 E=2048 H=16 (hd=128), RoPE"),
+        Workload("gqa8_prefill_16k", 2, 16384, 2048, 16, 8, 1, flags=8 | 16,
+                 description="GQA-8 bf16 prefill baseline: B=2 S=16384 E=2048 H=16 Hkv=8 (hd=128), RoPE"),
     ]
 }
 
