@@ -38,7 +38,8 @@ class CCAError(RuntimeError):
 class cca_config_t(ctypes.Structure):
     _fields_ = [("d_model", c_int), ("n_heads", c_int), ("n_kv_heads", c_int),
                 ("compression", c_int), ("conv_kernel", c_int), ("chan_conv_kernel", c_int),
-                ("rope_base", c_float), ("norm_eps", c_float), ("flags", c_uint), ("dtype", c_int)]
+                ("rope_base", c_float), ("norm_eps", c_float), ("flags", c_uint), ("dtype", c_int),
+                ("tp_size", c_int), ("tp_rank", c_int)]
 
 
 class cca_weights_t(ctypes.Structure):
@@ -124,9 +125,10 @@ def _stream(stream):
 
 
 def make_config(d_model, n_heads, n_kv_heads, compression, conv_kernel=4, chan_conv_kernel=1,
-                rope_base=10000.0, norm_eps=1e-6, flags=CCA_DEFAULT_FLAGS, dtype=CCA_BF16):
+                rope_base=10000.0, norm_eps=1e-6, flags=CCA_DEFAULT_FLAGS, dtype=CCA_BF16,
+                tp_size=1, tp_rank=0):
     return cca_config_t(d_model, n_heads, n_kv_heads, compression, conv_kernel, chan_conv_kernel,
-                        rope_base, norm_eps, flags, dtype)
+                        rope_base, norm_eps, flags, dtype, tp_size, tp_rank)
 
 
 def make_weights(w_qkv, w_o, conv_seq, conv_chan) -> cca_weights_t:

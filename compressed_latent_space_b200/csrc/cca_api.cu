@@ -76,16 +76,26 @@ int make_dims(const cca_config_t *cfg, cca::Dims &d) {
   if (!(cfg->norm_eps >= 0.f)) return fail(CCA_ERR_INVALID_ARG, "norm_eps must be >= 0");
   if ((cfg->flags & CCA_ROPE) && !(cfg->rope_base > 1.f))
     return fail(CCA_ERR_INVALID_ARG, "rope_base must be > 1");
+  const int tp = cfg->tp_size <= 1 ? 1 : cfg->tp_size;
+  if (cfg->tp_size < 0 || cfg->tp_rank < 0 || cfg->tp_rank >= tp)
+    return fail(CCA_ERR_INVALID_ARG, "tp_rank %d outside [0, tp_size %d)", cfg->tp_rank, tp);
+  if (cfg->n_kv_heads % tp)
+    return fail(CCA_ERR_INVALID_ARG, "n_kv_heads %d is not a multiple of tp_size %d", cfg->n_kv_heads, tp);
   d.E = cfg->d_model;
-  d.H = cfg->n_heads;
-  d.Hkv = cfg->n_kv_heads;
+  d.H = cfg->n_heads / tp;              // this rank's heads (all of them without TP)
+  d.Hkv = cfg->n_kv_heads / tp;
   d.G = d.H / d.Hkv;
   d.DL = dl;
   d.NQ = d.H * dl;
   d.NKV = d.Hkv * dl;
   d.NQKV = d.NQ + 2 * d.NKV;
   d.KC = cfg->conv_kernel;
-  d.VS0 = d.NKV / 2;
+  {
+    // value channels >= n_kv/2 of the whole layer are shifted; this rank holds global value
+    // channels [rank * NKV, (rank + 1) * NKV)
+    const int vs = cfg->n_kv_heads * dl / 2 - (tp > 1 ? cfg->tp_rank : 0) * d.NKV;
+    d.VS0 = vs < 0 ? 0 : vs > d.NKV ? d.NKV : vs;
+  }
   d.flags = cfg->flags;
   d.eps = cfg->norm_eps;
   d.rope_base = cfg->rope_base;

@@ -657,9 +657,9 @@ cudaError_t launch(const Dims &d, const StencilArgs &a, cudaStream_t st) {
 // Q-K-Mean (whose pre- and post-conv terms then coincide), value-shift, RMS norm and RoPE as
 // selected.  With C = 1 and only RoPE on, this is the projection-to-attention step of plain
 // multi-head (or grouped-query) attention with rotary embeddings, for any latent width up to
-// 128.  One warp per (token, head) item, reading its P row segment straight from global
-// memory (lane i holds channels i and i + d~/2, the RoPE pair, of the row); no shared memory,
-// so many warps per SM hide the load latency of this memory-bound pass.
+// 128.  One CTA per token, one warp per (token, head) item, reading its P row segment straight
+// from global memory (lane i holds channels i and i + d~/2, the RoPE pair, of the row); no
+// shared memory, so many warps per SM hide the load latency of this memory-bound pass.
 template <typename T>
 struct PointParams {
   using TL = typename LatentType<T>::type;
@@ -675,17 +675,13 @@ struct PointParams {
 template <typename T>
 __global__ void __launch_bounds__(256) pointwise_kernel(const PointParams<T> p) {
   using TL = typename LatentType<T>::type;
-  const int lane = threadIdx.x & 31;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
   const int per_tok = p.H + 2 * p.Hkv;
-  const long long items = static_cast<long long>(p.B) * p.S * per_tok;
-  const long long nwarps = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
   const int DL = p.DL, HALF = DL / 2;
-  for (long long it = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
-       it < items; it += nwarps) {
-    const long long bt = it / per_tok;               // b * S + t
-    const int hh = static_cast<int>(it % per_tok);
-    const int b = static_cast<int>(bt / p.S), t = static_cast<int>(bt % p.S);
-    const float *row = p.P + bt * p.NQKV;
+  const int bt = blockIdx.x;                         // one CTA per token: b * S + t
+  const int b = bt / p.S, t = bt - b * p.S;
+  const float *row = p.P + static_cast<size_t>(bt) * p.NQKV;
+  for (int hh = warp; hh < per_tok; hh += nwarps) {
     if (hh < p.H + p.Hkv) {                         // a query or key head
       const bool is_q = hh < p.H;
       const int g = is_q ? hh / p.G : hh - p.H;
@@ -777,11 +773,9 @@ cudaError_t launch_pointwise(const Dims &d, const StencilArgs &a, cudaStream_t s
   p.eps = d.eps;
   for (int i = 0; i < 64; ++i)
     p.theta[i] = i < d.DL / 2 ? pow(static_cast<double>(d.rope_base), -2.0 * i / d.DL) : 0.0;
-  const long long items = static_cast<long long>(d.B) * d.S * (d.H + 2 * d.Hkv);
-  long long blocks = (items + 7) / 8;
-  const long long cap = static_cast<long long>(num_sms()) * 8 * 16;   // a grid-stride loop beyond
-  if (blocks > cap) blocks = cap;
-  pointwise_kernel<T><<<static_cast<unsigned>(blocks), 256, 0, st>>>(p);
+  const int per_tok = d.H + 2 * d.Hkv;
+  const int threads = per_tok >= 8 ? 256 : 32 * per_tok;   // a warp per (token, head) item
+  pointwise_kernel<T><<<static_cast<unsigned>(d.B * d.S), threads, 0, st>>>(p);
   return cudaGetLastError();
 }
 

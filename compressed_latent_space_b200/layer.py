@@ -29,17 +29,18 @@ class Cache:
 
         c = layer.cfg
         dl = layer.dl
-        self.k = view(self.struct.k, batch * c.n_kv_heads * max_seq * dl, layer.latent_dtype, es,
-                      (batch, c.n_kv_heads, max_seq, dl))
-        self.v = view(self.struct.v, batch * c.n_kv_heads * max_seq * dl, layer.latent_dtype, es,
-                      (batch, c.n_kv_heads, max_seq, dl))
+        hkv = layer.n_kv_heads_local
+        self.k = view(self.struct.k, batch * hkv * max_seq * dl, layer.latent_dtype, es,
+                      (batch, hkv, max_seq, dl))
+        self.v = view(self.struct.v, batch * hkv * max_seq * dl, layer.latent_dtype, es,
+                      (batch, hkv, max_seq, dl))
         kc1 = c.conv_kernel - 1
         if kc1 > 0:
             self.conv_state = view(self.struct.conv_state, batch * kc1 * (layer.n_q + layer.n_kv),
                                    torch.float32, 4, (batch, kc1, layer.n_q + layer.n_kv))
         else:
             self.conv_state = None
-        half = layer.n_kv - layer.n_kv // 2
+        half = layer.n_kv - layer.vshift_begin
         self.vshift_state = view(self.struct.vshift_state, batch * half, torch.float32, 4,
                                  (batch, half))
         self.lengths = view(self.struct.lengths, batch, torch.int32, 4, (batch,))
@@ -48,17 +49,26 @@ class Cache:
 class CCALayer:
     def __init__(self, d_model, n_heads, n_kv_heads, compression, w_qkv, w_o, conv_seq, conv_chan,
                  conv_kernel=4, rope_base=10000.0, norm_eps=1e-6, flags=CCA_DEFAULT_FLAGS,
-                 dtype="bf16", device="cuda"):
+                 dtype="bf16", device="cuda", tp_size=1, tp_rank=0):
+        """Global layer shape; with tp_size > 1 the weights are rank tp_rank's slices (see
+        compressed_latent_space_b200.tp) and prefill / decode return its share of y."""
         self.dtype = torch.bfloat16 if dtype == "bf16" else torch.float32
         # latent q, k, v and the K/V cache: float16 in 16-bit layers, float32 otherwise
         self.latent_dtype = torch.float16 if dtype == "bf16" else torch.float32
         self.esize = 2 if dtype == "bf16" else 4
         self.device = torch.device(device)
         self.cfg = make_config(d_model, n_heads, n_kv_heads, compression, conv_kernel, 1, rope_base,
-                               norm_eps, flags, CCA_BF16 if dtype == "bf16" else CCA_F32)
+                               norm_eps, flags, CCA_BF16 if dtype == "bf16" else CCA_F32,
+                               tp_size, tp_rank)
+        tp = max(tp_size, 1)
         self.dl = d_model // n_heads // compression
-        self.n_q = n_heads * self.dl
-        self.n_kv = n_kv_heads * self.dl
+        self.n_heads_local = n_heads // tp
+        self.n_kv_heads_local = n_kv_heads // tp
+        self.n_q = self.n_heads_local * self.dl
+        self.n_kv = self.n_kv_heads_local * self.dl
+        # first value channel of this rank taken from the previous token (the layer's split
+        # at n_kv/2 of all key/value heads, in this rank's channel numbering)
+        self.vshift_begin = min(max(n_kv_heads * self.dl // 2 - tp_rank * self.n_kv, 0), self.n_kv)
         self.w_qkv = w_qkv.to(self.device, self.dtype).contiguous()
         self.w_o = w_o.to(self.device, self.dtype).contiguous()
         # CCA_NO_CONV layers take no conv filters

@@ -95,7 +95,25 @@ typedef struct {
   float norm_eps;
   unsigned flags;
   int dtype;                /* cca_dtype_t */
+  int tp_size;              /* tensor-parallel ranks sharing the layer (0 or 1: none)       */
+  int tp_rank;              /* this rank, 0 <= tp_rank < tp_size                            */
 } cca_config_t;
+
+/* Tensor parallelism by key/value group (gist.science explainer, 5. Significance and
+ * Implications, Scalability: the method works with tensor parallelism).  Every step before the
+ * up-projection is local to a key/value group (the channel conv is per head, Q-K-Mean pairs a
+ * query head with its group's key head, attention reads only its group), so with
+ * tp_size = R (Hkv % R == 0) rank r holds query heads [r H/R, (r+1) H/R) and key/value heads
+ * [r Hkv/R, (r+1) Hkv/R) and computes them alone.  All sizes (workspace, cache, decode) are
+ * then the rank's own, and the weights passed are the rank's slices:
+ *   w_qkv     its query rows, then its key rows, then its value rows (of the global W_q, W_k, W_v)
+ *   w_o       [E, n_q / R]: its columns of the global W_o
+ *   conv_seq  its query channels' rows, then its key channels' rows
+ *   conv_chan its query heads' filters, then its key heads' filters
+ * y is the rank's share of the up-projection; the layer's output is the sum of y over the
+ * ranks (one all-reduce of [tokens, E], done by the caller).  The value-shift keeps the
+ * global split: value channel c of the layer comes from the previous token when
+ * c >= n_kv / 2 of the whole layer, whichever rank holds it. */
 
 /* Layer parameters (device pointers).
  *   w_qkv     [n_q + 2*n_kv, E]  rows: W_q (n_q = H*d~), W_k (n_kv = Hkv*d~), W_v
