@@ -194,12 +194,16 @@ def bench_prefill(cls, w, steps, warmup, world, seed, e2e=True):
     stage_ms, calls = cls.cca_stage_times(8)
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     ms = statistics.median(step_ms)
-    stages = {n: t / max(calls, 1) for n, t in
-              zip(["weights_to_16bit", "qkv_projection", "latent_stencil", "latent_attention",
-                   "out_projection"], stage_ms)}
+    names = (["weights_to_16bit", "qkv_projection", "latent_stencil", "latent_attention",
+              "out_projection"] if len(stage_ms) == 5 else
+             ["weights_to_16bit", "qkv_projection_stencil", "latent_attention", "out_projection"])
+    stages = {n: t / max(calls, 1) for n, t in zip(names, stage_ms)}
+    # kernels per forward: one per timed slot, plus the channel-filter split that shares the
+    # first slot with the W_o conversion (layers with convolutions)
+    per_step = len(stage_ms) + (0 if w.flags & 16 else 1)
 
     if not e2e:
-        return dict(ms=ms, stages=stages, calls=calls, launches=6 * steps)
+        return dict(ms=ms, stages=stages, calls=calls, launches=per_step * steps)
 
     # end to end through the public API, the way a server would overlap the copies: each
     # sequence's x goes host -> device on one copy stream, its forward runs on the compute
@@ -243,7 +247,7 @@ def bench_prefill(cls, w, steps, warmup, world, seed, e2e=True):
     e2e_ms = statistics.median(s.elapsed_time(e) for s, e in zip(e2e_s, e2e_e))
     nbytes = x.numel() * x.element_size()
     return dict(ms=ms, stages=stages, calls=calls, e2e_ms=e2e_ms, h2d=nbytes, d2h=nbytes,
-                launches=6 * steps)
+                launches=per_step * steps)
 
 
 # Decode steps rotate over this many independent layers (weights and caches), in the order a
@@ -475,7 +479,7 @@ def bench_baselines(cls, steps, warmup, world, seed, ccgqa_ms):
     out = {}
     for name, w in W.BASELINES.items():
         r = bench_prefill(cls, w, steps, warmup, world, seed, e2e=False)
-        out[name] = {"description": w.description, "ms_per_step": r["ms"],
+        out[name] = {"description": w.description, "ms_per_step": r["ms"], "launches": r["launches"],
                      "tokens_per_s": job_throughput(w.batch * w.seq, world, r["ms"]),
                      "tflops": prefill_flops(w) / (r["ms"] * 1e-3) / 1e12,
                      "attention_tflops": attention_flops(w) / (r["stages"]["latent_attention"] * 1e-3) / 1e12,
@@ -513,7 +517,7 @@ def run_cuda(args):
         for name in W.BASELINES:
             base[name]["ms_per_step"] = max_over_ranks(base[name]["ms_per_step"], world)
         line["baselines"] = base
-        line["gpu_launches"] += sum(6 * args.steps for _ in W.BASELINES)
+        line["gpu_launches"] += sum(base[name]["launches"] for name in W.BASELINES)
     line["clocks"] = clk.summary()
     peak_clk = measured_peak_clock()
     if peak_clk and line["clocks"].get("sm_mhz"):

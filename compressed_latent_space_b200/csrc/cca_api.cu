@@ -37,6 +37,22 @@ int ok() {
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
+// Which kernels a 16-bit prefill with the convolutions uses for the down-projection and the
+// stencil.  The fused kernel keeps P on chip but runs its stencil epilogue between tiles (its
+// 384-column accumulator leaves no room for a second one in tensor memory); measured on B200 it
+// wins where one CTA packs four or more key/value groups (small groups, where the separate
+// stencil kernel spreads thinly: cca_prefill_4k 0.39 -> 0.25 ms) and loses ~7 % at four query
+// heads per group (ccgqa_prefill_16k / _32k).  CCA_PREFILL_PATH=fused or =unfused overrides the
+// choice (for comparing the two paths).
+bool use_fused(const cca::Dims &d) {
+  const int ng = cca::fused_group_set(d);
+  if (ng == 0) return false;
+  const char *f = getenv("CCA_PREFILL_PATH");
+  if (f && strcmp(f, "fused") == 0) return true;
+  if (f && strcmp(f, "unfused") == 0) return false;
+  return ng >= 4;
+}
+
 // Host-side fault injection for the error paths: CCA_FAULT_INJECT=launch makes every call
 // that would launch kernels fail with CCA_ERR_CUDA before touching the device.
 bool injected_launch_failure() {
@@ -368,22 +384,56 @@ CCA_API int cca_prefill_forward(const cca_config_t *cfg, const cca_weights_t *w,
   const int M = batch * seq;
   CallRecorder rec(st);
   rec.mark();
+  // The projection fused with the stencil where the kernel supports the shape (16-bit layers
+  // with the convolutions); P then never reaches global memory.
+  const bool fused = d.bf16 && !no_conv && use_fused(d);
   // 16-bit layers: the up-projection runs on float16 operands (the attention output is
   // float16), so W_o is converted once per call.
   void *wo = const_cast<void *>(w->w_o);
+  char *fhi = ws + L.wsplit, *flo = fhi + static_cast<size_t>(d.H + d.Hkv) * d.DL * d.DL * 2;
   if (d.bf16) {
     wo = ws + L.wo16;
     if ((e = cca::convert_bf16_to_f16(w->w_o, wo, static_cast<size_t>(d.E) * d.NQ, status, st)) !=
         cudaSuccess)
       return cuda_fail(e, "W_o conversion launch");
-    if (!no_conv && (e = cca::split_conv_chan(d, w->conv_chan, ws + L.wsplit, st)) != cudaSuccess)
-      return cuda_fail(e, "channel-conv weight split launch");
+    if (fused)
+      e = cca::split_filter_planes(d, w->conv_chan, fhi, flo, st);
+    else if (!no_conv)
+      e = cca::split_conv_chan(d, w->conv_chan, ws + L.wsplit, st);
+    if (e != cudaSuccess) return cuda_fail(e, "channel-conv weight split launch");
   }
   rec.mark();
   void *P = ws + L.P, *q = ws + L.q, *o = ws + L.o;
   void *k = cache ? cache->k : ws + L.k;
   void *v = cache ? cache->v : ws + L.v;
   const int kv_stride = cache ? cache->max_seq : seq;
+
+  if (fused) {
+    cca::FusedArgs fa;
+    fa.x = x;
+    fa.w_qkv = w->w_qkv;
+    fa.conv_seq = w->conv_seq;
+    fa.filt_hi = fhi;
+    fa.filt_lo = flo;
+    fa.q = q;
+    fa.k = k;
+    fa.v = v;
+    fa.kv_stride = kv_stride;
+    fa.conv_state = cache ? static_cast<float *>(cache->conv_state) : nullptr;
+    fa.vshift_state = cache ? static_cast<float *>(cache->vshift_state) : nullptr;
+    fa.lengths = cache ? cache->lengths : nullptr;
+    fa.write_state = cache != nullptr;
+    fa.status = status;
+    if ((e = cca::fused_qkv_stencil(d, fa, st)) != cudaSuccess)
+      return cuda_fail(e, "fused projection + stencil launch");
+    rec.mark();
+    if ((e = cca::latent_attention(d, q, k, v, kv_stride, o, status, st)) != cudaSuccess)
+      return cuda_fail(e, "attention launch");
+    rec.mark();
+    if ((rc = gemm_dispatch(CCA_F16, 0, o, wo, y, M, d.E, d.NQ, status, st))) return rc;
+    rec.mark();
+    return ok();
+  }
 
   const int dt = d.bf16 ? CCA_BF16 : CCA_F32;
   if ((rc = gemm_dispatch(dt, 1, x, w->w_qkv, P, M, d.NQKV, d.E, status, st))) return rc;

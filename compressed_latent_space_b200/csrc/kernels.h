@@ -68,6 +68,29 @@ cudaError_t latent_stencil(const Dims &d, const StencilArgs &a, cudaStream_t st)
 size_t conv_chan_split_bytes(const Dims &d);
 cudaError_t split_conv_chan(const Dims &d, const float *conv_chan, void *out, cudaStream_t st);
 
+// Down-projection fused with the latent stencil (16-bit layers): x [B, S, E] and W_qkv ->
+// q, k, v as latent_stencil writes them (and the decode state with write_state), without P
+// ever reaching global memory.  fused_group_set: the key/value groups one CTA takes (0 when
+// the shape is not supported by the fused kernel).  filt_hi / filt_lo: the channel filters as
+// bf16 leading terms and remainders, [(H + Hkv) * DL, DL] each (split_filter_planes, into
+// fused_filter_bytes of scratch).
+struct FusedArgs {
+  const void *x, *w_qkv;
+  const float *conv_seq;
+  const void *filt_hi, *filt_lo;
+  void *q, *k, *v;
+  int kv_stride;
+  float *conv_state, *vshift_state;
+  int *lengths;
+  bool write_state;
+  int *status;
+};
+int fused_group_set(const Dims &d);
+size_t fused_filter_bytes(const Dims &d);
+cudaError_t split_filter_planes(const Dims &d, const float *conv_chan, void *hi, void *lo,
+                                cudaStream_t st);
+cudaError_t fused_qkv_stencil(const Dims &d, const FusedArgs &a, cudaStream_t st);
+
 // Causal latent attention: q [B, H, S, DL], k/v [B, Hkv, kv_stride, DL] -> o [B*S, NQ].
 cudaError_t latent_attention(const Dims &d, const void *q, const void *k, const void *v,
                              int kv_stride, void *o, int *status, cudaStream_t st);

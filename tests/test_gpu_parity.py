@@ -425,3 +425,41 @@ def test_no_conv_rejects_decode(cuda_lib):
     with pytest.raises(cls.CCAError) as e:
         cls.cca_cache_alloc(cfg, 2, 64)
     assert e.value.code == cls.CCA_ERR_UNSUPPORTED
+
+
+# ------------------------------------------------------------------ fused projection + stencil
+@pytest.mark.parametrize("shape", [
+    dict(d_model=512, n_heads=8, n_kv_heads=2, compression=1, seq=300),     # d~=64, G=4, NG=1
+    dict(d_model=512, n_heads=8, n_kv_heads=4, compression=2, seq=250),     # d~=32, G=2
+    dict(d_model=256, n_heads=4, n_kv_heads=4, compression=4, seq=131),     # d~=16, G=1, NG=4
+    dict(d_model=512, n_heads=16, n_kv_heads=4, compression=1, seq=129, conv_kernel=6),
+    dict(d_model=512, n_heads=16, n_kv_heads=8, compression=1, seq=64, conv_kernel=1),
+])
+def test_prefill_fused_and_unfused_paths(cuda_lib, shape, monkeypatch):
+    """The fused down-projection + stencil kernel and the separate GEMM + stencil kernels both
+    match the oracle (and each other) on the same inputs, with a cache (decode state) too."""
+    w = small("fused", **shape)
+    inp = W.make_inputs(w, seed=12, conv_std=0.4, identity_conv=True)
+    ocfg = oracle_config(w)
+    ow = oracle_weights(ocfg, inp)
+    ref = O.prefill(ocfg, ow, f64(inp.x))
+    outs = []
+    for unfused in ("fused", "unfused"):
+        monkeypatch.setenv("CCA_PREFILL_PATH", unfused)
+        layer = cuda_lib.CCALayer.from_workload(w, inp)
+        cache = layer.new_cache(w.batch, w.seq + 8)
+        y = layer.prefill(inp.x.cuda(), cache=cache)
+        torch.cuda.synchronize()
+        cuda_lib.cca_workspace_status(layer._ws)
+        assert bf16_err(f64(y), ref) <= BF16_TOL, unfused
+        for b in range(w.batch):
+            _, st = O.prefill_sequence(ocfg, ow, f64(inp.x[b]))
+            S = w.seq
+            assert bf16_err(f64(cache.k[b, :, :S]).transpose(1, 0, 2).reshape(S, -1), st.k_cache) <= BF16_TOL
+            assert bf16_err(f64(cache.v[b, :, :S]).transpose(1, 0, 2).reshape(S, -1), st.v_cache) <= BF16_TOL
+            if w.conv_kernel > 1:
+                assert bf16_err(f64(cache.conv_state[b]), st.conv_state) <= BF16_TOL
+            assert bf16_err(f64(cache.vshift_state[b]), st.vshift_state) <= BF16_TOL
+        assert cache.lengths.tolist() == [w.seq] * w.batch
+        outs.append(f64(y))
+    assert bf16_err(outs[0], outs[1]) <= BF16_TOL
