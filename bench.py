@@ -471,6 +471,49 @@ def result_line(w, world, steps, warmup, pre, ms, e2e_ms, dec, dms, peaks):
     return line
 
 
+def backward_flops(w) -> float:
+    """Algorithmic flops of one backward pass: twice the forward projections' (the input and
+    the weight gradient of each GEMM) and 2.5x the forward attention's (dS and dP, dQ, dK, dV:
+    five S x S x d~ products against the forward's two), counted once each."""
+    tokens = w.batch * w.seq
+    proj = 2.0 * tokens * w.d_model * (w.n_q + 2 * w.n_kv) + 2.0 * tokens * w.n_q * w.d_model
+    return 2.0 * proj + 2.5 * attention_flops(w)
+
+
+def bench_backward(cls, w, steps, warmup, seed):
+    """cca_backward on the workload (forward intermediates recomputed inside), median step."""
+    inp = W.make_inputs(w, seed=seed)
+    layer = cls.CCALayer.from_workload(w, inp)
+    x = inp.x.cuda()
+    dy = torch.randn(x.shape, generator=torch.Generator("cpu").manual_seed(seed + 1)).to(x.dtype).cuda()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    for _ in range(warmup):
+        layer.backward(x, dy)
+    torch.cuda.synchronize()
+    cls.cca_stage_timing(True)
+    times = []
+    for i in range(steps):
+        flush.fill_(i & 0xFF)
+        s0 = torch.cuda.Event(enable_timing=True)
+        e0 = torch.cuda.Event(enable_timing=True)
+        s0.record()
+        layer.backward(x, dy)
+        e0.record()
+        times.append((s0, e0))
+    torch.cuda.synchronize()
+    cls.cca_stage_timing(False)
+    stage_ms, calls = cls.cca_stage_times(8)
+    cls.cca_workspace_status(layer._ws)
+    ms = statistics.median(s.elapsed_time(e) for s, e in times)
+    names = ["forward_recompute", "dO_and_rowsum", "attention_backward", "stencil_backward",
+             "gradient_gemms"]
+    return {"workload": w.name, "ms_per_step": ms, "tokens_per_s": w.batch * w.seq / (ms * 1e-3),
+            "tflops": backward_flops(w) / (ms * 1e-3) / 1e12,
+            "flops_counted": "2x forward projections + 2.5x forward attention (algorithmic)",
+            "stages_ms": {n: t / max(calls, 1) for n, t in zip(names, stage_ms)},
+            "launches": 19 * steps}
+
+
 def bench_baselines(cls, steps, warmup, world, seed, ccgqa_ms):
     """The systems the pages compare CCA / CCGQA prefill with at 16k tokens (MHA and GQA-8,
     head width 128, RoPE, same d_model / heads / batch as the CCGQA workload), run on this
@@ -508,11 +551,18 @@ def run_cuda(args):
         base = None
         if not args.no_baselines and w.name == DEFAULT_WORKLOAD:
             base = bench_baselines(cls, args.steps, args.warmup, world, rank, pre["ms"])
+        bwd = None
+        if not args.no_backward and w.dtype == "bf16" and not (w.flags & 16):
+            bwd = bench_backward(cls, w, max(3, args.steps // 2), args.warmup, rank)
     ms = max_over_ranks(pre["ms"], world)
     e2e_ms = max_over_ranks(pre["e2e_ms"], world)
     dms = max_over_ranks(dec["ms"], world) if dec else None
     line = result_line(w, world, args.steps, args.warmup, pre, ms, e2e_ms, dec, dms,
                        measured_peaks())
+    if bwd:
+        bwd["ms_per_step"] = max_over_ranks(bwd["ms_per_step"], world)
+        line["backward"] = bwd
+        line["gpu_launches"] += bwd["launches"]
     if base:
         for name in W.BASELINES:
             base[name]["ms_per_step"] = max_over_ranks(base[name]["ms_per_step"], world)
@@ -571,6 +621,7 @@ def main():
                     help="independent layers the decode steps rotate over (fewer for profiling "
                          "captures that must stay small; the timing needs the default)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-backward", action="store_true", help="skip the backward-pass timing")
     ap.add_argument("--no-baselines", action="store_true",
                     help="skip the same-box MHA / GQA-8 prefill baselines")
     ap.add_argument("--cpu-full", action="store_true",

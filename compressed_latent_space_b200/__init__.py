@@ -80,6 +80,10 @@ _SIGS = {
     "cca_decode_step_static": (c_int, [POINTER(cca_config_t), POINTER(cca_weights_t), c_void_p,
                                        c_void_p, POINTER(cca_cache_t), c_void_p]),
     "cca_stage_wait_probe": (c_int, [ctypes.c_longlong, c_int, c_void_p, c_void_p]),
+    "cca_backward_workspace_size": (c_size_t, [POINTER(cca_config_t), c_int, c_int]),
+    "cca_backward": (c_int, [POINTER(cca_config_t), POINTER(cca_weights_t), c_void_p, c_void_p,
+                             c_int, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                             c_void_p, c_size_t, c_void_p]),
     "cca_stage_timing": (c_int, [c_int]),
     "cca_stage_times": (c_int, [POINTER(ctypes.c_double), c_int, POINTER(c_int)]),
 }
@@ -187,6 +191,18 @@ def cca_decode_step_static(cfg, weights, x, y, cache, stream=None):
     """Decode step whose scratch is the library's built-in device array (no workspace)."""
     _check(load().cca_decode_step_static(ctypes.byref(cfg), ctypes.byref(weights), _ptr(x), _ptr(y),
                                          ctypes.byref(cache), _stream(stream)))
+
+
+def cca_backward_workspace_size(cfg: cca_config_t, batch: int, seq: int) -> int:
+    return load().cca_backward_workspace_size(ctypes.byref(cfg), batch, seq)
+
+
+def cca_backward(cfg, weights, x, dy, batch, seq, dx, dw_qkv, dw_o, dconv_seq, dconv_chan,
+                 workspace, stream=None):
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(load().cca_backward(ctypes.byref(cfg), ctypes.byref(weights), _ptr(x), _ptr(dy), batch,
+                               seq, _ptr(dx), _ptr(dw_qkv), _ptr(dw_o), _ptr(dconv_seq),
+                               _ptr(dconv_chan), _ptr(workspace), ws_bytes, _stream(stream)))
 
 
 def cca_cache_check(cache, stream=None):

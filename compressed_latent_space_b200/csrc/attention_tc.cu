@@ -132,7 +132,8 @@ __global__ void __launch_bounds__(AttnCfg<DL>::THREADS, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap mapQ,
                    const __grid_constant__ CUtensorMap mapK,
                    const __grid_constant__ CUtensorMap mapV, __half *__restrict__ O, int S,
-                   int H, int Hkv, int G, int gp_log2, int nqt, float scale_log2, int *status) {
+                   int H, int Hkv, int G, int gp_log2, int nqt, float scale_log2, int *status,
+                   float *__restrict__ lse) {
   using C = AttnCfg<DL>;
   constexpr int NTILE = C::NTILE;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -385,6 +386,10 @@ __global__ void __launch_bounds__(AttnCfg<DL>::THREADS, 1)
         u.w = pack_f16x2(__uint_as_float(o[6]) * inv, __uint_as_float(o[7]) * inv);
         if (qpos < S) reinterpret_cast<uint4 *>(dst)[c] = u;
       }
+      // log2-domain log-sum-exp of the row's scaled scores, for the backward pass:
+      // p = 2^(s * scale * log2(e) - lse) are the row's probabilities
+      if (lse && qpos < S)
+        lse[(static_cast<size_t>(b) * H + hrow) * S + qpos] = m_ref + log2f(l);
     }
   }
 
@@ -407,7 +412,7 @@ inline int pack_log2(int G) {
 
 template <int DL>
 cudaError_t launch_tc(const Dims &d, const void *q, const void *k, const void *v, int kv_stride,
-                      void *o, float scale_log2, int *status, cudaStream_t st) {
+                      void *o, float scale_log2, int *status, cudaStream_t st, float *lse) {
   using C = AttnCfg<DL>;
   const int gpl = pack_log2(d.G);
   const int GP = 1 << gpl, TT = TM >> gpl;
@@ -436,19 +441,19 @@ cudaError_t launch_tc(const Dims &d, const void *q, const void *k, const void *v
   dim3 grid(d.H / GP, d.B, (nqt + C::NTILE - 1) / C::NTILE);
   attn_tc_kernel<DL><<<grid, C::THREADS, C::SMEM, st>>>(mq, mk, mv, static_cast<__half *>(o), d.S,
                                                         d.H, d.Hkv, d.G, gpl, nqt, scale_log2,
-                                                        status);
+                                                        status, lse);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t latent_attention_tc(const Dims &d, const void *q, const void *k, const void *v,
-                                int kv_stride, void *o, int *status, cudaStream_t st) {
+                                int kv_stride, void *o, int *status, cudaStream_t st, float *lse) {
   const float scale_log2 = static_cast<float>(1.4426950408889634 / sqrt(static_cast<double>(d.DL)));
-  if (d.DL == 16) return launch_tc<16>(d, q, k, v, kv_stride, o, scale_log2, status, st);
-  if (d.DL == 32) return launch_tc<32>(d, q, k, v, kv_stride, o, scale_log2, status, st);
-  if (d.DL == 64) return launch_tc<64>(d, q, k, v, kv_stride, o, scale_log2, status, st);
-  if (d.DL == 128) return launch_tc<128>(d, q, k, v, kv_stride, o, scale_log2, status, st);
+  if (d.DL == 16) return launch_tc<16>(d, q, k, v, kv_stride, o, scale_log2, status, st, lse);
+  if (d.DL == 32) return launch_tc<32>(d, q, k, v, kv_stride, o, scale_log2, status, st, lse);
+  if (d.DL == 64) return launch_tc<64>(d, q, k, v, kv_stride, o, scale_log2, status, st, lse);
+  if (d.DL == 128) return launch_tc<128>(d, q, k, v, kv_stride, o, scale_log2, status, st, lse);
   return cudaErrorInvalidValue;
 }
 

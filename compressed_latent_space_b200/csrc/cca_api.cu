@@ -463,6 +463,177 @@ CCA_API int cca_prefill_forward(const cca_config_t *cfg, const cca_weights_t *w,
   return ok();
 }
 
+}  // extern "C"
+
+namespace {
+// ------------------------------------------------------------------ backward pass
+struct BackwardLayout {
+  size_t status, wsplit, P, q, k, v, o, lse, D, woT, dO, dyT, oT, dq, dk, dv, dA, dPpart, dP,
+      wqkvT, dPT, xT, total;
+};
+
+BackwardLayout backward_layout(const cca::Dims &d, int B, int S) {
+  BackwardLayout L;
+  const size_t M = static_cast<size_t>(B) * S, M8 = (M + 7) & ~static_cast<size_t>(7);
+  const size_t rows = static_cast<size_t>(B) * d.H * S;
+  size_t off = 0;
+  auto take = [&](size_t bytes) { const size_t o = off; off += align256(bytes); return o; };
+  L.status = take(256);
+  L.wsplit = take(cca::conv_chan_split_bytes(d));
+  L.P = take(M * d.NQKV * 4);
+  L.q = take(M * d.NQ * 2);
+  L.k = take(M * d.NKV * 2);
+  L.v = take(M * d.NKV * 2);
+  L.o = take(M * d.NQ * 2);
+  L.lse = take(rows * 4);
+  L.D = take(rows * 4);
+  L.woT = take(static_cast<size_t>(d.NQ) * d.E * 2);
+  L.dO = take(M * d.NQ * 2);
+  L.dyT = take(static_cast<size_t>(d.E) * M8 * 2);
+  L.oT = take(static_cast<size_t>(d.NQ) * M8 * 2);
+  L.dq = take(M * d.NQ * 4);
+  L.dk = take(M * d.NKV * 4);
+  L.dv = take(M * d.NKV * 4);
+  L.dA = take(M * (d.NQ + d.NKV) * 4);
+  L.dPpart = take(M * d.NQKV * 4);
+  L.dP = take(M * d.NQKV * 2);
+  L.wqkvT = take(static_cast<size_t>(d.E) * d.NQKV * 2);
+  L.dPT = take(static_cast<size_t>(d.NQKV) * M8 * 2);
+  L.xT = take(static_cast<size_t>(d.E) * M8 * 2);
+  L.total = off;
+  return L;
+}
+
+int check_backward_shape(const cca::Dims &d) {
+  if (!d.bf16) return fail(CCA_ERR_UNSUPPORTED, "the backward pass runs bfloat16 layers");
+  if (!cca::stencil_backward_supported(d))
+    return fail(CCA_ERR_UNSUPPORTED, "backward pass: needs the convolutions, latent width <= 64 "
+                "and (H/Hkv + 1) * d~^2 <= 20480");
+  if (d.E % 8) return fail(CCA_ERR_UNSUPPORTED, "backward pass: d_model must be a multiple of 8");
+  return CCA_OK;
+}
+}  // namespace
+
+extern "C" {
+
+CCA_API size_t cca_backward_workspace_size(const cca_config_t *cfg, int batch, int seq) {
+  cca::Dims d;
+  if (make_dims(cfg, d) || check_backward_shape(d) || batch < 0 || seq < 0) return 0;
+  return backward_layout(d, batch, seq).total;
+}
+
+CCA_API int cca_backward(const cca_config_t *cfg, const cca_weights_t *w, const void *x,
+                         const void *dy, int batch, int seq, void *dx, float *dw_qkv,
+                         float *dw_o, float *dconv_seq, float *dconv_chan, void *workspace,
+                         size_t ws_bytes, void *stream) {
+  cca::Dims d;
+  int rc = make_dims(cfg, d);
+  if (rc) return rc;
+  if ((rc = check_backward_shape(d))) return rc;
+  if (!w || !w->w_qkv || !w->w_o || !w->conv_seq || !w->conv_chan)
+    return fail(CCA_ERR_INVALID_ARG, "weights (or one of their pointers) NULL");
+  if (batch <= 0 || seq <= 0) return fail(CCA_ERR_INVALID_ARG, "batch and seq must be positive");
+  if (!x || !dy || !dx || !dw_qkv || !dw_o || !dconv_seq || !dconv_chan)
+    return fail(CCA_ERR_INVALID_ARG, "x, dy or an output NULL");
+  if (static_cast<long long>(batch) * seq > (1LL << 31) / 4)
+    return fail(CCA_ERR_UNSUPPORTED, "batch*seq %lld too large", static_cast<long long>(batch) * seq);
+  if (!aligned16(x) || !aligned16(dy) || !aligned16(dx) || !aligned16(dw_qkv) || !aligned16(dw_o) ||
+      !aligned16(w->w_qkv) || !aligned16(w->w_o) || !aligned16(workspace))
+    return fail(CCA_ERR_ALIGNMENT, "tensors and workspace must be 16-byte aligned");
+  d.B = batch;
+  d.S = seq;
+  const BackwardLayout L = backward_layout(d, batch, seq);
+  if (!workspace || ws_bytes < L.total)
+    return fail(CCA_ERR_WORKSPACE, "workspace of %zu bytes, %zu needed", workspace ? ws_bytes : 0, L.total);
+  if (injected_launch_failure()) return fail(CCA_ERR_CUDA, "injected launch failure");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char *ws = static_cast<char *>(workspace);
+  int *status = reinterpret_cast<int *>(ws + L.status);
+  const int M = batch * seq, M8 = (M + 7) & ~7;
+  cudaError_t e = cudaMemsetAsync(status, 0, 256, st);
+  if (e == cudaSuccess)
+    e = cudaMemsetAsync(dconv_seq, 0, static_cast<size_t>(d.NQ + d.NKV) * d.KC * 4, st);
+  if (e == cudaSuccess)
+    e = cudaMemsetAsync(dconv_chan, 0, static_cast<size_t>(d.H + d.Hkv) * d.DL * d.DL * 4, st);
+  if (e != cudaSuccess) return cuda_fail(e, "backward set-up");
+  CallRecorder rec(st);
+  rec.mark();
+  // forward recomputation: projections (kept), latents, attention output and log-sum-exp
+  void *P = ws + L.P, *q = ws + L.q, *k = ws + L.k, *v = ws + L.v, *o = ws + L.o;
+  float *lse = reinterpret_cast<float *>(ws + L.lse), *Dd = reinterpret_cast<float *>(ws + L.D);
+  if ((rc = gemm_dispatch(CCA_BF16, 1, x, w->w_qkv, P, M, d.NQKV, d.E, status, st))) return rc;
+  if ((e = cca::split_conv_chan(d, w->conv_chan, ws + L.wsplit, st)) != cudaSuccess)
+    return cuda_fail(e, "channel-conv weight split launch");
+  cca::StencilArgs sa{};
+  sa.P = static_cast<const float *>(P);
+  sa.conv_seq = w->conv_seq;
+  sa.conv_chan = w->conv_chan;
+  sa.conv_chan_split = ws + L.wsplit;
+  sa.q = q;
+  sa.k = k;
+  sa.v = v;
+  sa.kv_stride = seq;
+  sa.status = status;
+  if ((e = cca::latent_stencil(d, sa, st)) != cudaSuccess) return cuda_fail(e, "stencil launch");
+  if ((e = cca::latent_attention_tc(d, q, k, v, seq, o, status, st, lse)) != cudaSuccess)
+    return cuda_fail(e, "attention launch");
+  rec.mark();
+  // dO = dy W_o (float16, the attention backward's operand type), D = rowsum(dO * O)
+  void *woT = ws + L.woT, *dO = ws + L.dO;
+  if ((e = cca::transpose16(w->w_o, woT, d.E, d.NQ, d.E, false, st)) != cudaSuccess)
+    return cuda_fail(e, "W_o transpose launch");
+  if ((e = cca::gemm_tcgen05_f16out(dy, woT, dO, M, d.NQ, d.E, 0, status, st)) != cudaSuccess)
+    return cuda_fail(e, "dO GEMM launch");
+  if ((e = cca::attention_rowdot(d, dO, o, Dd, st)) != cudaSuccess)
+    return cuda_fail(e, "rowdot launch");
+  rec.mark();
+  // attention backward
+  cca::AttnBwdArgs ab;
+  ab.q = q;
+  ab.k = k;
+  ab.v = v;
+  ab.dO = dO;
+  ab.kv_stride = seq;
+  ab.lse = lse;
+  ab.D = Dd;
+  ab.dq = reinterpret_cast<float *>(ws + L.dq);
+  ab.dk = reinterpret_cast<float *>(ws + L.dk);
+  ab.dv = reinterpret_cast<float *>(ws + L.dv);
+  ab.status = status;
+  if ((e = cca::latent_attention_backward(d, ab, st)) != cudaSuccess)
+    return cuda_fail(e, "attention backward launch");
+  rec.mark();
+  // stencil backward -> dP (bf16) and the conv filters' gradients
+  cca::StencilBwdArgs sb;
+  sb.P = static_cast<const float *>(P);
+  sb.dq = ab.dq;
+  sb.dk = ab.dk;
+  sb.dv = ab.dv;
+  sb.conv_seq = w->conv_seq;
+  sb.conv_chan = w->conv_chan;
+  sb.dA = reinterpret_cast<float *>(ws + L.dA);
+  sb.dPpart = reinterpret_cast<float *>(ws + L.dPpart);
+  sb.dP = ws + L.dP;
+  sb.dconv_seq = dconv_seq;
+  sb.dconv_chan = dconv_chan;
+  if ((e = cca::stencil_backward(d, sb, st)) != cudaSuccess)
+    return cuda_fail(e, "stencil backward launch");
+  rec.mark();
+  // dx = dP W_qkv, dW_qkv = dP^T x, dW_o = dy^T o (token dimension padded to a multiple of 8)
+  void *wqkvT = ws + L.wqkvT, *dPT = ws + L.dPT, *xT = ws + L.xT, *dyT = ws + L.dyT, *oT = ws + L.oT;
+  if ((e = cca::transpose16(w->w_qkv, wqkvT, d.NQKV, d.E, d.NQKV, false, st)) != cudaSuccess ||
+      (e = cca::transpose16(ws + L.dP, dPT, M, d.NQKV, M8, false, st)) != cudaSuccess ||
+      (e = cca::transpose16(x, xT, M, d.E, M8, false, st)) != cudaSuccess ||
+      (e = cca::transpose16(dy, dyT, M, d.E, M8, false, st)) != cudaSuccess ||
+      (e = cca::transpose16(o, oT, M, d.NQ, M8, true, st)) != cudaSuccess)
+    return cuda_fail(e, "transpose launch");
+  if ((rc = gemm_dispatch(CCA_BF16, 0, ws + L.dP, wqkvT, dx, M, d.E, d.NQKV, status, st))) return rc;
+  if ((rc = gemm_dispatch(CCA_BF16, 1, dPT, xT, dw_qkv, d.NQKV, d.E, M8, status, st))) return rc;
+  if ((rc = gemm_dispatch(CCA_BF16, 1, dyT, oT, dw_o, d.E, d.NQ, M8, status, st))) return rc;
+  rec.mark();
+  return ok();
+}
+
 CCA_API int cca_decode_step(const cca_config_t *cfg, const cca_weights_t *w, const void *x,
                             void *y, cca_cache_t *cache, void *workspace, size_t ws_bytes,
                             void *stream) {

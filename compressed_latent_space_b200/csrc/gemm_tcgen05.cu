@@ -15,6 +15,8 @@
 // after releasing its tensor memory.
 #include <cuda.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -154,13 +156,15 @@ __global__ void __launch_bounds__(THREADS, 1)
           OutT *dst = C + static_cast<size_t>(m) * N + n;
           if (n + 32 <= N && (N & 7) == 0) {
             if constexpr (sizeof(OutT) == 2) {
+              constexpr bool kHalf = std::is_same<OutT, __half>::value;
+              auto pk = [](float a, float b2) { return kHalf ? pack_f16x2(a, b2) : pack_bf16x2(a, b2); };
 #pragma unroll
               for (int v = 0; v < 4; ++v) {
                 uint4 u;
-                u.x = pack_bf16x2(__uint_as_float(r[8 * v + 0]), __uint_as_float(r[8 * v + 1]));
-                u.y = pack_bf16x2(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3]));
-                u.z = pack_bf16x2(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5]));
-                u.w = pack_bf16x2(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7]));
+                u.x = pk(__uint_as_float(r[8 * v + 0]), __uint_as_float(r[8 * v + 1]));
+                u.y = pk(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3]));
+                u.z = pk(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5]));
+                u.w = pk(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7]));
                 reinterpret_cast<uint4 *>(dst)[v] = u;
               }
             } else {
@@ -244,6 +248,17 @@ static cudaError_t launch_gemm(const CUtensorMap &ma, const CUtensorMap &mb, voi
   gemm_bf16_kernel<OutT, AB_F16><<<grid, THREADS, SMEM_BYTES, st>>>(ma, mb, static_cast<OutT *>(C), M,
                                                              N, K, status);
   return cudaGetLastError();
+}
+
+cudaError_t gemm_tcgen05_f16out(const void *A, const void *B, void *C, int M, int N, int K,
+                                int ab_f16, int *status, cudaStream_t st) {
+  if (M <= 0 || N <= 0) return cudaSuccess;
+  if (K % 8 != 0) return cudaErrorInvalidValue;
+  CUtensorMap ma, mb;
+  if (!make_map_2d(&ma, A, M, K, BM, ab_f16) || !make_map_2d(&mb, B, N, K, BN, ab_f16))
+    return cudaErrorInvalidValue;
+  return ab_f16 ? launch_gemm<__half, 1>(ma, mb, C, M, N, K, status, st)
+                : launch_gemm<__half, 0>(ma, mb, C, M, N, K, status, st);
 }
 
 cudaError_t gemm_tcgen05(const void *A, const void *B, void *C, int M, int N, int K, int ab_f16,

@@ -38,6 +38,10 @@ enum : unsigned { F_QK_MEAN = 1u, F_VALUE_SHIFT = 2u, F_QK_NORM = 4u, F_ROPE = 8
 // out (tcgen05 + TMA).
 cudaError_t gemm_tcgen05(const void *A, const void *B, void *C, int M, int N, int K, int ab_f16,
                          int out_f32, int *status, cudaStream_t st);
+// The same contraction with a float16 result (the backward pass's dO, an operand of the
+// float16 attention-backward MMAs).
+cudaError_t gemm_tcgen05_f16out(const void *A, const void *B, void *C, int M, int N, int K,
+                                int ab_f16, int *status, cudaStream_t st);
 // dst[i] = float16(src[i]) for a bf16 tensor of n elements (n % 8 == 0); a value beyond the
 // float16 range records DEV_RANGE in *status.
 cudaError_t convert_bf16_to_f16(const void *src, void *dst, size_t n, int *status, cudaStream_t st);
@@ -95,8 +99,43 @@ cudaError_t fused_qkv_stencil(const Dims &d, const FusedArgs &a, cudaStream_t st
 cudaError_t latent_attention(const Dims &d, const void *q, const void *k, const void *v,
                              int kv_stride, void *o, int *status, cudaStream_t st);
 // The tcgen05 kernel behind latent_attention for 16-bit layers (float16 q, k, v, o).
+// lse (optional, [B, H, S] float32): per query row, the log2-domain log-sum-exp of its scaled
+// scores (the backward pass recomputes the probabilities from it).
 cudaError_t latent_attention_tc(const Dims &d, const void *q, const void *k, const void *v,
-                                int kv_stride, void *o, int *status, cudaStream_t st);
+                                int kv_stride, void *o, int *status, cudaStream_t st,
+                                float *lse = nullptr);
+
+// Backward pass of the latent attention (16-bit layers): q [B, H, S, DL], k / v
+// [B, Hkv, kv_stride, DL], dO [B*S, NQ] (float16, the layout of the forward's o), lse [B, H, S]
+// (from the forward), D = rowsum(dO * O) [B, H, S] -> dq [B, H, S, DL], dk / dv [B, Hkv, S, DL]
+// (float32).
+struct AttnBwdArgs {
+  const void *q, *k, *v, *dO;
+  int kv_stride;
+  const float *lse, *D;
+  float *dq, *dk, *dv;
+  int *status;
+};
+cudaError_t latent_attention_backward(const Dims &d, const AttnBwdArgs &a, cudaStream_t st);
+cudaError_t attention_rowdot(const Dims &d, const void *dO, const void *O, float *D,
+                             cudaStream_t st);
+
+// Backward pass of the latent stencil: P (the forward's projections), dq / dk / dv (float32,
+// the attention backward's layouts) -> dP [B*S, NQKV] bfloat16, and the conv filters'
+// gradients added to dconv_seq [NQ+NKV, KC] and dconv_chan [H+Hkv, DL, DL] (float32, zeroed by
+// the caller).  dA and dPpart are float32 scratch, [B*S, NQ+NKV] and [B*S, NQKV].
+struct StencilBwdArgs {
+  const float *P, *dq, *dk, *dv, *conv_seq, *conv_chan;
+  float *dA, *dPpart;
+  void *dP;
+  float *dconv_seq, *dconv_chan;
+};
+bool stencil_backward_supported(const Dims &d);
+cudaError_t stencil_backward(const Dims &d, const StencilBwdArgs &a, cudaStream_t st);
+// out[c][r] = in[r][c] for 16-bit elements ([R, C] -> [C, R8], rows R..R8-1 of the output
+// zero), float16 converted to bfloat16 when from_f16.
+cudaError_t transpose16(const void *in, void *out, int R, int C, int R8, bool from_f16,
+                        cudaStream_t st);
 
 // Decode step kernels.
 struct DecodeArgs {

@@ -5,7 +5,8 @@ from __future__ import annotations
 
 import torch
 
-from . import (CCA_BF16, CCA_DEFAULT_FLAGS, CCA_F32, cca_cache_alloc, cca_decode_step,
+from . import (CCA_BF16, CCA_DEFAULT_FLAGS, CCA_F32, cca_backward, cca_backward_workspace_size,
+               cca_cache_alloc, cca_decode_step,
                cca_decode_workspace_size, cca_prefill_forward, cca_prefill_workspace_size,
                make_config, make_weights)
 
@@ -103,6 +104,20 @@ class CCALayer:
         cca_prefill_forward(self.cfg, self.weights, x, B, S, y,
                             cache.struct if cache is not None else None, ws, stream)
         return y
+
+    def backward(self, x: torch.Tensor, dy: torch.Tensor, stream=None):
+        """Gradients of sum(y * dy) for the prefill of x: (dx, dw_qkv, dw_o, dconv_seq,
+        dconv_chan); weight gradients in float32."""
+        B, S, E = x.shape
+        dx = torch.empty_like(x)
+        dw_qkv = torch.empty(self.w_qkv.shape, dtype=torch.float32, device=self.device)
+        dw_o = torch.empty(self.w_o.shape, dtype=torch.float32, device=self.device)
+        dconv_seq = torch.empty(self.conv_seq.shape, dtype=torch.float32, device=self.device)
+        dconv_chan = torch.empty(self.conv_chan.shape, dtype=torch.float32, device=self.device)
+        ws = self.workspace(cca_backward_workspace_size(self.cfg, B, S))
+        cca_backward(self.cfg, self.weights, x, dy, B, S, dx, dw_qkv, dw_o, dconv_seq, dconv_chan,
+                     ws, stream)
+        return dx, dw_qkv, dw_o, dconv_seq, dconv_chan
 
     def decode(self, x: torch.Tensor, cache: Cache, out: torch.Tensor | None = None,
                stream=None) -> torch.Tensor:

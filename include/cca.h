@@ -223,6 +223,30 @@ CCA_API int cca_decode_step(const cca_config_t *cfg, const cca_weights_t *w, con
 CCA_API int cca_decode_step_static(const cca_config_t *cfg, const cca_weights_t *w,
                                    const void *x, void *y, cca_cache_t *cache, void *stream);
 
+/* Scratch bytes needed by cca_backward (0 if the config is invalid or outside what the
+ * backward kernels take). */
+CCA_API size_t cca_backward_workspace_size(const cca_config_t *cfg, int batch, int seq);
+
+/* Backward pass of the layer for `batch` sequences of `seq` tokens from position 0 (the pages
+ * measure it against MHA's: gist.science explainer, 4. Experimental Results, "Backward Pass").
+ * Given x [batch, seq, E] and dy = dL/dy [batch, seq, E] (bfloat16), writes
+ *   dx         [batch, seq, E] bfloat16
+ *   dw_qkv     [n_q + 2 n_kv, E] float32     dw_o [E, n_q] float32
+ *   dconv_seq  [n_q + n_kv, conv_kernel] float32
+ *   dconv_chan [H + Hkv, d~, d~, 1] float32
+ * (every output overwritten).  The forward's intermediates are recomputed in the workspace (the
+ * projections, the latents, the attention output and its per-row log-sum-exp); then the
+ * gradient of the up-projection, the attention's backward pass (probabilities recomputed from
+ * the log-sum-exp), the stencil's (RoPE, norm, Q-K-Mean, value-shift and both convolutions
+ * taken back), and the down-projection's.  With tp_size > 1 the gradients are the rank's, and
+ * dx is the rank's share (the caller sums it over the ranks).  bfloat16 layers with the
+ * convolutions, d~ <= 64, (H/Hkv + 1) d~^2 <= 20480, E % 8 == 0 (CCA_ERR_UNSUPPORTED
+ * otherwise).  Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, ALIGNMENT, CUDA. */
+CCA_API int cca_backward(const cca_config_t *cfg, const cca_weights_t *w, const void *x,
+                         const void *dy, int batch, int seq, void *dx, float *dw_qkv,
+                         float *dw_o, float *dconv_seq, float *dconv_chan, void *workspace,
+                         size_t ws_bytes, void *stream);
+
 /* Waits for `stream`, then returns the cache's sticky status word (CCA_OK or
  * CCA_ERR_CACHE_FULL) and clears it. */
 CCA_API int cca_cache_check(cca_cache_t *cache, void *stream);
