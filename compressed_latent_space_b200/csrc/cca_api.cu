@@ -38,19 +38,14 @@ inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 
 inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 // Which kernels a 16-bit prefill with the convolutions uses for the down-projection and the
-// stencil.  The fused kernel keeps P on chip but runs its stencil epilogue between tiles (its
-// 384-column accumulator leaves no room for a second one in tensor memory); measured on B200 it
-// wins where one CTA packs four or more key/value groups (small groups, where the separate
-// stencil kernel spreads thinly: cca_prefill_4k 0.39 -> 0.25 ms) and loses ~7 % at four query
-// heads per group (ccgqa_prefill_16k / _32k).  CCA_PREFILL_PATH=fused or =unfused overrides the
-// choice (for comparing the two paths).
+// stencil: the fused kernel (P stays on chip) wherever it supports the shape; measured on B200
+// it is as fast or faster than the separate GEMM + stencil kernels on every workload
+// (cca_prefill_4k 0.39 -> 0.22 ms, ccgqa_prefill_16k 0.43 -> 0.39 ms, ccgqa_prefill_32k 0.61 vs
+// 0.63 ms).  CCA_PREFILL_PATH=fused or =unfused overrides the choice (for comparing the paths).
 bool use_fused(const cca::Dims &d) {
-  const int ng = cca::fused_group_set(d);
-  if (ng == 0) return false;
+  if (cca::fused_group_set(d) == 0) return false;
   const char *f = getenv("CCA_PREFILL_PATH");
-  if (f && strcmp(f, "fused") == 0) return true;
-  if (f && strcmp(f, "unfused") == 0) return false;
-  return ng >= 4;
+  return !(f && strcmp(f, "unfused") == 0);
 }
 
 // Host-side fault injection for the error paths: CCA_FAULT_INJECT=launch makes every call

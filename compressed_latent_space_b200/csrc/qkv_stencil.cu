@@ -17,7 +17,8 @@
 //              [384, 384 + d~), with A and W_c split into bfloat16 leading terms and
 //              remainders (A_hi W_hi + A_lo W_hi + A_hi W_lo, about 16 significand bits); the
 //              filters of each head stream in by TMA through a two-deep buffer.
-//   warps 2-5  epilogue, one token row per thread (the TMEM lane quadrant of its warp):
+//   warps 2-9  epilogue, one token row per thread (the TMEM lane quadrant of its warp), two
+//              warps per row each on half of every head's columns:
 //              values with the value-shift (the previous token's row through shared memory),
 //              then per head: the causal sequence conv of P's columns (rows exchanged through
 //              shared memory), A written as hi / lo bfloat16 in the MMA's swizzled layout, the
@@ -40,8 +41,9 @@ constexpr int FBK = 32;            // K columns per stage: 64-byte rows
 constexpr int FST = 4;             // stages
 constexpr int FN_MAX = 384;        // accumulator columns
 constexpr uint32_t FCONV0 = 384;   // TMEM column of the channel-conv result
-constexpr int F_THREADS = 192;
-constexpr int XS_LD = 33;          // row stride (floats) of the row-exchange buffer
+constexpr int F_EPI_WARPS = 8;     // two per TMEM lane quadrant, each on half of a head's columns
+constexpr int F_THREADS = 64 + 32 * F_EPI_WARPS;
+constexpr int XS_LD = 17;          // row stride (floats) of a half's row-exchange buffer
 
 struct FusedParams {
   const float *conv_seq;
@@ -78,8 +80,8 @@ __host__ __device__ inline FusedSmem fused_smem(int DL, int N, int NG, int G, in
   off = (off + 1023) & ~1023;
   m.off_abuf = off;                              // {hi, lo} x [128 x d~] bf16
   off += 2 * FM * DL * 2;
-  m.off_xs = off;
-  off += FM * XS_LD * 4;
+  m.off_xs = off;                                // one exchange buffer per half, then the
+  off += 2 * FM * XS_LD * 4 + 2 * FM * 4;        // halves' norm partial sums
   m.off_taps = off;
   off += NG * (G + 1) * DL * KC * 4;
   off = (off + 15) & ~15;
@@ -92,8 +94,11 @@ __host__ __device__ inline FusedSmem fused_smem(int DL, int N, int NG, int G, in
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
-__device__ __forceinline__ void epi_sync() {   // the four epilogue warps only
-  asm volatile("bar.sync 1, 128;" ::: "memory");
+__device__ __forceinline__ void epi_sync() {   // all eight epilogue warps
+  asm volatile("bar.sync 1, 256;" ::: "memory");
+}
+__device__ __forceinline__ void half_sync(int hf) {   // the four epilogue warps of one half
+  asm volatile("bar.sync %0, 128;" ::"r"(2 + hf) : "memory");
 }
 // Byte offset of 16-byte chunk j of row r in a K-major tile with ROWB-byte rows, in the
 // 128/64/32-byte swizzled layout that TMA writes and tcgen05.mma reads (ROWB = 128, 64, 32).
@@ -111,7 +116,21 @@ __host__ __device__ constexpr uint32_t swz_mode() {
 template <int W>
 __device__ __forceinline__ void tmem_ldw(uint32_t taddr, uint32_t (&r)[W]) {
   if constexpr (W == 32) tmem_ld32(taddr, r);
-  else tmem_ld16(taddr, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
+  else if constexpr (W == 16) tmem_ld16(taddr, r);
+  else if constexpr (W == 8) tmem_ld8(taddr, r);
+  else tmem_ld4(taddr, r);
+}
+// Stores Q (16, 8 or 4) consecutive 16-bit values, as pairs in v, at the 2-byte-aligned dst.
+template <int Q>
+__device__ __forceinline__ void store_halves(__half *dst, const uint32_t (&v)[Q / 2]) {
+  if constexpr (Q == 16) {
+    reinterpret_cast<uint4 *>(dst)[0] = make_uint4(v[0], v[1], v[2], v[3]);
+    reinterpret_cast<uint4 *>(dst)[1] = make_uint4(v[4], v[5], v[6], v[7]);
+  } else if constexpr (Q == 8) {
+    *reinterpret_cast<uint4 *>(dst) = make_uint4(v[0], v[1], v[2], v[3]);
+  } else {
+    *reinterpret_cast<uint2 *>(dst) = make_uint2(v[0], v[1]);
+  }
 }
 
 template <int DL>
@@ -152,8 +171,8 @@ __global__ void __launch_bounds__(F_THREADS, 1)
       mbar_init(&bars->empty[s], 1);
     }
     mbar_init(&bars->acc_full, 1);
-    mbar_init(&bars->acc_empty, 4);
-    mbar_init(&bars->a_ready, 4);
+    mbar_init(&bars->acc_empty, F_EPI_WARPS);
+    mbar_init(&bars->a_ready, F_EPI_WARPS);
     mbar_init(&bars->conv_done, 1);
     mbar_init(&bars->filt_full[0], 1);
     mbar_init(&bars->filt_full[1], 1);
@@ -289,14 +308,22 @@ __global__ void __launch_bounds__(F_THREADS, 1)
       }
     }
   } else {
-    // ---------------------------------------------------------------- epilogue warps 2-5
-    const int quad = warp & 3;
+    // ---------------------------------------------------------------- epilogue warps 2-9
+    // Two warps per TMEM lane quadrant; half hf of a head's d~ columns belongs to the warps
+    // (2 + 4 hf .. 5 + 4 hf): columns [hf Q, hf Q + Q) and [d~/2 + hf Q, d~/2 + hf Q + Q) with
+    // Q = d~/4, so both members of every RoPE pair (i, i + d~/2) stay with one thread.  Rows are
+    // exchanged within a half (its own buffer and named barrier); the halves meet at the MMA
+    // hand-off and for the norm's sum of squares.
+    constexpr int Q = DL / 4;
+    const int quad = warp & 3, hf = (warp - 2) >> 2;
     const int row = quad * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
     const uint32_t tP = tmem + lane_off, tC = tmem + FCONV0 + lane_off;
     uint8_t *ahi = abuf, *alo = abuf + FM * ROWB;
+    float *xh = xs + hf * FM * XS_LD;                 // this half's exchange buffer
+    float *nrm = xs + 2 * FM * XS_LD;                 // [half][row] partial sums of squares
     // A failed (timed-out) wait sets the CTA's abort flag, after which every wait returns at
-    // once; the epilogue still runs its whole loop so that all four warps meet at every named
+    // once; the epilogue still runs its whole loop so that its warps meet at every named
     // barrier, and only its stores are skipped.
     int local = 0;
     uint32_t convs = 0;
@@ -310,36 +337,41 @@ __global__ void __launch_bounds__(F_THREADS, 1)
       const bool last_tok = last_tile && t == p.S - 1;
       const int ts = out ? t : 0;                     // a row of the tensors for address math
       tc_fence_after();
-      // ---- values, with the value-shift (the previous row's value through shared memory)
+      // ---- values, with the value-shift (the previous row's value through shared memory);
+      // this half takes the columns [hf d~/2, (hf+1) d~/2), Q at a time
       for (int gi = 0; gi < NG; ++gi) {
         const int g = gs * NG + gi;
         const int vcol = NG * G * DL + NG * DL + gi * DL;
 #pragma unroll
-        for (int c = 0; c < NCH; ++c) {
-          uint32_t r[CW];
-          tmem_ldw<CW>(tP + vcol + c * CW, r);
+        for (int blk = 0; blk < 2; ++blk) {
+          const int c0 = hf * (DL / 2) + blk * Q;
+          uint32_t r[Q];
+          tmem_ldw<Q>(tP + vcol + c0, r);
           tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < CW; ++j) xs[row * XS_LD + j] = __uint_as_float(r[j]);
-          epi_sync();
-          __half *dst = p.v + ((static_cast<size_t>(b) * p.Hkv + g) * p.kv_stride + ts) * DL + c * CW;
+          for (int j = 0; j < Q; ++j) xh[row * XS_LD + j] = __uint_as_float(r[j]);
+          half_sync(hf);
+          uint32_t pk[Q / 2];
           bool fits = true;
 #pragma unroll
-          for (int j = 0; j < CW; j += 2) {
+          for (int j = 0; j < Q; j += 2) {
             float val[2];
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
-              const int gvc = g * DL + c * CW + j + e;
+              const int gvc = g * DL + c0 + j + e;
               const bool shifted = (p.flags & F_VALUE_SHIFT) && gvc >= p.VS0;
-              val[e] = shifted ? (row > 0 ? xs[(row - 1) * XS_LD + j + e] : 0.f) : __uint_as_float(r[j + e]);
+              val[e] = shifted ? (row > 0 ? xh[(row - 1) * XS_LD + j + e] : 0.f) : __uint_as_float(r[j + e]);
               if (last_tok && gvc >= p.VS0)
                 p.vshift_state[static_cast<size_t>(b) * (p.NKV - p.VS0) + (gvc - p.VS0)] = __uint_as_float(r[j + e]);
             }
             fits &= fabsf(val[0]) <= kF16Max && fabsf(val[1]) <= kF16Max;
-            if (out) *reinterpret_cast<uint32_t *>(dst + j) = pack_f16x2(val[0], val[1]);
+            pk[j / 2] = pack_f16x2(val[0], val[1]);
           }
-          if (out && !fits) report(status, DEV_RANGE);
-          epi_sync();
+          if (out) {
+            store_halves<Q>(p.v + ((static_cast<size_t>(b) * p.Hkv + g) * p.kv_stride + ts) * DL + c0, pk);
+            if (!fits) report(status, DEV_RANGE);
+          }
+          half_sync(hf);
         }
       }
       // ---- query and key heads
@@ -350,43 +382,47 @@ __global__ void __launch_bounds__(F_THREADS, 1)
         const int pcol = is_q ? (gi * G + hh) * DL : NG * G * DL + gi * DL;     // P column
         const int kcol = NG * G * DL + gi * DL;                                  // its k head
         const int gch = is_q ? (g * G + hh) * DL : p.NQ + g * DL;             // q|k channel
-        const int lc = pcol;                           // CTA-local channel (taps)
-        // sequence conv, CW columns at a time, into A (hi / lo) in the MMA's layout
+        // sequence conv of this half's two column blocks, into A (hi / lo) in the MMA's layout
 #pragma unroll
-        for (int c = 0; c < NCH; ++c) {
-          uint32_t r[CW];
-          tmem_ldw<CW>(tP + pcol + c * CW, r);
+        for (int blk = 0; blk < 2; ++blk) {
+          const int c0 = blk * (DL / 2) + hf * Q;
+          uint32_t r[Q];
+          tmem_ldw<Q>(tP + pcol + c0, r);
           tmem_ld_wait();
           if (last_tile && t >= p.S - (KC - 1) && t >= 0 && t < p.S) {   // the last KC-1 tokens
             float *cs = p.conv_state + (static_cast<size_t>(b) * (KC - 1) + (t - (p.S - KC + 1))) *
                                            (p.NQ + p.NKV);
 #pragma unroll
-            for (int j = 0; j < CW; ++j) cs[gch + c * CW + j] = __uint_as_float(r[j]);
+            for (int j = 0; j < Q; ++j) cs[gch + c0 + j] = __uint_as_float(r[j]);
           }
 #pragma unroll
-          for (int j = 0; j < CW; ++j) xs[row * XS_LD + j] = __uint_as_float(r[j]);
-          epi_sync();
-          float a[CW];
+          for (int j = 0; j < Q; ++j) xh[row * XS_LD + j] = __uint_as_float(r[j]);
+          half_sync(hf);
+          float a[Q];
 #pragma unroll
-          for (int j = 0; j < CW; ++j) a[j] = 0.f;
+          for (int j = 0; j < Q; ++j) a[j] = 0.f;
           for (int tap = 0; tap < KC; ++tap) {
             const int rr = max(row - (KC - 1) + tap, 0);
-            const float *tp = taps + (lc + c * CW) * KC + tap;
+            const float *tp = taps + (pcol + c0) * KC + tap;
 #pragma unroll
-            for (int j = 0; j < CW; ++j) a[j] = fmaf(tp[j * KC], xs[rr * XS_LD + j], a[j]);
+            for (int j = 0; j < Q; ++j) a[j] = fmaf(tp[j * KC], xh[rr * XS_LD + j], a[j]);
           }
+          uint32_t hi[Q / 2], lo[Q / 2];
 #pragma unroll
-          for (int q8 = 0; q8 < CW / 8; ++q8) {
-            uint4 h4, l4;
-            split_bf16x2(make_float2(a[q8 * 8 + 0], a[q8 * 8 + 1]), h4.x, l4.x);
-            split_bf16x2(make_float2(a[q8 * 8 + 2], a[q8 * 8 + 3]), h4.y, l4.y);
-            split_bf16x2(make_float2(a[q8 * 8 + 4], a[q8 * 8 + 5]), h4.z, l4.z);
-            split_bf16x2(make_float2(a[q8 * 8 + 6], a[q8 * 8 + 7]), h4.w, l4.w);
-            const uint32_t o = swz_off<ROWB>(row, c * (CW / 8) + q8);
-            *reinterpret_cast<uint4 *>(ahi + o) = h4;
-            *reinterpret_cast<uint4 *>(alo + o) = l4;
+          for (int j = 0; j < Q; j += 2) split_bf16x2(make_float2(a[j], a[j + 1]), hi[j / 2], lo[j / 2]);
+          if constexpr (Q >= 8) {
+#pragma unroll
+            for (int q8 = 0; q8 < Q / 8; ++q8) {
+              const uint32_t o = swz_off<ROWB>(row, c0 / 8 + q8);
+              *reinterpret_cast<uint4 *>(ahi + o) = make_uint4(hi[4 * q8], hi[4 * q8 + 1], hi[4 * q8 + 2], hi[4 * q8 + 3]);
+              *reinterpret_cast<uint4 *>(alo + o) = make_uint4(lo[4 * q8], lo[4 * q8 + 1], lo[4 * q8 + 2], lo[4 * q8 + 3]);
+            }
+          } else {                                     // 4 columns: half of a 16-byte piece
+            const uint32_t o = swz_off<ROWB>(row, c0 / 8) + (c0 % 8) * 2;
+            *reinterpret_cast<uint2 *>(ahi + o) = make_uint2(hi[0], hi[1]);
+            *reinterpret_cast<uint2 *>(alo + o) = make_uint2(lo[0], lo[1]);
           }
-          epi_sync();                                  // xs is rewritten by the next chunk
+          half_sync(hf);                               // xh is rewritten by the next block
         }
         fence_proxy_async_smem();                      // A visible to the tensor cores
         tc_fence_before();
@@ -395,41 +431,43 @@ __global__ void __launch_bounds__(F_THREADS, 1)
         ok = __all_sync(0xffffffffu, mbar_wait(&bars->conv_done, convs & 1, abort, status)) && ok;
         ++convs;
         tc_fence_after();
-        float u[DL];
+        float uu[2 * Q];                               // [low block | high block]
 #pragma unroll
-        for (int c = 0; c < NCH; ++c) {
-          uint32_t r[CW];
-          tmem_ldw<CW>(tC + c * CW, r);
+        for (int blk = 0; blk < 2; ++blk) {
+          const int c0 = blk * (DL / 2) + hf * Q;
+          uint32_t r[Q];
+          tmem_ldw<Q>(tC + c0, r);
           tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < CW; ++j) u[c * CW + j] = __uint_as_float(r[j]);
+          for (int j = 0; j < Q; ++j) uu[blk * Q + j] = __uint_as_float(r[j]);
         }
         if (p.flags & F_QK_MEAN) {                     // + (pre-conv q + pre-conv k) / 2
 #pragma unroll
-          for (int c = 0; c < NCH; ++c) {
-            uint32_t rk[CW], rq[CW];
-            tmem_ldw<CW>(tP + kcol + c * CW, rk);
-            float mq[CW];
+          for (int blk = 0; blk < 2; ++blk) {
+            const int c0 = blk * (DL / 2) + hf * Q;
+            uint32_t rk[Q], rq[Q];
+            tmem_ldw<Q>(tP + kcol + c0, rk);
+            float mq[Q];
             if (is_q) {
-              tmem_ldw<CW>(tP + pcol + c * CW, rq);
+              tmem_ldw<Q>(tP + pcol + c0, rq);
               tmem_ld_wait();
 #pragma unroll
-              for (int j = 0; j < CW; ++j) mq[j] = __uint_as_float(rq[j]);
+              for (int j = 0; j < Q; ++j) mq[j] = __uint_as_float(rq[j]);
             } else {
 #pragma unroll
-              for (int j = 0; j < CW; ++j) mq[j] = 0.f;
+              for (int j = 0; j < Q; ++j) mq[j] = 0.f;
               for (int h2 = 0; h2 < G; ++h2) {
-                tmem_ldw<CW>(tP + (gi * G + h2) * DL + c * CW, rq);
+                tmem_ldw<Q>(tP + (gi * G + h2) * DL + c0, rq);
                 tmem_ld_wait();
 #pragma unroll
-                for (int j = 0; j < CW; ++j) mq[j] += __uint_as_float(rq[j]);
+                for (int j = 0; j < Q; ++j) mq[j] += __uint_as_float(rq[j]);
               }
 #pragma unroll
-              for (int j = 0; j < CW; ++j) mq[j] /= static_cast<float>(G);
+              for (int j = 0; j < Q; ++j) mq[j] /= static_cast<float>(G);
             }
             tmem_ld_wait();
 #pragma unroll
-            for (int j = 0; j < CW; ++j) u[c * CW + j] += 0.5f * (mq[j] + __uint_as_float(rk[j]));
+            for (int j = 0; j < Q; ++j) uu[blk * Q + j] += 0.5f * (mq[j] + __uint_as_float(rk[j]));
           }
         }
         if (hidx == nheads - 1) {                      // every P column this tile needs is read
@@ -440,19 +478,22 @@ __global__ void __launch_bounds__(F_THREADS, 1)
         if (p.flags & F_QK_NORM) {
           float ss = 0.f;
 #pragma unroll
-          for (int i = 0; i < DL; ++i) ss += u[i] * u[i];
+          for (int i = 0; i < 2 * Q; ++i) ss += uu[i] * uu[i];
+          nrm[hf * FM + row] = ss;
+          epi_sync();
+          ss = nrm[row] + nrm[FM + row];
           const float inv = 1.0f / sqrtf(ss / static_cast<float>(DL) + p.eps);
 #pragma unroll
-          for (int i = 0; i < DL; ++i) u[i] *= inv;
+          for (int i = 0; i < 2 * Q; ++i) uu[i] *= inv;
         }
         if ((p.flags & F_ROPE) && out) {
 #pragma unroll
-          for (int i = 0; i < HALF; ++i) {
+          for (int j = 0; j < Q; ++j) {
             float cs, sn;
-            rope_cos_sin(static_cast<double>(t) * p.theta[i], cs, sn);
-            const float x1 = u[i], x2 = u[i + HALF];
-            u[i] = x1 * cs - x2 * sn;
-            u[i + HALF] = x1 * sn + x2 * cs;
+            rope_cos_sin(static_cast<double>(t) * p.theta[hf * Q + j], cs, sn);
+            const float x1 = uu[j], x2 = uu[Q + j];
+            uu[j] = x1 * cs - x2 * sn;
+            uu[Q + j] = x1 * sn + x2 * cs;
           }
         }
         if (out && ok) {
@@ -460,20 +501,19 @@ __global__ void __launch_bounds__(F_THREADS, 1)
                              : p.k + ((static_cast<size_t>(b) * p.Hkv + g) * p.kv_stride + t) * DL;
           bool fits = true;
 #pragma unroll
-          for (int i = 0; i < DL; i += 8) {
-            uint4 w;
-            w.x = pack_f16x2(u[i], u[i + 1]);
-            w.y = pack_f16x2(u[i + 2], u[i + 3]);
-            w.z = pack_f16x2(u[i + 4], u[i + 5]);
-            w.w = pack_f16x2(u[i + 6], u[i + 7]);
+          for (int blk = 0; blk < 2; ++blk) {
+            uint32_t pk[Q / 2];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) fits &= fabsf(u[i + e]) <= kF16Max;
-            *reinterpret_cast<uint4 *>(dst + i) = w;
+            for (int j = 0; j < Q; j += 2) {
+              pk[j / 2] = pack_f16x2(uu[blk * Q + j], uu[blk * Q + j + 1]);
+              fits &= fabsf(uu[blk * Q + j]) <= kF16Max && fabsf(uu[blk * Q + j + 1]) <= kF16Max;
+            }
+            store_halves<Q>(dst + blk * (DL / 2) + hf * Q, pk);
           }
           if (!fits) report(status, DEV_RANGE);
         }
       }
-      if (last_tile && gs == 0 && row == HALO) p.lengths[b] = p.S;
+      if (last_tile && gs == 0 && row == HALO && hf == 0) p.lengths[b] = p.S;
     }
   }
 
