@@ -9,17 +9,19 @@
 //   dV = P^T dO (summed over the group's heads).
 // Two kernels, so that no gradient needs atomics:
 //   attn_bwd_dq_kernel    one CTA per (query head, sequence, 128-query tile): S = Q K_j^T and
-//                         dP = dO V_j^T per key tile j into tensor memory, dS written back over
-//                         S as float16 pairs, dQ += dS K_j with dS as the MMA's A operand from
+//                         dP = dO V_j^T per key tile j into tensor memory, dS written back as
+//                         float16 pairs, dQ += dS K_j with dS as the MMA's A operand from
 //                         tensor memory and the staged K tile read as the (MN-major) B operand.
 //   attn_bwd_dkdv_kernel  one CTA per (key/value head, sequence, 128-key tile), walking every
 //                         (query tile, query head of the group) pair at or after the diagonal:
 //                         S^T = K Q^T and dP^T = V dO^T with the keys on the tensor-memory
 //                         lanes, P^T and dS^T written back as float16 pairs, then
 //                         dV += P^T dO and dK += dS^T Q straight from tensor memory.
-// Warps 0-3 compute the elementwise part (one tensor-memory lane, i.e. one query or key row,
-// per thread), warp 4 is the TMA producer, warp 5 issues the MMAs.  The tensor pipe executes in
-// issue order, so a tile's next S overwrites dS only after the MMA that reads dS.  Every wait
+// Warps 0-7 compute the elementwise part, two per tensor-memory lane quadrant (one query or
+// key row per thread, each warp on half of the tile's 128 columns); warp 8 is the TMA producer,
+// warp 9 issues the MMAs.  P / dS go to their own tensor-memory columns, so as soon as every
+// elementwise warp has loaded its scores the next item's S / dP MMAs start, overlapping this
+// item's exponentials; a commit after the gradient MMAs guards the P / dS columns.  Every wait
 // is bounded; on a timeout the CTA records it in the status word, stops, and frees its TMEM.
 #include <math.h>
 
@@ -30,9 +32,13 @@ namespace cca {
 namespace {
 
 constexpr int BT = 128;              // rows of every tile (queries or keys)
-constexpr int BW_TMA = 4, BW_MMA = 5;
-constexpr int B_THREADS = 192;
+constexpr int B_EW = 8;              // elementwise warps: two per TMEM lane quadrant
+constexpr int BW_TMA = B_EW, BW_MMA = B_EW + 1;
+constexpr int B_THREADS = (B_EW + 2) * 32;
 constexpr int BSLOTS = 3;            // ring depth of the streamed tiles
+// TMEM columns: S (or S^T) 0..127, dP (dP^T) 128..255, gradient accumulators from 256,
+// the float16 pairs of P / dS (P^T / dS^T) the gradient MMAs read at 384..447 / 448..511
+constexpr uint32_t C_S = 0, C_DP = 128, C_ACC = 256, C_P = 384, C_DS = 448;
 
 template <int DL>
 struct BwdCfg {
@@ -40,13 +46,14 @@ struct BwdCfg {
   static constexpr int TILE = BT * ROWB;
   static constexpr uint32_t SW = ROWB == 128 ? 2u : ROWB == 64 ? 4u : 6u;
   static constexpr int SBO = 8 * ROWB;
+  static_assert(C_ACC + 2 * DL <= C_P, "accumulators below the P / dS columns");
 };
 
 struct BwdBars {
   uint64_t first_full;               // dq: Q and dO; dkdv: K and V
   uint64_t a_full[BSLOTS], a_empty[BSLOTS];   // dq: K ring; dkdv: Q + dO ring
   uint64_t b_full[BSLOTS], b_empty[BSLOTS];   // dq: V ring
-  uint64_t s_full, p_full, done;
+  uint64_t s_full, s_free, p_full, pds_free, done;
   uint32_t tmem_base;
   int abort;
 };
@@ -65,8 +72,17 @@ __device__ __forceinline__ bool elect_one() {
   return pred != 0;
 }
 
-__device__ __forceinline__ void soft_sync() {   // the four elementwise warps only
-  asm volatile("bar.sync 1, 128;" ::: "memory");
+__device__ __forceinline__ void ew_sync() {      // the eight elementwise warps only
+  asm volatile("bar.sync 1, 256;" ::: "memory");
+}
+
+// The elementwise warp's 64 columns of S and dP (its half of the tile's 128) for its TMEM lane.
+__device__ __forceinline__ void load_half(uint32_t base, uint32_t (&rs)[64], uint32_t (&rp)[64]) {
+  tmem_ld32(base + C_S, *reinterpret_cast<uint32_t(*)[32]>(&rs[0]));
+  tmem_ld32(base + C_S + 32, *reinterpret_cast<uint32_t(*)[32]>(&rs[32]));
+  tmem_ld32(base + C_DP, *reinterpret_cast<uint32_t(*)[32]>(&rp[0]));
+  tmem_ld32(base + C_DP + 32, *reinterpret_cast<uint32_t(*)[32]>(&rp[32]));
+  tmem_ld_wait();
 }
 
 // ------------------------------------------------------------------------------------ dQ
@@ -101,7 +117,9 @@ __global__ void __launch_bounds__(B_THREADS, 1)
       mbar_init(&bars->b_empty[s], 1);
     }
     mbar_init(&bars->s_full, 1);
-    mbar_init(&bars->p_full, 4);
+    mbar_init(&bars->s_free, B_EW);
+    mbar_init(&bars->p_full, B_EW);
+    mbar_init(&bars->pds_free, 1);
     mbar_init(&bars->done, 1);
     bars->abort = 0;
     fence_mbar_init();
@@ -113,7 +131,7 @@ __global__ void __launch_bounds__(B_THREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = bars->tmem_base;          // S: cols 0..127, dP: 128..255, dQ: 256..
+  const uint32_t tmem = bars->tmem_base;
   volatile int *abort = &bars->abort;
 
   if (warp == BW_TMA) {
@@ -144,8 +162,8 @@ __global__ void __launch_bounds__(B_THREADS, 1)
       if (leader) {
 #pragma unroll
         for (int kk = 0; kk < DL / 16; ++kk) {
-          umma_f16_ss(tmem, qd + 2 * kk, kd + 2 * kk, idesc_s, kk > 0 ? 1u : 0u);
-          umma_f16_ss(tmem + 128, dod + 2 * kk, vd + 2 * kk, idesc_s, kk > 0 ? 1u : 0u);
+          umma_f16_ss(tmem + C_S, qd + 2 * kk, kd + 2 * kk, idesc_s, kk > 0 ? 1u : 0u);
+          umma_f16_ss(tmem + C_DP, dod + 2 * kk, vd + 2 * kk, idesc_s, kk > 0 ? 1u : 0u);
         }
         umma_commit(&bars->s_full);
         umma_commit(&bars->b_empty[s]);              // V_j is read only by dP
@@ -161,64 +179,72 @@ __global__ void __launch_bounds__(B_THREADS, 1)
     }
     for (int j = 0; ok && j < nk; ++j) {
       const int s = j % BSLOTS;
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars->p_full, j & 1, abort, status));
-      if (!ok) break;
-      tc_fence_after();
-      // dQ += dS K_j: dS (float16 pairs over S's columns) as A, K_j as the MN-major B
-      const uint64_t kb = smem_desc(smem_u32(sK + s * C::TILE), C::TILE, C::SBO, C::SW);
-      if (leader) {
-#pragma unroll
-        for (int kk = 0; kk < BT / 16; ++kk)
-          umma_f16_ts(tmem + 256, tmem + kk * 8, kb + kk * (2 * C::SBO / 16), idesc_q,
-                      (j > 0 || kk > 0) ? 1u : 0u);
-        umma_commit(&bars->a_empty[s]);
-        if (j + 1 == nk) umma_commit(&bars->done);
-      }
-      __syncwarp();
-      if (j + 1 < nk) {
+      if (j + 1 < nk) {                              // next tile's S / dP once this one is read
         const int s1 = (j + 1) % BSLOTS;
-        ok = __all_sync(0xffffffffu, mbar_wait(&bars->a_full[s1], ((j + 1) / BSLOTS) & 1, abort, status) &&
+        ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_free, j & 1, abort, status) &&
+                                         mbar_wait(&bars->a_full[s1], ((j + 1) / BSLOTS) & 1, abort, status) &&
                                          mbar_wait(&bars->b_full[s1], ((j + 1) / BSLOTS) & 1, abort, status));
         if (!ok) break;
         tc_fence_after();
         issue_s(j + 1);
       }
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->p_full, j & 1, abort, status));
+      if (!ok) break;
+      tc_fence_after();
+      // dQ += dS K_j: dS (float16 pairs) as A from TMEM, K_j as the MN-major B
+      const uint64_t kb = smem_desc(smem_u32(sK + s * C::TILE), C::TILE, C::SBO, C::SW);
+      if (leader) {
+#pragma unroll
+        for (int kk = 0; kk < BT / 16; ++kk)
+          umma_f16_ts(tmem + C_ACC, tmem + C_DS + kk * 8, kb + kk * (2 * C::SBO / 16), idesc_q,
+                      (j > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(&bars->pds_free);
+        umma_commit(&bars->a_empty[s]);
+        if (j + 1 == nk) umma_commit(&bars->done);
+      }
+      __syncwarp();
     }
   } else {
-    const int row = warp * 32 + lane;
+    const int quad = warp & 3, hf = warp >> 2;       // lanes of quadrant, key columns of half
+    const int row = quad * 32 + lane;
     const int qpos = qt * BT + row;
     const bool valid = qpos < S;
     const size_t ridx = (static_cast<size_t>(b) * H + h) * S + (valid ? qpos : 0);
     const float lrow = valid ? lse[ridx] : INFINITY;   // invalid rows: every p is 0
     const float drow = valid ? Dd[ridx] : 0.f;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    const uint32_t base = tmem + lane_off + hf * 64;
     bool ok = true;
     for (int j = 0; ok && j < nk; ++j) {
       ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full, j & 1, abort, status));
       if (!ok) break;
       tc_fence_after();
+      uint32_t rs[64], rp[64];
+      load_half(base, rs, rp);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->s_free);    // the next tile's S / dP may overwrite
       const bool diag = j == qt;
+      uint32_t pk[32];
 #pragma unroll
-      for (int c = 0; c < BT / 32; ++c) {
-        uint32_t rs[32], rp[32];
-        tmem_ld32(tmem + lane_off + c * 32, rs);
-        tmem_ld32(tmem + lane_off + 128 + c * 32, rp);
-        tmem_ld_wait();
-        uint32_t pk[16];
+      for (int e = 0; e < 32; ++e) {
+        float ds[2];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          float ds[2];
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int kcol = c * 32 + 2 * e + u;
-            float p = ex2(__uint_as_float(rs[2 * e + u]) * scale_log2 - lrow);
-            if (diag && kcol > row) p = 0.f;
-            ds[u] = p * (__uint_as_float(rp[2 * e + u]) - drow);
-          }
-          pk[e] = pack_f16x2(ds[0], ds[1]);
+        for (int u = 0; u < 2; ++u) {
+          const int kcol = hf * 64 + 2 * e + u;
+          float p = ex2(__uint_as_float(rs[2 * e + u]) * scale_log2 - lrow);
+          if (diag && kcol > row) p = 0.f;
+          ds[u] = p * (__uint_as_float(rp[2 * e + u]) - drow);
         }
-        tmem_st16(tmem + lane_off + c * 16, pk);     // dS over the S columns already read
+        pk[e] = pack_f16x2(ds[0], ds[1]);
       }
+      // the previous tile's dQ MMA must have read its dS before this one is written
+      if (j > 0) ok = __all_sync(0xffffffffu, mbar_wait(&bars->pds_free, (j - 1) & 1, abort, status));
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t pd = tmem + lane_off + C_DS + hf * 32;
+      tmem_st16(pd, *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
+      tmem_st16(pd + 16, *reinterpret_cast<uint32_t(*)[16]>(&pk[16]));
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
@@ -229,17 +255,18 @@ __global__ void __launch_bounds__(B_THREADS, 1)
       tc_fence_after();
       float *dst = dq + ridx * DL;
 #pragma unroll
-      for (int c = 0; c < DL / 8; ++c) {
+      for (int c = 0; c < DL / 16; ++c) {           // this half's DL/2 columns, 8 at a time
         uint32_t o[8];
-        tmem_ld8(tmem + lane_off + 256 + c * 8, o);
+        const int col = hf * (DL / 2) + c * 8;
+        tmem_ld8(tmem + lane_off + C_ACC + col, o);
         tmem_ld_wait();
         if (valid) {
-          float4 a = make_float4(__uint_as_float(o[0]) * scale, __uint_as_float(o[1]) * scale,
-                                 __uint_as_float(o[2]) * scale, __uint_as_float(o[3]) * scale);
-          float4 bq = make_float4(__uint_as_float(o[4]) * scale, __uint_as_float(o[5]) * scale,
-                                  __uint_as_float(o[6]) * scale, __uint_as_float(o[7]) * scale);
-          reinterpret_cast<float4 *>(dst)[2 * c] = a;
-          reinterpret_cast<float4 *>(dst)[2 * c + 1] = bq;
+          reinterpret_cast<float4 *>(dst + col)[0] =
+              make_float4(__uint_as_float(o[0]) * scale, __uint_as_float(o[1]) * scale,
+                          __uint_as_float(o[2]) * scale, __uint_as_float(o[3]) * scale);
+          reinterpret_cast<float4 *>(dst + col)[1] =
+              make_float4(__uint_as_float(o[4]) * scale, __uint_as_float(o[5]) * scale,
+                          __uint_as_float(o[6]) * scale, __uint_as_float(o[7]) * scale);
         }
       }
     }
@@ -283,7 +310,9 @@ __global__ void __launch_bounds__(B_THREADS, 1)
       mbar_init(&bars->a_empty[s], 1);
     }
     mbar_init(&bars->s_full, 1);
-    mbar_init(&bars->p_full, 4);
+    mbar_init(&bars->s_free, B_EW);
+    mbar_init(&bars->p_full, B_EW);
+    mbar_init(&bars->pds_free, 1);
     mbar_init(&bars->done, 1);
     bars->abort = 0;
     fence_mbar_init();
@@ -295,7 +324,7 @@ __global__ void __launch_bounds__(B_THREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = bars->tmem_base;   // S^T 0..127, dP^T 128..255, dV 256.., dK 256+DL..
+  const uint32_t tmem = bars->tmem_base;
   volatile int *abort = &bars->abort;
 
   if (warp == BW_TMA) {
@@ -325,8 +354,8 @@ __global__ void __launch_bounds__(B_THREADS, 1)
       if (leader) {
 #pragma unroll
         for (int kk = 0; kk < DL / 16; ++kk) {
-          umma_f16_ss(tmem, kd + 2 * kk, qd + 2 * kk, idesc_s, kk > 0 ? 1u : 0u);
-          umma_f16_ss(tmem + 128, vd + 2 * kk, dod + 2 * kk, idesc_s, kk > 0 ? 1u : 0u);
+          umma_f16_ss(tmem + C_S, kd + 2 * kk, qd + 2 * kk, idesc_s, kk > 0 ? 1u : 0u);
+          umma_f16_ss(tmem + C_DP, vd + 2 * kk, dod + 2 * kk, idesc_s, kk > 0 ? 1u : 0u);
         }
         umma_commit(&bars->s_full);
       }
@@ -341,42 +370,45 @@ __global__ void __launch_bounds__(B_THREADS, 1)
     }
     for (int n = 0; ok && n < nitems; ++n) {
       const int s = n % BSLOTS;
+      if (n + 1 < nitems) {                          // the next item's S^T / dP^T once read
+        ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_free, n & 1, abort, status) &&
+                                         mbar_wait(&bars->a_full[(n + 1) % BSLOTS], ((n + 1) / BSLOTS) & 1, abort, status));
+        if (!ok) break;
+        tc_fence_after();
+        issue_s(n + 1);
+      }
       ok = __all_sync(0xffffffffu, mbar_wait(&bars->p_full, n & 1, abort, status));
       if (!ok) break;
       tc_fence_after();
-      // dV += P^T dO and dK += dS^T Q, A operands from tensor memory, the staged dO and Q tiles
+      // dV += P^T dO and dK += dS^T Q, A operands from tensor memory, the item's dO and Q tiles
       // as MN-major B operands
       const uint64_t dob = smem_desc(smem_u32(sDO + s * C::TILE), C::TILE, C::SBO, C::SW);
       const uint64_t qb = smem_desc(smem_u32(sQ + s * C::TILE), C::TILE, C::SBO, C::SW);
       if (leader) {
 #pragma unroll
         for (int kk = 0; kk < BT / 16; ++kk) {
-          umma_f16_ts(tmem + 256, tmem + kk * 8, dob + kk * (2 * C::SBO / 16), idesc_o,
+          umma_f16_ts(tmem + C_ACC, tmem + C_P + kk * 8, dob + kk * (2 * C::SBO / 16), idesc_o,
                       (n > 0 || kk > 0) ? 1u : 0u);
-          umma_f16_ts(tmem + 256 + DL, tmem + 128 + kk * 8, qb + kk * (2 * C::SBO / 16), idesc_o,
-                      (n > 0 || kk > 0) ? 1u : 0u);
+          umma_f16_ts(tmem + C_ACC + DL, tmem + C_DS + kk * 8, qb + kk * (2 * C::SBO / 16),
+                      idesc_o, (n > 0 || kk > 0) ? 1u : 0u);
         }
+        umma_commit(&bars->pds_free);
         umma_commit(&bars->a_empty[s]);
         if (n + 1 == nitems) umma_commit(&bars->done);
       }
       __syncwarp();
-      if (n + 1 < nitems) {
-        const int s1 = (n + 1) % BSLOTS;
-        ok = __all_sync(0xffffffffu, mbar_wait(&bars->a_full[s1], ((n + 1) / BSLOTS) & 1, abort, status));
-        if (!ok) break;
-        tc_fence_after();
-        issue_s(n + 1);
-      }
     }
   } else {
-    const int row = warp * 32 + lane;
+    const int quad = warp & 3, hf = warp >> 2;       // lanes of quadrant, query columns of half
+    const int row = quad * 32 + lane;
     const int kpos = kt * BT + row;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    const uint32_t base = tmem + lane_off + hf * 64;
     // per-item lse and D of the item's 128 queries, staged in shared memory one item ahead
     auto stage_stats = [&](int n) {
-      if (n >= nitems) return;
+      if (n >= nitems || threadIdx.x >= BT) return;
       const int qt = kt + n / G, h = g * G + n % G;
-      const int q = qt * BT + threadIdx.x;          // threadIdx.x < 128 here
+      const int q = qt * BT + threadIdx.x;
       const size_t ridx = (static_cast<size_t>(b) * H + h) * S + q;
       float *buf = sL + (n & 1) * 2 * BT;
       buf[threadIdx.x] = q < S ? lse[ridx] : INFINITY;
@@ -385,36 +417,40 @@ __global__ void __launch_bounds__(B_THREADS, 1)
     stage_stats(0);
     bool ok = true;
     for (int n = 0; n < nitems; ++n) {
-      soft_sync();                                   // stats of item n visible, n-1's read
+      ew_sync();                                     // stats of item n visible, n-1's read
       stage_stats(n + 1);
       ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full, n & 1, abort, status)) && ok;
       tc_fence_after();
+      uint32_t rs[64], rp[64];
+      load_half(base, rs, rp);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->s_free);
       const int qt = kt + n / G;
       const bool diag = qt == kt;
-      const float *bl = sL + (n & 1) * 2 * BT, *bd = bl + BT;
+      const float *bl = sL + (n & 1) * 2 * BT + hf * 64, *bd = bl + BT;
+      uint32_t pkp[32], pks[32];
 #pragma unroll
-      for (int c = 0; c < BT / 32; ++c) {
-        uint32_t rs[32], rp[32];
-        tmem_ld32(tmem + lane_off + c * 32, rs);
-        tmem_ld32(tmem + lane_off + 128 + c * 32, rp);
-        tmem_ld_wait();
-        uint32_t pkp[16], pks[16];
+      for (int e = 0; e < 32; ++e) {
+        float pp[2], ds[2];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          float p[2], ds[2];
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int qcol = c * 32 + 2 * e + u;
-            p[u] = ex2(__uint_as_float(rs[2 * e + u]) * scale_log2 - bl[qcol]);
-            if (diag && qcol < row) p[u] = 0.f;          // a query before this key
-            ds[u] = p[u] * (__uint_as_float(rp[2 * e + u]) - bd[qcol]);
-          }
-          pkp[e] = pack_f16x2(p[0], p[1]);
-          pks[e] = pack_f16x2(ds[0], ds[1]);
+        for (int u = 0; u < 2; ++u) {
+          const int qcol = 2 * e + u;                // within this half
+          pp[u] = ex2(__uint_as_float(rs[2 * e + u]) * scale_log2 - bl[qcol]);
+          if (diag && hf * 64 + qcol < row) pp[u] = 0.f;   // a query before this key
+          ds[u] = pp[u] * (__uint_as_float(rp[2 * e + u]) - bd[qcol]);
         }
-        tmem_st16(tmem + lane_off + c * 16, pkp);        // P^T over S^T's read columns
-        tmem_st16(tmem + lane_off + 128 + c * 16, pks);  // dS^T over dP^T's read columns
+        pkp[e] = pack_f16x2(pp[0], pp[1]);
+        pks[e] = pack_f16x2(ds[0], ds[1]);
       }
+      // the previous item's dV / dK MMAs must have read P^T / dS^T before they are rewritten
+      if (n > 0) ok = __all_sync(0xffffffffu, mbar_wait(&bars->pds_free, (n - 1) & 1, abort, status)) && ok;
+      tc_fence_after();
+      const uint32_t pp = tmem + lane_off + C_P + hf * 32, pd = tmem + lane_off + C_DS + hf * 32;
+      tmem_st16(pp, *reinterpret_cast<uint32_t(*)[16]>(&pkp[0]));
+      tmem_st16(pp + 16, *reinterpret_cast<uint32_t(*)[16]>(&pkp[16]));
+      tmem_st16(pd, *reinterpret_cast<uint32_t(*)[16]>(&pks[0]));
+      tmem_st16(pd + 16, *reinterpret_cast<uint32_t(*)[16]>(&pks[16]));
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
@@ -426,13 +462,14 @@ __global__ void __launch_bounds__(B_THREADS, 1)
       const bool valid = kpos < S;
       const size_t ridx = (static_cast<size_t>(b) * Hkv + g) * S + (valid ? kpos : 0);
 #pragma unroll
-      for (int c = 0; c < DL / 8; ++c) {
+      for (int c = 0; c < DL / 16; ++c) {           // this half's DL/2 columns, 8 at a time
+        const int col = hf * (DL / 2) + c * 8;
         uint32_t ov[8], okk[8];
-        tmem_ld8(tmem + lane_off + 256 + c * 8, ov);
-        tmem_ld8(tmem + lane_off + 256 + DL + c * 8, okk);
+        tmem_ld8(tmem + lane_off + C_ACC + col, ov);
+        tmem_ld8(tmem + lane_off + C_ACC + DL + col, okk);
         tmem_ld_wait();
         if (valid && nitems > 0) {
-          float *pv = dv + ridx * DL + c * 8, *pk = dk + ridx * DL + c * 8;
+          float *pv = dv + ridx * DL + col, *pk = dk + ridx * DL + col;
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             pv[e] = __uint_as_float(ov[e]);

@@ -22,7 +22,8 @@ namespace {
 
 constexpr int S1_TT = 16;          // tokens per pass-1 tile
 constexpr int S1_THREADS = 256;
-constexpr int S1_MAX_PER_THREAD = 80;   // channel-filter gradient entries a thread accumulates
+constexpr int S1_MAX_BLOCKS = 5;        // 4 x 4 blocks of filter-gradient entries per thread
+constexpr int S1_MAX_PER_THREAD = 16 * S1_MAX_BLOCKS;
 
 struct S1Params {
   const float *P;                  // [B*S, NQKV] forward projections
@@ -38,12 +39,13 @@ struct S1Params {
   double theta[32];
 };
 
-// smem (floats): Wc [(G+1) DL x (DL+1)] (rows padded by one float, so reading a column across
-// a warp's rows and reading a row across its columns are both free of bank conflicts) |
-// Ps [(TT + KC-1) x (G+2)DL] | A [TT x (G+1)DL] | U [same] | dU [same] | N [same]
+// smem (floats): Wc [(G+1) DL x (DL+4)] (rows padded by four floats: 16-byte aligned rows whose
+// 128-bit reads across a quarter warp's rows hit distinct banks, and column reads across a
+// warp's columns stay contiguous) | Ps [(TT + KC-1) x (G+2)DL] | A [TT x (G+1)DL] | U [same] |
+// dU [same] | N [same]
 __host__ __device__ inline size_t s1_smem_floats(int G, int DL, int KC) {
   const size_t QK = static_cast<size_t>(G + 1) * DL;
-  return QK * (DL + 1) + static_cast<size_t>(S1_TT + KC - 1) * (G + 2) * DL + 4 * S1_TT * QK;
+  return QK * (DL + 4) + static_cast<size_t>(S1_TT + KC - 1) * (G + 2) * DL + 4 * S1_TT * QK;
 }
 
 __global__ void __launch_bounds__(S1_THREADS, 1) stencil_bwd1_kernel(const S1Params p, int cpg,
@@ -51,7 +53,7 @@ __global__ void __launch_bounds__(S1_THREADS, 1) stencil_bwd1_kernel(const S1Par
   extern __shared__ __align__(16) float sm[];
   const int G = p.G, DL = p.DL, KC = p.KC, KC1 = KC - 1;
   const int QK = (G + 1) * DL, CH = (G + 2) * DL;
-  const int WL = DL + 1;                             // padded filter row
+  const int WL = DL + 4;                             // padded filter row
   float *Wc = sm;
   float *Ps = Wc + QK * WL;
   float *A = Ps + (S1_TT + KC1) * CH;
@@ -71,7 +73,8 @@ __global__ void __launch_bounds__(S1_THREADS, 1) stencil_bwd1_kernel(const S1Par
     const int hh = e / (DL * DL), r = e % (DL * DL);
     Wc[(hh * DL + r / DL) * WL + r % DL] = p.conv_chan[static_cast<size_t>(head_glob(hh)) * DL * DL + r];
   }
-  const int NE = QK * DL;                            // filter-gradient entries of the group
+  const int BPH = (DL / 4) * (DL / 4);               // 4 x 4 filter-gradient blocks per head
+  const int NB = (G + 1) * BPH;
   float acc[S1_MAX_PER_THREAD];
 #pragma unroll
   for (int m = 0; m < S1_MAX_PER_THREAD; ++m) acc[m] = 0.f;
@@ -96,27 +99,40 @@ __global__ void __launch_bounds__(S1_THREADS, 1) stencil_bwd1_kernel(const S1Par
       A[e] = a;
     }
     __syncthreads();
-    // channel conv and Q-K-Mean: U = W_c A + skip
-    for (int e = tid; e < S1_TT * QK; e += nt) {
-      const int tt = e / QK, hc = e % QK, hh = hc / DL, i = hc % DL;
-      const float *w = Wc + (hh * DL + i) * WL;
-      const float *a = A + tt * QK + hh * DL;
-      float v = 0.f;
-      for (int c = 0; c < DL; ++c) v = fmaf(w[c], a[c], v);
-      if (p.flags & F_QK_MEAN) {
-        const float *pr = Ps + (tt + KC1) * CH;
-        const float pk = pr[G * DL + i];
-        float pq;
-        if (hh < G) {
-          pq = pr[hh * DL + i];
-        } else {
-          pq = 0.f;
-          for (int h2 = 0; h2 < G; ++h2) pq += pr[h2 * DL + i];
-          pq /= static_cast<float>(G);
+    // channel conv and Q-K-Mean: U = W_c A + skip; a thread per output channel, all TT tokens,
+    // the filter row and the tokens' inputs read four floats at a time
+    for (int hc = tid; hc < QK; hc += nt) {
+      const int hh = hc / DL, i = hc % DL;
+      const float4 *w4 = reinterpret_cast<const float4 *>(Wc + (hh * DL + i) * WL);
+      float v[S1_TT];
+#pragma unroll
+      for (int tt = 0; tt < S1_TT; ++tt) v[tt] = 0.f;
+      for (int c4 = 0; c4 < DL / 4; ++c4) {
+        const float4 w = w4[c4];
+#pragma unroll
+        for (int tt = 0; tt < S1_TT; ++tt) {
+          const float4 a = reinterpret_cast<const float4 *>(A + tt * QK + hh * DL)[c4];
+          v[tt] = fmaf(w.x, a.x, fmaf(w.y, a.y, fmaf(w.z, a.z, fmaf(w.w, a.w, v[tt]))));
         }
-        v += 0.5f * (pq + pk);
       }
-      U[e] = v;
+#pragma unroll
+      for (int tt = 0; tt < S1_TT; ++tt) {
+        float x = v[tt];
+        if (p.flags & F_QK_MEAN) {
+          const float *pr = Ps + (tt + KC1) * CH;
+          const float pk = pr[G * DL + i];
+          float pq;
+          if (hh < G) {
+            pq = pr[hh * DL + i];
+          } else {
+            pq = 0.f;
+            for (int h2 = 0; h2 < G; ++h2) pq += pr[h2 * DL + i];
+            pq /= static_cast<float>(G);
+          }
+          x += 0.5f * (pq + pk);
+        }
+        U[tt * QK + hc] = x;
+      }
     }
     __syncthreads();
     // per (token, head): norm statistics, dn = RoPE^-1(dq or dk), du; one warp per pair
@@ -163,29 +179,42 @@ __global__ void __launch_bounds__(S1_THREADS, 1) stencil_bwd1_kernel(const S1Par
       }
     }
     __syncthreads();
-    // dA = W_c^T dU per head, and the Q-K-Mean skip gradients of the q | k projections
-    for (int e = tid; e < S1_TT * QK; e += nt) {
-      const int tt = e / QK, hc = e % QK, hh = hc / DL, c = hc % DL;
-      const int t = t0 + tt;
-      if (t >= p.S) continue;
-      const float *du = dU + tt * QK + hh * DL;
-      float v = 0.f;
-      for (int i = 0; i < DL; ++i) v = fmaf(Wc[(hh * DL + i) * WL + c], du[i], v);
-      const size_t row = static_cast<size_t>(b) * p.S + t;
-      const int gc = hh < G ? qcol0 + hh * DL + c : kcol0 + c;
-      p.dA[row * (p.NQ + p.NKV) + gc] = v;
-      float skip = 0.f;
-      if (p.flags & F_QK_MEAN) {
-        const float duk = dU[tt * QK + G * DL + c];
-        if (hh < G) {
-          skip = 0.5f * du[c] + duk / (2.0f * static_cast<float>(G));
-        } else {
-          float sq = 0.f;
-          for (int h2 = 0; h2 < G; ++h2) sq += dU[tt * QK + h2 * DL + c];
-          skip = 0.5f * sq + 0.5f * duk;
+    // dA = W_c^T dU per head, and the Q-K-Mean skip gradients of the q | k projections; a
+    // thread per input channel, all TT tokens, the tokens' dU read four floats at a time
+    for (int hc = tid; hc < QK; hc += nt) {
+      const int hh = hc / DL, c = hc % DL;
+      float v[S1_TT];
+#pragma unroll
+      for (int tt = 0; tt < S1_TT; ++tt) v[tt] = 0.f;
+      for (int i4 = 0; i4 < DL / 4; ++i4) {
+        const float *wc = Wc + (hh * DL + 4 * i4) * WL + c;
+        const float w0 = wc[0], w1 = wc[WL], w2 = wc[2 * WL], w3 = wc[3 * WL];
+#pragma unroll
+        for (int tt = 0; tt < S1_TT; ++tt) {
+          const float4 d = reinterpret_cast<const float4 *>(dU + tt * QK + hh * DL)[i4];
+          v[tt] = fmaf(w0, d.x, fmaf(w1, d.y, fmaf(w2, d.z, fmaf(w3, d.w, v[tt]))));
         }
       }
-      p.dPpart[row * p.NQKV + gc] = skip;
+      const int gc = hh < G ? qcol0 + hh * DL + c : kcol0 + c;
+#pragma unroll
+      for (int tt = 0; tt < S1_TT; ++tt) {
+        const int t = t0 + tt;
+        if (t >= p.S) continue;
+        const size_t row = static_cast<size_t>(b) * p.S + t;
+        p.dA[row * (p.NQ + p.NKV) + gc] = v[tt];
+        float skip = 0.f;
+        if (p.flags & F_QK_MEAN) {
+          const float duk = dU[tt * QK + G * DL + c];
+          if (hh < G) {
+            skip = 0.5f * dU[tt * QK + hh * DL + c] + duk / (2.0f * static_cast<float>(G));
+          } else {
+            float sq = 0.f;
+            for (int h2 = 0; h2 < G; ++h2) sq += dU[tt * QK + h2 * DL + c];
+            skip = 0.5f * sq + 0.5f * duk;
+          }
+        }
+        p.dPpart[row * p.NQKV + gc] = skip;
+      }
     }
     // values: dPv[t, c] = dv[t, c] unshifted, dv[t+1, c] shifted
     for (int e = tid; e < S1_TT * DL; e += nt) {
@@ -198,25 +227,41 @@ __global__ void __launch_bounds__(S1_THREADS, 1) stencil_bwd1_kernel(const S1Par
       const float val = ts < p.S ? p.dv[((static_cast<size_t>(b) * p.Hkv + g) * p.S + ts) * DL + c] : 0.f;
       p.dPpart[(static_cast<size_t>(b) * p.S + t) * p.NQKV + vcol0 + c] = val;
     }
-    // channel-filter gradient: dW_c[h][i][c] += sum_tt dU[tt][h][i] A[tt][h][c]
+    // channel-filter gradient: dW_c[h][i][c] += sum_tt dU[tt][h][i] A[tt][h][c], a 4 x 4 block
+    // of (i, c) per thread and block slot
 #pragma unroll
-    for (int m = 0; m < S1_MAX_PER_THREAD; ++m) {
-      const int e = tid + m * S1_THREADS;
-      if (e < NE) {
-        const int hh = e / (DL * DL), r = e % (DL * DL), i = r / DL, c = r % DL;
-        float s = 0.f;
-        for (int tt = 0; tt < S1_TT; ++tt) s = fmaf(dU[tt * QK + hh * DL + i], A[tt * QK + hh * DL + c], s);
-        acc[m] += s;
+    for (int m = 0; m < S1_MAX_BLOCKS; ++m) {
+      const int blk = tid + m * S1_THREADS;
+      if (blk < NB) {
+        const int hh = blk / BPH, r = blk % BPH;
+        const int i0 = (r / (DL / 4)) * 4, c0 = (r % (DL / 4)) * 4;
+#pragma unroll
+        for (int tt = 0; tt < S1_TT; ++tt) {
+          const float4 d = *reinterpret_cast<const float4 *>(dU + tt * QK + hh * DL + i0);
+          const float4 a = *reinterpret_cast<const float4 *>(A + tt * QK + hh * DL + c0);
+          const float dv4[4] = {d.x, d.y, d.z, d.w}, av4[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+          for (int ii = 0; ii < 4; ++ii)
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc)
+              acc[m * 16 + ii * 4 + cc] = fmaf(dv4[ii], av4[cc], acc[m * 16 + ii * 4 + cc]);
+        }
       }
     }
     __syncthreads();                                 // Ps, A, U, dU rewritten by the next tile
   }
 #pragma unroll
-  for (int m = 0; m < S1_MAX_PER_THREAD; ++m) {
-    const int e = tid + m * S1_THREADS;
-    if (e < NE && u_end > u_beg) {
-      const int hh = e / (DL * DL), r = e % (DL * DL);
-      atomicAdd(p.dconv_chan + static_cast<size_t>(head_glob(hh)) * DL * DL + r, acc[m]);
+  for (int m = 0; m < S1_MAX_BLOCKS; ++m) {
+    const int blk = tid + m * S1_THREADS;
+    if (blk < NB && u_end > u_beg) {
+      const int hh = blk / BPH, r = blk % BPH;
+      const int i0 = (r / (DL / 4)) * 4, c0 = (r % (DL / 4)) * 4;
+      float *dst = p.dconv_chan + static_cast<size_t>(head_glob(hh)) * DL * DL;
+#pragma unroll
+      for (int ii = 0; ii < 4; ++ii)
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc)
+          atomicAdd(dst + (i0 + ii) * DL + c0 + cc, acc[m * 16 + ii * 4 + cc]);
     }
   }
 }
@@ -291,7 +336,7 @@ __global__ void __launch_bounds__(256) transpose16_kernel(const uint16_t *__rest
 
 bool stencil_backward_supported(const Dims &d) {
   return d.bf16 && !(d.flags & F_NO_CONV) && d.DL <= 64 && d.KC <= 8 &&
-         (d.G + 1) * d.DL * d.DL <= S1_MAX_PER_THREAD * S1_THREADS &&
+         (d.G + 1) * (d.DL / 4) * (d.DL / 4) <= S1_MAX_BLOCKS * S1_THREADS &&
          s1_smem_floats(d.G, d.DL, d.KC) * 4 <= 200 * 1024;
 }
 
