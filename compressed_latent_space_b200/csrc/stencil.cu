@@ -657,9 +657,10 @@ cudaError_t launch(const Dims &d, const StencilArgs &a, cudaStream_t st) {
 // Q-K-Mean (whose pre- and post-conv terms then coincide), value-shift, RMS norm and RoPE as
 // selected.  With C = 1 and only RoPE on, this is the projection-to-attention step of plain
 // multi-head (or grouped-query) attention with rotary embeddings, for any latent width up to
-// 128.  One CTA per token, one warp per (token, head) item, reading its P row segment straight
-// from global memory (lane i holds channels i and i + d~/2, the RoPE pair, of the row); no
-// shared memory, so many warps per SM hide the load latency of this memory-bound pass.
+// 128.  A memory-bound pass: one (token, head row) unit per d~/8 consecutive threads, each
+// thread holding four RoPE pairs (channels i..i+3 and i+d~/2..i+d~/2+3) as two float4 loads of
+// the P row (the q heads, k groups and v groups of a token lie at row offset unit * d~ in
+// that order), the row's sum of squares reduced over the unit's lanes by shuffles.
 template <typename T>
 struct PointParams {
   using TL = typename LatentType<T>::type;
@@ -669,97 +670,187 @@ struct PointParams {
   int B, S, H, Hkv, G, DL, NQ, NKV, NQKV, VS0, kv_stride;
   unsigned flags;
   float eps;
-  double theta[64];        // RoPE frequencies base^(-2i/d~), i < d~/2, computed on the host
+  // RoPE frequency base^(-2i/d~) / (2 pi) in turns, i < d~/2, as a float pair hi + lo
+  // (computed on the host in double)
+  float turns_hi[64], turns_lo[64];
 };
 
-template <typename T>
-__global__ void __launch_bounds__(256) pointwise_kernel(const PointParams<T> p) {
-  using TL = typename LatentType<T>::type;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-  const int per_tok = p.H + 2 * p.Hkv;
-  const int DL = p.DL, HALF = DL / 2;
-  const int bt = blockIdx.x;                         // one CTA per token: b * S + t
-  const int b = bt / p.S, t = bt - b * p.S;
+// cos and sin of t * theta_i without double precision: the angle in turns is t * (hi + lo);
+// t * hi is split into its rounded product and the product's exact rounding error (an FMA),
+// the rounded product's whole turns are dropped exactly, and the rest (|r| <= 1/2 + tiny) is
+// scaled to radians.  The reduced angle is good to a few 1e-8 turns for t < 2^24.
+__device__ __forceinline__ void rope_cos_sin_turns(int t, float hi, float lo, float &c, float &s) {
+  const float tf = static_cast<float>(t);
+  const float prod = tf * hi;
+  const float err = fmaf(tf, hi, -prod);
+  const float r = (prod - rintf(prod)) + fmaf(tf, lo, err);
+  __sincosf(r * 6.2831853071795865f, &s, &c);
+}
+
+template <typename TL>
+__device__ __forceinline__ void store4(TL *dst, const float (&x)[4]) {
+  if constexpr (sizeof(TL) == 2) {
+    uint2 u;
+    u.x = pack_f16x2(x[0], x[1]);
+    u.y = pack_f16x2(x[2], x[3]);
+    *reinterpret_cast<uint2 *>(dst) = u;
+  } else {
+    *reinterpret_cast<float4 *>(dst) = make_float4(x[0], x[1], x[2], x[3]);
+  }
+}
+
+__device__ __forceinline__ void load4(const float *src, float (&x)[4]) {
+  const float4 f = __ldg(reinterpret_cast<const float4 *>(src));
+  x[0] = f.x; x[1] = f.y; x[2] = f.z; x[3] = f.w;
+}
+
+// Loads one unit's eight channels (Q-K-Mean applied for query / key heads, the value-shift
+// for value groups).
+template <typename T, int DL, bool QKM>
+__device__ __forceinline__ void pointwise_load(const PointParams<T> &p, int bt, int hh, int i0,
+                                               float (&u0)[4], float (&u1)[4]) {
+  constexpr int HALF = DL / 2;
   const float *row = p.P + static_cast<size_t>(bt) * p.NQKV;
-  for (int hh = warp; hh < per_tok; hh += nwarps) {
-    if (hh < p.H + p.Hkv) {                         // a query or key head
-      const bool is_q = hh < p.H;
-      const int g = is_q ? hh / p.G : hh - p.H;
-      const int off = is_q ? hh * DL : p.NQ + g * DL;
-      float u[2][2];                                // pairs (i, i + d~/2), i = lane + 32e
-      float ss = 0.f;
+  if (hh < p.H + p.Hkv) {                           // a query or key head
+    const bool is_q = hh < p.H;
+    const int g = is_q ? hh / p.G : hh - p.H;
+    load4(row + hh * DL + i0, u0);
+    load4(row + hh * DL + HALF + i0, u1);
+    if (QKM) {                                      // post-conv == pre-conv here
+      float k0[4], k1[4], m0[4], m1[4];
+      load4(row + p.NQ + g * DL + i0, k0);
+      load4(row + p.NQ + g * DL + HALF + i0, k1);
+      if (is_q) {
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int i = lane + 32 * e;
+        for (int e = 0; e < 4; ++e) { m0[e] = u0[e]; m1[e] = u1[e]; }
+      } else {
 #pragma unroll
-        for (int s2 = 0; s2 < 2; ++s2) {
-          float x = 0.f;
-          if (i < HALF) {
-            const int c = i + s2 * HALF;
-            x = row[off + c];
-            if (p.flags & F_QK_MEAN) {              // post-conv == pre-conv here
-              const float pk = row[p.NQ + g * DL + c];
-              float pq;
-              if (is_q) {
-                pq = x;
-              } else {
-                pq = 0.f;
-                for (int h2 = 0; h2 < p.G; ++h2) pq += row[(g * p.G + h2) * DL + c];
-                pq /= static_cast<float>(p.G);
-              }
-              x += 0.5f * (pq + pk);
-            }
-          }
-          u[e][s2] = x;
-          ss += x * x;
+        for (int e = 0; e < 4; ++e) { m0[e] = 0.f; m1[e] = 0.f; }
+        for (int h2 = 0; h2 < p.G; ++h2) {
+          float a0[4], a1[4];
+          load4(row + (g * p.G + h2) * DL + i0, a0);
+          load4(row + (g * p.G + h2) * DL + HALF + i0, a1);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) { m0[e] += a0[e]; m1[e] += a1[e]; }
         }
-      }
-      if (p.flags & F_QK_NORM) {
+        const float inv_g = 1.f / static_cast<float>(p.G);
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-        const float inv = 1.0f / sqrtf(ss / static_cast<float>(DL) + p.eps);
-#pragma unroll
-        for (int e = 0; e < 2; ++e) { u[e][0] *= inv; u[e][1] *= inv; }
+        for (int e = 0; e < 4; ++e) { m0[e] *= inv_g; m1[e] *= inv_g; }
       }
-      TL *dst = is_q ? p.q + ((static_cast<size_t>(b) * p.H + hh) * p.S + t) * DL
-                     : p.k + ((static_cast<size_t>(b) * p.Hkv + g) * p.kv_stride + t) * DL;
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int i = lane + 32 * e;
-        if (i < HALF) {
-          float a = u[e][0], c2 = u[e][1];
-          if (p.flags & F_ROPE) {
-            float cs, sn;
-            rope_cos_sin(static_cast<double>(t) * p.theta[i], cs, sn);
-            const float x1 = a, x2 = c2;
-            a = x1 * cs - x2 * sn;
-            c2 = x1 * sn + x2 * cs;
-          }
-          check_latent<TL>(a, p.status);
-          check_latent<TL>(c2, p.status);
-          dst[i] = from_f32<TL>(a);
-          dst[i + HALF] = from_f32<TL>(c2);
-        }
-      }
-    } else {                                        // a value head, with the value-shift
-      const int g = hh - p.H - p.Hkv;
-      TL *dst = p.v + ((static_cast<size_t>(b) * p.Hkv + g) * p.kv_stride + t) * DL;
-      for (int c = lane; c < DL; c += 32) {
-        const bool shifted = (p.flags & F_VALUE_SHIFT) && (g * DL + c >= p.VS0);
-        float x = 0.f;
-        if (!shifted) x = row[p.NQ + p.NKV + g * DL + c];
-        else if (t > 0) x = row[static_cast<long long>(-p.NQKV) + p.NQ + p.NKV + g * DL + c];
-        check_latent<TL>(x, p.status);
-        dst[c] = from_f32<TL>(x);
+      for (int e = 0; e < 4; ++e) {
+        u0[e] += 0.5f * (m0[e] + k0[e]);
+        u1[e] += 0.5f * (m1[e] + k1[e]);
       }
     }
+  } else {                                          // a value group, with the value-shift
+    const int g = hh - p.H - p.Hkv;
+    const int t = bt % p.S;
+    // the channel boundary of the shift is a multiple of 4 (checked on the host), so each
+    // 4-channel run is shifted or not as a whole
+    const int c0 = g * DL + i0, c1 = c0 + HALF;
+    const bool sh0 = (p.flags & F_VALUE_SHIFT) && c0 >= p.VS0;
+    const bool sh1 = (p.flags & F_VALUE_SHIFT) && c1 >= p.VS0;
+    const float *vrow = row + p.NQ + p.NKV;
+    const float *prev = vrow - p.NQKV;              // the previous token's row (t > 0 only)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) { u0[e] = 0.f; u1[e] = 0.f; }
+    if (!sh0) load4(vrow + c0, u0);
+    else if (t > 0) load4(prev + c0, u0);
+    if (!sh1) load4(vrow + c1, u1);
+    else if (t > 0) load4(prev + c1, u1);
+  }
+}
+
+// Norm (its sum of squares reduced over the unit's lanes; every lane of the warp takes part),
+// RoPE, range check and store of one unit.
+template <typename T, int DL>
+__device__ __forceinline__ void pointwise_finish(const PointParams<T> &p, const float2 *turns,
+                                                 int bt, int hh, int i0, bool live,
+                                                 float (&u0)[4], float (&u1)[4]) {
+  using TL = typename LatentType<T>::type;
+  constexpr int TPU = DL / 8, HALF = DL / 2;
+  const bool is_qk = hh < p.H + p.Hkv;
+  if (p.flags & F_QK_NORM) {                        // uniform over the grid
+    float ss = 0.f;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) ss += u0[e] * u0[e] + u1[e] * u1[e];
+#pragma unroll
+    for (int o = TPU / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if (is_qk) {
+      const float inv = 1.0f / sqrtf(ss / static_cast<float>(DL) + p.eps);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) { u0[e] *= inv; u1[e] *= inv; }
+    }
+  }
+  if (!live) return;
+  const int b = bt / p.S, t = bt - b * p.S;
+  TL *dst;
+  if (is_qk) {
+    if (p.flags & F_ROPE) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        float cs, sn;
+        const float2 tr = turns[i0 + e];
+        rope_cos_sin_turns(t, tr.x, tr.y, cs, sn);
+        const float x1 = u0[e], x2 = u1[e];
+        u0[e] = x1 * cs - x2 * sn;
+        u1[e] = x1 * sn + x2 * cs;
+      }
+    }
+    const bool is_q = hh < p.H;
+    dst = is_q ? p.q + ((static_cast<size_t>(b) * p.H + hh) * p.S + t) * DL
+               : p.k + ((static_cast<size_t>(b) * p.Hkv + (hh - p.H)) * p.kv_stride + t) * DL;
+  } else {
+    const int g = hh - p.H - p.Hkv;
+    dst = p.v + ((static_cast<size_t>(b) * p.Hkv + g) * p.kv_stride + t) * DL;
+  }
+#pragma unroll
+  for (int e = 0; e < 4; ++e) { check_latent<TL>(u0[e], p.status); check_latent<TL>(u1[e], p.status); }
+  store4(dst + i0, u0);
+  store4(dst + HALF + i0, u1);
+}
+
+// Grid-stride over units, two units per thread per pass with both units' loads issued first.
+// Lanes of a warp walk together: the warp's pass continues while its first unit exists, and
+// lanes whose unit lies past the end redo the last unit without storing.
+template <typename T, int DL, bool QKM>
+__global__ void __launch_bounds__(256, QKM ? 3 : 6) pointwise_kernel(const PointParams<T> p) {
+  constexpr int TPU = DL / 8;                       // threads per unit (divides 32)
+  const unsigned per_tok = p.H + 2 * p.Hkv;
+  const unsigned units = static_cast<unsigned>(p.B) * p.S * per_tok;   // < 2^31 (host check)
+  const unsigned total = gridDim.x * blockDim.x;
+  const unsigned lane = threadIdx.x & 31;
+  const int i0 = static_cast<int>(lane % TPU) * 4;  // pairs i0..i0+3 with i0+HALF..
+  // the RoPE frequencies in shared memory: lanes of a warp read different ones, which a
+  // constant-bank access would serialise
+  __shared__ float2 turns[64];
+  if (threadIdx.x < 64) turns[threadIdx.x] = make_float2(p.turns_hi[threadIdx.x], p.turns_lo[threadIdx.x]);
+  __syncthreads();
+  for (unsigned wb = blockIdx.x * blockDim.x + (threadIdx.x & ~31u); wb / TPU < units;
+       wb += 2 * total) {
+    float u0[2][4], u1[2][4];
+    int bt[2], hh[2];
+    bool live[2];
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const unsigned g = (wb + r * total + lane) / TPU;
+      live[r] = g < units;
+      const unsigned unit = live[r] ? g : units - 1;
+      bt[r] = static_cast<int>(unit / per_tok);
+      hh[r] = static_cast<int>(unit % per_tok);
+      pointwise_load<T, DL, QKM>(p, bt[r], hh[r], i0, u0[r], u1[r]);
+    }
+#pragma unroll
+    for (int r = 0; r < 2; ++r) pointwise_finish<T, DL>(p, turns, bt[r], hh[r], i0, live[r], u0[r], u1[r]);
   }
 }
 
 template <typename T>
 cudaError_t launch_pointwise(const Dims &d, const StencilArgs &a, cudaStream_t st) {
   using TL = typename LatentType<T>::type;
-  if (d.DL > 128) return cudaErrorInvalidValue;
+  if (d.DL != 16 && d.DL != 32 && d.DL != 64 && d.DL != 128) return cudaErrorInvalidValue;
+  if (d.VS0 % 4 != 0 || d.NQKV % 4 != 0) return cudaErrorInvalidValue;
   PointParams<T> p;
   p.P = a.P;
   p.q = static_cast<TL *>(a.q);
@@ -771,11 +862,37 @@ cudaError_t launch_pointwise(const Dims &d, const StencilArgs &a, cudaStream_t s
   p.kv_stride = a.kv_stride;
   p.flags = d.flags;
   p.eps = d.eps;
-  for (int i = 0; i < 64; ++i)
-    p.theta[i] = i < d.DL / 2 ? pow(static_cast<double>(d.rope_base), -2.0 * i / d.DL) : 0.0;
-  const int per_tok = d.H + 2 * d.Hkv;
-  const int threads = per_tok >= 8 ? 256 : 32 * per_tok;   // a warp per (token, head) item
-  pointwise_kernel<T><<<static_cast<unsigned>(d.B * d.S), threads, 0, st>>>(p);
+  for (int i = 0; i < 64; ++i) {
+    const double turns = i < d.DL / 2
+        ? pow(static_cast<double>(d.rope_base), -2.0 * i / d.DL) / 6.283185307179586 : 0.0;
+    p.turns_hi[i] = static_cast<float>(turns);
+    p.turns_lo[i] = static_cast<float>(turns - static_cast<double>(p.turns_hi[i]));
+  }
+  const long long units = static_cast<long long>(d.B) * d.S * (d.H + 2 * d.Hkv);
+  const long long threads = units * (d.DL / 8);
+  if (threads >= (1LL << 30) || d.S >= (1 << 24)) return cudaErrorInvalidValue;
+  const long long want = (threads + 511) / 512;      // two units per thread
+  const long long cap = static_cast<long long>(num_sms()) * ((d.flags & F_QK_MEAN) ? 3 : 6);
+  const unsigned blocks = static_cast<unsigned>(want < cap ? want : cap);
+  const bool qkm = (d.flags & F_QK_MEAN) != 0;
+  switch (d.DL) {
+    case 16:
+      if (qkm) pointwise_kernel<T, 16, true><<<blocks, 256, 0, st>>>(p);
+      else pointwise_kernel<T, 16, false><<<blocks, 256, 0, st>>>(p);
+      break;
+    case 32:
+      if (qkm) pointwise_kernel<T, 32, true><<<blocks, 256, 0, st>>>(p);
+      else pointwise_kernel<T, 32, false><<<blocks, 256, 0, st>>>(p);
+      break;
+    case 64:
+      if (qkm) pointwise_kernel<T, 64, true><<<blocks, 256, 0, st>>>(p);
+      else pointwise_kernel<T, 64, false><<<blocks, 256, 0, st>>>(p);
+      break;
+    default:
+      if (qkm) pointwise_kernel<T, 128, true><<<blocks, 256, 0, st>>>(p);
+      else pointwise_kernel<T, 128, false><<<blocks, 256, 0, st>>>(p);
+      break;
+  }
   return cudaGetLastError();
 }
 

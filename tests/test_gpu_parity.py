@@ -390,6 +390,9 @@ def test_latent_range_is_reported(cuda_lib):
     dict(d_model=512, n_heads=4, n_kv_heads=4, compression=1, seq=300),   # MHA, hd=128
     dict(d_model=512, n_heads=4, n_kv_heads=2, compression=1, seq=257),   # GQA, hd=128
     dict(d_model=256, n_heads=4, n_kv_heads=2, compression=2, seq=130),   # d~=32
+    dict(d_model=256, n_heads=4, n_kv_heads=2, compression=1, seq=333),   # d~=64
+    dict(d_model=256, n_heads=4, n_kv_heads=4, compression=4, seq=99),    # d~=16
+    dict(d_model=256, n_heads=4, n_kv_heads=2, compression=2, seq=77, dtype="f32"),
 ])
 def test_prefill_no_conv(cuda_lib, shape, flags):
     """CCA_NO_CONV: both convolutions are the identity.  With C = 1 and RoPE alone this is
@@ -399,7 +402,10 @@ def test_prefill_no_conv(cuda_lib, shape, flags):
     _, y = run_prefill(cuda_lib, w, inp, flags)
     ocfg = oracle_config(w, flags)
     ref = O.prefill(ocfg, oracle_weights(ocfg, inp, no_conv=True), f64(inp.x))
-    assert bf16_err(f64(y), ref) <= BF16_TOL
+    if w.dtype == "f32":
+        assert_fp32_close(f64(y), ref)
+    else:
+        assert bf16_err(f64(y), ref) <= BF16_TOL
 
 
 @pytest.mark.parametrize("name", ["mha_prefill_16k", "gqa8_prefill_16k"])
