@@ -20,106 +20,179 @@
 namespace cca {
 namespace {
 
-constexpr int S1_TT = 16;          // tokens per pass-1 tile
+constexpr int S1_TT = 16;          // tokens per pass-1 tile (the M of its mma.sync tiles)
 constexpr int S1_THREADS = 256;
-constexpr int S1_MAX_BLOCKS = 5;        // 4 x 4 blocks of filter-gradient entries per thread
-constexpr int S1_MAX_PER_THREAD = 16 * S1_MAX_BLOCKS;
+constexpr int S1_WARPS = S1_THREADS / 32;
+constexpr int S1_MAXB = 20;        // filter-gradient 16 x 8 blocks per warp
+constexpr int S1_KCMAX = 8;
 
 struct S1Params {
   const float *P;                  // [B*S, NQKV] forward projections
   const float *dq, *dk, *dv;       // [B, H, S, DL], [B, Hkv, S, DL] float32
   const float *conv_seq;           // [NQ + NKV, KC]
-  const float *conv_chan;          // [H + Hkv, DL, DL]
+  const uint2 *wsplit;             // channel filters as bf16 hi/lo pairs, [head][out i][in pair]
+  const uint2 *wsplitT;            // the same transposed, [head][in c][out pair]
   float *dA;                       // [B*S, NQ + NKV] gradient of the sequence-conv output
   float *dPpart;                   // [B*S, NQKV] Q-K-Mean skip and value gradients
   float *dconv_chan;               // [H + Hkv, DL, DL] (accumulated)
-  int B, S, H, Hkv, G, DL, NQ, NKV, NQKV, KC, VS0;
+  int B, S, H, Hkv, G, NQ, NKV, NQKV, KC, VS0;
   unsigned flags;
   float eps;
-  double theta[32];
+  float turns_hi[32], turns_lo[32];  // RoPE frequencies in turns, as float pairs
 };
 
-// smem (floats): Wc [(G+1) DL x (DL+4)] (rows padded by four floats: 16-byte aligned rows whose
-// 128-bit reads across a quarter warp's rows hit distinct banks, and column reads across a
-// warp's columns stay contiguous) | Ps [(TT + KC-1) x (G+2)DL] | A [TT x (G+1)DL] | U [same] |
-// dU [same] | N [same]
+// Row strides of the shared-memory tiles: a multiple of 32 floats plus 4, so that the mma
+// fragment reads (eight rows x four column pairs, or four row pairs x eight columns) fall on
+// distinct banks.
+__host__ __device__ constexpr int s1_pad(int w) { return (w + 31) / 32 * 32 + 4; }
+
+// smem (floats): Ps [2][(TT + KC-1) x CHP] (P rows with the conv halo, double-buffered) |
+// Dq [2][TT x QKP] (dq of the G heads and dk) | Dv [2][(TT + 1) x DL] | A [TT x QKP] (sequence-
+// conv output) | U [TT x QKP] (channel-conv output, then its gradient in place) |
+// Rt [TT x DL] (cos, sin of the tile's RoPE angles) | turns [2 x 32]
 __host__ __device__ inline size_t s1_smem_floats(int G, int DL, int KC) {
-  const size_t QK = static_cast<size_t>(G + 1) * DL;
-  return QK * (DL + 4) + static_cast<size_t>(S1_TT + KC - 1) * (G + 2) * DL + 4 * S1_TT * QK;
+  const size_t QKP = s1_pad((G + 1) * DL), CHP = s1_pad((G + 2) * DL);
+  return 2 * static_cast<size_t>(S1_TT + KC - 1) * CHP + 2 * S1_TT * QKP +
+         2 * static_cast<size_t>(S1_TT + 1) * DL + 2 * S1_TT * QKP + S1_TT * DL + 64;
 }
 
+// Pass 1, persistent: CTA (ci, g) walks the 16-token tiles u_beg .. u_end-1 of key/value group
+// g, the next tile's P rows, dq / dk and dv copied in (16-byte asynchronous copies) while the
+// current one is computed.  The three channel-conv products are warp mma.sync tiles on bf16
+// hi / lo splits (three products each: hi*hi + hi*lo + lo*hi, about fp32 accuracy):
+//   U  = A W^T per head (tokens x out channels), then Q-K-Mean's skip terms
+//   dA = dU W  per head (tokens x in channels)
+//   dW += dU^T A per head (out x in channels, the tile's tokens as K), accumulated in
+//         registers over the CTA's tiles and added to the output once.
+template <int DL>
 __global__ void __launch_bounds__(S1_THREADS, 1) stencil_bwd1_kernel(const S1Params p, int cpg,
                                                                      int tiles_per_seq) {
   extern __shared__ __align__(16) float sm[];
-  const int G = p.G, DL = p.DL, KC = p.KC, KC1 = KC - 1;
+  constexpr int TT = S1_TT, HALF = DL / 2, NTI = DL / 8, KST = DL / 16, MT = DL / 16;
+  const int G = p.G, KC = p.KC, KC1 = KC - 1, S = p.S;
   const int QK = (G + 1) * DL, CH = (G + 2) * DL;
-  const int WL = DL + 4;                             // padded filter row
-  float *Wc = sm;
-  float *Ps = Wc + QK * WL;
-  float *A = Ps + (S1_TT + KC1) * CH;
-  float *U = A + S1_TT * QK;
-  float *dU = U + S1_TT * QK;
-  float *Nn = dU + S1_TT * QK;
-  const int tid = threadIdx.x, nt = blockDim.x;
-  const int warp = tid >> 5, lane = tid & 31, nwarps = nt >> 5;
+  const int QKP = s1_pad(QK), CHP = s1_pad(CH), PR = TT + KC1;
+  float *Ps = sm;
+  float *Dq = Ps + 2 * PR * CHP;
+  float *Dv = Dq + 2 * TT * QKP;
+  float *A = Dv + 2 * (TT + 1) * DL;
+  float *U = A + TT * QKP;
+  float *Rt = U + TT * QKP;
+  float2 *turns = reinterpret_cast<float2 *>(Rt + TT * DL);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int gr = lane >> 2, qc = lane & 3;
   const int g = blockIdx.y, ci = blockIdx.x;
   const int units = p.B * tiles_per_seq;
   const int u_beg = static_cast<int>(static_cast<long long>(units) * ci / cpg);
   const int u_end = static_cast<int>(static_cast<long long>(units) * (ci + 1) / cpg);
   const int qcol0 = g * G * DL, kcol0 = p.NQ + g * DL, vcol0 = p.NQ + p.NKV + g * DL;
+  const bool qkm = (p.flags & F_QK_MEAN) != 0, norm = (p.flags & F_QK_NORM) != 0;
+  const bool rope = (p.flags & F_ROPE) != 0;
   auto head_glob = [&](int hh) { return hh < G ? g * G + hh : p.H + g; };
-  // the group's channel filters, [head][out i][in c]
-  for (int e = tid; e < QK * DL; e += nt) {
-    const int hh = e / (DL * DL), r = e % (DL * DL);
-    Wc[(hh * DL + r / DL) * WL + r % DL] = p.conv_chan[static_cast<size_t>(head_glob(hh)) * DL * DL + r];
-  }
-  const int BPH = (DL / 4) * (DL / 4);               // 4 x 4 filter-gradient blocks per head
-  const int NB = (G + 1) * BPH;
-  float acc[S1_MAX_PER_THREAD];
-#pragma unroll
-  for (int m = 0; m < S1_MAX_PER_THREAD; ++m) acc[m] = 0.f;
-  __syncthreads();
+  if (tid < 32) turns[tid] = make_float2(p.turns_hi[tid], p.turns_lo[tid]);
 
-  for (int u = u_beg; u < u_end; ++u) {
-    const int b = u / tiles_per_seq, t0 = (u % tiles_per_seq) * S1_TT;
-    // P rows t0-KC1 .. t0+TT-1 of the group's q | k | v channels (zero outside the sequence)
-    for (int e = tid; e < (S1_TT + KC1) * CH; e += nt) {
-      const int r = e / CH, c = e % CH;
+  auto issue = [&](int u, int k) {                  // tile u's inputs into buffer k
+    const int b = u / tiles_per_seq, t0 = (u % tiles_per_seq) * TT;
+    float *ps = Ps + k * PR * CHP, *dqs = Dq + k * TT * QKP, *dvs = Dv + k * (TT + 1) * DL;
+    const int C4 = CH / 4;
+    for (int e = tid; e < PR * C4; e += S1_THREADS) {
+      const int r = e / C4, c = (e % C4) * 4;
       const int t = t0 - KC1 + r;
       const int gc = c < G * DL ? qcol0 + c : (c < QK ? kcol0 + (c - G * DL) : vcol0 + (c - QK));
-      Ps[e] = (t >= 0 && t < p.S) ? p.P[(static_cast<size_t>(b) * p.S + t) * p.NQKV + gc] : 0.f;
+      const bool ok = t >= 0 && t < S;
+      cp_async16_zfill(ps + r * CHP + c, p.P + (static_cast<size_t>(b) * S + (ok ? t : 0)) * p.NQKV + gc, ok);
     }
+    constexpr int D4 = DL / 4;
+    for (int e = tid; e < TT * (G + 1) * D4; e += S1_THREADS) {
+      const int tt = e / ((G + 1) * D4), rem = e % ((G + 1) * D4), hh = rem / D4, i = (rem % D4) * 4;
+      const int t = t0 + tt;
+      const bool ok = t < S;
+      const size_t tr = ok ? t : 0;
+      const float *src = hh < G ? p.dq + ((static_cast<size_t>(b) * p.H + g * G + hh) * S + tr) * DL + i
+                                : p.dk + ((static_cast<size_t>(b) * p.Hkv + g) * S + tr) * DL + i;
+      cp_async16_zfill(dqs + tt * QKP + hh * DL + i, src, ok);
+    }
+    for (int e = tid; e < (TT + 1) * D4; e += S1_THREADS) {
+      const int tt = e / D4, i = (e % D4) * 4;
+      const int t = t0 + tt;
+      const bool ok = t < S;
+      cp_async16_zfill(dvs + tt * DL + i,
+                       p.dv + ((static_cast<size_t>(b) * p.Hkv + g) * S + (ok ? t : 0)) * DL + i, ok);
+    }
+  };
+
+  // filter-gradient blocks of this warp: (head, 16 out channels, 8 in channels)
+  const int NB = (G + 1) * MT * NTI;
+  const int BPW = (NB + S1_WARPS - 1) / S1_WARPS;
+  float accW[S1_MAXB][4];
+#pragma unroll
+  for (int m = 0; m < S1_MAXB; ++m) accW[m][0] = accW[m][1] = accW[m][2] = accW[m][3] = 0.f;
+
+  if (u_beg < u_end) issue(u_beg, 0);
+  cp_async_commit();
+  int k = 0;
+  for (int u = u_beg; u < u_end; ++u, k ^= 1) {
+    if (u + 1 < u_end) issue(u + 1, k ^ 1);
+    cp_async_commit();
+    cp_async_wait_one();                             // tile u's copies have landed
     __syncthreads();
-    // sequence conv of the q | k channels
-    for (int e = tid; e < S1_TT * QK; e += nt) {
-      const int tt = e / QK, c = e % QK;
+    const int b = u / tiles_per_seq, t0 = (u % tiles_per_seq) * TT;
+    const float *ps = Ps + k * PR * CHP, *dqs = Dq + k * TT * QKP, *dvs = Dv + k * (TT + 1) * DL;
+
+    // 1. sequence conv of the q | k channels (tap j of token t reads token t - (KC-1) + j),
+    //    and the tile's RoPE angles
+    for (int c = tid; c < QK; c += S1_THREADS) {
       const int gc = c < G * DL ? qcol0 + c : kcol0 + (c - G * DL);
-      float a = 0.f;
-      for (int j = 0; j < KC; ++j) a = fmaf(p.conv_seq[static_cast<size_t>(gc) * KC + j], Ps[(tt + j) * CH + c], a);
-      A[e] = a;
+      float w[S1_KCMAX];
+#pragma unroll
+      for (int j = 0; j < S1_KCMAX; ++j) w[j] = j < KC ? __ldg(p.conv_seq + static_cast<size_t>(gc) * KC + j) : 0.f;
+#pragma unroll 4
+      for (int tt = 0; tt < TT; ++tt) {
+        float a = 0.f;
+#pragma unroll
+        for (int j = 0; j < S1_KCMAX; ++j)
+          if (j < KC) a = fmaf(w[j], ps[(tt + j) * CHP + c], a);
+        A[tt * QKP + c] = a;
+      }
     }
+    if (rope)
+      for (int e = tid; e < TT * HALF; e += S1_THREADS) {
+        const int tt = e / HALF, i = e % HALF;
+        float cs, sn;
+        const float2 tr = turns[i];
+        rope_cos_sin_turns(t0 + tt, tr.x, tr.y, cs, sn);
+        Rt[2 * e] = cs;
+        Rt[2 * e + 1] = sn;
+      }
     __syncthreads();
-    // channel conv and Q-K-Mean: U = W_c A + skip; a thread per output channel, all TT tokens,
-    // the filter row and the tokens' inputs read four floats at a time
-    for (int hc = tid; hc < QK; hc += nt) {
-      const int hh = hc / DL, i = hc % DL;
-      const float4 *w4 = reinterpret_cast<const float4 *>(Wc + (hh * DL + i) * WL);
-      float v[S1_TT];
+
+    // 2. U = A W^T per head (+ Q-K-Mean's skip terms); a warp per (head, 8 out channels)
+    for (int task = warp; task < (G + 1) * NTI; task += S1_WARPS) {
+      const int hh = task / NTI, nt = task % NTI;
+      const uint2 *wb = p.wsplit + static_cast<size_t>(head_glob(hh)) * DL * (DL / 2);
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      const float *a0p = A + gr * QKP + hh * DL, *a1p = a0p + 8 * QKP;
 #pragma unroll
-      for (int tt = 0; tt < S1_TT; ++tt) v[tt] = 0.f;
-      for (int c4 = 0; c4 < DL / 4; ++c4) {
-        const float4 w = w4[c4];
-#pragma unroll
-        for (int tt = 0; tt < S1_TT; ++tt) {
-          const float4 a = reinterpret_cast<const float4 *>(A + tt * QK + hh * DL)[c4];
-          v[tt] = fmaf(w.x, a.x, fmaf(w.y, a.y, fmaf(w.z, a.z, fmaf(w.w, a.w, v[tt]))));
-        }
+      for (int ks = 0; ks < KST; ++ks) {
+        const int k0 = ks * 16 + 2 * qc;
+        uint32_t ah[4], al[4];
+        split_bf16x2(*reinterpret_cast<const float2 *>(a0p + k0), ah[0], al[0]);
+        split_bf16x2(*reinterpret_cast<const float2 *>(a1p + k0), ah[1], al[1]);
+        split_bf16x2(*reinterpret_cast<const float2 *>(a0p + k0 + 8), ah[2], al[2]);
+        split_bf16x2(*reinterpret_cast<const float2 *>(a1p + k0 + 8), ah[3], al[3]);
+        const uint2 *wr = wb + (nt * 8 + gr) * (DL / 2) + k0 / 2;
+        const uint2 w0 = __ldg(wr), w1 = __ldg(wr + 4);
+        const uint32_t bh[2] = {w0.x, w1.x}, bl[2] = {w0.y, w1.y};
+        mma_bf16_16816(acc, ah, bh);
+        mma_bf16_16816(acc, ah, bl);
+        mma_bf16_16816(acc, al, bh);
       }
 #pragma unroll
-      for (int tt = 0; tt < S1_TT; ++tt) {
-        float x = v[tt];
-        if (p.flags & F_QK_MEAN) {
-          const float *pr = Ps + (tt + KC1) * CH;
+      for (int e = 0; e < 4; ++e) {
+        const int tt = gr + 8 * (e >> 1), i = nt * 8 + 2 * qc + (e & 1);
+        float x = acc[e];
+        if (qkm) {                                   // post-conv + (pre-conv q + k) / 2
+          const float *pr = ps + (tt + KC1) * CHP;
           const float pk = pr[G * DL + i];
           float pq;
           if (hh < G) {
@@ -131,176 +204,260 @@ __global__ void __launch_bounds__(S1_THREADS, 1) stencil_bwd1_kernel(const S1Par
           }
           x += 0.5f * (pq + pk);
         }
-        U[tt * QK + hc] = x;
+        U[tt * QKP + hh * DL + i] = x;
       }
     }
     __syncthreads();
-    // per (token, head): norm statistics, dn = RoPE^-1(dq or dk), du; one warp per pair
-    for (int it = warp; it < S1_TT * (G + 1); it += nwarps) {
+
+    // 3. per (token, head): norm statistics, dn = RoPE^-1(dq or dk), du (over U in place); a
+    //    warp per pair, lane i holding the RoPE pair (i, i + d~/2)
+    for (int it = warp; it < TT * (G + 1); it += S1_WARPS) {
       const int tt = it / (G + 1), hh = it % (G + 1);
-      const int t = t0 + tt;
-      float *uu = U + tt * QK + hh * DL, *nn = Nn + tt * QK + hh * DL, *du = dU + tt * QK + hh * DL;
-      if (t >= p.S) {                                // past the sequence: no gradient
-        for (int c = lane; c < DL; c += 32) { du[c] = 0.f; nn[c] = 0.f; }
+      float *uu = U + tt * QKP + hh * DL;
+      const bool act = lane < HALF;
+      if (t0 + tt >= S) {                            // past the sequence: no gradient
+        if (act) { uu[lane] = 0.f; uu[lane + HALF] = 0.f; }
         continue;
       }
-      float ss = 0.f;
-      for (int c = lane; c < DL; c += 32) ss += uu[c] * uu[c];
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-      const bool norm = (p.flags & F_QK_NORM) != 0;
-      const float r = norm ? sqrtf(ss / static_cast<float>(DL) + p.eps) : 1.f;
-      const float *src = hh < G ? p.dq + ((static_cast<size_t>(b) * p.H + g * G + hh) * p.S + t) * DL
-                                : p.dk + ((static_cast<size_t>(b) * p.Hkv + g) * p.S + t) * DL;
-      const int HALF = DL / 2;
-      float dot = 0.f;
-      for (int i = lane; i < HALF; i += 32) {
-        float d1 = src[i], d2 = src[i + HALF];
-        if (p.flags & F_ROPE) {                      // rotate back by -t theta_i
-          float cs, sn;
-          rope_cos_sin(static_cast<double>(t) * p.theta[i], cs, sn);
+      const float *ds = dqs + tt * QKP + hh * DL;
+      float u1 = 0.f, u2 = 0.f, d1 = 0.f, d2 = 0.f;
+      if (act) {
+        u1 = uu[lane];
+        u2 = uu[lane + HALF];
+        d1 = ds[lane];
+        d2 = ds[lane + HALF];
+        if (rope) {                                  // rotate back by -t theta_i
+          const float cs = Rt[2 * (tt * HALF + lane)], sn = Rt[2 * (tt * HALF + lane) + 1];
           const float a1 = d1 * cs + d2 * sn, a2 = -d1 * sn + d2 * cs;
           d1 = a1;
           d2 = a2;
         }
-        const float n1 = uu[i] / r, n2 = uu[i + HALF] / r;
-        nn[i] = n1;
-        nn[i + HALF] = n2;
-        du[i] = d1;                                  // dn for now
-        du[i + HALF] = d2;
-        dot += d1 * n1 + d2 * n2;
       }
+      float ss = u1 * u1 + u2 * u2;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      const float inv_r = norm ? rsqrtf(ss / static_cast<float>(DL) + p.eps) : 1.f;
+      const float n1 = u1 * inv_r, n2 = u2 * inv_r;
+      float dot = d1 * n1 + d2 * n2;
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-      __syncwarp();
       if (norm) {
         const float mdn = dot / static_cast<float>(DL);
-        for (int c = lane; c < DL; c += 32) du[c] = (du[c] - nn[c] * mdn) / r;
+        d1 = (d1 - n1 * mdn) * inv_r;
+        d2 = (d2 - n2 * mdn) * inv_r;
+      }
+      if (act) {
+        uu[lane] = d1;
+        uu[lane + HALF] = d2;
       }
     }
     __syncthreads();
-    // dA = W_c^T dU per head, and the Q-K-Mean skip gradients of the q | k projections; a
-    // thread per input channel, all TT tokens, the tokens' dU read four floats at a time
-    for (int hc = tid; hc < QK; hc += nt) {
-      const int hh = hc / DL, c = hc % DL;
-      float v[S1_TT];
+
+    // 4. dA = dU W per head (the channel conv's transpose); a warp per (head, 8 in channels)
+    for (int task = warp; task < (G + 1) * NTI; task += S1_WARPS) {
+      const int hh = task / NTI, nt = task % NTI;
+      const uint2 *wt = p.wsplitT + static_cast<size_t>(head_glob(hh)) * DL * (DL / 2);
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      const float *a0p = U + gr * QKP + hh * DL, *a1p = a0p + 8 * QKP;
 #pragma unroll
-      for (int tt = 0; tt < S1_TT; ++tt) v[tt] = 0.f;
-      for (int i4 = 0; i4 < DL / 4; ++i4) {
-        const float *wc = Wc + (hh * DL + 4 * i4) * WL + c;
-        const float w0 = wc[0], w1 = wc[WL], w2 = wc[2 * WL], w3 = wc[3 * WL];
-#pragma unroll
-        for (int tt = 0; tt < S1_TT; ++tt) {
-          const float4 d = reinterpret_cast<const float4 *>(dU + tt * QK + hh * DL)[i4];
-          v[tt] = fmaf(w0, d.x, fmaf(w1, d.y, fmaf(w2, d.z, fmaf(w3, d.w, v[tt]))));
-        }
+      for (int ks = 0; ks < KST; ++ks) {
+        const int k0 = ks * 16 + 2 * qc;
+        uint32_t ah[4], al[4];
+        split_bf16x2(*reinterpret_cast<const float2 *>(a0p + k0), ah[0], al[0]);
+        split_bf16x2(*reinterpret_cast<const float2 *>(a1p + k0), ah[1], al[1]);
+        split_bf16x2(*reinterpret_cast<const float2 *>(a0p + k0 + 8), ah[2], al[2]);
+        split_bf16x2(*reinterpret_cast<const float2 *>(a1p + k0 + 8), ah[3], al[3]);
+        const uint2 *wr = wt + (nt * 8 + gr) * (DL / 2) + k0 / 2;
+        const uint2 w0 = __ldg(wr), w1 = __ldg(wr + 4);
+        const uint32_t bh[2] = {w0.x, w1.x}, bl[2] = {w0.y, w1.y};
+        mma_bf16_16816(acc, ah, bh);
+        mma_bf16_16816(acc, ah, bl);
+        mma_bf16_16816(acc, al, bh);
       }
+      const int c = nt * 8 + 2 * qc;
       const int gc = hh < G ? qcol0 + hh * DL + c : kcol0 + c;
 #pragma unroll
-      for (int tt = 0; tt < S1_TT; ++tt) {
-        const int t = t0 + tt;
-        if (t >= p.S) continue;
-        const size_t row = static_cast<size_t>(b) * p.S + t;
-        p.dA[row * (p.NQ + p.NKV) + gc] = v[tt];
+      for (int h2 = 0; h2 < 2; ++h2) {
+        const int t = t0 + gr + 8 * h2;
+        if (t < S)
+          *reinterpret_cast<float2 *>(p.dA + (static_cast<size_t>(b) * S + t) * (p.NQ + p.NKV) + gc) =
+              make_float2(acc[2 * h2], acc[2 * h2 + 1]);
+      }
+    }
+    // Q-K-Mean's skip gradients of the q | k projections, and the value gradients (the
+    // value-shift undone: a shifted channel of token t received dv of token t + 1)
+    for (int e = tid; e < TT * CH; e += S1_THREADS) {
+      const int tt = e / CH, c = e % CH;
+      const int t = t0 + tt;
+      if (t >= S) continue;
+      const size_t row = static_cast<size_t>(b) * S + t;
+      if (c < QK) {
         float skip = 0.f;
-        if (p.flags & F_QK_MEAN) {
-          const float duk = dU[tt * QK + G * DL + c];
-          if (hh < G) {
-            skip = 0.5f * dU[tt * QK + hh * DL + c] + duk / (2.0f * static_cast<float>(G));
+        if (qkm) {
+          const int i = c % DL;
+          const float duk = U[tt * QKP + G * DL + i];
+          if (c < G * DL) {
+            skip = 0.5f * U[tt * QKP + c] + duk / (2.0f * static_cast<float>(G));
           } else {
             float sq = 0.f;
-            for (int h2 = 0; h2 < G; ++h2) sq += dU[tt * QK + h2 * DL + c];
+            for (int h2 = 0; h2 < G; ++h2) sq += U[tt * QKP + h2 * DL + i];
             skip = 0.5f * sq + 0.5f * duk;
           }
         }
+        const int gc = c < G * DL ? qcol0 + c : kcol0 + (c - G * DL);
         p.dPpart[row * p.NQKV + gc] = skip;
+      } else {
+        const int i = c - QK;
+        const bool shifted = (p.flags & F_VALUE_SHIFT) && g * DL + i >= p.VS0;
+        p.dPpart[row * p.NQKV + vcol0 + i] = dvs[(tt + (shifted ? 1 : 0)) * DL + i];
       }
     }
-    // values: dPv[t, c] = dv[t, c] unshifted, dv[t+1, c] shifted
-    for (int e = tid; e < S1_TT * DL; e += nt) {
-      const int tt = e / DL, c = e % DL;
-      const int t = t0 + tt;
-      if (t >= p.S) continue;
-      const int gvc = g * DL + c;
-      const bool shifted = (p.flags & F_VALUE_SHIFT) && gvc >= p.VS0;
-      const int ts = shifted ? t + 1 : t;
-      const float val = ts < p.S ? p.dv[((static_cast<size_t>(b) * p.Hkv + g) * p.S + ts) * DL + c] : 0.f;
-      p.dPpart[(static_cast<size_t>(b) * p.S + t) * p.NQKV + vcol0 + c] = val;
-    }
-    // channel-filter gradient: dW_c[h][i][c] += sum_tt dU[tt][h][i] A[tt][h][c], a 4 x 4 block
-    // of (i, c) per thread and block slot
+    // 5. dW[h][i][c] += sum over the tile's tokens of dU[t][h][i] A[t][h][c]
 #pragma unroll
-    for (int m = 0; m < S1_MAX_BLOCKS; ++m) {
-      const int blk = tid + m * S1_THREADS;
-      if (blk < NB) {
-        const int hh = blk / BPH, r = blk % BPH;
-        const int i0 = (r / (DL / 4)) * 4, c0 = (r % (DL / 4)) * 4;
-#pragma unroll
-        for (int tt = 0; tt < S1_TT; ++tt) {
-          const float4 d = *reinterpret_cast<const float4 *>(dU + tt * QK + hh * DL + i0);
-          const float4 a = *reinterpret_cast<const float4 *>(A + tt * QK + hh * DL + c0);
-          const float dv4[4] = {d.x, d.y, d.z, d.w}, av4[4] = {a.x, a.y, a.z, a.w};
-#pragma unroll
-          for (int ii = 0; ii < 4; ++ii)
-#pragma unroll
-            for (int cc = 0; cc < 4; ++cc)
-              acc[m * 16 + ii * 4 + cc] = fmaf(dv4[ii], av4[cc], acc[m * 16 + ii * 4 + cc]);
-        }
+    for (int m = 0; m < S1_MAXB; ++m) {
+      const int blk = warp * BPW + m;
+      if (m < BPW && blk < NB) {
+        const int hh = blk / (MT * NTI), rem = blk % (MT * NTI);
+        const int cu = hh * DL + (rem / NTI) * 16 + gr;   // dU column (out channel i)
+        const int ca = hh * DL + (rem % NTI) * 8 + gr;    // A column (in channel c)
+        uint32_t ah[4], al[4], bh[2], bl[2];
+        split_bf16x2(make_float2(U[(2 * qc) * QKP + cu], U[(2 * qc + 1) * QKP + cu]), ah[0], al[0]);
+        split_bf16x2(make_float2(U[(2 * qc) * QKP + cu + 8], U[(2 * qc + 1) * QKP + cu + 8]), ah[1], al[1]);
+        split_bf16x2(make_float2(U[(2 * qc + 8) * QKP + cu], U[(2 * qc + 9) * QKP + cu]), ah[2], al[2]);
+        split_bf16x2(make_float2(U[(2 * qc + 8) * QKP + cu + 8], U[(2 * qc + 9) * QKP + cu + 8]), ah[3], al[3]);
+        split_bf16x2(make_float2(A[(2 * qc) * QKP + ca], A[(2 * qc + 1) * QKP + ca]), bh[0], bl[0]);
+        split_bf16x2(make_float2(A[(2 * qc + 8) * QKP + ca], A[(2 * qc + 9) * QKP + ca]), bh[1], bl[1]);
+        mma_bf16_16816(accW[m], ah, bh);
+        mma_bf16_16816(accW[m], ah, bl);
+        mma_bf16_16816(accW[m], al, bh);
       }
     }
-    __syncthreads();                                 // Ps, A, U, dU rewritten by the next tile
+    __syncthreads();                                 // A, U and this buffer reused next
   }
+  cp_async_wait_none();
 #pragma unroll
-  for (int m = 0; m < S1_MAX_BLOCKS; ++m) {
-    const int blk = tid + m * S1_THREADS;
-    if (blk < NB && u_end > u_beg) {
-      const int hh = blk / BPH, r = blk % BPH;
-      const int i0 = (r / (DL / 4)) * 4, c0 = (r % (DL / 4)) * 4;
+  for (int m = 0; m < S1_MAXB; ++m) {
+    const int blk = warp * BPW + m;
+    if (m < BPW && blk < NB && u_end > u_beg) {
+      const int hh = blk / (MT * NTI), rem = blk % (MT * NTI);
+      const int i = (rem / NTI) * 16 + gr, c = (rem % NTI) * 8 + 2 * qc;
       float *dst = p.dconv_chan + static_cast<size_t>(head_glob(hh)) * DL * DL;
-#pragma unroll
-      for (int ii = 0; ii < 4; ++ii)
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc)
-          atomicAdd(dst + (i0 + ii) * DL + c0 + cc, acc[m * 16 + ii * 4 + cc]);
+      atomicAdd(dst + i * DL + c, accW[m][0]);
+      atomicAdd(dst + i * DL + c + 1, accW[m][1]);
+      atomicAdd(dst + (i + 8) * DL + c, accW[m][2]);
+      atomicAdd(dst + (i + 8) * DL + c + 1, accW[m][3]);
     }
   }
 }
 
-// Pass 2: one thread per (q|k channel, token range); the sequence conv's transpose and its
-// filter gradient, then dP in bfloat16 (the value columns are converted as they are).
-constexpr int S2_TOK = 256;                          // tokens per thread's range
+// The channel filters transposed and split: out[(head * DL + c) * DL/2 + i/2] = the bf16 hi / lo
+// pairs of (W[head][i][c], W[head][i+1][c]).
+__global__ void split_conv_chan_t_kernel(const float *__restrict__ w, uint2 *__restrict__ out,
+                                         int heads, int DL) {
+  const int half = DL / 2;
+  const size_t n = static_cast<size_t>(heads) * DL * half;
+  for (size_t e = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < n;
+       e += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const int ip = static_cast<int>(e % half);
+    const int c = static_cast<int>((e / half) % DL);
+    const size_t h = e / (static_cast<size_t>(half) * DL);
+    const float *wh = w + h * DL * DL;
+    uint2 r;
+    split_bf16x2(make_float2(wh[(2 * ip) * DL + c], wh[(2 * ip + 1) * DL + c]), r.x, r.y);
+    out[e] = r;
+  }
+}
+
+// Pass 2: a CTA per (32 columns of dP, 256 rows), a warp per 32-row slice of them (so every
+// load and store of a warp covers 32 consecutive columns of one row); the sequence conv's
+// transpose and its filter gradient from sliding windows of dA (rows t .. t+KC-1) and P (rows
+// t-KC+1 .. t) held in registers, then dP in bfloat16 (the value columns converted as they
+// are).  The filter gradient is summed over the CTA's warps in shared memory and added once
+// per CTA.
+constexpr int S2_COLS = 32;
+constexpr int S2_SUB = 32;                           // rows per warp
+constexpr int S2_WARPS = 8;
+constexpr int S2_KCMAX = 8;
 
 __global__ void __launch_bounds__(256) stencil_bwd2_kernel(
     const float *__restrict__ P, const float *__restrict__ dA, const float *__restrict__ dPpart,
     const float *__restrict__ conv_seq, __nv_bfloat16 *__restrict__ dP, float *__restrict__ dconv_seq,
     int B, int S, int NQ, int NKV, int NQKV, int KC) {
-  const int c = blockIdx.x * blockDim.x + threadIdx.x;   // column of dP (all NQKV)
-  const int seg = blockIdx.y;                            // token range of (B*S)
-  if (c >= NQKV) return;
+  __shared__ float red[S2_WARPS][S2_KCMAX][S2_COLS];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int c = blockIdx.x * S2_COLS + lane;             // column of dP (all NQKV)
   const long long M = static_cast<long long>(B) * S;
-  const long long t_beg = static_cast<long long>(seg) * S2_TOK;
-  const long long t_end = t_beg + S2_TOK < M ? t_beg + S2_TOK : M;
-  const bool qk = c < NQ + NKV;
-  float w[8], dw[8];
-  for (int j = 0; j < 8; ++j) {
+  const long long r_beg = (static_cast<long long>(blockIdx.y) * S2_WARPS + warp) * S2_SUB;
+  const long long r_end = r_beg + S2_SUB < M ? r_beg + S2_SUB : M;
+  const int W = NQ + NKV;
+  const bool live = c < NQKV;
+  const bool qk = live && c < W;
+  float w[S2_KCMAX], dw[S2_KCMAX];
+#pragma unroll
+  for (int j = 0; j < S2_KCMAX; ++j) {
     w[j] = (qk && j < KC) ? conv_seq[static_cast<size_t>(c) * KC + j] : 0.f;
     dw[j] = 0.f;
   }
-  const int W = NQ + NKV;
-  for (long long row = t_beg; row < t_end; ++row) {
-    const int t = static_cast<int>(row % S);
-    float v = dPpart[row * NQKV + c];
-    if (qk) {
-      for (int j = 0; j < KC; ++j) {
-        const int lag = KC - 1 - j;                      // output t + lag read input t by tap j
-        if (t + lag < S) v = fmaf(w[j], dA[(row + lag) * W + c], v);
-        if (t - lag >= 0) dw[j] = fmaf(dA[row * W + c], P[(row - lag) * NQKV + c], dw[j]);
+  if (qk) {
+    // windows: da[l] = dA[row + l] (l < KC, zero past the sequence), pp[l] = P[row - l]
+    // (zero before the sequence start), for the current row
+    float da[S2_KCMAX], pp[S2_KCMAX];
+    if (r_beg < r_end) {
+      const int t0 = static_cast<int>(r_beg % S);
+#pragma unroll
+      for (int l = 0; l < S2_KCMAX; ++l) {
+        da[l] = (l < KC && t0 + l < S) ? dA[(r_beg + l) * W + c] : 0.f;
+        pp[l] = (l < KC && t0 - l >= 0) ? P[(r_beg - l) * NQKV + c] : 0.f;
       }
     }
-    dP[row * NQKV + c] = __float2bfloat16_rn(v);
+    for (long long row = r_beg; row < r_end; ++row) {
+      const int t = static_cast<int>(row % S);
+      float v = dPpart[row * NQKV + c];
+#pragma unroll
+      for (int j = 0; j < S2_KCMAX; ++j) {
+        if (j < KC) {
+          const int lag = KC - 1 - j;                    // output t + lag read input t by tap j
+          v = fmaf(w[j], da[lag], v);                    // da[lag] is zero past the sequence
+          dw[j] = fmaf(da[0], pp[lag], dw[j]);           // pp[lag] is zero before its start
+        }
+      }
+      dP[row * NQKV + c] = __float2bfloat16_rn(v);
+      // slide both windows by one row
+#pragma unroll
+      for (int l = S2_KCMAX - 1; l > 0; --l) pp[l] = pp[l - 1];
+#pragma unroll
+      for (int l = 0; l + 1 < S2_KCMAX; ++l) da[l] = da[l + 1];
+      const long long nrow = row + 1;
+      if (nrow < r_end) {
+        const int nt = t + 1 == S ? 0 : t + 1;           // a new sequence starts at nt == 0
+        pp[0] = P[nrow * NQKV + c];
+        if (nt == 0) {
+#pragma unroll
+          for (int l = 1; l < S2_KCMAX; ++l) pp[l] = 0.f;
+#pragma unroll
+          for (int l = 0; l < S2_KCMAX; ++l)
+            da[l] = (l < KC && l < S) ? dA[(nrow + l) * W + c] : 0.f;
+        } else {
+          const int l = KC - 1;                          // the window's new last row
+          if (l < S2_KCMAX) da[l] = nt + l < S ? dA[(nrow + l) * W + c] : 0.f;
+        }
+      }
+    }
+  } else if (live) {
+    for (long long row = r_beg; row < r_end; ++row)
+      dP[row * NQKV + c] = __float2bfloat16_rn(dPpart[row * NQKV + c]);
   }
-  if (qk)
-    for (int j = 0; j < KC; ++j) atomicAdd(dconv_seq + static_cast<size_t>(c) * KC + j, dw[j]);
+#pragma unroll
+  for (int j = 0; j < S2_KCMAX; ++j) red[warp][j][lane] = dw[j];
+  __syncthreads();
+  if (warp == 0 && qk) {
+    for (int j = 0; j < KC; ++j) {
+      float sum = 0.f;
+#pragma unroll
+      for (int w2 = 0; w2 < S2_WARPS; ++w2) sum += red[w2][j][lane];
+      atomicAdd(dconv_seq + static_cast<size_t>(c) * KC + j, sum);
+    }
+  }
 }
 
 // out[c][r] = in[r][c] for r < R, zero for R <= r < R8 (R8 = R rounded up to 8, so every output
@@ -335,41 +492,59 @@ __global__ void __launch_bounds__(256) transpose16_kernel(const uint16_t *__rest
 }  // namespace
 
 bool stencil_backward_supported(const Dims &d) {
-  return d.bf16 && !(d.flags & F_NO_CONV) && d.DL <= 64 && d.KC <= 8 &&
-         (d.G + 1) * (d.DL / 4) * (d.DL / 4) <= S1_MAX_BLOCKS * S1_THREADS &&
+  return d.bf16 && !(d.flags & F_NO_CONV) && (d.DL == 16 || d.DL == 32 || d.DL == 64) &&
+         d.KC <= S1_KCMAX && (d.G + 1) * (d.DL / 16) * (d.DL / 8) <= S1_WARPS * S1_MAXB &&
          s1_smem_floats(d.G, d.DL, d.KC) * 4 <= 200 * 1024;
+}
+
+template <int DL>
+cudaError_t launch_bwd1(const Dims &d, const S1Params &p, int cpg, int tiles, cudaStream_t st) {
+  const size_t smem = s1_smem_floats(d.G, DL, d.KC) * 4;
+  cudaError_t e;
+  if ((e = ensure_dyn_smem<stencil_bwd1_kernel<DL>>(smem)) != cudaSuccess) return e;
+  stencil_bwd1_kernel<DL><<<dim3(cpg, d.Hkv), S1_THREADS, smem, st>>>(p, cpg, tiles);
+  return cudaGetLastError();
 }
 
 cudaError_t stencil_backward(const Dims &d, const StencilBwdArgs &a, cudaStream_t st) {
   if (d.B == 0 || d.S == 0) return cudaSuccess;
+  if (!stencil_backward_supported(d)) return cudaErrorInvalidValue;
+  cudaError_t e;
+  {
+    const int heads = d.H + d.Hkv;
+    const size_t n = static_cast<size_t>(heads) * d.DL * (d.DL / 2);
+    const int blocks = static_cast<int>((n + 255) / 256);
+    split_conv_chan_t_kernel<<<blocks, 256, 0, st>>>(a.conv_chan, static_cast<uint2 *>(a.conv_chan_split_t),
+                                                     heads, d.DL);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
   S1Params p;
   p.P = a.P;
   p.dq = a.dq;
   p.dk = a.dk;
   p.dv = a.dv;
   p.conv_seq = a.conv_seq;
-  p.conv_chan = a.conv_chan;
+  p.wsplit = static_cast<const uint2 *>(a.conv_chan_split);
+  p.wsplitT = static_cast<const uint2 *>(a.conv_chan_split_t);
   p.dA = a.dA;
   p.dPpart = a.dPpart;
   p.dconv_chan = a.dconv_chan;
-  p.B = d.B; p.S = d.S; p.H = d.H; p.Hkv = d.Hkv; p.G = d.G; p.DL = d.DL;
+  p.B = d.B; p.S = d.S; p.H = d.H; p.Hkv = d.Hkv; p.G = d.G;
   p.NQ = d.NQ; p.NKV = d.NKV; p.NQKV = d.NQKV; p.KC = d.KC; p.VS0 = d.VS0;
   p.flags = d.flags;
   p.eps = d.eps;
-  for (int i = 0; i < 32; ++i)
-    p.theta[i] = i < d.DL / 2 ? pow(static_cast<double>(d.rope_base), -2.0 * i / d.DL) : 0.0;
+  rope_turns_host(d.DL, d.rope_base, p.turns_hi, p.turns_lo, 32);
   const int tiles = (d.S + S1_TT - 1) / S1_TT;
   const int units = d.B * tiles;
   int cpg = num_sms() / d.Hkv;
   if (cpg < 1) cpg = 1;
   if (cpg > units) cpg = units;
-  const size_t smem = s1_smem_floats(d.G, d.DL, d.KC) * 4;
-  cudaError_t e;
-  if ((e = ensure_dyn_smem<stencil_bwd1_kernel>(smem)) != cudaSuccess) return e;
-  stencil_bwd1_kernel<<<dim3(cpg, d.Hkv), S1_THREADS, smem, st>>>(p, cpg, tiles);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  e = d.DL == 16 ? launch_bwd1<16>(d, p, cpg, tiles, st)
+    : d.DL == 32 ? launch_bwd1<32>(d, p, cpg, tiles, st) : launch_bwd1<64>(d, p, cpg, tiles, st);
+  if (e != cudaSuccess) return e;
   const long long M = static_cast<long long>(d.B) * d.S;
-  const dim3 g2((d.NQKV + 255) / 256, static_cast<unsigned>((M + S2_TOK - 1) / S2_TOK));
+  const long long rows_per_cta = static_cast<long long>(S2_WARPS) * S2_SUB;
+  const dim3 g2((d.NQKV + S2_COLS - 1) / S2_COLS, static_cast<unsigned>((M + rows_per_cta - 1) / rows_per_cta));
   stencil_bwd2_kernel<<<g2, 256, 0, st>>>(a.P, a.dA, a.dPpart, a.conv_seq,
                                          static_cast<__nv_bfloat16 *>(a.dP), a.dconv_seq, d.B, d.S,
                                          d.NQ, d.NKV, d.NQKV, d.KC);

@@ -463,8 +463,8 @@ CCA_API int cca_prefill_forward(const cca_config_t *cfg, const cca_weights_t *w,
 namespace {
 // ------------------------------------------------------------------ backward pass
 struct BackwardLayout {
-  size_t status, wsplit, P, q, k, v, o, lse, D, woT, dO, dyT, oT, dq, dk, dv, dA, dPpart, dP,
-      wqkvT, dPT, xT, total;
+  size_t status, wsplit, wsplitT, P, q, k, v, o, lse, D, woT, dO, dyT, oT, dq, dk, dv, dA, dPpart,
+      dP, wqkvT, dPT, xT, total;
 };
 
 BackwardLayout backward_layout(const cca::Dims &d, int B, int S) {
@@ -475,6 +475,7 @@ BackwardLayout backward_layout(const cca::Dims &d, int B, int S) {
   auto take = [&](size_t bytes) { const size_t o = off; off += align256(bytes); return o; };
   L.status = take(256);
   L.wsplit = take(cca::conv_chan_split_bytes(d));
+  L.wsplitT = take(cca::conv_chan_split_bytes(d));
   L.P = take(M * d.NQKV * 4);
   L.q = take(M * d.NQ * 2);
   L.k = take(M * d.NKV * 2);
@@ -606,6 +607,8 @@ CCA_API int cca_backward(const cca_config_t *cfg, const cca_weights_t *w, const 
   sb.dv = ab.dv;
   sb.conv_seq = w->conv_seq;
   sb.conv_chan = w->conv_chan;
+  sb.conv_chan_split = ws + L.wsplit;
+  sb.conv_chan_split_t = ws + L.wsplitT;
   sb.dA = reinterpret_cast<float *>(ws + L.dA);
   sb.dPpart = reinterpret_cast<float *>(ws + L.dPpart);
   sb.dP = ws + L.dP;

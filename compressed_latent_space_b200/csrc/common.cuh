@@ -6,6 +6,7 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
+#include <math.h>
 #include <stdint.h>
 
 #include <atomic>
@@ -182,6 +183,28 @@ __device__ __forceinline__ void rope_cos_sin(double angle, float &c, float &s) {
   const double k = rint(angle * (1.0 / two_pi));
   const float r = static_cast<float>(fma(-k, two_pi, angle));
   __sincosf(r, &s, &c);
+}
+
+// cos and sin of t * theta_i without double precision: the angle in turns is t * (hi + lo);
+// t * hi is split into its rounded product and the product's exact rounding error (an FMA),
+// the rounded product's whole turns are dropped exactly, and the rest (|r| <= 1/2 + tiny) is
+// scaled to radians.  The reduced angle is good to a few 1e-8 turns for t < 2^24.
+__device__ __forceinline__ void rope_cos_sin_turns(int t, float hi, float lo, float &c, float &s) {
+  const float tf = static_cast<float>(t);
+  const float prod = tf * hi;
+  const float err = fmaf(tf, hi, -prod);
+  const float r = (prod - rintf(prod)) + fmaf(tf, lo, err);
+  __sincosf(r * 6.2831853071795865f, &s, &c);
+}
+
+// Host side of rope_cos_sin_turns: frequency i of a d~-wide latent, base^(-2i/d~) / (2 pi)
+// turns, as a float pair hi + lo (n entries, zero past d~/2).
+inline void rope_turns_host(int DL, double base, float *hi, float *lo, int n) {
+  for (int i = 0; i < n; ++i) {
+    const double turns = i < DL / 2 ? pow(base, -2.0 * i / DL) / 6.283185307179586 : 0.0;
+    hi[i] = static_cast<float>(turns);
+    lo[i] = static_cast<float>(turns - static_cast<double>(hi[i]));
+  }
 }
 
 // ----------------------------------------------------------------------------- cp.async

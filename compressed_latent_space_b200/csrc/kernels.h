@@ -126,6 +126,8 @@ cudaError_t attention_rowdot(const Dims &d, const void *dO, const void *O, float
 // the caller).  dA and dPpart are float32 scratch, [B*S, NQ+NKV] and [B*S, NQKV].
 struct StencilBwdArgs {
   const float *P, *dq, *dk, *dv, *conv_seq, *conv_chan;
+  const void *conv_chan_split;     // split_conv_chan's output for these filters
+  void *conv_chan_split_t;         // scratch of conv_chan_split_bytes: the transposed split
   float *dA, *dPpart;
   void *dP;
   float *dconv_seq, *dconv_chan;

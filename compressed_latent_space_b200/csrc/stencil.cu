@@ -675,18 +675,6 @@ struct PointParams {
   float turns_hi[64], turns_lo[64];
 };
 
-// cos and sin of t * theta_i without double precision: the angle in turns is t * (hi + lo);
-// t * hi is split into its rounded product and the product's exact rounding error (an FMA),
-// the rounded product's whole turns are dropped exactly, and the rest (|r| <= 1/2 + tiny) is
-// scaled to radians.  The reduced angle is good to a few 1e-8 turns for t < 2^24.
-__device__ __forceinline__ void rope_cos_sin_turns(int t, float hi, float lo, float &c, float &s) {
-  const float tf = static_cast<float>(t);
-  const float prod = tf * hi;
-  const float err = fmaf(tf, hi, -prod);
-  const float r = (prod - rintf(prod)) + fmaf(tf, lo, err);
-  __sincosf(r * 6.2831853071795865f, &s, &c);
-}
-
 template <typename TL>
 __device__ __forceinline__ void store4(TL *dst, const float (&x)[4]) {
   if constexpr (sizeof(TL) == 2) {
@@ -862,12 +850,7 @@ cudaError_t launch_pointwise(const Dims &d, const StencilArgs &a, cudaStream_t s
   p.kv_stride = a.kv_stride;
   p.flags = d.flags;
   p.eps = d.eps;
-  for (int i = 0; i < 64; ++i) {
-    const double turns = i < d.DL / 2
-        ? pow(static_cast<double>(d.rope_base), -2.0 * i / d.DL) / 6.283185307179586 : 0.0;
-    p.turns_hi[i] = static_cast<float>(turns);
-    p.turns_lo[i] = static_cast<float>(turns - static_cast<double>(p.turns_hi[i]));
-  }
+  rope_turns_host(d.DL, d.rope_base, p.turns_hi, p.turns_lo, 64);
   const long long units = static_cast<long long>(d.B) * d.S * (d.H + 2 * d.Hkv);
   const long long threads = units * (d.DL / 8);
   if (threads >= (1LL << 30) || d.S >= (1 << 24)) return cudaErrorInvalidValue;

@@ -51,6 +51,29 @@ def test_backward_matches_oracle(cuda_lib, shape, flags):
     check(grads, ref, w.dl)
 
 
+@pytest.mark.parametrize("shape", [
+    dict(d_model=256, n_heads=4, n_kv_heads=2, compression=2, seq=77, conv_kernel=1),
+    dict(d_model=256, n_heads=4, n_kv_heads=2, compression=2, seq=150, conv_kernel=2),
+    dict(d_model=256, n_heads=4, n_kv_heads=2, compression=2, seq=33, conv_kernel=6),
+    dict(d_model=256, n_heads=4, n_kv_heads=2, compression=2, seq=260, conv_kernel=8),
+    dict(d_model=512, n_heads=8, n_kv_heads=1, compression=2, seq=140),    # d~=32, G=8
+    dict(d_model=256, n_heads=2, n_kv_heads=1, compression=2, seq=5),      # d~=64, G=2, S < tile
+])
+def test_backward_conv_widths_and_groups(cuda_lib, shape):
+    """Conv widths 1..8 (the halo of the sequence conv's transpose across tiles and sequence
+    starts), a group of 8 query heads, a sequence shorter than one tile."""
+    shape = dict(shape)
+    S = shape.pop("seq")
+    w = W.Workload("bwd_kc", 2, S, **shape)
+    inp = W.make_inputs(w, seed=31, conv_std=0.4, identity_conv=True)
+    g = torch.Generator("cpu").manual_seed(32)
+    dy = torch.randn(w.batch, S, w.d_model, generator=g).to(torch.bfloat16)
+    grads = run_backward(cuda_lib, w, inp, dy)
+    ocfg = oracle_config(w)
+    ref = OB.backward(ocfg, oracle_weights(ocfg, inp), f64(inp.x), f64(dy))
+    check(grads, ref, w.dl)
+
+
 def test_backward_long_sequence(cuda_lib):
     """The 16k workload's heads (E=2048, 16 query / 4 kv heads, d~=64) over 1024 tokens: many
     key and query tiles per head, the conv widths' halo across tiles."""
