@@ -224,19 +224,25 @@ __global__ void __launch_bounds__(B_THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->s_free);    // the next tile's S / dP may overwrite
+      // dS = P * (dP - D) on pairs of keys: one packed FMA for the exponents, two MUFU ex2,
+      // packed subtract and multiply; keys past this row's query masked on the diagonal tile
       const bool diag = j == qt;
+      const uint64_t sc2 = f2(scale_log2, scale_log2), nl2 = f2(-lrow, -lrow), nd2 = f2(-drow, -drow);
       uint32_t pk[32];
 #pragma unroll
       for (int e = 0; e < 32; ++e) {
-        float ds[2];
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int kcol = hf * 64 + 2 * e + u;
-          float p = ex2(__uint_as_float(rs[2 * e + u]) * scale_log2 - lrow);
-          if (diag && kcol > row) p = 0.f;
-          ds[u] = p * (__uint_as_float(rp[2 * e + u]) - drow);
+        float x0, x1;
+        unf2(fma2(f2(__uint_as_float(rs[2 * e]), __uint_as_float(rs[2 * e + 1])), sc2, nl2), x0, x1);
+        float p0 = ex2(x0), p1 = ex2(x1);
+        if (diag) {
+          const int kcol = hf * 64 + 2 * e;
+          if (kcol > row) p0 = 0.f;
+          if (kcol + 1 > row) p1 = 0.f;
         }
-        pk[e] = pack_f16x2(ds[0], ds[1]);
+        const uint64_t t2 = add2(f2(__uint_as_float(rp[2 * e]), __uint_as_float(rp[2 * e + 1])), nd2);
+        float d0, d1;
+        unf2(mul2(f2(p0, p1), t2), d0, d1);
+        pk[e] = pack_f16x2(d0, d1);
       }
       // the previous tile's dQ MMA must have read its dS before this one is written
       if (j > 0) ok = __all_sync(0xffffffffu, mbar_wait(&bars->pds_free, (j - 1) & 1, abort, status));
@@ -410,9 +416,9 @@ __global__ void __launch_bounds__(B_THREADS, 1)
       const int qt = kt + n / G, h = g * G + n % G;
       const int q = qt * BT + threadIdx.x;
       const size_t ridx = (static_cast<size_t>(b) * H + h) * S + q;
-      float *buf = sL + (n & 1) * 2 * BT;
-      buf[threadIdx.x] = q < S ? lse[ridx] : INFINITY;
-      buf[BT + threadIdx.x] = q < S ? Dd[ridx] : 0.f;
+      float *buf = sL + (n & 1) * 2 * BT;             // negated, for the packed FMA / add
+      buf[threadIdx.x] = q < S ? -lse[ridx] : -INFINITY;
+      buf[BT + threadIdx.x] = q < S ? -Dd[ridx] : 0.f;
     };
     stage_stats(0);
     bool ok = true;
@@ -428,20 +434,28 @@ __global__ void __launch_bounds__(B_THREADS, 1)
       if (lane == 0) mbar_arrive(&bars->s_free);
       const int qt = kt + n / G;
       const bool diag = qt == kt;
+      // per query column: -lse and -D (broadcast 8-byte shared-memory reads), then P^T and
+      // dS^T on pairs of queries with packed FMA / subtract / multiply
       const float *bl = sL + (n & 1) * 2 * BT + hf * 64, *bd = bl + BT;
+      const uint64_t sc2 = f2(scale_log2, scale_log2);
       uint32_t pkp[32], pks[32];
 #pragma unroll
       for (int e = 0; e < 32; ++e) {
-        float pp[2], ds[2];
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int qcol = 2 * e + u;                // within this half
-          pp[u] = ex2(__uint_as_float(rs[2 * e + u]) * scale_log2 - bl[qcol]);
-          if (diag && hf * 64 + qcol < row) pp[u] = 0.f;   // a query before this key
-          ds[u] = pp[u] * (__uint_as_float(rp[2 * e + u]) - bd[qcol]);
+        const float2 nl = *reinterpret_cast<const float2 *>(bl + 2 * e);
+        const float2 nd = *reinterpret_cast<const float2 *>(bd + 2 * e);
+        float x0, x1;
+        unf2(fma2(f2(__uint_as_float(rs[2 * e]), __uint_as_float(rs[2 * e + 1])), sc2, f2(nl.x, nl.y)), x0, x1);
+        float p0 = ex2(x0), p1 = ex2(x1);
+        if (diag) {                                  // a query before this key
+          const int qcol = hf * 64 + 2 * e;
+          if (qcol < row) p0 = 0.f;
+          if (qcol + 1 < row) p1 = 0.f;
         }
-        pkp[e] = pack_f16x2(pp[0], pp[1]);
-        pks[e] = pack_f16x2(ds[0], ds[1]);
+        const uint64_t t2 = add2(f2(__uint_as_float(rp[2 * e]), __uint_as_float(rp[2 * e + 1])), f2(nd.x, nd.y));
+        float d0, d1;
+        unf2(mul2(f2(p0, p1), t2), d0, d1);
+        pkp[e] = pack_f16x2(p0, p1);
+        pks[e] = pack_f16x2(d0, d1);
       }
       // the previous item's dV / dK MMAs must have read P^T / dS^T before they are rewritten
       if (n > 0) ok = __all_sync(0xffffffffu, mbar_wait(&bars->pds_free, (n - 1) & 1, abort, status)) && ok;

@@ -41,46 +41,60 @@ struct S1Params {
   float turns_hi[32], turns_lo[32];  // RoPE frequencies in turns, as float pairs
 };
 
-// Row strides of the shared-memory tiles: a multiple of 32 floats plus 4, so that the mma
-// fragment reads (eight rows x four column pairs, or four row pairs x eight columns) fall on
-// distinct banks.
+// Row strides of the float32 shared-memory tiles: a multiple of 32 floats plus 4, so that
+// fragment-pattern reads (eight rows x four column pairs) fall on distinct banks.
 __host__ __device__ constexpr int s1_pad(int w) { return (w + 31) / 32 * 32 + 4; }
+// Row stride (bf16 elements) of the bf16 planes: a multiple of 128 bytes plus 16, so that the
+// eight 16-byte rows of an ldmatrix phase hit distinct bank groups.
+__host__ __device__ constexpr int s1_plane_ld(int w) { return ((w * 2 + 127) / 128 * 128 + 16) / 2; }
 
-// smem (floats): Ps [2][(TT + KC-1) x CHP] (P rows with the conv halo, double-buffered) |
-// Dq [2][TT x QKP] (dq of the G heads and dk) | Dv [2][(TT + 1) x DL] | A [TT x QKP] (sequence-
-// conv output) | U [TT x QKP] (channel-conv output, then its gradient in place) |
-// Rt [TT x DL] (cos, sin of the tile's RoPE angles) | turns [2 x 32]
-__host__ __device__ inline size_t s1_smem_floats(int G, int DL, int KC) {
+// smem: Ps [2][(TT + KC-1) x CHP] f32 (P rows with the conv halo, double-buffered) | Dq [2][TT x
+// QKP] f32 (dq of the G heads and dk) | Dv [2][(TT + 1) x DL] f32 | U [TT x QKP] f32 (channel-
+// conv output, then its gradient in place) | Rt [TT x DL] f32 (cos, sin of the tile's RoPE
+// angles) | turns [64] f32 | planes [4][TT x PLD] bf16: the sequence-conv output A and the
+// gradient dU, each as a bf16 leading term and remainder (about 16 significand bits in all)
+__host__ __device__ inline size_t s1_smem_bytes(int G, int DL, int KC) {
   const size_t QKP = s1_pad((G + 1) * DL), CHP = s1_pad((G + 2) * DL);
-  return 2 * static_cast<size_t>(S1_TT + KC - 1) * CHP + 2 * S1_TT * QKP +
-         2 * static_cast<size_t>(S1_TT + 1) * DL + 2 * S1_TT * QKP + S1_TT * DL + 64;
+  const size_t floats = 2 * static_cast<size_t>(S1_TT + KC - 1) * CHP + 2 * S1_TT * QKP +
+                        2 * static_cast<size_t>(S1_TT + 1) * DL + S1_TT * QKP + S1_TT * DL + 64;
+  return floats * 4 + 4 * static_cast<size_t>(S1_TT) * s1_plane_ld((G + 1) * DL) * 2;
+}
+
+__device__ __forceinline__ void split_store(__nv_bfloat16 *hi, __nv_bfloat16 *lo, float v) {
+  const __nv_bfloat16 h = __float2bfloat16_rn(v);
+  *hi = h;
+  *lo = __float2bfloat16_rn(v - __bfloat162float(h));
 }
 
 // Pass 1, persistent: CTA (ci, g) walks the 16-token tiles u_beg .. u_end-1 of key/value group
 // g, the next tile's P rows, dq / dk and dv copied in (16-byte asynchronous copies) while the
 // current one is computed.  The three channel-conv products are warp mma.sync tiles on bf16
-// hi / lo splits (three products each: hi*hi + hi*lo + lo*hi, about fp32 accuracy):
+// hi / lo splits (three products each: hi*hi + hi*lo + lo*hi, about fp32 accuracy), their
+// activation fragments read from the split planes by ldmatrix:
 //   U  = A W^T per head (tokens x out channels), then Q-K-Mean's skip terms
 //   dA = dU W  per head (tokens x in channels)
-//   dW += dU^T A per head (out x in channels, the tile's tokens as K), accumulated in
-//         registers over the CTA's tiles and added to the output once.
+//   dW += dU^T A per head (out x in channels, the tile's tokens as K, both operands through
+//         ldmatrix.trans), accumulated in registers over the CTA's tiles, added once.
 template <int DL>
 __global__ void __launch_bounds__(S1_THREADS, 1) stencil_bwd1_kernel(const S1Params p, int cpg,
                                                                      int tiles_per_seq) {
   extern __shared__ __align__(16) float sm[];
   constexpr int TT = S1_TT, HALF = DL / 2, NTI = DL / 8, KST = DL / 16, MT = DL / 16;
+  constexpr int D4 = DL / 4;
   const int G = p.G, KC = p.KC, KC1 = KC - 1, S = p.S;
   const int QK = (G + 1) * DL, CH = (G + 2) * DL;
-  const int QKP = s1_pad(QK), CHP = s1_pad(CH), PR = TT + KC1;
+  const int QKP = s1_pad(QK), CHP = s1_pad(CH), PR = TT + KC1, PLD = s1_plane_ld(QK);
   float *Ps = sm;
   float *Dq = Ps + 2 * PR * CHP;
   float *Dv = Dq + 2 * TT * QKP;
-  float *A = Dv + 2 * (TT + 1) * DL;
-  float *U = A + TT * QKP;
+  float *U = Dv + 2 * (TT + 1) * DL;
   float *Rt = U + TT * QKP;
   float2 *turns = reinterpret_cast<float2 *>(Rt + TT * DL);
+  __nv_bfloat16 *Ahi = reinterpret_cast<__nv_bfloat16 *>(Rt + TT * DL + 64);
+  __nv_bfloat16 *Alo = Ahi + TT * PLD, *Dhi = Alo + TT * PLD, *Dlo = Dhi + TT * PLD;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int gr = lane >> 2, qc = lane & 3;
+  const int lr = lane & 7, lm = lane >> 3;          // ldmatrix: row of matrix lm
   const int g = blockIdx.y, ci = blockIdx.x;
   const int units = p.B * tiles_per_seq;
   const int u_beg = static_cast<int>(static_cast<long long>(units) * ci / cpg);
@@ -91,33 +105,35 @@ __global__ void __launch_bounds__(S1_THREADS, 1) stencil_bwd1_kernel(const S1Par
   auto head_glob = [&](int hh) { return hh < G ? g * G + hh : p.H + g; };
   if (tid < 32) turns[tid] = make_float2(p.turns_hi[tid], p.turns_lo[tid]);
 
+  // copy assignments fixed per thread: P rows by C4 16-byte pieces, dq / dk rows by D4
+  const int C4 = CH / 4;                            // <= 256 (host check)
+  const int p_rows_pass = S1_THREADS / C4, p_r0 = tid / C4, p_c = (tid % C4) * 4;
+  const int p_gc = p_c < G * DL ? qcol0 + p_c : (p_c < QK ? kcol0 + (p_c - G * DL) : vcol0 + (p_c - QK));
+  constexpr int q_rows_pass = S1_THREADS / D4;
+  const int q_r0 = tid / D4, q_i = (tid % D4) * 4;
   auto issue = [&](int u, int k) {                  // tile u's inputs into buffer k
     const int b = u / tiles_per_seq, t0 = (u % tiles_per_seq) * TT;
     float *ps = Ps + k * PR * CHP, *dqs = Dq + k * TT * QKP, *dvs = Dv + k * (TT + 1) * DL;
-    const int C4 = CH / 4;
-    for (int e = tid; e < PR * C4; e += S1_THREADS) {
-      const int r = e / C4, c = (e % C4) * 4;
-      const int t = t0 - KC1 + r;
-      const int gc = c < G * DL ? qcol0 + c : (c < QK ? kcol0 + (c - G * DL) : vcol0 + (c - QK));
-      const bool ok = t >= 0 && t < S;
-      cp_async16_zfill(ps + r * CHP + c, p.P + (static_cast<size_t>(b) * S + (ok ? t : 0)) * p.NQKV + gc, ok);
-    }
-    constexpr int D4 = DL / 4;
-    for (int e = tid; e < TT * (G + 1) * D4; e += S1_THREADS) {
-      const int tt = e / ((G + 1) * D4), rem = e % ((G + 1) * D4), hh = rem / D4, i = (rem % D4) * 4;
+    if (p_r0 < p_rows_pass)
+      for (int r = p_r0; r < PR; r += p_rows_pass) {
+        const int t = t0 - KC1 + r;
+        const bool ok = t >= 0 && t < S;
+        cp_async16_zfill(ps + r * CHP + p_c, p.P + (static_cast<size_t>(b) * S + (ok ? t : 0)) * p.NQKV + p_gc, ok);
+      }
+    for (int r = q_r0; r < TT * (G + 1); r += q_rows_pass) {   // (token, head) rows
+      const int tt = r / (G + 1), hh = r % (G + 1);
       const int t = t0 + tt;
       const bool ok = t < S;
       const size_t tr = ok ? t : 0;
-      const float *src = hh < G ? p.dq + ((static_cast<size_t>(b) * p.H + g * G + hh) * S + tr) * DL + i
-                                : p.dk + ((static_cast<size_t>(b) * p.Hkv + g) * S + tr) * DL + i;
-      cp_async16_zfill(dqs + tt * QKP + hh * DL + i, src, ok);
+      const float *src = hh < G ? p.dq + ((static_cast<size_t>(b) * p.H + g * G + hh) * S + tr) * DL + q_i
+                                : p.dk + ((static_cast<size_t>(b) * p.Hkv + g) * S + tr) * DL + q_i;
+      cp_async16_zfill(dqs + tt * QKP + hh * DL + q_i, src, ok);
     }
-    for (int e = tid; e < (TT + 1) * D4; e += S1_THREADS) {
-      const int tt = e / D4, i = (e % D4) * 4;
-      const int t = t0 + tt;
+    for (int r = q_r0; r < TT + 1; r += q_rows_pass) {
+      const int t = t0 + r;
       const bool ok = t < S;
-      cp_async16_zfill(dvs + tt * DL + i,
-                       p.dv + ((static_cast<size_t>(b) * p.Hkv + g) * S + (ok ? t : 0)) * DL + i, ok);
+      cp_async16_zfill(dvs + r * DL + q_i,
+                       p.dv + ((static_cast<size_t>(b) * p.Hkv + g) * S + (ok ? t : 0)) * DL + q_i, ok);
     }
   };
 
@@ -127,6 +143,7 @@ __global__ void __launch_bounds__(S1_THREADS, 1) stencil_bwd1_kernel(const S1Par
   float accW[S1_MAXB][4];
 #pragma unroll
   for (int m = 0; m < S1_MAXB; ++m) accW[m][0] = accW[m][1] = accW[m][2] = accW[m][3] = 0.f;
+  const uint32_t ahi_s = smem_u32(Ahi), alo_s = smem_u32(Alo), dhi_s = smem_u32(Dhi), dlo_s = smem_u32(Dlo);
 
   if (u_beg < u_end) issue(u_beg, 0);
   cp_async_commit();
@@ -140,7 +157,7 @@ __global__ void __launch_bounds__(S1_THREADS, 1) stencil_bwd1_kernel(const S1Par
     const float *ps = Ps + k * PR * CHP, *dqs = Dq + k * TT * QKP, *dvs = Dv + k * (TT + 1) * DL;
 
     // 1. sequence conv of the q | k channels (tap j of token t reads token t - (KC-1) + j),
-    //    and the tile's RoPE angles
+    //    stored as bf16 hi / lo planes, and the tile's RoPE angles
     for (int c = tid; c < QK; c += S1_THREADS) {
       const int gc = c < G * DL ? qcol0 + c : kcol0 + (c - G * DL);
       float w[S1_KCMAX];
@@ -152,7 +169,7 @@ __global__ void __launch_bounds__(S1_THREADS, 1) stencil_bwd1_kernel(const S1Par
 #pragma unroll
         for (int j = 0; j < S1_KCMAX; ++j)
           if (j < KC) a = fmaf(w[j], ps[(tt + j) * CHP + c], a);
-        A[tt * QKP + c] = a;
+        split_store(Ahi + tt * PLD + c, Alo + tt * PLD + c, a);
       }
     }
     if (rope)
@@ -166,21 +183,20 @@ __global__ void __launch_bounds__(S1_THREADS, 1) stencil_bwd1_kernel(const S1Par
       }
     __syncthreads();
 
-    // 2. U = A W^T per head (+ Q-K-Mean's skip terms); a warp per (head, 8 out channels)
+    // 2. U = A W^T per head (+ Q-K-Mean's skip terms); a warp per (head, 8 out channels).
+    //    A fragments: ldmatrix rows = tokens (lm & 1) * 8 + lr, columns k0 + (lm >> 1) * 8
+    const uint32_t frag_off = static_cast<uint32_t>((((lm & 1) * 8 + lr) * PLD + (lm >> 1) * 8) * 2);
     for (int task = warp; task < (G + 1) * NTI; task += S1_WARPS) {
       const int hh = task / NTI, nt = task % NTI;
       const uint2 *wb = p.wsplit + static_cast<size_t>(head_glob(hh)) * DL * (DL / 2);
       float acc[4] = {0.f, 0.f, 0.f, 0.f};
-      const float *a0p = A + gr * QKP + hh * DL, *a1p = a0p + 8 * QKP;
 #pragma unroll
       for (int ks = 0; ks < KST; ++ks) {
-        const int k0 = ks * 16 + 2 * qc;
+        const uint32_t off = frag_off + (hh * DL + ks * 16) * 2;
         uint32_t ah[4], al[4];
-        split_bf16x2(*reinterpret_cast<const float2 *>(a0p + k0), ah[0], al[0]);
-        split_bf16x2(*reinterpret_cast<const float2 *>(a1p + k0), ah[1], al[1]);
-        split_bf16x2(*reinterpret_cast<const float2 *>(a0p + k0 + 8), ah[2], al[2]);
-        split_bf16x2(*reinterpret_cast<const float2 *>(a1p + k0 + 8), ah[3], al[3]);
-        const uint2 *wr = wb + (nt * 8 + gr) * (DL / 2) + k0 / 2;
+        ldsm_x4(ahi_s + off, ah[0], ah[1], ah[2], ah[3]);
+        ldsm_x4(alo_s + off, al[0], al[1], al[2], al[3]);
+        const uint2 *wr = wb + (nt * 8 + gr) * (DL / 2) + (ks * 16 + 2 * qc) / 2;
         const uint2 w0 = __ldg(wr), w1 = __ldg(wr + 4);
         const uint32_t bh[2] = {w0.x, w1.x}, bl[2] = {w0.y, w1.y};
         mma_bf16_16816(acc, ah, bh);
@@ -209,14 +225,20 @@ __global__ void __launch_bounds__(S1_THREADS, 1) stencil_bwd1_kernel(const S1Par
     }
     __syncthreads();
 
-    // 3. per (token, head): norm statistics, dn = RoPE^-1(dq or dk), du (over U in place); a
-    //    warp per pair, lane i holding the RoPE pair (i, i + d~/2)
+    // 3. per (token, head): norm statistics, dn = RoPE^-1(dq or dk), du (over U in place, and
+    //    into the dU planes); a warp per pair, lane i holding the RoPE pair (i, i + d~/2)
     for (int it = warp; it < TT * (G + 1); it += S1_WARPS) {
       const int tt = it / (G + 1), hh = it % (G + 1);
       float *uu = U + tt * QKP + hh * DL;
       const bool act = lane < HALF;
+      const int pc = tt * PLD + hh * DL + lane;
       if (t0 + tt >= S) {                            // past the sequence: no gradient
-        if (act) { uu[lane] = 0.f; uu[lane + HALF] = 0.f; }
+        if (act) {
+          uu[lane] = 0.f;
+          uu[lane + HALF] = 0.f;
+          split_store(Dhi + pc, Dlo + pc, 0.f);
+          split_store(Dhi + pc + HALF, Dlo + pc + HALF, 0.f);
+        }
         continue;
       }
       const float *ds = dqs + tt * QKP + hh * DL;
@@ -249,6 +271,8 @@ __global__ void __launch_bounds__(S1_THREADS, 1) stencil_bwd1_kernel(const S1Par
       if (act) {
         uu[lane] = d1;
         uu[lane + HALF] = d2;
+        split_store(Dhi + pc, Dlo + pc, d1);
+        split_store(Dhi + pc + HALF, Dlo + pc + HALF, d2);
       }
     }
     __syncthreads();
@@ -258,16 +282,13 @@ __global__ void __launch_bounds__(S1_THREADS, 1) stencil_bwd1_kernel(const S1Par
       const int hh = task / NTI, nt = task % NTI;
       const uint2 *wt = p.wsplitT + static_cast<size_t>(head_glob(hh)) * DL * (DL / 2);
       float acc[4] = {0.f, 0.f, 0.f, 0.f};
-      const float *a0p = U + gr * QKP + hh * DL, *a1p = a0p + 8 * QKP;
 #pragma unroll
       for (int ks = 0; ks < KST; ++ks) {
-        const int k0 = ks * 16 + 2 * qc;
+        const uint32_t off = frag_off + (hh * DL + ks * 16) * 2;
         uint32_t ah[4], al[4];
-        split_bf16x2(*reinterpret_cast<const float2 *>(a0p + k0), ah[0], al[0]);
-        split_bf16x2(*reinterpret_cast<const float2 *>(a1p + k0), ah[1], al[1]);
-        split_bf16x2(*reinterpret_cast<const float2 *>(a0p + k0 + 8), ah[2], al[2]);
-        split_bf16x2(*reinterpret_cast<const float2 *>(a1p + k0 + 8), ah[3], al[3]);
-        const uint2 *wr = wt + (nt * 8 + gr) * (DL / 2) + k0 / 2;
+        ldsm_x4(dhi_s + off, ah[0], ah[1], ah[2], ah[3]);
+        ldsm_x4(dlo_s + off, al[0], al[1], al[2], al[3]);
+        const uint2 *wr = wt + (nt * 8 + gr) * (DL / 2) + (ks * 16 + 2 * qc) / 2;
         const uint2 w0 = __ldg(wr), w1 = __ldg(wr + 4);
         const uint32_t bh[2] = {w0.x, w1.x}, bl[2] = {w0.y, w1.y};
         mma_bf16_16816(acc, ah, bh);
@@ -286,53 +307,58 @@ __global__ void __launch_bounds__(S1_THREADS, 1) stencil_bwd1_kernel(const S1Par
     }
     // Q-K-Mean's skip gradients of the q | k projections, and the value gradients (the
     // value-shift undone: a shifted channel of token t received dv of token t + 1)
-    for (int e = tid; e < TT * CH; e += S1_THREADS) {
-      const int tt = e / CH, c = e % CH;
-      const int t = t0 + tt;
-      if (t >= S) continue;
-      const size_t row = static_cast<size_t>(b) * S + t;
-      if (c < QK) {
-        float skip = 0.f;
-        if (qkm) {
-          const int i = c % DL;
-          const float duk = U[tt * QKP + G * DL + i];
-          if (c < G * DL) {
-            skip = 0.5f * U[tt * QKP + c] + duk / (2.0f * static_cast<float>(G));
-          } else {
-            float sq = 0.f;
-            for (int h2 = 0; h2 < G; ++h2) sq += U[tt * QKP + h2 * DL + i];
-            skip = 0.5f * sq + 0.5f * duk;
+    for (int c = tid; c < CH; c += S1_THREADS) {
+      const bool is_qk = c < QK;
+      const int i = is_qk ? c % DL : c - QK;
+      const int gc = c < G * DL ? qcol0 + c : (is_qk ? kcol0 + (c - G * DL) : vcol0 + i);
+      const int vsh = (!is_qk && (p.flags & F_VALUE_SHIFT) && g * DL + i >= p.VS0) ? 1 : 0;
+      for (int tt = 0; tt < TT; ++tt) {
+        const int t = t0 + tt;
+        if (t >= S) break;
+        float val;
+        if (is_qk) {
+          val = 0.f;
+          if (qkm) {
+            const float *ur = U + tt * QKP;
+            const float duk = ur[G * DL + i];
+            if (c < G * DL) {
+              val = 0.5f * ur[c] + duk / (2.0f * static_cast<float>(G));
+            } else {
+              float sq = 0.f;
+              for (int h2 = 0; h2 < G; ++h2) sq += ur[h2 * DL + i];
+              val = 0.5f * sq + 0.5f * duk;
+            }
           }
+        } else {
+          val = dvs[(tt + vsh) * DL + i];
         }
-        const int gc = c < G * DL ? qcol0 + c : kcol0 + (c - G * DL);
-        p.dPpart[row * p.NQKV + gc] = skip;
-      } else {
-        const int i = c - QK;
-        const bool shifted = (p.flags & F_VALUE_SHIFT) && g * DL + i >= p.VS0;
-        p.dPpart[row * p.NQKV + vcol0 + i] = dvs[(tt + (shifted ? 1 : 0)) * DL + i];
+        p.dPpart[(static_cast<size_t>(b) * S + t) * p.NQKV + gc] = val;
       }
     }
-    // 5. dW[h][i][c] += sum over the tile's tokens of dU[t][h][i] A[t][h][c]
+    // 5. dW[h][i][c] += sum over the tile's tokens of dU[t][h][i] A[t][h][c].  A operand dU^T
+    //    (16 out channels x 16 tokens): ldmatrix.trans of the dU plane, matrix lm at tokens
+    //    (lm >> 1) * 8 + lr, channels (lm & 1) * 8; B operand (16 tokens x 8 in channels):
+    //    ldmatrix.trans of the A plane, matrix (lm & 1) at tokens (lm & 1) * 8 + lr
+    const uint32_t ta_off = static_cast<uint32_t>((((lm >> 1) * 8 + lr) * PLD + (lm & 1) * 8) * 2);
+    const uint32_t tb_off = static_cast<uint32_t>((((lm & 1) * 8 + lr) * PLD) * 2);
 #pragma unroll
     for (int m = 0; m < S1_MAXB; ++m) {
       const int blk = warp * BPW + m;
       if (m < BPW && blk < NB) {
         const int hh = blk / (MT * NTI), rem = blk % (MT * NTI);
-        const int cu = hh * DL + (rem / NTI) * 16 + gr;   // dU column (out channel i)
-        const int ca = hh * DL + (rem % NTI) * 8 + gr;    // A column (in channel c)
+        const int cu = hh * DL + (rem / NTI) * 16;   // first out channel of the block
+        const int ca = hh * DL + (rem % NTI) * 8;    // first in channel
         uint32_t ah[4], al[4], bh[2], bl[2];
-        split_bf16x2(make_float2(U[(2 * qc) * QKP + cu], U[(2 * qc + 1) * QKP + cu]), ah[0], al[0]);
-        split_bf16x2(make_float2(U[(2 * qc) * QKP + cu + 8], U[(2 * qc + 1) * QKP + cu + 8]), ah[1], al[1]);
-        split_bf16x2(make_float2(U[(2 * qc + 8) * QKP + cu], U[(2 * qc + 9) * QKP + cu]), ah[2], al[2]);
-        split_bf16x2(make_float2(U[(2 * qc + 8) * QKP + cu + 8], U[(2 * qc + 9) * QKP + cu + 8]), ah[3], al[3]);
-        split_bf16x2(make_float2(A[(2 * qc) * QKP + ca], A[(2 * qc + 1) * QKP + ca]), bh[0], bl[0]);
-        split_bf16x2(make_float2(A[(2 * qc + 8) * QKP + ca], A[(2 * qc + 9) * QKP + ca]), bh[1], bl[1]);
+        ldsm_x4_t(dhi_s + ta_off + cu * 2, ah[0], ah[1], ah[2], ah[3]);
+        ldsm_x4_t(dlo_s + ta_off + cu * 2, al[0], al[1], al[2], al[3]);
+        ldsm_x2_t(ahi_s + tb_off + ca * 2, bh[0], bh[1]);
+        ldsm_x2_t(alo_s + tb_off + ca * 2, bl[0], bl[1]);
         mma_bf16_16816(accW[m], ah, bh);
         mma_bf16_16816(accW[m], ah, bl);
         mma_bf16_16816(accW[m], al, bh);
       }
     }
-    __syncthreads();                                 // A, U and this buffer reused next
+    __syncthreads();                                 // planes, U and this buffer reused next
   }
   cp_async_wait_none();
 #pragma unroll
@@ -369,15 +395,16 @@ __global__ void split_conv_chan_t_kernel(const float *__restrict__ w, uint2 *__r
 }
 
 // Pass 2: a CTA per (32 columns of dP, 256 rows), a warp per 32-row slice of them (so every
-// load and store of a warp covers 32 consecutive columns of one row); the sequence conv's
-// transpose and its filter gradient from sliding windows of dA (rows t .. t+KC-1) and P (rows
-// t-KC+1 .. t) held in registers, then dP in bfloat16 (the value columns converted as they
-// are).  The filter gradient is summed over the CTA's warps in shared memory and added once
-// per CTA.
+// load and store of a warp covers 32 consecutive columns of one row), walked in chunks of 8
+// rows whose loads (dPpart, the P rows back to KC-1 before the chunk, the dA rows up to KC-1
+// after it) are all issued before any is used; the sequence conv's transpose and its filter
+// gradient, then dP in bfloat16 (the value columns converted as they are).  The filter
+// gradient is summed over the CTA's warps in shared memory and added once per CTA.
 constexpr int S2_COLS = 32;
 constexpr int S2_SUB = 32;                           // rows per warp
 constexpr int S2_WARPS = 8;
 constexpr int S2_KCMAX = 8;
+constexpr int S2_CH = 8;                             // rows per chunk
 
 __global__ void __launch_bounds__(256) stencil_bwd2_kernel(
     const float *__restrict__ P, const float *__restrict__ dA, const float *__restrict__ dPpart,
@@ -388,73 +415,60 @@ __global__ void __launch_bounds__(256) stencil_bwd2_kernel(
   const int c = blockIdx.x * S2_COLS + lane;             // column of dP (all NQKV)
   const long long M = static_cast<long long>(B) * S;
   const long long r_beg = (static_cast<long long>(blockIdx.y) * S2_WARPS + warp) * S2_SUB;
-  const long long r_end = r_beg + S2_SUB < M ? r_beg + S2_SUB : M;
   const int W = NQ + NKV;
   const bool live = c < NQKV;
   const bool qk = live && c < W;
-  float w[S2_KCMAX], dw[S2_KCMAX];
+  const int KC1 = KC - 1;
+  // per lag (tap j = KC-1 - lag): wl[lag] = w[c][j], dwl[lag] accumulates the gradient of w[c][j]
+  float wl[S2_KCMAX], dwl[S2_KCMAX];
 #pragma unroll
-  for (int j = 0; j < S2_KCMAX; ++j) {
-    w[j] = (qk && j < KC) ? conv_seq[static_cast<size_t>(c) * KC + j] : 0.f;
-    dw[j] = 0.f;
+  for (int l = 0; l < S2_KCMAX; ++l) {
+    wl[l] = (qk && l < KC) ? conv_seq[static_cast<size_t>(c) * KC + (KC1 - l)] : 0.f;
+    dwl[l] = 0.f;
   }
-  if (qk) {
-    // windows: da[l] = dA[row + l] (l < KC, zero past the sequence), pp[l] = P[row - l]
-    // (zero before the sequence start), for the current row
-    float da[S2_KCMAX], pp[S2_KCMAX];
-    if (r_beg < r_end) {
-      const int t0 = static_cast<int>(r_beg % S);
+  constexpr int NW = S2_CH + S2_KCMAX - 1;
+  for (int ch = 0; ch < S2_SUB / S2_CH; ++ch) {
+    const long long r0 = r_beg + ch * S2_CH;
+    if (r0 >= M || !live) break;
+    // da[m] = dA[r0 + m], pq[m] = P[r0 + m - (KCMAX-1)] (zero outside [0, M) and outside the
+    // halo this chunk needs); the sequence boundaries are applied per use below
+    float da[NW], pq[NW], dpp[S2_CH];
 #pragma unroll
-      for (int l = 0; l < S2_KCMAX; ++l) {
-        da[l] = (l < KC && t0 + l < S) ? dA[(r_beg + l) * W + c] : 0.f;
-        pp[l] = (l < KC && t0 - l >= 0) ? P[(r_beg - l) * NQKV + c] : 0.f;
+    for (int e = 0; e < S2_CH; ++e) dpp[e] = r0 + e < M ? dPpart[(r0 + e) * NQKV + c] : 0.f;
+    if (qk) {
+#pragma unroll
+      for (int m = 0; m < NW; ++m) {
+        const long long rd = r0 + m, rp = r0 + m - (S2_KCMAX - 1);
+        da[m] = (m < S2_CH + KC1 && rd < M) ? dA[rd * W + c] : 0.f;
+        pq[m] = (m >= S2_KCMAX - KC && rp >= 0 && rp < M) ? P[rp * NQKV + c] : 0.f;
       }
     }
-    for (long long row = r_beg; row < r_end; ++row) {
-      const int t = static_cast<int>(row % S);
-      float v = dPpart[row * NQKV + c];
 #pragma unroll
-      for (int j = 0; j < S2_KCMAX; ++j) {
-        if (j < KC) {
-          const int lag = KC - 1 - j;                    // output t + lag read input t by tap j
-          v = fmaf(w[j], da[lag], v);                    // da[lag] is zero past the sequence
-          dw[j] = fmaf(da[0], pp[lag], dw[j]);           // pp[lag] is zero before its start
+    for (int e = 0; e < S2_CH; ++e) {
+      const long long row = r0 + e;
+      if (row >= M) break;
+      float v = dpp[e];
+      if (qk) {
+        const int t = static_cast<int>(row % S);
+#pragma unroll
+        for (int l = 0; l < S2_KCMAX; ++l) {
+          if (l < KC) {                                  // output t + l read input t by tap KC-1-l
+            if (t + l < S) v = fmaf(wl[l], da[e + l], v);
+            if (t - l >= 0) dwl[l] = fmaf(da[e], pq[e + S2_KCMAX - 1 - l], dwl[l]);
+          }
         }
       }
       dP[row * NQKV + c] = __float2bfloat16_rn(v);
-      // slide both windows by one row
-#pragma unroll
-      for (int l = S2_KCMAX - 1; l > 0; --l) pp[l] = pp[l - 1];
-#pragma unroll
-      for (int l = 0; l + 1 < S2_KCMAX; ++l) da[l] = da[l + 1];
-      const long long nrow = row + 1;
-      if (nrow < r_end) {
-        const int nt = t + 1 == S ? 0 : t + 1;           // a new sequence starts at nt == 0
-        pp[0] = P[nrow * NQKV + c];
-        if (nt == 0) {
-#pragma unroll
-          for (int l = 1; l < S2_KCMAX; ++l) pp[l] = 0.f;
-#pragma unroll
-          for (int l = 0; l < S2_KCMAX; ++l)
-            da[l] = (l < KC && l < S) ? dA[(nrow + l) * W + c] : 0.f;
-        } else {
-          const int l = KC - 1;                          // the window's new last row
-          if (l < S2_KCMAX) da[l] = nt + l < S ? dA[(nrow + l) * W + c] : 0.f;
-        }
-      }
     }
-  } else if (live) {
-    for (long long row = r_beg; row < r_end; ++row)
-      dP[row * NQKV + c] = __float2bfloat16_rn(dPpart[row * NQKV + c]);
   }
 #pragma unroll
-  for (int j = 0; j < S2_KCMAX; ++j) red[warp][j][lane] = dw[j];
+  for (int l = 0; l < S2_KCMAX; ++l) red[warp][l][lane] = dwl[l];
   __syncthreads();
   if (warp == 0 && qk) {
     for (int j = 0; j < KC; ++j) {
       float sum = 0.f;
 #pragma unroll
-      for (int w2 = 0; w2 < S2_WARPS; ++w2) sum += red[w2][j][lane];
+      for (int w2 = 0; w2 < S2_WARPS; ++w2) sum += red[w2][KC1 - j][lane];
       atomicAdd(dconv_seq + static_cast<size_t>(c) * KC + j, sum);
     }
   }
@@ -494,12 +508,12 @@ __global__ void __launch_bounds__(256) transpose16_kernel(const uint16_t *__rest
 bool stencil_backward_supported(const Dims &d) {
   return d.bf16 && !(d.flags & F_NO_CONV) && (d.DL == 16 || d.DL == 32 || d.DL == 64) &&
          d.KC <= S1_KCMAX && (d.G + 1) * (d.DL / 16) * (d.DL / 8) <= S1_WARPS * S1_MAXB &&
-         s1_smem_floats(d.G, d.DL, d.KC) * 4 <= 200 * 1024;
+         (d.G + 2) * d.DL / 4 <= S1_THREADS && s1_smem_bytes(d.G, d.DL, d.KC) <= 200 * 1024;
 }
 
 template <int DL>
 cudaError_t launch_bwd1(const Dims &d, const S1Params &p, int cpg, int tiles, cudaStream_t st) {
-  const size_t smem = s1_smem_floats(d.G, DL, d.KC) * 4;
+  const size_t smem = s1_smem_bytes(d.G, DL, d.KC);
   cudaError_t e;
   if ((e = ensure_dyn_smem<stencil_bwd1_kernel<DL>>(smem)) != cudaSuccess) return e;
   stencil_bwd1_kernel<DL><<<dim3(cpg, d.Hkv), S1_THREADS, smem, st>>>(p, cpg, tiles);
