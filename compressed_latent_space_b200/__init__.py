@@ -80,6 +80,7 @@ _SIGS = {
     "cca_decode_step_static": (c_int, [POINTER(cca_config_t), POINTER(cca_weights_t), c_void_p,
                                        c_void_p, POINTER(cca_cache_t), c_void_p]),
     "cca_stage_wait_probe": (c_int, [ctypes.c_longlong, c_int, c_void_p, c_void_p]),
+    "cca_stage_exp2_poly": (c_int, [c_void_p, c_void_p, c_int, c_void_p]),
     "cca_backward_workspace_size": (c_size_t, [POINTER(cca_config_t), c_int, c_int]),
     "cca_backward": (c_int, [POINTER(cca_config_t), POINTER(cca_weights_t), c_void_p, c_void_p,
                              c_int, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
@@ -232,6 +233,11 @@ def cca_stage_attention(cfg, q, k, v, batch, seq, kv_stride, o, status=None, str
 
 def cca_workspace_status(workspace, stream=None):
     _check(load().cca_workspace_status(_ptr(workspace), _stream(stream)))
+
+
+def cca_stage_exp2_poly(x, y, stream=None):
+    """y = 2^x (float32 device tensors of one even length) by the attention's FMA-pipe cubic."""
+    _check(load().cca_stage_exp2_poly(_ptr(x), _ptr(y), int(x.numel()), _stream(stream)))
 
 
 def cca_stage_wait_probe(limit_ns: int, arm: bool, status, stream=None):

@@ -311,8 +311,10 @@ __global__ void __launch_bounds__(AttnCfg<DL>::THREADS, 1)
           tmem_st16(tO + c * 16, o);
         }
       }
-      // p = 2^(s * scale - m_ref): pairs scaled with one packed FMA, one MUFU ex2 each,
-      // rounded to float16 pairs (written over this tile's scores), four paired partial sums.
+      // p = 2^(s * scale - m_ref): pairs scaled with one packed FMA, one MUFU ex2 each (at
+      // d~ <= 64, where the exponential unit is the kernel's busiest pipe, three pairs in
+      // sixteen by a cubic on the FMA pipes instead), rounded to float16 pairs (written over
+      // this tile's scores), four paired partial sums.
       const uint64_t nm2 = f2(-m_ref, -m_ref);
       uint64_t l2[4];
 #pragma unroll
@@ -324,9 +326,15 @@ __global__ void __launch_bounds__(AttnCfg<DL>::THREADS, 1)
         for (int e = 0; e < 16; ++e) {
           const int i = c * 32 + 2 * e;
           const uint64_t x2 = fma2(f2(__uint_as_float(r[i]), __uint_as_float(r[i + 1])), sc2, nm2);
-          float x0, x1;
-          unf2(x2, x0, x1);
-          const float p0 = ex2(x0), p1 = ex2(x1);
+          float p0, p1;
+          if (DL < 128 && e % 5 == 4) {               // pairs 4, 9, 14 of 16: FMA pipes
+            ex2_poly2(x2, p0, p1);
+          } else {
+            float x0, x1;
+            unf2(x2, x0, x1);
+            p0 = ex2(x0);
+            p1 = ex2(x1);
+          }
           l2[e & 3] = add2(l2[e & 3], f2(p0, p1));
           pk[e] = pack_f16x2(p0, p1);
         }

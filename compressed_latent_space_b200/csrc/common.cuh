@@ -486,6 +486,29 @@ __device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
   return d;
 }
 
+// 2^x for a pair of floats on the FMA pipes instead of the MUFU unit: x = n + f with n the
+// nearest integer (added to and taken back from 1.5 * 2^23, which leaves n in the low bits of
+// the sum) and f in [-1/2, 1/2]; 2^f by the degree-3 minimax polynomial under relative error
+// (Remez exchange; coefficients from exp2_poly_coeffs.py, levelled relative error 7.5e-5, below
+// float16's 2^-11 rounding of the probabilities); 2^n added to the result's exponent field.
+// Arguments below -125 are clamped there (2^-125 rounds to 0 in float16; the clamp also keeps
+// the result's exponent field normal).
+__device__ __forceinline__ void ex2_poly2(uint64_t x2, float &p0, float &p1) {
+  float x0, x1;
+  unf2(x2, x0, x1);
+  const uint64_t xc = f2(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+  const uint64_t j2 = add2(xc, f2(12582912.f, 12582912.f));
+  const uint64_t fr = fma2(add2(j2, f2(-12582912.f, -12582912.f)), f2(-1.f, -1.f), xc);
+  uint64_t p = fma2(f2(0.0551716685f, 0.0551716685f), fr, f2(0.242611125f, 0.242611125f));
+  p = fma2(p, fr, f2(0.693260968f, 0.693260968f));
+  p = fma2(p, fr, f2(0.999928057f, 0.999928057f));
+  float q0, q1, j0, j1;
+  unf2(p, q0, q1);
+  unf2(j2, j0, j1);
+  p0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(j0) << 23));
+  p1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(j1) << 23));
+}
+
 // ----------------------------------------------------------------------------- ldmatrix
 // Four (two) 8x8 16-bit matrices from shared memory, lanes 8i..8i+7 giving the row addresses
 // of matrix i; .trans delivers each matrix transposed.

@@ -1,4 +1,5 @@
-// Diagnostic of the kernels' failure detection: one CTA runs the same bounded mbarrier wait
+// Stage entry of the attention's FMA-pipe exponential (ex2_poly2), so that its error bound is
+// tested on the device, and the diagnostic of the kernels' failure detection: one CTA runs the same bounded mbarrier wait
 // the tcgen05 kernels use, on a barrier that nothing arrives on unless the caller asks for it,
 // with a limit the caller chooses.  It shows, on the device, that a wait which can never
 // complete gives up after its limit, records DEV_WAIT_TIMEOUT in the status word and lets the
@@ -25,8 +26,29 @@ __global__ void wait_probe_kernel(unsigned long long limit_ns, int arm, int *sta
   __syncthreads();
 }
 
+__global__ void exp2_poly_kernel(const float *__restrict__ x, float *__restrict__ y, int npairs) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < npairs; i += gridDim.x * blockDim.x) {
+    float p0, p1;
+    ex2_poly2(f2(x[2 * i], x[2 * i + 1]), p0, p1);
+    y[2 * i] = p0;
+    y[2 * i + 1] = p1;
+  }
+}
+
 }  // namespace
 }  // namespace cca
+
+extern "C" CCA_API int cca_stage_exp2_poly(const float *x, float *y, int n, void *stream) {
+  if (n < 0 || (n & 1)) return cca::set_last_error(CCA_ERR_INVALID_ARG, "n must be even and >= 0");
+  if (n > 0 && (!x || !y)) return cca::set_last_error(CCA_ERR_INVALID_ARG, "x or y is NULL");
+  if (n > 0) {
+    const int pairs = n / 2, blocks = (pairs + 255) / 256 < 1024 ? (pairs + 255) / 256 : 1024;
+    cca::exp2_poly_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, pairs);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cca::set_last_error(CCA_ERR_CUDA, cudaGetErrorString(e));
+  }
+  return cca::set_last_error(CCA_OK, "");
+}
 
 extern "C" CCA_API int cca_stage_wait_probe(long long limit_ns, int arm, int *status,
                                             void *stream) {

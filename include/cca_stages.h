@@ -49,6 +49,14 @@ CCA_API int cca_stage_attention(const cca_config_t *cfg, const void *q, const vo
  * of its kernels recorded an internal error. */
 CCA_API int cca_workspace_status(const void *workspace, void *stream);
 
+/* y[i] = 2^x[i] for i < n (n even; x, y caller-owned device float32 arrays, enqueued on
+ * `stream`) by the cubic on the FMA pipes that the latent attention uses for part of its
+ * softmax probabilities (gist.science/de explainer, 2. Methodik: Softmax(QK^T)V): x = n + f,
+ * f in [-1/2, 1/2], 2^f by the minimax cubic under relative error, 2^n into the exponent;
+ * relative error below 1e-4 for x in [-125, 126], arguments below -125 treated as -125.
+ * Errors: INVALID_ARG (odd or negative n, NULL pointers), CUDA (launch). */
+CCA_API int cca_stage_exp2_poly(const float *x, float *y, int n, void *stream);
+
 /* Failure-detection diagnostic (the paper has no counterpart).  Launches one CTA that runs
  * the bounded mbarrier wait of the tcgen05 kernels on a shared-memory barrier, with a limit of
  * limit_ns nanoseconds (1e3 .. 1e9) instead of the kernels' 2 s.  arm == 0: nothing ever

@@ -469,3 +469,30 @@ def test_prefill_fused_and_unfused_paths(cuda_lib, shape, monkeypatch):
         assert cache.lengths.tolist() == [w.seq] * w.batch
         outs.append(f64(y))
     assert bf16_err(outs[0], outs[1]) <= BF16_TOL
+
+
+# ------------------------------------------------------------------ FMA-pipe exponential
+def test_exp2_poly_stage(cuda_lib):
+    """The cubic exp2 the latent attention evaluates part of its probabilities with, on the
+    device: relative error below 1e-4 against float64 exp2 on [-125, 126]; arguments below
+    -125 give about 2^-125 (zero once rounded to float16); odd lengths are refused."""
+    cls = cuda_lib
+    g = torch.Generator("cpu").manual_seed(5)
+    x = torch.cat([torch.rand(1 << 20, generator=g, dtype=torch.float64) * 251 - 125,
+                   torch.arange(-125, 126.5, 0.5, dtype=torch.float64),
+                   torch.tensor([0.0, 1e-7, -1e-7, 0.4999999, -0.4999999])]).float()
+    x = x[: x.numel() // 2 * 2].contiguous()
+    xd = x.cuda()
+    yd = torch.empty_like(xd)
+    cls.cca_stage_exp2_poly(xd, yd)
+    torch.cuda.synchronize()
+    y = yd.cpu().double()
+    ref = torch.exp2(x.double())
+    assert float((y / ref - 1).abs().max()) < 1e-4
+    low = torch.tensor([-126.0, -500.0, float("-inf"), -125.0], device="cuda")
+    ylow = torch.empty_like(low)
+    cls.cca_stage_exp2_poly(low, ylow)
+    torch.cuda.synchronize()
+    assert bool((ylow > 0).all()) and float(ylow.max()) <= 2.0 ** -124.9
+    with pytest.raises(cls.CCAError):
+        cls.cca_stage_exp2_poly(low[:3], ylow[:3])
