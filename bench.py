@@ -382,8 +382,9 @@ def cpu_oracle_sample(w, seed=0, full=False):
 # capture of the current kernel (scaled by tokens from a smaller case of the same shape); a
 # workload without one reports null.
 ATTN_TRAFFIC = {
-    # 25.43 MB read on one 8192-token sequence (B=1) of the same shape, x 4 for 2 x 16384 tokens
-    "ccgqa_prefill_16k": 4 * 25.428992e6,
+    # 25.66 MB read, 0 written on one 8192-token sequence (B=1) of the same shape (the kernel
+    # with part of its exponentials on the FMA pipes), x 4 for 2 x 16384 tokens
+    "ccgqa_prefill_16k": 4 * 25.658112e6,
 }
 
 
