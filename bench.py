@@ -310,8 +310,9 @@ def bench_decode(cls, w, steps, warmup, seed, layers=DECODE_LAYERS):
     for layer, cache in stack:
         cls.cca_cache_check(cache.struct)
     nk = decode_launches(cls, stack[0][0], w.batch, max_seq)
-    names = (["qkv_projection", "stencil_append", "split_kv_attention", "merge", "out_projection"]
-             if nk == 5 else ["qkv_projection", "stencil_append", "attention", "out_projection"])
+    names = {5: ["qkv_projection", "stencil_append", "split_kv_attention", "merge", "out_projection"],
+             4: ["qkv_projection", "stencil_append", "attention", "out_projection"],
+             3: ["qkv_projection", "stencil_append_attention", "out_projection"]}[nk]
     return dict(ms=ms, stages={n: t / max(calls, 1) for n, t in zip(names, stage_ms)},
                 launches=nk * steps, layers=layers)
 

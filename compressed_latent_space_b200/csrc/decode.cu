@@ -601,14 +601,27 @@ template <int DL>
 __host__ __device__ constexpr size_t tc_smem_bytes() {
   return static_cast<size_t>(tc_slots<DL>()) * TC_SUB * DL * 4 + 4 * 8 * (DL + 2) * 4;
 }
-
+// With the stencil fused in: the new token's queries [8][DL], key and value [2][DL] (float16-
+// rounded) and the G heads' scores of the new key [8], after the combine area.
 template <int DL>
+__host__ __device__ constexpr size_t tc_fused_smem_bytes() {
+  return tc_smem_bytes<DL>() + (8 * DL + 2 * DL + 8) * 4;
+}
+
+// STENCIL: the decode stencil of the new token (D2) runs inside this kernel, one CTA per
+// (sequence, group) with the keys unsplit.  Its filters are staged before the grid-dependency
+// wait into the ring's last slot (free until the first loop iteration refills it); after the
+// wait the CTA starts streaming cache rows 0..L-1, computes the new token's queries (kept in
+// shared memory), key and value (appended to the cache as before, and kept), and the new key
+// enters the softmax as one more partial (m = its score, l = 1, o = its value) in the combine.
+template <int DL, bool STENCIL>
 __global__ void __launch_bounds__(128, 1) decode_attn_tc_kernel(
     const float *__restrict__ q_new, const __half *__restrict__ k_cache,
     const __half *__restrict__ v_cache, const int *__restrict__ lengths,
     float *__restrict__ part_o, float *__restrict__ part_ml, __nv_bfloat16 *__restrict__ o_hi,
     __nv_bfloat16 *__restrict__ o_lo, int H, int Hkv, int G, int max_seq, int chunk, int nchunk,
-    float scale_log2, const uint8_t *__restrict__ next_w, size_t next_w_bytes) {
+    float scale_log2, const uint8_t *__restrict__ next_w, size_t next_w_bytes,
+    const D2Params<__nv_bfloat16> p2) {
   constexpr int CPR = DL / 8;                        // 16-byte pieces (8 dims) per row
   constexpr int NSLOT = tc_slots<DL>();
   constexpr int NT = TC_SUB / 32;                    // 8-key n-tiles per warp step
@@ -631,14 +644,26 @@ __global__ void __launch_bounds__(128, 1) decode_attn_tc_kernel(
     for (size_t i = id * per + tid; i < min(lines, (id + 1) * per); i += blockDim.x)
       prefetch_l2(next_w + i * 128);
   }
+  float *scratch = reinterpret_cast<float *>(ring + (NSLOT - 1) * SLOT);
+  float *qn = wst + 4 * 8 * (DL + 2);                // STENCIL: [8][DL] queries
+  float *kvn = qn + 8 * DL;                          // [2][DL] new key, value
+  float *sn = kvn + 2 * DL;                          // [8] scores of the new key
+  if constexpr (STENCIL) {
+    const D2Smem<DL> m(scratch, p2.G, p2.KC);
+    d2_stage(p2, g, b, m);
+    __syncthreads();                                 // staged filters visible to every thread
+  }
   pdl_wait();
   const int L = lengths[b];
   const int s0 = ch * chunk;
-  const int n = L < max_seq ? min(chunk, L + 1 - s0) : 0;
+  // keys streamed from the cache: with the stencil fused in, rows 0..L-1 (row L is the new key,
+  // written by this kernel and taken from shared memory)
+  const int n = L < max_seq ? (STENCIL ? L : min(chunk, L + 1 - s0)) : 0;
   float *po = part_o + ((static_cast<size_t>(b) * H + g * G) * nchunk + ch) * DL;
   float *pml = part_ml + ((static_cast<size_t>(b) * H + g * G) * nchunk + ch) * 2;
   const bool whole = nchunk == 1;                    // one split: write the merged o itself
-  if (n <= 0) {
+  if (STENCIL && L >= max_seq && tid == 0) report(p2.status, DEV_CACHE_FULL);
+  if (STENCIL ? L >= max_seq : n <= 0) {
     for (int i = tid; i < G * DL; i += blockDim.x) {
       if (whole) {
         o_hi[(static_cast<size_t>(b) * H + g * G) * DL + i] = __float2bfloat16_rn(0.f);
@@ -674,10 +699,31 @@ __global__ void __launch_bounds__(128, 1) decode_attn_tc_kernel(
 #pragma unroll
   for (int s = 0; s < NSLOT - 1; ++s) issue(s);
 
+  if constexpr (STENCIL) {
+    // the new token's stencil while the first sub-chunks are in flight
+    const D2Smem<DL> m(scratch, p2.G, p2.KC);
+    d2_load(p2, g, b, m);                            // each thread reads back only its own loads
+    d2_compute(p2, g, b, L, m, qn);
+    __syncthreads();                                 // q and the appended row L are visible
+    const size_t rowL = ((static_cast<size_t>(b) * Hkv + g) * max_seq + L) * DL;
+    for (int i = tid; i < 2 * DL; i += blockDim.x)   // read back through the writable pointers
+      kvn[i] = __half2float(i < DL ? p2.k_cache[rowL + i] : p2.v_cache[rowL + i - DL]);
+    __syncthreads();
+    // the new key's score per head, with q rounded to float16 as the MMA fragments below
+    for (int h = warp; h < G; h += 4) {
+      float acc = 0.f;
+      for (int i = lane; i < DL; i += 32)
+        acc = fmaf(__half2float(__float2half_rn(qn[h * DL + i])), kvn[i], acc);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if (lane == 0) sn[h] = acc * scale_log2;
+    }
+  }
+
   // Q fragments (rows = heads; a1, a3 are rows 8..15 and stay zero)
   uint32_t qa[DL / 16][2];
   {
-    const float *qh = q_new + (static_cast<size_t>(b) * H + g * G + gr) * DL;
+    const float *qh = STENCIL ? qn + gr * DL : q_new + (static_cast<size_t>(b) * H + g * G + gr) * DL;
 #pragma unroll
     for (int kk = 0; kk < DL / 16; ++kk) {
       float v0 = 0.f, v1 = 0.f, v2 = 0.f, v3 = 0.f;
@@ -794,7 +840,7 @@ __global__ void __launch_bounds__(128, 1) decode_attn_tc_kernel(
   __syncthreads();
   for (int i = tid; i < G * DL; i += blockDim.x) {
     const int h = i / DL, d = i % DL;
-    float mw[4], M = -INFINITY;
+    float mw[4], M = STENCIL ? sn[h] : -INFINITY;
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
       mw[w] = wst[(w * 8 + h) * WS + DL];
@@ -806,6 +852,11 @@ __global__ void __launch_bounds__(128, 1) decode_attn_tc_kernel(
       const float c = mw[w] == -INFINITY ? 0.f : exp2f(mw[w] - M);
       acc = fmaf(c, wst[(w * 8 + h) * WS + d], acc);
       lsum = fmaf(c, wst[(w * 8 + h) * WS + DL + 1], lsum);
+    }
+    if constexpr (STENCIL) {                         // the new key: one more partial, l = 1
+      const float c = exp2f(sn[h] - M);
+      acc = fmaf(c, kvn[DL + d], acc);
+      lsum += c;
     }
     if (whole) {
       const float v = acc / lsum;
@@ -917,11 +968,23 @@ int decode_chunk(const Dims &d, int max_seq) {
   return static_cast<int>((per + TC_SUB - 1) / TC_SUB * TC_SUB);
 }
 
+// 16-bit layers whose keys run unsplit and whose stencil scratch fits one slot of the
+// attention's copy ring run the stencil inside the attention kernel.
+static bool decode_fused(const Dims &d, int max_seq) {
+  const int chunk = decode_chunk(d, max_seq);
+  const int nchunk = (max_seq + chunk - 1) / chunk;
+  if (!d.bf16 || nchunk != 1 || d.DL > 32) return false;
+  const size_t slot_bytes = static_cast<size_t>(2) * TC_SUB * d.DL * 2;
+  return d2_smem_floats(d.G, d.DL, d.KC) * 4 <= slot_bytes;
+}
+
 // projection, stencil, attention, output projection, and the merge of the attention's key
-// splits (16-bit layers merge only when they split; float32 layers always run it)
+// splits (16-bit layers merge only when they split; float32 layers always run it); the
+// stencil shares the attention's kernel where decode_fused says so
 int decode_kernel_count(const Dims &d, int max_seq) {
   const int chunk = decode_chunk(d, max_seq);
   const int nchunk = (max_seq + chunk - 1) / chunk;
+  if (decode_fused(d, max_seq)) return 3;
   return d.bf16 && nchunk == 1 ? 4 : 5;
 }
 
@@ -956,20 +1019,30 @@ void decode_workspace_carve(const Dims &d, int max_seq, void *ws, DecodeArgs &a)
   a.chunk = chunk;
 }
 
+template <int DL, bool STENCIL>
+static cudaError_t launch_decode_tc(const Dims &d, const DecodeArgs &a, float scale_log2,
+                                    const D2Params<__nv_bfloat16> &p2, cudaStream_t st) {
+  const size_t smem = STENCIL ? tc_fused_smem_bytes<DL>() : tc_smem_bytes<DL>();
+  cudaError_t e = ensure_dyn_smem<decode_attn_tc_kernel<DL, STENCIL>>(smem);
+  if (e != cudaSuccess) return e;
+  __nv_bfloat16 *o_hi = static_cast<__nv_bfloat16 *>(a.o);
+  return launch_pdl(decode_attn_tc_kernel<DL, STENCIL>, dim3(a.nchunk, d.Hkv, d.B), dim3(128),
+                    smem, st, a.q_new, static_cast<const __half *>(a.k_cache),
+                    static_cast<const __half *>(a.v_cache), a.lengths, a.part_o, a.part_ml, o_hi,
+                    o_hi + static_cast<size_t>(d.B) * d.NQ, d.H, d.Hkv, d.G, a.max_seq, a.chunk,
+                    a.nchunk, scale_log2, static_cast<const uint8_t *>(a.w_o),
+                    static_cast<size_t>(d.E) * d.NQ * 2, p2);
+}
+
 template <int DL, typename TL>
 static cudaError_t launch_decode_attn(const Dims &d, const DecodeArgs &a, float scale_log2,
-                                      cudaStream_t st) {
+                                      const D2Params<__nv_bfloat16> *p2, cudaStream_t st) {
   if constexpr (sizeof(TL) == 2) {
-    const size_t smem = tc_smem_bytes<DL>();
-    cudaError_t e = ensure_dyn_smem<decode_attn_tc_kernel<DL>>(smem);
-    if (e != cudaSuccess) return e;
-    __nv_bfloat16 *o_hi = static_cast<__nv_bfloat16 *>(a.o);
-    return launch_pdl(decode_attn_tc_kernel<DL>, dim3(a.nchunk, d.Hkv, d.B), dim3(128), smem, st,
-                      a.q_new, static_cast<const __half *>(a.k_cache),
-                      static_cast<const __half *>(a.v_cache), a.lengths, a.part_o, a.part_ml,
-                      o_hi, o_hi + static_cast<size_t>(d.B) * d.NQ, d.H, d.Hkv, d.G, a.max_seq,
-                      a.chunk, a.nchunk, scale_log2, static_cast<const uint8_t *>(a.w_o),
-                      static_cast<size_t>(d.E) * d.NQ * sizeof(TL));
+    if (p2) {
+      if constexpr (DL <= 32) return launch_decode_tc<DL, true>(d, a, scale_log2, *p2, st);
+      return cudaErrorInvalidValue;
+    }
+    return launch_decode_tc<DL, false>(d, a, scale_log2, D2Params<__nv_bfloat16>{}, st);
   }
   const int KS = 128 / (DL / 2);
   const size_t smem = 4 * static_cast<size_t>(SUB) * DL * sizeof(TL) +
@@ -1020,22 +1093,27 @@ static cudaError_t decode_typed(const Dims &d, const DecodeArgs &a, cudaStream_t
   p2.eps = d.eps;
   for (int i = 0; i < d.DL / 2; ++i)
     p2.theta[i] = pow(static_cast<double>(d.rope_base), -2.0 * i / d.DL);
-  const size_t sm2 = d2_smem_floats(d.G, d.DL, d.KC) * 4;
-  auto d2 = d.DL == 16 ? decode_stencil_kernel<T, 16>
-                       : (d.DL == 32 ? decode_stencil_kernel<T, 32> : decode_stencil_kernel<T, 64>);
-  if (sm2 > 48 * 1024) {
-    e = d.DL == 16 ? ensure_dyn_smem<decode_stencil_kernel<T, 16>>(sm2)
-                   : (d.DL == 32 ? ensure_dyn_smem<decode_stencil_kernel<T, 32>>(sm2)
-                                 : ensure_dyn_smem<decode_stencil_kernel<T, 64>>(sm2));
-    if (e != cudaSuccess) return e;
+  const bool fused = decode_fused(d, a.max_seq);
+  if (!fused) {
+    const size_t sm2 = d2_smem_floats(d.G, d.DL, d.KC) * 4;
+    auto d2 = d.DL == 16 ? decode_stencil_kernel<T, 16>
+                         : (d.DL == 32 ? decode_stencil_kernel<T, 32> : decode_stencil_kernel<T, 64>);
+    if (sm2 > 48 * 1024) {
+      e = d.DL == 16 ? ensure_dyn_smem<decode_stencil_kernel<T, 16>>(sm2)
+                     : (d.DL == 32 ? ensure_dyn_smem<decode_stencil_kernel<T, 32>>(sm2)
+                                   : ensure_dyn_smem<decode_stencil_kernel<T, 64>>(sm2));
+      if (e != cudaSuccess) return e;
+    }
+    if ((e = launch_pdl(d2, dim3(d.Hkv, d.B), dim3(256), sm2, st, p2)) != cudaSuccess) return e;
+    mark();
   }
-  if ((e = launch_pdl(d2, dim3(d.Hkv, d.B), dim3(256), sm2, st, p2)) != cudaSuccess) return e;
-  mark();
-  // D3
+  // D3 (with D2 inside when fused)
   const float scale_log2 = static_cast<float>(1.4426950408889634 / sqrt(static_cast<double>(d.DL)));
-  if (d.DL == 16) e = launch_decode_attn<16, TL>(d, a, scale_log2, st);
-  else if (d.DL == 32) e = launch_decode_attn<32, TL>(d, a, scale_log2, st);
-  else e = launch_decode_attn<64, TL>(d, a, scale_log2, st);
+  const D2Params<__nv_bfloat16> *p2f = nullptr;
+  if constexpr (sizeof(T) == 2) p2f = fused ? &p2 : nullptr;
+  if (d.DL == 16) e = launch_decode_attn<16, TL>(d, a, scale_log2, p2f, st);
+  else if (d.DL == 32) e = launch_decode_attn<32, TL>(d, a, scale_log2, p2f, st);
+  else e = launch_decode_attn<64, TL>(d, a, scale_log2, p2f, st);
   if (e != cudaSuccess) return e;
   mark();
   // D3b (+ lengths advance for float32 layers; the 16-bit D4 advances them)

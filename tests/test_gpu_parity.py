@@ -286,21 +286,28 @@ def test_decode_step_full_size(cuda_lib):
 
 def test_decode_kernel_count(cuda_lib):
     """The step launches projection, stencil, attention and output kernels, plus the merge of
-    the attention's key splits when the (sequence, group) pairs are fewer than the SMs."""
+    the attention's key splits when the (sequence, group) pairs are fewer than the SMs; with
+    unsplit keys and d~ <= 32 the stencil runs inside the attention kernel."""
     cls = cuda_lib
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     cfg = cls.make_config(2048, 16, 4, 4)
-    assert cls.cca_decode_kernel_count(cfg, 64, 8300) == (4 if 64 * 4 >= sms else 5)
+    assert cls.cca_decode_kernel_count(cfg, 64, 8300) == (3 if 64 * 4 >= sms else 5)
+    cfg64 = cls.make_config(2048, 16, 4, 2)                  # d~ = 64: stencil kernel of its own
+    assert cls.cca_decode_kernel_count(cfg64, 64, 8300) == (4 if 64 * 4 >= sms else 5)
     assert cls.cca_decode_kernel_count(cfg, 2, 8300) == 5
     assert cls.cca_decode_kernel_count(cls.make_config(256, 4, 4, 4, dtype=cls.CCA_F32), 64, 300) == 5
     assert cls.cca_decode_kernel_count(cfg, 0, 8300) < 0
 
 
-def test_decode_ragged_lengths(cuda_lib):
-    w = W.Workload("dec", 5, 300, 256, 4, 2, 2, decode=True)
-    lengths = [0, 1, 255, 256, 300]
+@pytest.mark.parametrize("C,max_seq,lengths", [
+    (2, 320, [0, 1, 255, 256, 300]),      # d~=32, keys split over CTAs (merge kernel)
+    (2, 256, [0, 1, 129, 255, 200]),      # d~=32, unsplit: stencil inside the attention kernel
+    (4, 256, [3, 0, 255, 64, 77]),        # d~=16, unsplit, fused
+])
+def test_decode_ragged_lengths(cuda_lib, C, max_seq, lengths):
+    w = W.Workload("dec", 5, max(lengths), 256, 4, 2, C, decode=True)
     inp = W.make_inputs(w, seed=2, conv_std=0.4, lengths=lengths)
-    _, cache, y, (ry, *_rest) = decode_vs_oracle(cuda_lib, w, inp, 320)
+    _, cache, y, (ry, *_rest) = decode_vs_oracle(cuda_lib, w, inp, max_seq)
     assert bf16_err(f64(y), ry) <= BF16_TOL
     assert cache.lengths.cpu().tolist() == [l + 1 for l in lengths]
 
