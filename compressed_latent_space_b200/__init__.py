@@ -68,6 +68,8 @@ _SIGS = {
     "cca_decode_step": (c_int, [POINTER(cca_config_t), POINTER(cca_weights_t), c_void_p, c_void_p,
                                 POINTER(cca_cache_t), c_void_p, c_size_t, c_void_p]),
     "cca_cache_check": (c_int, [POINTER(cca_cache_t), c_void_p]),
+    "cca_gemm_t": (c_int, [c_int, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int,
+                           c_void_p, c_void_p]),
     "cca_gemm": (c_int, [c_int, c_int, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int,
                          c_void_p, c_void_p]),
     "cca_stage_stencil": (c_int, [POINTER(cca_config_t), c_void_p, c_int, c_int, c_void_p,
@@ -208,6 +210,11 @@ def cca_backward(cfg, weights, x, dy, batch, seq, dx, dw_qkv, dw_o, dconv_seq, d
 
 def cca_cache_check(cache, stream=None):
     _check(load().cca_cache_check(ctypes.byref(cache), _stream(stream)))
+
+
+def cca_gemm_t(out_dtype, A, B, C, M, N, K, a_trans, b_trans, status=None, stream=None):
+    _check(load().cca_gemm_t(out_dtype, _ptr(A), _ptr(B), _ptr(C), M, N, K, 1 if a_trans else 0,
+                             1 if b_trans else 0, _ptr(status), _stream(stream)))
 
 
 def cca_gemm(dtype, out_dtype, A, B, C, M, N, K, status=None, stream=None):

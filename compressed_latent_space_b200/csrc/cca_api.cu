@@ -463,13 +463,13 @@ CCA_API int cca_prefill_forward(const cca_config_t *cfg, const cca_weights_t *w,
 namespace {
 // ------------------------------------------------------------------ backward pass
 struct BackwardLayout {
-  size_t status, wsplit, wsplitT, P, q, k, v, o, lse, D, woT, dO, dyT, oT, dq, dk, dv, dA, dPpart,
-      dP, wqkvT, dPT, xT, total;
+  size_t status, wsplit, wsplitT, P, q, k, v, o, lse, D, woT, dO, oB, dq, dk, dv, dA, dPpart,
+      dP, total;
 };
 
 BackwardLayout backward_layout(const cca::Dims &d, int B, int S) {
   BackwardLayout L;
-  const size_t M = static_cast<size_t>(B) * S, M8 = (M + 7) & ~static_cast<size_t>(7);
+  const size_t M = static_cast<size_t>(B) * S;
   const size_t rows = static_cast<size_t>(B) * d.H * S;
   size_t off = 0;
   auto take = [&](size_t bytes) { const size_t o = off; off += align256(bytes); return o; };
@@ -485,17 +485,13 @@ BackwardLayout backward_layout(const cca::Dims &d, int B, int S) {
   L.D = take(rows * 4);
   L.woT = take(static_cast<size_t>(d.NQ) * d.E * 2);
   L.dO = take(M * d.NQ * 2);
-  L.dyT = take(static_cast<size_t>(d.E) * M8 * 2);
-  L.oT = take(static_cast<size_t>(d.NQ) * M8 * 2);
+  L.oB = take(M * d.NQ * 2);
   L.dq = take(M * d.NQ * 4);
   L.dk = take(M * d.NKV * 4);
   L.dv = take(M * d.NKV * 4);
   L.dA = take(M * (d.NQ + d.NKV) * 4);
   L.dPpart = take(M * d.NQKV * 4);
   L.dP = take(M * d.NQKV * 2);
-  L.wqkvT = take(static_cast<size_t>(d.E) * d.NQKV * 2);
-  L.dPT = take(static_cast<size_t>(d.NQKV) * M8 * 2);
-  L.xT = take(static_cast<size_t>(d.E) * M8 * 2);
   L.total = off;
   return L;
 }
@@ -545,7 +541,7 @@ CCA_API int cca_backward(const cca_config_t *cfg, const cca_weights_t *w, const 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char *ws = static_cast<char *>(workspace);
   int *status = reinterpret_cast<int *>(ws + L.status);
-  const int M = batch * seq, M8 = (M + 7) & ~7;
+  const int M = batch * seq;
   cudaError_t e = cudaMemsetAsync(status, 0, 256, st);
   if (e == cudaSuccess)
     e = cudaMemsetAsync(dconv_seq, 0, static_cast<size_t>(d.NQ + d.NKV) * d.KC * 4, st);
@@ -617,17 +613,15 @@ CCA_API int cca_backward(const cca_config_t *cfg, const cca_weights_t *w, const 
   if ((e = cca::stencil_backward(d, sb, st)) != cudaSuccess)
     return cuda_fail(e, "stencil backward launch");
   rec.mark();
-  // dx = dP W_qkv, dW_qkv = dP^T x, dW_o = dy^T o (token dimension padded to a multiple of 8)
-  void *wqkvT = ws + L.wqkvT, *dPT = ws + L.dPT, *xT = ws + L.xT, *dyT = ws + L.dyT, *oT = ws + L.oT;
-  if ((e = cca::transpose16(w->w_qkv, wqkvT, d.NQKV, d.E, d.NQKV, false, st)) != cudaSuccess ||
-      (e = cca::transpose16(ws + L.dP, dPT, M, d.NQKV, M8, false, st)) != cudaSuccess ||
-      (e = cca::transpose16(x, xT, M, d.E, M8, false, st)) != cudaSuccess ||
-      (e = cca::transpose16(dy, dyT, M, d.E, M8, false, st)) != cudaSuccess ||
-      (e = cca::transpose16(o, oT, M, d.NQ, M8, true, st)) != cudaSuccess)
-    return cuda_fail(e, "transpose launch");
-  if ((rc = gemm_dispatch(CCA_BF16, 0, ws + L.dP, wqkvT, dx, M, d.E, d.NQKV, status, st))) return rc;
-  if ((rc = gemm_dispatch(CCA_BF16, 1, dPT, xT, dw_qkv, d.NQKV, d.E, M8, status, st))) return rc;
-  if ((rc = gemm_dispatch(CCA_BF16, 1, dyT, oT, dw_o, d.E, d.NQ, M8, status, st))) return rc;
+  // dx = dP W_qkv, dW_qkv = dP^T x, dW_o = dy^T o: the operands read as stored (row-major
+  // activations as MN-major tiles of the products over tokens); o in bfloat16 for dW_o
+  void *oB = ws + L.oB;
+  if ((e = cca::convert_f16_to_bf16(o, oB, static_cast<size_t>(M) * d.NQ, st)) != cudaSuccess)
+    return cuda_fail(e, "attention output conversion launch");
+  if ((e = cca::gemm_tcgen05_t(ws + L.dP, w->w_qkv, dx, M, d.E, d.NQKV, 0, 1, 0, status, st)) != cudaSuccess ||
+      (e = cca::gemm_tcgen05_t(ws + L.dP, x, dw_qkv, d.NQKV, d.E, M, 1, 1, 1, status, st)) != cudaSuccess ||
+      (e = cca::gemm_tcgen05_t(dy, oB, dw_o, d.E, d.NQ, M, 1, 1, 1, status, st)) != cudaSuccess)
+    return cuda_fail(e, "gradient GEMM launch");
   rec.mark();
   return ok();
 }
@@ -719,6 +713,22 @@ CCA_API int cca_gemm(int dtype, int out_dtype, const void *A, const void *B, voi
   int rc = gemm_dispatch(dtype, out_dtype == CCA_F32, A, B, C, M, N, K, status,
                          static_cast<cudaStream_t>(stream));
   return rc ? rc : ok();
+}
+
+CCA_API int cca_gemm_t(int out_dtype, const void *A, const void *B, void *C, int M, int N, int K,
+                       int a_trans, int b_trans, int *status, void *stream) {
+  if (out_dtype != CCA_F32 && out_dtype != CCA_BF16)
+    return fail(CCA_ERR_INVALID_ARG, "bad out dtype %d", out_dtype);
+  if (M < 0 || N < 0 || K <= 0) return fail(CCA_ERR_INVALID_ARG, "bad shape %d x %d x %d", M, N, K);
+  if (M > 0 && N > 0 && (!A || !B || !C)) return fail(CCA_ERR_INVALID_ARG, "NULL operand");
+  if (!aligned16(A) || !aligned16(B) || !aligned16(C)) return fail(CCA_ERR_ALIGNMENT, "operands must be 16-byte aligned");
+  if ((a_trans ? M : K) % 8 != 0 || (b_trans ? N : K) % 8 != 0)
+    return fail(CCA_ERR_UNSUPPORTED, "each operand's contiguous extent must be a multiple of 8");
+  if (injected_launch_failure()) return fail(CCA_ERR_CUDA, "injected launch failure");
+  const cudaError_t e = cca::gemm_tcgen05_t(A, B, C, M, N, K, a_trans ? 1 : 0, b_trans ? 1 : 0,
+                                            out_dtype == CCA_F32, status,
+                                            static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? ok() : cuda_fail(e, "GEMM launch");
 }
 
 CCA_API size_t cca_stage_stencil_workspace_size(const cca_config_t *cfg) {

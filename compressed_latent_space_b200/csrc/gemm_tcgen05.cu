@@ -2,8 +2,12 @@
 //
 // Used for the down-projection x W_qkv^T and the up-projection o W_o^T of the layer
 // (gist.science explainer, 2. Methodology, Core Mechanism: "Down-Projection"; the result of
-// the latent attention returns to width E through one output matrix).  Both operands are
-// K-major (PyTorch Linear layout), bf16 or f16, accumulated in fp32 in tensor memory.
+// the latent attention returns to width E through one output matrix), and for the backward
+// pass's gradient products.  Operands are K-major (PyTorch Linear layout) or, per operand,
+// MN-major (stored [K][M] / [K][N], as a row-major activation is for a product over its
+// rows), bf16 or f16, accumulated in fp32 in tensor memory.  An MN-major tile is TMA-loaded
+// as 64-element (128-byte) column chunks of 64 K rows in the 128-byte swizzle, which is the
+// UMMA MN-major layout with the chunks LBO = 8 KB apart and 8-row groups SBO = 1 KB apart.
 //
 // Persistent, warp-specialised kernel, one CTA per SM:
 //   warp 0  : TMA producer, 4-stage ring of 128x64 (A) + 256x64 (B) tiles, 128B swizzle
@@ -40,7 +44,9 @@ struct Bars {
 };
 constexpr size_t SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + sizeof(Bars);
 
-template <typename OutT, int AB_F16>
+constexpr int MN_CHUNK_BYTES = 64 * BK * 2;         // one 64-element MN chunk of a stage
+
+template <typename OutT, int AB_F16, int A_MN, int B_MN>
 __global__ void __launch_bounds__(THREADS, 1)
     gemm_bf16_kernel(const __grid_constant__ CUtensorMap mapA,
                      const __grid_constant__ CUtensorMap mapB, OutT *__restrict__ C,
@@ -93,15 +99,28 @@ __global__ void __launch_bounds__(THREADS, 1)
           if (!mbar_wait(&bars->empty[stage], phase ^ 1u, abort, status)) { ok = false; break; }
           uint8_t *sa = smem + stage * STAGE_BYTES;
           mbar_arrive_expect_tx(&bars->full[stage], STAGE_BYTES);
-          tma_load_2d(sa, &mapA, &bars->full[stage], kb * BK, m0);
-          tma_load_2d(sa + A_BYTES, &mapB, &bars->full[stage], kb * BK, n0);
+          if constexpr (A_MN) {
+#pragma unroll
+            for (int c = 0; c < BM / 64; ++c)
+              tma_load_2d(sa + c * MN_CHUNK_BYTES, &mapA, &bars->full[stage], m0 + 64 * c, kb * BK);
+          } else {
+            tma_load_2d(sa, &mapA, &bars->full[stage], kb * BK, m0);
+          }
+          if constexpr (B_MN) {
+#pragma unroll
+            for (int c = 0; c < BN / 64; ++c)
+              tma_load_2d(sa + A_BYTES + c * MN_CHUNK_BYTES, &mapB, &bars->full[stage], n0 + 64 * c,
+                          kb * BK);
+          } else {
+            tma_load_2d(sa + A_BYTES, &mapB, &bars->full[stage], kb * BK, n0);
+          }
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_f16_f32(BM, BN, 0, 0, AB_F16);
+      constexpr uint32_t idesc = idesc_f16_f32(BM, BN, A_MN, B_MN, AB_F16);
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
@@ -119,8 +138,12 @@ __global__ void __launch_bounds__(THREADS, 1)
           const uint32_t b_addr = a_addr + A_BYTES;
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {
-            const uint64_t ad = smem_desc(a_addr + k * 32, 16, 1024, 2);
-            const uint64_t bd = smem_desc(b_addr + k * 32, 16, 1024, 2);
+            // K-major: 16 K elements are 32 bytes along the row; MN-major: 16 K rows are two
+            // 8-row (1 KB) groups
+            const uint64_t ad = A_MN ? smem_desc(a_addr + k * 2048, MN_CHUNK_BYTES, 1024, 2)
+                                     : smem_desc(a_addr + k * 32, 16, 1024, 2);
+            const uint64_t bd = B_MN ? smem_desc(b_addr + k * 2048, MN_CHUNK_BYTES, 1024, 2)
+                                     : smem_desc(b_addr + k * 32, 16, 1024, 2);
             umma_f16_ss(d_tmem, ad, bd, idesc, (kb > 0 || k > 0) ? 1u : 0u);
           }
           umma_commit(&bars->empty[stage]);
@@ -210,13 +233,14 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2-D bf16 row-major tensor [rows, cols] -> box [box_rows, 64 cols], 128B swizzle.
+// 2-D bf16 row-major tensor [rows, cols] -> box [box_rows, 64 cols], 128B swizzle (a
+// K-major operand: box_rows MN rows of 64 K; an MN-major one: 64 K rows of 64 MN columns).
 bool make_map_2d(CUtensorMap *map, const void *ptr, int rows, int cols, int box_rows, int f16) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
-  cuuint32_t box[2] = {static_cast<cuuint32_t>(BK), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(box_rows)};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -237,17 +261,43 @@ int num_sms() {
   return n;
 }
 
-template <typename OutT, int AB_F16>
+template <typename OutT, int AB_F16, int A_MN = 0, int B_MN = 0>
 static cudaError_t launch_gemm(const CUtensorMap &ma, const CUtensorMap &mb, void *C, int M,
                                int N, int K, int *status, cudaStream_t st) {
-  if (cudaError_t e = ensure_dyn_smem<gemm_bf16_kernel<OutT, AB_F16>>(SMEM_BYTES);
+  if (cudaError_t e = ensure_dyn_smem<gemm_bf16_kernel<OutT, AB_F16, A_MN, B_MN>>(SMEM_BYTES);
       e != cudaSuccess)
     return e;
   const int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
   const int grid = tiles < num_sms() ? tiles : num_sms();
-  gemm_bf16_kernel<OutT, AB_F16><<<grid, THREADS, SMEM_BYTES, st>>>(ma, mb, static_cast<OutT *>(C), M,
-                                                             N, K, status);
+  gemm_bf16_kernel<OutT, AB_F16, A_MN, B_MN><<<grid, THREADS, SMEM_BYTES, st>>>(
+      ma, mb, static_cast<OutT *>(C), M, N, K, status);
   return cudaGetLastError();
+}
+
+cudaError_t gemm_tcgen05_t(const void *A, const void *B, void *C, int M, int N, int K, int a_mn,
+                           int b_mn, int out_f32, int *status, cudaStream_t st) {
+  if (M <= 0 || N <= 0) return cudaSuccess;
+  // every TMA row pitch a multiple of 16 bytes: the contiguous extent of each operand % 8
+  if ((a_mn ? M : K) % 8 != 0 || (b_mn ? N : K) % 8 != 0) return cudaErrorInvalidValue;
+  CUtensorMap ma, mb;
+  const bool okA = a_mn ? make_map_2d(&ma, A, K, M, BK, 0) : make_map_2d(&ma, A, M, K, BM, 0);
+  const bool okB = b_mn ? make_map_2d(&mb, B, K, N, BK, 0) : make_map_2d(&mb, B, N, K, BN, 0);
+  if (!okA || !okB) return cudaErrorInvalidValue;
+  const int sel = (a_mn ? 2 : 0) + (b_mn ? 1 : 0);
+  if (out_f32) {
+    switch (sel) {
+      case 0: return launch_gemm<float, 0, 0, 0>(ma, mb, C, M, N, K, status, st);
+      case 1: return launch_gemm<float, 0, 0, 1>(ma, mb, C, M, N, K, status, st);
+      case 2: return launch_gemm<float, 0, 1, 0>(ma, mb, C, M, N, K, status, st);
+      default: return launch_gemm<float, 0, 1, 1>(ma, mb, C, M, N, K, status, st);
+    }
+  }
+  switch (sel) {
+    case 0: return launch_gemm<__nv_bfloat16, 0, 0, 0>(ma, mb, C, M, N, K, status, st);
+    case 1: return launch_gemm<__nv_bfloat16, 0, 0, 1>(ma, mb, C, M, N, K, status, st);
+    case 2: return launch_gemm<__nv_bfloat16, 0, 1, 0>(ma, mb, C, M, N, K, status, st);
+    default: return launch_gemm<__nv_bfloat16, 0, 1, 1>(ma, mb, C, M, N, K, status, st);
+  }
 }
 
 cudaError_t gemm_tcgen05_f16out(const void *A, const void *B, void *C, int M, int N, int K,
@@ -300,7 +350,36 @@ __global__ void __launch_bounds__(256) bf16_to_f16_kernel(const __nv_bfloat16 *_
   }
 }
 
+__global__ void __launch_bounds__(256) f16_to_bf16_kernel(const __half *__restrict__ src,
+                                                          __nv_bfloat16 *__restrict__ dst, size_t n8) {
+  for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const uint4 u = reinterpret_cast<const uint4 *>(src)[i];
+    const __half2 *h = reinterpret_cast<const __half2 *>(&u);
+    uint4 o;
+    uint32_t *ow = reinterpret_cast<uint32_t *>(&o);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = __half22float2(h[e]);
+      ow[e] = pack_bf16x2(f.x, f.y);
+    }
+    reinterpret_cast<uint4 *>(dst)[i] = o;
+  }
+}
+
 }  // namespace
+
+cudaError_t convert_f16_to_bf16(const void *src, void *dst, size_t n, cudaStream_t st) {
+  if (n == 0) return cudaSuccess;
+  if (n % 8) return cudaErrorInvalidValue;
+  const size_t n8 = n / 8;
+  size_t blocks = (n8 + 255) / 256;
+  const size_t cap = static_cast<size_t>(num_sms()) * 8;
+  if (blocks > cap) blocks = cap;
+  f16_to_bf16_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+      static_cast<const __half *>(src), static_cast<__nv_bfloat16 *>(dst), n8);
+  return cudaGetLastError();
+}
 
 cudaError_t convert_bf16_to_f16(const void *src, void *dst, size_t n, int *status, cudaStream_t st) {
   if (n == 0) return cudaSuccess;

@@ -38,6 +38,11 @@ enum : unsigned { F_QK_MEAN = 1u, F_VALUE_SHIFT = 2u, F_QK_NORM = 4u, F_ROPE = 8
 // out (tcgen05 + TMA).
 cudaError_t gemm_tcgen05(const void *A, const void *B, void *C, int M, int N, int K, int ab_f16,
                          int out_f32, int *status, cudaStream_t st);
+// C[M, N] = sum_k A'[m, k] B'[n, k] on bf16 operands, A' = A [M, K] (a_mn == 0) or the
+// transpose of A stored [K, M] (a_mn == 1), B' likewise ([N, K] or [K, N]); fp32 or bf16 out.
+// The contiguous extent of each operand must be a multiple of 8.
+cudaError_t gemm_tcgen05_t(const void *A, const void *B, void *C, int M, int N, int K, int a_mn,
+                           int b_mn, int out_f32, int *status, cudaStream_t st);
 // The same contraction with a float16 result (the backward pass's dO, an operand of the
 // float16 attention-backward MMAs).
 cudaError_t gemm_tcgen05_f16out(const void *A, const void *B, void *C, int M, int N, int K,
@@ -45,6 +50,8 @@ cudaError_t gemm_tcgen05_f16out(const void *A, const void *B, void *C, int M, in
 // dst[i] = float16(src[i]) for a bf16 tensor of n elements (n % 8 == 0); a value beyond the
 // float16 range records DEV_RANGE in *status.
 cudaError_t convert_bf16_to_f16(const void *src, void *dst, size_t n, int *status, cudaStream_t st);
+// dst[i] = bfloat16(src[i]) for a float16 tensor of n elements (n % 8 == 0).
+cudaError_t convert_f16_to_bf16(const void *src, void *dst, size_t n, cudaStream_t st);
 // Same contraction on CUDA cores; element type float (bf16 == 0) or bf16.
 cudaError_t gemm_simt(int bf16, const void *A, const void *B, void *C, int M, int N, int K,
                       cudaStream_t st);

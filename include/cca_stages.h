@@ -22,6 +22,16 @@ extern "C" {
 CCA_API int cca_gemm(int dtype, int out_dtype, const void *A, const void *B, void *C, int M,
                      int N, int K, int *status, void *stream);
 
+/* The same contraction on bfloat16 operands either of which may be stored transposed:
+ * C[m, n] = sum_k A'[m, k] * B'[n, k] with A' = A [M, K] (a_trans == 0) or A stored [K, M]
+ * (a_trans == 1), B' = B [N, K] (b_trans == 0) or B stored [K, N] (b_trans == 1); C [M, N]
+ * float32 (out_dtype CCA_F32) or bfloat16.  The contiguous extent of each operand (K, or M /
+ * N when transposed) must be a multiple of 8.  The backward pass's gradient products
+ * (dx = dP W_qkv, dW_qkv = dP^T x, dW_o = dy^T o) read their operands this way, untransposed
+ * in memory.  Errors: INVALID_ARG, ALIGNMENT, UNSUPPORTED (extents), CUDA. */
+CCA_API int cca_gemm_t(int out_dtype, const void *A, const void *B, void *C, int M, int N, int K,
+                       int a_trans, int b_trans, int *status, void *stream);
+
 /* Latent stencil: P [batch*seq, n_q + 2 n_kv] (the projections, float32) ->
  * q [batch, H, seq, d~], k and v [batch, Hkv, kv_stride, d~] with kv_stride >= seq
  * (q, k and v of the latent element type of cca.h: float16 for bfloat16 layers).

@@ -26,6 +26,43 @@ def small(name, **kw):
 
 
 # ------------------------------------------------------------------ single kernels
+@pytest.mark.parametrize("a_trans,b_trans", [(0, 0), (0, 1), (1, 0), (1, 1)])
+@pytest.mark.parametrize("M,N,K", [(128, 256, 64), (200, 264, 77), (1536, 2048, 1000),
+                                   (2048, 1024, 4099), (64, 520, 8)])
+def test_gemm_transposed_operands(cuda_lib, M, N, K, a_trans, b_trans):
+    """cca_gemm_t: either operand read as stored transposed ([K, M] / [K, N], the MN-major
+    tiles of the backward's gradient products), ragged M, N and K, against a float64 product."""
+    cls = cuda_lib
+    if (not a_trans or not b_trans) and K % 8:      # a K-major operand needs K % 8 == 0
+        K += 8 - K % 8
+    g = torch.Generator("cpu").manual_seed(M * 7 + N * 3 + K + a_trans * 2 + b_trans)
+    A = torch.randn(M, K, generator=g).to(torch.bfloat16)
+    B = (torch.randn(N, K, generator=g) * 0.05).to(torch.bfloat16)
+    ref = A.double() @ B.double().T
+    As = (A.t() if a_trans else A).contiguous().cuda()
+    Bs = (B.t() if b_trans else B).contiguous().cuda()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    C32 = torch.empty(M, N, dtype=torch.float32, device="cuda")
+    cls.cca_gemm_t(cls.CCA_F32, As, Bs, C32, M, N, K, a_trans, b_trans, status)
+    C16 = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    cls.cca_gemm_t(cls.CCA_BF16, As, Bs, C16, M, N, K, a_trans, b_trans, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    err = (C32.double().cpu() - ref).abs()
+    assert (err <= 2e-5 * ref.abs() + 1e-4 * ref.pow(2).mean().sqrt()).all(), float(err.max())
+    err16 = (C16.double().cpu() - ref).abs()
+    assert (err16 <= 8e-3 * ref.abs() + 2e-3 * ref.pow(2).mean().sqrt()).all(), float(err16.max())
+
+
+def test_gemm_transposed_rejects_ragged_rows(cuda_lib):
+    cls = cuda_lib
+    A = torch.zeros(12, 16, dtype=torch.bfloat16, device="cuda")
+    C = torch.zeros(16, 16, dtype=torch.float32, device="cuda")
+    with pytest.raises(cls.CCAError) as e:       # A stored [K=12, M=16]: fine; B [K, N=12]: not
+        cls.cca_gemm_t(cls.CCA_F32, A, A, C, 16, 12, 12, 1, 1)
+    assert e.value.code == cls.CCA_ERR_UNSUPPORTED
+
+
 @pytest.mark.parametrize("M,N,K", [(128, 256, 64), (300, 520, 200), (1000, 1536, 2048),
                                    (257, 768, 512), (64, 2048, 512), (4096, 2048, 1024)])
 def test_gemm_bf16_tcgen05(cuda_lib, M, N, K):
