@@ -17,9 +17,9 @@
 //                         S^T = K Q^T and dP^T = V dO^T with the keys on the tensor-memory
 //                         lanes, P^T and dS^T written back as float16 pairs, then
 //                         dV += P^T dO and dK += dS^T Q straight from tensor memory.
-// Warps 0-7 compute the elementwise part, two per tensor-memory lane quadrant (one query or
-// key row per thread, each warp on half of the tile's 128 columns); warp 8 is the TMA producer,
-// warp 9 issues the MMAs.  P / dS go to their own tensor-memory columns, so as soon as every
+// Warps 0-15 compute the elementwise part, four per tensor-memory lane quadrant (one query or
+// key row per thread, each warp on a quarter of the tile's 128 columns); warp 16 is the TMA
+// producer, warp 17 issues the MMAs.  P / dS go to their own tensor-memory columns, so as soon as every
 // elementwise warp has loaded its scores the next item's S / dP MMAs start, overlapping this
 // item's exponentials; a commit after the gradient MMAs guards the P / dS columns.  Every wait
 // is bounded; on a timeout the CTA records it in the status word, stops, and frees its TMEM.
@@ -32,7 +32,9 @@ namespace cca {
 namespace {
 
 constexpr int BT = 128;              // rows of every tile (queries or keys)
-constexpr int B_EW = 8;              // elementwise warps: two per TMEM lane quadrant
+constexpr int B_EW = 16;             // elementwise warps: four per TMEM lane quadrant
+constexpr int NPART = B_EW / 4;      // column parts of a tile per lane quadrant
+constexpr int CW = BT / NPART;       // score columns (keys or queries) per elementwise warp
 constexpr int BW_TMA = B_EW, BW_MMA = B_EW + 1;
 constexpr int B_THREADS = (B_EW + 2) * 32;
 constexpr int BSLOTS = 3;            // ring depth of the streamed tiles
@@ -72,17 +74,37 @@ __device__ __forceinline__ bool elect_one() {
   return pred != 0;
 }
 
-__device__ __forceinline__ void ew_sync() {      // the eight elementwise warps only
-  asm volatile("bar.sync 1, 256;" ::: "memory");
+__device__ __forceinline__ void ew_sync() {      // the elementwise warps only
+  asm volatile("bar.sync 1, %0;" ::"n"(B_EW * 32) : "memory");
 }
 
-// The elementwise warp's 64 columns of S and dP (its half of the tile's 128) for its TMEM lane.
-__device__ __forceinline__ void load_half(uint32_t base, uint32_t (&rs)[64], uint32_t (&rp)[64]) {
-  tmem_ld32(base + C_S, *reinterpret_cast<uint32_t(*)[32]>(&rs[0]));
-  tmem_ld32(base + C_S + 32, *reinterpret_cast<uint32_t(*)[32]>(&rs[32]));
-  tmem_ld32(base + C_DP, *reinterpret_cast<uint32_t(*)[32]>(&rp[0]));
-  tmem_ld32(base + C_DP + 32, *reinterpret_cast<uint32_t(*)[32]>(&rp[32]));
+// The elementwise warp's CW columns of S and dP (its part of the tile's 128) for its TMEM lane.
+__device__ __forceinline__ void load_part(uint32_t base, uint32_t (&rs)[CW], uint32_t (&rp)[CW]) {
+  static_assert(CW == 32, "one 32-column load each");
+  tmem_ld32(base + C_S, rs);
+  tmem_ld32(base + C_DP, rp);
   tmem_ld_wait();
+}
+
+// This warp's PW = DL / NPART accumulator columns [col, col + PW) of its lane, as floats.
+template <int PW>
+__device__ __forceinline__ void load_acc(uint32_t taddr, float (&o)[PW]) {
+  if constexpr (PW == 4) {
+    uint32_t r[4];
+    tmem_ld4(taddr, r);
+    tmem_ld_wait();
+#pragma unroll
+    for (int e = 0; e < 4; ++e) o[e] = __uint_as_float(r[e]);
+  } else {
+#pragma unroll
+    for (int c = 0; c < PW / 8; ++c) {
+      uint32_t r[8];
+      tmem_ld8(taddr + c * 8, r);
+      tmem_ld_wait();
+#pragma unroll
+      for (int e = 0; e < 8; ++e) o[c * 8 + e] = __uint_as_float(r[e]);
+    }
+  }
 }
 
 // ------------------------------------------------------------------------------------ dQ
@@ -205,7 +227,7 @@ __global__ void __launch_bounds__(B_THREADS, 1)
       __syncwarp();
     }
   } else {
-    const int quad = warp & 3, hf = warp >> 2;       // lanes of quadrant, key columns of half
+    const int quad = warp & 3, hf = warp >> 2;       // lanes of quadrant, key columns of part
     const int row = quad * 32 + lane;
     const int qpos = qt * BT + row;
     const bool valid = qpos < S;
@@ -213,14 +235,14 @@ __global__ void __launch_bounds__(B_THREADS, 1)
     const float lrow = valid ? lse[ridx] : INFINITY;   // invalid rows: every p is 0
     const float drow = valid ? Dd[ridx] : 0.f;
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-    const uint32_t base = tmem + lane_off + hf * 64;
+    const uint32_t base = tmem + lane_off + hf * CW;
     bool ok = true;
     for (int j = 0; ok && j < nk; ++j) {
       ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full, j & 1, abort, status));
       if (!ok) break;
       tc_fence_after();
-      uint32_t rs[64], rp[64];
-      load_half(base, rs, rp);
+      uint32_t rs[CW], rp[CW];
+      load_part(base, rs, rp);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->s_free);    // the next tile's S / dP may overwrite
@@ -228,14 +250,14 @@ __global__ void __launch_bounds__(B_THREADS, 1)
       // packed subtract and multiply; keys past this row's query masked on the diagonal tile
       const bool diag = j == qt;
       const uint64_t sc2 = f2(scale_log2, scale_log2), nl2 = f2(-lrow, -lrow), nd2 = f2(-drow, -drow);
-      uint32_t pk[32];
+      uint32_t pk[CW / 2];
 #pragma unroll
-      for (int e = 0; e < 32; ++e) {
+      for (int e = 0; e < CW / 2; ++e) {
         float x0, x1;
         unf2(fma2(f2(__uint_as_float(rs[2 * e]), __uint_as_float(rs[2 * e + 1])), sc2, nl2), x0, x1);
         float p0 = ex2(x0), p1 = ex2(x1);
         if (diag) {
-          const int kcol = hf * 64 + 2 * e;
+          const int kcol = hf * CW + 2 * e;
           if (kcol > row) p0 = 0.f;
           if (kcol + 1 > row) p1 = 0.f;
         }
@@ -248,9 +270,7 @@ __global__ void __launch_bounds__(B_THREADS, 1)
       if (j > 0) ok = __all_sync(0xffffffffu, mbar_wait(&bars->pds_free, (j - 1) & 1, abort, status));
       if (!ok) break;
       tc_fence_after();
-      const uint32_t pd = tmem + lane_off + C_DS + hf * 32;
-      tmem_st16(pd, *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
-      tmem_st16(pd + 16, *reinterpret_cast<uint32_t(*)[16]>(&pk[16]));
+      tmem_st16(tmem + lane_off + C_DS + hf * (CW / 2), pk);
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
@@ -259,21 +279,15 @@ __global__ void __launch_bounds__(B_THREADS, 1)
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars->done, 0, abort, status));
     if (ok) {
       tc_fence_after();
-      float *dst = dq + ridx * DL;
+      constexpr int PW = DL / NPART;                 // this part's dQ columns
+      float o[PW];
+      load_acc<PW>(tmem + lane_off + C_ACC + hf * PW, o);
+      if (valid) {
+        float *dst = dq + ridx * DL + hf * PW;
 #pragma unroll
-      for (int c = 0; c < DL / 16; ++c) {           // this half's DL/2 columns, 8 at a time
-        uint32_t o[8];
-        const int col = hf * (DL / 2) + c * 8;
-        tmem_ld8(tmem + lane_off + C_ACC + col, o);
-        tmem_ld_wait();
-        if (valid) {
-          reinterpret_cast<float4 *>(dst + col)[0] =
-              make_float4(__uint_as_float(o[0]) * scale, __uint_as_float(o[1]) * scale,
-                          __uint_as_float(o[2]) * scale, __uint_as_float(o[3]) * scale);
-          reinterpret_cast<float4 *>(dst + col)[1] =
-              make_float4(__uint_as_float(o[4]) * scale, __uint_as_float(o[5]) * scale,
-                          __uint_as_float(o[6]) * scale, __uint_as_float(o[7]) * scale);
-        }
+        for (int c = 0; c < PW / 4; ++c)
+          reinterpret_cast<float4 *>(dst)[c] = make_float4(o[4 * c] * scale, o[4 * c + 1] * scale,
+                                                           o[4 * c + 2] * scale, o[4 * c + 3] * scale);
       }
     }
   }
@@ -405,11 +419,11 @@ __global__ void __launch_bounds__(B_THREADS, 1)
       __syncwarp();
     }
   } else {
-    const int quad = warp & 3, hf = warp >> 2;       // lanes of quadrant, query columns of half
+    const int quad = warp & 3, hf = warp >> 2;       // lanes of quadrant, query columns of part
     const int row = quad * 32 + lane;
     const int kpos = kt * BT + row;
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-    const uint32_t base = tmem + lane_off + hf * 64;
+    const uint32_t base = tmem + lane_off + hf * CW;
     // per-item lse and D of the item's 128 queries, staged in shared memory one item ahead
     auto stage_stats = [&](int n) {
       if (n >= nitems || threadIdx.x >= BT) return;
@@ -427,8 +441,8 @@ __global__ void __launch_bounds__(B_THREADS, 1)
       stage_stats(n + 1);
       ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full, n & 1, abort, status)) && ok;
       tc_fence_after();
-      uint32_t rs[64], rp[64];
-      load_half(base, rs, rp);
+      uint32_t rs[CW], rp[CW];
+      load_part(base, rs, rp);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->s_free);
@@ -436,18 +450,18 @@ __global__ void __launch_bounds__(B_THREADS, 1)
       const bool diag = qt == kt;
       // per query column: -lse and -D (broadcast 8-byte shared-memory reads), then P^T and
       // dS^T on pairs of queries with packed FMA / subtract / multiply
-      const float *bl = sL + (n & 1) * 2 * BT + hf * 64, *bd = bl + BT;
+      const float *bl = sL + (n & 1) * 2 * BT + hf * CW, *bd = bl + BT;
       const uint64_t sc2 = f2(scale_log2, scale_log2);
-      uint32_t pkp[32], pks[32];
+      uint32_t pkp[CW / 2], pks[CW / 2];
 #pragma unroll
-      for (int e = 0; e < 32; ++e) {
+      for (int e = 0; e < CW / 2; ++e) {
         const float2 nl = *reinterpret_cast<const float2 *>(bl + 2 * e);
         const float2 nd = *reinterpret_cast<const float2 *>(bd + 2 * e);
         float x0, x1;
         unf2(fma2(f2(__uint_as_float(rs[2 * e]), __uint_as_float(rs[2 * e + 1])), sc2, f2(nl.x, nl.y)), x0, x1);
         float p0 = ex2(x0), p1 = ex2(x1);
         if (diag) {                                  // a query before this key
-          const int qcol = hf * 64 + 2 * e;
+          const int qcol = hf * CW + 2 * e;
           if (qcol < row) p0 = 0.f;
           if (qcol + 1 < row) p1 = 0.f;
         }
@@ -460,11 +474,8 @@ __global__ void __launch_bounds__(B_THREADS, 1)
       // the previous item's dV / dK MMAs must have read P^T / dS^T before they are rewritten
       if (n > 0) ok = __all_sync(0xffffffffu, mbar_wait(&bars->pds_free, (n - 1) & 1, abort, status)) && ok;
       tc_fence_after();
-      const uint32_t pp = tmem + lane_off + C_P + hf * 32, pd = tmem + lane_off + C_DS + hf * 32;
-      tmem_st16(pp, *reinterpret_cast<uint32_t(*)[16]>(&pkp[0]));
-      tmem_st16(pp + 16, *reinterpret_cast<uint32_t(*)[16]>(&pkp[16]));
-      tmem_st16(pd, *reinterpret_cast<uint32_t(*)[16]>(&pks[0]));
-      tmem_st16(pd + 16, *reinterpret_cast<uint32_t(*)[16]>(&pks[16]));
+      tmem_st16(tmem + lane_off + C_P + hf * (CW / 2), pkp);
+      tmem_st16(tmem + lane_off + C_DS + hf * (CW / 2), pks);
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
@@ -475,20 +486,17 @@ __global__ void __launch_bounds__(B_THREADS, 1)
       tc_fence_after();
       const bool valid = kpos < S;
       const size_t ridx = (static_cast<size_t>(b) * Hkv + g) * S + (valid ? kpos : 0);
+      constexpr int PW = DL / NPART;                 // this part's dV / dK columns
+      float ov[PW], ok2[PW];
+      load_acc<PW>(tmem + lane_off + C_ACC + hf * PW, ov);
+      load_acc<PW>(tmem + lane_off + C_ACC + DL + hf * PW, ok2);
+      if (valid && nitems > 0) {
+        float *pv = dv + ridx * DL + hf * PW, *pk = dk + ridx * DL + hf * PW;
 #pragma unroll
-      for (int c = 0; c < DL / 16; ++c) {           // this half's DL/2 columns, 8 at a time
-        const int col = hf * (DL / 2) + c * 8;
-        uint32_t ov[8], okk[8];
-        tmem_ld8(tmem + lane_off + C_ACC + col, ov);
-        tmem_ld8(tmem + lane_off + C_ACC + DL + col, okk);
-        tmem_ld_wait();
-        if (valid && nitems > 0) {
-          float *pv = dv + ridx * DL + col, *pk = dk + ridx * DL + col;
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            pv[e] = __uint_as_float(ov[e]);
-            pk[e] = __uint_as_float(okk[e]) * scale;
-          }
+        for (int c = 0; c < PW / 4; ++c) {
+          reinterpret_cast<float4 *>(pv)[c] = make_float4(ov[4 * c], ov[4 * c + 1], ov[4 * c + 2], ov[4 * c + 3]);
+          reinterpret_cast<float4 *>(pk)[c] = make_float4(ok2[4 * c] * scale, ok2[4 * c + 1] * scale,
+                                                          ok2[4 * c + 2] * scale, ok2[4 * c + 3] * scale);
         }
       }
     }
