@@ -628,6 +628,9 @@ __global__ void __launch_bounds__(128, 1) decode_attn_tc_kernel(
   constexpr int WK = NT * 8;                         // keys per warp per sub-chunk
   constexpr int SLOT = 2 * TC_SUB * DL;              // halves per slot: [K | V]
   static_assert(4 * WK == TC_SUB && NT % 2 == 0, "four warps cover a sub-chunk");
+  // cp.async.wait_group NSLOT - 2 below: a 12-slot ring (wait_group 10) raised an illegal
+  // instruction on this GPU, 6 slots (wait_group 4) run; keep the count of groups in flight small
+  static_assert(NSLOT <= 6, "at most five copy groups in flight");
   extern __shared__ __align__(16) uint8_t smraw[];
   __half *ring = reinterpret_cast<__half *>(smraw);  // [NSLOT][K, V][TC_SUB][DL], swizzled
   float *wst = reinterpret_cast<float *>(ring + NSLOT * SLOT);     // [4][8 heads][DL + 2]
