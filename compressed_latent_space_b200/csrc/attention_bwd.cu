@@ -74,9 +74,6 @@ __device__ __forceinline__ bool elect_one() {
   return pred != 0;
 }
 
-__device__ __forceinline__ void ew_sync() {      // the elementwise warps only
-  asm volatile("bar.sync 1, %0;" ::"n"(B_EW * 32) : "memory");
-}
 
 // The elementwise warp's CW columns of S and dP (its part of the tile's 128) for its TMEM lane.
 __device__ __forceinline__ void load_part(uint32_t base, uint32_t (&rs)[CW], uint32_t (&rp)[CW]) {
@@ -314,8 +311,9 @@ __global__ void __launch_bounds__(B_THREADS, 1)
   extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t *sK = smem, *sV = smem + C::TILE, *sQ = smem + 2 * C::TILE;
   uint8_t *sDO = sQ + BSLOTS * C::TILE;
-  float *sL = reinterpret_cast<float *>(sDO + BSLOTS * C::TILE);   // [2][lse 128 | D 128]
-  BwdBars *bars = reinterpret_cast<BwdBars *>(sL + 2 * 2 * BT);
+  // per elementwise warp: [2 items][-lse 32 | -D 32] of its 32 query columns
+  float *sL = reinterpret_cast<float *>(sDO + BSLOTS * C::TILE);
+  BwdBars *bars = reinterpret_cast<BwdBars *>(sL + B_EW * 2 * 2 * CW);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = blockIdx.x, b = blockIdx.y, kt = blockIdx.z;       // small kt: most work first
   const int nitems = G * (nqt - kt);                // (query tile kt + n / G, head g*G + n % G)
@@ -424,20 +422,23 @@ __global__ void __launch_bounds__(B_THREADS, 1)
     const int kpos = kt * BT + row;
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
     const uint32_t base = tmem + lane_off + hf * CW;
-    // per-item lse and D of the item's 128 queries, staged in shared memory one item ahead
+    // each warp stages the negated lse and D of its own 32 query columns one item ahead in its
+    // own shared-memory slice (lane i the i-th column), so only __syncwarp orders them
+    float *wsl = sL + warp * 2 * 2 * CW;
     auto stage_stats = [&](int n) {
-      if (n >= nitems || threadIdx.x >= BT) return;
+      if (n >= nitems) return;
       const int qt = kt + n / G, h = g * G + n % G;
-      const int q = qt * BT + threadIdx.x;
+      const int q = qt * BT + hf * CW + lane;
       const size_t ridx = (static_cast<size_t>(b) * H + h) * S + q;
-      float *buf = sL + (n & 1) * 2 * BT;             // negated, for the packed FMA / add
-      buf[threadIdx.x] = q < S ? -lse[ridx] : -INFINITY;
-      buf[BT + threadIdx.x] = q < S ? -Dd[ridx] : 0.f;
+      float *buf = wsl + (n & 1) * 2 * CW;
+      buf[lane] = q < S ? -lse[ridx] : -INFINITY;
+      buf[CW + lane] = q < S ? -Dd[ridx] : 0.f;
     };
+    static_assert(CW == 32, "a lane per query column");
     stage_stats(0);
     bool ok = true;
     for (int n = 0; n < nitems; ++n) {
-      ew_sync();                                     // stats of item n visible, n-1's read
+      __syncwarp();                                  // stats of item n visible, n-1's read
       stage_stats(n + 1);
       ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full, n & 1, abort, status)) && ok;
       tc_fence_after();
@@ -450,7 +451,7 @@ __global__ void __launch_bounds__(B_THREADS, 1)
       const bool diag = qt == kt;
       // per query column: -lse and -D (broadcast 8-byte shared-memory reads), then P^T and
       // dS^T on pairs of queries with packed FMA / subtract / multiply
-      const float *bl = sL + (n & 1) * 2 * BT + hf * CW, *bd = bl + BT;
+      const float *bl = wsl + (n & 1) * 2 * CW, *bd = bl + CW;
       const uint64_t sc2 = f2(scale_log2, scale_log2);
       uint32_t pkp[CW / 2], pks[CW / 2];
 #pragma unroll
@@ -563,7 +564,7 @@ cudaError_t launch_bwd(const Dims &d, const AttnBwdArgs &a, cudaStream_t st) {
   const float scale_log2 = static_cast<float>(1.4426950408889634) * scale;
   const int nt = (d.S + BT - 1) / BT;
   const size_t smem_dq = (2 + 2 * BSLOTS) * C::TILE + sizeof(BwdBars);
-  const size_t smem_kv = (2 + 2 * BSLOTS) * C::TILE + 2 * 2 * BT * 4 + sizeof(BwdBars);
+  const size_t smem_kv = (2 + 2 * BSLOTS) * C::TILE + B_EW * 2 * 2 * CW * 4 + sizeof(BwdBars);
   cudaError_t e;
   if ((e = ensure_dyn_smem<attn_bwd_dq_kernel<DL>>(smem_dq)) != cudaSuccess) return e;
   if ((e = ensure_dyn_smem<attn_bwd_dkdv_kernel<DL>>(smem_kv)) != cudaSuccess) return e;
