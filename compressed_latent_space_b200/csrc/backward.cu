@@ -21,9 +21,9 @@ namespace cca {
 namespace {
 
 constexpr int S1_TT = 16;          // tokens per pass-1 tile (the M of its mma.sync tiles)
-constexpr int S1_THREADS = 256;
+constexpr int S1_THREADS = 512;    // sixteen warps: more of each phase in flight (8 warps: +25 %)
 constexpr int S1_WARPS = S1_THREADS / 32;
-constexpr int S1_MAXB = 20;        // filter-gradient 16 x 8 blocks per warp
+constexpr int S1_MAXB = 10;        // filter-gradient 16 x 8 blocks per warp (160 per CTA)
 constexpr int S1_KCMAX = 8;
 
 struct S1Params {

@@ -241,7 +241,7 @@ CCA_API size_t cca_backward_workspace_size(const cca_config_t *cfg, int batch, i
  * taken back), and the down-projection's.  With tp_size > 1 the gradients are the rank's, and
  * dx is the rank's share (the caller sums it over the ranks).  bfloat16 layers with the
  * convolutions, d~ in {16, 32, 64}, conv_kernel <= 8, (H/Hkv + 1) d~^2 <= 20480,
- * (H/Hkv + 2) d~ <= 1024, E % 8 == 0, and the stencil backward's per-CTA tiles within 200 KB of
+ * (H/Hkv + 2) d~ <= 2048, E % 8 == 0, and the stencil backward's per-CTA tiles within 200 KB of
  * shared memory (CCA_ERR_UNSUPPORTED otherwise; cca_backward_workspace_size returns 0 then).
  * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, ALIGNMENT, CUDA. */
 CCA_API int cca_backward(const cca_config_t *cfg, const cca_weights_t *w, const void *x,
