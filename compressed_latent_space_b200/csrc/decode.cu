@@ -197,13 +197,14 @@ __host__ __device__ inline size_t d2_smem_floats(int G, int DL, int KC) {
   return static_cast<size_t>(DL) * d2_ld(QKC)   // wt
          + QKC * KC                             // sequence filters
          + static_cast<size_t>(QKC) * (KC - 1)  // old conv state
-         + CH + 2 * QKC + 16;                   // pn, av, uv, inv
+         + CH + 2 * QKC + 16                    // pn, av, uv, inv
+         + DL;                                  // the value-shift state of the group's channels
 }
 
-// D2's shared-memory carve ([wt | wseq | old | pn | a | u | inv], floats)
+// D2's shared-memory carve ([wt | wseq | old | pn | a | u | inv | vsh], floats)
 template <int DL>
 struct D2Smem {
-  float *wt, *wseq, *old, *pn, *a, *u, *inv;
+  float *wt, *wseq, *old, *pn, *a, *u, *inv, *vsh;
   __device__ D2Smem(float *sm, int G, int KC) {
     const int QKC = (G + 1) * DL, CH = (G + 2) * DL;
     wt = sm;
@@ -213,27 +214,68 @@ struct D2Smem {
     a = pn + CH;
     u = a + QKC;
     inv = u + QKC;
+    vsh = inv + 16;
   }
 };
 
 // Before the grid-dependency wait: the group's filters into shared memory (no __syncthreads),
-// the sequence's conv state towards L2.
-template <typename T, int DL>
+// the sequence's conv and value-shift state towards L2.  The filters are read in batches of
+// independent loads, so that a CTA which only becomes resident after the previous kernel's
+// CTAs leave (and stages them with nothing to hide behind) pays one or two memory round trips.
+template <typename T, int DL, int BATCH = 8>
 __device__ __forceinline__ void d2_stage(const D2Params<T> &p, int g, int b, const D2Smem<DL> &m) {
   const int tid = threadIdx.x, nt = blockDim.x;
   const int G = p.G, QKC = (G + 1) * DL, KC = p.KC, KC1 = KC - 1;
   const int LD = d2_ld(QKC);
-  // filters: q heads g*G.., then k head H+g; W_head[i][j] -> wt[j][head * DL + i]
-  for (int e = tid; e < (G + 1) * DL * DL; e += nt) {
-    const int hh = e / (DL * DL), r = e % (DL * DL), i = r / DL, j = r % DL;
-    const int head = hh < G ? g * G + hh : p.H + g;
-    m.wt[j * LD + hh * DL + i] = p.conv_chan[static_cast<size_t>(head) * DL * DL + r];
+  // filters: q heads g*G.., then k head H+g; W_head[i][j] -> wt[j][head * DL + i], four
+  // consecutive j of one (head, i) per load (16-byte loads when the filters are so aligned)
+  const int nf4 = (G + 1) * DL * DL / 4;
+  const bool vec = (reinterpret_cast<uintptr_t>(p.conv_chan) & 15u) == 0;
+  for (int e0 = tid; e0 < nf4; e0 += BATCH * nt) {
+    float4 v[BATCH];
+#pragma unroll
+    for (int k = 0; k < BATCH; ++k) {
+      const int e = (e0 + k * nt) * 4;
+      if (e0 + k * nt < nf4) {
+        const int hh = e / (DL * DL), r = e % (DL * DL);
+        const int head = hh < G ? g * G + hh : p.H + g;
+        const float *src = p.conv_chan + static_cast<size_t>(head) * DL * DL + r;
+        v[k] = vec ? *reinterpret_cast<const float4 *>(src) : make_float4(src[0], src[1], src[2], src[3]);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < BATCH; ++k) {
+      const int e = (e0 + k * nt) * 4;
+      if (e0 + k * nt < nf4) {
+        const int hh = e / (DL * DL), r = e % (DL * DL), i = r / DL, j = r % DL;
+        float *dst = m.wt + j * LD + hh * DL + i;
+        dst[0] = v[k].x;
+        dst[LD] = v[k].y;
+        dst[2 * LD] = v[k].z;
+        dst[3 * LD] = v[k].w;
+      }
+    }
   }
   const int qcol0 = g * G * DL, kcol0 = p.NQ + g * DL;
-  for (int e = tid; e < QKC * KC; e += nt) {
-    const int c = e / KC, t = e % KC;
-    const int gc = c < G * DL ? qcol0 + c : kcol0 + (c - G * DL);
-    m.wseq[e] = p.conv_seq[static_cast<size_t>(gc) * KC + t];
+  for (int e0 = tid; e0 < QKC * KC; e0 += BATCH * nt) {
+    float v[BATCH];
+#pragma unroll
+    for (int k = 0; k < BATCH; ++k) {
+      const int e = e0 + k * nt;
+      if (e < QKC * KC) {
+        const int c = e / KC, t = e % KC;
+        const int gc = c < G * DL ? qcol0 + c : kcol0 + (c - G * DL);
+        v[k] = p.conv_seq[static_cast<size_t>(gc) * KC + t];
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < BATCH; ++k)
+      if (e0 + k * nt < QKC * KC) m.wseq[e0 + k * nt] = v[k];
+  }
+  if (p.flags & F_VALUE_SHIFT) {                     // the shifted channels of this group
+    const float *vs = p.vshift_state + static_cast<size_t>(b) * (p.NKV - p.VS0);
+    for (int c = max(g * DL, p.VS0) + tid * 32; c < (g + 1) * DL; c += nt * 32)
+      prefetch_l2(vs + (c - p.VS0));
   }
   const int W = p.NQ + p.NKV;
   const float *cs = p.conv_state + static_cast<size_t>(b) * KC1 * W;
@@ -246,33 +288,53 @@ __device__ __forceinline__ void d2_stage(const D2Params<T> &p, int g, int b, con
   }
 }
 
-// After the wait: the token's projections (sum of the split-K partials) and the old conv
-// state into shared memory, thread c taking channel c (the compute below keeps that mapping).
+// After the wait: the token's projections (sum of the split-K partials), the old conv state and
+// the value-shift state into shared memory, thread c taking channel c (the compute below keeps
+// that mapping for the projections and the conv state).
 template <typename T, int DL>
-__device__ __forceinline__ void d2_load(const D2Params<T> &p, int g, int b, const D2Smem<DL> &m) {
-  const int tid = threadIdx.x, nt = blockDim.x;
+__device__ __forceinline__ void d2_load(const D2Params<T> &p, int g, int b, const D2Smem<DL> &m,
+                                        int tid, int nt) {
   const int G = p.G, CH = (G + 2) * DL, QKC = (G + 1) * DL, KC1 = p.KC - 1;
   const int qcol0 = g * G * DL, kcol0 = p.NQ + g * DL, vcol0 = p.NQ + p.NKV + g * DL;
   const int W = p.NQ + p.NKV;
   const float *cs = p.conv_state + static_cast<size_t>(b) * KC1 * W;
+  const size_t kstride = static_cast<size_t>(p.B) * p.NQKV;
+  const float *vs = p.vshift_state + static_cast<size_t>(b) * (p.NKV - p.VS0);
   for (int c = tid; c < CH; c += nt) {
     const int gc = c < G * DL ? qcol0 + c : (c < QKC ? kcol0 + (c - G * DL) : vcol0 + (c - QKC));
-    float v = 0.f;
-    for (int ks = 0; ks < p.ksplit; ++ks) v += p.p_part[(static_cast<size_t>(ks) * p.B + b) * p.NQKV + gc];
+    const float *pp = p.p_part + static_cast<size_t>(b) * p.NQKV + gc;
+    // the first eight split-K partials and the state rows (KC <= 8) as independent loads, so
+    // they share one memory round trip
+    float part[8], st[7];
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) part[ks] = ks < p.ksplit ? pp[ks * kstride] : 0.f;
+#pragma unroll
+    for (int j = 0; j < 7; ++j)
+      st[j] = c < QKC && j < KC1 ? cs[static_cast<size_t>(j) * W + gc] : 0.f;
+    const int vc = g * DL + (c - QKC);              // a value channel's index in N_kv
+    const bool shifted = c >= QKC && (p.flags & F_VALUE_SHIFT) && vc >= p.VS0;
+    const float vsv = shifted ? vs[vc - p.VS0] : 0.f;
+    float v = ((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7]));
+    for (int ks = 8; ks < p.ksplit; ++ks) v += pp[ks * kstride];
     m.pn[c] = v;
+    if (c >= QKC) m.vsh[c - QKC] = vsv;
     if (c < QKC)
-      for (int j = 0; j < KC1; ++j) m.old[j * QKC + c] = cs[static_cast<size_t>(j) * W + gc];
+#pragma unroll
+      for (int j = 0; j < 7; ++j)
+        if (j < KC1) m.old[j * QKC + c] = st[j];
   }
 }
 
 // The stencil of the new token at position L (< max_seq): k and v rows appended to the cache,
 // the G query heads' rotated latents to q (head hh at q + hh * DL; global or shared memory),
-// conv / value-shift state advanced.  Every thread of the block takes part (__syncthreads).
+// conv / value-shift state advanced.  Threads tid = 0..nt-1 (the ones that ran d2_load, with
+// the same numbering) take part and meet at named barrier `bar`; kv_keep (optional, shared
+// memory [2][DL]) receives the appended key and value as the cache holds them.
 template <typename T, int DL>
 __device__ __forceinline__ void d2_compute(const D2Params<T> &p, int g, int b, int L,
-                                           const D2Smem<DL> &m, float *q) {
+                                           const D2Smem<DL> &m, float *q, int tid, int nt, int bar,
+                                           float *kv_keep = nullptr) {
   using TL = typename D2Params<T>::TL;
-  const int tid = threadIdx.x, nt = blockDim.x;
   const int G = p.G, QKC = (G + 1) * DL, KC = p.KC, KC1 = KC - 1;
   const int LD = d2_ld(QKC);
   const int qcol0 = g * G * DL, kcol0 = p.NQ + g * DL;
@@ -289,7 +351,7 @@ __device__ __forceinline__ void d2_compute(const D2Params<T> &p, int g, int b, i
     for (int j = 0; j < KC1; ++j) acc = fmaf(w[j], m.old[j * QKC + c], acc);
     m.a[c] = fmaf(w[KC1], m.pn[c], acc);
   }
-  __syncthreads();
+  bar_sync(bar, nt);
   // channel conv (thread per output) and q-k-mean
   for (int o = tid; o < QKC; o += nt) {
     const int hh = o / DL, i = o % DL;
@@ -309,7 +371,7 @@ __device__ __forceinline__ void d2_compute(const D2Params<T> &p, int g, int b, i
     }
     m.u[o] = acc;
   }
-  __syncthreads();
+  bar_sync(bar, nt);
   // RMS norm per head: one warp per head
   const int warp = tid >> 5, lane = tid & 31;
   for (int hh = warp; hh <= G; hh += nt / 32) {
@@ -320,7 +382,7 @@ __device__ __forceinline__ void d2_compute(const D2Params<T> &p, int g, int b, i
     if (lane == 0)
       m.inv[hh] = (p.flags & F_QK_NORM) ? 1.0f / sqrtf(ss / static_cast<float>(DL) + p.eps) : 1.0f;
   }
-  __syncthreads();
+  bar_sync(bar, nt);
   // RoPE at position L on (i, i + DL/2) pairs, then store q and k (cache); every pair a thread
   // takes has i = tid mod DL/2 (DL/2 divides the block size), whose rotation it computed above
   for (int o = tid; o < (G + 1) * HALF; o += nt) {
@@ -338,8 +400,13 @@ __device__ __forceinline__ void d2_compute(const D2Params<T> &p, int g, int b, i
       auto *kd = p.k_cache + ((static_cast<size_t>(b) * p.Hkv + g) * p.max_seq + L) * DL;
       check_latent<TL>(x1, p.status);
       check_latent<TL>(x2, p.status);
-      kd[ip] = from_f32<TL>(x1);
-      kd[ip + HALF] = from_f32<TL>(x2);
+      const TL k1 = from_f32<TL>(x1), k2 = from_f32<TL>(x2);
+      kd[ip] = k1;
+      kd[ip + HALF] = k2;
+      if (kv_keep) {                                 // the appended key as the cache holds it
+        kv_keep[ip] = to_f32(k1);
+        kv_keep[ip + HALF] = to_f32(k2);
+      }
     }
   }
   // value with the value-shift, appended at position L
@@ -348,9 +415,11 @@ __device__ __forceinline__ void d2_compute(const D2Params<T> &p, int g, int b, i
   for (int c = tid; c < DL; c += nt) {
     const int vc = g * DL + c;
     const bool shifted = vc >= vhalf;
-    const float val = ((p.flags & F_VALUE_SHIFT) && shifted) ? vs[vc - vhalf] : m.pn[QKC + c];
+    const float val = ((p.flags & F_VALUE_SHIFT) && shifted) ? m.vsh[c] : m.pn[QKC + c];
     check_latent<TL>(val, p.status);
-    p.v_cache[((static_cast<size_t>(b) * p.Hkv + g) * p.max_seq + L) * DL + c] = from_f32<TL>(val);
+    const TL vv = from_f32<TL>(val);
+    p.v_cache[((static_cast<size_t>(b) * p.Hkv + g) * p.max_seq + L) * DL + c] = vv;
+    if (kv_keep) kv_keep[DL + c] = to_f32(vv);
   }
   // state advance (thread c rewrites only channel c's state, which it alone read)
   for (int c = tid; c < QKC; c += nt) {
@@ -373,13 +442,14 @@ __global__ void __launch_bounds__(256) decode_stencil_kernel(const D2Params<T> p
   d2_stage(p, g, b, m);
   __syncthreads();                                   // staged filters visible to every thread
   pdl_wait();
-  d2_load(p, g, b, m);                               // loads in flight before the position
+  d2_load(p, g, b, m, threadIdx.x, blockDim.x);      // loads in flight before the position
   const int L = p.lengths[b];
   if (L >= p.max_seq) {
     if (threadIdx.x == 0) report(p.status, DEV_CACHE_FULL);
     return;
   }
-  d2_compute(p, g, b, L, m, p.q_new + (static_cast<size_t>(b) * p.H + g * p.G) * DL);
+  d2_compute(p, g, b, L, m, p.q_new + (static_cast<size_t>(b) * p.H + g * p.G) * DL, threadIdx.x,
+             blockDim.x, 0);
 }
 
 // ------------------------------------------------------------------ D3 split-KV attention
@@ -601,27 +671,14 @@ template <int DL>
 __host__ __device__ constexpr size_t tc_smem_bytes() {
   return static_cast<size_t>(tc_slots<DL>()) * TC_SUB * DL * 4 + 4 * 8 * (DL + 2) * 4;
 }
-// With the stencil fused in: the new token's queries [8][DL], key and value [2][DL] (float16-
-// rounded) and the G heads' scores of the new key [8], after the combine area.
-template <int DL>
-__host__ __device__ constexpr size_t tc_fused_smem_bytes() {
-  return tc_smem_bytes<DL>() + (8 * DL + 2 * DL + 8) * 4;
-}
 
-// STENCIL: the decode stencil of the new token (D2) runs inside this kernel, one CTA per
-// (sequence, group) with the keys unsplit.  Its filters are staged before the grid-dependency
-// wait into the ring's last slot (free until the first loop iteration refills it); after the
-// wait the CTA starts streaming cache rows 0..L-1, computes the new token's queries (kept in
-// shared memory), key and value (appended to the cache as before, and kept), and the new key
-// enters the softmax as one more partial (m = its score, l = 1, o = its value) in the combine.
-template <int DL, bool STENCIL>
+template <int DL>
 __global__ void __launch_bounds__(128, 1) decode_attn_tc_kernel(
     const float *__restrict__ q_new, const __half *__restrict__ k_cache,
     const __half *__restrict__ v_cache, const int *__restrict__ lengths,
     float *__restrict__ part_o, float *__restrict__ part_ml, __nv_bfloat16 *__restrict__ o_hi,
     __nv_bfloat16 *__restrict__ o_lo, int H, int Hkv, int G, int max_seq, int chunk, int nchunk,
-    float scale_log2, const uint8_t *__restrict__ next_w, size_t next_w_bytes,
-    const D2Params<__nv_bfloat16> p2) {
+    float scale_log2, const uint8_t *__restrict__ next_w, size_t next_w_bytes) {
   constexpr int CPR = DL / 8;                        // 16-byte pieces (8 dims) per row
   constexpr int NSLOT = tc_slots<DL>();
   constexpr int NT = TC_SUB / 32;                    // 8-key n-tiles per warp step
@@ -647,26 +704,14 @@ __global__ void __launch_bounds__(128, 1) decode_attn_tc_kernel(
     for (size_t i = id * per + tid; i < min(lines, (id + 1) * per); i += blockDim.x)
       prefetch_l2(next_w + i * 128);
   }
-  float *scratch = reinterpret_cast<float *>(ring + (NSLOT - 1) * SLOT);
-  float *qn = wst + 4 * 8 * (DL + 2);                // STENCIL: [8][DL] queries
-  float *kvn = qn + 8 * DL;                          // [2][DL] new key, value
-  float *sn = kvn + 2 * DL;                          // [8] scores of the new key
-  if constexpr (STENCIL) {
-    const D2Smem<DL> m(scratch, p2.G, p2.KC);
-    d2_stage(p2, g, b, m);
-    __syncthreads();                                 // staged filters visible to every thread
-  }
   pdl_wait();
   const int L = lengths[b];
   const int s0 = ch * chunk;
-  // keys streamed from the cache: with the stencil fused in, rows 0..L-1 (row L is the new key,
-  // written by this kernel and taken from shared memory)
-  const int n = L < max_seq ? (STENCIL ? L : min(chunk, L + 1 - s0)) : 0;
+  const int n = L < max_seq ? min(chunk, L + 1 - s0) : 0;   // keys of this split
   float *po = part_o + ((static_cast<size_t>(b) * H + g * G) * nchunk + ch) * DL;
   float *pml = part_ml + ((static_cast<size_t>(b) * H + g * G) * nchunk + ch) * 2;
   const bool whole = nchunk == 1;                    // one split: write the merged o itself
-  if (STENCIL && L >= max_seq && tid == 0) report(p2.status, DEV_CACHE_FULL);
-  if (STENCIL ? L >= max_seq : n <= 0) {
+  if (n <= 0) {
     for (int i = tid; i < G * DL; i += blockDim.x) {
       if (whole) {
         o_hi[(static_cast<size_t>(b) * H + g * G) * DL + i] = __float2bfloat16_rn(0.f);
@@ -702,31 +747,11 @@ __global__ void __launch_bounds__(128, 1) decode_attn_tc_kernel(
 #pragma unroll
   for (int s = 0; s < NSLOT - 1; ++s) issue(s);
 
-  if constexpr (STENCIL) {
-    // the new token's stencil while the first sub-chunks are in flight
-    const D2Smem<DL> m(scratch, p2.G, p2.KC);
-    d2_load(p2, g, b, m);                            // each thread reads back only its own loads
-    d2_compute(p2, g, b, L, m, qn);
-    __syncthreads();                                 // q and the appended row L are visible
-    const size_t rowL = ((static_cast<size_t>(b) * Hkv + g) * max_seq + L) * DL;
-    for (int i = tid; i < 2 * DL; i += blockDim.x)   // read back through the writable pointers
-      kvn[i] = __half2float(i < DL ? p2.k_cache[rowL + i] : p2.v_cache[rowL + i - DL]);
-    __syncthreads();
-    // the new key's score per head, with q rounded to float16 as the MMA fragments below
-    for (int h = warp; h < G; h += 4) {
-      float acc = 0.f;
-      for (int i = lane; i < DL; i += 32)
-        acc = fmaf(__half2float(__float2half_rn(qn[h * DL + i])), kvn[i], acc);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-      if (lane == 0) sn[h] = acc * scale_log2;
-    }
-  }
 
   // Q fragments (rows = heads; a1, a3 are rows 8..15 and stay zero)
   uint32_t qa[DL / 16][2];
   {
-    const float *qh = STENCIL ? qn + gr * DL : q_new + (static_cast<size_t>(b) * H + g * G + gr) * DL;
+    const float *qh = q_new + (static_cast<size_t>(b) * H + g * G + gr) * DL;
 #pragma unroll
     for (int kk = 0; kk < DL / 16; ++kk) {
       float v0 = 0.f, v1 = 0.f, v2 = 0.f, v3 = 0.f;
@@ -843,7 +868,7 @@ __global__ void __launch_bounds__(128, 1) decode_attn_tc_kernel(
   __syncthreads();
   for (int i = tid; i < G * DL; i += blockDim.x) {
     const int h = i / DL, d = i % DL;
-    float mw[4], M = STENCIL ? sn[h] : -INFINITY;
+    float mw[4], M = -INFINITY;
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
       mw[w] = wst[(w * 8 + h) * WS + DL];
@@ -855,11 +880,6 @@ __global__ void __launch_bounds__(128, 1) decode_attn_tc_kernel(
       const float c = mw[w] == -INFINITY ? 0.f : exp2f(mw[w] - M);
       acc = fmaf(c, wst[(w * 8 + h) * WS + d], acc);
       lsum = fmaf(c, wst[(w * 8 + h) * WS + DL + 1], lsum);
-    }
-    if constexpr (STENCIL) {                         // the new key: one more partial, l = 1
-      const float c = exp2f(sn[h] - M);
-      acc = fmaf(c, kvn[DL + d], acc);
-      lsum += c;
     }
     if (whole) {
       const float v = acc / lsum;
@@ -874,6 +894,395 @@ __global__ void __launch_bounds__(128, 1) decode_attn_tc_kernel(
         pml[static_cast<size_t>(h) * nchunk * 2 + 1] = lsum;
       }
     }
+  }
+}
+
+// ------------------------------------------------------------------ D2 + D3, cache buffered in TMEM
+// The stencil of the new token sits on the path to the first score (no score exists before q),
+// and in decode_attn_tc_kernel the cache stream meanwhile stops after the two sub-chunks its
+// copy ring has free (the third slot holds the stencil's filters).  This kernel adds four
+// filler warps (4..7) beside the four compute warps (0..3): while the compute warps run the
+// stencil, the fillers stream the first sub-chunks through the two free slots and park each in
+// tensor memory already in the compute warps' MMA fragment form (filler warp 4 + w issues
+// exactly the ldmatrix reads compute warp w would, and stores the words to the TMEM lanes of
+// their common lane quadrant, one column per word), then leave the next sub-chunks in the free
+// slots.  The compute warps take the parked sub-chunks from TMEM (tcgen05.ld straight into
+// fragments), then continue through the ring as decode_attn_tc_kernel does.  Hand-offs use
+// named barriers: FZ_BAR_TM + i (sub-chunk i parked; fillers arrive, compute warps wait),
+// FZ_BAR_HO (both sides: the fillers' copies have landed, the compute warps are done with
+// TMEM, which warp 4 then frees), FZ_BAR_C / FZ_BAR_F (within the compute / filler warps).
+constexpr int FZ_TMEM_COLS = 256;            // per CTA: two CTAs per SM share the 512 columns
+constexpr int FZ_BAR_C = 1, FZ_BAR_F = 2, FZ_BAR_TM = 3;
+
+template <int DL>
+__host__ __device__ constexpr int fz_words() {   // fragment words per thread per sub-chunk
+  return 2 * (TC_SUB / 32) * (DL / 8);
+}
+// sub-chunks parked in TMEM: as many as the columns hold, rounded down to a multiple of the
+// free slots (so the ring positions the fillers leave match the compute warps' ring order)
+template <int DL>
+__host__ __device__ constexpr int fz_parked() {
+  return FZ_TMEM_COLS / fz_words<DL>() / (tc_slots<DL>() - 1) * (tc_slots<DL>() - 1);
+}
+// the ring and combine area of decode_attn_tc_kernel, then the new token's queries [8][DL],
+// key and value [2][DL] (float16-rounded), the G heads' scores of the new key [8] and the TMEM
+// address
+template <int DL>
+__host__ __device__ constexpr size_t fz_smem_bytes() {
+  return tc_smem_bytes<DL>() + (8 * DL + 2 * DL + 8) * 4 + 16;
+}
+
+template <int DL>
+__global__ void __launch_bounds__(256, 2) decode_attn_fused_kernel(
+    const __half *__restrict__ k_cache, const __half *__restrict__ v_cache,
+    const int *__restrict__ lengths, __nv_bfloat16 *__restrict__ o_hi,
+    __nv_bfloat16 *__restrict__ o_lo, int H, int Hkv, int G, int max_seq, float scale_log2,
+    const uint8_t *__restrict__ next_w, size_t next_w_bytes, const D2Params<__nv_bfloat16> p2) {
+  constexpr int CPR = DL / 8;                        // 16-byte pieces (8 dims) per row
+  constexpr int NSLOT = tc_slots<DL>();
+  constexpr int NT = TC_SUB / 32;                    // 8-key n-tiles per warp step
+  constexpr int WK = NT * 8;                         // keys per warp per sub-chunk
+  constexpr int SLOT = 2 * TC_SUB * DL;              // halves per slot: [K | V]
+  constexpr int KW = NT * CPR;                       // K (and V) fragment words per thread
+  constexpr int FW = 2 * KW;
+  constexpr int NPARK = fz_parked<DL>();
+  constexpr int FREE = NSLOT - 1;                    // slots free while the stencil runs
+  constexpr int FZ_BAR_HO = FZ_BAR_TM + NPARK;
+  static_assert(4 * WK == TC_SUB && NT % 2 == 0, "four warps cover a sub-chunk");
+  static_assert(KW % 16 == 0, "TMEM stores of 16 columns");
+  static_assert(NPARK >= FREE && NPARK * FW <= FZ_TMEM_COLS && FZ_BAR_HO < 16, "TMEM parking");
+  static_assert(NSLOT <= 6, "at most five copy groups in flight");
+  extern __shared__ __align__(16) uint8_t smraw[];
+  __half *ring = reinterpret_cast<__half *>(smraw);  // [NSLOT][K, V][TC_SUB][DL], swizzled
+  float *wst = reinterpret_cast<float *>(ring + NSLOT * SLOT);     // [4][8 heads][DL + 2]
+  float *qn = wst + 4 * 8 * (DL + 2);                // [8][DL] queries of the new token
+  float *kvn = qn + 8 * DL;                          // [2][DL] its key and value
+  float *sn = kvn + 2 * DL;                          // [8] scores of the new key
+  uint32_t *taddr_s = reinterpret_cast<uint32_t *>(sn + 8);
+  float *scratch = reinterpret_cast<float *>(ring + (NSLOT - 1) * SLOT);
+  const int g = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31, gr = lane >> 2, qd = lane & 3;
+  const int t = tid & 127;                           // index within the compute or filler half
+  const bool filler = warp >= 4;
+  {
+    // the up-projection weights, which nothing in the step writes, towards L2 for the step's
+    // last kernel (the evict-first cache stream leaves them there); an equal share per CTA
+    const size_t lines = (next_w_bytes + 127) / 128;
+    const size_t ctas = static_cast<size_t>(gridDim.y) * gridDim.z;
+    const size_t id = static_cast<size_t>(b) * gridDim.y + g;
+    const size_t per = (lines + ctas - 1) / ctas;
+    for (size_t i = id * per + tid; i < min(lines, (id + 1) * per); i += blockDim.x)
+      prefetch_l2(next_w + i * 128);
+  }
+  if (warp == 4) {
+    tmem_alloc(taddr_s, FZ_TMEM_COLS);
+    tmem_relinquish();
+  }
+  // the dependents launch only once this CTA holds its columns (two CTAs of this kernel fill
+  // an SM's shared memory, so their 2 x 256 columns never wait on each other)
+  pdl_launch_dependents();
+  const D2Smem<DL> m(scratch, p2.G, p2.KC);
+  d2_stage<__nv_bfloat16, DL, 5>(p2, g, b, m);       // 5 x 256 loads: a group of 4 + 1 heads of 32
+  tc_fence_before();
+  __syncthreads();                                   // filters staged, TMEM address posted
+  tc_fence_after();
+  const uint32_t tmem = *taddr_s + ((static_cast<uint32_t>(warp & 3) * 32) << 16);
+  pdl_wait();
+  const int L = lengths[b];
+  if (!filler) d2_load(p2, g, b, m, t, 128);         // shares the length's round trip
+  if (L >= max_seq) {                                // cache full: o = 0, nothing appended
+    if (tid == 0) report(p2.status, DEV_CACHE_FULL);
+    for (int i = tid; i < G * DL; i += blockDim.x) {
+      o_hi[(static_cast<size_t>(b) * H + g * G) * DL + i] = __float2bfloat16_rn(0.f);
+      o_lo[(static_cast<size_t>(b) * H + g * G) * DL + i] = __float2bfloat16_rn(0.f);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 4) {
+      tc_fence_after();
+      tmem_dealloc(*taddr_s, FZ_TMEM_COLS);
+    }
+    return;
+  }
+  const int n = L;                                   // cache rows 0..L-1; row L is the new key
+  const size_t row0 = (static_cast<size_t>(b) * Hkv + g) * max_seq;
+  const int nsub = (n + TC_SUB - 1) / TC_SUB;
+  const uint64_t stream_pol = l2_evict_first_policy();
+  auto issue = [&](int sbi, int slot) {              // sub-chunk sbi into `slot` by this half's
+    if (sbi < nsub) {                                // 128 threads; an empty group past the end
+      const int base = sbi * TC_SUB, cnt = min(TC_SUB, n - base);  // rows past cnt: zeros
+      __half *kd = ring + slot * SLOT, *vd = kd + TC_SUB * DL;
+      for (int i = t; i < TC_SUB * CPR; i += 128) {
+        const int r = i / CPR, j = i % CPR;
+        const bool ok = r < cnt;
+        const size_t src = (row0 + base + (ok ? r : 0)) * DL + j * 8;
+        const int dst = r * DL + (j ^ kv_swz<CPR>(r)) * 8;
+        cp_async16_zfill_stream(kd + dst, k_cache + src, ok, stream_pol);
+        cp_async16_zfill_stream(vd + dst, v_cache + src, ok, stream_pol);
+      }
+    }
+    cp_async_commit();
+  };
+  const int kb = (warp & 3) * WK;                    // the compute warp's first key in a sub-chunk
+
+  if (filler) {
+    // ---- park sub-chunks 0..NPARK-1 in TMEM; leave NPARK..NPARK+FREE-1 in slots 0..FREE-1
+#pragma unroll
+    for (int s = 0; s < FREE; ++s) issue(s, s);
+    for (int i = 0; i < NPARK; ++i) {
+      const int slot = i % FREE;
+      cp_async_wait_group<FREE - 1>();               // sub-chunk i has landed (own copies)
+      bar_sync(FZ_BAR_F, 128);                       // ... everyone's
+      if (i < nsub) {
+        const uint32_t ks_base = smem_u32(ring + slot * SLOT);
+        const uint32_t vs_base = ks_base + TC_SUB * DL * 2;
+        uint32_t w[FW];
+#pragma unroll
+        for (int m0 = 0; m0 < KW; m0 += 4) {         // K: the S = Q K^T B fragments
+          const int id = m0 + (lane >> 3);
+          const int nt = id / CPR, j = id % CPR;
+          const int r = kb + nt * 8 + (lane & 7);
+          ldsm_x4(ks_base + (r * DL + (j ^ kv_swz<CPR>(r)) * 8) * 2, w[m0], w[m0 + 1], w[m0 + 2],
+                  w[m0 + 3]);
+        }
+#pragma unroll
+        for (int kk = 0; kk < NT / 2; ++kk) {        // V: the O += P V B fragments
+#pragma unroll
+          for (int t0 = 0; t0 < DL / 8; t0 += 2) {
+            const int id = lane >> 3;
+            const int r = kb + kk * 16 + (id & 1) * 8 + (lane & 7);
+            const int j = t0 + (id >> 1);
+            const int o = KW + (kk * (DL / 16) + t0 / 2) * 4;
+            ldsm_x4_t(vs_base + (r * DL + (j ^ kv_swz<CPR>(r)) * 8) * 2, w[o], w[o + 1], w[o + 2],
+                      w[o + 3]);
+          }
+        }
+#pragma unroll
+        for (int c = 0; c < FW; c += 16) {
+          uint32_t w16[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) w16[e] = w[c + e];
+          tmem_st16(tmem + i * FW + c, w16);
+        }
+        tmem_st_wait();
+      }
+      bar_sync(FZ_BAR_F, 128);                       // every filler is done with the slot
+      issue(i + FREE, slot);                         // -> slot (i + FREE) % FREE == slot
+      tc_fence_before();
+      bar_arrive(FZ_BAR_TM + i, 256);                // sub-chunk i is in TMEM
+    }
+    cp_async_wait_group<0>();                        // the ring's sub-chunks have landed
+    bar_sync(FZ_BAR_HO, 256);                        // ... and the compute warps are off TMEM
+    if (warp == 4) {
+      tc_fence_after();
+      tmem_dealloc(*taddr_s, FZ_TMEM_COLS);
+    }
+    return;
+  }
+
+  // ---- compute warps: the stencil of the new token (the fillers stream meanwhile)
+  d2_compute(p2, g, b, L, m, qn, t, 128, FZ_BAR_C, kvn);
+  bar_sync(FZ_BAR_C, 128);                           // q, the new key and value are visible
+
+  // Q fragments (rows = heads; a1, a3 are rows 8..15 and stay zero)
+  uint32_t qa[DL / 16][2];
+  {
+    const float *qh = qn + gr * DL;
+#pragma unroll
+    for (int kk = 0; kk < DL / 16; ++kk) {
+      float v0 = 0.f, v1 = 0.f, v2 = 0.f, v3 = 0.f;
+      if (gr < G) {
+        v0 = qh[16 * kk + 2 * qd];
+        v1 = qh[16 * kk + 2 * qd + 1];
+        v2 = qh[16 * kk + 2 * qd + 8];
+        v3 = qh[16 * kk + 2 * qd + 9];
+      }
+      qa[kk][0] = pack_f16x2(v0, v1);
+      qa[kk][1] = pack_f16x2(v2, v3);
+    }
+  }
+  float o[DL / 8][4];
+#pragma unroll
+  for (int u = 0; u < DL / 8; ++u) o[u][0] = o[u][1] = o[u][2] = o[u][3] = 0.f;
+  float m_run = -INFINITY, l_run = 0.f;              // of head row gr (lanes of one quad agree)
+
+  // online softmax of row gr over this warp's keys of one sub-chunk; P as f16 A fragments
+  auto softmax = [&](float (&sc)[NT][4], int valid, uint32_t (&pa)[NT / 2][2]) {
+    float mx = -INFINITY;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        sc[nt][e] = nt * 8 + 2 * qd + e < valid ? sc[nt][e] * scale_log2 : -INFINITY;
+        mx = fmaxf(mx, sc[nt][e]);
+      }
+    }
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    const float m_new = fmaxf(m_run, mx);            // finite: key kb of this slice is valid
+    const float f = exp2f(m_run - m_new);            // 0 while m_run = -inf
+    m_run = m_new;
+    float ls = 0.f;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const float p0 = exp2f(sc[nt][0] - m_new), p1 = exp2f(sc[nt][1] - m_new);
+      ls += p0 + p1;
+      pa[nt / 2][nt & 1] = pack_f16x2(p0, p1);
+    }
+    l_run = l_run * f + ls;
+#pragma unroll
+    for (int u = 0; u < DL / 8; ++u) {
+      o[u][0] *= f;
+      o[u][1] *= f;
+    }
+  };
+
+  // ---- the parked sub-chunks, fragments straight from TMEM
+  for (int i = 0; i < NPARK; ++i) {
+    bar_sync(FZ_BAR_TM + i, 256);
+    tc_fence_after();
+    const int valid = n - i * TC_SUB - kb;
+    if (i < nsub && valid > 0) {
+      float sc[NT][4];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+#pragma unroll
+      for (int h = 0; h < KW; h += 16) {             // K words, 16 columns per load
+        uint32_t kw[16];
+        tmem_ld16(tmem + i * FW + h, kw);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 16; e += 2) {
+          const int idm = h + e, ntm = idm / CPR, kk = (idm % CPR) / 2;
+          const uint32_t a[4] = {qa[kk][0], 0u, qa[kk][1], 0u};
+          const uint32_t bb[2] = {kw[e], kw[e + 1]};
+          mma_f16_16816(sc[ntm], a, bb);
+        }
+      }
+      uint32_t pa[NT / 2][2];
+      softmax(sc, valid, pa);
+      constexpr int WPK = DL / 4;                    // V words per 16-key step
+#pragma unroll
+      for (int h = 0; h < KW; h += 16) {
+        uint32_t vw[16];
+        tmem_ld16(tmem + i * FW + KW + h, vw);
+        tmem_ld_wait();
+#pragma unroll
+        for (int kk = h / WPK; kk < (h + 16) / WPK; ++kk) {
+          const uint32_t a[4] = {pa[kk][0], 0u, pa[kk][1], 0u};
+#pragma unroll
+          for (int t0 = 0; t0 < DL / 8; t0 += 2) {
+            const int w0 = kk * WPK + (t0 / 2) * 4 - h;
+            const uint32_t b0[2] = {vw[w0], vw[w0 + 1]}, b1[2] = {vw[w0 + 2], vw[w0 + 3]};
+            mma_f16_16816(o[t0], a, b0);
+            mma_f16_16816(o[t0 + 1], a, b1);
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  bar_sync(FZ_BAR_HO, 256);                          // slots 0..FREE-1 hold sub-chunks NPARK..
+
+  // ---- the rest through the ring: sub-chunk s >= NPARK in slot (s - NPARK) % NSLOT
+#pragma unroll
+  for (int s = 0; s < FREE; ++s) cp_async_commit();  // stand-ins for the fillers' groups
+  for (int sbi = NPARK; sbi < nsub; ++sbi) {
+    cp_async_wait_group<NSLOT - 2>();                // sub-chunk sbi has landed
+    bar_sync(FZ_BAR_C, 128);                         // ... for every thread; and every warp
+    issue(sbi + NSLOT - 1, (sbi + NSLOT - 1 - NPARK) % NSLOT);  // is done with that slot
+    const uint32_t ks_base = smem_u32(ring + ((sbi - NPARK) % NSLOT) * SLOT);
+    const uint32_t vs_base = ks_base + TC_SUB * DL * 2;
+    const int valid = n - sbi * TC_SUB - kb;         // keys of this warp's slice that exist
+    if (valid > 0) {
+      float sc[NT][4];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+#pragma unroll
+      for (int m0 = 0; m0 < KW; m0 += 4) {           // four (n-tile, piece) matrices per load
+        const int id = m0 + (lane >> 3);
+        const int nt = id / CPR, j = id % CPR;
+        const int r = kb + nt * 8 + (lane & 7);
+        uint32_t f[4];
+        ldsm_x4(ks_base + (r * DL + (j ^ kv_swz<CPR>(r)) * 8) * 2, f[0], f[1], f[2], f[3]);
+#pragma unroll
+        for (int e = 0; e < 4; e += 2) {
+          const int idm = m0 + e, ntm = idm / CPR, kk = (idm % CPR) / 2;
+          const uint32_t a[4] = {qa[kk][0], 0u, qa[kk][1], 0u};
+          const uint32_t bb[2] = {f[e], f[e + 1]};
+          mma_f16_16816(sc[ntm], a, bb);
+        }
+      }
+      uint32_t pa[NT / 2][2];
+      softmax(sc, valid, pa);
+#pragma unroll
+      for (int kk = 0; kk < NT / 2; ++kk) {
+        const uint32_t a[4] = {pa[kk][0], 0u, pa[kk][1], 0u};
+#pragma unroll
+        for (int t0 = 0; t0 < DL / 8; t0 += 2) {      // two dim n-tiles (4 matrices) per load
+          const int id = lane >> 3;
+          const int r = kb + kk * 16 + (id & 1) * 8 + (lane & 7);
+          const int j = t0 + (id >> 1);
+          uint32_t f4[4];
+          ldsm_x4_t(vs_base + (r * DL + (j ^ kv_swz<CPR>(r)) * 8) * 2, f4[0], f4[1], f4[2], f4[3]);
+          const uint32_t b0[2] = {f4[0], f4[1]}, b1[2] = {f4[2], f4[3]};
+          mma_f16_16816(o[t0], a, b0);
+          mma_f16_16816(o[t0 + 1], a, b1);
+        }
+      }
+    }
+  }
+  cp_async_wait_group<0>();                          // only empty groups can be left
+
+  // ---- the new key's score per head, with q rounded to float16 as in the fragments
+  for (int h = warp; h < G; h += 4) {
+    float acc = 0.f;
+    for (int i = lane; i < DL; i += 32)
+      acc = fmaf(__half2float(__float2half_rn(qn[h * DL + i])), kvn[i], acc);
+#pragma unroll
+    for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
+    if (lane == 0) sn[h] = acc * scale_log2;
+  }
+  // ---- combine the four warps and the new key (one more partial: m = its score, l = 1)
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
+  constexpr int WS = DL + 2;
+  if (gr < G) {
+    float *w = wst + (warp * 8 + gr) * WS;
+#pragma unroll
+    for (int u = 0; u < DL / 8; ++u) {
+      w[u * 8 + 2 * qd] = o[u][0];
+      w[u * 8 + 2 * qd + 1] = o[u][1];
+    }
+    if (qd == 0) {
+      w[DL] = m_run;
+      w[DL + 1] = l_run;
+    }
+  }
+  bar_sync(FZ_BAR_C, 128);
+  for (int i = t; i < G * DL; i += 128) {
+    const int h = i / DL, d = i % DL;
+    float mw[4], M = sn[h];
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      mw[w] = wst[(w * 8 + h) * WS + DL];
+      M = fmaxf(M, mw[w]);
+    }
+    float acc = 0.f, lsum = 0.f;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const float c = mw[w] == -INFINITY ? 0.f : exp2f(mw[w] - M);
+      acc = fmaf(c, wst[(w * 8 + h) * WS + d], acc);
+      lsum = fmaf(c, wst[(w * 8 + h) * WS + DL + 1], lsum);
+    }
+    const float c = exp2f(sn[h] - M);
+    acc = fmaf(c, kvn[DL + d], acc);
+    lsum += c;
+    const float v = acc / lsum;
+    const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+    const size_t idx = (static_cast<size_t>(b) * H + g * G) * DL + i;
+    o_hi[idx] = hi;
+    o_lo[idx] = __float2bfloat16_rn(v - __bfloat162float(hi));
   }
 }
 
@@ -1022,18 +1431,32 @@ void decode_workspace_carve(const Dims &d, int max_seq, void *ws, DecodeArgs &a)
   a.chunk = chunk;
 }
 
-template <int DL, bool STENCIL>
+template <int DL>
 static cudaError_t launch_decode_tc(const Dims &d, const DecodeArgs &a, float scale_log2,
-                                    const D2Params<__nv_bfloat16> &p2, cudaStream_t st) {
-  const size_t smem = STENCIL ? tc_fused_smem_bytes<DL>() : tc_smem_bytes<DL>();
-  cudaError_t e = ensure_dyn_smem<decode_attn_tc_kernel<DL, STENCIL>>(smem);
+                                    cudaStream_t st) {
+  const size_t smem = tc_smem_bytes<DL>();
+  cudaError_t e = ensure_dyn_smem<decode_attn_tc_kernel<DL>>(smem);
   if (e != cudaSuccess) return e;
   __nv_bfloat16 *o_hi = static_cast<__nv_bfloat16 *>(a.o);
-  return launch_pdl(decode_attn_tc_kernel<DL, STENCIL>, dim3(a.nchunk, d.Hkv, d.B), dim3(128),
+  return launch_pdl(decode_attn_tc_kernel<DL>, dim3(a.nchunk, d.Hkv, d.B), dim3(128),
                     smem, st, a.q_new, static_cast<const __half *>(a.k_cache),
                     static_cast<const __half *>(a.v_cache), a.lengths, a.part_o, a.part_ml, o_hi,
                     o_hi + static_cast<size_t>(d.B) * d.NQ, d.H, d.Hkv, d.G, a.max_seq, a.chunk,
                     a.nchunk, scale_log2, static_cast<const uint8_t *>(a.w_o),
+                    static_cast<size_t>(d.E) * d.NQ * 2);
+}
+
+template <int DL>
+static cudaError_t launch_decode_fused(const Dims &d, const DecodeArgs &a, float scale_log2,
+                                       const D2Params<__nv_bfloat16> &p2, cudaStream_t st) {
+  const size_t smem = fz_smem_bytes<DL>();
+  cudaError_t e = ensure_dyn_smem<decode_attn_fused_kernel<DL>>(smem);
+  if (e != cudaSuccess) return e;
+  __nv_bfloat16 *o_hi = static_cast<__nv_bfloat16 *>(a.o);
+  return launch_pdl(decode_attn_fused_kernel<DL>, dim3(1, d.Hkv, d.B), dim3(256), smem, st,
+                    static_cast<const __half *>(a.k_cache), static_cast<const __half *>(a.v_cache),
+                    a.lengths, o_hi, o_hi + static_cast<size_t>(d.B) * d.NQ, d.H, d.Hkv, d.G,
+                    a.max_seq, scale_log2, static_cast<const uint8_t *>(a.w_o),
                     static_cast<size_t>(d.E) * d.NQ * 2, p2);
 }
 
@@ -1042,10 +1465,10 @@ static cudaError_t launch_decode_attn(const Dims &d, const DecodeArgs &a, float 
                                       const D2Params<__nv_bfloat16> *p2, cudaStream_t st) {
   if constexpr (sizeof(TL) == 2) {
     if (p2) {
-      if constexpr (DL <= 32) return launch_decode_tc<DL, true>(d, a, scale_log2, *p2, st);
+      if constexpr (DL <= 32) return launch_decode_fused<DL>(d, a, scale_log2, *p2, st);
       return cudaErrorInvalidValue;
     }
-    return launch_decode_tc<DL, false>(d, a, scale_log2, D2Params<__nv_bfloat16>{}, st);
+    return launch_decode_tc<DL>(d, a, scale_log2, st);
   }
   const int KS = 128 / (DL / 2);
   const size_t smem = 4 * static_cast<size_t>(SUB) * DL * sizeof(TL) +

@@ -349,6 +349,29 @@ def test_decode_ragged_lengths(cuda_lib, C, max_seq, lengths):
     assert cache.lengths.cpu().tolist() == [l + 1 for l in lengths]
 
 
+@pytest.mark.parametrize("C,max_seq", [(2, 2048), (4, 3072)])
+def test_decode_ragged_long_unsplit(cuda_lib, C, max_seq):
+    """Unsplit keys (160 (sequence, group) pairs) over many 256-key sub-chunks: lengths on and
+    around the sub-chunk boundaries, the end of the sub-chunks the fused kernel parks in tensor
+    memory (4 at d~=32, 5 at d~=16) and the end of those it leaves in the copy ring."""
+    edges = [0, 1, 255, 256, 257, 511, 512, 767, 768, 1023, 1024, 1025, 1279, 1280, 1281,
+             1535, 1536, 1537, 1791, 1792, 2047]
+    rng = np.random.default_rng(5)
+    lengths = [min(e, max_seq - 1) for e in edges] + \
+        [int(v) for v in rng.integers(0, max_seq, 40 - len(edges))]
+    w = W.Workload("dec_long", 40, max(lengths), 512, 8, 4, C, decode=True)
+    inp = W.make_inputs(w, seed=4, conv_std=0.4, lengths=lengths)
+    assert cuda_lib.cca_decode_kernel_count(cuda_lib.make_config(512, 8, 4, C), 40, max_seq) == 3
+    _, cache, y, (ry, rk, rv, *_rest) = decode_vs_oracle(cuda_lib, w, inp, max_seq)
+    assert bf16_err(f64(y), ry) <= BF16_TOL
+    assert cache.lengths.cpu().tolist() == [l + 1 for l in lengths]
+    idx = torch.tensor(lengths)
+    ar = torch.arange(w.batch)
+    gk = f64(cache.k[ar, :, idx]).reshape(w.batch, -1)
+    gv = f64(cache.v[ar, :, idx]).reshape(w.batch, -1)
+    assert bf16_err(gk, rk) <= BF16_TOL and bf16_err(gv, rv) <= BF16_TOL
+
+
 @pytest.mark.parametrize("KC", [4, 2, 6])
 def test_decode_equals_prefill_gpu(cuda_lib, KC):
     """Prefill S0 tokens into the cache, then n decode steps == prefill of S0 + n tokens (the
