@@ -300,28 +300,42 @@ __device__ __forceinline__ void d2_load(const D2Params<T> &p, int g, int b, cons
   const float *cs = p.conv_state + static_cast<size_t>(b) * KC1 * W;
   const size_t kstride = static_cast<size_t>(p.B) * p.NQKV;
   const float *vs = p.vshift_state + static_cast<size_t>(b) * (p.NKV - p.VS0);
-  for (int c = tid; c < CH; c += nt) {
+  // channel c's first eight split-K partials, state rows (KC <= 8) and value-shift entry
+  auto fetch = [&](int c, float (&part)[8], float (&st)[7], float &vsv) {
     const int gc = c < G * DL ? qcol0 + c : (c < QKC ? kcol0 + (c - G * DL) : vcol0 + (c - QKC));
     const float *pp = p.p_part + static_cast<size_t>(b) * p.NQKV + gc;
-    // the first eight split-K partials and the state rows (KC <= 8) as independent loads, so
-    // they share one memory round trip
-    float part[8], st[7];
 #pragma unroll
-    for (int ks = 0; ks < 8; ++ks) part[ks] = ks < p.ksplit ? pp[ks * kstride] : 0.f;
+    for (int ks = 0; ks < 8; ++ks) part[ks] = c < CH && ks < p.ksplit ? pp[ks * kstride] : 0.f;
 #pragma unroll
     for (int j = 0; j < 7; ++j)
       st[j] = c < QKC && j < KC1 ? cs[static_cast<size_t>(j) * W + gc] : 0.f;
     const int vc = g * DL + (c - QKC);              // a value channel's index in N_kv
-    const bool shifted = c >= QKC && (p.flags & F_VALUE_SHIFT) && vc >= p.VS0;
-    const float vsv = shifted ? vs[vc - p.VS0] : 0.f;
+    const bool shifted = c >= QKC && c < CH && (p.flags & F_VALUE_SHIFT) && vc >= p.VS0;
+    vsv = shifted ? vs[vc - p.VS0] : 0.f;
+  };
+  auto put = [&](int c, const float (&part)[8], const float (&st)[7], float vsv) {
+    if (c >= CH) return;
     float v = ((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7]));
-    for (int ks = 8; ks < p.ksplit; ++ks) v += pp[ks * kstride];
+    if (p.ksplit > 8) {
+      const int gc = c < G * DL ? qcol0 + c : (c < QKC ? kcol0 + (c - G * DL) : vcol0 + (c - QKC));
+      const float *pp = p.p_part + static_cast<size_t>(b) * p.NQKV + gc;
+      for (int ks = 8; ks < p.ksplit; ++ks) v += pp[ks * kstride];
+    }
     m.pn[c] = v;
     if (c >= QKC) m.vsh[c - QKC] = vsv;
     if (c < QKC)
 #pragma unroll
       for (int j = 0; j < 7; ++j)
         if (j < KC1) m.old[j * QKC + c] = st[j];
+  };
+  // two channels per thread and pass, both channels' loads issued before either is stored, so
+  // that a CTA with more channels than threads still pays one memory round trip
+  for (int c = tid; c < CH; c += 2 * nt) {
+    float pa[8], sa[7], va, pb[8], sb[7], vb;
+    fetch(c, pa, sa, va);
+    fetch(c + nt, pb, sb, vb);
+    put(c, pa, sa, va);
+    put(c + nt, pb, sb, vb);
   }
 }
 
