@@ -194,20 +194,24 @@ struct D2Params {
 __host__ __device__ constexpr int d2_ld(int QKC) { return QKC | 1; }
 __host__ __device__ inline size_t d2_smem_floats(int G, int DL, int KC) {
   const int QKC = (G + 1) * DL, CH = (G + 2) * DL;
-  return static_cast<size_t>(DL) * d2_ld(QKC)   // wt
+  return 64                                     // RoPE frequencies (32 doubles)
+         + static_cast<size_t>(DL) * d2_ld(QKC)   // wt
          + QKC * KC                             // sequence filters
          + static_cast<size_t>(QKC) * (KC - 1)  // old conv state
          + CH + 2 * QKC + 16                    // pn, av, uv, inv
          + DL;                                  // the value-shift state of the group's channels
 }
 
-// D2's shared-memory carve ([wt | wseq | old | pn | a | u | inv | vsh], floats)
+// D2's shared-memory carve ([th | wt | wseq | old | pn | a | u | inv | vsh], floats; th holds
+// doubles, so `sm` is 8-byte aligned)
 template <int DL>
 struct D2Smem {
+  double *th;
   float *wt, *wseq, *old, *pn, *a, *u, *inv, *vsh;
   __device__ D2Smem(float *sm, int G, int KC) {
     const int QKC = (G + 1) * DL, CH = (G + 2) * DL;
-    wt = sm;
+    th = reinterpret_cast<double *>(sm);
+    wt = sm + 64;
     wseq = wt + DL * d2_ld(QKC);
     old = wseq + QKC * KC;                           // [KC-1][QKC] conv state before the step
     pn = old + QKC * (KC - 1);
@@ -272,6 +276,7 @@ __device__ __forceinline__ void d2_stage(const D2Params<T> &p, int g, int b, con
     for (int k = 0; k < BATCH; ++k)
       if (e0 + k * nt < QKC * KC) m.wseq[e0 + k * nt] = v[k];
   }
+  for (int i = tid; i < DL / 2; i += nt) m.th[i] = p.theta[i];   // read once, off the param bank
   if (p.flags & F_VALUE_SHIFT) {                     // the shifted channels of this group
     const float *vs = p.vshift_state + static_cast<size_t>(b) * (p.NKV - p.VS0);
     for (int c = max(g * DL, p.VS0) + tid * 32; c < (g + 1) * DL; c += nt * 32)
@@ -357,7 +362,7 @@ __device__ __forceinline__ void d2_compute(const D2Params<T> &p, int g, int b, i
   constexpr int HALF = DL / 2;
   float rc = 1.f, rs = 0.f;                          // RoPE rotation of this thread's pairs
   if ((p.flags & F_ROPE) && tid < (G + 1) * HALF)
-    rope_cos_sin(static_cast<double>(L) * p.theta[tid % HALF], rc, rs);
+    rope_cos_sin(static_cast<double>(L) * m.th[tid % HALF], rc, rs);
   // the sequence conv of the q|k channels (each thread reads only what it loaded)
   for (int c = tid; c < QKC; c += nt) {
     const float *w = m.wseq + c * KC;
