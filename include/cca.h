@@ -200,6 +200,10 @@ CCA_API int cca_prefill_forward(const cca_config_t *cfg, const cca_weights_t *w,
  * cache status word is set to CCA_ERR_CACHE_FULL (read it with cca_cache_check).  The decode
  * kernels take at most 8 query heads per kv head (CCA_ERR_UNSUPPORTED otherwise).  A new
  * latent key or value beyond the float16 range sets it to CCA_ERR_RANGE.
+ * Where the stencil runs inside the attention kernel (bfloat16 layers, d~ <= 32, keys unsplit:
+ * cca_decode_kernel_count == 3), each CTA of that kernel holds 256 tensor-memory columns of its
+ * SM while it buffers the first cache rows; a kernel of another stream that allocates tensor
+ * memory on the same SM meanwhile waits for them to be released.
  * Errors (host): INVALID_ARG, UNSUPPORTED, WORKSPACE, ALIGNMENT, CUDA. */
 CCA_API int cca_decode_step(const cca_config_t *cfg, const cca_weights_t *w, const void *x,
                             void *y, cca_cache_t *cache, void *workspace, size_t ws_bytes,
