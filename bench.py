@@ -269,6 +269,11 @@ def bench_prefill(cls, w, steps, warmup, world, seed, e2e=True):
 # (8 GB) and weights (160 MB) pass through L2, so no step finds its own in L2 from its
 # previous use, as in a real decode.
 DECODE_LAYERS = 32
+# The decode step is timed over at least this many steps back to back: the window's first step
+# has no earlier kernel to start under (about 24 us of the chain's start are paid once per
+# window), so a short window overstates the per-step time a serving loop sees.  200 steps
+# are 12 ms of device time.
+DECODE_MIN_STEPS = 200
 
 
 def decode_launches(cls, layer, batch, max_seq):
@@ -328,7 +333,7 @@ def bench_decode(cls, w, steps, warmup, seed, layers=DECODE_LAYERS):
              4: ["qkv_projection", "stencil_append", "attention", "out_projection"],
              3: ["qkv_projection", "stencil_append_attention", "out_projection"]}[nk]
     return dict(ms=ms, stages={n: t / max(calls, 1) for n, t in zip(names, stage_ms)},
-                launches=nk * steps, layers=layers)
+                launches=nk * steps, layers=layers, steps=steps)
 
 
 def cpu_model() -> str:
@@ -482,7 +487,7 @@ def result_line(w, world, steps, warmup, pre, ms, e2e_ms, dec, dms, peaks):
                           "tokens_per_s": job_throughput(dw.batch, world, dms), "GB/s": gbs,
                           "frac_of_hbm": gbs / hbm, "hbm_peak_GB/s": hbm,
                           "bytes_per_step": decode_bytes(dw), "stages_ms": dec["stages"],
-                          "peak_source": peak_src,
+                          "peak_source": peak_src, "steps": dec["steps"],
                           "layers": f"steps rotate over {dec['layers']} independent layers "
                                     "(weights + caches), so none is in L2 from its last use"}
     return line
@@ -563,8 +568,8 @@ def run_cuda(args):
         dec = None
         if not args.no_decode:
             dw = W.WORKLOADS[DECODE_WORKLOAD]
-            dec = bench_decode(cls, dw, args.steps, args.warmup, seed=rank,
-                               layers=args.decode_layers)
+            dec = bench_decode(cls, dw, max(args.steps, DECODE_MIN_STEPS), args.warmup,
+                               seed=rank, layers=args.decode_layers)
         base = None
         if not args.no_baselines and w.name == DEFAULT_WORKLOAD:
             base = bench_baselines(cls, args.steps, args.warmup, world, rank, pre["ms"])

@@ -21,7 +21,7 @@ def _pre(ms):
 
 
 def _dec(ms):
-    return {"ms": ms, "launches": 120, "layers": 32,
+    return {"ms": ms, "launches": 600, "layers": 32, "steps": 200,
             "stages": {"qkv_projection": 0.011, "stencil_append": 0.015,
                        "split_kv_attention": 0.05, "merge": 0.0, "out_projection": 0.011}}
 
@@ -46,12 +46,13 @@ def test_result_line_contract(world):
         assert key in roof, key
     assert roof["achieved"] == pytest.approx(bench.attention_flops(w) / 1.39e-3 / 1e12)
     assert roof["frac"] == pytest.approx(roof["achieved"] / 1670.0)
-    assert line["gpu_launches"] == 300
+    assert line["gpu_launches"] == 780
     d = line["decode"]
     dw = W.WORKLOADS[bench.DECODE_WORKLOAD]
     assert d["GB/s"] == pytest.approx(bench.decode_bytes(dw) / 0.0656e-3 / 1e9)
     assert d["frac_of_hbm"] == pytest.approx(d["GB/s"] / 6453.7)
     assert d["tokens_per_s"] == pytest.approx(world * dw.batch / 0.0656e-3)
+    assert d["steps"] == 200 >= bench.DECODE_MIN_STEPS
     json.loads(json.dumps(line))
 
 
